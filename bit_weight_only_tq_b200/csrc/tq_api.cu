@@ -1,0 +1,261 @@
+// tq_api.cu -- the extern "C" boundary of libtq.so (declared in include/tq.h): argument
+// validation, path dispatch, and host utilities (tensor maps, device properties).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "../../include/tq.h"
+#include "tq_common.cuh"
+
+namespace tq {
+
+bool decode_supported(bool int4, int64_t M, int64_t N, int64_t K);
+bool prefill_supported(bool int4, int64_t M, int64_t N, int64_t K);
+
+static constexpr int kMaxDevices = 64;
+
+DeviceInfo current_device_info() {
+  static int sms[kMaxDevices] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  DeviceInfo d{dev, 148};
+  if (dev >= 0 && dev < kMaxDevices) {
+    if (sms[dev] == 0) {
+      int v = 0;
+      if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+        sms[dev] = v;
+    }
+    if (sms[dev] > 0) d.num_sms = sms[dev];
+  }
+  return d;
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
+                  uint64_t rows, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows,
+                  CUtensorMapSwizzle swizzle) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {row_stride_bytes};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+cudaError_t ensure_smem_attr(const void* func, int bytes) {
+  struct Entry {
+    const void* f;
+    int dev;
+    int bytes;
+  };
+  static Entry cache[256];
+  static int n = 0;
+  static std::mutex mu;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    for (int i = 0; i < n; ++i)
+      if (cache[i].f == func && cache[i].dev == dev && cache[i].bytes >= bytes) return cudaSuccess;
+  }
+  const int want = 227 * 1024;  // set the maximum once per (function, device)
+  cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       bytes > want ? bytes : want);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(mu);
+  if (n < 256) cache[n++] = Entry{func, dev, bytes > want ? bytes : want};
+  return cudaSuccess;
+}
+
+}  // namespace tq
+
+// =============================================================================================
+// extern "C" entry points
+// =============================================================================================
+namespace {
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline int to_status(cudaError_t e) { return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA; }
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Checks common to both GEMMs.  Returns TQ_OK, or an error; sets *empty for M == 0 or N == 0.
+int check_gemm_args(const void* x, const void* w, const void* sc, const void* y, int64_t M,
+                    int64_t N, int64_t K, bool* empty) {
+  if (M < 0 || N < 0 || K <= 0) return TQ_ERR_SHAPE;
+  if (M > (int64_t(1) << 31) || N > (int64_t(1) << 31) || K > (int64_t(1) << 28))
+    return TQ_ERR_SHAPE;
+  *empty = (M == 0 || N == 0);
+  if (*empty) return TQ_OK;
+  if (!x || !w || !sc || !y) return TQ_ERR_NULL;
+  return TQ_OK;
+}
+
+int resolve_path(int fmt, int path, int64_t M, int64_t N, int64_t K, bool all_aligned) {
+  const bool int4 = fmt == TQ_FMT_W4G128;
+  switch (path) {
+    case TQ_PATH_AUTO:
+      return tq_select_path(fmt, M, N, K, all_aligned ? 1 : 0);
+    case TQ_PATH_GENERIC:
+      return TQ_PATH_GENERIC;
+    case TQ_PATH_DECODE:
+      if (!tq::decode_supported(int4, M, N, K)) return TQ_ERR_PATH;
+      return all_aligned ? static_cast<int>(TQ_PATH_DECODE) : static_cast<int>(TQ_ERR_ALIGN);
+    case TQ_PATH_PREFILL:
+      if (!tq::prefill_supported(int4, M, N, K)) return TQ_ERR_PATH;
+      return all_aligned ? static_cast<int>(TQ_PATH_PREFILL) : static_cast<int>(TQ_ERR_ALIGN);
+    default:
+      return TQ_ERR_PATH;
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+int tq_version(void) { return (1 << 16) | 0; }
+
+const char* tq_status_string(int status) {
+  switch (status) {
+    case TQ_OK: return "ok";
+    case TQ_ERR_NULL: return "a required pointer is NULL";
+    case TQ_ERR_SHAPE: return "invalid shape";
+    case TQ_ERR_ALIGN: return "misaligned pointer for the requested path";
+    case TQ_ERR_DTYPE: return "unknown dtype";
+    case TQ_ERR_CUDA: return "CUDA runtime or launch error";
+    case TQ_ERR_TIMEOUT: return "a bounded device-side wait ran out";
+    case TQ_ERR_INVALID_CODE: return "packed data holds the invalid ternary code 0b11";
+    case TQ_ERR_PATH: return "unknown path, or the forced path cannot take this shape";
+    default: return "unknown status";
+  }
+}
+
+int tq_select_path(int fmt, int64_t M, int64_t N, int64_t K, int aligned) {
+  if (fmt != TQ_FMT_TERNARY && fmt != TQ_FMT_W4G128) return TQ_ERR_PATH;
+  const bool int4 = fmt == TQ_FMT_W4G128;
+  if (M < 0 || N < 0 || K <= 0) return TQ_ERR_SHAPE;
+  if (int4 && K % 128 != 0) return TQ_ERR_SHAPE;
+  if (M == 0 || N == 0 || !aligned) return TQ_PATH_GENERIC;
+  // Ridge of the fp16 tensor-core roofline: the decode kernel streams weights at HBM speed and
+  // wins for skinny M; the tensor-core prefill kernel takes over above 16 tokens.
+  if (M <= 16 && tq::decode_supported(int4, M, N, K)) return TQ_PATH_DECODE;
+  if (tq::prefill_supported(int4, M, N, K)) return TQ_PATH_PREFILL;
+  if (M <= 16) return TQ_PATH_GENERIC;
+  return TQ_PATH_GENERIC;
+}
+
+int tq_quantize_pack(const void* w, int w_dtype, uint8_t* packed, uint16_t* scale, int64_t N,
+                     int64_t K, void* stream) {
+  if (w_dtype != TQ_F32 && w_dtype != TQ_F16) return TQ_ERR_DTYPE;
+  if (N < 0 || K <= 0 || K > (int64_t(1) << 28)) return TQ_ERR_SHAPE;
+  if (N == 0) return TQ_OK;
+  if (!w || !packed || !scale) return TQ_ERR_NULL;
+  return to_status(tq::launch_tq_pack(w, w_dtype == TQ_F16, packed, scale, N, K, as_stream(stream)));
+}
+
+int w4g_quantize_pack(const void* w, int w_dtype, int32_t* qweight, uint16_t* scales, int64_t N,
+                      int64_t K, void* stream) {
+  if (w_dtype != TQ_F32 && w_dtype != TQ_F16) return TQ_ERR_DTYPE;
+  if (N < 0 || K <= 0 || K % 128 != 0 || K > (int64_t(1) << 28)) return TQ_ERR_SHAPE;
+  if (N == 0) return TQ_OK;
+  if (!w || !qweight || !scales) return TQ_ERR_NULL;
+  return to_status(tq::launch_w4g_pack(w, w_dtype == TQ_F16, qweight, scales, N, K, as_stream(stream)));
+}
+
+int tq_gemm_ex(const uint16_t* x, const uint8_t* packed, const uint16_t* scale,
+               const uint16_t* bias, uint16_t* y, int64_t M, int64_t N, int64_t K, int path,
+               void* stream) {
+  bool empty = false;
+  int st = check_gemm_args(x, packed, scale, y, M, N, K, &empty);
+  if (st != TQ_OK) return st;
+  if (path < TQ_PATH_AUTO || path > TQ_PATH_GENERIC) return TQ_ERR_PATH;
+  if (empty) return TQ_OK;
+  const bool al = aligned16(x) && aligned16(packed) && aligned16(y);
+  const int p = resolve_path(TQ_FMT_TERNARY, path, M, N, K, al);
+  if (p < 0) return p;
+  const __half* xh = reinterpret_cast<const __half*>(x);
+  const __half* sh = reinterpret_cast<const __half*>(scale);
+  const __half* bh = reinterpret_cast<const __half*>(bias);
+  __half* yh = reinterpret_cast<__half*>(y);
+  cudaStream_t s = as_stream(stream);
+  switch (p) {
+    case TQ_PATH_DECODE: return to_status(tq::launch_tq_gemm_decode(xh, packed, sh, bh, yh, M, N, K, s));
+    case TQ_PATH_PREFILL: return to_status(tq::launch_tq_gemm_prefill(xh, packed, sh, bh, yh, M, N, K, s));
+    default: return to_status(tq::launch_tq_gemm_generic(xh, packed, sh, bh, yh, M, N, K, s));
+  }
+}
+
+int tq_gemm(const uint16_t* x, const uint8_t* packed, const uint16_t* scale, const uint16_t* bias,
+            uint16_t* y, int64_t M, int64_t N, int64_t K, void* stream) {
+  return tq_gemm_ex(x, packed, scale, bias, y, M, N, K, TQ_PATH_AUTO, stream);
+}
+
+int w4g_gemm_ex(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
+                const uint16_t* bias, uint16_t* y, int64_t M, int64_t N, int64_t K, int path,
+                void* stream) {
+  bool empty = false;
+  int st = check_gemm_args(x, qweight, scales, y, M, N, K, &empty);
+  if (st != TQ_OK) return st;
+  if (K % 128 != 0) return TQ_ERR_SHAPE;
+  if (path < TQ_PATH_AUTO || path > TQ_PATH_GENERIC) return TQ_ERR_PATH;
+  if (empty) return TQ_OK;
+  const bool al = aligned16(x) && aligned16(qweight) && aligned16(y) && aligned16(scales);
+  const int p = resolve_path(TQ_FMT_W4G128, path, M, N, K, al);
+  if (p < 0) return p;
+  const __half* xh = reinterpret_cast<const __half*>(x);
+  const __half* sh = reinterpret_cast<const __half*>(scales);
+  const __half* bh = reinterpret_cast<const __half*>(bias);
+  __half* yh = reinterpret_cast<__half*>(y);
+  cudaStream_t s = as_stream(stream);
+  switch (p) {
+    case TQ_PATH_DECODE: return to_status(tq::launch_w4g_gemm_decode(xh, qweight, sh, bh, yh, M, N, K, s));
+    case TQ_PATH_PREFILL: return to_status(tq::launch_w4g_gemm_prefill(xh, qweight, sh, bh, yh, M, N, K, s));
+    default: return to_status(tq::launch_w4g_gemm_generic(xh, qweight, sh, bh, yh, M, N, K, s));
+  }
+}
+
+int w4g_gemm(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
+             const uint16_t* bias, uint16_t* y, int64_t M, int64_t N, int64_t K, void* stream) {
+  return w4g_gemm_ex(x, qweight, scales, bias, y, M, N, K, TQ_PATH_AUTO, stream);
+}
+
+int tq_validate_packed(const uint8_t* packed, int64_t N, int64_t K, int* bad_count, void* stream) {
+  if (N < 0 || K <= 0) return TQ_ERR_SHAPE;
+  if (!bad_count) return TQ_ERR_NULL;
+  if (N > 0 && !packed) return TQ_ERR_NULL;
+  if (N == 0) return to_status(cudaMemsetAsync(bad_count, 0, sizeof(int), as_stream(stream)));
+  return to_status(tq::launch_tq_validate(packed, N, K, bad_count, as_stream(stream)));
+}
+
+int tq_device_status(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return TQ_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, tq::g_tq_device_status, sizeof(int)) != cudaSuccess) return TQ_ERR_CUDA;
+  const int zero = 0;
+  if (v != 0 && cudaMemcpyToSymbol(tq::g_tq_device_status, &zero, sizeof(int)) != cudaSuccess)
+    return TQ_ERR_CUDA;
+  return v == 0 ? TQ_OK : TQ_ERR_TIMEOUT;
+}
+
+}  // extern "C"

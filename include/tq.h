@@ -38,6 +38,12 @@
 
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define TQ_API __attribute__((visibility("default")))
+#else
+#define TQ_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -84,7 +90,7 @@ typedef enum { TQ_FMT_TERNARY = 0, TQ_FMT_W4G128 = 1 } tq_format;
  * The result is bit-exact: it does not depend on summation order.
  * Requires K <= 2^28, N*ceil(K/4) < 2^62.  Returns TQ_OK or an error listed above.
  * ------------------------------------------------------------------------------------------ */
-int tq_quantize_pack(const void* w, int w_dtype, uint8_t* packed, uint16_t* scale,
+TQ_API int tq_quantize_pack(const void* w, int w_dtype, uint8_t* packed, uint16_t* scale,
                      int64_t N, int64_t K, void* stream);
 
 /* --------------------------------------------------------------------------------------------
@@ -100,9 +106,9 @@ int tq_quantize_pack(const void* w, int w_dtype, uint8_t* packed, uint16_t* scal
  * x / packed; PREFILL needs K % 64 == 0 and 16-byte aligned x / packed / y; otherwise
  * TQ_ERR_PATH (shape) or TQ_ERR_ALIGN (pointers).  GENERIC takes any shape.
  * ------------------------------------------------------------------------------------------ */
-int tq_gemm(const uint16_t* x, const uint8_t* packed, const uint16_t* scale, const uint16_t* bias,
+TQ_API int tq_gemm(const uint16_t* x, const uint8_t* packed, const uint16_t* scale, const uint16_t* bias,
             uint16_t* y, int64_t M, int64_t N, int64_t K, void* stream);
-int tq_gemm_ex(const uint16_t* x, const uint8_t* packed, const uint16_t* scale,
+TQ_API int tq_gemm_ex(const uint16_t* x, const uint8_t* packed, const uint16_t* scale,
                const uint16_t* bias, uint16_t* y, int64_t M, int64_t N, int64_t K, int path,
                void* stream);
 
@@ -119,15 +125,15 @@ int tq_gemm_ex(const uint16_t* x, const uint8_t* packed, const uint16_t* scale,
  * clamp(rint(w / s), -8, 7) with the fp64 quotient by the STORED fp16 s, ties to even.
  * Bit-exact.  Calibration-based GPTQ (Hessian error feedback) is not performed.
  * ------------------------------------------------------------------------------------------ */
-int w4g_quantize_pack(const void* w, int w_dtype, int32_t* qweight, uint16_t* scales,
+TQ_API int w4g_quantize_pack(const void* w, int w_dtype, int32_t* qweight, uint16_t* scales,
                       int64_t N, int64_t K, void* stream);
 
 /* w4g_gemm -- y = x . What^T (+ bias), What = scales[n,k/128] * (u - 8) ([VQ] §5 forward:
  * INT4 weight x fp16 activation -> fp16 output).  Shapes as tq_gemm with K % 128 == 0.
  * DECODE needs M <= 16 and 16-byte aligned x / qweight; PREFILL needs 16-byte aligned pointers. */
-int w4g_gemm(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
+TQ_API int w4g_gemm(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
              const uint16_t* bias, uint16_t* y, int64_t M, int64_t N, int64_t K, void* stream);
-int w4g_gemm_ex(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
+TQ_API int w4g_gemm_ex(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
                 const uint16_t* bias, uint16_t* y, int64_t M, int64_t N, int64_t K, int path,
                 void* stream);
 
@@ -135,23 +141,23 @@ int w4g_gemm_ex(const uint16_t* x, const int32_t* qweight, const uint16_t* scale
  * the unused code 0b11 in one of their first K codes of the row ([TQ] §3.1: the table maps
  * 00/01/10 only).  *bad_count (device int) is OVERWRITTEN with the count (set to 0 first, on
  * `stream`).  Returns TQ_OK or an argument error; the count is ready when the stream is. */
-int tq_validate_packed(const uint8_t* packed, int64_t N, int64_t K, int* bad_count, void* stream);
+TQ_API int tq_validate_packed(const uint8_t* packed, int64_t N, int64_t K, int* bad_count, void* stream);
 
 /* tq_select_path -- the host-side dispatch rule used by TQ_PATH_AUTO, exposed so that it can be
  * tested without a GPU.  fmt is a tq_format; aligned16 says whether every pointer is 16-byte
  * aligned.  Returns a tq_path (never AUTO) or a negative tq_status for an invalid shape. */
-int tq_select_path(int fmt, int64_t M, int64_t N, int64_t K, int aligned16);
+TQ_API int tq_select_path(int fmt, int64_t M, int64_t N, int64_t K, int aligned16);
 
 /* tq_device_status -- synchronise the current device, then read and clear the device-side
  * status word written by kernels whose bounded waits ran out.  Returns TQ_OK,
  * TQ_ERR_TIMEOUT, or TQ_ERR_CUDA if the synchronisation itself failed. */
-int tq_device_status(void);
+TQ_API int tq_device_status(void);
 
 /* tq_status_string -- static, human-readable text for a tq_status value. */
-const char* tq_status_string(int status);
+TQ_API const char* tq_status_string(int status);
 
 /* tq_version -- library ABI version, (major << 16) | minor. */
-int tq_version(void);
+TQ_API int tq_version(void);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,89 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every function
+declared in include/tq.h, validates arguments before touching the device, and applies the
+documented dispatch rule."""
+import ctypes
+
+import pytest
+
+import bit_weight_only_tq_b200 as tq
+
+
+def test_library_exports_every_header_function():
+    names = tq.header_functions()
+    assert len(names) == 11
+    for n in names:
+        assert hasattr(tq.lib, n), n
+    for n in ("tq_quantize_pack", "tq_gemm", "w4g_quantize_pack", "w4g_gemm", "tq_validate_packed",
+              "tq_select_path", "tq_device_status", "tq_status_string"):
+        assert n in names
+
+
+def test_status_strings():
+    assert tq.tq_status_string(0) == "ok"
+    for s in range(-8, 0):
+        assert tq.tq_status_string(s) != "unknown status"
+    assert tq.tq_status_string(-99) == "unknown status"
+    assert tq.lib.tq_version() >> 16 == 1
+
+
+NULL = None
+
+
+@pytest.mark.parametrize("N,K,expect", [(-1, 8, -2), (4, 0, -2), (4, -3, -2), (4, 2 ** 29, -2)])
+def test_pack_rejects_bad_shapes(N, K, expect):
+    assert tq.lib.tq_quantize_pack(ctypes.c_void_p(16), 0, ctypes.c_void_p(16), ctypes.c_void_p(16),
+                                   N, K, NULL) == expect
+
+
+def test_pack_rejects_dtype_and_null():
+    assert tq.lib.tq_quantize_pack(ctypes.c_void_p(16), 7, ctypes.c_void_p(16), ctypes.c_void_p(16), 4, 8, NULL) == -4
+    assert tq.lib.tq_quantize_pack(NULL, 0, ctypes.c_void_p(16), ctypes.c_void_p(16), 4, 8, NULL) == -1
+    assert tq.lib.w4g_quantize_pack(ctypes.c_void_p(16), 0, ctypes.c_void_p(16), ctypes.c_void_p(16), 4, 100, NULL) == -2
+    # empty problem: nothing to do, no pointer needed
+    assert tq.lib.tq_quantize_pack(NULL, 0, NULL, NULL, 0, 8, NULL) == 0
+
+
+def test_gemm_argument_errors_without_gpu():
+    p = ctypes.c_void_p(4096)
+    assert tq.lib.tq_gemm(p, p, p, NULL, p, -1, 4, 8, NULL) == -2
+    assert tq.lib.tq_gemm(p, p, p, NULL, p, 1, 4, 0, NULL) == -2
+    assert tq.lib.tq_gemm(NULL, p, p, NULL, p, 1, 4, 8, NULL) == -1
+    assert tq.lib.tq_gemm(p, p, NULL, NULL, p, 1, 4, 8, NULL) == -1
+    assert tq.lib.tq_gemm(NULL, NULL, NULL, NULL, NULL, 0, 4, 8, NULL) == 0   # empty
+    assert tq.lib.tq_gemm(NULL, NULL, NULL, NULL, NULL, 3, 0, 8, NULL) == 0   # empty
+    assert tq.lib.tq_gemm_ex(p, p, p, NULL, p, 1, 4, 64, 9, NULL) == -8       # unknown path
+    assert tq.lib.w4g_gemm(p, p, p, NULL, p, 1, 4, 100, NULL) == -2           # K % 128
+    # forced fast paths refuse shapes they cannot take / misaligned pointers
+    assert tq.lib.tq_gemm_ex(p, p, p, NULL, p, 17, 4, 64, 1, NULL) == -8      # decode needs M<=16
+    assert tq.lib.tq_gemm_ex(p, p, p, NULL, p, 1, 4, 100, 1, NULL) == -8      # decode needs K%64
+    assert tq.lib.tq_gemm_ex(p, p, p, NULL, p, 256, 4, 100, 2, NULL) == -8    # prefill needs K%64
+    q = ctypes.c_void_p(4098)
+    assert tq.lib.tq_gemm_ex(q, p, p, NULL, p, 1, 4, 64, 1, NULL) == -3       # misaligned x
+    assert tq.lib.w4g_gemm_ex(p, p, q, NULL, p, 300, 4, 128, 2, NULL) == -3   # misaligned scales
+
+
+def test_validate_argument_errors():
+    assert tq.lib.tq_validate_packed(ctypes.c_void_p(16), 4, 0, ctypes.c_void_p(16), NULL) == -2
+    assert tq.lib.tq_validate_packed(ctypes.c_void_p(16), 4, 8, NULL, NULL) == -1
+
+
+def test_dispatch_rule():
+    T, W = tq.FMT_TERNARY, tq.FMT_W4G128
+    # decode for skinny M on shapes the decode kernel takes
+    for M in (1, 2, 4, 8, 9, 16):
+        assert tq.tq_select_path(T, M, 4096, 4096) == tq.PATH_DECODE
+        assert tq.tq_select_path(W, M, 4096, 14336) == tq.PATH_DECODE
+    assert tq.tq_select_path(T, 1, 4096, 14336) == tq.PATH_DECODE
+    assert tq.tq_select_path(T, 1, 3584, 18944) == tq.PATH_DECODE
+    assert tq.tq_select_path(T, 16, 37888, 3584) == tq.PATH_DECODE
+    # tensor-core path above the ridge
+    for M in (17, 32, 512, 2048, 8192):
+        assert tq.tq_select_path(T, M, 4096, 4096) == tq.PATH_PREFILL
+        assert tq.tq_select_path(W, M, 14336, 4096) == tq.PATH_PREFILL
+    # shapes / alignment the fast kernels do not take
+    assert tq.tq_select_path(T, 1, 4096, 4100) == tq.PATH_GENERIC
+    assert tq.tq_select_path(T, 1, 4096, 4096, aligned=False) == tq.PATH_GENERIC
+    assert tq.tq_select_path(T, 512, 4096, 4095) == tq.PATH_GENERIC
+    assert tq.tq_select_path(W, 1, 4096, 4000) == -2
+    assert tq.tq_select_path(T, 1, 4096, 0) == -2
+    assert tq.tq_select_path(5, 1, 4096, 4096) == -8

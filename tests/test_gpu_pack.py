@@ -1,0 +1,115 @@
+"""tq_quantize_pack / w4g_quantize_pack on the GPU must equal the oracle bit for bit."""
+import numpy as np
+import pytest
+import torch
+
+import bit_weight_only_tq_b200 as tq
+import oracle as O
+import tq_inputs as I
+from gpu_util import bits, gpu, need_cuda
+
+pytestmark = gpu
+
+
+def _check_tq(w_cpu, rows=None, offset=0):
+    need_cuda()
+    if offset:
+        buf = torch.zeros(w_cpu.numel() + offset, dtype=w_cpu.dtype, device="cuda")
+        buf[offset:] = w_cpu.reshape(-1).cuda()
+        wg = buf[offset:].view(w_cpu.shape)
+    else:
+        wg = w_cpu.cuda()
+    p, s = tq.tq_quantize_pack(wg)
+    torch.cuda.synchronize()
+    wn = w_cpu.numpy()
+    idx = np.arange(wn.shape[0]) if rows is None else np.asarray(rows)
+    pr, sr = O.tq_quantize_pack(wn[idx])
+    assert np.array_equal(p.cpu().numpy()[idx], pr), "packed bytes differ"
+    assert np.array_equal(bits(s)[idx], sr), "scales differ"
+
+
+def test_pack_config0_fp32_1024x1024():
+    _check_tq(I.weights(1024, 1024, I.seed_for(0, 0, 0)))
+
+
+def test_pack_fp16_rows():
+    _check_tq(I.weights(300, 3584, I.seed_for(4, 0, 1), dtype=torch.float16))
+
+
+@pytest.mark.parametrize("K", [1, 2, 3, 5, 63, 65, 1001, 4095])
+def test_pack_ragged_k(K):
+    _check_tq(I.weights(17, K, 77 + K))
+    _check_tq(I.weights(9, K, 78 + K, dtype=torch.float16))
+
+
+def test_pack_unaligned_input():
+    _check_tq(I.weights(33, 4096, 5), offset=1)
+    _check_tq(I.weights(33, 4096, 6, dtype=torch.float16), offset=3)
+
+
+def test_pack_adversarial_rows():
+    g = torch.Generator().manual_seed(11)
+    K = 2048
+    rows = []
+    rows.append(torch.zeros(K))                                           # all zero
+    rows.append(torch.full((K,), 0.02))                                   # constant
+    e = torch.randint(-140, 100, (K,), generator=g).float()
+    rows.append(torch.randn(K, generator=g) * torch.exp2(e))              # huge exponent range
+    sub = torch.randint(1, 2 ** 23, (K,), generator=g, dtype=torch.int32).view(torch.float32)
+    rows.append(sub)                                                      # fp32 subnormals only
+    one = torch.zeros(K)
+    one[777] = -3.0
+    rows.append(one)                                                      # a single nonzero
+    q = torch.randn(K, generator=g) * 0.02
+    q[::3] = 1e-30
+    rows.append(q)                                                        # many tiny values
+    w = torch.stack(rows).float()
+    _check_tq(w)
+    _check_tq(w.clamp(-60000, 60000).to(torch.float16))
+
+
+def test_pack_llama_gate_sampled_rows():
+    need_cuda()
+    w = I.weights(14336, 4096, I.seed_for(1, 0, 4), device="cuda")
+    p, s = tq.tq_quantize_pack(w)
+    torch.cuda.synchronize()
+    rows = np.random.default_rng(0).choice(14336, 48, replace=False)
+    rows = np.concatenate([rows, [0, 14335]])
+    wn = w[torch.as_tensor(rows, device="cuda")].cpu().numpy()
+    pr, sr = O.tq_quantize_pack(wn)
+    assert np.array_equal(p.cpu().numpy()[rows], pr)
+    assert np.array_equal(bits(s)[rows], sr)
+
+
+def _check_w4g(w_cpu, offset=0):
+    need_cuda()
+    if offset:
+        buf = torch.zeros(w_cpu.numel() + offset, dtype=w_cpu.dtype, device="cuda")
+        buf[offset:] = w_cpu.reshape(-1).cuda()
+        wg = buf[offset:].view(w_cpu.shape)
+    else:
+        wg = w_cpu.cuda()
+    qw, s = tq.w4g_quantize_pack(wg)
+    torch.cuda.synchronize()
+    qr, sr = O.w4g_quantize_pack(w_cpu.numpy())
+    assert np.array_equal(qw.cpu().numpy(), qr), "qweight differs"
+    assert np.array_equal(bits(s), sr), "scales differ"
+
+
+def test_w4g_pack_config3_outliers():
+    _check_w4g(I.weights(512, 4096, I.seed_for(3, 0, 0), outlier_frac=0.001, outlier_mult=10.0))
+
+
+def test_w4g_pack_fp16_and_unaligned():
+    _check_w4g(I.weights(64, 1024, 9, dtype=torch.float16))
+    _check_w4g(I.weights(40, 512, 10), offset=1)
+
+
+def test_w4g_pack_edge_groups():
+    w = torch.zeros(4, 256)
+    w[1, 0] = 9.6 * 2.0 ** -24           # subnormal scale, clamping to -8 / +7
+    w[1, 1] = -9.6 * 2.0 ** -24
+    s0 = 0.0999755859375
+    w[2, :6] = torch.tensor([7 * s0, 2.5 * s0, 3.5 * s0, -2.5 * s0, 0.5 * s0, -0.5 * s0])  # ties
+    w[3] = torch.randn(256, generator=torch.Generator().manual_seed(3)) * 1e4
+    _check_w4g(w)
