@@ -1,0 +1,548 @@
+"""Benchmark of the weight-only low-bit linear layer on B200.
+
+Headline workload (one "step"): the Llama-3-8B-shaped ternary decode sweep -- 32 distinct layers
+x 7 linears (q, k, v, o, gate, up, down) x M in {1, 4, 16} tokens, x ~ N(0,1) fp16, weights
+~ N(0, 0.02) ternarised and packed by tq_quantize_pack (1.745 GB packed, larger than L2, so no
+L2 flush is needed between steps).  Every GEMM goes through the public tq_gemm C-ABI call
+(path chosen by the library's dispatch); the 672 calls of a step are captured in CUDA graphs.
+
+metric: decode packed-weight GB/s (algorithmic bytes: packed weights + scales + x + y) ; the
+other hot-path rows (prefill TFLOP/s, W4A16, pack) are measured after the headline step and
+reported under "rows", each with its own roofline fraction.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--detail]
+
+With N > 1 (torchrun), every rank runs the same per-GPU workload on its own seeded weights
+(replicas, weak scaling; the path has no exchange step); time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode packed-weight GB/s & prefill TFLOP/s vs B200 roofline (1 GPU)"
+LLAMA = [("q_proj", 4096, 4096), ("k_proj", 1024, 4096), ("v_proj", 1024, 4096),
+         ("o_proj", 4096, 4096), ("gate_proj", 14336, 4096), ("up_proj", 14336, 4096),
+         ("down_proj", 4096, 14336)]
+DECODE_M = (1, 4, 16)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def decode_bytes(M, N, K, bias=False):
+    return N * K // 4 + 2 * N + 2 * M * K + 2 * M * N + (2 * N if bias else 0)
+
+
+def w4g_decode_bytes(M, N, K):
+    return N * K // 2 + 2 * N * (K // 128) + 2 * M * K + 2 * M * N
+
+
+class ClockSampler:
+    """Samples nvidia-smi clocks / throttle reasons while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.th = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.th = threading.Thread(target=self._read, daemon=True)
+        self.th.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.th:
+            self.th.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup():
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier_sync(world):
+    import torch
+    import torch.distributed as dist
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(v, world):
+    import torch
+    import torch.distributed as dist
+
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------------------------------------
+# our implementation
+# ------------------------------------------------------------------------------------------------
+def build_ternary_layers(rank, n_layers, config=1, shapes=LLAMA, dtype=None):
+    import torch
+
+    import bit_weight_only_tq_b200 as tq
+    import tq_inputs as I
+
+    layers = []
+    for l in range(n_layers):
+        row = []
+        for mid, (name, N, K) in enumerate(shapes):
+            w = I.weights(N, K, I.seed_for(config, l, mid) + 100003 * rank, device="cuda")
+            p, s = tq.tq_quantize_pack(w)
+            row.append((name, N, K, p, s))
+            del w
+        layers.append(row)
+    torch.cuda.synchronize()
+    return layers
+
+
+def capture(fn):
+    import torch
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()  # warm-up (also sets kernel attributes outside capture)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def time_graph(g, iters, warm=3):
+    import torch
+
+    for _ in range(warm):
+        g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(True), torch.cuda.Event(True)
+    a.record()
+    for _ in range(iters):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / iters
+
+
+def run_ours(args, world, rank, local):
+    import torch
+
+    import bit_weight_only_tq_b200 as tq
+    import tq_inputs as I
+
+    peaks, peak_src = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    n_layers = 32
+    layers = build_ternary_layers(rank, n_layers)
+
+    # inputs / outputs of a step: one x per (M, K); one output buffer per M (slices per GEMM)
+    Ks = sorted({K for _, _, K in LLAMA})
+    xs = {(M, K): I.activations(M, K, I.seed_for(1, 99, M) + K, device="cuda") for M in DECODE_M for K in Ks}
+    out_cols = n_layers * sum(N for _, N, _ in LLAMA)
+    ys = {M: torch.empty(M * out_cols, dtype=torch.float16, device="cuda") for M in DECODE_M}
+
+    def step_fn():
+        for M in DECODE_M:
+            off = 0
+            for row in layers:
+                for name, N, K, p, s in row:
+                    y = ys[M][off: off + M * N].view(M, N)
+                    tq.tq_gemm(xs[(M, K)], p, s, None, y)
+                    off += M * N
+
+    bytes_step = sum(decode_bytes(M, N, K) for M in DECODE_M for _ in range(n_layers) for _, N, K in LLAMA)
+    launches_step = len(DECODE_M) * n_layers * len(LLAMA)
+    g = capture(step_fn)
+    for _ in range(args.warmup):
+        g.replay()
+    barrier_sync(world)
+    clk = ClockSampler(local)
+    clk.start()
+    ev0, ev1 = torch.cuda.Event(True), torch.cuda.Event(True)
+    ev0.record()
+    for _ in range(args.steps):
+        g.replay()
+    ev1.record()
+    barrier_sync(world)
+    clocks = clk.stop()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    ms_max = max_over_ranks(ms, world)
+    value = bytes_step * world / (ms_max * 1e-3) / 1e9
+
+    # end-to-end through the public API: pinned-host x in, y out, every step
+    h_x = {k: v.cpu().pin_memory() for k, v in xs.items()}
+    h_y = {M: torch.empty(ys[M].numel(), dtype=torch.float16).pin_memory() for M in DECODE_M}
+    bi = sum(v.numel() * 2 for v in h_x.values())
+    bo = sum(v.numel() * 2 for v in h_y.values())
+
+    def e2e_step():
+        for k, v in h_x.items():
+            xs[k].copy_(v, non_blocking=True)
+        g.replay()
+        for M in DECODE_M:
+            h_y[M].copy_(ys[M], non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    barrier_sync(world)
+    e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
+    e0.record()
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record()
+    barrier_sync(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    e2e_val = bytes_step * world / (e2e_ms * 1e-3) / 1e9
+
+    # roofline of the dominant kernel (the decode GEMM is every launch of the step)
+    per_launch_us = ms * 1e3 / launches_step
+    achieved = bytes_step / launches_step / (per_launch_us * 1e-6) / 1e9
+    traffic = load_traffic()
+    roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+            "frac": round(achieved / hbm, 4), "traffic": traffic,
+            "kernel": "decode_gemm_kernel (ternary, mma.sync m16n8k16, TMA ring, cluster split-K)",
+            "peak_source": f"{peak_src} hbm_gbs"}
+
+    detail = {}
+    if args.detail and rank == 0:
+        detail = per_shape_detail(layers, xs)
+
+    rows = {}
+    if not args.no_rows:
+        rows = secondary_rows(args, rank, layers, peaks)
+
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic (seeded N(0,0.02) weights ternarised on the GPU; x ~ N(0,1) fp16)",
+        "config": {"workload": "Llama-3-8B-shaped ternary decode linears: 32 layers x "
+                               "{q,k,v,o 4096x4096/1024x4096, gate/up 14336x4096, down 4096x14336} "
+                               "x M in {1,4,16}",
+                   "layers": n_layers, "M": list(DECODE_M), "launches_per_step": launches_step,
+                   "bytes_per_step": bytes_step, "l2": "inputs larger than L2 (1.745 GB packed)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+                   "graph": "one CUDA graph per step, PDL between GEMMs"},
+        "roofline": roof,
+        "e2e": {"value": round(e2e_val, 1), "unit": "GB/s", "h2d_bytes_per_step": bi,
+                "d2h_bytes_per_step": bo, "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": launches_step * args.steps,
+        "clocks": clocks,
+        "rows": rows,
+    }
+    if detail:
+        result["detail"] = detail
+    if rank == 0 and world == 1 and not args.no_cpu:
+        result["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
+    return result
+
+
+def per_shape_detail(layers, xs):
+    import torch
+
+    import bit_weight_only_tq_b200 as tq
+
+    out = {}
+    for mid, (name, N, K) in enumerate(LLAMA):
+        for M in DECODE_M:
+            y = torch.empty(M, N, dtype=torch.float16, device="cuda")
+
+            def fn():
+                for row in layers:
+                    _, _, _, p, s = row[mid]
+                    tq.tq_gemm(xs[(M, K)], p, s, None, y)
+
+            g = capture(fn)
+            ms = time_graph(g, 10)
+            per = ms * 1e3 / len(layers)
+            out[f"{name} M={M}"] = {"us": round(per, 2),
+                                     "GB/s": round(decode_bytes(M, N, K) / (per * 1e-6) / 1e9, 1)}
+            del g
+    return out
+
+
+def secondary_rows(args, rank, layers, peaks):
+    """One measurement per remaining hot-path row (prefill, W4A16, pack), each timed on the GPU
+    with CUDA events over several launches of the public API."""
+    import torch
+
+    import bit_weight_only_tq_b200 as tq
+    import tq_inputs as I
+
+    hbm = float(peaks["hbm_gbs"])
+    tc = float(peaks["bf16_tflops"])
+    rows = {}
+    # ---- ternary prefill (config 2): 4 layers x 7 shapes, M = 2048, bias, outlier tokens
+    M = 2048
+    xs = {K: I.activations(M, K, I.seed_for(2, 0, K), device="cuda", outlier_row_frac=0.01)
+          for K in (4096, 14336)}
+    bs = {N: I.bias(N, I.seed_for(2, 1, N), device="cuda") for N in (1024, 4096, 14336)}
+    ys = {N: torch.empty(M, N, dtype=torch.float16, device="cuda") for N in (1024, 4096, 14336)}
+    sub = layers[:4]
+
+    def pf():
+        for row in sub:
+            for name, N, K, p, s in row:
+                tq.tq_gemm(xs[K], p, s, bs[N], ys[N])
+
+    g = capture(pf)
+    ms = time_graph(g, 3)
+    flops = sum(2 * M * N * K for row in sub for _, N, K, _, _ in row)
+    tf = flops / (ms * 1e-3) / 1e12
+    rows["ternary_prefill_M2048"] = {"value": round(tf, 1), "unit": "TFLOP/s", "frac": round(tf / tc, 4),
+                                     "peak": tc, "bound": "tensor", "sample": "4 layers x 7 shapes, M=2048"}
+    del g
+    # ---- W4A16 decode / prefill (config 3): 8 layers
+    w4 = []
+    for l in range(8):
+        row = []
+        for mid, (name, N, K) in enumerate(LLAMA):
+            w = I.weights(N, K, I.seed_for(3, l, mid) + 100003 * rank, device="cuda", outlier_frac=0.001)
+            qw, sc = tq.w4g_quantize_pack(w)
+            row.append((name, N, K, qw, sc))
+            del w
+        w4.append(row)
+    for M in (1, 16):
+        xq = {K: I.activations(M, K, I.seed_for(3, 2, K) + M, device="cuda") for K in (4096, 14336)}
+        yq = {N: torch.empty(M, N, dtype=torch.float16, device="cuda") for N in (1024, 4096, 14336)}
+
+        def wd():
+            for row in w4:
+                for name, N, K, qw, sc in row:
+                    tq.w4g_gemm(xq[K], qw, sc, None, yq[N])
+
+        g = capture(wd)
+        ms = time_graph(g, 20)
+        byts = sum(w4g_decode_bytes(M, N, K) for row in w4 for _, N, K, _, _ in row)
+        gbs = byts / (ms * 1e-3) / 1e9
+        rows[f"w4g_decode_M{M}"] = {"value": round(gbs, 1), "unit": "GB/s", "frac": round(gbs / hbm, 4),
+                                    "peak": hbm, "bound": "hbm", "sample": "8 layers x 7 shapes"}
+        del g
+    M = 4096
+    xq = {K: I.activations(M, K, I.seed_for(3, 3, K), device="cuda") for K in (4096, 14336)}
+    yq = {N: torch.empty(M, N, dtype=torch.float16, device="cuda") for N in (1024, 4096, 14336)}
+
+    def wp():
+        for name, N, K, qw, sc in w4[0]:
+            tq.w4g_gemm(xq[K], qw, sc, None, yq[N])
+
+    g = capture(wp)
+    ms = time_graph(g, 3)
+    flops = sum(2 * M * N * K for _, N, K, _, _ in w4[0])
+    tf = flops / (ms * 1e-3) / 1e12
+    rows["w4g_prefill_M4096"] = {"value": round(tf, 1), "unit": "TFLOP/s", "frac": round(tf / tc, 4),
+                                 "peak": tc, "bound": "tensor", "sample": "1 layer x 7 shapes, M=4096"}
+    del g, w4
+    # ---- pack throughput (config 4): Qwen2-7B fp16 weights, 2 layers x 4 shapes
+    qshapes = [(4608, 3584), (3584, 3584), (37888, 3584), (3584, 18944)]
+    tot_ms, tot_b = 0.0, 0
+    for l in range(2):
+        for mid, (N, K) in enumerate(qshapes):
+            w = I.weights(N, K, I.seed_for(4, l, mid), device="cuda", dtype=torch.float16)
+            p = torch.empty(N, K // 4, dtype=torch.uint8, device="cuda")
+            s = torch.empty(N, dtype=torch.float16, device="cuda")
+            tq.tq_quantize_pack(w, p, s)
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(True), torch.cuda.Event(True)
+            a.record()
+            for _ in range(3):
+                tq.tq_quantize_pack(w, p, s)
+            b.record()
+            torch.cuda.synchronize()
+            tot_ms += a.elapsed_time(b) / 3
+            tot_b += N * K * 2 + N * K // 4 + 2 * N
+            del w, p, s
+    gbs = tot_b / (tot_ms * 1e-3) / 1e9
+    rows["tq_quantize_pack_qwen2_fp16"] = {"value": round(gbs, 1), "unit": "GB/s", "frac": round(gbs / hbm, 4),
+                                           "peak": hbm, "bound": "hbm", "sample": "2 Qwen2-7B layers x 4 shapes"}
+    torch.cuda.synchronize()
+    return rows
+
+
+def load_traffic():
+    """DRAM bytes per decode launch from the committed ncu summary, if one matches this kernel."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("decode_gemm_bytes_per_launch")
+    except (OSError, ValueError):
+        return None
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU oracle (reference arm and cpu_baseline)
+# ------------------------------------------------------------------------------------------------
+def cpu_baseline(seconds=12.0):
+    """The oracle as it stands, on the host cores, on a bounded sample of the decode workload:
+    the first 1024 output rows of each layer-0 Llama linear (q, k, v, o, gate, up, down), packed
+    by the oracle, then oracle tq_gemm at M = 1, 4, 16 cycled until `seconds` of GEMM time."""
+    import oracle as O
+    import tq_inputs as I
+
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # noqa: BLE001
+        cores = os.cpu_count() or 1
+    rows = 1024
+    mats = []
+    for mid, (name, N, K) in enumerate(LLAMA):
+        w = I.weights(N, K, I.seed_for(1, 0, mid))[:rows].numpy()
+        p, s = O.tq_quantize_pack(w)
+        mats.append((name, min(N, rows), K, p, s))
+    xs = {(M, K): I.activations(M, K, 1).numpy() for M in DECODE_M for K in {4096, 14336}}
+    done_b, gemm_time, n_items = 0, 0.0, 0
+    while gemm_time < seconds:
+        name, N, K, p, s = mats[n_items % len(mats)]
+        M = DECODE_M[(n_items // len(mats)) % len(DECODE_M)]
+        t1 = time.perf_counter()
+        O.tq_gemm(xs[(M, K)], p, s, None, K)
+        gemm_time += time.perf_counter() - t1
+        done_b += decode_bytes(M, N, K)
+        n_items += 1
+    return {"value": round(done_b / gemm_time / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n_items} oracle tq_gemm calls on the first {rows} output rows of each layer-0 "
+                      f"Llama linear, M cycling 1/4/16 ({gemm_time:.1f} s of GEMM)"}
+
+
+def run_reference(args, world, rank):
+    """Reference arm: the CPU oracle timed on this host, same metric/config (bounded sample)."""
+    t0 = time.perf_counter()
+    per_step = []
+    res = None
+    for i in range(args.warmup + args.steps):
+        r = cpu_baseline(seconds=max(2.0, args.cpu_seconds / max(1, args.steps)))
+        if i >= args.warmup:
+            per_step.append(r)
+        res = r
+    val = statistics.median([r["value"] for r in per_step]) if per_step else res["value"]
+    return {
+        "metric": METRIC, "value": val, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (same seeds as the GPU arm)",
+        "config": {"workload": "Llama-3-8B-shaped ternary decode linears (oracle on a bounded sample)",
+                   "M": list(DECODE_M)},
+        "impl": "reference",
+        "cpu_baseline": {"value": val, "unit": "GB/s", "cores": res["cores"], "kind": "oracle",
+                         "sample": res["sample"]},
+        "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "wall_s": round(time.perf_counter() - t0, 1),
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--detail", action="store_true", help="per-shape decode breakdown")
+    ap.add_argument("--no-rows", action="store_true", help="skip the secondary hot-path rows")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, world, rank)), flush=True)
+        return 0
+
+    world, rank, local = dist_setup()
+    res = run_ours(args, world, rank, local)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

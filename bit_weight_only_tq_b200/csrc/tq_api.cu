@@ -14,6 +14,7 @@
 namespace tq {
 
 bool decode_supported(bool int4, int64_t M, int64_t N, int64_t K);
+static bool decode_ok(bool int4, int64_t M, int64_t N, int64_t K) { return decode_supported(int4, M, N, K); }
 bool prefill_supported(bool int4, int64_t M, int64_t N, int64_t K);
 
 static constexpr int kMaxDevices = 64;
@@ -120,7 +121,7 @@ int resolve_path(int fmt, int path, int64_t M, int64_t N, int64_t K, bool all_al
     case TQ_PATH_GENERIC:
       return TQ_PATH_GENERIC;
     case TQ_PATH_DECODE:
-      if (!tq::decode_supported(int4, M, N, K)) return TQ_ERR_PATH;
+      if (!tq::decode_ok(int4, M, N, K)) return TQ_ERR_PATH;
       return all_aligned ? static_cast<int>(TQ_PATH_DECODE) : static_cast<int>(TQ_ERR_ALIGN);
     case TQ_PATH_PREFILL:
       if (!tq::prefill_supported(int4, M, N, K)) return TQ_ERR_PATH;
@@ -159,7 +160,7 @@ int tq_select_path(int fmt, int64_t M, int64_t N, int64_t K, int aligned) {
   if (M == 0 || N == 0 || !aligned) return TQ_PATH_GENERIC;
   // Ridge of the fp16 tensor-core roofline: the decode kernel streams weights at HBM speed and
   // wins for skinny M; the tensor-core prefill kernel takes over above 16 tokens.
-  if (M <= 16 && tq::decode_supported(int4, M, N, K)) return TQ_PATH_DECODE;
+  if (M <= 16 && tq::decode_ok(int4, M, N, K)) return TQ_PATH_DECODE;
   if (tq::prefill_supported(int4, M, N, K)) return TQ_PATH_PREFILL;
   if (M <= 16) return TQ_PATH_GENERIC;
   return TQ_PATH_GENERIC;

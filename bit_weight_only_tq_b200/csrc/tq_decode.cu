@@ -4,24 +4,30 @@
 // of packed codes; [TQ] §4.2: codes are decoded into fp16 tensor-core fragments, accumulated in
 // fp32, and the per-row scale is applied after the MMA.
 //
-// Layout of the work (one CTA = 128 output rows x one K-slice; a cluster of S CTAs covers the
-// whole K of its 128 rows and reduces through distributed shared memory, in a fixed order):
-//   * warp 4 (one lane) streams 128-row x 128-byte tiles of packed weights with TMA (128-byte
-//     swizzle, so the 16-byte reads below are bank-conflict free) into a ring of stages; it
-//     starts before griddepcontrol.wait, since weights never depend on the previous kernel;
-//   * warps 0-3 each own 32 rows (two 16-row MMA tiles).  Weights are the A operand of
-//     mma.sync.m16n8k16 ("swap AB") and the tokens are the N=8 operand, so M <= 8 costs one MMA
-//     per 256 weights and M <= 16 two.
+// Work layout.  One CTA = 128 output rows x one K-slice; a cluster of S CTAs (S <= 8) covers
+// the whole K of its 128 rows and reduces through distributed shared memory in a fixed order
+// (deterministic, no global scratch).  Per CTA:
+//   * warps 0-3 (consumers) each own 32 rows = two 16-row MMA tiles.  Weights are the A operand
+//     of mma.sync.m16n8k16 ("swap AB"), the tokens the N = 8 operand: one MMA per 256 weights
+//     for M <= 8, two for M <= 16;
+//   * warp 4 (producer): lane 0 streams 128-row x 128-byte packed tiles with TMA (128-byte
+//     swizzle: the 16-byte fragment reads are bank-conflict free) into a ring, starting before
+//     griddepcontrol.wait because weights never depend on the previous kernel; all 32 lanes then
+//     copy the activations of each stage (cp.async, padded, conflict-free), rearrange them into
+//     ready-made B fragments in the k order the decode produces (byte permutes), and compute the
+//     per-token sums of x on the tensor core (an MMA with an all-ones A).
 //
-// In-register decode ("subnormal" trick).  Masking a packed word leaves small integers in the
-// fraction bits of each fp16 half, i.e. exact subnormal values c * 2^-24 (or c * 2^-22 when the
-// code sits two bits higher).  Per 32-bit word of 16 ternary codes: 3 shifts + 8 ANDs give 8
-// fp16x2 registers.  The 4x scale of the second mask position is folded into the activation
-// fragment (x/4), so every product carries the same 2^-24 and a single fp32 accumulator per
-// output suffices; the epilogue multiplies by 2^24 and subtracts sum_k x (codes are c = w + 1).
-// The order of k inside an MMA is permuted; the activation fragments are built (once per CTA,
-// in shared memory) in the matching order, so the weights are used in their canonical layout.
-// W4A16 uses the same scheme with 4-bit fields (masks 0x000F000F / 0x00F000F0, x/16 fold) and
+// In-register decode ("subnormal" trick).  ANDing a packed 32-bit word with 0x00030003 << 2p
+// leaves, in each fp16 half, the code at bits 2p..2p+1: the exact value c * 2^(2p-24) (fp16
+// subnormals for p <= 4, and still exactly linear for p = 5 where the code fills the two lowest
+// exponent bits).  Positions 6, 7 are shifted down by 12 first.  So one word of 16 codes costs
+// 1 shift + 8 ANDs for 8 fp16x2 registers, ~0.56 integer operations per weight.  The odd
+// positions carry an extra factor 4, folded into their activation fragments (x / 4); the
+// remaining factors 2^-24, 2^-20, 2^-16 are kept apart in separate accumulators and applied
+// exactly (powers of two) in the epilogue, which also subtracts sum_k x (codes are c = w + 1).
+// One accumulator per position pair keeps the dependent MMA chains short (latency, not issue,
+// bounds a skinny GEMM).
+// W4A16 uses the same scheme with 4-bit fields (masks 0x000F000F / 0x00F000F0, x / 16 fold) and
 // one 128-wide quantisation group per 64-byte sub-chunk: y += s[n,g] * (2^24 * C_g - 8 sum_g x).
 #include <cuda.h>
 #include <cuda_fp16.h>
@@ -32,12 +38,27 @@
 
 namespace tq {
 
-constexpr int kDRows = 128;                      // output rows per CTA
-constexpr int kDConsumers = 4;                   // consumer warps (32 rows each)
+constexpr int kDRows = 128;                 // output rows per CTA
+constexpr int kDConsumers = 4;              // consumer warps (32 rows each)
 constexpr int kDThreads = (kDConsumers + 1) * 32;
-constexpr int kDStageBytes = kDRows * 128;       // one TMA box: 128 rows x 128 bytes
-constexpr int kDMaxRing = 4;
+constexpr int kDStageBytes = kDRows * 128;  // one TMA box: 128 rows x 128 bytes
+constexpr int kDMaxRing = 6;                // weight stages resident in shared memory
+constexpr int kDXRing = 2;                  // activation-fragment stages
 constexpr int kDMaxCluster = 8;
+constexpr int kDRedRows = kDRows + kDMaxCluster;  // >= S * ceil(128 / S)
+constexpr int kDSmemBudget = 113 * 1024;    // two CTAs per SM
+
+template <bool kInt4>
+struct DecFmt {
+  static constexpr int kStageK = kInt4 ? 256 : 512;  // codes per stage (128 bytes of a row)
+  static constexpr int kSubK = kStageK / 2;          // codes per 64-byte sub-chunk
+  static constexpr int kLaneK = kSubK / 4;           // codes per lane (16 bytes) per sub-chunk
+  static constexpr int kMmas = kInt4 ? 8 : 16;       // MMAs per 16-row tile per sub-chunk
+  static constexpr int kFragU4 = kMmas / 2;          // uint4 B fragments per lane per sub-chunk
+  static constexpr int kFragBytes = kFragU4 * 32 * 16;
+  static constexpr int kXLaneBytes = kLaneK * 2;     // activation bytes per lane per sub-chunk
+  static constexpr int kXStride = kXLaneBytes + 16;  // padded: conflict-free 16-byte reads
+};
 
 struct DecodeArgs {
   const __half* x;
@@ -45,339 +66,419 @@ struct DecodeArgs {
   const __half* bias;  // may be null
   __half* y;
   int64_t M, N, K;
-  int C;          // stages along K (128 packed bytes of every row per stage)
-  int S;          // CTAs per cluster (K-slices)
-  int ring;       // stages resident in shared memory
-  int max_local;  // ceil(C / S)
-};
-
-template <bool kInt4>
-struct DecFmt {
-  static constexpr int kSubK = kInt4 ? 128 : 256;   // codes per 64-byte sub-chunk
-  static constexpr int kLaneK = kInt4 ? 32 : 64;     // codes per lane (16 bytes) per sub-chunk
-  static constexpr int kMmas = kInt4 ? 8 : 16;       // MMAs per 16-row tile per sub-chunk
-  static constexpr int kFragU4 = kMmas / 2;          // uint4 activation fragments per lane
-  static constexpr int kFragBytes = kFragU4 * 32 * 16;
-};
-
-struct DecodeSmem {
-  uint8_t* stage;
-  uint4* xf;
-  float* sx;
-  float* part;
-  uint64_t* full;
-  uint64_t* empty;
+  int C;     // stages along K
+  int S;     // CTAs per cluster (K-slices)
+  int ring;  // weight stages resident in shared memory (all of a CTA's stages when they fit)
 };
 
 template <bool kInt4, int NT>
-__device__ __forceinline__ DecodeSmem decode_smem_carve(uint8_t* base, const DecodeArgs& a) {
-  DecodeSmem s;
-  uint8_t* p = base;
-  s.stage = p;
-  p += a.ring * kDStageBytes;
-  const int nsub = 2 * a.max_local;
-  s.xf = reinterpret_cast<uint4*>(p);
-  p += nsub * NT * DecFmt<kInt4>::kFragBytes;
-  s.sx = reinterpret_cast<float*>(p);
-  p += nsub * 16 * sizeof(float);
-  s.part = reinterpret_cast<float*>(p);
-  p += kDRows * 16 * sizeof(float);
-  s.full = reinterpret_cast<uint64_t*>(p);
-  p += kDMaxRing * sizeof(uint64_t);
-  s.empty = reinterpret_cast<uint64_t*>(p);
-  return s;
-}
-
-__host__ __device__ constexpr int decode_smem_bytes(bool int4, int NT, int ring, int max_local) {
-  return 1024 /* alignment slack */ + ring * kDStageBytes +
-         2 * max_local * NT * (int4 ? 8 * 32 * 8 : 16 * 32 * 8) + 2 * max_local * 16 * 4 +
-         kDRows * 16 * 4 + 2 * kDMaxRing * 8;
-}
-
-__device__ __forceinline__ uint32_t h2_bits(__half2 v) { return *reinterpret_cast<uint32_t*>(&v); }
+struct DecLayout {
+  using F = DecFmt<kInt4>;
+  static constexpr int kXfStage = 2 * NT * F::kFragBytes;
+  static constexpr int kXgStage = kInt4 ? 2 * 16 * 4 : 0;
+  static constexpr int kXsBuf = 2 * NT * 32 * F::kXStride;
+  static constexpr int kRed = kDRedRows * 16 * 4;
+  static constexpr int kSxr = kDMaxCluster * 16 * 4;
+  __host__ __device__ static constexpr int bytes(int ring) {
+    return 1024 + ring * kDStageBytes + kDXRing * (kXfStage + kXgStage) + 2 * kXsBuf + kRed + kSxr +
+           (2 * kDMaxRing + 2 * kDXRing) * 8;
+  }
+};
 
 template <bool kInt4, int NT>
 __global__ void __launch_bounds__(kDThreads)
     decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeArgs a) {
-  extern __shared__ uint8_t smem_raw[];
   using F = DecFmt<kInt4>;
+  using L = DecLayout<kInt4, NT>;
+  extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const DecodeSmem sm = decode_smem_carve<kInt4, NT>(base, a);
+  uint8_t* wst = base;                                                // ring x 16 KB weight tiles
+  uint8_t* xf = wst + a.ring * kDStageBytes;                          // 2 x B fragments
+  float* xg = reinterpret_cast<float*>(xf + kDXRing * L::kXfStage);   // 2 x [2][16] group sums
+  uint8_t* xs = reinterpret_cast<uint8_t*>(xg) + kDXRing * L::kXgStage;  // 2 x natural x
+  float* red = reinterpret_cast<float*>(xs + 2 * L::kXsBuf);          // [S][rows/S][16] partials
+  float* sxr = red + kDRedRows * 16;                                  // [S][16] slice sums of x
+  uint64_t* wfull = reinterpret_cast<uint64_t*>(sxr + kDMaxCluster * 16);
+  uint64_t* wempty = wfull + kDMaxRing;
+  uint64_t* xfull = wempty + kDMaxRing;
+  uint64_t* xempty = xfull + kDXRing;
 
   pdl_allow_dependents();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
   const int rank = static_cast<int>(cluster_ctarank());
   const int rb = blockIdx.y;
   const int st_begin = static_cast<int>((static_cast<int64_t>(rank) * a.C) / a.S);
   const int st_end = static_cast<int>((static_cast<int64_t>(rank + 1) * a.C) / a.S);
   const int nst = st_end - st_begin;
+  const int own_cap = (kDRows + a.S - 1) / a.S;  // row slots per owner in `red`
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < a.ring; ++i) {
-      mbar_init(&sm.full[i], 1);
-      mbar_init(&sm.empty[i], kDConsumers);
+      mbar_init(&wfull[i], 1);
+      mbar_init(&wempty[i], kDConsumers);
+    }
+    for (int i = 0; i < kDXRing; ++i) {
+      mbar_init(&xfull[i], 32);
+      mbar_init(&xempty[i], kDConsumers);
     }
     fence_mbar_init();
   }
   __syncthreads();
 
   if (warp == kDConsumers) {
-    // ------------------------------------------------------------- producer: weight tiles
+    // ================================================================== producer warp
     if (lane == 0) {
       tma_prefetch_desc(&tmap);
-      for (int i = 0; i < nst; ++i) {
-        const int slot = i % a.ring;
-        if (i >= a.ring && !mbar_wait(&sm.empty[slot], static_cast<uint32_t>((i / a.ring) - 1) & 1u)) break;
-        mbar_arrive_expect_tx(&sm.full[slot], kDStageBytes);
-        tma_load_2d(sm.stage + slot * kDStageBytes, &tmap, &sm.full[slot], (st_begin + i) * 128,
-                    rb * kDRows);
+      const int pre = nst < a.ring ? nst : a.ring;
+      for (int i = 0; i < pre; ++i) {
+        mbar_arrive_expect_tx(&wfull[i], kDStageBytes);
+        tma_load_2d(wst + i * kDStageBytes, &tmap, &wfull[i], (st_begin + i) * 128, rb * kDRows);
       }
     }
-    pdl_wait_prior_grids();  // this warp also writes y in the epilogue
-  } else {
-    // ------------------------------------------------------------- consumers
-    const int g = lane >> 2, t = lane & 3;
-    pdl_wait_prior_grids();  // x (and y) may belong to the previous kernel in the stream
+    pdl_wait_prior_grids();  // activations may come from the previous kernel
 
-    // Stage the activation fragments of this CTA's K-slice, in MMA order.
-    const int nsub = 2 * nst;
-    for (int p = warp; p < nsub * NT; p += kDConsumers) {
-      const int scl = p / NT, T = p - scl * NT;
-      const int m = 8 * T + g;
-      const int64_t kb = static_cast<int64_t>(st_begin * 2 + scl) * F::kSubK + t * F::kLaneK;
-      __align__(16) __half X[F::kLaneK];
-      if (m < a.M && kb + F::kLaneK <= a.K) {
-        const uint4* src = reinterpret_cast<const uint4*>(a.x + m * a.K + kb);
+    auto issue_x = [&](int i) {
+      if (i < nst) {
+        uint8_t* buf = xs + (i & 1) * L::kXsBuf;
 #pragma unroll
-        for (int i = 0; i < F::kLaneK / 8; ++i) reinterpret_cast<uint4*>(X)[i] = __ldg(src + i);
-      } else {
+        for (int sub = 0; sub < 2; ++sub)
 #pragma unroll
-        for (int i = 0; i < F::kLaneK; ++i)
-          X[i] = (m < a.M && kb + i < a.K) ? a.x[m * a.K + kb + i] : __float2half_rn(0.0f);
+          for (int T = 0; T < NT; ++T) {
+            const int m = 8 * T + g;
+            const int64_t k0 = static_cast<int64_t>(st_begin + i) * F::kStageK + sub * F::kSubK + t * F::kLaneK;
+            const bool valid = (m < a.M) && (k0 < a.K);
+            const __half* src = valid ? a.x + m * a.K + k0 : a.x;
+            uint8_t* dst = buf + ((sub * NT + T) * 32 + lane) * F::kXStride;
+#pragma unroll
+            for (int j = 0; j < F::kXLaneBytes / 16; ++j)
+              cp_async_16(dst + 16 * j, src + (valid ? 8 * j : 0), valid ? 16u : 0u);
+          }
       }
-      float sum = 0.0f;
+      cp_async_commit();  // one group per stage (possibly empty) keeps the accounting uniform
+    };
+    issue_x(0);
+    issue_x(1);
+
+    const uint32_t ONE = 0x3C003C00u, FOUR = 0x44004400u, SIXTEEN = 0x4C004C00u;
+    const __half2 q4 = __floats2half2_rn(0.25f, 0.25f);
+    const __half2 q16 = __floats2half2_rn(0.0625f, 0.0625f);
+    float ssum[NT][4][4];  // four independent MMA chains per token tile
 #pragma unroll
-      for (int i = 0; i < F::kLaneK; ++i) sum += __half2float(X[i]);
-      sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
-      sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
-      if (t == 0) sm.sx[scl * 16 + m] = sum;
-      const __half2 q4 = __floats2half2_rn(0.25f, 0.25f);
-      const __half2 q16 = __floats2half2_rn(0.0625f, 0.0625f);
+    for (int T = 0; T < NT; ++T)
 #pragma unroll
-      for (int ip = 0; ip < F::kFragU4; ++ip) {
-        uint32_t r[4];
+      for (int j = 0; j < 4; ++j)
 #pragma unroll
-        for (int cls = 0; cls < 2; ++cls) {
-          __half2 b01, b23;
-          if (!kInt4) {
-            const int h = ip >> 2, s = ip & 3, pp = 2 * s + cls;
-            b01 = __halves2half2(X[32 * h + pp], X[32 * h + 8 + pp]);
-            b23 = __halves2half2(X[32 * h + 16 + pp], X[32 * h + 24 + pp]);
-            if (cls) {
-              b01 = __hmul2(b01, q4);
-              b23 = __hmul2(b23, q4);
+        for (int c = 0; c < 4; ++c) ssum[T][j][c] = 0.0f;
+
+    for (int i = 0; i < nst; ++i) {
+      const int xslot = i & 1;
+      if (i >= kDXRing) {
+        // consumers are done with stage i-2: its fragment slot and its weight slot are free
+        if (!mbar_wait(&xempty[xslot], static_cast<uint32_t>((i >> 1) - 1) & 1u)) break;
+        const int j = i - kDXRing + a.ring;  // refill the freed weight slot with stage j
+        if (j >= a.ring && j < nst) {
+          const int ws = j % a.ring;
+          if (!mbar_wait(&wempty[ws], static_cast<uint32_t>((j / a.ring) - 1) & 1u)) break;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&wfull[ws], kDStageBytes);
+            tma_load_2d(wst + ws * kDStageBytes, &tmap, &wfull[ws], (st_begin + j) * 128, rb * kDRows);
+          }
+        }
+      }
+      cp_async_wait<1>();  // this lane's copies of stage i have landed
+      const uint8_t* buf = xs + (i & 1) * L::kXsBuf;
+      uint4* xfs = reinterpret_cast<uint4*>(xf + xslot * L::kXfStage);
+#pragma unroll
+      for (int sub = 0; sub < 2; ++sub)
+#pragma unroll
+        for (int T = 0; T < NT; ++T) {
+          const uint4* src = reinterpret_cast<const uint4*>(buf + ((sub * NT + T) * 32 + lane) * F::kXStride);
+          uint32_t P[F::kLaneK / 2];
+#pragma unroll
+          for (int j = 0; j < F::kLaneK / 8; ++j) {
+            const uint4 v = src[j];
+            P[4 * j] = v.x;
+            P[4 * j + 1] = v.y;
+            P[4 * j + 2] = v.z;
+            P[4 * j + 3] = v.w;
+          }
+          float cg[4][4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) cg[j][c] = 0.0f;
+#pragma unroll
+          for (int f = 0; f < F::kFragU4; ++f) {
+            uint32_t Pa, Pb, Pc, Pd;
+            if (!kInt4) {  // f = h*4 + pp: positions p = 2pp (even), 2pp+1 (odd) of word pair h
+              const int h = f >> 2, pp = f & 3;
+              Pa = P[16 * h + pp];
+              Pb = P[16 * h + 4 + pp];
+              Pc = P[16 * h + 8 + pp];
+              Pd = P[16 * h + 12 + pp];
+            } else {       // f = h*2 + s: nibble positions 2s (class 0), 2s+1 (class 1)
+              const int h = f >> 1, s = f & 1;
+              Pa = P[8 * h + s];
+              Pb = P[8 * h + 2 + s];
+              Pc = P[8 * h + 4 + s];
+              Pd = P[8 * h + 6 + s];
             }
-          } else {
-            const int h = ip >> 1, s = ip & 1, pp = 2 * s + cls;
-            b01 = __halves2half2(X[16 * h + pp], X[16 * h + 4 + pp]);
-            b23 = __halves2half2(X[16 * h + 8 + pp], X[16 * h + 12 + pp]);
-            if (cls) {
-              b01 = __hmul2(b01, q16);
-              b23 = __hmul2(b23, q16);
+            const uint32_t e01 = __byte_perm(Pa, Pb, 0x5410), e23 = __byte_perm(Pc, Pd, 0x5410);
+            const uint32_t o01 = __byte_perm(Pa, Pb, 0x7632), o23 = __byte_perm(Pc, Pd, 0x7632);
+            __half2 so01 = *reinterpret_cast<const __half2*>(&o01);
+            __half2 so23 = *reinterpret_cast<const __half2*>(&o23);
+            so01 = __hmul2(so01, kInt4 ? q16 : q4);
+            so23 = __hmul2(so23, kInt4 ? q16 : q4);
+            const uint32_t s01 = *reinterpret_cast<const uint32_t*>(&so01);
+            const uint32_t s23 = *reinterpret_cast<const uint32_t*>(&so23);
+            xfs[((sub * NT + T) * F::kFragU4 + f) * 32 + lane] = make_uint4(e01, e23, s01, s23);
+            // sum_k x on the tensor core: A = all ones (x4 / x16 undoes the fold)
+            const uint32_t up = kInt4 ? SIXTEEN : FOUR;
+            if (!kInt4) {
+              mma_16816(ssum[T][(2 * f) & 3], ONE, ONE, ONE, ONE, e01, e23);
+              mma_16816(ssum[T][(2 * f + 1) & 3], up, up, up, up, s01, s23);
+            } else {
+              mma_16816(cg[(2 * f) & 3], ONE, ONE, ONE, ONE, e01, e23);
+              mma_16816(cg[(2 * f + 1) & 3], up, up, up, up, s01, s23);
             }
           }
-          r[2 * cls] = h2_bits(b01);
-          r[2 * cls + 1] = h2_bits(b23);
+          if (kInt4 && g == 0) {  // row 0 of the all-ones product holds the token sums
+            xg[(xslot * 2 + sub) * 16 + 8 * T + 2 * t] = (cg[0][0] + cg[1][0]) + (cg[2][0] + cg[3][0]);
+            xg[(xslot * 2 + sub) * 16 + 8 * T + 2 * t + 1] = (cg[0][1] + cg[1][1]) + (cg[2][1] + cg[3][1]);
+          }
         }
-        sm.xf[((scl * NT + T) * F::kFragU4 + ip) * 32 + lane] = make_uint4(r[0], r[1], r[2], r[3]);
+      mbar_arrive(&xfull[xslot]);
+      issue_x(i + 2);
+    }
+    cp_async_wait<0>();
+    if (!kInt4 && g == 0) {  // push this slice's token sums of x to every CTA of the cluster
+      const uint32_t loc = smem_u32(sxr + rank * 16);
+#pragma unroll
+      for (int T = 0; T < NT; ++T) {
+        const float s0 = (ssum[T][0][0] + ssum[T][1][0]) + (ssum[T][2][0] + ssum[T][3][0]);
+        const float s1 = (ssum[T][0][1] + ssum[T][1][1]) + (ssum[T][2][1] + ssum[T][3][1]);
+        for (int q = 0; q < a.S; ++q) {
+          st_shared_cluster_f32(mapa_shared(loc + (8 * T + 2 * t) * 4, q), s0);
+          st_shared_cluster_f32(mapa_shared(loc + (8 * T + 2 * t + 1) * 4, q), s1);
+        }
       }
     }
-    asm volatile("bar.sync 1, %0;" ::"n"(kDConsumers * 32) : "memory");
-
-    float acc[2][NT][4];
+  } else {
+    // ================================================================== consumer warps
+    constexpr int NG = kInt4 ? 1 : 4;  // accumulator groups: one per position pair (chains)
+    float acc[NG][2][NT][4];
 #pragma unroll
-    for (int rt = 0; rt < 2; ++rt)
+    for (int q = 0; q < NG; ++q)
 #pragma unroll
-      for (int T = 0; T < NT; ++T)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) acc[rt][T][c] = 0.0f;
-
-    const int64_t G = a.K >> 7;
-    for (int i = 0; i < nst; ++i) {
-      const int slot = i % a.ring;
-      if (!mbar_wait(&sm.full[slot], static_cast<uint32_t>(i / a.ring) & 1u)) break;
-      const uint8_t* st = sm.stage + slot * kDStageBytes;
-#pragma unroll
-      for (int sub = 0; sub < 2; ++sub) {
-        const int scl = 2 * i + sub;
-        uint4 bf[NT][F::kFragU4];
+      for (int rt = 0; rt < 2; ++rt)
 #pragma unroll
         for (int T = 0; T < NT; ++T)
 #pragma unroll
-          for (int ip = 0; ip < F::kFragU4; ++ip)
-            bf[T][ip] = sm.xf[((scl * NT + T) * F::kFragU4 + ip) * 32 + lane];
-        float xg[NT][2];
-        int64_t gi = 0;
-        if (kInt4) {
-          gi = static_cast<int64_t>(st_begin + i) * 2 + sub;
+          for (int c = 0; c < 4; ++c) acc[q][rt][T][c] = 0.0f;
+    const int64_t G = a.K >> 7;
+
+    for (int i = 0; i < nst; ++i) {
+      const int ws = i % a.ring, xslot = i & 1;
+      if (!mbar_wait(&wfull[ws], static_cast<uint32_t>(i / a.ring) & 1u) ||
+          !mbar_wait(&xfull[xslot], static_cast<uint32_t>(i >> 1) & 1u))
+        break;
+      const uint8_t* st = wst + ws * kDStageBytes;
+      const uint4* xfs = reinterpret_cast<const uint4*>(xf + xslot * L::kXfStage);
 #pragma unroll
-          for (int T = 0; T < NT; ++T) {
-            xg[T][0] = 8.0f * sm.sx[scl * 16 + 8 * T + 2 * t];
-            xg[T][1] = 8.0f * sm.sx[scl * 16 + 8 * T + 2 * t + 1];
-          }
-        }
+      for (int sub = 0; sub < 2; ++sub) {
         const int chunk = sub * 4 + t;
+        uint32_t w0[2][4], w1[2][4];
 #pragma unroll
         for (int rt = 0; rt < 2; ++rt) {
           const int r0 = warp * 32 + rt * 16 + g, r1 = r0 + 8;
           const uint4 U0 = *reinterpret_cast<const uint4*>(st + r0 * 128 + ((chunk ^ (r0 & 7)) << 4));
           const uint4 U1 = *reinterpret_cast<const uint4*>(st + r1 * 128 + ((chunk ^ (r1 & 7)) << 4));
-          const uint32_t w0[4] = {U0.x, U0.y, U0.z, U0.w};
-          const uint32_t w1[4] = {U1.x, U1.y, U1.z, U1.w};
-          if (!kInt4) {
+          w0[rt][0] = U0.x; w0[rt][1] = U0.y; w0[rt][2] = U0.z; w0[rt][3] = U0.w;
+          w1[rt][0] = U1.x; w1[rt][1] = U1.y; w1[rt][2] = U1.z; w1[rt][3] = U1.w;
+        }
+        if (!kInt4) {
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
+          for (int h = 0; h < 2; ++h) {
+            uint32_t sh[2][4];
 #pragma unroll
-              for (int s = 0; s < 4; ++s) {
-                const uint32_t x0 = w0[2 * h] >> (4 * s), x1 = w1[2 * h] >> (4 * s);
-                const uint32_t x2 = w0[2 * h + 1] >> (4 * s), x3 = w1[2 * h + 1] >> (4 * s);
+            for (int rt = 0; rt < 2; ++rt) {
+              sh[rt][0] = w0[rt][2 * h] >> 12;
+              sh[rt][1] = w1[rt][2 * h] >> 12;
+              sh[rt][2] = w0[rt][2 * h + 1] >> 12;
+              sh[rt][3] = w1[rt][2 * h + 1] >> 12;
+            }
 #pragma unroll
-                for (int cls = 0; cls < 2; ++cls) {
-                  const uint32_t mk = cls ? 0x000C000Cu : 0x00030003u;
-                  const int ip = h * 4 + s;
+            for (int pp = 0; pp < 4; ++pp) {
+              uint4 B[NT];
 #pragma unroll
-                  for (int T = 0; T < NT; ++T) {
-                    const uint32_t b0 = cls ? bf[T][ip].z : bf[T][ip].x;
-                    const uint32_t b1 = cls ? bf[T][ip].w : bf[T][ip].y;
-                    mma_16816(acc[rt][T], x0 & mk, x1 & mk, x2 & mk, x3 & mk, b0, b1);
+              for (int T = 0; T < NT; ++T) B[T] = xfs[((sub * NT + T) * 8 + h * 4 + pp) * 32 + lane];
+#pragma unroll
+              for (int q = 0; q < 2; ++q) {
+                const int p = 2 * pp + q;
+#pragma unroll
+                for (int rt = 0; rt < 2; ++rt) {
+                  uint32_t a0, a1, a2, a3;
+                  if (p < 6) {
+                    const uint32_t mk = 0x00030003u << (2 * p);
+                    a0 = w0[rt][2 * h] & mk;
+                    a1 = w1[rt][2 * h] & mk;
+                    a2 = w0[rt][2 * h + 1] & mk;
+                    a3 = w1[rt][2 * h + 1] & mk;
+                  } else {
+                    const uint32_t mk = (p == 6) ? 0x00030003u : 0x000C000Cu;
+                    a0 = sh[rt][0] & mk;
+                    a1 = sh[rt][1] & mk;
+                    a2 = sh[rt][2] & mk;
+                    a3 = sh[rt][3] & mk;
                   }
+#pragma unroll
+                  for (int T = 0; T < NT; ++T)
+                    mma_16816(acc[pp % NG][rt][T], a0, a1, a2, a3, q ? B[T].z : B[T].x, q ? B[T].w : B[T].y);
                 }
               }
-          } else {
-            float cg[NT][4];
+            }
+          }
+        } else {
+          const int64_t gi = static_cast<int64_t>(st_begin + i) * 2 + sub;
+          const float* xgs = xg + (xslot * 2 + sub) * 16;
+          float xgt[NT][2];
 #pragma unroll
-            for (int T = 0; T < NT; ++T)
+          for (int T = 0; T < NT; ++T) {
+            xgt[T][0] = 8.0f * xgs[8 * T + 2 * t];
+            xgt[T][1] = 8.0f * xgs[8 * T + 2 * t + 1];
+          }
 #pragma unroll
-              for (int c = 0; c < 4; ++c) cg[T][c] = 0.0f;
+          for (int rt = 0; rt < 2; ++rt) {
+            float cg[2][NT][4];  // two chains (class 0 / class 1 fields)
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+              for (int T = 0; T < NT; ++T)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) cg[j][T][c] = 0.0f;
 #pragma unroll
             for (int h = 0; h < 2; ++h)
 #pragma unroll
               for (int s = 0; s < 2; ++s) {
-                const uint32_t x0 = w0[2 * h] >> (8 * s), x1 = w1[2 * h] >> (8 * s);
-                const uint32_t x2 = w0[2 * h + 1] >> (8 * s), x3 = w1[2 * h + 1] >> (8 * s);
+                const uint32_t x0 = w0[rt][2 * h] >> (8 * s), x1 = w1[rt][2 * h] >> (8 * s);
+                const uint32_t x2 = w0[rt][2 * h + 1] >> (8 * s), x3 = w1[rt][2 * h + 1] >> (8 * s);
+                uint4 B[NT];
+#pragma unroll
+                for (int T = 0; T < NT; ++T) B[T] = xfs[((sub * NT + T) * 4 + h * 2 + s) * 32 + lane];
 #pragma unroll
                 for (int cls = 0; cls < 2; ++cls) {
                   const uint32_t mk = cls ? 0x00F000F0u : 0x000F000Fu;
-                  const int ip = h * 2 + s;
 #pragma unroll
-                  for (int T = 0; T < NT; ++T) {
-                    const uint32_t b0 = cls ? bf[T][ip].z : bf[T][ip].x;
-                    const uint32_t b1 = cls ? bf[T][ip].w : bf[T][ip].y;
-                    mma_16816(cg[T], x0 & mk, x1 & mk, x2 & mk, x3 & mk, b0, b1);
-                  }
+                  for (int T = 0; T < NT; ++T)
+                    mma_16816(cg[cls][T], x0 & mk, x1 & mk, x2 & mk, x3 & mk, cls ? B[T].z : B[T].x,
+                              cls ? B[T].w : B[T].y);
                 }
               }
-            const int64_t n0 = static_cast<int64_t>(rb) * kDRows + r0, n1 = n0 + 8;
+            const int64_t n0 = static_cast<int64_t>(rb) * kDRows + warp * 32 + rt * 16 + g, n1 = n0 + 8;
             // groups past K (a zero-filled half stage) contribute nothing
             const float s0 = (n0 < a.N && gi < G) ? __half2float(a.sc[n0 * G + gi]) : 0.0f;
             const float s1 = (n1 < a.N && gi < G) ? __half2float(a.sc[n1 * G + gi]) : 0.0f;
 #pragma unroll
             for (int T = 0; T < NT; ++T) {
-              acc[rt][T][0] = fmaf(s0, fmaf(cg[T][0], 16777216.0f, -xg[T][0]), acc[rt][T][0]);
-              acc[rt][T][1] = fmaf(s0, fmaf(cg[T][1], 16777216.0f, -xg[T][1]), acc[rt][T][1]);
-              acc[rt][T][2] = fmaf(s1, fmaf(cg[T][2], 16777216.0f, -xg[T][0]), acc[rt][T][2]);
-              acc[rt][T][3] = fmaf(s1, fmaf(cg[T][3], 16777216.0f, -xg[T][1]), acc[rt][T][3]);
+              float c4[4];
+#pragma unroll
+              for (int c = 0; c < 4; ++c) c4[c] = cg[0][T][c] + cg[1][T][c];
+              acc[0][rt][T][0] = fmaf(s0, fmaf(c4[0], 16777216.0f, -xgt[T][0]), acc[0][rt][T][0]);
+              acc[0][rt][T][1] = fmaf(s0, fmaf(c4[1], 16777216.0f, -xgt[T][1]), acc[0][rt][T][1]);
+              acc[0][rt][T][2] = fmaf(s1, fmaf(c4[2], 16777216.0f, -xgt[T][0]), acc[0][rt][T][2]);
+              acc[0][rt][T][3] = fmaf(s1, fmaf(c4[3], 16777216.0f, -xgt[T][1]), acc[0][rt][T][3]);
             }
           }
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.empty[slot]);
-    }
-
-    // partial results of this K-slice -> shared memory part[row][token]
-    float sxt[NT][2];
-#pragma unroll
-    for (int T = 0; T < NT; ++T) {
-      sxt[T][0] = 0.0f;
-      sxt[T][1] = 0.0f;
-      if (!kInt4) {
-        for (int scl = 0; scl < nsub; ++scl) {
-          sxt[T][0] += sm.sx[scl * 16 + 8 * T + 2 * t];
-          sxt[T][1] += sm.sx[scl * 16 + 8 * T + 2 * t + 1];
-        }
+      if (lane == 0) {
+        mbar_arrive(&wempty[ws]);
+        mbar_arrive(&xempty[xslot]);
       }
     }
+    // push this slice's partial results to the CTA that owns each row (the rows of the row block
+    // are split evenly over the cluster: owner q holds rows [q*128/S, (q+1)*128/S))
+    const uint32_t red_local = smem_u32(red);
 #pragma unroll
-    for (int rt = 0; rt < 2; ++rt) {
-      const int r0 = warp * 32 + rt * 16 + g, r1 = r0 + 8;
+    for (int rt = 0; rt < 2; ++rt)
 #pragma unroll
-      for (int T = 0; T < NT; ++T) {
-        const int m0 = 8 * T + 2 * t;
-        if (!kInt4) {
-          sm.part[r0 * 16 + m0] = fmaf(acc[rt][T][0], 16777216.0f, -sxt[T][0]);
-          sm.part[r0 * 16 + m0 + 1] = fmaf(acc[rt][T][1], 16777216.0f, -sxt[T][1]);
-          sm.part[r1 * 16 + m0] = fmaf(acc[rt][T][2], 16777216.0f, -sxt[T][0]);
-          sm.part[r1 * 16 + m0 + 1] = fmaf(acc[rt][T][3], 16777216.0f, -sxt[T][1]);
-        } else {
-          sm.part[r0 * 16 + m0] = acc[rt][T][0];
-          sm.part[r0 * 16 + m0 + 1] = acc[rt][T][1];
-          sm.part[r1 * 16 + m0] = acc[rt][T][2];
-          sm.part[r1 * 16 + m0 + 1] = acc[rt][T][3];
-        }
+      for (int hr = 0; hr < 2; ++hr) {
+        const int r = warp * 32 + rt * 16 + g + 8 * hr;
+        const int q = (r * a.S + a.S - 1) / kDRows;
+        const int slot = r - (q * kDRows) / a.S;
+        const uint32_t dst = mapa_shared(red_local + ((rank * own_cap + slot) * 16) * 4, static_cast<uint32_t>(q));
+#pragma unroll
+        for (int T = 0; T < NT; ++T)
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const int ci = 2 * hr + c;
+            float v;
+            // factors 2^-24 (pairs 0 and 3), 2^-20 (pair 1), 2^-16 (pair 2): exact rescaling
+            if (!kInt4)
+              v = fmaf(acc[0][rt][T][ci] + acc[NG - 1][rt][T][ci], 16777216.0f,
+                       fmaf(acc[1 % NG][rt][T][ci], 1048576.0f, acc[2 % NG][rt][T][ci] * 65536.0f));
+            else
+              v = acc[0][rt][T][ci];
+            st_shared_cluster_f32(dst + (8 * T + 2 * t + c) * 4, v);
+          }
       }
-    }
   }
 
-  // --------------------------------------------------------------- cluster reduction, epilogue
-  cluster_sync_all();
+  // ==================================================================== cluster reduction
+  cluster_sync_all();  // every partial and slice sum has landed in its owner's shared memory
   {
     const int rr0 = (rank * kDRows) / a.S, rr1 = ((rank + 1) * kDRows) / a.S;
     const int nrows = rr1 - rr0;
     const int Mv = static_cast<int>(a.M < 8 * NT ? a.M : 8 * NT);
-    const uint32_t part_local = smem_u32(sm.part);
     for (int idx = threadIdx.x; idx < nrows * Mv; idx += kDThreads) {
-      const int m = idx / nrows, r = rr0 + (idx - m * nrows);
-      const int64_t n = static_cast<int64_t>(rb) * kDRows + r;
+      const int m = idx / nrows, slot = idx - m * nrows;
+      const int64_t n = static_cast<int64_t>(rb) * kDRows + rr0 + slot;
       if (n >= a.N) continue;
-      float v = 0.0f;
-      const uint32_t off = static_cast<uint32_t>((r * 16 + m) * sizeof(float));
-      for (int q = 0; q < a.S; ++q) v += ld_shared_cluster_f32(mapa_shared(part_local + off, q));
-      if (!kInt4) v *= __half2float(a.sc[n]);
+      float v = 0.0f, sx = 0.0f;
+      for (int q = 0; q < a.S; ++q) {  // fixed order: deterministic
+        v += red[(q * own_cap + slot) * 16 + m];
+        if (!kInt4) sx += sxr[q * 16 + m];
+      }
+      if (!kInt4) v = (v - sx) * __half2float(a.sc[n]);
       if (a.bias) v += __half2float(a.bias[n]);
       a.y[m * a.N + n] = __float2half_rn(v);
     }
   }
-  cluster_sync_all();
 }
 
 // ---------------------------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------------------------
 struct DecodePlan {
-  int S, C, ring, max_local, smem;
+  int S, C, ring, smem;
 };
 
-static bool plan_decode(bool int4, int NT, int64_t N, int64_t K, int num_sms, DecodePlan* p) {
-  const int64_t kbytes = int4 ? K / 2 : K / 4;
-  const int C = static_cast<int>((kbytes + 127) / 128);
+template <bool kInt4, int NT>
+static bool plan_decode_t(int64_t N, int64_t K, int num_sms, DecodePlan* p) {
+  using F = DecFmt<kInt4>;
+  const int C = static_cast<int>((K + F::kStageK - 1) / F::kStageK);
   const int64_t RB = (N + kDRows - 1) / kDRows;
-  const int64_t target = 2 * static_cast<int64_t>(num_sms);
-  int S = static_cast<int>((target + RB - 1) / RB);
+  // weight ring: every stage of the CTA's slice if it fits (then the whole slice is in flight
+  // before griddepcontrol.wait), else as many as two CTAs per SM allow
+  int ring = kDMaxRing;
+  while (ring > 2 && DecLayout<kInt4, NT>::bytes(ring) > kDSmemBudget) --ring;
+  const int smem = DecLayout<kInt4, NT>::bytes(ring);
+  if (smem > 227 * 1024) return false;
+  // one wave of two CTAs per SM, at most 8 K-slices per row block
+  int64_t S = (2 * static_cast<int64_t>(num_sms)) / RB;
   if (S < 1) S = 1;
-  const int smax = C < kDMaxCluster ? C : kDMaxCluster;
-  if (S > smax) S = smax;
-  for (;; ++S) {
-    const int ml = (C + S - 1) / S;
-    const int ring = ml < kDMaxRing ? ml : kDMaxRing;
-    const int bytes = decode_smem_bytes(int4, NT, ring, ml);
-    if (bytes <= 227 * 1024) {
-      *p = DecodePlan{S, C, ring, ml, bytes};
-      return true;
-    }
-    if (S >= smax) return false;
-  }
+  if (S > kDMaxCluster) S = kDMaxCluster;
+  if (S > C) S = C;
+  *p = DecodePlan{static_cast<int>(S), C, ring, smem};
+  return true;
+}
+
+static bool plan_decode(bool int4, int NT, int64_t N, int64_t K, int num_sms, DecodePlan* p) {
+  if (int4) return NT == 1 ? plan_decode_t<true, 1>(N, K, num_sms, p) : plan_decode_t<true, 2>(N, K, num_sms, p);
+  return NT == 1 ? plan_decode_t<false, 1>(N, K, num_sms, p) : plan_decode_t<false, 2>(N, K, num_sms, p);
 }
 
 template <bool kInt4, int NT>
@@ -433,7 +534,6 @@ static cudaError_t launch_decode(const __half* x, const void* w, const __half* s
   a.C = p.C;
   a.S = p.S;
   a.ring = p.ring;
-  a.max_local = p.max_local;
   return NT == 1 ? launch_decode_t<kInt4, 1>(tmap, a, p, s) : launch_decode_t<kInt4, 2>(tmap, a, p, s);
 }
 
