@@ -138,15 +138,26 @@ def barrier_sync(world):
     torch.cuda.synchronize()
 
 
-def max_over_ranks(v, world):
+def max_over_ranks(v, world, device="cuda"):
+    """Max of a per-rank scalar over all ranks (the job time is the slowest rank's)."""
     import torch
     import torch.distributed as dist
 
     if world == 1:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed_offset(rank: int) -> int:
+    """Every replica packs its own, distinct weights (weak scaling over independent replicas)."""
+    return 100003 * rank
+
+
+def weak_scaling_value(bytes_per_rank: int, world: int, ms_max: float) -> float:
+    """Whole-job GB/s: the bytes all ranks processed over the slowest rank's step time."""
+    return bytes_per_rank * world / (ms_max * 1e-3) / 1e9
 
 
 # ------------------------------------------------------------------------------------------------
@@ -162,7 +173,7 @@ def build_ternary_layers(rank, n_layers, config=1, shapes=LLAMA, dtype=None):
     for l in range(n_layers):
         row = []
         for mid, (name, N, K) in enumerate(shapes):
-            w = I.weights(N, K, I.seed_for(config, l, mid) + 100003 * rank, device="cuda")
+            w = I.weights(N, K, I.seed_for(config, l, mid) + rank_seed_offset(rank), device="cuda")
             p, s = tq.tq_quantize_pack(w)
             row.append((name, N, K, p, s))
             del w
@@ -245,7 +256,7 @@ def run_ours(args, world, rank, local):
     clocks = clk.stop()
     ms = ev0.elapsed_time(ev1) / args.steps
     ms_max = max_over_ranks(ms, world)
-    value = bytes_step * world / (ms_max * 1e-3) / 1e9
+    value = weak_scaling_value(bytes_step, world, ms_max)
 
     # end-to-end through the public API: pinned-host x in, y out, every step
     h_x = {k: v.cpu().pin_memory() for k, v in xs.items()}
@@ -270,7 +281,7 @@ def run_ours(args, world, rank, local):
     e1.record()
     barrier_sync(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
-    e2e_val = bytes_step * world / (e2e_ms * 1e-3) / 1e9
+    e2e_val = weak_scaling_value(bytes_step, world, e2e_ms)
 
     # roofline of the dominant kernel (the decode GEMM is every launch of the step)
     per_launch_us = ms * 1e3 / launches_step
@@ -375,7 +386,7 @@ def secondary_rows(args, rank, layers, peaks):
     for l in range(8):
         row = []
         for mid, (name, N, K) in enumerate(LLAMA):
-            w = I.weights(N, K, I.seed_for(3, l, mid) + 100003 * rank, device="cuda", outlier_frac=0.001)
+            w = I.weights(N, K, I.seed_for(3, l, mid) + rank_seed_offset(rank), device="cuda", outlier_frac=0.001)
             qw, sc = tq.w4g_quantize_pack(w)
             row.append((name, N, K, qw, sc))
             del w

@@ -39,8 +39,12 @@
 namespace tq {
 
 constexpr int kDRows = 128;                 // output rows per CTA
-constexpr int kDConsumers = 4;              // consumer warps (32 rows each)
-constexpr int kDThreads = (kDConsumers + 1) * 32;
+constexpr int kDConsumers = 8;              // consumer warps (16 rows = one MMA tile each)
+constexpr int kDRT = kDRows / (16 * kDConsumers);  // 16-row MMA tiles per consumer warp
+constexpr int kDBuilders = 2;               // activation warps: one per 64-byte sub-chunk
+constexpr int kDBuildWarp0 = kDConsumers;
+constexpr int kDTmaWarp = kDConsumers + kDBuilders;  // issues the weight TMA stream
+constexpr int kDThreads = (kDConsumers + kDBuilders + 1) * 32;
 constexpr int kDStageBytes = kDRows * 128;  // one TMA box: 128 rows x 128 bytes
 constexpr int kDMaxRing = 6;                // weight stages resident in shared memory
 constexpr int kDXRing = 2;                  // activation-fragment stages
@@ -74,19 +78,19 @@ struct DecodeArgs {
 template <bool kInt4, int NT>
 struct DecLayout {
   using F = DecFmt<kInt4>;
-  static constexpr int kXfStage = 2 * NT * F::kFragBytes;
-  static constexpr int kXgStage = kInt4 ? 2 * 16 * 4 : 0;
-  static constexpr int kXsBuf = 2 * NT * 32 * F::kXStride;
+  static constexpr int kXfStage = 2 * NT * F::kFragBytes;      // B fragments of one stage
+  static constexpr int kXsSub = NT * 32 * F::kXStride;          // natural x of one sub-chunk
+  static constexpr int kXgStage = 2 * 16 * 4;                   // W4A16 group sums [sub][token]
   static constexpr int kRed = kDRedRows * 16 * 4;
   static constexpr int kSxr = kDMaxCluster * 16 * 4;
   __host__ __device__ static constexpr int bytes(int ring) {
-    return 1024 + ring * kDStageBytes + kDXRing * (kXfStage + kXgStage) + 2 * kXsBuf + kRed + kSxr +
-           (2 * kDMaxRing + 2 * kDXRing) * 8;
+    return 1024 + ring * kDStageBytes + kDXRing * (kXfStage + kXgStage) + 2 * kDBuilders * kXsSub +
+           kRed + kSxr + 2 * 16 * 4 + (2 * kDMaxRing + 2 * kDXRing) * 8;
   }
 };
 
 template <bool kInt4, int NT>
-__global__ void __launch_bounds__(kDThreads)
+__global__ void __launch_bounds__(kDThreads, 2)
     decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeArgs a) {
   using F = DecFmt<kInt4>;
   using L = DecLayout<kInt4, NT>;
@@ -95,13 +99,14 @@ __global__ void __launch_bounds__(kDThreads)
   uint8_t* wst = base;                                                // ring x 16 KB weight tiles
   uint8_t* xf = wst + a.ring * kDStageBytes;                          // 2 x B fragments
   float* xg = reinterpret_cast<float*>(xf + kDXRing * L::kXfStage);   // 2 x [2][16] group sums
-  uint8_t* xs = reinterpret_cast<uint8_t*>(xg) + kDXRing * L::kXgStage;  // 2 x natural x
-  float* red = reinterpret_cast<float*>(xs + 2 * L::kXsBuf);          // [S][rows/S][16] partials
+  uint8_t* xs = reinterpret_cast<uint8_t*>(xg + kDXRing * 2 * 16);    // [builder][2] natural x
+  float* red = reinterpret_cast<float*>(xs + 2 * kDBuilders * L::kXsSub);  // [S][rows/S][16]
   float* sxr = red + kDRedRows * 16;                                  // [S][16] slice sums of x
-  uint64_t* wfull = reinterpret_cast<uint64_t*>(sxr + kDMaxCluster * 16);
+  float* sxb = sxr + kDMaxCluster * 16;                               // [builder][16] sums of x
+  uint64_t* wfull = reinterpret_cast<uint64_t*>(sxb + 2 * 16);
   uint64_t* wempty = wfull + kDMaxRing;
-  uint64_t* xfull = wempty + kDMaxRing;
-  uint64_t* xempty = xfull + kDXRing;
+  uint64_t* xfull = wempty + kDMaxRing;     // B fragments of a stage built (builder warps)
+  uint64_t* xempty = xfull + kDXRing;       // ... and consumed (consumer warps)
 
   pdl_allow_dependents();
 
@@ -120,15 +125,15 @@ __global__ void __launch_bounds__(kDThreads)
       mbar_init(&wempty[i], kDConsumers);
     }
     for (int i = 0; i < kDXRing; ++i) {
-      mbar_init(&xfull[i], 32);
+      mbar_init(&xfull[i], kDBuilders * 32);
       mbar_init(&xempty[i], kDConsumers);
     }
     fence_mbar_init();
   }
   __syncthreads();
 
-  if (warp == kDConsumers) {
-    // ================================================================== producer warp
+  if (warp == kDTmaWarp) {
+    // ================================================================== weight TMA warp
     if (lane == 0) {
       tma_prefetch_desc(&tmap);
       const int pre = nst < a.ring ? nst : a.ring;
@@ -136,149 +141,124 @@ __global__ void __launch_bounds__(kDThreads)
         mbar_arrive_expect_tx(&wfull[i], kDStageBytes);
         tma_load_2d(wst + i * kDStageBytes, &tmap, &wfull[i], (st_begin + i) * 128, rb * kDRows);
       }
+      // refill each weight slot as soon as the consumers release it (they start only once the
+      // previous kernel is done, so block in griddepcontrol.wait instead of polling meanwhile)
+      if (a.ring < nst) pdl_wait_prior_grids();
+      for (int j = a.ring; j < nst; ++j) {
+        const int ws = j % a.ring;
+        if (!mbar_wait(&wempty[ws], static_cast<uint32_t>((j / a.ring) - 1) & 1u)) break;
+        mbar_arrive_expect_tx(&wfull[ws], kDStageBytes);
+        tma_load_2d(wst + ws * kDStageBytes, &tmap, &wfull[ws], (st_begin + j) * 128, rb * kDRows);
+      }
     }
+  } else if (warp >= kDBuildWarp0) {
+    // ================================================================== builder warps
+    // Builder `sub` owns the 64-byte sub-chunk `sub` of every stage: it copies those
+    // activations (cp.async, padded), lays them out as B fragments in the k order the decode
+    // produces (odd positions pre-scaled by 1/4 or 1/16), and sums x on the CUDA cores.
+    const int sub = warp - kDBuildWarp0;
     pdl_wait_prior_grids();  // activations may come from the previous kernel
-
+    uint8_t* mybuf = xs + sub * 2 * L::kXsSub;
     auto issue_x = [&](int i) {
       if (i < nst) {
-        uint8_t* buf = xs + (i & 1) * L::kXsBuf;
+        uint8_t* buf = mybuf + (i & 1) * L::kXsSub;
 #pragma unroll
-        for (int sub = 0; sub < 2; ++sub)
+        for (int T = 0; T < NT; ++T) {
+          const int m = 8 * T + g;
+          const int64_t k0 = static_cast<int64_t>(st_begin + i) * F::kStageK + sub * F::kSubK + t * F::kLaneK;
+          const bool valid = (m < a.M) && (k0 < a.K);
+          const __half* src = valid ? a.x + m * a.K + k0 : a.x;
+          uint8_t* dst = buf + (T * 32 + lane) * F::kXStride;
 #pragma unroll
-          for (int T = 0; T < NT; ++T) {
-            const int m = 8 * T + g;
-            const int64_t k0 = static_cast<int64_t>(st_begin + i) * F::kStageK + sub * F::kSubK + t * F::kLaneK;
-            const bool valid = (m < a.M) && (k0 < a.K);
-            const __half* src = valid ? a.x + m * a.K + k0 : a.x;
-            uint8_t* dst = buf + ((sub * NT + T) * 32 + lane) * F::kXStride;
-#pragma unroll
-            for (int j = 0; j < F::kXLaneBytes / 16; ++j)
-              cp_async_16(dst + 16 * j, src + (valid ? 8 * j : 0), valid ? 16u : 0u);
-          }
+          for (int j = 0; j < F::kXLaneBytes / 16; ++j)
+            cp_async_16(dst + 16 * j, src + (valid ? 8 * j : 0), valid ? 16u : 0u);
+        }
       }
       cp_async_commit();  // one group per stage (possibly empty) keeps the accounting uniform
     };
     issue_x(0);
     issue_x(1);
-
-    const uint32_t ONE = 0x3C003C00u, FOUR = 0x44004400u, SIXTEEN = 0x4C004C00u;
-    const __half2 q4 = __floats2half2_rn(0.25f, 0.25f);
-    const __half2 q16 = __floats2half2_rn(0.0625f, 0.0625f);
-    float ssum[NT][4][4];  // four independent MMA chains per token tile
+    const __half2 fold = kInt4 ? __floats2half2_rn(0.0625f, 0.0625f) : __floats2half2_rn(0.25f, 0.25f);
+    float sxl[NT];  // running sum of this lane's activations (ternary)
 #pragma unroll
-    for (int T = 0; T < NT; ++T)
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) ssum[T][j][c] = 0.0f;
-
+    for (int T = 0; T < NT; ++T) sxl[T] = 0.0f;
     for (int i = 0; i < nst; ++i) {
       const int xslot = i & 1;
-      if (i >= kDXRing) {
-        // consumers are done with stage i-2: its fragment slot and its weight slot are free
-        if (!mbar_wait(&xempty[xslot], static_cast<uint32_t>((i >> 1) - 1) & 1u)) break;
-        const int j = i - kDXRing + a.ring;  // refill the freed weight slot with stage j
-        if (j >= a.ring && j < nst) {
-          const int ws = j % a.ring;
-          if (!mbar_wait(&wempty[ws], static_cast<uint32_t>((j / a.ring) - 1) & 1u)) break;
-          if (lane == 0) {
-            mbar_arrive_expect_tx(&wfull[ws], kDStageBytes);
-            tma_load_2d(wst + ws * kDStageBytes, &tmap, &wfull[ws], (st_begin + j) * 128, rb * kDRows);
-          }
-        }
-      }
+      if (i >= kDXRing && !mbar_wait(&xempty[xslot], static_cast<uint32_t>((i >> 1) - 1) & 1u)) break;
       cp_async_wait<1>();  // this lane's copies of stage i have landed
-      const uint8_t* buf = xs + (i & 1) * L::kXsBuf;
+      const uint8_t* buf = mybuf + (i & 1) * L::kXsSub;
       uint4* xfs = reinterpret_cast<uint4*>(xf + xslot * L::kXfStage);
 #pragma unroll
-      for (int sub = 0; sub < 2; ++sub)
+      for (int T = 0; T < NT; ++T) {
+        const uint4* src = reinterpret_cast<const uint4*>(buf + (T * 32 + lane) * F::kXStride);
+        uint32_t P[F::kLaneK / 2];
 #pragma unroll
-        for (int T = 0; T < NT; ++T) {
-          const uint4* src = reinterpret_cast<const uint4*>(buf + ((sub * NT + T) * 32 + lane) * F::kXStride);
-          uint32_t P[F::kLaneK / 2];
-#pragma unroll
-          for (int j = 0; j < F::kLaneK / 8; ++j) {
-            const uint4 v = src[j];
-            P[4 * j] = v.x;
-            P[4 * j + 1] = v.y;
-            P[4 * j + 2] = v.z;
-            P[4 * j + 3] = v.w;
-          }
-          float cg[4][4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-#pragma unroll
-            for (int c = 0; c < 4; ++c) cg[j][c] = 0.0f;
-#pragma unroll
-          for (int f = 0; f < F::kFragU4; ++f) {
-            uint32_t Pa, Pb, Pc, Pd;
-            if (!kInt4) {  // f = h*4 + pp: positions p = 2pp (even), 2pp+1 (odd) of word pair h
-              const int h = f >> 2, pp = f & 3;
-              Pa = P[16 * h + pp];
-              Pb = P[16 * h + 4 + pp];
-              Pc = P[16 * h + 8 + pp];
-              Pd = P[16 * h + 12 + pp];
-            } else {       // f = h*2 + s: nibble positions 2s (class 0), 2s+1 (class 1)
-              const int h = f >> 1, s = f & 1;
-              Pa = P[8 * h + s];
-              Pb = P[8 * h + 2 + s];
-              Pc = P[8 * h + 4 + s];
-              Pd = P[8 * h + 6 + s];
-            }
-            const uint32_t e01 = __byte_perm(Pa, Pb, 0x5410), e23 = __byte_perm(Pc, Pd, 0x5410);
-            const uint32_t o01 = __byte_perm(Pa, Pb, 0x7632), o23 = __byte_perm(Pc, Pd, 0x7632);
-            __half2 so01 = *reinterpret_cast<const __half2*>(&o01);
-            __half2 so23 = *reinterpret_cast<const __half2*>(&o23);
-            so01 = __hmul2(so01, kInt4 ? q16 : q4);
-            so23 = __hmul2(so23, kInt4 ? q16 : q4);
-            const uint32_t s01 = *reinterpret_cast<const uint32_t*>(&so01);
-            const uint32_t s23 = *reinterpret_cast<const uint32_t*>(&so23);
-            xfs[((sub * NT + T) * F::kFragU4 + f) * 32 + lane] = make_uint4(e01, e23, s01, s23);
-            // sum_k x on the tensor core: A = all ones (x4 / x16 undoes the fold)
-            const uint32_t up = kInt4 ? SIXTEEN : FOUR;
-            if (!kInt4) {
-              mma_16816(ssum[T][(2 * f) & 3], ONE, ONE, ONE, ONE, e01, e23);
-              mma_16816(ssum[T][(2 * f + 1) & 3], up, up, up, up, s01, s23);
-            } else {
-              mma_16816(cg[(2 * f) & 3], ONE, ONE, ONE, ONE, e01, e23);
-              mma_16816(cg[(2 * f + 1) & 3], up, up, up, up, s01, s23);
-            }
-          }
-          if (kInt4 && g == 0) {  // row 0 of the all-ones product holds the token sums
-            xg[(xslot * 2 + sub) * 16 + 8 * T + 2 * t] = (cg[0][0] + cg[1][0]) + (cg[2][0] + cg[3][0]);
-            xg[(xslot * 2 + sub) * 16 + 8 * T + 2 * t + 1] = (cg[0][1] + cg[1][1]) + (cg[2][1] + cg[3][1]);
-          }
+        for (int j = 0; j < F::kLaneK / 8; ++j) {
+          const uint4 v = src[j];
+          P[4 * j] = v.x;
+          P[4 * j + 1] = v.y;
+          P[4 * j + 2] = v.z;
+          P[4 * j + 3] = v.w;
         }
+        float ps = 0.0f;  // sum of this lane's activations in the sub-chunk (fixed order)
+#pragma unroll
+        for (int j = 0; j < F::kLaneK / 2; ++j) {
+          const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&P[j]));
+          ps += f2.x + f2.y;
+        }
+#pragma unroll
+        for (int f = 0; f < F::kFragU4; ++f) {
+          uint32_t Pa, Pb, Pc, Pd;
+          if (!kInt4) {  // f = h*4 + pp: positions p = 2pp (even), 2pp+1 (odd) of word pair h
+            const int h = f >> 2, pp = f & 3;
+            Pa = P[16 * h + pp];
+            Pb = P[16 * h + 4 + pp];
+            Pc = P[16 * h + 8 + pp];
+            Pd = P[16 * h + 12 + pp];
+          } else {       // f = h*2 + s: nibble positions 2s (class 0), 2s+1 (class 1)
+            const int h = f >> 1, s2 = f & 1;
+            Pa = P[8 * h + s2];
+            Pb = P[8 * h + 2 + s2];
+            Pc = P[8 * h + 4 + s2];
+            Pd = P[8 * h + 6 + s2];
+          }
+          const uint32_t e01 = __byte_perm(Pa, Pb, 0x5410), e23 = __byte_perm(Pc, Pd, 0x5410);
+          uint32_t o01 = __byte_perm(Pa, Pb, 0x7632), o23 = __byte_perm(Pc, Pd, 0x7632);
+          __half2 so01 = __hmul2(*reinterpret_cast<__half2*>(&o01), fold);
+          __half2 so23 = __hmul2(*reinterpret_cast<__half2*>(&o23), fold);
+          xfs[((sub * NT + T) * F::kFragU4 + f) * 32 + lane] =
+              make_uint4(e01, e23, *reinterpret_cast<uint32_t*>(&so01), *reinterpret_cast<uint32_t*>(&so23));
+        }
+        ps += __shfl_xor_sync(0xFFFFFFFFu, ps, 1);  // the four lanes of one token
+        ps += __shfl_xor_sync(0xFFFFFFFFu, ps, 2);
+        if (kInt4) {
+          if (t == 0) xg[(xslot * 2 + sub) * 16 + 8 * T + g] = ps;
+        } else {
+          sxl[T] += ps;
+        }
+      }
       mbar_arrive(&xfull[xslot]);
       issue_x(i + 2);
     }
     cp_async_wait<0>();
-    if (!kInt4 && g == 0) {  // push this slice's token sums of x to every CTA of the cluster
-      const uint32_t loc = smem_u32(sxr + rank * 16);
+    if (!kInt4 && t == 0) {
 #pragma unroll
-      for (int T = 0; T < NT; ++T) {
-        const float s0 = (ssum[T][0][0] + ssum[T][1][0]) + (ssum[T][2][0] + ssum[T][3][0]);
-        const float s1 = (ssum[T][0][1] + ssum[T][1][1]) + (ssum[T][2][1] + ssum[T][3][1]);
-        for (int q = 0; q < a.S; ++q) {
-          st_shared_cluster_f32(mapa_shared(loc + (8 * T + 2 * t) * 4, q), s0);
-          st_shared_cluster_f32(mapa_shared(loc + (8 * T + 2 * t + 1) * 4, q), s1);
-        }
-      }
+      for (int T = 0; T < NT; ++T) sxb[sub * 16 + 8 * T + g] = sxl[T];
     }
   } else {
     // ================================================================== consumer warps
     constexpr int NG = kInt4 ? 1 : 4;  // accumulator groups: one per position pair (chains)
-    float acc[NG][2][NT][4];
+    float acc[NG][kDRT][NT][4];
 #pragma unroll
     for (int q = 0; q < NG; ++q)
 #pragma unroll
-      for (int rt = 0; rt < 2; ++rt)
+      for (int rt = 0; rt < kDRT; ++rt)
 #pragma unroll
         for (int T = 0; T < NT; ++T)
 #pragma unroll
           for (int c = 0; c < 4; ++c) acc[q][rt][T][c] = 0.0f;
     const int64_t G = a.K >> 7;
-
+    pdl_wait_prior_grids();  // block (not poll) until the activations can exist
     for (int i = 0; i < nst; ++i) {
       const int ws = i % a.ring, xslot = i & 1;
       if (!mbar_wait(&wfull[ws], static_cast<uint32_t>(i / a.ring) & 1u) ||
@@ -289,10 +269,10 @@ __global__ void __launch_bounds__(kDThreads)
 #pragma unroll
       for (int sub = 0; sub < 2; ++sub) {
         const int chunk = sub * 4 + t;
-        uint32_t w0[2][4], w1[2][4];
+        uint32_t w0[kDRT][4], w1[kDRT][4];
 #pragma unroll
-        for (int rt = 0; rt < 2; ++rt) {
-          const int r0 = warp * 32 + rt * 16 + g, r1 = r0 + 8;
+        for (int rt = 0; rt < kDRT; ++rt) {
+          const int r0 = warp * (16 * kDRT) + rt * 16 + g, r1 = r0 + 8;
           const uint4 U0 = *reinterpret_cast<const uint4*>(st + r0 * 128 + ((chunk ^ (r0 & 7)) << 4));
           const uint4 U1 = *reinterpret_cast<const uint4*>(st + r1 * 128 + ((chunk ^ (r1 & 7)) << 4));
           w0[rt][0] = U0.x; w0[rt][1] = U0.y; w0[rt][2] = U0.z; w0[rt][3] = U0.w;
@@ -301,9 +281,9 @@ __global__ void __launch_bounds__(kDThreads)
         if (!kInt4) {
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            uint32_t sh[2][4];
+            uint32_t sh[kDRT][4];
 #pragma unroll
-            for (int rt = 0; rt < 2; ++rt) {
+            for (int rt = 0; rt < kDRT; ++rt) {
               sh[rt][0] = w0[rt][2 * h] >> 12;
               sh[rt][1] = w1[rt][2 * h] >> 12;
               sh[rt][2] = w0[rt][2 * h + 1] >> 12;
@@ -318,7 +298,7 @@ __global__ void __launch_bounds__(kDThreads)
               for (int q = 0; q < 2; ++q) {
                 const int p = 2 * pp + q;
 #pragma unroll
-                for (int rt = 0; rt < 2; ++rt) {
+                for (int rt = 0; rt < kDRT; ++rt) {
                   uint32_t a0, a1, a2, a3;
                   if (p < 6) {
                     const uint32_t mk = 0x00030003u << (2 * p);
@@ -342,15 +322,14 @@ __global__ void __launch_bounds__(kDThreads)
           }
         } else {
           const int64_t gi = static_cast<int64_t>(st_begin + i) * 2 + sub;
-          const float* xgs = xg + (xslot * 2 + sub) * 16;
           float xgt[NT][2];
 #pragma unroll
           for (int T = 0; T < NT; ++T) {
-            xgt[T][0] = 8.0f * xgs[8 * T + 2 * t];
-            xgt[T][1] = 8.0f * xgs[8 * T + 2 * t + 1];
+            xgt[T][0] = 8.0f * xg[(xslot * 2 + sub) * 16 + 8 * T + 2 * t];
+            xgt[T][1] = 8.0f * xg[(xslot * 2 + sub) * 16 + 8 * T + 2 * t + 1];
           }
 #pragma unroll
-          for (int rt = 0; rt < 2; ++rt) {
+          for (int rt = 0; rt < kDRT; ++rt) {
             float cg[2][NT][4];  // two chains (class 0 / class 1 fields)
 #pragma unroll
             for (int j = 0; j < 2; ++j)
@@ -361,12 +340,12 @@ __global__ void __launch_bounds__(kDThreads)
 #pragma unroll
             for (int h = 0; h < 2; ++h)
 #pragma unroll
-              for (int s = 0; s < 2; ++s) {
-                const uint32_t x0 = w0[rt][2 * h] >> (8 * s), x1 = w1[rt][2 * h] >> (8 * s);
-                const uint32_t x2 = w0[rt][2 * h + 1] >> (8 * s), x3 = w1[rt][2 * h + 1] >> (8 * s);
+              for (int s2 = 0; s2 < 2; ++s2) {
+                const uint32_t x0 = w0[rt][2 * h] >> (8 * s2), x1 = w1[rt][2 * h] >> (8 * s2);
+                const uint32_t x2 = w0[rt][2 * h + 1] >> (8 * s2), x3 = w1[rt][2 * h + 1] >> (8 * s2);
                 uint4 B[NT];
 #pragma unroll
-                for (int T = 0; T < NT; ++T) B[T] = xfs[((sub * NT + T) * 4 + h * 2 + s) * 32 + lane];
+                for (int T = 0; T < NT; ++T) B[T] = xfs[((sub * NT + T) * 4 + h * 2 + s2) * 32 + lane];
 #pragma unroll
                 for (int cls = 0; cls < 2; ++cls) {
                   const uint32_t mk = cls ? 0x00F000F0u : 0x000F000Fu;
@@ -376,7 +355,7 @@ __global__ void __launch_bounds__(kDThreads)
                               cls ? B[T].w : B[T].y);
                 }
               }
-            const int64_t n0 = static_cast<int64_t>(rb) * kDRows + warp * 32 + rt * 16 + g, n1 = n0 + 8;
+            const int64_t n0 = static_cast<int64_t>(rb) * kDRows + warp * (16 * kDRT) + rt * 16 + g, n1 = n0 + 8;
             // groups past K (a zero-filled half stage) contribute nothing
             const float s0 = (n0 < a.N && gi < G) ? __half2float(a.sc[n0 * G + gi]) : 0.0f;
             const float s1 = (n1 < a.N && gi < G) ? __half2float(a.sc[n1 * G + gi]) : 0.0f;
@@ -403,10 +382,10 @@ __global__ void __launch_bounds__(kDThreads)
     // are split evenly over the cluster: owner q holds rows [q*128/S, (q+1)*128/S))
     const uint32_t red_local = smem_u32(red);
 #pragma unroll
-    for (int rt = 0; rt < 2; ++rt)
+    for (int rt = 0; rt < kDRT; ++rt)
 #pragma unroll
       for (int hr = 0; hr < 2; ++hr) {
-        const int r = warp * 32 + rt * 16 + g + 8 * hr;
+        const int r = warp * (16 * kDRT) + rt * 16 + g + 8 * hr;
         const int q = (r * a.S + a.S - 1) / kDRows;
         const int slot = r - (q * kDRows) / a.S;
         const uint32_t dst = mapa_shared(red_local + ((rank * own_cap + slot) * 16) * 4, static_cast<uint32_t>(q));
@@ -428,7 +407,14 @@ __global__ void __launch_bounds__(kDThreads)
   }
 
   // ==================================================================== cluster reduction
+  __syncthreads();  // the builders' sums of x are in shared memory
+  if (!kInt4 && threadIdx.x < 16) {  // push this slice's token sums of x to every owner
+    const float sx = sxb[threadIdx.x] + sxb[16 + threadIdx.x];
+    const uint32_t loc = smem_u32(sxr + rank * 16 + threadIdx.x);
+    for (int q = 0; q < a.S; ++q) st_shared_cluster_f32(mapa_shared(loc, q), sx);
+  }
   cluster_sync_all();  // every partial and slice sum has landed in its owner's shared memory
+  pdl_wait_prior_grids();
   {
     const int rr0 = (rank * kDRows) / a.S, rr1 = ((rank + 1) * kDRows) / a.S;
     const int nrows = rr1 - rr0;

@@ -187,6 +187,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
+    pdl_wait_prior_grids();  // x arrives only after the previous kernel: block, do not poll
     if (lane == 0) {
       const uint32_t idesc = idesc_f16_f32(kPBM, kPBN);
       const uint32_t a_base = smem_u32(sm + L::kOffA), b_base = smem_u32(sm + L::kOffB);
