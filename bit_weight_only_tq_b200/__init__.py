@@ -23,6 +23,7 @@ __all__ = [
     "TQ_OK", "TQ_F32", "TQ_F16", "PATH_AUTO", "PATH_DECODE", "PATH_PREFILL", "PATH_GENERIC",
     "FMT_TERNARY", "FMT_W4G128",
     "tq_quantize_pack", "tq_gemm", "w4g_quantize_pack", "w4g_gemm", "tq_validate_packed",
+    "tq_gemm_grouped", "w4g_gemm_grouped",
     "tq_select_path", "tq_device_status", "tq_status_string", "header_functions",
 ]
 
@@ -55,6 +56,8 @@ _SIGS = {
     "w4g_gemm": [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp],
     "w4g_gemm_ex": [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _vp],
     "tq_validate_packed": [_vp, _i64, _i64, _vp, _vp],
+    "tq_gemm_grouped": [_vp, _int, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _vp],
+    "w4g_gemm_grouped": [_vp, _int, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _vp],
     "tq_select_path": [_int, _i64, _i64, _i64, _int],
     "tq_device_status": [],
     "tq_status_string": [_int],
@@ -181,6 +184,51 @@ def w4g_gemm(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, bias=
     _check(lib.w4g_gemm_ex(_ptr(x), _ptr(qweight), _ptr(scales), _ptr(bias), _ptr(y), M, N, K,
                            int(path), _stream(stream)), "w4g_gemm")
     return y
+
+
+def _ptr_array(ts):
+    arr = (ctypes.c_void_p * len(ts))()
+    for i, t in enumerate(ts):
+        arr[i] = None if t is None else t.data_ptr()
+    return arr
+
+
+def _grouped(fn, x, weights, scales, biases, ys, wdtype, sdim, what, stream):
+    _need(x, torch.float16, "x", 2)
+    M, K = x.shape
+    count = len(weights)
+    if not (1 <= count <= 4) or len(scales) != count:
+        raise ValueError("1..4 matrices with one scale tensor each")
+    biases = [None] * count if biases is None else list(biases)
+    Ns = []
+    for w, s, b in zip(weights, scales, biases):
+        _need(w, wdtype, "weights", 2)
+        _need(s, torch.float16, "scales", sdim)
+        _need(b, torch.float16, "bias", 1)
+        Ns.append(w.shape[0])
+    if ys is None:
+        ys = [torch.empty(M, n, dtype=torch.float16, device=x.device) for n in Ns]
+    for yv, n in zip(ys, Ns):
+        _need(yv, torch.float16, "y", 2)
+        if tuple(yv.shape) != (M, n):
+            raise ValueError("y shape mismatch")
+    nar = (ctypes.c_int64 * count)(*Ns)
+    has_bias = any(b is not None for b in biases)
+    _check(fn(_ptr(x), count, _ptr_array(weights), _ptr_array(scales),
+              _ptr_array(biases) if has_bias else None, _ptr_array(ys), nar, M, K, _stream(stream)), what)
+    return ys
+
+
+def tq_gemm_grouped(x, packed_list, scale_list, bias_list=None, y_list=None, stream=None):
+    """Several ternary linears sharing x (e.g. q, k, v) in one launch: returns [y_g]."""
+    return _grouped(lib.tq_gemm_grouped, x, packed_list, scale_list, bias_list, y_list, torch.uint8, 1,
+                    "tq_gemm_grouped", stream)
+
+
+def w4g_gemm_grouped(x, qweight_list, scales_list, bias_list=None, y_list=None, stream=None):
+    """Several W4A16 linears sharing x in one launch: returns [y_g]."""
+    return _grouped(lib.w4g_gemm_grouped, x, qweight_list, scales_list, bias_list, y_list, torch.int32, 2,
+                    "w4g_gemm_grouped", stream)
 
 
 def tq_validate_packed(packed: torch.Tensor, K: int, stream=None) -> int:

@@ -131,6 +131,41 @@ int resolve_path(int fmt, int path, int64_t M, int64_t N, int64_t K, bool all_al
   }
 }
 
+// Shared driver of the grouped entry points: one decode launch when every matrix takes the
+// decode path, otherwise one single-matrix GEMM per matrix.
+template <bool kInt4, typename WT, typename Single, typename Group>
+static int gemm_grouped_impl(const uint16_t* x, int count, const WT* const* w,
+                             const uint16_t* const* sc, const uint16_t* const* bias,
+                             uint16_t* const* y, const int64_t* N, int64_t M, int64_t K,
+                             void* stream, Single single, Group group) {
+  if (count < 1 || count > 4) return TQ_ERR_SHAPE;
+  if (!w || !sc || !y || !N) return TQ_ERR_NULL;
+  if (M < 0 || K <= 0 || K > (int64_t(1) << 28) || M > (int64_t(1) << 31)) return TQ_ERR_SHAPE;
+  if (kInt4 && K % 128 != 0) return TQ_ERR_SHAPE;
+  bool all_decode = M >= 1 && M <= 16 && x && aligned16(x);
+  for (int g = 0; g < count; ++g) {
+    if (N[g] < 0 || N[g] > (int64_t(1) << 31)) return TQ_ERR_SHAPE;
+    if (M > 0 && N[g] > 0 && (!w[g] || !sc[g] || !y[g])) return TQ_ERR_NULL;
+    if (N[g] == 0) { all_decode = false; continue; }
+    all_decode = all_decode && tq::decode_supported(kInt4, M, N[g], K) && aligned16(w[g]) &&
+                 aligned16(y[g]) && (!kInt4 || aligned16(sc[g]));
+  }
+  if (M == 0) return TQ_OK;
+  if (!x) return TQ_ERR_NULL;
+  if (all_decode) {
+    const __half* bh[4] = {nullptr, nullptr, nullptr, nullptr};
+    for (int g = 0; g < count; ++g) bh[g] = bias ? reinterpret_cast<const __half*>(bias[g]) : nullptr;
+    return to_status(group(reinterpret_cast<const __half*>(x), count, w,
+                           reinterpret_cast<const __half* const*>(sc), bh,
+                           reinterpret_cast<__half* const*>(y), N, M, K, as_stream(stream)));
+  }
+  for (int g = 0; g < count; ++g) {
+    const int st = single(x, w[g], sc[g], bias ? bias[g] : nullptr, y[g], M, N[g], K, stream);
+    if (st != TQ_OK) return st;
+  }
+  return TQ_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -239,6 +274,20 @@ int w4g_gemm_ex(const uint16_t* x, const int32_t* qweight, const uint16_t* scale
 int w4g_gemm(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
              const uint16_t* bias, uint16_t* y, int64_t M, int64_t N, int64_t K, void* stream) {
   return w4g_gemm_ex(x, qweight, scales, bias, y, M, N, K, TQ_PATH_AUTO, stream);
+}
+
+int tq_gemm_grouped(const uint16_t* x, int count, const uint8_t* const* packed,
+                    const uint16_t* const* scale, const uint16_t* const* bias, uint16_t* const* y,
+                    const int64_t* N, int64_t M, int64_t K, void* stream) {
+  return gemm_grouped_impl<false>(x, count, packed, scale, bias, y, N, M, K, stream, tq_gemm,
+                                  tq::launch_tq_gemm_decode_group);
+}
+
+int w4g_gemm_grouped(const uint16_t* x, int count, const int32_t* const* qweight,
+                     const uint16_t* const* scales, const uint16_t* const* bias,
+                     uint16_t* const* y, const int64_t* N, int64_t M, int64_t K, void* stream) {
+  return gemm_grouped_impl<true>(x, count, qweight, scales, bias, y, N, M, K, stream, w4g_gemm,
+                                 tq::launch_w4g_gemm_decode_group);
 }
 
 int tq_validate_packed(const uint8_t* packed, int64_t N, int64_t K, int* bad_count, void* stream) {

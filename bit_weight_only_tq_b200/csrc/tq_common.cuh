@@ -192,6 +192,14 @@ cudaError_t launch_tq_validate(const uint8_t* packed, int64_t N, int64_t K, int*
 cudaError_t launch_tq_gemm_decode(const __half* x, const uint8_t* packed, const __half* scale,
                                   const __half* bias, __half* y, int64_t M, int64_t N, int64_t K,
                                   cudaStream_t s);
+cudaError_t launch_tq_gemm_decode_group(const __half* x, int count, const uint8_t* const* packed,
+                                        const __half* const* scale, const __half* const* bias,
+                                        __half* const* y, const int64_t* N, int64_t M, int64_t K,
+                                        cudaStream_t s);
+cudaError_t launch_w4g_gemm_decode_group(const __half* x, int count, const int32_t* const* qweight,
+                                         const __half* const* scales, const __half* const* bias,
+                                         __half* const* y, const int64_t* N, int64_t M, int64_t K,
+                                         cudaStream_t s);
 cudaError_t launch_w4g_gemm_decode(const __half* x, const int32_t* qweight, const __half* scales,
                                    const __half* bias, __half* y, int64_t M, int64_t N, int64_t K,
                                    cudaStream_t s);

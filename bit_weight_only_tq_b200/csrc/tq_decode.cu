@@ -64,15 +64,24 @@ struct DecFmt {
   static constexpr int kXStride = kXLaneBytes + 16;  // padded: conflict-free 16-byte reads
 };
 
+constexpr int kDMaxGroup = 4;  // weight matrices sharing x in one launch (e.g. q, k, v)
+
 struct DecodeArgs {
   const __half* x;
-  const __half* sc;    // ternary: scale[N]; W4A16: scales[N, K/128]
-  const __half* bias;  // may be null
-  __half* y;
-  int64_t M, N, K;
+  int64_t M, K;
   int C;     // stages along K
   int S;     // CTAs per cluster (K-slices)
   int ring;  // weight stages resident in shared memory (all of a CTA's stages when they fit)
+  int count;                        // matrices in the group
+  int rb_start[kDMaxGroup + 1];     // first 128-row block of each matrix in grid.y
+  int64_t N[kDMaxGroup];
+  const __half* sc[kDMaxGroup];     // ternary: scale[N]; W4A16: scales[N, K/128]
+  const __half* bias[kDMaxGroup];   // may be null
+  __half* y[kDMaxGroup];
+};
+
+struct DecodeMaps {
+  CUtensorMap m[kDMaxGroup];        // packed weights of each matrix
 };
 
 template <bool kInt4, int NT>
@@ -91,7 +100,7 @@ struct DecLayout {
 
 template <bool kInt4, int NT>
 __global__ void __launch_bounds__(kDThreads, 2)
-    decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeArgs a) {
+    decode_gemm_kernel(const __grid_constant__ DecodeMaps maps, const __grid_constant__ DecodeArgs a) {
   using F = DecFmt<kInt4>;
   using L = DecLayout<kInt4, NT>;
   extern __shared__ uint8_t smem_raw[];
@@ -113,7 +122,17 @@ __global__ void __launch_bounds__(kDThreads, 2)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int rank = static_cast<int>(cluster_ctarank());
-  const int rb = blockIdx.y;
+  // which matrix of the group this CTA works on, and its 128-row block within that matrix
+  int grp = 0;
+#pragma unroll
+  for (int q = 1; q < kDMaxGroup; ++q)
+    if (q < a.count && static_cast<int>(blockIdx.y) >= a.rb_start[q]) grp = q;
+  const int rb = static_cast<int>(blockIdx.y) - a.rb_start[grp];
+  const CUtensorMap* tmap = &maps.m[grp];
+  const int64_t Nm = a.N[grp];
+  const __half* scm = a.sc[grp];
+  const __half* biasm = a.bias[grp];
+  __half* ym = a.y[grp];
   const int st_begin = static_cast<int>((static_cast<int64_t>(rank) * a.C) / a.S);
   const int st_end = static_cast<int>((static_cast<int64_t>(rank + 1) * a.C) / a.S);
   const int nst = st_end - st_begin;
@@ -135,11 +154,11 @@ __global__ void __launch_bounds__(kDThreads, 2)
   if (warp == kDTmaWarp) {
     // ================================================================== weight TMA warp
     if (lane == 0) {
-      tma_prefetch_desc(&tmap);
+      tma_prefetch_desc(tmap);
       const int pre = nst < a.ring ? nst : a.ring;
       for (int i = 0; i < pre; ++i) {
         mbar_arrive_expect_tx(&wfull[i], kDStageBytes);
-        tma_load_2d(wst + i * kDStageBytes, &tmap, &wfull[i], (st_begin + i) * 128, rb * kDRows);
+        tma_load_2d(wst + i * kDStageBytes, tmap, &wfull[i], (st_begin + i) * 128, rb * kDRows);
       }
       // refill each weight slot as soon as the consumers release it (they start only once the
       // previous kernel is done, so block in griddepcontrol.wait instead of polling meanwhile)
@@ -148,7 +167,7 @@ __global__ void __launch_bounds__(kDThreads, 2)
         const int ws = j % a.ring;
         if (!mbar_wait(&wempty[ws], static_cast<uint32_t>((j / a.ring) - 1) & 1u)) break;
         mbar_arrive_expect_tx(&wfull[ws], kDStageBytes);
-        tma_load_2d(wst + ws * kDStageBytes, &tmap, &wfull[ws], (st_begin + j) * 128, rb * kDRows);
+        tma_load_2d(wst + ws * kDStageBytes, tmap, &wfull[ws], (st_begin + j) * 128, rb * kDRows);
       }
     }
   } else if (warp >= kDBuildWarp0) {
@@ -357,8 +376,8 @@ __global__ void __launch_bounds__(kDThreads, 2)
               }
             const int64_t n0 = static_cast<int64_t>(rb) * kDRows + warp * (16 * kDRT) + rt * 16 + g, n1 = n0 + 8;
             // groups past K (a zero-filled half stage) contribute nothing
-            const float s0 = (n0 < a.N && gi < G) ? __half2float(a.sc[n0 * G + gi]) : 0.0f;
-            const float s1 = (n1 < a.N && gi < G) ? __half2float(a.sc[n1 * G + gi]) : 0.0f;
+            const float s0 = (n0 < Nm && gi < G) ? __half2float(scm[n0 * G + gi]) : 0.0f;
+            const float s1 = (n1 < Nm && gi < G) ? __half2float(scm[n1 * G + gi]) : 0.0f;
 #pragma unroll
             for (int T = 0; T < NT; ++T) {
               float c4[4];
@@ -422,15 +441,15 @@ __global__ void __launch_bounds__(kDThreads, 2)
     for (int idx = threadIdx.x; idx < nrows * Mv; idx += kDThreads) {
       const int m = idx / nrows, slot = idx - m * nrows;
       const int64_t n = static_cast<int64_t>(rb) * kDRows + rr0 + slot;
-      if (n >= a.N) continue;
+      if (n >= Nm) continue;
       float v = 0.0f, sx = 0.0f;
       for (int q = 0; q < a.S; ++q) {  // fixed order: deterministic
         v += red[(q * own_cap + slot) * 16 + m];
         if (!kInt4) sx += sxr[q * 16 + m];
       }
-      if (!kInt4) v = (v - sx) * __half2float(a.sc[n]);
-      if (a.bias) v += __half2float(a.bias[n]);
-      a.y[m * a.N + n] = __float2half_rn(v);
+      if (!kInt4) v = (v - sx) * __half2float(scm[n]);
+      if (biasm) v += __half2float(biasm[n]);
+      ym[m * Nm + n] = __float2half_rn(v);
     }
   }
 }
@@ -443,10 +462,9 @@ struct DecodePlan {
 };
 
 template <bool kInt4, int NT>
-static bool plan_decode_t(int64_t N, int64_t K, int num_sms, DecodePlan* p) {
+static bool plan_decode_t(int64_t RB, int64_t K, int num_sms, DecodePlan* p) {
   using F = DecFmt<kInt4>;
   const int C = static_cast<int>((K + F::kStageK - 1) / F::kStageK);
-  const int64_t RB = (N + kDRows - 1) / kDRows;
   // weight ring: every stage of the CTA's slice if it fits (then the whole slice is in flight
   // before griddepcontrol.wait), else as many as two CTAs per SM allow
   int ring = kDMaxRing;
@@ -462,19 +480,19 @@ static bool plan_decode_t(int64_t N, int64_t K, int num_sms, DecodePlan* p) {
   return true;
 }
 
-static bool plan_decode(bool int4, int NT, int64_t N, int64_t K, int num_sms, DecodePlan* p) {
-  if (int4) return NT == 1 ? plan_decode_t<true, 1>(N, K, num_sms, p) : plan_decode_t<true, 2>(N, K, num_sms, p);
-  return NT == 1 ? plan_decode_t<false, 1>(N, K, num_sms, p) : plan_decode_t<false, 2>(N, K, num_sms, p);
+static bool plan_decode(bool int4, int NT, int64_t RB, int64_t K, int num_sms, DecodePlan* p) {
+  if (int4) return NT == 1 ? plan_decode_t<true, 1>(RB, K, num_sms, p) : plan_decode_t<true, 2>(RB, K, num_sms, p);
+  return NT == 1 ? plan_decode_t<false, 1>(RB, K, num_sms, p) : plan_decode_t<false, 2>(RB, K, num_sms, p);
 }
 
 template <bool kInt4, int NT>
-static cudaError_t launch_decode_t(const CUtensorMap& tmap, const DecodeArgs& a, const DecodePlan& p,
+static cudaError_t launch_decode_t(const DecodeMaps& maps, const DecodeArgs& a, const DecodePlan& p,
                                    cudaStream_t s) {
   auto* kern = decode_gemm_kernel<kInt4, NT>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), p.smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(p.S), static_cast<unsigned>((a.N + kDRows - 1) / kDRows), 1);
+  cfg.gridDim = dim3(static_cast<unsigned>(p.S), static_cast<unsigned>(a.rb_start[a.count]), 1);
   cfg.blockDim = dim3(kDThreads, 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(p.smem);
   cfg.stream = s;
@@ -492,54 +510,86 @@ static cudaError_t launch_decode_t(const CUtensorMap& tmap, const DecodeArgs& a,
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, kern, tmap, a);
+  return cudaLaunchKernelEx(&cfg, kern, maps, a);
 }
 
+// One launch for `count` matrices that share x (same M and K): y_g = x . What_g^T (+ bias_g).
 template <bool kInt4>
-static cudaError_t launch_decode(const __half* x, const void* w, const __half* sc,
-                                 const __half* bias, __half* y, int64_t M, int64_t N, int64_t K,
-                                 cudaStream_t s) {
+static cudaError_t launch_decode_group(const __half* x, int count, const void* const* w,
+                                       const __half* const* sc, const __half* const* bias,
+                                       __half* const* y, const int64_t* N, int64_t M, int64_t K,
+                                       cudaStream_t s) {
+  if (count < 1 || count > kDMaxGroup) return cudaErrorInvalidValue;
   const DeviceInfo di = current_device_info();
   const int NT = M > 8 ? 2 : 1;
-  DecodePlan p;
-  if (!plan_decode(kInt4, NT, N, K, di.num_sms, &p)) return cudaErrorInvalidValue;
-  const int64_t kbytes = kInt4 ? K / 2 : K / 4;
-  CUtensorMap tmap;
-  if (!make_tmap_2d(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, w, static_cast<uint64_t>(kbytes),
-                    static_cast<uint64_t>(N), static_cast<uint64_t>(kbytes), 128, kDRows,
-                    CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
-  DecodeArgs a;
+  DecodeArgs a = {};
+  DecodeMaps maps;
   a.x = x;
-  a.sc = sc;
-  a.bias = bias;
-  a.y = y;
   a.M = M;
-  a.N = N;
   a.K = K;
+  a.count = count;
+  int64_t rbs = 0;
+  const int64_t kbytes = kInt4 ? K / 2 : K / 4;
+  for (int g = 0; g < count; ++g) {
+    a.rb_start[g] = static_cast<int>(rbs);
+    rbs += (N[g] + kDRows - 1) / kDRows;
+    a.N[g] = N[g];
+    a.sc[g] = sc[g];
+    a.bias[g] = bias ? bias[g] : nullptr;
+    a.y[g] = y[g];
+    if (!make_tmap_2d(&maps.m[g], CU_TENSOR_MAP_DATA_TYPE_UINT8, w[g], static_cast<uint64_t>(kbytes),
+                      static_cast<uint64_t>(N[g]), static_cast<uint64_t>(kbytes), 128, kDRows,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
+  for (int g = count; g < kDMaxGroup; ++g) maps.m[g] = maps.m[0];
+  a.rb_start[count] = static_cast<int>(rbs);
+  if (rbs > 65535) return cudaErrorInvalidValue;
+  DecodePlan p;
+  if (!plan_decode(kInt4, NT, rbs, K, di.num_sms, &p)) return cudaErrorInvalidValue;
   a.C = p.C;
   a.S = p.S;
   a.ring = p.ring;
-  return NT == 1 ? launch_decode_t<kInt4, 1>(tmap, a, p, s) : launch_decode_t<kInt4, 2>(tmap, a, p, s);
+  return NT == 1 ? launch_decode_t<kInt4, 1>(maps, a, p, s) : launch_decode_t<kInt4, 2>(maps, a, p, s);
 }
 
 bool decode_supported(bool int4, int64_t M, int64_t N, int64_t K) {
   if (M < 1 || M > 16 || N < 1) return false;
   if (int4 ? (K % 128 != 0) : (K % 64 != 0)) return false;
   DecodePlan p;
-  return plan_decode(int4, M > 8 ? 2 : 1, N, K, 148, &p);
+  return plan_decode(int4, M > 8 ? 2 : 1, (N + kDRows - 1) / kDRows, K, 148, &p);
 }
 
 cudaError_t launch_tq_gemm_decode(const __half* x, const uint8_t* packed, const __half* scale,
                                   const __half* bias, __half* y, int64_t M, int64_t N, int64_t K,
                                   cudaStream_t s) {
-  return launch_decode<false>(x, packed, scale, bias, y, M, N, K, s);
+  const void* w = packed;
+  return launch_decode_group<false>(x, 1, &w, &scale, &bias, &y, &N, M, K, s);
 }
 
 cudaError_t launch_w4g_gemm_decode(const __half* x, const int32_t* qweight, const __half* scales,
                                    const __half* bias, __half* y, int64_t M, int64_t N, int64_t K,
                                    cudaStream_t s) {
-  return launch_decode<true>(x, qweight, scales, bias, y, M, N, K, s);
+  const void* w = qweight;
+  return launch_decode_group<true>(x, 1, &w, &scales, &bias, &y, &N, M, K, s);
+}
+
+cudaError_t launch_tq_gemm_decode_group(const __half* x, int count, const uint8_t* const* packed,
+                                        const __half* const* scale, const __half* const* bias,
+                                        __half* const* y, const int64_t* N, int64_t M, int64_t K,
+                                        cudaStream_t s) {
+  const void* w[kDMaxGroup];
+  for (int g = 0; g < count && g < kDMaxGroup; ++g) w[g] = packed[g];
+  return launch_decode_group<false>(x, count, w, scale, bias, y, N, M, K, s);
+}
+
+cudaError_t launch_w4g_gemm_decode_group(const __half* x, int count, const int32_t* const* qweight,
+                                         const __half* const* scales, const __half* const* bias,
+                                         __half* const* y, const int64_t* N, int64_t M, int64_t K,
+                                         cudaStream_t s) {
+  const void* w[kDMaxGroup];
+  for (int g = 0; g < count && g < kDMaxGroup; ++g) w[g] = qweight[g];
+  return launch_decode_group<true>(x, count, w, scales, bias, y, N, M, K, s);
 }
 
 }  // namespace tq

@@ -137,6 +137,31 @@ TQ_API int w4g_gemm_ex(const uint16_t* x, const int32_t* qweight, const uint16_t
                 const uint16_t* bias, uint16_t* y, int64_t M, int64_t N, int64_t K, int path,
                 void* stream);
 
+/* --------------------------------------------------------------------------------------------
+ * tq_gemm_grouped / w4g_gemm_grouped -- several linears that read the same input, as a serving
+ * engine's fused q/k/v or gate/up projections do: for g < count,
+ *     y_g[M, N_g] = x[M, K] . What_g[N_g, K]^T (+ bias_g)
+ * Same results contract as `count` separate tq_gemm / w4g_gemm calls (each element within the
+ * stated bound; the split of K over CTAs may differ, so the bits may differ).  With M <= 16 on
+ * shapes the decode path takes, all matrices run in ONE kernel launch (one kernel boundary
+ * instead of `count`); otherwise the call issues `count` single-matrix GEMMs.
+ *   count              1 .. 4
+ *   packed / qweight   HOST array of `count` device pointers (layouts as in tq_gemm / w4g_gemm)
+ *   scale / scales     HOST array of `count` device pointers
+ *   bias               NULL (no bias) or a HOST array of `count` device pointers, each nullable
+ *   y                  HOST array of `count` device pointers to [M, N_g] fp16 outputs
+ *   N                  HOST array of `count` row counts
+ * The host arrays are read during the call only.  Errors as in tq_gemm (TQ_ERR_SHAPE for count
+ * outside 1..4 or a negative N_g).
+ * ------------------------------------------------------------------------------------------ */
+TQ_API int tq_gemm_grouped(const uint16_t* x, int count, const uint8_t* const* packed,
+                           const uint16_t* const* scale, const uint16_t* const* bias,
+                           uint16_t* const* y, const int64_t* N, int64_t M, int64_t K, void* stream);
+TQ_API int w4g_gemm_grouped(const uint16_t* x, int count, const int32_t* const* qweight,
+                            const uint16_t* const* scales, const uint16_t* const* bias,
+                            uint16_t* const* y, const int64_t* N, int64_t M, int64_t K,
+                            void* stream);
+
 /* tq_validate_packed -- count the bytes of a packed ternary matrix [N, ceil(K/4)] that hold
  * the unused code 0b11 in one of their first K codes of the row ([TQ] §3.1: the table maps
  * 00/01/10 only).  *bad_count (device int) is OVERWRITTEN with the count (set to 0 first, on

@@ -10,7 +10,7 @@ import bit_weight_only_tq_b200 as tq
 
 def test_library_exports_every_header_function():
     names = tq.header_functions()
-    assert len(names) == 11
+    assert len(names) == 13
     for n in names:
         assert hasattr(tq.lib, n), n
     for n in ("tq_quantize_pack", "tq_gemm", "w4g_quantize_pack", "w4g_gemm", "tq_validate_packed",
@@ -87,3 +87,16 @@ def test_dispatch_rule():
     assert tq.tq_select_path(W, 1, 4096, 4000) == -2
     assert tq.tq_select_path(T, 1, 4096, 0) == -2
     assert tq.tq_select_path(5, 1, 4096, 4096) == -8
+
+
+def test_grouped_argument_errors_without_gpu():
+    p = ctypes.c_void_p(4096)
+    arr = (ctypes.c_void_p * 3)(4096, 4096, 4096)
+    ns = (ctypes.c_int64 * 3)(64, 64, 64)
+    assert tq.lib.tq_gemm_grouped(p, 0, arr, arr, None, arr, ns, 1, 64, None) == -2   # count
+    assert tq.lib.tq_gemm_grouped(p, 5, arr, arr, None, arr, ns, 1, 64, None) == -2
+    assert tq.lib.tq_gemm_grouped(p, 3, None, arr, None, arr, ns, 1, 64, None) == -1  # null array
+    bad = (ctypes.c_int64 * 3)(64, -1, 64)
+    assert tq.lib.tq_gemm_grouped(p, 3, arr, arr, None, arr, bad, 1, 64, None) == -2
+    assert tq.lib.w4g_gemm_grouped(p, 3, arr, arr, None, arr, ns, 1, 100, None) == -2  # K % 128
+    assert tq.lib.tq_gemm_grouped(p, 3, arr, arr, None, arr, ns, 0, 64, None) == 0    # M = 0
