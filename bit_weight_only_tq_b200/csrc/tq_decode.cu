@@ -4,18 +4,21 @@
 // of packed codes; [TQ] §4.2: codes are decoded into fp16 tensor-core fragments, accumulated in
 // fp32, and the per-row scale is applied after the MMA.
 //
-// Work layout.  One CTA = 128 output rows x one K-slice; a cluster of S CTAs (S <= 8) covers
-// the whole K of its 128 rows and reduces through distributed shared memory in a fixed order
-// (deterministic, no global scratch).  Per CTA:
+// Work layout.  One CTA = one block of output rows (127 ternary rows plus one virtual row, or 128
+// W4A16 rows) x one K-slice; a cluster of S CTAs (S <= 8) covers the whole K of its rows and
+// reduces through distributed shared memory in a fixed order (deterministic, no global scratch).
+// A stage is 128 bytes of every packed row (512 ternary or 256 INT4 codes) plus the activations
+// of those k for all M tokens.  Per CTA:
+//   * warp 4 (producer) streams each stage with TMA into a ring: the 128-row x 128-byte packed
+//     tile (issued before griddepcontrol.wait, weights never depend on the previous kernel) and
+//     the activations, one 64-element block x M tokens per box (issued after it), both
+//     128-byte swizzled so that every 16-byte read below is bank-conflict free.  For W4A16 it
+//     also sums each 128-wide group of x per token;
 //   * warps 0-3 (consumers) each own 32 rows = two 16-row MMA tiles.  Weights are the A operand
 //     of mma.sync.m16n8k16 ("swap AB"), the tokens the N = 8 operand: one MMA per 256 weights
-//     for M <= 8, two for M <= 16;
-//   * warp 4 (producer): lane 0 streams 128-row x 128-byte packed tiles with TMA (128-byte
-//     swizzle: the 16-byte fragment reads are bank-conflict free) into a ring, starting before
-//     griddepcontrol.wait because weights never depend on the previous kernel; all 32 lanes then
-//     copy the activations of each stage (cp.async, padded, conflict-free), rearrange them into
-//     ready-made B fragments in the k order the decode produces (byte permutes), and compute the
-//     per-token sums of x on the tensor core (an MMA with an all-ones A).
+//     for M <= 8, two for M <= 16.  Each lane builds its B fragments from the activations in
+//     shared memory (byte permutes into the k order the decode produces, see below); with two
+//     row tiles per warp one fragment feeds four MMAs.
 //
 // In-register decode ("subnormal" trick).  ANDing a packed 32-bit word with 0x00030003 << 2p
 // leaves, in each fp16 half, the code at bits 2p..2p+1: the exact value c * 2^(2p-24) (fp16
@@ -23,10 +26,10 @@
 // exponent bits).  Positions 6, 7 are shifted down by 12 first.  So one word of 16 codes costs
 // 1 shift + 8 ANDs for 8 fp16x2 registers, ~0.56 integer operations per weight.  The odd
 // positions carry an extra factor 4, folded into their activation fragments (x / 4); the
-// remaining factors 2^-24, 2^-20, 2^-16 are kept apart in separate accumulators and applied
-// exactly (powers of two) in the epilogue, which also subtracts sum_k x (codes are c = w + 1).
-// One accumulator per position pair keeps the dependent MMA chains short (latency, not issue,
-// bounds a skinny GEMM).
+// factors 2^-24 (position pairs 0 and 3), 2^-20 (pair 1) and 2^-16 (pair 2) are kept in three
+// accumulators and applied exactly (powers of two) after the loop.  The codes are c = w + 1, so
+// the result is sum_k c x - sum_k x; sum_k x comes out of the same MMAs as a virtual 128th row
+// whose codes are all 01 (c = 1).
 // W4A16 uses the same scheme with 4-bit fields (masks 0x000F000F / 0x00F000F0, x / 16 fold) and
 // one 128-wide quantisation group per 64-byte sub-chunk: y += s[n,g] * (2^24 * C_g - 8 sum_g x).
 #include <cuda.h>
@@ -38,42 +41,34 @@
 
 namespace tq {
 
-constexpr int kDRows = 128;                 // output rows per CTA
-constexpr int kDConsumers = 8;              // consumer warps (16 rows = one MMA tile each)
-constexpr int kDRT = kDRows / (16 * kDConsumers);  // 16-row MMA tiles per consumer warp
-constexpr int kDBuilders = 2;               // activation warps: one per 64-byte sub-chunk
-constexpr int kDBuildWarp0 = kDConsumers;
-constexpr int kDTmaWarp = kDConsumers + kDBuilders;  // issues the weight TMA stream
-constexpr int kDThreads = (kDConsumers + kDBuilders + 1) * 32;
-constexpr int kDStageBytes = kDRows * 128;  // one TMA box: 128 rows x 128 bytes
-constexpr int kDMaxRing = 6;                // weight stages resident in shared memory
-constexpr int kDXRing = 2;                  // activation-fragment stages
+constexpr int kDTile = 128;                 // rows of one packed TMA tile
+constexpr int kDConsumers = 4;              // consumer warps (32 rows = two MMA tiles each)
+constexpr int kDRT = 2;                     // 16-row MMA tiles per consumer warp
+constexpr int kDProducer = kDConsumers;     // TMA warp
+constexpr int kDThreads = (kDConsumers + 1) * 32;
+constexpr int kDWBytes = kDTile * 128;      // weights of one stage: 128 rows x 128 bytes
+constexpr int kDMaxRing = 8;                // stages resident in shared memory
 constexpr int kDMaxCluster = 8;
-constexpr int kDRedRows = kDRows + kDMaxCluster;  // >= S * ceil(128 / S)
+constexpr int kDRedRows = kDTile + kDMaxCluster;  // >= S * ceil(rows / S)
 constexpr int kDSmemBudget = 113 * 1024;    // two CTAs per SM
 
 template <bool kInt4>
 struct DecFmt {
   static constexpr int kStageK = kInt4 ? 256 : 512;  // codes per stage (128 bytes of a row)
-  static constexpr int kSubK = kStageK / 2;          // codes per 64-byte sub-chunk
-  static constexpr int kLaneK = kSubK / 4;           // codes per lane (16 bytes) per sub-chunk
-  static constexpr int kMmas = kInt4 ? 8 : 16;       // MMAs per 16-row tile per sub-chunk
-  static constexpr int kFragU4 = kMmas / 2;          // uint4 B fragments per lane per sub-chunk
-  static constexpr int kFragBytes = kFragU4 * 32 * 16;
-  static constexpr int kXLaneBytes = kLaneK * 2;     // activation bytes per lane per sub-chunk
-  static constexpr int kXStride = kXLaneBytes + 16;  // padded: conflict-free 16-byte reads
+  static constexpr int kKB = kStageK / 64;           // 64-element activation blocks per stage
+  static constexpr int kRows = kInt4 ? 128 : 127;    // real output rows per CTA
 };
 
 constexpr int kDMaxGroup = 4;  // weight matrices sharing x in one launch (e.g. q, k, v)
 
 struct DecodeArgs {
-  const __half* x;
   int64_t M, K;
-  int C;     // stages along K
-  int S;     // CTAs per cluster (K-slices)
-  int ring;  // weight stages resident in shared memory (all of a CTA's stages when they fit)
+  int C;          // stages along K
+  int S;          // CTAs per cluster (K-slices)
+  int ring;       // stages resident in shared memory
+  int stage;      // bytes of one stage (weights + activations, multiple of 1024)
   int count;                        // matrices in the group
-  int rb_start[kDMaxGroup + 1];     // first 128-row block of each matrix in grid.y
+  int rb_start[kDMaxGroup + 1];     // first row block of each matrix in grid.y
   int64_t N[kDMaxGroup];
   const __half* sc[kDMaxGroup];     // ternary: scale[N]; W4A16: scales[N, K/128]
   const __half* bias[kDMaxGroup];   // may be null
@@ -82,52 +77,69 @@ struct DecodeArgs {
 
 struct DecodeMaps {
   CUtensorMap m[kDMaxGroup];        // packed weights of each matrix
+  CUtensorMap x;                    // activations [M][K] fp16, box 64 x M, 128-byte swizzle
 };
 
-template <bool kInt4, int NT>
+template <bool kInt4>
 struct DecLayout {
-  using F = DecFmt<kInt4>;
-  static constexpr int kXfStage = 2 * NT * F::kFragBytes;      // B fragments of one stage
-  static constexpr int kXsSub = NT * 32 * F::kXStride;          // natural x of one sub-chunk
-  static constexpr int kXgStage = 2 * 16 * 4;                   // W4A16 group sums [sub][token]
+  static constexpr int kXg = kInt4 ? 2 * 16 * 4 : 0;  // W4A16 group sums of a stage [2][16]
   static constexpr int kRed = kDRedRows * 16 * 4;
   static constexpr int kSxr = kDMaxCluster * 16 * 4;
-  __host__ __device__ static constexpr int bytes(int ring) {
-    return 1024 + ring * kDStageBytes + kDXRing * (kXfStage + kXgStage) + 2 * kDBuilders * kXsSub +
-           kRed + kSxr + 2 * 16 * 4 + (2 * kDMaxRing + 2 * kDXRing) * 8;
-  }
+  __host__ __device__ static constexpr int fixed() { return 1024 + kRed + kSxr + 3 * kDMaxRing * 8; }
+  __host__ __device__ static constexpr int bytes(int ring, int stage) { return fixed() + ring * (stage + kXg); }
 };
 
+// 16-byte chunk c (0..7) of token row m of one activation block (128-byte swizzle: the chunk
+// index is XORed with the row index within the 1024-byte atom).
+__device__ __forceinline__ uint4 ld_x_chunk(const uint8_t* blk, int m, int c) {
+  return *reinterpret_cast<const uint4*>(blk + m * 128 + ((c ^ (m & 7)) << 4));
+}
+
+// B fragments of one MMA pair from four activation words: even positions (x) and odd positions
+// (x times `fold`), in the k order of the decode.
+__device__ __forceinline__ void make_frag(uint32_t Pa, uint32_t Pb, uint32_t Pc, uint32_t Pd,
+                                          __half2 fold, uint32_t& e0, uint32_t& e1, uint32_t& o0,
+                                          uint32_t& o1) {
+  e0 = __byte_perm(Pa, Pb, 0x5410);
+  e1 = __byte_perm(Pc, Pd, 0x5410);
+  uint32_t u01 = __byte_perm(Pa, Pb, 0x7632), u23 = __byte_perm(Pc, Pd, 0x7632);
+  __half2 s01 = __hmul2(*reinterpret_cast<__half2*>(&u01), fold);
+  __half2 s23 = __hmul2(*reinterpret_cast<__half2*>(&u23), fold);
+  o0 = *reinterpret_cast<uint32_t*>(&s01);
+  o1 = *reinterpret_cast<uint32_t*>(&s23);
+}
+
+// Two CTAs of five warps per SM (the launch bound keeps the registers within that).
 template <bool kInt4, int NT>
 __global__ void __launch_bounds__(kDThreads, 2)
     decode_gemm_kernel(const __grid_constant__ DecodeMaps maps, const __grid_constant__ DecodeArgs a) {
   using F = DecFmt<kInt4>;
-  using L = DecLayout<kInt4, NT>;
+  using L = DecLayout<kInt4>;
+  constexpr int kXSlot = 8 * NT * 128;  // one activation block: up to 8*NT token rows
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* wst = base;                                                // ring x 16 KB weight tiles
-  uint8_t* xf = wst + a.ring * kDStageBytes;                          // 2 x B fragments
-  float* xg = reinterpret_cast<float*>(xf + kDXRing * L::kXfStage);   // 2 x [2][16] group sums
-  uint8_t* xs = reinterpret_cast<uint8_t*>(xg + kDXRing * 2 * 16);    // [builder][2] natural x
-  float* red = reinterpret_cast<float*>(xs + 2 * kDBuilders * L::kXsSub);  // [S][rows/S][16]
-  float* sxr = red + kDRedRows * 16;                                  // [S][16] slice sums of x
-  float* sxb = sxr + kDMaxCluster * 16;                               // [builder][16] sums of x
-  uint64_t* wfull = reinterpret_cast<uint64_t*>(sxb + 2 * 16);
-  uint64_t* wempty = wfull + kDMaxRing;
-  uint64_t* xfull = wempty + kDMaxRing;     // B fragments of a stage built (builder warps)
-  uint64_t* xempty = xfull + kDXRing;       // ... and consumed (consumer warps)
+  // 1024-byte aligned; pointer arithmetic on the __shared__ array keeps the shared address
+  // space visible to the compiler (plain ld/st.shared instead of generic accesses)
+  uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* stg = base;                                                  // ring x [weights | x]
+  float* xg = reinterpret_cast<float*>(stg + a.ring * a.stage);         // ring x [2][16]
+  float* red = xg + a.ring * (L::kXg / 4);                              // [S][rows/S][16]
+  float* sxr = red + kDRedRows * 16;                                    // [S][16] slice sums of x
+  uint64_t* full = reinterpret_cast<uint64_t*>(sxr + kDMaxCluster * 16);
+  uint64_t* xready = full + kDMaxRing;  // W4A16 group sums of the stage written
+  uint64_t* empty = xready + kDMaxRing;
 
   pdl_allow_dependents();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int rank = static_cast<int>(cluster_ctarank());
-  // which matrix of the group this CTA works on, and its 128-row block within that matrix
+  // which matrix of the group this CTA works on, and its row block within that matrix
   int grp = 0;
 #pragma unroll
   for (int q = 1; q < kDMaxGroup; ++q)
     if (q < a.count && static_cast<int>(blockIdx.y) >= a.rb_start[q]) grp = q;
   const int rb = static_cast<int>(blockIdx.y) - a.rb_start[grp];
+  const int64_t row0 = static_cast<int64_t>(rb) * F::kRows;  // first output row of the block
   const CUtensorMap* tmap = &maps.m[grp];
   const int64_t Nm = a.N[grp];
   const __half* scm = a.sc[grp];
@@ -136,137 +148,112 @@ __global__ void __launch_bounds__(kDThreads, 2)
   const int st_begin = static_cast<int>((static_cast<int64_t>(rank) * a.C) / a.S);
   const int st_end = static_cast<int>((static_cast<int64_t>(rank + 1) * a.C) / a.S);
   const int nst = st_end - st_begin;
-  const int own_cap = (kDRows + a.S - 1) / a.S;  // row slots per owner in `red`
+  const int own_cap = (F::kRows + a.S - 1) / a.S;  // row slots per owner in `red`
+  const int Mi = static_cast<int>(a.M);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < a.ring; ++i) {
-      mbar_init(&wfull[i], 1);
-      mbar_init(&wempty[i], kDConsumers);
-    }
-    for (int i = 0; i < kDXRing; ++i) {
-      mbar_init(&xfull[i], kDBuilders * 32);
-      mbar_init(&xempty[i], kDConsumers);
+      mbar_init(&full[i], 1);
+      mbar_init(&xready[i], 32);
+      mbar_init(&empty[i], kDConsumers);
     }
     fence_mbar_init();
   }
   __syncthreads();
 
-  if (warp == kDTmaWarp) {
-    // ================================================================== weight TMA warp
+  // this thread's output row of the epilogue and its scale / bias, fetched before any wait
+  // (they never depend on the previous kernel) so that the epilogue does not wait on them
+  const int rr0 = (rank * F::kRows) / a.S, rr1 = ((rank + 1) * F::kRows) / a.S;
+  const int nrows = rr1 - rr0;
+  const int ep_row = threadIdx.x;
+  const int64_t ep_n = row0 + rr0 + ep_row;
+  const bool ep_on = ep_row < nrows && ep_n < Nm;
+  float ep_s = 1.0f, ep_b = 0.0f;
+  if (ep_on) {
+    if (!kInt4) ep_s = __half2float(scm[ep_n]);
+    if (biasm) ep_b = __half2float(biasm[ep_n]);
+  }
+
+  if (warp == kDProducer) {
+    // ================================================================== producer warp
+    const uint32_t tx = static_cast<uint32_t>(kDWBytes + F::kKB * Mi * 128);
+    auto load_w = [&](int i) {
+      tma_load_2d(stg + (i % a.ring) * a.stage, tmap, &full[i % a.ring], (st_begin + i) * 128,
+                  static_cast<int>(row0));
+    };
+    auto load_x = [&](int i) {
+      uint8_t* dst = stg + (i % a.ring) * a.stage + kDWBytes;
+#pragma unroll
+      for (int b = 0; b < F::kKB; ++b)
+        tma_load_2d(dst + b * kXSlot, &maps.x, &full[i % a.ring], (st_begin + i) * F::kStageK + 64 * b, 0);
+    };
+    const int pre = nst < a.ring ? nst : a.ring;
     if (lane == 0) {
       tma_prefetch_desc(tmap);
-      const int pre = nst < a.ring ? nst : a.ring;
+      tma_prefetch_desc(&maps.x);
       for (int i = 0; i < pre; ++i) {
-        mbar_arrive_expect_tx(&wfull[i], kDStageBytes);
-        tma_load_2d(wst + i * kDStageBytes, tmap, &wfull[i], (st_begin + i) * 128, rb * kDRows);
-      }
-      // refill each weight slot as soon as the consumers release it (they start only once the
-      // previous kernel is done, so block in griddepcontrol.wait instead of polling meanwhile)
-      if (a.ring < nst) pdl_wait_prior_grids();
-      for (int j = a.ring; j < nst; ++j) {
-        const int ws = j % a.ring;
-        if (!mbar_wait(&wempty[ws], static_cast<uint32_t>((j / a.ring) - 1) & 1u)) break;
-        mbar_arrive_expect_tx(&wfull[ws], kDStageBytes);
-        tma_load_2d(wst + ws * kDStageBytes, tmap, &wfull[ws], (st_begin + j) * 128, rb * kDRows);
+        mbar_arrive_expect_tx(&full[i], tx);
+        load_w(i);
       }
     }
-  } else if (warp >= kDBuildWarp0) {
-    // ================================================================== builder warps
-    // Builder `sub` owns the 64-byte sub-chunk `sub` of every stage: it copies those
-    // activations (cp.async, padded), lays them out as B fragments in the k order the decode
-    // produces (odd positions pre-scaled by 1/4 or 1/16), and sums x on the CUDA cores.
-    const int sub = warp - kDBuildWarp0;
-    pdl_wait_prior_grids();  // activations may come from the previous kernel
-    uint8_t* mybuf = xs + sub * 2 * L::kXsSub;
-    auto issue_x = [&](int i) {
-      if (i < nst) {
-        uint8_t* buf = mybuf + (i & 1) * L::kXsSub;
-#pragma unroll
-        for (int T = 0; T < NT; ++T) {
-          const int m = 8 * T + g;
-          const int64_t k0 = static_cast<int64_t>(st_begin + i) * F::kStageK + sub * F::kSubK + t * F::kLaneK;
-          const bool valid = (m < a.M) && (k0 < a.K);
-          const __half* src = valid ? a.x + m * a.K + k0 : a.x;
-          uint8_t* dst = buf + (T * 32 + lane) * F::kXStride;
-#pragma unroll
-          for (int j = 0; j < F::kXLaneBytes / 16; ++j)
-            cp_async_16(dst + 16 * j, src + (valid ? 8 * j : 0), valid ? 16u : 0u);
+    pdl_wait_prior_grids();  // the activations may come from the previous kernel
+    if (lane == 0)
+      for (int i = 0; i < pre; ++i) load_x(i);
+    if (!kInt4) {
+      if (lane == 0)
+        for (int j = a.ring; j < nst; ++j) {
+          const int slot = j % a.ring;
+          if (!mbar_wait(&empty[slot], static_cast<uint32_t>((j / a.ring) - 1) & 1u)) break;
+          mbar_arrive_expect_tx(&full[slot], tx);
+          load_w(j);
+          load_x(j);
         }
-      }
-      cp_async_commit();  // one group per stage (possibly empty) keeps the accounting uniform
-    };
-    issue_x(0);
-    issue_x(1);
-    const __half2 fold = kInt4 ? __floats2half2_rn(0.0625f, 0.0625f) : __floats2half2_rn(0.25f, 0.25f);
-    float sxl[NT];  // running sum of this lane's activations (ternary)
+    } else {
+      // group sums: lane -> token m = lane % (8*NT), block part = lane / (8*NT)
+      constexpr int MP = 8 * NT, PARTS = 32 / MP, KBL = F::kKB / PARTS;
+      const int m = lane % MP, part = lane / MP;
+      for (int i = 0; i < nst; ++i) {
+        const int slot = i % a.ring;
+        const uint32_t ph = static_cast<uint32_t>(i / a.ring) & 1u;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full[slot], ph))) break;  // warp-uniform exit
+        const uint8_t* xs = stg + slot * a.stage + kDWBytes;
+        float ps = 0.0f;
+        if (m < Mi) {
 #pragma unroll
-    for (int T = 0; T < NT; ++T) sxl[T] = 0.0f;
-    for (int i = 0; i < nst; ++i) {
-      const int xslot = i & 1;
-      if (i >= kDXRing && !mbar_wait(&xempty[xslot], static_cast<uint32_t>((i >> 1) - 1) & 1u)) break;
-      cp_async_wait<1>();  // this lane's copies of stage i have landed
-      const uint8_t* buf = mybuf + (i & 1) * L::kXsSub;
-      uint4* xfs = reinterpret_cast<uint4*>(xf + xslot * L::kXfStage);
+          for (int bb = 0; bb < KBL; ++bb) {
+            const uint8_t* blk = xs + (part * KBL + bb) * kXSlot;
 #pragma unroll
-      for (int T = 0; T < NT; ++T) {
-        const uint4* src = reinterpret_cast<const uint4*>(buf + (T * 32 + lane) * F::kXStride);
-        uint32_t P[F::kLaneK / 2];
+            for (int c = 0; c < 8; ++c) {
+              const uint4 v = ld_x_chunk(blk, m, c);
+              const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int j = 0; j < F::kLaneK / 8; ++j) {
-          const uint4 v = src[j];
-          P[4 * j] = v.x;
-          P[4 * j + 1] = v.y;
-          P[4 * j + 2] = v.z;
-          P[4 * j + 3] = v.w;
-        }
-        float ps = 0.0f;  // sum of this lane's activations in the sub-chunk (fixed order)
-#pragma unroll
-        for (int j = 0; j < F::kLaneK / 2; ++j) {
-          const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&P[j]));
-          ps += f2.x + f2.y;
-        }
-#pragma unroll
-        for (int f = 0; f < F::kFragU4; ++f) {
-          uint32_t Pa, Pb, Pc, Pd;
-          if (!kInt4) {  // f = h*4 + pp: positions p = 2pp (even), 2pp+1 (odd) of word pair h
-            const int h = f >> 2, pp = f & 3;
-            Pa = P[16 * h + pp];
-            Pb = P[16 * h + 4 + pp];
-            Pc = P[16 * h + 8 + pp];
-            Pd = P[16 * h + 12 + pp];
-          } else {       // f = h*2 + s: nibble positions 2s (class 0), 2s+1 (class 1)
-            const int h = f >> 1, s2 = f & 1;
-            Pa = P[8 * h + s2];
-            Pb = P[8 * h + 2 + s2];
-            Pc = P[8 * h + 4 + s2];
-            Pd = P[8 * h + 6 + s2];
+              for (int j = 0; j < 4; ++j) {
+                const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&u[j]));
+                ps += f2.x + f2.y;
+              }
+            }
           }
-          const uint32_t e01 = __byte_perm(Pa, Pb, 0x5410), e23 = __byte_perm(Pc, Pd, 0x5410);
-          uint32_t o01 = __byte_perm(Pa, Pb, 0x7632), o23 = __byte_perm(Pc, Pd, 0x7632);
-          __half2 so01 = __hmul2(*reinterpret_cast<__half2*>(&o01), fold);
-          __half2 so23 = __hmul2(*reinterpret_cast<__half2*>(&o23), fold);
-          xfs[((sub * NT + T) * F::kFragU4 + f) * 32 + lane] =
-              make_uint4(e01, e23, *reinterpret_cast<uint32_t*>(&so01), *reinterpret_cast<uint32_t*>(&so23));
         }
-        ps += __shfl_xor_sync(0xFFFFFFFFu, ps, 1);  // the four lanes of one token
-        ps += __shfl_xor_sync(0xFFFFFFFFu, ps, 2);
-        if (kInt4) {
-          if (t == 0) xg[(xslot * 2 + sub) * 16 + 8 * T + g] = ps;
-        } else {
-          sxl[T] += ps;
+        // a group is 128 elements = 2 blocks: combine the two parts of one group
+        if (KBL == 1) ps += __shfl_xor_sync(0xFFFFFFFFu, ps, MP);
+        const int gq = (part * KBL) >> 1;
+        if (KBL == 2 || (part & 1) == 0) xg[(slot * 2 + gq) * 16 + m] = ps;
+        mbar_arrive(&xready[slot]);
+        const int j = i + a.ring;
+        if (j < nst) {
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait(&empty[slot], ph))) break;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&full[slot], tx);
+            load_w(j);
+            load_x(j);
+          }
         }
       }
-      mbar_arrive(&xfull[xslot]);
-      issue_x(i + 2);
-    }
-    cp_async_wait<0>();
-    if (!kInt4 && t == 0) {
-#pragma unroll
-      for (int T = 0; T < NT; ++T) sxb[sub * 16 + 8 * T + g] = sxl[T];
     }
   } else {
     // ================================================================== consumer warps
-    constexpr int NG = kInt4 ? 1 : 4;  // accumulator groups: one per position pair (chains)
+    // accumulator groups by exact power-of-two factor: pairs 0 and 3 (2^-24), 1 (2^-20), 2 (2^-16)
+    constexpr int NG = kInt4 ? 1 : 3;
     float acc[NG][kDRT][NT][4];
 #pragma unroll
     for (int q = 0; q < NG; ++q)
@@ -276,43 +263,69 @@ __global__ void __launch_bounds__(kDThreads, 2)
         for (int T = 0; T < NT; ++T)
 #pragma unroll
           for (int c = 0; c < 4; ++c) acc[q][rt][T][c] = 0.0f;
+    bool tokv[NT];
+#pragma unroll
+    for (int T = 0; T < NT; ++T) tokv[T] = 8 * T + g < Mi;
+    const __half2 fold = kInt4 ? __floats2half2_rn(0.0625f, 0.0625f) : __floats2half2_rn(0.25f, 0.25f);
+    const int rw = warp * 16 * kDRT + g;  // row of tile 0, lower half; tile rt adds 16 rt, upper +8
+    // ternary: tile row 127 is the virtual all-01 row (its result is sum_k x)
+    const bool virt = !kInt4 && rw + 16 * (kDRT - 1) + 8 == kDTile - 1;
     const int64_t G = a.K >> 7;
-    pdl_wait_prior_grids();  // block (not poll) until the activations can exist
+    pdl_wait_prior_grids();  // block (not poll) until the previous kernel is done
     for (int i = 0; i < nst; ++i) {
-      const int ws = i % a.ring, xslot = i & 1;
-      if (!mbar_wait(&wfull[ws], static_cast<uint32_t>(i / a.ring) & 1u) ||
-          !mbar_wait(&xfull[xslot], static_cast<uint32_t>(i >> 1) & 1u))
-        break;
-      const uint8_t* st = wst + ws * kDStageBytes;
-      const uint4* xfs = reinterpret_cast<const uint4*>(xf + xslot * L::kXfStage);
-#pragma unroll
+      const int slot = i % a.ring;
+      const uint32_t ph = static_cast<uint32_t>(i / a.ring) & 1u;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full[slot], ph))) break;  // warp-uniform exit
+      const uint8_t* st = stg + slot * a.stage;
+      const uint8_t* xs = st + kDWBytes;
+#pragma unroll 1
       for (int sub = 0; sub < 2; ++sub) {
-        const int chunk = sub * 4 + t;
-        uint32_t w0[kDRT][4], w1[kDRT][4];
+        const int chunk = sub * 4 + t;  // this lane's 16 bytes of the packed rows
+        // rows rw + 16 rt + 8 hr all have (row & 7) == g: swizzled chunk position chunk ^ g
+        uint32_t w[kDRT][2][4];
 #pragma unroll
-        for (int rt = 0; rt < kDRT; ++rt) {
-          const int r0 = warp * (16 * kDRT) + rt * 16 + g, r1 = r0 + 8;
-          const uint4 U0 = *reinterpret_cast<const uint4*>(st + r0 * 128 + ((chunk ^ (r0 & 7)) << 4));
-          const uint4 U1 = *reinterpret_cast<const uint4*>(st + r1 * 128 + ((chunk ^ (r1 & 7)) << 4));
-          w0[rt][0] = U0.x; w0[rt][1] = U0.y; w0[rt][2] = U0.z; w0[rt][3] = U0.w;
-          w1[rt][0] = U1.x; w1[rt][1] = U1.y; w1[rt][2] = U1.z; w1[rt][3] = U1.w;
-        }
+        for (int rt = 0; rt < kDRT; ++rt)
+#pragma unroll
+          for (int hr = 0; hr < 2; ++hr) {
+            uint4 U = *reinterpret_cast<const uint4*>(st + (rw + 16 * rt + 8 * hr) * 128 + ((chunk ^ g) << 4));
+            if (virt && rt == kDRT - 1 && hr == 1) U = make_uint4(0x55555555u, 0x55555555u, 0x55555555u, 0x55555555u);
+            w[rt][hr][0] = U.x;
+            w[rt][hr][1] = U.y;
+            w[rt][hr][2] = U.z;
+            w[rt][hr][3] = U.w;
+          }
         if (!kInt4) {
+          // the 64 codes of the chunk are k = 64*chunk + 0..63: activation block `chunk`
+          const uint8_t* blk = xs + chunk * kXSlot;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
+            // P[T][j] = x[8T+g][64*chunk + 32h + 2j .. +1]
+            uint32_t P[NT][16];
+#pragma unroll
+            for (int T = 0; T < NT; ++T)
+#pragma unroll
+              for (int jj = 0; jj < 4; ++jj) {
+                uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                if (tokv[T]) v = ld_x_chunk(blk, 8 * T + g, 4 * h + jj);
+                P[T][4 * jj] = v.x;
+                P[T][4 * jj + 1] = v.y;
+                P[T][4 * jj + 2] = v.z;
+                P[T][4 * jj + 3] = v.w;
+              }
             uint32_t sh[kDRT][4];
 #pragma unroll
             for (int rt = 0; rt < kDRT; ++rt) {
-              sh[rt][0] = w0[rt][2 * h] >> 12;
-              sh[rt][1] = w1[rt][2 * h] >> 12;
-              sh[rt][2] = w0[rt][2 * h + 1] >> 12;
-              sh[rt][3] = w1[rt][2 * h + 1] >> 12;
+              sh[rt][0] = w[rt][0][2 * h] >> 12;
+              sh[rt][1] = w[rt][1][2 * h] >> 12;
+              sh[rt][2] = w[rt][0][2 * h + 1] >> 12;
+              sh[rt][3] = w[rt][1][2 * h + 1] >> 12;
             }
 #pragma unroll
             for (int pp = 0; pp < 4; ++pp) {
-              uint4 B[NT];
+              uint32_t be0[NT], be1[NT], bo0[NT], bo1[NT];
 #pragma unroll
-              for (int T = 0; T < NT; ++T) B[T] = xfs[((sub * NT + T) * 8 + h * 4 + pp) * 32 + lane];
+              for (int T = 0; T < NT; ++T)
+                make_frag(P[T][pp], P[T][4 + pp], P[T][8 + pp], P[T][12 + pp], fold, be0[T], be1[T], bo0[T], bo1[T]);
 #pragma unroll
               for (int q = 0; q < 2; ++q) {
                 const int p = 2 * pp + q;
@@ -321,10 +334,10 @@ __global__ void __launch_bounds__(kDThreads, 2)
                   uint32_t a0, a1, a2, a3;
                   if (p < 6) {
                     const uint32_t mk = 0x00030003u << (2 * p);
-                    a0 = w0[rt][2 * h] & mk;
-                    a1 = w1[rt][2 * h] & mk;
-                    a2 = w0[rt][2 * h + 1] & mk;
-                    a3 = w1[rt][2 * h + 1] & mk;
+                    a0 = w[rt][0][2 * h] & mk;
+                    a1 = w[rt][1][2 * h] & mk;
+                    a2 = w[rt][0][2 * h + 1] & mk;
+                    a3 = w[rt][1][2 * h + 1] & mk;
                   } else {
                     const uint32_t mk = (p == 6) ? 0x00030003u : 0x000C000Cu;
                     a0 = sh[rt][0] & mk;
@@ -334,47 +347,70 @@ __global__ void __launch_bounds__(kDThreads, 2)
                   }
 #pragma unroll
                   for (int T = 0; T < NT; ++T)
-                    mma_16816(acc[pp % NG][rt][T], a0, a1, a2, a3, q ? B[T].z : B[T].x, q ? B[T].w : B[T].y);
+                    mma_16816(acc[pp == 3 ? 0 : pp][rt][T], a0, a1, a2, a3, q ? bo0[T] : be0[T], q ? bo1[T] : be1[T]);
                 }
               }
             }
           }
         } else {
-          const int64_t gi = static_cast<int64_t>(st_begin + i) * 2 + sub;
-          float xgt[NT][2];
+          // the 32 codes of the chunk are k = 32*chunk + 0..31: half (chunk & 1) of activation
+          // block chunk / 2, its 16-byte chunks 4*(chunk & 1) + 0..3
+          const uint8_t* blk = xs + (chunk >> 1) * kXSlot;
+          uint32_t P[NT][16];
 #pragma unroll
-          for (int T = 0; T < NT; ++T) {
-            xgt[T][0] = 8.0f * xg[(xslot * 2 + sub) * 16 + 8 * T + 2 * t];
-            xgt[T][1] = 8.0f * xg[(xslot * 2 + sub) * 16 + 8 * T + 2 * t + 1];
-          }
+          for (int T = 0; T < NT; ++T)
 #pragma unroll
-          for (int rt = 0; rt < kDRT; ++rt) {
-            float cg[2][NT][4];  // two chains (class 0 / class 1 fields)
+            for (int jj = 0; jj < 4; ++jj) {
+              uint4 v = make_uint4(0u, 0u, 0u, 0u);
+              if (tokv[T]) v = ld_x_chunk(blk, 8 * T + g, 4 * (chunk & 1) + jj);
+              P[T][4 * jj] = v.x;
+              P[T][4 * jj + 1] = v.y;
+              P[T][4 * jj + 2] = v.z;
+              P[T][4 * jj + 3] = v.w;
+            }
+          float cg[2][kDRT][NT][4];  // two chains (class 0 / class 1 fields)
 #pragma unroll
-            for (int j = 0; j < 2; ++j)
+          for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int rt = 0; rt < kDRT; ++rt)
 #pragma unroll
               for (int T = 0; T < NT; ++T)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) cg[j][T][c] = 0.0f;
+                for (int c = 0; c < 4; ++c) cg[j][rt][T][c] = 0.0f;
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
+          for (int h = 0; h < 2; ++h)
 #pragma unroll
-              for (int s2 = 0; s2 < 2; ++s2) {
-                const uint32_t x0 = w0[rt][2 * h] >> (8 * s2), x1 = w1[rt][2 * h] >> (8 * s2);
-                const uint32_t x2 = w0[rt][2 * h + 1] >> (8 * s2), x3 = w1[rt][2 * h + 1] >> (8 * s2);
-                uint4 B[NT];
+            for (int s2 = 0; s2 < 2; ++s2) {
+              uint32_t be0[NT], be1[NT], bo0[NT], bo1[NT];
 #pragma unroll
-                for (int T = 0; T < NT; ++T) B[T] = xfs[((sub * NT + T) * 4 + h * 2 + s2) * 32 + lane];
+              for (int T = 0; T < NT; ++T)
+                make_frag(P[T][8 * h + s2], P[T][8 * h + 2 + s2], P[T][8 * h + 4 + s2], P[T][8 * h + 6 + s2], fold,
+                          be0[T], be1[T], bo0[T], bo1[T]);
+#pragma unroll
+              for (int rt = 0; rt < kDRT; ++rt) {
+                const uint32_t x0 = w[rt][0][2 * h] >> (8 * s2), x1 = w[rt][1][2 * h] >> (8 * s2);
+                const uint32_t x2 = w[rt][0][2 * h + 1] >> (8 * s2), x3 = w[rt][1][2 * h + 1] >> (8 * s2);
 #pragma unroll
                 for (int cls = 0; cls < 2; ++cls) {
                   const uint32_t mk = cls ? 0x00F000F0u : 0x000F000Fu;
 #pragma unroll
                   for (int T = 0; T < NT; ++T)
-                    mma_16816(cg[cls][T], x0 & mk, x1 & mk, x2 & mk, x3 & mk, cls ? B[T].z : B[T].x,
-                              cls ? B[T].w : B[T].y);
+                    mma_16816(cg[cls][rt][T], x0 & mk, x1 & mk, x2 & mk, x3 & mk, cls ? bo0[T] : be0[T],
+                              cls ? bo1[T] : be1[T]);
                 }
               }
-            const int64_t n0 = static_cast<int64_t>(rb) * kDRows + warp * (16 * kDRT) + rt * 16 + g, n1 = n0 + 8;
+            }
+          if (sub == 0) (void)__all_sync(0xFFFFFFFFu, mbar_wait(&xready[slot], ph));
+          const int64_t gi = static_cast<int64_t>(st_begin + i) * 2 + sub;
+          float xg0[NT], xg1[NT];
+#pragma unroll
+          for (int T = 0; T < NT; ++T) {
+            xg0[T] = 8.0f * xg[(slot * 2 + sub) * 16 + 8 * T + 2 * t];
+            xg1[T] = 8.0f * xg[(slot * 2 + sub) * 16 + 8 * T + 2 * t + 1];
+          }
+#pragma unroll
+          for (int rt = 0; rt < kDRT; ++rt) {
+            const int64_t n0 = row0 + rw + 16 * rt, n1 = n0 + 8;
             // groups past K (a zero-filled half stage) contribute nothing
             const float s0 = (n0 < Nm && gi < G) ? __half2float(scm[n0 * G + gi]) : 0.0f;
             const float s1 = (n1 < Nm && gi < G) ? __half2float(scm[n1 * G + gi]) : 0.0f;
@@ -382,32 +418,29 @@ __global__ void __launch_bounds__(kDThreads, 2)
             for (int T = 0; T < NT; ++T) {
               float c4[4];
 #pragma unroll
-              for (int c = 0; c < 4; ++c) c4[c] = cg[0][T][c] + cg[1][T][c];
-              acc[0][rt][T][0] = fmaf(s0, fmaf(c4[0], 16777216.0f, -xgt[T][0]), acc[0][rt][T][0]);
-              acc[0][rt][T][1] = fmaf(s0, fmaf(c4[1], 16777216.0f, -xgt[T][1]), acc[0][rt][T][1]);
-              acc[0][rt][T][2] = fmaf(s1, fmaf(c4[2], 16777216.0f, -xgt[T][0]), acc[0][rt][T][2]);
-              acc[0][rt][T][3] = fmaf(s1, fmaf(c4[3], 16777216.0f, -xgt[T][1]), acc[0][rt][T][3]);
+              for (int c = 0; c < 4; ++c) c4[c] = cg[0][rt][T][c] + cg[1][rt][T][c];
+              acc[0][rt][T][0] = fmaf(s0, fmaf(c4[0], 16777216.0f, -xg0[T]), acc[0][rt][T][0]);
+              acc[0][rt][T][1] = fmaf(s0, fmaf(c4[1], 16777216.0f, -xg1[T]), acc[0][rt][T][1]);
+              acc[0][rt][T][2] = fmaf(s1, fmaf(c4[2], 16777216.0f, -xg0[T]), acc[0][rt][T][2]);
+              acc[0][rt][T][3] = fmaf(s1, fmaf(c4[3], 16777216.0f, -xg1[T]), acc[0][rt][T][3]);
             }
           }
         }
       }
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&wempty[ws]);
-        mbar_arrive(&xempty[xslot]);
-      }
+      if (lane == 0) mbar_arrive(&empty[slot]);
     }
-    // push this slice's partial results to the CTA that owns each row (the rows of the row block
-    // are split evenly over the cluster: owner q holds rows [q*128/S, (q+1)*128/S))
-    const uint32_t red_local = smem_u32(red);
+    // push this slice's partial results to the CTA that owns each row (owner q holds rows
+    // [q*R/S, (q+1)*R/S) of the R real rows); the virtual row goes to every owner
+    const uint32_t red_local = smem_u32(red), sxr_local = smem_u32(sxr);
 #pragma unroll
     for (int rt = 0; rt < kDRT; ++rt)
 #pragma unroll
       for (int hr = 0; hr < 2; ++hr) {
-        const int r = warp * (16 * kDRT) + rt * 16 + g + 8 * hr;
-        const int q = (r * a.S + a.S - 1) / kDRows;
-        const int slot = r - (q * kDRows) / a.S;
-        const uint32_t dst = mapa_shared(red_local + ((rank * own_cap + slot) * 16) * 4, static_cast<uint32_t>(q));
+        const int r = rw + 16 * rt + 8 * hr;
+        const bool vrow = virt && rt == kDRT - 1 && hr == 1;
+        const int q = ((r + 1) * a.S - 1) / F::kRows;
+        const int slot = r - (q * F::kRows) / a.S;
 #pragma unroll
         for (int T = 0; T < NT; ++T)
 #pragma unroll
@@ -416,40 +449,35 @@ __global__ void __launch_bounds__(kDThreads, 2)
             float v;
             // factors 2^-24 (pairs 0 and 3), 2^-20 (pair 1), 2^-16 (pair 2): exact rescaling
             if (!kInt4)
-              v = fmaf(acc[0][rt][T][ci] + acc[NG - 1][rt][T][ci], 16777216.0f,
+              v = fmaf(acc[0][rt][T][ci], 16777216.0f,
                        fmaf(acc[1 % NG][rt][T][ci], 1048576.0f, acc[2 % NG][rt][T][ci] * 65536.0f));
             else
               v = acc[0][rt][T][ci];
-            st_shared_cluster_f32(dst + (8 * T + 2 * t + c) * 4, v);
+            const int tok = 8 * T + 2 * t + c;
+            if (vrow) {
+              for (int o = 0; o < a.S; ++o)
+                st_shared_cluster_f32(mapa_shared(sxr_local + (rank * 16 + tok) * 4, static_cast<uint32_t>(o)), v);
+            } else if (r < F::kRows) {
+              st_shared_cluster_f32(
+                  mapa_shared(red_local + ((rank * own_cap + slot) * 16 + tok) * 4, static_cast<uint32_t>(q)), v);
+            }
           }
       }
   }
 
   // ==================================================================== cluster reduction
-  __syncthreads();  // the builders' sums of x are in shared memory
-  if (!kInt4 && threadIdx.x < 16) {  // push this slice's token sums of x to every owner
-    const float sx = sxb[threadIdx.x] + sxb[16 + threadIdx.x];
-    const uint32_t loc = smem_u32(sxr + rank * 16 + threadIdx.x);
-    for (int q = 0; q < a.S; ++q) st_shared_cluster_f32(mapa_shared(loc, q), sx);
-  }
   cluster_sync_all();  // every partial and slice sum has landed in its owner's shared memory
   pdl_wait_prior_grids();
-  {
-    const int rr0 = (rank * kDRows) / a.S, rr1 = ((rank + 1) * kDRows) / a.S;
-    const int nrows = rr1 - rr0;
-    const int Mv = static_cast<int>(a.M < 8 * NT ? a.M : 8 * NT);
-    for (int idx = threadIdx.x; idx < nrows * Mv; idx += kDThreads) {
-      const int m = idx / nrows, slot = idx - m * nrows;
-      const int64_t n = static_cast<int64_t>(rb) * kDRows + rr0 + slot;
-      if (n >= Nm) continue;
+  if (ep_on) {
+    const int Mv = Mi < 8 * NT ? Mi : 8 * NT;
+    for (int mm = 0; mm < Mv; ++mm) {
       float v = 0.0f, sx = 0.0f;
       for (int q = 0; q < a.S; ++q) {  // fixed order: deterministic
-        v += red[(q * own_cap + slot) * 16 + m];
-        if (!kInt4) sx += sxr[q * 16 + m];
+        v += red[(q * own_cap + ep_row) * 16 + mm];
+        if (!kInt4) sx += sxr[q * 16 + mm];
       }
-      if (!kInt4) v = (v - sx) * __half2float(scm[n]);
-      if (biasm) v += __half2float(biasm[n]);
-      ym[m * Nm + n] = __float2half_rn(v);
+      if (!kInt4) v = (v - sx) * ep_s;
+      ym[mm * Nm + ep_n] = __float2half_rn(v + ep_b);
     }
   }
 }
@@ -458,38 +486,41 @@ __global__ void __launch_bounds__(kDThreads, 2)
 // host side
 // ---------------------------------------------------------------------------------------------
 struct DecodePlan {
-  int S, C, ring, smem;
+  int S, C, ring, stage, smem;
 };
 
-template <bool kInt4, int NT>
-static bool plan_decode_t(int64_t RB, int64_t K, int num_sms, DecodePlan* p) {
+// Stage ring and cluster size for RB row blocks of one launch.
+template <bool kInt4>
+static bool plan_decode_t(int64_t RB, int64_t M, int64_t K, int num_sms, DecodePlan* p) {
   using F = DecFmt<kInt4>;
+  using L = DecLayout<kInt4>;
   const int C = static_cast<int>((K + F::kStageK - 1) / F::kStageK);
-  // weight ring: every stage of the CTA's slice if it fits (then the whole slice is in flight
-  // before griddepcontrol.wait), else as many as two CTAs per SM allow
+  const int xbytes = F::kKB * (M > 8 ? 2 : 1) * 1024;  // one 8- or 16-row slot per block
+  const int stage = kDWBytes + xbytes;
+  // as many stages as two CTAs per SM allow (a CTA's whole slice when it fits, so that all its
+  // weights are in flight before griddepcontrol.wait)
   int ring = kDMaxRing;
-  while (ring > 2 && DecLayout<kInt4, NT>::bytes(ring) > kDSmemBudget) --ring;
-  const int smem = DecLayout<kInt4, NT>::bytes(ring);
-  if (smem > 227 * 1024) return false;
+  while (ring > 2 && L::bytes(ring, stage) > kDSmemBudget) --ring;
+  const int smem = L::bytes(ring, stage);
+  if (smem > kDSmemBudget) return false;
   // one wave of two CTAs per SM, at most 8 K-slices per row block
   int64_t S = (2 * static_cast<int64_t>(num_sms)) / RB;
   if (S < 1) S = 1;
   if (S > kDMaxCluster) S = kDMaxCluster;
   if (S > C) S = C;
-  *p = DecodePlan{static_cast<int>(S), C, ring, smem};
+  *p = DecodePlan{static_cast<int>(S), C, ring, stage, smem};
   return true;
 }
 
-static bool plan_decode(bool int4, int NT, int64_t RB, int64_t K, int num_sms, DecodePlan* p) {
-  if (int4) return NT == 1 ? plan_decode_t<true, 1>(RB, K, num_sms, p) : plan_decode_t<true, 2>(RB, K, num_sms, p);
-  return NT == 1 ? plan_decode_t<false, 1>(RB, K, num_sms, p) : plan_decode_t<false, 2>(RB, K, num_sms, p);
+static bool plan_decode(bool int4, int64_t RB, int64_t M, int64_t K, int num_sms, DecodePlan* p) {
+  return int4 ? plan_decode_t<true>(RB, M, K, num_sms, p) : plan_decode_t<false>(RB, M, K, num_sms, p);
 }
 
 template <bool kInt4, int NT>
 static cudaError_t launch_decode_t(const DecodeMaps& maps, const DecodeArgs& a, const DecodePlan& p,
                                    cudaStream_t s) {
   auto* kern = decode_gemm_kernel<kInt4, NT>;
-  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), p.smem);
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), kDSmemBudget);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(p.S), static_cast<unsigned>(a.rb_start[a.count]), 1);
@@ -519,12 +550,12 @@ static cudaError_t launch_decode_group(const __half* x, int count, const void* c
                                        const __half* const* sc, const __half* const* bias,
                                        __half* const* y, const int64_t* N, int64_t M, int64_t K,
                                        cudaStream_t s) {
+  using F = DecFmt<kInt4>;
   if (count < 1 || count > kDMaxGroup) return cudaErrorInvalidValue;
   const DeviceInfo di = current_device_info();
   const int NT = M > 8 ? 2 : 1;
   DecodeArgs a = {};
   DecodeMaps maps;
-  a.x = x;
   a.M = M;
   a.K = K;
   a.count = count;
@@ -532,24 +563,30 @@ static cudaError_t launch_decode_group(const __half* x, int count, const void* c
   const int64_t kbytes = kInt4 ? K / 2 : K / 4;
   for (int g = 0; g < count; ++g) {
     a.rb_start[g] = static_cast<int>(rbs);
-    rbs += (N[g] + kDRows - 1) / kDRows;
+    rbs += (N[g] + F::kRows - 1) / F::kRows;
     a.N[g] = N[g];
     a.sc[g] = sc[g];
     a.bias[g] = bias ? bias[g] : nullptr;
     a.y[g] = y[g];
     if (!make_tmap_2d(&maps.m[g], CU_TENSOR_MAP_DATA_TYPE_UINT8, w[g], static_cast<uint64_t>(kbytes),
-                      static_cast<uint64_t>(N[g]), static_cast<uint64_t>(kbytes), 128, kDRows,
+                      static_cast<uint64_t>(N[g]), static_cast<uint64_t>(kbytes), 128, kDTile,
                       CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   }
   for (int g = count; g < kDMaxGroup; ++g) maps.m[g] = maps.m[0];
+  // activations: one box = 64 elements (128 bytes) x all M tokens
+  if (!make_tmap_2d(&maps.x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, static_cast<uint64_t>(K),
+                    static_cast<uint64_t>(M), static_cast<uint64_t>(K) * 2, 64,
+                    static_cast<uint32_t>(M), CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
   a.rb_start[count] = static_cast<int>(rbs);
   if (rbs > 65535) return cudaErrorInvalidValue;
   DecodePlan p;
-  if (!plan_decode(kInt4, NT, rbs, K, di.num_sms, &p)) return cudaErrorInvalidValue;
+  if (!plan_decode(kInt4, rbs, M, K, di.num_sms, &p)) return cudaErrorInvalidValue;
   a.C = p.C;
   a.S = p.S;
   a.ring = p.ring;
+  a.stage = p.stage;
   return NT == 1 ? launch_decode_t<kInt4, 1>(maps, a, p, s) : launch_decode_t<kInt4, 2>(maps, a, p, s);
 }
 
@@ -557,7 +594,8 @@ bool decode_supported(bool int4, int64_t M, int64_t N, int64_t K) {
   if (M < 1 || M > 16 || N < 1) return false;
   if (int4 ? (K % 128 != 0) : (K % 64 != 0)) return false;
   DecodePlan p;
-  return plan_decode(int4, M > 8 ? 2 : 1, (N + kDRows - 1) / kDRows, K, 148, &p);
+  const int64_t rows = int4 ? DecFmt<true>::kRows : DecFmt<false>::kRows;
+  return plan_decode(int4, (N + rows - 1) / rows, M, K, 148, &p);
 }
 
 cudaError_t launch_tq_gemm_decode(const __half* x, const uint8_t* packed, const __half* scale,

@@ -1,7 +1,7 @@
 // tq_pack.cu -- quantise-and-pack kernels.
 //
 // Ternary ([TQ] §1 ternarisation, §3.1 threshold 0.7*mean|w|, code table and byte layout, §3.2
-// ceil(K/4) row stride): one CTA per row.  The row sums that decide the threshold and the
+// ceil(K/4) row stride): one warp per row.  The row sums that decide the threshold and the
 // scale are computed EXACTLY (then rounded once to fp64), so the codes and the scale do not
 // depend on the order in which the GPU adds:
 //   * fp16 input: |w| * 2^24 is an integer below 2^40, so an int64 accumulator is exact for
@@ -9,8 +9,10 @@
 //   * fp32 input: |w| is binned by its exponent relative to the row's largest exponent; inside
 //     a bin of `binw` binades every value is a multiple of the bin's quantum and the bin total
 //     stays below 2^53 quanta (binw = 30 - ceil(log2 K)), so fp64 additions in a bin are exact
-//     in any order.  Bins 0 and 1 live in registers, deeper (rare) bins in shared memory.  The
-//     bins are finally added exactly in fixed point and rounded once.
+//     in any order.  Bins 0 and 1 live in registers, deeper (rare) bins in the warp's slice of
+//     shared memory.  The bins are finally added exactly in fixed point and rounded once.
+// The code decision |w| > t is an integer compare of the magnitude's bit pattern against the
+// pattern of the largest representable value <= t, which equals the fp64 compare exactly.
 // W4A16 ([VQ] §4.2, §5: 4-bit, group 128, symmetric, 8 per int32): one warp per (row, group).
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -21,7 +23,6 @@
 namespace tq {
 
 constexpr int kPackThreads = 256;
-constexpr int kMaxBins = 256;
 
 // Load the 4 elements of byte j of a row (k = 4j .. 4j+3), as raw bit patterns widened to
 // uint32 (fp32 bits, or fp16 bits in the low half).  Elements past K read as 0.
@@ -57,11 +58,6 @@ __device__ __forceinline__ void load4(const void* row, int64_t j, int64_t K, boo
   }
 }
 
-__device__ __forceinline__ double elem_to_f64(uint32_t bits, bool f16) {
-  return f16 ? static_cast<double>(__half2float(__ushort_as_half(static_cast<uint16_t>(bits))))
-             : static_cast<double>(__uint_as_float(bits));
-}
-
 // |w| of an fp16 pattern, as an integer multiple of 2^-24 (exact).
 __device__ __forceinline__ long long f16_abs_units(uint32_t h) {
   const uint32_t e = (h >> 10) & 0x1Fu, f = h & 0x3FFu;
@@ -93,103 +89,124 @@ struct ExactAcc {
   }
 };
 
-// Block-wide exact total of the per-thread accumulators, rounded once to fp64.
-// Every thread must call; every thread gets the result.
+// Warp-wide exact total of per-lane accumulators, rounded once to fp64 (all lanes get it).
+// `wbins` is this warp's shared-memory bin array (fp32 input only).
 template <bool kF16>
-__device__ double exact_total(const ExactAcc<kF16>& acc, double* s_bins, int nbins,
-                              long long* s_red_ll, double* s_red_d, double* s_result) {
+__device__ double warp_exact_total(const ExactAcc<kF16>& acc, double* wbins, int nbins) {
   if (kF16) {
-    const long long tot = block_sum<long long>(acc.i64, s_red_ll);
-    return __ll2double_rn(tot) * 0x1p-24;
+    long long v = acc.i64;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    return __ll2double_rn(v) * 0x1p-24;
   } else {
-    const double t0 = block_sum<double>(acc.b0, s_red_d);
-    const double t1 = block_sum<double>(acc.b1, s_red_d);
-    __syncthreads();  // all deep-bin atomics are done
-    if (threadIdx.x == 0) {
-      s_bins[0] = t0;
-      s_bins[1] = t1;
-      *s_result = exact_sum_fixed149(s_bins, nbins);
+    double b0 = acc.b0, b1 = acc.b1;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {  // exact: every partial sum of one bin is representable
+      b0 += __shfl_xor_sync(0xFFFFFFFFu, b0, o);
+      b1 += __shfl_xor_sync(0xFFFFFFFFu, b1, o);
     }
-    __syncthreads();
-    return *s_result;
+    __syncwarp();  // deep-bin atomics of all lanes are done
+    double r = 0.0;
+    if ((threadIdx.x & 31) == 0) {
+      wbins[0] = b0;
+      wbins[1] = b1;
+      r = exact_sum_fixed149(wbins, nbins);
+    }
+    return __shfl_sync(0xFFFFFFFFu, r, 0);
   }
 }
 
+// Largest magnitude bit pattern whose value is <= t (t >= 0).  Positive IEEE patterns are
+// ordered like their values, so for any element |w| > t  <=>  (bits(w) & ~sign) > this.
+template <bool kF16>
+__device__ __forceinline__ uint32_t magnitude_floor_bits(double t) {
+  if (kF16) {
+    const uint16_t h = f64_to_f16_rne(t);  // nearest; step down if it rounded up
+    const uint32_t m = h & 0x7FFFu;
+    if (m != 0u && f16_bits_to_f64(static_cast<uint16_t>(m)) > t) return m - 1u;
+    return m >= 0x7C00u ? 0x7BFFu : m;
+  } else {
+    const float f = __double2float_rd(t);  // round toward -inf: largest float <= t
+    const uint32_t m = __float_as_uint(f) & 0x7FFFFFFFu;
+    return m >= 0x7F800000u ? 0x7F7FFFFFu : m;
+  }
+}
+
+// One warp per row.  Pass 1 (fp32 only): largest exponent.  Pass 2: exact sum of |w| -> t.
+// Pass 3: codes (an integer compare against the threshold pattern), packed bytes, exact sum of
+// the nonzero magnitudes and their count -> scale.  Rows are re-read from L2 between passes.
 template <bool kF16>
 __global__ void __launch_bounds__(kPackThreads)
     tq_pack_kernel(const void* __restrict__ w, uint8_t* __restrict__ packed,
                    uint16_t* __restrict__ scale, int64_t N, int64_t K, int binw, int vec) {
-  __shared__ double s_bins[kMaxBins];
-  __shared__ long long s_red_ll[32];
-  __shared__ double s_red_d[32];
-  __shared__ int s_red_i[32];
-  __shared__ double s_result;
-
+  constexpr int kWarps = kPackThreads / 32;
+  constexpr int kWarpBins = 130;  // fp32 bins per warp: 254 / binw + 2 with binw >= 2 (K <= 2^28)
+  __shared__ double s_bins[kF16 ? 1 : kWarps * kWarpBins];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  double* wbins = kF16 ? s_bins : s_bins + wid * kWarpBins;
   const int64_t KB = (K + 3) >> 2;
-  const int nbins = kF16 ? 0 : min(kMaxBins, 254 / binw + 2);
+  const int nbins = kF16 ? 0 : min(kWarpBins, 254 / binw + 2);
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
 
-  for (int64_t n = blockIdx.x; n < N; n += gridDim.x) {
+  for (int64_t n = static_cast<int64_t>(blockIdx.x) * kWarps + wid; n < N; n += nwarps) {
     const void* row = kF16 ? static_cast<const void*>(static_cast<const uint16_t*>(w) + n * K)
                            : static_cast<const void*>(static_cast<const float*>(w) + n * K);
-    // ---- pass 1 (fp32 only): largest biased exponent of the row
     int emax = 1;
     if (!kF16) {
       int m = 1;
-      for (int64_t j = threadIdx.x; j < KB; j += blockDim.x) {
+      for (int64_t j = lane; j < KB; j += 32) {
         uint32_t v[4];
         load4<kF16>(row, j, K, vec, v);
 #pragma unroll
         for (int i = 0; i < 4; ++i) m = max(m, static_cast<int>((v[i] & 0x7FFFFFFFu) >> 23));
       }
-      emax = block_max_int(m, s_red_i);
-      for (int i = threadIdx.x; i < nbins; i += blockDim.x) s_bins[i] = 0.0;
-      __syncthreads();
+      emax = warp_max_int(m);
+      __syncwarp();  // lane 0 is done with the previous row's bins
+      for (int i = lane; i < nbins; i += 32) wbins[i] = 0.0;
+      __syncwarp();
     }
-    // ---- pass 2: S = exact sum |w|;  t = 0.7 * (S / K)
     ExactAcc<kF16> accS;
 #pragma unroll 4
-    for (int64_t j = threadIdx.x; j < KB; j += blockDim.x) {
+    for (int64_t j = lane; j < KB; j += 32) {
       uint32_t v[4];
       load4<kF16>(row, j, K, vec, v);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) accS.add(v[i], emax, binw, s_bins);
+      for (int i = 0; i < 4; ++i) accS.add(v[i], emax, binw, wbins);
     }
-    const double S = exact_total<kF16>(accS, s_bins, nbins, s_red_ll, s_red_d, &s_result);
+    const double S = warp_exact_total<kF16>(accS, wbins, nbins);
     const double t = 0.7 * (S / static_cast<double>(K));
+    const uint32_t tb = magnitude_floor_bits<kF16>(t);
+    const uint32_t magmask = kF16 ? 0x7FFFu : 0x7FFFFFFFu;
+    const uint32_t signbit = kF16 ? 0x8000u : 0x80000000u;
     if (!kF16) {
-      for (int i = threadIdx.x; i < nbins; i += blockDim.x) s_bins[i] = 0.0;
-      __syncthreads();
+      __syncwarp();
+      for (int i = lane; i < nbins; i += 32) wbins[i] = 0.0;
+      __syncwarp();
     }
-    // ---- pass 3: codes, packed bytes, A = exact sum |w| over nonzero codes, nz
     ExactAcc<kF16> accA;
     int nz = 0;
     uint8_t* prow = packed + n * KB;
-#pragma unroll 2
-    for (int64_t j = threadIdx.x; j < KB; j += blockDim.x) {
+#pragma unroll 4
+    for (int64_t j = lane; j < KB; j += 32) {
       uint32_t v[4];
       load4<kF16>(row, j, K, vec, v);
       uint32_t byte = 0;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         uint32_t code = 1u;  // padding past K is the zero code 0b01
-        if (4 * j + i < K) {
-          const double wd = elem_to_f64(v[i], kF16);
-          code = (wd < -t) ? 0u : ((wd > t) ? 2u : 1u);
-          if (code != 1u) {
-            accA.add(v[i], emax, binw, s_bins);
-            ++nz;
-          }
+        if (4 * j + i < K && (v[i] & magmask) > tb) {  // |w| > t
+          code = (v[i] & signbit) ? 0u : 2u;
+          accA.add(v[i], emax, binw, wbins);
+          ++nz;
         }
         byte |= code << (2 * i);
       }
       prow[j] = static_cast<uint8_t>(byte);
     }
-    const double A = exact_total<kF16>(accA, s_bins, nbins, s_red_ll, s_red_d, &s_result);
-    const int nzt = block_sum<int>(nz, s_red_i);
-    if (threadIdx.x == 0) {
+    const double A = warp_exact_total<kF16>(accA, wbins, nbins);
+    const int nzt = warp_sum(nz);
+    if (lane == 0)
       scale[n] = nzt > 0 ? f64_to_f16_rne(A / static_cast<double>(nzt)) : static_cast<uint16_t>(0);
-    }
-    __syncthreads();  // shared scratch is reused by the next row
   }
 }
 
@@ -249,7 +266,9 @@ static int ceil_log2_i64(int64_t v) {
 cudaError_t launch_tq_pack(const void* w, bool w_f16, uint8_t* packed, uint16_t* scale, int64_t N,
                            int64_t K, cudaStream_t s) {
   const DeviceInfo di = current_device_info();
-  const int64_t grid = N < int64_t(di.num_sms) * 8 ? N : int64_t(di.num_sms) * 8;
+  const int64_t rows_per_cta = kPackThreads / 32;
+  int64_t grid = (N + rows_per_cta - 1) / rows_per_cta;
+  if (grid > int64_t(di.num_sms) * 8) grid = int64_t(di.num_sms) * 8;
   const int binw = 30 - ceil_log2_i64(K);
   const uintptr_t a = reinterpret_cast<uintptr_t>(w);
   const int vec = (K % 4 == 0) && (a % (w_f16 ? 8 : 16) == 0);

@@ -117,7 +117,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
   using L = PrefillLayout<kInt4>;
   using F = PFmt<kInt4>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned; pointer arithmetic on the __shared__ array keeps the shared address
+  // space visible to the compiler (plain ld/st.shared instead of generic accesses)
+  uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kOffBar);
   uint64_t* fullL = bars;
   uint64_t* emptyA = bars + kPRingL;

@@ -113,3 +113,34 @@ def test_w4g_pack_edge_groups():
     w[2, :6] = torch.tensor([7 * s0, 2.5 * s0, 3.5 * s0, -2.5 * s0, 0.5 * s0, -0.5 * s0])  # ties
     w[3] = torch.randn(256, generator=torch.Generator().manual_seed(3)) * 1e4
     _check_w4g(w)
+
+
+def _near_threshold_row(K, seed, np_dtype):
+    """A row whose elements include the representable values just below, at and just above its
+    own threshold 0.7*mean|w| (iterated until the threshold no longer moves), both signs."""
+    rng = np.random.default_rng(seed)
+    w = (rng.standard_normal(K) * 0.02).astype(np_dtype)
+    for _ in range(6):
+        t = O.ternary_threshold(w.astype(np.float64))
+        c = np.asarray(t, dtype=np_dtype)
+        lo = np.nextafter(c, np_dtype(0))
+        hi = np.nextafter(c, np_dtype(np.inf))
+        near = np.array([lo, c, hi, -lo, -c, -hi], dtype=np_dtype)
+        w[: 6 * 16] = np.tile(near, 16)
+    return w
+
+
+def test_pack_threshold_boundary():
+    for np_dtype, tdt in ((np.float32, torch.float32), (np.float16, torch.float16)):
+        rows = [_near_threshold_row(K, 100 + K, np_dtype) for K in (512, 4096, 4099)]
+        for r in rows:
+            _check_tq(torch.from_numpy(r[None, :].copy()).to(tdt))
+
+
+def test_pack_fp32_deep_bins_long_row():
+    # K = 2^20 -> narrow exponent bins; a wide exponent spread lands values in many bins.
+    g = torch.Generator().manual_seed(12)
+    K = 1 << 20
+    e = torch.randint(-120, 60, (3, K), generator=g).float()
+    w = torch.randn(3, K, generator=g) * torch.exp2(e)
+    _check_tq(w)
