@@ -9,16 +9,18 @@
 // reduces through distributed shared memory in a fixed order (deterministic, no global scratch).
 // A stage is 128 bytes of every packed row (512 ternary or 256 INT4 codes) plus the activations
 // of those k for all M tokens.  Per CTA:
-//   * warp 4 (producer) streams each stage with TMA into a ring: the 128-row x 128-byte packed
+//   * warp 8 (producer) streams each stage with TMA into a ring: the 128-row x 128-byte packed
 //     tile (issued before griddepcontrol.wait, weights never depend on the previous kernel) and
 //     the activations, one 64-element block x M tokens per box (issued after it), both
 //     128-byte swizzled so that every 16-byte read below is bank-conflict free.  For W4A16 it
 //     also sums each 128-wide group of x per token;
-//   * warps 0-3 (consumers) each own 32 rows = two 16-row MMA tiles.  Weights are the A operand
-//     of mma.sync.m16n8k16 ("swap AB"), the tokens the N = 8 operand: one MMA per 256 weights
-//     for M <= 8, two for M <= 16.  Each lane builds its B fragments from the activations in
-//     shared memory (byte permutes into the k order the decode produces, see below); with two
-//     row tiles per warp one fragment feeds four MMAs.
+//   * warps 0-7 (consumers): warp w owns rows 32 (w & 3) .. +31 (two 16-row MMA tiles) and,
+//     for M > 8, the token group w >> 2 over the whole stage, for M <= 8 the K half w >> 2 of
+//     every stage (the two halves are added in shared memory, in a fixed order, at the end).
+//     Weights are the A operand of mma.sync.m16n8k16 ("swap AB"), the tokens the N = 8
+//     operand: one MMA per 256 weights and token group.  Each lane builds its B fragments from
+//     the activations in shared memory (byte permutes into the k order the decode produces, see
+//     below); with two row tiles per warp one fragment feeds four MMAs.
 //
 // In-register decode ("subnormal" trick).  ANDing a packed 32-bit word with 0x00030003 << 2p
 // leaves, in each fp16 half, the code at bits 2p..2p+1: the exact value c * 2^(2p-24) (fp16
@@ -42,14 +44,15 @@
 namespace tq {
 
 constexpr int kDTile = 128;                 // rows of one packed TMA tile
-constexpr int kDConsumers = 4;              // consumer warps (32 rows = two MMA tiles each)
+constexpr int kDConsumers = 8;              // consumer warps: 4 row sets x 2 (token groups or K halves)
+constexpr int kDRowSets = 4;                // 32 rows = two 16-row MMA tiles per consumer warp
 constexpr int kDRT = 2;                     // 16-row MMA tiles per consumer warp
 constexpr int kDProducer = kDConsumers;     // TMA warp
 constexpr int kDThreads = (kDConsumers + 1) * 32;
 constexpr int kDWBytes = kDTile * 128;      // weights of one stage: 128 rows x 128 bytes
 constexpr int kDMaxRing = 8;                // stages resident in shared memory
 constexpr int kDMaxCluster = 8;
-constexpr int kDRedRows = kDTile + kDMaxCluster;  // >= S * ceil(rows / S)
+constexpr int kDRedRows = kDTile + kDMaxCluster;  // >= S * ceil(rows / S): red holds [S][16][ceil(rows / S)]
 constexpr int kDSmemBudget = 113 * 1024;    // two CTAs per SM
 
 template <bool kInt4>
@@ -85,7 +88,8 @@ struct DecLayout {
   static constexpr int kXg = kInt4 ? 2 * 16 * 4 : 0;  // W4A16 group sums of a stage [2][16]
   static constexpr int kRed = kDRedRows * 16 * 4;
   static constexpr int kSxr = kDMaxCluster * 16 * 4;
-  __host__ __device__ static constexpr int fixed() { return 1024 + kRed + kSxr + 3 * kDMaxRing * 8; }
+  static constexpr int kPart = kDTile * 8 * 4;        // second K half's partials (M <= 8)
+  __host__ __device__ static constexpr int fixed() { return 1024 + kRed + kSxr + kPart + 3 * kDMaxRing * 8; }
   __host__ __device__ static constexpr int bytes(int ring, int stage) { return fixed() + ring * (stage + kXg); }
 };
 
@@ -109,9 +113,10 @@ __device__ __forceinline__ void make_frag(uint32_t Pa, uint32_t Pb, uint32_t Pc,
   o1 = *reinterpret_cast<uint32_t*>(&s23);
 }
 
-// Two CTAs of five warps per SM (the launch bound keeps the registers within that).
+// Two CTAs of nine warps per SM: five warps share one SM sub-partition's 16K registers, so a
+// thread may use at most 102; 96 it is.
 template <bool kInt4, int NT>
-__global__ void __launch_bounds__(kDThreads, 2)
+__global__ void __maxnreg__(96)
     decode_gemm_kernel(const __grid_constant__ DecodeMaps maps, const __grid_constant__ DecodeArgs a) {
   using F = DecFmt<kInt4>;
   using L = DecLayout<kInt4>;
@@ -122,9 +127,10 @@ __global__ void __launch_bounds__(kDThreads, 2)
   uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* stg = base;                                                  // ring x [weights | x]
   float* xg = reinterpret_cast<float*>(stg + a.ring * a.stage);         // ring x [2][16]
-  float* red = xg + a.ring * (L::kXg / 4);                              // [S][rows/S][16]
+  float* red = xg + a.ring * (L::kXg / 4);                              // [S][16][own_cap]
   float* sxr = red + kDRedRows * 16;                                    // [S][16] slice sums of x
-  uint64_t* full = reinterpret_cast<uint64_t*>(sxr + kDMaxCluster * 16);
+  float* part = sxr + kDMaxCluster * 16;                                // [128 rows][8 tokens]
+  uint64_t* full = reinterpret_cast<uint64_t*>(part + kDTile * 8);
   uint64_t* xready = full + kDMaxRing;  // W4A16 group sums of the stage written
   uint64_t* empty = xready + kDMaxRing;
 
@@ -254,20 +260,20 @@ __global__ void __launch_bounds__(kDThreads, 2)
     // ================================================================== consumer warps
     // accumulator groups by exact power-of-two factor: pairs 0 and 3 (2^-24), 1 (2^-20), 2 (2^-16)
     constexpr int NG = kInt4 ? 1 : 3;
-    float acc[NG][kDRT][NT][4];
+    const int rs = warp & (kDRowSets - 1), hi = warp / kDRowSets;
+    const int T0 = NT == 2 ? hi : 0;                  // token group of this warp
+    const int sub_lo = NT == 2 ? 0 : hi, sub_hi = NT == 2 ? 2 : hi + 1;  // its K halves
+    const int m = 8 * T0 + g;                         // this lane's token (B column)
+    const bool tokv = m < Mi;
+    float acc[NG][kDRT][4];
 #pragma unroll
     for (int q = 0; q < NG; ++q)
 #pragma unroll
       for (int rt = 0; rt < kDRT; ++rt)
 #pragma unroll
-        for (int T = 0; T < NT; ++T)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) acc[q][rt][T][c] = 0.0f;
-    bool tokv[NT];
-#pragma unroll
-    for (int T = 0; T < NT; ++T) tokv[T] = 8 * T + g < Mi;
+        for (int c = 0; c < 4; ++c) acc[q][rt][c] = 0.0f;
     const __half2 fold = kInt4 ? __floats2half2_rn(0.0625f, 0.0625f) : __floats2half2_rn(0.25f, 0.25f);
-    const int rw = warp * 16 * kDRT + g;  // row of tile 0, lower half; tile rt adds 16 rt, upper +8
+    const int rw = rs * 16 * kDRT + g;  // row of tile 0, lower half; tile rt adds 16 rt, upper +8
     // ternary: tile row 127 is the virtual all-01 row (its result is sum_k x)
     const bool virt = !kInt4 && rw + 16 * (kDRT - 1) + 8 == kDTile - 1;
     const int64_t G = a.K >> 7;
@@ -279,7 +285,7 @@ __global__ void __launch_bounds__(kDThreads, 2)
       const uint8_t* st = stg + slot * a.stage;
       const uint8_t* xs = st + kDWBytes;
 #pragma unroll 1
-      for (int sub = 0; sub < 2; ++sub) {
+      for (int sub = sub_lo; sub < sub_hi; ++sub) {
         const int chunk = sub * 4 + t;  // this lane's 16 bytes of the packed rows
         // rows rw + 16 rt + 8 hr all have (row & 7) == g: swizzled chunk position chunk ^ g
         uint32_t w[kDRT][2][4];
@@ -299,19 +305,17 @@ __global__ void __launch_bounds__(kDThreads, 2)
           const uint8_t* blk = xs + chunk * kXSlot;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            // P[T][j] = x[8T+g][64*chunk + 32h + 2j .. +1]
-            uint32_t P[NT][16];
+            // P[j] = x[m][64*chunk + 32h + 2j .. +1]
+            uint32_t P[16];
 #pragma unroll
-            for (int T = 0; T < NT; ++T)
-#pragma unroll
-              for (int jj = 0; jj < 4; ++jj) {
-                uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                if (tokv[T]) v = ld_x_chunk(blk, 8 * T + g, 4 * h + jj);
-                P[T][4 * jj] = v.x;
-                P[T][4 * jj + 1] = v.y;
-                P[T][4 * jj + 2] = v.z;
-                P[T][4 * jj + 3] = v.w;
-              }
+            for (int jj = 0; jj < 4; ++jj) {
+              uint4 v = make_uint4(0u, 0u, 0u, 0u);
+              if (tokv) v = ld_x_chunk(blk, m, 4 * h + jj);
+              P[4 * jj] = v.x;
+              P[4 * jj + 1] = v.y;
+              P[4 * jj + 2] = v.z;
+              P[4 * jj + 3] = v.w;
+            }
             uint32_t sh[kDRT][4];
 #pragma unroll
             for (int rt = 0; rt < kDRT; ++rt) {
@@ -322,10 +326,8 @@ __global__ void __launch_bounds__(kDThreads, 2)
             }
 #pragma unroll
             for (int pp = 0; pp < 4; ++pp) {
-              uint32_t be0[NT], be1[NT], bo0[NT], bo1[NT];
-#pragma unroll
-              for (int T = 0; T < NT; ++T)
-                make_frag(P[T][pp], P[T][4 + pp], P[T][8 + pp], P[T][12 + pp], fold, be0[T], be1[T], bo0[T], bo1[T]);
+              uint32_t be0, be1, bo0, bo1;
+              make_frag(P[pp], P[4 + pp], P[8 + pp], P[12 + pp], fold, be0, be1, bo0, bo1);
 #pragma unroll
               for (int q = 0; q < 2; ++q) {
                 const int p = 2 * pp + q;
@@ -345,9 +347,7 @@ __global__ void __launch_bounds__(kDThreads, 2)
                     a2 = sh[rt][2] & mk;
                     a3 = sh[rt][3] & mk;
                   }
-#pragma unroll
-                  for (int T = 0; T < NT; ++T)
-                    mma_16816(acc[pp == 3 ? 0 : pp][rt][T], a0, a1, a2, a3, q ? bo0[T] : be0[T], q ? bo1[T] : be1[T]);
+                  mma_16816(acc[pp == 3 ? 0 : pp][rt], a0, a1, a2, a3, q ? bo0 : be0, q ? bo1 : be1);
                 }
               }
             }
@@ -356,113 +356,112 @@ __global__ void __launch_bounds__(kDThreads, 2)
           // the 32 codes of the chunk are k = 32*chunk + 0..31: half (chunk & 1) of activation
           // block chunk / 2, its 16-byte chunks 4*(chunk & 1) + 0..3
           const uint8_t* blk = xs + (chunk >> 1) * kXSlot;
-          uint32_t P[NT][16];
+          uint32_t P[16];
 #pragma unroll
-          for (int T = 0; T < NT; ++T)
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-              uint4 v = make_uint4(0u, 0u, 0u, 0u);
-              if (tokv[T]) v = ld_x_chunk(blk, 8 * T + g, 4 * (chunk & 1) + jj);
-              P[T][4 * jj] = v.x;
-              P[T][4 * jj + 1] = v.y;
-              P[T][4 * jj + 2] = v.z;
-              P[T][4 * jj + 3] = v.w;
-            }
-          float cg[2][kDRT][NT][4];  // two chains (class 0 / class 1 fields)
+          for (int jj = 0; jj < 4; ++jj) {
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (tokv) v = ld_x_chunk(blk, m, 4 * (chunk & 1) + jj);
+            P[4 * jj] = v.x;
+            P[4 * jj + 1] = v.y;
+            P[4 * jj + 2] = v.z;
+            P[4 * jj + 3] = v.w;
+          }
+          float cg[2][kDRT][4];  // two chains (class 0 / class 1 fields)
 #pragma unroll
           for (int j = 0; j < 2; ++j)
 #pragma unroll
             for (int rt = 0; rt < kDRT; ++rt)
 #pragma unroll
-              for (int T = 0; T < NT; ++T)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) cg[j][rt][T][c] = 0.0f;
+              for (int c = 0; c < 4; ++c) cg[j][rt][c] = 0.0f;
 #pragma unroll
           for (int h = 0; h < 2; ++h)
 #pragma unroll
             for (int s2 = 0; s2 < 2; ++s2) {
-              uint32_t be0[NT], be1[NT], bo0[NT], bo1[NT];
-#pragma unroll
-              for (int T = 0; T < NT; ++T)
-                make_frag(P[T][8 * h + s2], P[T][8 * h + 2 + s2], P[T][8 * h + 4 + s2], P[T][8 * h + 6 + s2], fold,
-                          be0[T], be1[T], bo0[T], bo1[T]);
+              uint32_t be0, be1, bo0, bo1;
+              make_frag(P[8 * h + s2], P[8 * h + 2 + s2], P[8 * h + 4 + s2], P[8 * h + 6 + s2], fold, be0, be1, bo0, bo1);
 #pragma unroll
               for (int rt = 0; rt < kDRT; ++rt) {
                 const uint32_t x0 = w[rt][0][2 * h] >> (8 * s2), x1 = w[rt][1][2 * h] >> (8 * s2);
                 const uint32_t x2 = w[rt][0][2 * h + 1] >> (8 * s2), x3 = w[rt][1][2 * h + 1] >> (8 * s2);
-#pragma unroll
-                for (int cls = 0; cls < 2; ++cls) {
-                  const uint32_t mk = cls ? 0x00F000F0u : 0x000F000Fu;
-#pragma unroll
-                  for (int T = 0; T < NT; ++T)
-                    mma_16816(cg[cls][rt][T], x0 & mk, x1 & mk, x2 & mk, x3 & mk, cls ? bo0[T] : be0[T],
-                              cls ? bo1[T] : be1[T]);
-                }
+                mma_16816(cg[0][rt], x0 & 0x000F000Fu, x1 & 0x000F000Fu, x2 & 0x000F000Fu, x3 & 0x000F000Fu, be0, be1);
+                mma_16816(cg[1][rt], x0 & 0x00F000F0u, x1 & 0x00F000F0u, x2 & 0x00F000F0u, x3 & 0x00F000F0u, bo0, bo1);
               }
             }
-          if (sub == 0) (void)__all_sync(0xFFFFFFFFu, mbar_wait(&xready[slot], ph));
+          if (sub == sub_lo) (void)__all_sync(0xFFFFFFFFu, mbar_wait(&xready[slot], ph));
           const int64_t gi = static_cast<int64_t>(st_begin + i) * 2 + sub;
-          float xg0[NT], xg1[NT];
-#pragma unroll
-          for (int T = 0; T < NT; ++T) {
-            xg0[T] = 8.0f * xg[(slot * 2 + sub) * 16 + 8 * T + 2 * t];
-            xg1[T] = 8.0f * xg[(slot * 2 + sub) * 16 + 8 * T + 2 * t + 1];
-          }
+          const float xg0 = 8.0f * xg[(slot * 2 + sub) * 16 + 8 * T0 + 2 * t];
+          const float xg1 = 8.0f * xg[(slot * 2 + sub) * 16 + 8 * T0 + 2 * t + 1];
 #pragma unroll
           for (int rt = 0; rt < kDRT; ++rt) {
             const int64_t n0 = row0 + rw + 16 * rt, n1 = n0 + 8;
             // groups past K (a zero-filled half stage) contribute nothing
             const float s0 = (n0 < Nm && gi < G) ? __half2float(scm[n0 * G + gi]) : 0.0f;
             const float s1 = (n1 < Nm && gi < G) ? __half2float(scm[n1 * G + gi]) : 0.0f;
+            float c4[4];
 #pragma unroll
-            for (int T = 0; T < NT; ++T) {
-              float c4[4];
-#pragma unroll
-              for (int c = 0; c < 4; ++c) c4[c] = cg[0][rt][T][c] + cg[1][rt][T][c];
-              acc[0][rt][T][0] = fmaf(s0, fmaf(c4[0], 16777216.0f, -xg0[T]), acc[0][rt][T][0]);
-              acc[0][rt][T][1] = fmaf(s0, fmaf(c4[1], 16777216.0f, -xg1[T]), acc[0][rt][T][1]);
-              acc[0][rt][T][2] = fmaf(s1, fmaf(c4[2], 16777216.0f, -xg0[T]), acc[0][rt][T][2]);
-              acc[0][rt][T][3] = fmaf(s1, fmaf(c4[3], 16777216.0f, -xg1[T]), acc[0][rt][T][3]);
-            }
+            for (int c = 0; c < 4; ++c) c4[c] = cg[0][rt][c] + cg[1][rt][c];
+            acc[0][rt][0] = fmaf(s0, fmaf(c4[0], 16777216.0f, -xg0), acc[0][rt][0]);
+            acc[0][rt][1] = fmaf(s0, fmaf(c4[1], 16777216.0f, -xg1), acc[0][rt][1]);
+            acc[0][rt][2] = fmaf(s1, fmaf(c4[2], 16777216.0f, -xg0), acc[0][rt][2]);
+            acc[0][rt][3] = fmaf(s1, fmaf(c4[3], 16777216.0f, -xg1), acc[0][rt][3]);
           }
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);
     }
-    // push this slice's partial results to the CTA that owns each row (owner q holds rows
-    // [q*R/S, (q+1)*R/S) of the R real rows); the virtual row goes to every owner
-    const uint32_t red_local = smem_u32(red), sxr_local = smem_u32(sxr);
+    // this warp's results: factors 2^-24 (pairs 0 and 3), 2^-20 (pair 1), 2^-16 (pair 2) applied
+    // exactly; rows rw + 16 rt + 8 hr, tokens 8 T0 + 2t + c
+    float v[kDRT][4];
 #pragma unroll
     for (int rt = 0; rt < kDRT; ++rt)
 #pragma unroll
-      for (int hr = 0; hr < 2; ++hr) {
-        const int r = rw + 16 * rt + 8 * hr;
-        const bool vrow = virt && rt == kDRT - 1 && hr == 1;
-        const int q = ((r + 1) * a.S - 1) / F::kRows;
-        const int slot = r - (q * F::kRows) / a.S;
+      for (int ci = 0; ci < 4; ++ci)
+        v[rt][ci] = kInt4 ? acc[0][rt][ci]
+                          : fmaf(acc[0][rt][ci], 16777216.0f,
+                                 fmaf(acc[1 % NG][rt][ci], 1048576.0f, acc[2 % NG][rt][ci] * 65536.0f));
+    if (NT == 1) {  // M <= 8: add the second K half (warps 4-7) to the first, fixed order
+      if (hi == 1) {
 #pragma unroll
-        for (int T = 0; T < NT; ++T)
+        for (int rt = 0; rt < kDRT; ++rt)
+#pragma unroll
+          for (int ci = 0; ci < 4; ++ci)
+            part[(rw + 16 * rt + 8 * (ci >> 1)) * 8 + 2 * t + (ci & 1)] = v[rt][ci];
+      }
+      named_barrier_sync(1, kDConsumers * 32);
+      if (hi == 1) goto consumers_done;
+#pragma unroll
+      for (int rt = 0; rt < kDRT; ++rt)
+#pragma unroll
+        for (int ci = 0; ci < 4; ++ci) v[rt][ci] += part[(rw + 16 * rt + 8 * (ci >> 1)) * 8 + 2 * t + (ci & 1)];
+    }
+    {
+      // push this slice's partial results to the CTA that owns each row (owner q holds rows
+      // [q*R/S, (q+1)*R/S) of the R real rows); the virtual row goes to every owner
+      const uint32_t red_local = smem_u32(red), sxr_local = smem_u32(sxr);
+#pragma unroll
+      for (int rt = 0; rt < kDRT; ++rt)
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+          const int r = rw + 16 * rt + 8 * hr;
+          const bool vrow = virt && rt == kDRT - 1 && hr == 1;
+          const int q = ((r + 1) * a.S - 1) / F::kRows;
+          const int slot = r - (q * F::kRows) / a.S;
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
-            const int ci = 2 * hr + c;
-            float v;
-            // factors 2^-24 (pairs 0 and 3), 2^-20 (pair 1), 2^-16 (pair 2): exact rescaling
-            if (!kInt4)
-              v = fmaf(acc[0][rt][T][ci], 16777216.0f,
-                       fmaf(acc[1 % NG][rt][T][ci], 1048576.0f, acc[2 % NG][rt][T][ci] * 65536.0f));
-            else
-              v = acc[0][rt][T][ci];
-            const int tok = 8 * T + 2 * t + c;
+            const float val = v[rt][2 * hr + c];
+            const int tok = 8 * T0 + 2 * t + c;
             if (vrow) {
               for (int o = 0; o < a.S; ++o)
-                st_shared_cluster_f32(mapa_shared(sxr_local + (rank * 16 + tok) * 4, static_cast<uint32_t>(o)), v);
+                st_shared_cluster_f32(mapa_shared(sxr_local + (rank * 16 + tok) * 4, static_cast<uint32_t>(o)), val);
             } else if (r < F::kRows) {
               st_shared_cluster_f32(
-                  mapa_shared(red_local + ((rank * own_cap + slot) * 16 + tok) * 4, static_cast<uint32_t>(q)), v);
+                  mapa_shared(red_local + ((rank * 16 + tok) * own_cap + slot) * 4, static_cast<uint32_t>(q)), val);
             }
           }
-      }
+        }
+    }
+  consumers_done:;
   }
 
   // ==================================================================== cluster reduction
@@ -473,7 +472,7 @@ __global__ void __launch_bounds__(kDThreads, 2)
     for (int mm = 0; mm < Mv; ++mm) {
       float v = 0.0f, sx = 0.0f;
       for (int q = 0; q < a.S; ++q) {  // fixed order: deterministic
-        v += red[(q * own_cap + ep_row) * 16 + mm];
+        v += red[(q * 16 + mm) * own_cap + ep_row];  // consecutive rows: conflict free
         if (!kInt4) sx += sxr[q * 16 + mm];
       }
       if (!kInt4) v = (v - sx) * ep_s;
