@@ -216,6 +216,10 @@ bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
                   uint64_t rows, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows,
                   CUtensorMapSwizzle swizzle);
 
+// 3-D variant: dims[0] innermost (elements), strides_bytes[i] = stride of dimension i + 1.
+bool make_tmap_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, const uint64_t dims[3],
+                  const uint64_t strides_bytes[2], const uint32_t box[3], CUtensorMapSwizzle swizzle);
+
 // Set the dynamic shared-memory limit of `func` on the current device once.
 cudaError_t ensure_smem_attr(const void* func, int bytes);
 

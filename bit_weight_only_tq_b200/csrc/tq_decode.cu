@@ -70,6 +70,7 @@ struct DecodeArgs {
   int S;          // CTAs per cluster (K-slices)
   int ring;       // stages resident in shared memory
   int stage;      // bytes of one stage (weights + activations, multiple of 1024)
+  int xhalf;      // bytes of one activation box [M][4 blocks][64] (multiple of 1024)
   int count;                        // matrices in the group
   int rb_start[kDMaxGroup + 1];     // first row block of each matrix in grid.y
   int64_t N[kDMaxGroup];
@@ -80,7 +81,8 @@ struct DecodeArgs {
 
 struct DecodeMaps {
   CUtensorMap m[kDMaxGroup];        // packed weights of each matrix
-  CUtensorMap x;                    // activations [M][K] fp16, box 64 x M, 128-byte swizzle
+  CUtensorMap x;                    // activations viewed as [M][K/64][64], box 64 x 4 x M,
+                                    // 128-byte swizzle
 };
 
 template <bool kInt4>
@@ -93,10 +95,14 @@ struct DecLayout {
   __host__ __device__ static constexpr int bytes(int ring, int stage) { return fixed() + ring * (stage + kXg); }
 };
 
-// 16-byte chunk c (0..7) of token row m of one activation block (128-byte swizzle: the chunk
-// index is XORed with the row index within the 1024-byte atom).
-__device__ __forceinline__ uint4 ld_x_chunk(const uint8_t* blk, int m, int c) {
-  return *reinterpret_cast<const uint4*>(blk + m * 128 + ((c ^ (m & 7)) << 4));
+// Activations of a stage: one TMA box per four 64-element blocks (a ternary stage has two, a
+// W4A16 stage one), laid out token-major: 128-byte row 4 m + b for token m, block b.  128-byte
+// swizzle: 16-byte chunk c of row r sits at chunk position c ^ (r & 7).  128-bit shared loads
+// are served eight lanes at a time; the eight lanes g in {2j, 2j+1}, t in 0..3 read rows
+// 4 (8T + g) + t (+ const), whose swizzle phases 4 (g & 1) + t are all different, so every read
+// is bank-conflict free.
+__device__ __forceinline__ uint4 ld_x_chunk(const uint8_t* box, int row, int c) {
+  return *reinterpret_cast<const uint4*>(box + row * 128 + ((c ^ (row & 7)) << 4));
 }
 
 // B fragments of one MMA pair from four activation words: even positions (x) and odd positions
@@ -120,7 +126,6 @@ __global__ void __maxnreg__(96)
     decode_gemm_kernel(const __grid_constant__ DecodeMaps maps, const __grid_constant__ DecodeArgs a) {
   using F = DecFmt<kInt4>;
   using L = DecLayout<kInt4>;
-  constexpr int kXSlot = 8 * NT * 128;  // one activation block: up to 8*NT token rows
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned; pointer arithmetic on the __shared__ array keeps the shared address
   // space visible to the compiler (plain ld/st.shared instead of generic accesses)
@@ -190,8 +195,8 @@ __global__ void __maxnreg__(96)
     auto load_x = [&](int i) {
       uint8_t* dst = stg + (i % a.ring) * a.stage + kDWBytes;
 #pragma unroll
-      for (int b = 0; b < F::kKB; ++b)
-        tma_load_2d(dst + b * kXSlot, &maps.x, &full[i % a.ring], (st_begin + i) * F::kStageK + 64 * b, 0);
+      for (int hb = 0; hb < F::kKB / 4; ++hb)
+        tma_load_3d(dst + hb * a.xhalf, &maps.x, &full[i % a.ring], 0, (st_begin + i) * F::kKB + 4 * hb, 0);
     };
     const int pre = nst < a.ring ? nst : a.ring;
     if (lane == 0) {
@@ -221,16 +226,16 @@ __global__ void __maxnreg__(96)
       for (int i = 0; i < nst; ++i) {
         const int slot = i % a.ring;
         const uint32_t ph = static_cast<uint32_t>(i / a.ring) & 1u;
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full[slot], ph))) break;  // warp-uniform exit
+        if (!mbar_wait_warp(&full[slot], ph)) break;  // warp-uniform exit
         const uint8_t* xs = stg + slot * a.stage + kDWBytes;
         float ps = 0.0f;
         if (m < Mi) {
 #pragma unroll
           for (int bb = 0; bb < KBL; ++bb) {
-            const uint8_t* blk = xs + (part * KBL + bb) * kXSlot;
+            const int b = part * KBL + bb;  // W4A16: one box, rows 4 m + b
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
-              const uint4 v = ld_x_chunk(blk, m, c);
+              const uint4 v = ld_x_chunk(xs, 4 * m + b, c);
               const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
@@ -247,7 +252,7 @@ __global__ void __maxnreg__(96)
         mbar_arrive(&xready[slot]);
         const int j = i + a.ring;
         if (j < nst) {
-          if (!__all_sync(0xFFFFFFFFu, mbar_wait(&empty[slot], ph))) break;
+          if (!mbar_wait_warp(&empty[slot], ph)) break;
           if (lane == 0) {
             mbar_arrive_expect_tx(&full[slot], tx);
             load_w(j);
@@ -273,7 +278,10 @@ __global__ void __maxnreg__(96)
 #pragma unroll
         for (int c = 0; c < 4; ++c) acc[q][rt][c] = 0.0f;
     const __half2 fold = kInt4 ? __floats2half2_rn(0.0625f, 0.0625f) : __floats2half2_rn(0.25f, 0.25f);
-    const int rw = rs * 16 * kDRT + g;  // row of tile 0, lower half; tile rt adds 16 rt, upper +8
+    // MMA tile row g is stored row gp of its group of eight, gp = (g >> 1) | (g & 1) << 2: the
+    // eight lanes of a quarter warp then read rows of different swizzle phases (conflict free)
+    const int gp = (g >> 1) | ((g & 1) << 2);
+    const int rw = rs * 16 * kDRT + gp;  // row of tile 0, lower half; tile rt adds 16 rt, upper +8
     // ternary: tile row 127 is the virtual all-01 row (its result is sum_k x)
     const bool virt = !kInt4 && rw + 16 * (kDRT - 1) + 8 == kDTile - 1;
     const int64_t G = a.K >> 7;
@@ -281,19 +289,19 @@ __global__ void __maxnreg__(96)
     for (int i = 0; i < nst; ++i) {
       const int slot = i % a.ring;
       const uint32_t ph = static_cast<uint32_t>(i / a.ring) & 1u;
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full[slot], ph))) break;  // warp-uniform exit
+      if (!mbar_wait_warp(&full[slot], ph)) break;  // warp-uniform exit
       const uint8_t* st = stg + slot * a.stage;
       const uint8_t* xs = st + kDWBytes;
 #pragma unroll 1
       for (int sub = sub_lo; sub < sub_hi; ++sub) {
         const int chunk = sub * 4 + t;  // this lane's 16 bytes of the packed rows
-        // rows rw + 16 rt + 8 hr all have (row & 7) == g: swizzled chunk position chunk ^ g
+        // rows rw + 16 rt + 8 hr all have (row & 7) == gp: swizzled chunk position chunk ^ gp
         uint32_t w[kDRT][2][4];
 #pragma unroll
         for (int rt = 0; rt < kDRT; ++rt)
 #pragma unroll
           for (int hr = 0; hr < 2; ++hr) {
-            uint4 U = *reinterpret_cast<const uint4*>(st + (rw + 16 * rt + 8 * hr) * 128 + ((chunk ^ g) << 4));
+            uint4 U = *reinterpret_cast<const uint4*>(st + (rw + 16 * rt + 8 * hr) * 128 + ((chunk ^ gp) << 4));
             if (virt && rt == kDRT - 1 && hr == 1) U = make_uint4(0x55555555u, 0x55555555u, 0x55555555u, 0x55555555u);
             w[rt][hr][0] = U.x;
             w[rt][hr][1] = U.y;
@@ -301,8 +309,10 @@ __global__ void __maxnreg__(96)
             w[rt][hr][3] = U.w;
           }
         if (!kInt4) {
-          // the 64 codes of the chunk are k = 64*chunk + 0..63: activation block `chunk`
-          const uint8_t* blk = xs + chunk * kXSlot;
+          // the 64 codes of the chunk are k = 64*chunk + 0..63: activation block `chunk`, i.e.
+          // block t of the box of sub-chunk `sub`
+          const uint8_t* xbox = xs + sub * a.xhalf;
+          const int xrow = 4 * m + t;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             // P[j] = x[m][64*chunk + 32h + 2j .. +1]
@@ -310,7 +320,7 @@ __global__ void __maxnreg__(96)
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) {
               uint4 v = make_uint4(0u, 0u, 0u, 0u);
-              if (tokv) v = ld_x_chunk(blk, m, 4 * h + jj);
+              if (tokv) v = ld_x_chunk(xbox, xrow, 4 * h + jj);
               P[4 * jj] = v.x;
               P[4 * jj + 1] = v.y;
               P[4 * jj + 2] = v.z;
@@ -355,12 +365,12 @@ __global__ void __maxnreg__(96)
         } else {
           // the 32 codes of the chunk are k = 32*chunk + 0..31: half (chunk & 1) of activation
           // block chunk / 2, its 16-byte chunks 4*(chunk & 1) + 0..3
-          const uint8_t* blk = xs + (chunk >> 1) * kXSlot;
+          const int xrow = 4 * m + (chunk >> 1);
           uint32_t P[16];
 #pragma unroll
           for (int jj = 0; jj < 4; ++jj) {
             uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (tokv) v = ld_x_chunk(blk, m, 4 * (chunk & 1) + jj);
+            if (tokv) v = ld_x_chunk(xs, xrow, 4 * (chunk & 1) + jj);
             P[4 * jj] = v.x;
             P[4 * jj + 1] = v.y;
             P[4 * jj + 2] = v.z;
@@ -387,7 +397,7 @@ __global__ void __maxnreg__(96)
                 mma_16816(cg[1][rt], x0 & 0x00F000F0u, x1 & 0x00F000F0u, x2 & 0x00F000F0u, x3 & 0x00F000F0u, bo0, bo1);
               }
             }
-          if (sub == sub_lo) (void)__all_sync(0xFFFFFFFFu, mbar_wait(&xready[slot], ph));
+          if (sub == sub_lo) (void)mbar_wait_warp(&xready[slot], ph);
           const int64_t gi = static_cast<int64_t>(st_begin + i) * 2 + sub;
           const float xg0 = 8.0f * xg[(slot * 2 + sub) * 16 + 8 * T0 + 2 * t];
           const float xg1 = 8.0f * xg[(slot * 2 + sub) * 16 + 8 * T0 + 2 * t + 1];
@@ -485,7 +495,7 @@ __global__ void __maxnreg__(96)
 // host side
 // ---------------------------------------------------------------------------------------------
 struct DecodePlan {
-  int S, C, ring, stage, smem;
+  int S, C, ring, stage, xhalf, smem;
 };
 
 // Stage ring and cluster size for RB row blocks of one launch.
@@ -494,7 +504,8 @@ static bool plan_decode_t(int64_t RB, int64_t M, int64_t K, int num_sms, DecodeP
   using F = DecFmt<kInt4>;
   using L = DecLayout<kInt4>;
   const int C = static_cast<int>((K + F::kStageK - 1) / F::kStageK);
-  const int xbytes = F::kKB * (M > 8 ? 2 : 1) * 1024;  // one 8- or 16-row slot per block
+  const int xhalf = ((static_cast<int>(M) * 4 * 128 + 1023) / 1024) * 1024;
+  const int xbytes = (F::kKB / 4) * xhalf;  // activation boxes of one stage
   const int stage = kDWBytes + xbytes;
   // as many stages as two CTAs per SM allow (a CTA's whole slice when it fits, so that all its
   // weights are in flight before griddepcontrol.wait)
@@ -507,7 +518,7 @@ static bool plan_decode_t(int64_t RB, int64_t M, int64_t K, int num_sms, DecodeP
   if (S < 1) S = 1;
   if (S > kDMaxCluster) S = kDMaxCluster;
   if (S > C) S = C;
-  *p = DecodePlan{static_cast<int>(S), C, ring, stage, smem};
+  *p = DecodePlan{static_cast<int>(S), C, ring, stage, xhalf, smem};
   return true;
 }
 
@@ -573,11 +584,14 @@ static cudaError_t launch_decode_group(const __half* x, int count, const void* c
       return cudaErrorInvalidValue;
   }
   for (int g = count; g < kDMaxGroup; ++g) maps.m[g] = maps.m[0];
-  // activations: one box = 64 elements (128 bytes) x all M tokens
-  if (!make_tmap_2d(&maps.x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, static_cast<uint64_t>(K),
-                    static_cast<uint64_t>(M), static_cast<uint64_t>(K) * 2, 64,
-                    static_cast<uint32_t>(M), CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
+  {  // activations viewed as [M][K/64][64]: one box = four 64-element blocks x all M tokens
+    const uint64_t dims[3] = {64, static_cast<uint64_t>(K / 64), static_cast<uint64_t>(M)};
+    const uint64_t strides[2] = {128, static_cast<uint64_t>(K) * 2};
+    const uint32_t box[3] = {64, 4, static_cast<uint32_t>(M)};
+    if (!make_tmap_3d(&maps.x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, dims, strides, box,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
   a.rb_start[count] = static_cast<int>(rbs);
   if (rbs > 65535) return cudaErrorInvalidValue;
   DecodePlan p;
@@ -586,6 +600,7 @@ static cudaError_t launch_decode_group(const __half* x, int count, const void* c
   a.S = p.S;
   a.ring = p.ring;
   a.stage = p.stage;
+  a.xhalf = p.xhalf;
   return NT == 1 ? launch_decode_t<kInt4, 1>(maps, a, p, s) : launch_decode_t<kInt4, 2>(maps, a, p, s);
 }
 
