@@ -71,12 +71,16 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
             return
         self.th = threading.Thread(target=self._read, daemon=True)
         self.th.start()
+        t0 = time.time()  # nvidia-smi takes a moment to start: wait for its first sample
+        while not self.lines and time.time() - t0 < 3.0:
+            time.sleep(0.02)
+        self.lines.clear()  # keep only samples taken while the timed region runs
 
     def _read(self):
         for line in self.proc.stdout:
@@ -559,7 +563,7 @@ def run_reference(args, world, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--detail", action="store_true", help="per-shape decode breakdown")

@@ -32,6 +32,12 @@
  *     TQ_ERR_TIMEOUT in a device status word read by tq_device_status().
  *   - M == 0 or N == 0 is a valid empty problem (TQ_OK, nothing launched).  K must be > 0.
  *   - Inputs must be finite; results for Inf/NaN weights or activations are unspecified.
+ *   - The tensor-core GEMM kernels are launched with programmatic dependent launch: they start
+ *     while the preceding kernel on the stream is still running and wait for it before reading x
+ *     or writing y, but they read the packed weights, scales and bias (model constants) before
+ *     that wait.  Those must therefore not be written by the kernel enqueued immediately before
+ *     a GEMM call on the same stream (e.g. tq_quantize_pack followed directly by tq_gemm): put
+ *     any other operation, an event wait or a synchronisation in between.
  */
 #ifndef TQ_H
 #define TQ_H
