@@ -9,18 +9,19 @@
 // reduces through distributed shared memory in a fixed order (deterministic, no global scratch).
 // A stage is 128 bytes of every packed row (512 ternary or 256 INT4 codes) plus the activations
 // of those k for all M tokens.  Per CTA:
-//   * warp 8 (producer) streams each stage with TMA into a ring: the 128-row x 128-byte packed
+//   * the last warp (producer) streams each stage with TMA into a ring: the 128-row x 128-byte packed
 //     tile (issued before griddepcontrol.wait, weights never depend on the previous kernel) and
 //     the activations, one 64-element block x M tokens per box (issued after it), both
 //     128-byte swizzled so that every 16-byte read below is bank-conflict free.  For W4A16 it
 //     also sums each 128-wide group of x per token;
-//   * warps 0-7 (consumers): warp w owns rows 32 (w & 3) .. +31 (two 16-row MMA tiles) and,
-//     for M > 8, the token group w >> 2 over the whole stage, for M <= 8 the K half w >> 2 of
-//     every stage (the two halves are added in shared memory, in a fixed order, at the end).
-//     Weights are the A operand of mma.sync.m16n8k16 ("swap AB"), the tokens the N = 8
-//     operand: one MMA per 256 weights and token group.  Each lane builds its B fragments from
-//     the activations in shared memory (byte permutes into the k order the decode produces, see
-//     below); with two row tiles per warp one fragment feeds four MMAs.
+//   * consumers: warp w owns rows 32 (w & 3) .. +31 (two 16-row MMA tiles).  For M <= 8 there
+//     are eight, warp w taking the K half w >> 2 of every stage (the two halves are added in
+//     shared memory, in a fixed order, at the end); for M > 8 there are four, each holding both
+//     token groups, so that every decoded weight fragment feeds two MMAs.  Weights are the A
+//     operand of mma.sync.m16n8k16 ("swap AB"), the tokens the N = 8 operand: one MMA per 256
+//     weights and token group.  Each lane builds its B fragments from the activations in
+//     shared memory (byte permutes into the k order the decode produces, see below); with two
+//     row tiles per warp one fragment feeds four MMAs.
 //
 // In-register decode ("subnormal" trick).  ANDing a packed 32-bit word with 0x00030003 << 2p
 // leaves, in each fp16 half, the code at bits 2p..2p+1: the exact value c * 2^(2p-24) (fp16
@@ -44,11 +45,19 @@
 namespace tq {
 
 constexpr int kDTile = 128;                 // rows of one packed TMA tile
-constexpr int kDConsumers = 8;              // consumer warps: 4 row sets x 2 (token groups or K halves)
 constexpr int kDRowSets = 4;                // 32 rows = two 16-row MMA tiles per consumer warp
 constexpr int kDRT = 2;                     // 16-row MMA tiles per consumer warp
-constexpr int kDProducer = kDConsumers;     // TMA warp
-constexpr int kDThreads = (kDConsumers + 1) * 32;
+
+// Consumer warps per CTA, for NT token groups of which each warp holds TW: M <= 8 (NT = 1):
+// eight, the two K halves of every stage split between warps w and w + 4; M > 8 with TW = 2:
+// four, each holding both token groups (the decoded weights then feed two MMAs); M > 8 with
+// TW = 1: eight, warp w holding token group w >> 2 (more warps to hide latency when a CTA has a
+// single stage).  The producer is the warp after them.
+template <int NT, int TW>
+struct DecWarps {
+  static constexpr int kCons = (NT == 2 && TW == 2) ? 4 : 8;
+  static constexpr int kThreads = (kCons + 1) * 32;
+};
 constexpr int kDWBytes = kDTile * 128;      // weights of one stage: 128 rows x 128 bytes
 constexpr int kDMaxRing = 8;                // stages resident in shared memory
 constexpr int kDMaxCluster = 8;
@@ -119,12 +128,10 @@ __device__ __forceinline__ void make_frag(uint32_t Pa, uint32_t Pb, uint32_t Pc,
   o1 = *reinterpret_cast<uint32_t*>(&s23);
 }
 
-// Two CTAs of nine warps per SM: five warps share one SM sub-partition's 16K registers, so a
-// thread may use at most 102; 96 it is.
-template <bool kInt4, int NT>
-__global__ void __maxnreg__(96)
-    decode_gemm_kernel(const __grid_constant__ DecodeMaps maps, const __grid_constant__ DecodeArgs a) {
+template <bool kInt4, int NT, int TW>
+__device__ __forceinline__ void decode_gemm_body(const DecodeMaps& maps, const DecodeArgs& a) {
   using F = DecFmt<kInt4>;
+  using W = DecWarps<NT, TW>;
   using L = DecLayout<kInt4>;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned; pointer arithmetic on the __shared__ array keeps the shared address
@@ -166,7 +173,7 @@ __global__ void __maxnreg__(96)
     for (int i = 0; i < a.ring; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&xready[i], 32);
-      mbar_init(&empty[i], kDConsumers);
+      mbar_init(&empty[i], W::kCons);
     }
     fence_mbar_init();
   }
@@ -185,7 +192,7 @@ __global__ void __maxnreg__(96)
     if (biasm) ep_b = __half2float(biasm[ep_n]);
   }
 
-  if (warp == kDProducer) {
+  if (warp == W::kCons) {
     // ================================================================== producer warp
     const uint32_t tx = static_cast<uint32_t>(kDWBytes + F::kKB * Mi * 128);
     auto load_w = [&](int i) {
@@ -265,18 +272,21 @@ __global__ void __maxnreg__(96)
     // ================================================================== consumer warps
     // accumulator groups by exact power-of-two factor: pairs 0 and 3 (2^-24), 1 (2^-20), 2 (2^-16)
     constexpr int NG = kInt4 ? 1 : 3;
-    const int rs = warp & (kDRowSets - 1), hi = warp / kDRowSets;
-    const int T0 = NT == 2 ? hi : 0;                  // token group of this warp
-    const int sub_lo = NT == 2 ? 0 : hi, sub_hi = NT == 2 ? 2 : hi + 1;  // its K halves
-    const int m = 8 * T0 + g;                         // this lane's token (B column)
-    const bool tokv = m < Mi;
-    float acc[NG][kDRT][4];
+    const int rs = warp & (kDRowSets - 1), hi = warp / kDRowSets;  // hi: K half or token group
+    const int sub_lo = NT == 1 ? hi : 0, sub_hi = NT == 1 ? hi + 1 : 2;
+    const int Tb = TW < NT ? hi : 0;  // first token group of this warp
+    bool tokv[TW];  // this lane's token 8(Tb+T) + g (B column g of token group Tb+T) exists
+#pragma unroll
+    for (int T = 0; T < TW; ++T) tokv[T] = 8 * (Tb + T) + g < Mi;
+    float acc[NG][kDRT][TW][4];
 #pragma unroll
     for (int q = 0; q < NG; ++q)
 #pragma unroll
       for (int rt = 0; rt < kDRT; ++rt)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[q][rt][c] = 0.0f;
+        for (int T = 0; T < TW; ++T)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[q][rt][T][c] = 0.0f;
     const __half2 fold = kInt4 ? __floats2half2_rn(0.0625f, 0.0625f) : __floats2half2_rn(0.25f, 0.25f);
     // MMA tile row g is stored row gp of its group of eight, gp = (g >> 1) | (g & 1) << 2: the
     // eight lanes of a quarter warp then read rows of different swizzle phases (conflict free)
@@ -312,20 +322,21 @@ __global__ void __maxnreg__(96)
           // the 64 codes of the chunk are k = 64*chunk + 0..63: activation block `chunk`, i.e.
           // block t of the box of sub-chunk `sub`
           const uint8_t* xbox = xs + sub * a.xhalf;
-          const int xrow = 4 * m + t;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            // P[j] = x[m][64*chunk + 32h + 2j .. +1]
-            uint32_t P[16];
+            // P[T][j] = x[8(Tb+T)+g][64*chunk + 32h + 2j .. +1]
+            uint32_t P[TW][16];
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-              uint4 v = make_uint4(0u, 0u, 0u, 0u);
-              if (tokv) v = ld_x_chunk(xbox, xrow, 4 * h + jj);
-              P[4 * jj] = v.x;
-              P[4 * jj + 1] = v.y;
-              P[4 * jj + 2] = v.z;
-              P[4 * jj + 3] = v.w;
-            }
+            for (int T = 0; T < TW; ++T)
+#pragma unroll
+              for (int jj = 0; jj < 4; ++jj) {
+                uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                if (tokv[T]) v = ld_x_chunk(xbox, 4 * (8 * (Tb + T) + g) + t, 4 * h + jj);
+                P[T][4 * jj] = v.x;
+                P[T][4 * jj + 1] = v.y;
+                P[T][4 * jj + 2] = v.z;
+                P[T][4 * jj + 3] = v.w;
+              }
             uint32_t sh[kDRT][4];
 #pragma unroll
             for (int rt = 0; rt < kDRT; ++rt) {
@@ -336,8 +347,10 @@ __global__ void __maxnreg__(96)
             }
 #pragma unroll
             for (int pp = 0; pp < 4; ++pp) {
-              uint32_t be0, be1, bo0, bo1;
-              make_frag(P[pp], P[4 + pp], P[8 + pp], P[12 + pp], fold, be0, be1, bo0, bo1);
+              uint32_t be0[TW], be1[TW], bo0[TW], bo1[TW];
+#pragma unroll
+              for (int T = 0; T < TW; ++T)
+                make_frag(P[T][pp], P[T][4 + pp], P[T][8 + pp], P[T][12 + pp], fold, be0[T], be1[T], bo0[T], bo1[T]);
 #pragma unroll
               for (int q = 0; q < 2; ++q) {
                 const int p = 2 * pp + q;
@@ -357,7 +370,9 @@ __global__ void __maxnreg__(96)
                     a2 = sh[rt][2] & mk;
                     a3 = sh[rt][3] & mk;
                   }
-                  mma_16816(acc[pp == 3 ? 0 : pp][rt], a0, a1, a2, a3, q ? bo0 : be0, q ? bo1 : be1);
+#pragma unroll
+                  for (int T = 0; T < TW; ++T)
+                    mma_16816(acc[pp == 3 ? 0 : pp][rt][T], a0, a1, a2, a3, q ? bo0[T] : be0[T], q ? bo1[T] : be1[T]);
                 }
               }
             }
@@ -365,55 +380,70 @@ __global__ void __maxnreg__(96)
         } else {
           // the 32 codes of the chunk are k = 32*chunk + 0..31: half (chunk & 1) of activation
           // block chunk / 2, its 16-byte chunks 4*(chunk & 1) + 0..3
-          const int xrow = 4 * m + (chunk >> 1);
-          uint32_t P[16];
+          uint32_t P[TW][16];
 #pragma unroll
-          for (int jj = 0; jj < 4; ++jj) {
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (tokv) v = ld_x_chunk(xs, xrow, 4 * (chunk & 1) + jj);
-            P[4 * jj] = v.x;
-            P[4 * jj + 1] = v.y;
-            P[4 * jj + 2] = v.z;
-            P[4 * jj + 3] = v.w;
-          }
-          float cg[2][kDRT][4];  // two chains (class 0 / class 1 fields)
+          for (int T = 0; T < TW; ++T)
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+              uint4 v = make_uint4(0u, 0u, 0u, 0u);
+              if (tokv[T]) v = ld_x_chunk(xs, 4 * (8 * (Tb + T) + g) + (chunk >> 1), 4 * (chunk & 1) + jj);
+              P[T][4 * jj] = v.x;
+              P[T][4 * jj + 1] = v.y;
+              P[T][4 * jj + 2] = v.z;
+              P[T][4 * jj + 3] = v.w;
+            }
+          float cg[2][kDRT][TW][4];  // two chains (class 0 / class 1 fields)
 #pragma unroll
           for (int j = 0; j < 2; ++j)
 #pragma unroll
             for (int rt = 0; rt < kDRT; ++rt)
 #pragma unroll
-              for (int c = 0; c < 4; ++c) cg[j][rt][c] = 0.0f;
+              for (int T = 0; T < TW; ++T)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) cg[j][rt][T][c] = 0.0f;
 #pragma unroll
           for (int h = 0; h < 2; ++h)
 #pragma unroll
             for (int s2 = 0; s2 < 2; ++s2) {
-              uint32_t be0, be1, bo0, bo1;
-              make_frag(P[8 * h + s2], P[8 * h + 2 + s2], P[8 * h + 4 + s2], P[8 * h + 6 + s2], fold, be0, be1, bo0, bo1);
+              uint32_t be0[TW], be1[TW], bo0[TW], bo1[TW];
+#pragma unroll
+              for (int T = 0; T < TW; ++T)
+                make_frag(P[T][8 * h + s2], P[T][8 * h + 2 + s2], P[T][8 * h + 4 + s2], P[T][8 * h + 6 + s2], fold,
+                          be0[T], be1[T], bo0[T], bo1[T]);
 #pragma unroll
               for (int rt = 0; rt < kDRT; ++rt) {
                 const uint32_t x0 = w[rt][0][2 * h] >> (8 * s2), x1 = w[rt][1][2 * h] >> (8 * s2);
                 const uint32_t x2 = w[rt][0][2 * h + 1] >> (8 * s2), x3 = w[rt][1][2 * h + 1] >> (8 * s2);
-                mma_16816(cg[0][rt], x0 & 0x000F000Fu, x1 & 0x000F000Fu, x2 & 0x000F000Fu, x3 & 0x000F000Fu, be0, be1);
-                mma_16816(cg[1][rt], x0 & 0x00F000F0u, x1 & 0x00F000F0u, x2 & 0x00F000F0u, x3 & 0x00F000F0u, bo0, bo1);
+#pragma unroll
+                for (int cls = 0; cls < 2; ++cls) {
+                  const uint32_t mk = cls ? 0x00F000F0u : 0x000F000Fu;
+#pragma unroll
+                  for (int T = 0; T < TW; ++T)
+                    mma_16816(cg[cls][rt][T], x0 & mk, x1 & mk, x2 & mk, x3 & mk, cls ? bo0[T] : be0[T],
+                              cls ? bo1[T] : be1[T]);
+                }
               }
             }
           if (sub == sub_lo) (void)mbar_wait_warp(&xready[slot], ph);
           const int64_t gi = static_cast<int64_t>(st_begin + i) * 2 + sub;
-          const float xg0 = 8.0f * xg[(slot * 2 + sub) * 16 + 8 * T0 + 2 * t];
-          const float xg1 = 8.0f * xg[(slot * 2 + sub) * 16 + 8 * T0 + 2 * t + 1];
 #pragma unroll
           for (int rt = 0; rt < kDRT; ++rt) {
             const int64_t n0 = row0 + rw + 16 * rt, n1 = n0 + 8;
             // groups past K (a zero-filled half stage) contribute nothing
             const float s0 = (n0 < Nm && gi < G) ? __half2float(scm[n0 * G + gi]) : 0.0f;
             const float s1 = (n1 < Nm && gi < G) ? __half2float(scm[n1 * G + gi]) : 0.0f;
-            float c4[4];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) c4[c] = cg[0][rt][c] + cg[1][rt][c];
-            acc[0][rt][0] = fmaf(s0, fmaf(c4[0], 16777216.0f, -xg0), acc[0][rt][0]);
-            acc[0][rt][1] = fmaf(s0, fmaf(c4[1], 16777216.0f, -xg1), acc[0][rt][1]);
-            acc[0][rt][2] = fmaf(s1, fmaf(c4[2], 16777216.0f, -xg0), acc[0][rt][2]);
-            acc[0][rt][3] = fmaf(s1, fmaf(c4[3], 16777216.0f, -xg1), acc[0][rt][3]);
+            for (int T = 0; T < TW; ++T) {
+              const float xg0 = 8.0f * xg[(slot * 2 + sub) * 16 + 8 * (Tb + T) + 2 * t];
+              const float xg1 = 8.0f * xg[(slot * 2 + sub) * 16 + 8 * (Tb + T) + 2 * t + 1];
+              float c4[4];
+#pragma unroll
+              for (int c = 0; c < 4; ++c) c4[c] = cg[0][rt][T][c] + cg[1][rt][T][c];
+              acc[0][rt][T][0] = fmaf(s0, fmaf(c4[0], 16777216.0f, -xg0), acc[0][rt][T][0]);
+              acc[0][rt][T][1] = fmaf(s0, fmaf(c4[1], 16777216.0f, -xg1), acc[0][rt][T][1]);
+              acc[0][rt][T][2] = fmaf(s1, fmaf(c4[2], 16777216.0f, -xg0), acc[0][rt][T][2]);
+              acc[0][rt][T][3] = fmaf(s1, fmaf(c4[3], 16777216.0f, -xg1), acc[0][rt][T][3]);
+            }
           }
         }
       }
@@ -421,29 +451,31 @@ __global__ void __maxnreg__(96)
       if (lane == 0) mbar_arrive(&empty[slot]);
     }
     // this warp's results: factors 2^-24 (pairs 0 and 3), 2^-20 (pair 1), 2^-16 (pair 2) applied
-    // exactly; rows rw + 16 rt + 8 hr, tokens 8 T0 + 2t + c
-    float v[kDRT][4];
+    // exactly; rows rw + 16 rt + 8 hr, tokens 8 (Tb + T) + 2t + c
+    float v[kDRT][TW][4];
 #pragma unroll
     for (int rt = 0; rt < kDRT; ++rt)
 #pragma unroll
-      for (int ci = 0; ci < 4; ++ci)
-        v[rt][ci] = kInt4 ? acc[0][rt][ci]
-                          : fmaf(acc[0][rt][ci], 16777216.0f,
-                                 fmaf(acc[1 % NG][rt][ci], 1048576.0f, acc[2 % NG][rt][ci] * 65536.0f));
+      for (int T = 0; T < TW; ++T)
+#pragma unroll
+        for (int ci = 0; ci < 4; ++ci)
+          v[rt][T][ci] = kInt4 ? acc[0][rt][T][ci]
+                               : fmaf(acc[0][rt][T][ci], 16777216.0f,
+                                      fmaf(acc[1 % NG][rt][T][ci], 1048576.0f, acc[2 % NG][rt][T][ci] * 65536.0f));
     if (NT == 1) {  // M <= 8: add the second K half (warps 4-7) to the first, fixed order
       if (hi == 1) {
 #pragma unroll
         for (int rt = 0; rt < kDRT; ++rt)
 #pragma unroll
           for (int ci = 0; ci < 4; ++ci)
-            part[(rw + 16 * rt + 8 * (ci >> 1)) * 8 + 2 * t + (ci & 1)] = v[rt][ci];
+            part[(rw + 16 * rt + 8 * (ci >> 1)) * 8 + 2 * t + (ci & 1)] = v[rt][0][ci];
       }
-      named_barrier_sync(1, kDConsumers * 32);
+      named_barrier_sync(1, W::kCons * 32);
       if (hi == 1) goto consumers_done;
 #pragma unroll
       for (int rt = 0; rt < kDRT; ++rt)
 #pragma unroll
-        for (int ci = 0; ci < 4; ++ci) v[rt][ci] += part[(rw + 16 * rt + 8 * (ci >> 1)) * 8 + 2 * t + (ci & 1)];
+        for (int ci = 0; ci < 4; ++ci) v[rt][0][ci] += part[(rw + 16 * rt + 8 * (ci >> 1)) * 8 + 2 * t + (ci & 1)];
     }
     {
       // push this slice's partial results to the CTA that owns each row (owner q holds rows
@@ -458,17 +490,19 @@ __global__ void __maxnreg__(96)
           const int q = ((r + 1) * a.S - 1) / F::kRows;
           const int slot = r - (q * F::kRows) / a.S;
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const float val = v[rt][2 * hr + c];
-            const int tok = 8 * T0 + 2 * t + c;
-            if (vrow) {
-              for (int o = 0; o < a.S; ++o)
-                st_shared_cluster_f32(mapa_shared(sxr_local + (rank * 16 + tok) * 4, static_cast<uint32_t>(o)), val);
-            } else if (r < F::kRows) {
-              st_shared_cluster_f32(
-                  mapa_shared(red_local + ((rank * 16 + tok) * own_cap + slot) * 4, static_cast<uint32_t>(q)), val);
+          for (int T = 0; T < TW; ++T)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              const float val = v[rt][T][2 * hr + c];
+              const int tok = 8 * (Tb + T) + 2 * t + c;
+              if (vrow) {
+                for (int o = 0; o < a.S; ++o)
+                  st_shared_cluster_f32(mapa_shared(sxr_local + (rank * 16 + tok) * 4, static_cast<uint32_t>(o)), val);
+              } else if (r < F::kRows) {
+                st_shared_cluster_f32(
+                    mapa_shared(red_local + ((rank * 16 + tok) * own_cap + slot) * 4, static_cast<uint32_t>(q)), val);
+              }
             }
-          }
         }
     }
   consumers_done:;
@@ -489,6 +523,28 @@ __global__ void __maxnreg__(96)
       ym[mm * Nm + ep_n] = __float2half_rn(v + ep_b);
     }
   }
+}
+
+// M <= 8: two CTAs of nine warps per SM; five warps share one SM sub-partition's 16K registers,
+// so a thread may use at most 102 (96 it is).
+template <bool kInt4>
+__global__ void __maxnreg__(96)
+    decode_gemm_kernel_m8(const __grid_constant__ DecodeMaps maps, const __grid_constant__ DecodeArgs a) {
+  decode_gemm_body<kInt4, 1, 1>(maps, a);
+}
+
+// M <= 16, both token groups per warp: two CTAs of five warps per SM (at most 168 registers).
+template <bool kInt4>
+__global__ void __launch_bounds__(DecWarps<2, 2>::kThreads, 2)
+    decode_gemm_kernel_m16(const __grid_constant__ DecodeMaps maps, const __grid_constant__ DecodeArgs a) {
+  decode_gemm_body<kInt4, 2, 2>(maps, a);
+}
+
+// M <= 16, one token group per warp: two CTAs of nine warps per SM (96 registers, as above).
+template <bool kInt4>
+__global__ void __maxnreg__(96)
+    decode_gemm_kernel_m16s(const __grid_constant__ DecodeMaps maps, const __grid_constant__ DecodeArgs a) {
+  decode_gemm_body<kInt4, 2, 1>(maps, a);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -526,15 +582,16 @@ static bool plan_decode(bool int4, int64_t RB, int64_t M, int64_t K, int num_sms
   return int4 ? plan_decode_t<true>(RB, M, K, num_sms, p) : plan_decode_t<false>(RB, M, K, num_sms, p);
 }
 
-template <bool kInt4, int NT>
+template <bool kInt4, int NT, int TW>
 static cudaError_t launch_decode_t(const DecodeMaps& maps, const DecodeArgs& a, const DecodePlan& p,
                                    cudaStream_t s) {
-  auto* kern = decode_gemm_kernel<kInt4, NT>;
+  auto* kern = NT == 1 ? decode_gemm_kernel_m8<kInt4>
+                       : (TW == 2 ? decode_gemm_kernel_m16<kInt4> : decode_gemm_kernel_m16s<kInt4>);
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), kDSmemBudget);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(p.S), static_cast<unsigned>(a.rb_start[a.count]), 1);
-  cfg.blockDim = dim3(kDThreads, 1, 1);
+  cfg.blockDim = dim3(DecWarps<NT, TW>::kThreads, 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(p.smem);
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
@@ -601,7 +658,10 @@ static cudaError_t launch_decode_group(const __half* x, int count, const void* c
   a.ring = p.ring;
   a.stage = p.stage;
   a.xhalf = p.xhalf;
-  return NT == 1 ? launch_decode_t<kInt4, 1>(maps, a, p, s) : launch_decode_t<kInt4, 2>(maps, a, p, s);
+  if (NT == 1) return launch_decode_t<kInt4, 1, 1>(maps, a, p, s);
+  // a CTA with a single stage and two CTAs per SM: more, lighter warps hide the latency better
+  const bool single = (p.C + p.S - 1) / p.S <= 1 && static_cast<int64_t>(p.S) * rbs > di.num_sms;
+  return single ? launch_decode_t<kInt4, 2, 1>(maps, a, p, s) : launch_decode_t<kInt4, 2, 2>(maps, a, p, s);
 }
 
 bool decode_supported(bool int4, int64_t M, int64_t N, int64_t K) {

@@ -121,3 +121,18 @@ def test_validate_counts_code_11():
     p[3, 2] = 0b11_01_01_01          # code 11 in the padding of the last byte (k = 11 >= K): ok
     p[4, 2] = 0b01_01_01_11          # code 11 at k = 8 < K
     assert tq.tq_validate_packed(p, 10) == 2
+
+
+# M > 8 has two consumer layouts (both token groups per warp, or one group per warp when every
+# CTA has a single stage and there are more CTAs than SMs): cover both, with a partial second
+# token group, for both formats.
+@pytest.mark.parametrize("M", [9, 12, 16])
+@pytest.mark.parametrize("N,K", [(4096, 4096), (1024, 4096), (4096, 14336)])
+def test_decode_m_gt_8_layouts(M, N, K):
+    need_cuda()
+    x, p, s, b = _tq_problem(M, N, K, 700 + M + N // 64)
+    y = tq.tq_gemm(x, p, s, b, path=tq.PATH_DECODE)
+    check_tq_gemm(x, p, s, b, y, cols=np.arange(0, N, 7), label=f"tq decode M={M} {N}x{K}")
+    xw, qw, sc, bw = _w4_problem(M, N, K, 800 + M)
+    yw = tq.w4g_gemm(xw, qw, sc, bw, path=tq.PATH_DECODE)
+    check_w4g_gemm(xw, qw, sc, bw, yw, cols=np.arange(0, N, 7), label=f"w4g decode M={M} {N}x{K}")
