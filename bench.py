@@ -487,16 +487,24 @@ def secondary_rows(args, rank, layers, peaks):
 
 
 def load_traffic():
-    """DRAM bytes per decode launch from the committed ncu summary, if one matches this kernel."""
+    """DRAM bytes per decode launch from the committed ncu summary, only if it was taken on this
+    kernel source (the summary records the SHA-256 of the decode source file)."""
+    import hashlib
+
     p = os.path.join(ROOT, "profiles", "traffic.json")
-    if not os.path.exists(p):
+    src = os.path.join(ROOT, "bit_weight_only_tq_b200", "csrc", "tq_decode.cu")
+    if not os.path.exists(p) or not os.path.exists(src):
         return None
     try:
         with open(p) as f:
             d = json.load(f)
-        return d.get("decode_gemm_bytes_per_launch")
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
     except (OSError, ValueError):
         return None
+    if d.get("kernel_source_sha256") != sha:
+        return None
+    return d.get("decode_gemm_bytes_per_launch")
 
 
 # ------------------------------------------------------------------------------------------------
@@ -560,8 +568,64 @@ def run_reference(args, world, rank):
     }
 
 
+# ------------------------------------------------------------------------------------------------
+# small fixed cases for profiler captures (a few launches each, a few GB on the device at most)
+# ------------------------------------------------------------------------------------------------
+PROFILE_CASES = {
+    "decode": "ternary gate_proj 14336x4096 at M=1, 3 launches; q/k/v group (4096+1024+1024)x4096 at M=16, 3 launches",
+    "prefill": "ternary q_proj 4096x4096 at M=2048 (1 % outlier rows), 3 launches; W4A16 gate_proj 14336x4096 at M=512, 3 launches",
+    "pack": "tq_quantize_pack of an fp16 Qwen2-7B gate_up 37888x3584 (2 launches) and an fp32 4096x4096 (2 launches); w4g_quantize_pack of the latter (2 launches)",
+}
+
+
+def run_profile_case(name):
+    import torch
+
+    import bit_weight_only_tq_b200 as tq
+    import tq_inputs as I
+
+    if name == "decode":
+        w = I.weights(14336, 4096, 1, device="cuda")
+        p, s = tq.tq_quantize_pack(w)
+        del w
+        x = I.activations(1, 4096, 2, device="cuda")
+        for _ in range(3):
+            tq.tq_gemm(x, p, s)
+        ws = [tq.tq_quantize_pack(I.weights(N, 4096, 3 + i, device="cuda")) for i, N in enumerate((4096, 1024, 1024))]
+        x16 = I.activations(16, 4096, 4, device="cuda")
+        for _ in range(3):
+            tq.tq_gemm_grouped(x16, [a for a, _ in ws], [b for _, b in ws])
+    elif name == "prefill":
+        w = I.weights(4096, 4096, 1, device="cuda")
+        p, s = tq.tq_quantize_pack(w)
+        del w
+        x = I.activations(2048, 4096, 2, device="cuda", outlier_row_frac=0.01)
+        for _ in range(3):
+            tq.tq_gemm(x, p, s)
+        w = I.weights(14336, 4096, 5, device="cuda")
+        q, sc = tq.w4g_quantize_pack(w)
+        del w
+        x = I.activations(512, 4096, 6, device="cuda")
+        for _ in range(3):
+            tq.w4g_gemm(x, q, sc)
+    elif name == "pack":
+        w = I.weights(37888, 3584, 1, device="cuda", dtype=torch.float16)
+        for _ in range(2):
+            tq.tq_quantize_pack(w)
+        w = I.weights(4096, 4096, 2, device="cuda")
+        for _ in range(2):
+            tq.tq_quantize_pack(w)
+        for _ in range(2):
+            tq.w4g_quantize_pack(w)
+    torch.cuda.synchronize()
+    assert tq.tq_device_status() == 0
+    print(f"profile case {name} done: {PROFILE_CASES[name]}", flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
+    ap.add_argument("--case", choices=sorted(PROFILE_CASES),
+                    help="run one small fixed case for a profiler capture and exit (no timing)")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=3)
@@ -575,6 +639,9 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.case:
+        run_profile_case(args.case)
+        return 0
 
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))

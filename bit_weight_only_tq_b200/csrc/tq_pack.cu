@@ -211,6 +211,105 @@ __global__ void __launch_bounds__(kPackThreads)
 }
 
 // ---------------------------------------------------------------------------------------------
+// Ternary pack, fp16 rows with K % 8 == 0 and a 16-byte aligned base: the same semantics as
+// above with 16-byte loads and cheaper exact sums.  |w| is converted to fp64 by the hardware
+// (exact); a lane's fp64 partial sum stays exact while it is below 2^29 (every value is a
+// multiple of 2^-24), so it is flushed every 8192 elements into integer units of 2^-24, kept as
+// a high (>> 32) and a low part so that no row length overflows; the warp total is the sum of
+// the two exact parts, rounded once.  The code decision is a packed 16-bit compare of the
+// magnitude patterns against the threshold pattern.
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ double f16_mag_f64(uint32_t h) {  // |h| for the fp16 pattern in bits 0..15
+  double d;
+  const unsigned short m = static_cast<unsigned short>(h & 0x7FFFu);
+  asm("{\n\t.reg .f16 t;\n\tmov.b16 t, %1;\n\tcvt.f64.f16 %0, t;\n\t}" : "=d"(d) : "h"(m));
+  return d;
+}
+
+struct UnitsAcc {  // exact running sum of fp16 magnitudes
+  double part = 0.0;
+  long long hi = 0, lo = 0;
+  __device__ __forceinline__ void flush() {
+    const unsigned long long u = static_cast<unsigned long long>(part * 16777216.0);  // exact
+    hi += static_cast<long long>(u >> 32);
+    lo += static_cast<long long>(u & 0xFFFFFFFFull);
+    part = 0.0;
+  }
+  __device__ __forceinline__ double warp_total() {  // all lanes get the correctly rounded total
+    flush();
+    long long h = hi, l = lo;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      h += __shfl_xor_sync(0xFFFFFFFFu, h, o);
+      l += __shfl_xor_sync(0xFFFFFFFFu, l, o);
+    }
+    return __ll2double_rn(h) * 256.0 + __ll2double_rn(l) * 0x1p-24;  // two exact terms, one rounding
+  }
+};
+
+__global__ void __launch_bounds__(kPackThreads)
+    tq_pack_f16_kernel(const uint16_t* __restrict__ w, uint8_t* __restrict__ packed,
+                       uint16_t* __restrict__ scale, int64_t N, int64_t K) {
+  constexpr int kWarps = kPackThreads / 32;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int64_t C = K >> 3;  // 16-byte chunks (8 elements) per row
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
+  for (int64_t n = static_cast<int64_t>(blockIdx.x) * kWarps + wid; n < N; n += nwarps) {
+    const uint4* row = reinterpret_cast<const uint4*>(w + n * K);
+    UnitsAcc accS;
+    int cnt = 0;
+#pragma unroll 2
+    for (int64_t j = lane; j < C; j += 32) {
+      const uint4 v = __ldg(row + j);
+      accS.part += ((f16_mag_f64(v.x) + f16_mag_f64(v.x >> 16)) + (f16_mag_f64(v.y) + f16_mag_f64(v.y >> 16))) +
+                   ((f16_mag_f64(v.z) + f16_mag_f64(v.z >> 16)) + (f16_mag_f64(v.w) + f16_mag_f64(v.w >> 16)));
+      if (++cnt == 1024) {  // 8192 elements < 2^13: the partial stays below 2^29
+        accS.flush();
+        cnt = 0;
+      }
+    }
+    const double S = accS.warp_total();
+    const double t = 0.7 * (S / static_cast<double>(K));
+    const uint32_t tb = magnitude_floor_bits<true>(t);
+    const uint32_t tb2 = (tb | (tb << 16)) | 0x80008000u;
+    UnitsAcc accA;
+    int nz = 0;
+    cnt = 0;
+    uint16_t* prow = reinterpret_cast<uint16_t*>(packed + n * (K >> 2));
+#pragma unroll 2
+    for (int64_t j = lane; j < C; j += 32) {
+      const uint4 v = __ldg(row + j);
+      const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+      uint32_t out = 0;
+      double a = 0.0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        // per 16-bit half: bit 15 of D is set iff |h| <= t (0x8000 + tb - |h| never borrows
+        // across halves)
+        const uint32_t D = tb2 - (wd[i] & 0x7FFF7FFFu);
+        const uint32_t zero = (D >> 15) & 0x00010001u;           // code 01
+        const uint32_t pos = (~(D | wd[i]) >> 14) & 0x00020002u;  // |h| > t and h >= 0: code 10
+        const uint32_t c = zero | pos;                            // else 00
+        out |= ((c | (c >> 14)) & 0xFu) << (4 * i);
+        nz += __popc(~D & 0x80008000u);
+        if (!(D & 0x8000u)) a += f16_mag_f64(wd[i]);
+        if (!(D & 0x80000000u)) a += f16_mag_f64(wd[i] >> 16);
+      }
+      accA.part += a;
+      if (++cnt == 1024) {
+        accA.flush();
+        cnt = 0;
+      }
+      prow[j] = static_cast<uint16_t>(out);
+    }
+    const double A = accA.warp_total();
+    const int nzt = warp_sum(nz);
+    if (lane == 0)
+      scale[n] = nzt > 0 ? f64_to_f16_rne(A / static_cast<double>(nzt)) : static_cast<uint16_t>(0);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
 // W4A16 pack: one warp per (row n, group g of 128).  Lane l holds k = 128g + 4l .. 4l+3.
 // ---------------------------------------------------------------------------------------------
 template <bool kF16>
@@ -271,6 +370,11 @@ cudaError_t launch_tq_pack(const void* w, bool w_f16, uint8_t* packed, uint16_t*
   if (grid > int64_t(di.num_sms) * 8) grid = int64_t(di.num_sms) * 8;
   const int binw = 30 - ceil_log2_i64(K);
   const uintptr_t a = reinterpret_cast<uintptr_t>(w);
+  if (w_f16 && K % 8 == 0 && a % 16 == 0) {
+    tq_pack_f16_kernel<<<static_cast<unsigned>(grid), kPackThreads, 0, s>>>(
+        static_cast<const uint16_t*>(w), packed, scale, N, K);
+    return cudaGetLastError();
+  }
   const int vec = (K % 4 == 0) && (a % (w_f16 ? 8 : 16) == 0);
   if (w_f16)
     tq_pack_kernel<true><<<static_cast<unsigned>(grid), kPackThreads, 0, s>>>(w, packed, scale, N,
