@@ -1,21 +1,27 @@
 // tq_prefill.cu -- tensor-core GEMM for large M (prefill), ternary and W4A16 weights.
 //
-// This path is a dense contraction, so it runs on the 5th-generation tensor cores:
-//   y[m, n] = sum_k x[m,k] * What[n,k]   as   D(TMEM, fp32) += A(x tile, smem) * B(What tile, smem)^T
-// [TQ] §4.2-4.3 (prior art: decode the codes into fp16 tensor-core operands, accumulate in fp32,
-// apply the per-row scale after the MMA; stage weights through shared memory).  On sm_100a:
-//   * warp 0, one lane: TMA loads of the x tile (128 tokens x 64 k, fp16, 128-byte swizzle) and
-//     of the packed weight tile (256 rows x 16 bytes ternary / 32 bytes W4A16) into a ring;
-//   * warps 4-11 (256 threads, one weight row each): decode the packed row into fp16 and store
-//     it in the K-major 128-byte-swizzle layout the UMMA descriptor expects -- exactly what TMA
-//     would have written for an fp16 matrix, so A and B share one descriptor format;
+// This path is a dense contraction, so it runs on the 5th-generation tensor cores.  [TQ] §4.2-4.3
+// (prior art): decode the codes into fp16 tensor-core operands, accumulate in fp32, apply the
+// per-row scale after the MMA.  On sm_100a the decoded weights never touch shared memory: they
+// are the A operand of tcgen05.mma, written straight into tensor memory, and the activations are
+// the B operand:
+//   D[n, m] (TMEM, fp32) += A[n, k] (TMEM, fp16 decoded weights) * B[m, k]^T (smem, x tile)
+// One CTA = 128 weight rows (the TMEM lanes, UMMA M) x TN tokens (UMMA N = 256, or 128 for
+// small M):
+//   * warp 0, one lane: TMA loads of the x tile (TN tokens x 64 k, fp16, 128-byte swizzle, the
+//     K-major layout the UMMA descriptor expects) and of the packed weight tile (128 rows x 16
+//     bytes ternary / 32 bytes W4A16) into a ring;
+//   * warp 1: allocates the tensor memory (accumulator + a ring of decoded-weight slots); one
+//     lane issues tcgen05.mma (M=128, N=TN, K=16, A from tensor memory) and commits to
+//     mbarriers that free the input stages;
+//   * warps 4-7 (thread r = weight row r = TMEM lane r): decode the packed row into 32 fp16x2
+//     registers in natural k order and store them with one tcgen05.st per stage;
 //       ternary: (c - 1) is exact in fp16; the row scale is applied in the epilogue;
 //       W4A16:   fp16(q * s[n, k/128]) (one rounding, <= 2^-11 relative);
-//   * warp 1: allocates 256 TMEM columns (the 128 x 256 fp32 accumulator); one lane issues
-//     tcgen05.mma (M=128, N=256, K=16, fp16 x fp16 -> fp32) and commits to mbarriers that free
-//     the input stages;
-//   * warps 0-3: epilogue -- tcgen05.ld the accumulator (lane = token row), apply scale / bias,
-//     convert to fp16 and store.
+//     then the epilogue: tcgen05.ld 32 tokens of the row at a time, scale / bias, fp16, staged
+//     through shared memory for coalesced 16-byte stores of y.
+// Shared-memory traffic per MMA is the x tile only (read by the MMA, written by TMA); decoding
+// into shared memory would add the weight tile twice (written, then read).
 // Every wait is bounded; a wait that runs out records a timeout in the device status word and
 // the CTA skips the rest of its work, frees its TMEM and exits (kernels never trap).
 //
@@ -32,36 +38,34 @@
 
 namespace tq {
 
-constexpr int kPBM = 128;        // tokens per tile (UMMA M)
-constexpr int kPBN = 256;        // weight rows per tile (UMMA N)
-constexpr int kPBK = 64;         // K per stage: one 128-byte swizzle row of fp16
-constexpr int kPRingL = 4;       // stages of (x tile, packed tile)
-constexpr int kPRingB = 3;       // stages of decoded weight tiles
-constexpr int kPDecThreads = 256;
-constexpr int kPThreads = 128 + kPDecThreads;
-constexpr int kPTileA = kPBM * kPBK * 2;  // 16 KB
-constexpr int kPTileB = kPBN * kPBK * 2;  // 32 KB
-constexpr uint32_t kPTmemCols = 256;
+constexpr int kQM = 128;         // weight rows per CTA (UMMA M, TMEM lanes)
+constexpr int kQK = 64;          // K per stage: one 128-byte swizzle row of fp16
+constexpr int kQRing = 4;        // stages of (x tile, packed tile)
+constexpr int kQARing = 4;       // tensor-memory slots of decoded weights (32 columns each)
+constexpr int kQThreads = 256;   // warp 0 TMA, warp 1 MMA, warps 4-7 decode + epilogue
 
 template <bool kInt4>
 struct PFmt {
-  static constexpr int kRowBytes = kInt4 ? 32 : 16;  // packed bytes per row per k-block
-  static constexpr int kTileP = kPBN * kRowBytes;
+  static constexpr int kRowBytes = kInt4 ? 32 : 16;  // packed bytes per row per stage
+  static constexpr int kTileP = kQM * kRowBytes;
 };
 
-template <bool kInt4>
+template <bool kInt4, int TN>
 struct PrefillLayout {
-  static constexpr int kOffA = 0;
-  static constexpr int kOffB = kOffA + kPRingL * kPTileA;
-  static constexpr int kOffP = kOffB + kPRingB * kPTileB;
-  static constexpr int kOffScale = kOffP + kPRingL * PFmt<kInt4>::kTileP;
-  static constexpr int kOffBias = kOffScale + kPBN * 4;
-  static constexpr int kOffBar = kOffBias + kPBN * 4;
-  // barriers: fullL[4], emptyA[4], emptyP[4], fullB[3], emptyB[3], accFull, tmem slot
-  static constexpr int kNumBars = 3 * kPRingL + 2 * kPRingB + 1;
+  static constexpr int kTileX = TN * kQK * 2;  // x tile of one stage
+  static constexpr int kOffX = 0;
+  static constexpr int kOffP = kOffX + kQRing * kTileX;
+  static constexpr int kOffBar = kOffP + kQRing * PFmt<kInt4>::kTileP;
+  // barriers: full[R], emptyX[R], emptyP[R], afull[RA], aempty[RA], accFull; then the TMEM slot
+  static constexpr int kNumBars = 3 * kQRing + 2 * kQARing + 1;
   static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffTmemSlot + 16;
   static constexpr int kAlloc = kBytes + 1024;  // alignment slack
+  // tensor memory: accumulator columns [0, TN), decoded-weight slots after it
+  static constexpr uint32_t kColA = TN;
+  static constexpr uint32_t kTmemCols = TN + 32 * kQARing <= 256 ? 256u : 512u;
+  // epilogue staging (reuses the x ring): 32 tokens x 128 rows fp16
+  static_assert(32 * kQM * 2 <= kQRing * kTileX, "staging fits in the x ring");
 };
 
 struct PrefillArgs {
@@ -110,62 +114,53 @@ __device__ __forceinline__ uint4 decode_w4_8(uint32_t w, uint32_t s2) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-template <bool kInt4>
-__global__ void __launch_bounds__(kPThreads, 1)
+template <bool kInt4, int TN>
+__global__ void __launch_bounds__(kQThreads, 1)
     prefill_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
                         const __grid_constant__ CUtensorMap tmap_w, const PrefillArgs a) {
-  using L = PrefillLayout<kInt4>;
+  using L = PrefillLayout<kInt4, TN>;
   using F = PFmt<kInt4>;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned; pointer arithmetic on the __shared__ array keeps the shared address
   // space visible to the compiler (plain ld/st.shared instead of generic accesses)
   uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kOffBar);
-  uint64_t* fullL = bars;
-  uint64_t* emptyA = bars + kPRingL;
-  uint64_t* emptyP = bars + 2 * kPRingL;
-  uint64_t* fullB = bars + 3 * kPRingL;
-  uint64_t* emptyB = fullB + kPRingB;
-  uint64_t* accFull = emptyB + kPRingB;
+  uint64_t* full = bars;                     // x tile + packed tile landed (TMA)
+  uint64_t* emptyX = bars + kQRing;          // x tile consumed (MMA commit)
+  uint64_t* emptyP = bars + 2 * kQRing;      // packed tile consumed (decode warps)
+  uint64_t* afull = bars + 3 * kQRing;       // decoded weights in tensor memory
+  uint64_t* aempty = afull + kQARing;        // ... consumed (MMA commit)
+  uint64_t* accFull = aempty + kQARing;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::kOffTmemSlot);
-  float* sScale = reinterpret_cast<float*>(sm + L::kOffScale);
-  float* sBias = reinterpret_cast<float*>(sm + L::kOffBias);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kPBN;
-  const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kPBM;
-  const int nk = static_cast<int>(a.K / kPBK);
+  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kQM;  // first weight row
+  const int64_t m0 = static_cast<int64_t>(blockIdx.y) * TN;   // first token
+  const int nk = static_cast<int>(a.K / kQK);
   const int64_t G = a.K >> 7;
 
   pdl_allow_dependents();
-
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kPRingL; ++i) {
-      mbar_init(&fullL[i], 1);
-      mbar_init(&emptyA[i], 1);
-      mbar_init(&emptyP[i], kPDecThreads);
+    for (int i = 0; i < kQRing; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&emptyX[i], 1);
+      mbar_init(&emptyP[i], 4);
     }
-    for (int i = 0; i < kPRingB; ++i) {
-      mbar_init(&fullB[i], kPDecThreads);
-      mbar_init(&emptyB[i], 1);
+    for (int i = 0; i < kQARing; ++i) {
+      mbar_init(&afull[i], 4);
+      mbar_init(&aempty[i], 1);
     }
     mbar_init(accFull, 1);
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kPTmemCols);
+    tmem_alloc(tmem_slot, L::kTmemCols);
     tmem_relinquish();
-  }
-  if (warp >= 4) {
-    const int r = threadIdx.x - 128;
-    const int64_t n = n0 + r;
-    sScale[r] = (!kInt4 && n < a.N) ? __half2float(a.sc[n]) : 0.0f;
-    sBias[r] = (a.bias && n < a.N) ? __half2float(a.bias[n]) : 0.0f;
   }
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
-  const uint32_t tmem_d = *tmem_slot;
+  const uint32_t tmem = *tmem_slot;
 
   bool ok = true;
   if (warp == 0) {
@@ -175,15 +170,15 @@ __global__ void __launch_bounds__(kPThreads, 1)
       tma_prefetch_desc(&tmap_x);
       tma_prefetch_desc(&tmap_w);
       for (int kb = 0; kb < nk && ok; ++kb) {
-        const int s = kb % kPRingL;
-        if (kb >= kPRingL) {
-          const uint32_t par = static_cast<uint32_t>((kb / kPRingL) - 1) & 1u;
-          ok = mbar_wait(&emptyA[s], par) && mbar_wait(&emptyP[s], par);
+        const int s = kb % kQRing;
+        if (kb >= kQRing) {
+          const uint32_t par = static_cast<uint32_t>((kb / kQRing) - 1) & 1u;
+          ok = mbar_wait(&emptyX[s], par) && mbar_wait(&emptyP[s], par);
           if (!ok) break;
         }
-        mbar_arrive_expect_tx(&fullL[s], kPTileA + F::kTileP);
-        tma_load_2d(sm + L::kOffA + s * kPTileA, &tmap_x, &fullL[s], kb * kPBK, static_cast<int32_t>(m0));
-        tma_load_2d(sm + L::kOffP + s * F::kTileP, &tmap_w, &fullL[s], kb * F::kRowBytes,
+        mbar_arrive_expect_tx(&full[s], L::kTileX + F::kTileP);
+        tma_load_2d(sm + L::kOffX + s * L::kTileX, &tmap_x, &full[s], kb * kQK, static_cast<int32_t>(m0));
+        tma_load_2d(sm + L::kOffP + s * F::kTileP, &tmap_w, &full[s], kb * F::kRowBytes,
                     static_cast<int32_t>(n0));
       }
     }
@@ -191,96 +186,108 @@ __global__ void __launch_bounds__(kPThreads, 1)
     // ------------------------------------------------------------------ MMA issuer
     pdl_wait_prior_grids();  // x arrives only after the previous kernel: block, do not poll
     if (lane == 0) {
-      const uint32_t idesc = idesc_f16_f32(kPBM, kPBN);
-      const uint32_t a_base = smem_u32(sm + L::kOffA), b_base = smem_u32(sm + L::kOffB);
+      const uint32_t idesc = idesc_f16_f32(kQM, TN);
+      const uint32_t x_base = smem_u32(sm + L::kOffX);
       for (int kb = 0; kb < nk && ok; ++kb) {
-        const int s = kb % kPRingL, b = kb % kPRingB;
-        ok = mbar_wait(&fullL[s], static_cast<uint32_t>(kb / kPRingL) & 1u) &&
-             mbar_wait(&fullB[b], static_cast<uint32_t>(kb / kPRingB) & 1u);
+        const int s = kb % kQRing, as = kb % kQARing;
+        ok = mbar_wait(&full[s], static_cast<uint32_t>(kb / kQRing) & 1u) &&
+             mbar_wait(&afull[as], static_cast<uint32_t>(kb / kQARing) & 1u);
         if (!ok) break;
         tc_fence_after_sync();
-        const uint64_t adesc = sdesc_kmajor_sw128(a_base + s * kPTileA);
-        const uint64_t bdesc = sdesc_kmajor_sw128(b_base + b * kPTileB);
+        const uint64_t bdesc = sdesc_kmajor_sw128(x_base + s * L::kTileX);
+        const uint32_t a_tmem = tmem + L::kColA + 32 * as;
 #pragma unroll
-        for (int k16 = 0; k16 < kPBK / 16; ++k16) {
-          // +32 bytes along K inside the swizzle atom = +2 in the encoded start address
-          umma_f16(tmem_d, adesc + 2 * k16, bdesc + 2 * k16, idesc, (kb | k16) != 0 ? 1u : 0u);
+        for (int k16 = 0; k16 < kQK / 16; ++k16) {
+          // A: 8 columns (16 fp16) per K=16 step; B: +32 bytes along K = +2 in the descriptor
+          umma_f16_ts(tmem, a_tmem + 8 * k16, bdesc + 2 * k16, idesc, (kb | k16) != 0 ? 1u : 0u);
         }
-        umma_commit(&emptyA[s]);
-        umma_commit(&emptyB[b]);
+        umma_commit(&emptyX[s]);
+        umma_commit(&aempty[as]);
       }
       if (ok) umma_commit(accFull);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------------ decode warps
-    const int r = threadIdx.x - 128;  // weight row within the tile
+    const int r = threadIdx.x - 128;  // weight row within the tile = TMEM lane
     const int64_t n = n0 + r;
-    uint8_t* brow_base = sm + L::kOffB + (r >> 3) * 1024 + (r & 7) * 128;
-    const int sw = r & 7;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp - 4) * 32) << 16);
+    float ep_s = 1.0f, ep_b = 0.0f;  // epilogue scale / bias of this row (constants)
+    if (n < a.N) {
+      if (!kInt4) ep_s = __half2float(a.sc[n]);
+      if (a.bias) ep_b = __half2float(a.bias[n]);
+    }
     for (int kb = 0; kb < nk && ok; ++kb) {
-      const int s = kb % kPRingL, b = kb % kPRingB;
-      ok = mbar_wait(&fullL[s], static_cast<uint32_t>(kb / kPRingL) & 1u);
+      const int s = kb % kQRing, as = kb % kQARing;
+      ok = mbar_wait(&full[s], static_cast<uint32_t>(kb / kQRing) & 1u);
       if (!ok) break;
       const uint8_t* prow = sm + L::kOffP + s * F::kTileP + r * F::kRowBytes;
-      uint4 p0 = *reinterpret_cast<const uint4*>(prow);
+      const uint4 p0 = *reinterpret_cast<const uint4*>(prow);
       uint4 p1 = make_uint4(0u, 0u, 0u, 0u);
       if (kInt4) p1 = *reinterpret_cast<const uint4*>(prow + 16);
-      mbar_arrive(&emptyP[s]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&emptyP[s]);
       uint32_t s2 = 0u;
       if (kInt4) {
         const uint16_t sb = (n < a.N) ? __half_as_ushort(a.sc[n * G + (kb >> 1)]) : static_cast<uint16_t>(0);
         s2 = static_cast<uint32_t>(sb) | (static_cast<uint32_t>(sb) << 16);
       }
-      if (kb >= kPRingB) {
-        ok = mbar_wait(&emptyB[b], static_cast<uint32_t>((kb / kPRingB) - 1) & 1u);
-        if (!ok) break;
-      }
-      uint8_t* brow = brow_base + b * kPTileB;
       const uint32_t pw[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+      uint32_t v[32];  // column j = fp16 pair (k = 2j, 2j + 1) of this row
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const uint4 v = kInt4 ? decode_w4_8(pw[j], s2) : decode_tq_8(pw[j >> 1], j & 1);
-        *reinterpret_cast<uint4*>(brow + ((j ^ sw) << 4)) = v;
+        const uint4 d = kInt4 ? decode_w4_8(pw[j], s2) : decode_tq_8(pw[j >> 1], j & 1);
+        v[4 * j] = d.x;
+        v[4 * j + 1] = d.y;
+        v[4 * j + 2] = d.z;
+        v[4 * j + 3] = d.w;
       }
-      fence_proxy_async_smem();
-      mbar_arrive(&fullB[b]);
+      if (kb >= kQARing) {
+        ok = mbar_wait(&aempty[as], static_cast<uint32_t>((kb / kQARing) - 1) & 1u);
+        if (!ok) break;
+        tc_fence_after_sync();
+      }
+      tmem_st_32x32b_x32(lane_base + L::kColA + 32 * as, v);
+      tmem_st_wait();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&afull[as]);
     }
-  }
 
-  // -------------------------------------------------------------------- epilogue (warps 0-3)
-  if (warp < 4) {
-    if (warp != 0) pdl_wait_prior_grids();
-    __syncwarp();
-    const bool acc_ok = mbar_wait(accFull, 0u);
+    // ---------------------------------------------------------------- epilogue (same warps)
+    pdl_wait_prior_grids();  // y may still be read by the previous kernel
+    const bool acc_ok = ok && mbar_wait(accFull, 0u);
     tc_fence_after_sync();
-    const int64_t m = m0 + warp * 32 + lane;
-    const uint32_t taddr = tmem_d + (static_cast<uint32_t>(warp * 32) << 16);
-    if (acc_ok) {
-      const bool vec = ((a.N & 7) == 0);
+    __half* stage = reinterpret_cast<__half*>(sm + L::kOffX);  // [32 tokens][128 rows]
+    const int et = threadIdx.x - 128;                           // 0..127
+    const bool vec = (a.N & 7) == 0;
 #pragma unroll 1
-      for (int c = 0; c < kPBN / 32; ++c) {
-        uint32_t rr[32];
-        tmem_ld_32x32b_x32(taddr + c * 32, rr);
-        tmem_ld_wait();
-        if (m < a.M) {
-          const int64_t nb = n0 + c * 32;
-          __align__(16) __half o[32];
+    for (int c = 0; c < TN / 32 && acc_ok; ++c) {
+      uint32_t rr[32];
+      tmem_ld_32x32b_x32(lane_base + c * 32, rr);
+      tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float v = __uint_as_float(rr[j]);
-            const float yv = kInt4 ? (v + sBias[c * 32 + j]) : fmaf(v, sScale[c * 32 + j], sBias[c * 32 + j]);
-            o[j] = __float2half_rn(yv);
-          }
+      for (int j = 0; j < 32; ++j) {
+        const float v = __uint_as_float(rr[j]);
+        stage[j * kQM + r] = __float2half_rn(kInt4 ? v + ep_b : fmaf(v, ep_s, ep_b));
+      }
+      named_barrier_sync(1, 128);
+      // 32 tokens x 128 rows: 16 chunks of 16 bytes per token, four per thread
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int idx = et + 128 * q, tok = idx >> 4, ch = idx & 15;
+        const int64_t m = m0 + c * 32 + tok, nb = n0 + ch * 8;
+        if (m < a.M && nb < a.N) {
+          const uint4 val = *reinterpret_cast<const uint4*>(stage + tok * kQM + ch * 8);
           __half* dst = a.y + m * a.N + nb;
-          if (vec && nb + 32 <= a.N) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) reinterpret_cast<uint4*>(dst)[q] = reinterpret_cast<const uint4*>(o)[q];
+          if (vec && nb + 8 <= a.N) {
+            *reinterpret_cast<uint4*>(dst) = val;
           } else {
-            for (int j = 0; j < 32; ++j)
-              if (nb + j < a.N) dst[j] = o[j];
+            const __half* hv = reinterpret_cast<const __half*>(&val);
+            for (int e = 0; e < 8 && nb + e < a.N; ++e) dst[e] = hv[e];
           }
         }
       }
+      named_barrier_sync(1, 128);
     }
   }
 
@@ -288,34 +295,34 @@ __global__ void __launch_bounds__(kPThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem_d, kPTmemCols);
+    tmem_dealloc(tmem, L::kTmemCols);
   }
 }
 
 bool prefill_supported(bool int4, int64_t M, int64_t N, int64_t K) {
   if (M < 1 || N < 1) return false;
-  if (K < kPBK) return false;
+  if (K < kQK) return false;
   if (int4 ? (K % 128 != 0) : (K % 64 != 0)) return false;
-  if ((M + kPBM - 1) / kPBM > 65535) return false;
+  if ((M + 127) / 128 > 65535) return false;
   return true;
 }
 
-template <bool kInt4>
-static cudaError_t launch_prefill(const __half* x, const void* w, const __half* sc,
-                                  const __half* bias, __half* y, int64_t M, int64_t N, int64_t K,
-                                  cudaStream_t s) {
-  using L = PrefillLayout<kInt4>;
+template <bool kInt4, int TN>
+static cudaError_t launch_prefill_t(const __half* x, const void* w, const __half* sc,
+                                    const __half* bias, __half* y, int64_t M, int64_t N, int64_t K,
+                                    cudaStream_t s) {
+  using L = PrefillLayout<kInt4, TN>;
   using F = PFmt<kInt4>;
   CUtensorMap tx, tw;
   if (!make_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, static_cast<uint64_t>(K),
-                    static_cast<uint64_t>(M), static_cast<uint64_t>(K) * 2, kPBK, kPBM,
+                    static_cast<uint64_t>(M), static_cast<uint64_t>(K) * 2, kQK, TN,
                     CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   const uint64_t kbytes = kInt4 ? static_cast<uint64_t>(K) / 2 : static_cast<uint64_t>(K) / 4;
   if (!make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w, kbytes, static_cast<uint64_t>(N), kbytes,
-                    F::kRowBytes, kPBN, CU_TENSOR_MAP_SWIZZLE_NONE))
+                    F::kRowBytes, kQM, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
-  auto* kern = prefill_gemm_kernel<kInt4>;
+  auto* kern = prefill_gemm_kernel<kInt4, TN>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), L::kAlloc);
   if (e != cudaSuccess) return e;
   PrefillArgs a;
@@ -326,8 +333,8 @@ static cudaError_t launch_prefill(const __half* x, const void* w, const __half* 
   a.N = N;
   a.K = K;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>((N + kPBN - 1) / kPBN), static_cast<unsigned>((M + kPBM - 1) / kPBM), 1);
-  cfg.blockDim = dim3(kPThreads, 1, 1);
+  cfg.gridDim = dim3(static_cast<unsigned>((N + kQM - 1) / kQM), static_cast<unsigned>((M + TN - 1) / TN), 1);
+  cfg.blockDim = dim3(kQThreads, 1, 1);
   cfg.dynamicSmemBytes = L::kAlloc;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -336,6 +343,17 @@ static cudaError_t launch_prefill(const __half* x, const void* w, const __half* 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, tx, tw, a);
+}
+
+// 256 tokens per CTA (each x tile then feeds twice the MMA work) unless that leaves SMs idle.
+template <bool kInt4>
+static cudaError_t launch_prefill(const __half* x, const void* w, const __half* sc,
+                                  const __half* bias, __half* y, int64_t M, int64_t N, int64_t K,
+                                  cudaStream_t s) {
+  const DeviceInfo di = current_device_info();
+  const int64_t tiles256 = ((N + kQM - 1) / kQM) * ((M + 255) / 256);
+  if (tiles256 >= di.num_sms) return launch_prefill_t<kInt4, 256>(x, w, sc, bias, y, M, N, K, s);
+  return launch_prefill_t<kInt4, 128>(x, w, sc, bias, y, M, N, K, s);
 }
 
 cudaError_t launch_tq_gemm_prefill(const __half* x, const uint8_t* packed, const __half* scale,
