@@ -460,28 +460,70 @@ def secondary_rows(args, rank, layers, peaks):
     rows["w4g_prefill_M4096"] = {"value": round(tf, 1), "unit": "TFLOP/s", "frac": round(tf / tc, 4),
                                  "peak": tc, "bound": "tensor", "sample": "1 layer x 7 shapes, M=4096"}
     del g, w4
-    # ---- pack throughput (config 4): Qwen2-7B fp16 weights, 2 layers x 4 shapes
+    # ---- config 0: one ternary linear 1024x1024 at M = 1 (L2-resident: the time of one call)
+    w = I.weights(1024, 1024, I.seed_for(0, 0, 0), device="cuda")
+    p0, s0 = tq.tq_quantize_pack(w)
+    del w
+    x0 = I.activations(1, 1024, I.seed_for(0, 0, 0), device="cuda")
+    y0 = torch.empty(1, 1024, dtype=torch.float16, device="cuda")
+    g = capture(lambda: [tq.tq_gemm(x0, p0, s0, None, y0) for _ in range(32)])
+    ms = time_graph(g, 20) / 32
+    rows["config0_decode_1024x1024_M1"] = {"value": round(ms * 1e3, 2), "unit": "us/call",
+                                           "sample": "32 calls in a CUDA graph; weights L2-resident (256 KiB), "
+                                                     "so no roofline fraction"}
+    del g
+    # ---- config 4: Qwen2-7B, 28 layers x {qkv 4608x3584, o 3584x3584, gate_up 37888x3584,
+    # down 3584x18944}: tq_quantize_pack of all fp16 weights (13.05 GB read), then the M sweep
     qshapes = [(4608, 3584), (3584, 3584), (37888, 3584), (3584, 18944)]
-    tot_ms, tot_b = 0.0, 0
-    for l in range(2):
-        for mid, (N, K) in enumerate(qshapes):
-            w = I.weights(N, K, I.seed_for(4, l, mid), device="cuda", dtype=torch.float16)
-            p = torch.empty(N, K // 4, dtype=torch.uint8, device="cuda")
-            s = torch.empty(N, dtype=torch.float16, device="cuda")
-            tq.tq_quantize_pack(w, p, s)
-            torch.cuda.synchronize()
-            a, b = torch.cuda.Event(True), torch.cuda.Event(True)
-            a.record()
-            for _ in range(3):
-                tq.tq_quantize_pack(w, p, s)
-            b.record()
-            torch.cuda.synchronize()
-            tot_ms += a.elapsed_time(b) / 3
-            tot_b += N * K * 2 + N * K // 4 + 2 * N
-            del w, p, s
-    gbs = tot_b / (tot_ms * 1e-3) / 1e9
+    nl = 28
+    wq = [[I.weights(N, K, I.seed_for(4, l, mid) + rank_seed_offset(rank), device="cuda", dtype=torch.float16)
+           for mid, (N, K) in enumerate(qshapes)] for l in range(nl)]
+    pq = [[(torch.empty(N, K // 4, dtype=torch.uint8, device="cuda"), torch.empty(N, dtype=torch.float16, device="cuda"))
+           for (N, K) in qshapes] for _ in range(nl)]
+
+    def pack_all():
+        for l in range(nl):
+            for mid in range(len(qshapes)):
+                tq.tq_quantize_pack(wq[l][mid], pq[l][mid][0], pq[l][mid][1])
+
+    pack_all()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(True), torch.cuda.Event(True)
+    a.record()
+    pack_all()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    byts = nl * sum(N * K * 2 + N * K // 4 + 2 * N for N, K in qshapes)
+    gbs = byts / (ms * 1e-3) / 1e9
     rows["tq_quantize_pack_qwen2_fp16"] = {"value": round(gbs, 1), "unit": "GB/s", "frac": round(gbs / hbm, 4),
-                                           "peak": hbm, "bound": "hbm", "sample": "2 Qwen2-7B layers x 4 shapes"}
+                                           "peak": hbm, "bound": "hbm", "ms": round(ms, 3),
+                                           "sample": f"all {nl} Qwen2-7B layers x 4 shapes, fp16 in "
+                                                     f"({byts / 1e9:.2f} GB moved), inputs larger than L2"}
+    del wq
+    sweep = {}
+    for M in (1, 2, 8, 32, 128, 512, 2048, 8192):
+        xk = {K: I.activations(M, K, I.seed_for(4, 99, M) + K, device="cuda") for K in (3584, 18944)}
+        yn = {N: torch.empty(M, N, dtype=torch.float16, device="cuda") for N, _ in qshapes}
+
+        def qs():
+            for l in range(nl):
+                for mid, (N, K) in enumerate(qshapes):
+                    tq.tq_gemm(xk[K], pq[l][mid][0], pq[l][mid][1], None, yn[N])
+
+        g = capture(qs)
+        ms = time_graph(g, 10 if M <= 128 else 2)
+        byts = nl * sum(decode_bytes(M, N, K) for N, K in qshapes)
+        flops = nl * sum(2 * M * N * K for N, K in qshapes)
+        t_att = max(byts / (hbm * 1e9), flops / (tc * 1e12)) * 1e3  # ms at the attainable roofline
+        ent = {"ms": round(ms, 4), "GB/s": round(byts / (ms * 1e-3) / 1e9, 1),
+               "TFLOP/s": round(flops / (ms * 1e-3) / 1e12, 1), "attainable_frac": round(t_att / ms, 4),
+               "path": "decode" if tq.tq_select_path(0, M, 3584, 3584, 1) == tq.PATH_DECODE else "prefill"}
+        sweep[f"M{M}"] = ent
+        del g, xk, yn
+    rows["qwen2_sweep_28_layers"] = {"unit": "per M: ms for 28 layers x 4 shapes; attainable_frac = "
+                                             "max(bytes / HBM, flops / fp16 peak) / time", "values": sweep}
+    del pq
     torch.cuda.synchronize()
     return rows
 
@@ -575,6 +617,7 @@ PROFILE_CASES = {
     "decode": "ternary gate_proj 14336x4096 at M=1, 3 launches; q/k/v group (4096+1024+1024)x4096 at M=16, 3 launches",
     "prefill": "ternary q_proj 4096x4096 at M=2048 (1 % outlier rows), 3 launches; W4A16 gate_proj 14336x4096 at M=512, 3 launches",
     "pack": "tq_quantize_pack of an fp16 Qwen2-7B gate_up 37888x3584 (2 launches) and an fp32 4096x4096 (2 launches); w4g_quantize_pack of the latter (2 launches)",
+    "prefill_mid": "ternary Qwen2-7B down 3584x18944 at M=128, 3 launches; gate_up 37888x3584 at M=32, 3 launches",
 }
 
 
@@ -608,6 +651,19 @@ def run_profile_case(name):
         x = I.activations(512, 4096, 6, device="cuda")
         for _ in range(3):
             tq.w4g_gemm(x, q, sc)
+    elif name == "prefill_mid":
+        w = I.weights(3584, 18944, 1, device="cuda")
+        p, s = tq.tq_quantize_pack(w)
+        del w
+        x = I.activations(128, 18944, 2, device="cuda")
+        for _ in range(3):
+            tq.tq_gemm(x, p, s)
+        w = I.weights(37888, 3584, 3, device="cuda")
+        p2, s2 = tq.tq_quantize_pack(w)
+        del w
+        x2 = I.activations(32, 3584, 4, device="cuda")
+        for _ in range(3):
+            tq.tq_gemm(x2, p2, s2)
     elif name == "pack":
         w = I.weights(37888, 3584, 1, device="cuda", dtype=torch.float16)
         for _ in range(2):

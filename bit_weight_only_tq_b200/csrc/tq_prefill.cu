@@ -9,8 +9,9 @@
 // One CTA = 128 weight rows (the TMEM lanes, UMMA M) x TN tokens (UMMA N = 256, or 128 for
 // small M):
 //   * warp 0, one lane: TMA loads of the x tile (TN tokens x 64 k, fp16, 128-byte swizzle, the
-//     K-major layout the UMMA descriptor expects) and of the packed weight tile (128 rows x 16
-//     bytes ternary / 32 bytes W4A16) into a ring;
+//     K-major layout the UMMA descriptor expects) into a ring; warp 2, one lane: TMA loads of the
+//     packed weights, 128 rows x 128 bytes per tile (8 ternary / 4 W4A16 stages, 128-byte
+//     swizzle) into a ring of three;
 //   * warp 1: allocates the tensor memory (accumulator + a ring of decoded-weight slots); one
 //     lane issues tcgen05.mma (M=128, N=TN, K=16, A from tensor memory) and commits to
 //     mbarriers that free the input stages;
@@ -40,32 +41,49 @@ namespace tq {
 
 constexpr int kQM = 128;         // weight rows per CTA (UMMA M, TMEM lanes)
 constexpr int kQK = 64;          // K per stage: one 128-byte swizzle row of fp16
-constexpr int kQRing = 4;        // stages of (x tile, packed tile)
-constexpr int kQARing = 4;       // tensor-memory slots of decoded weights (32 columns each)
+constexpr int kQMaxRing = 12;    // stages of (x tile, packed tile), at most
+constexpr int kQMaxARing = 8;    // tensor-memory slots of decoded weights (32 columns each)
 constexpr int kQThreads = 256;   // warp 0 TMA, warp 1 MMA, warps 4-7 decode + epilogue
 
 template <bool kInt4>
 struct PFmt {
-  static constexpr int kRowBytes = kInt4 ? 32 : 16;  // packed bytes per row per stage
-  static constexpr int kTileP = kQM * kRowBytes;
+  static constexpr int kRowBytes = kInt4 ? 32 : 16;  // packed bytes per row per stage (64 k)
+  // the packed weights arrive in tiles of 128 bytes per row (8 ternary / 4 W4A16 stages),
+  // 128-byte swizzled: one DRAM burst per row instead of one 16- or 32-byte piece per stage
+  static constexpr int kSPP = 128 / kRowBytes;       // stages per packed tile
+  static constexpr int kTileP = kQM * 128;
+  static constexpr int kPRing = 3;
 };
 
 template <bool kInt4, int TN>
 struct PrefillLayout {
   static constexpr int kTileX = TN * kQK * 2;  // x tile of one stage
+  // ring depths: narrow tiles move little data per stage, so they keep more stages in flight
+  static constexpr int kRing = TN == 256 ? 4 : (TN == 128 ? 6 : 10);
+  static constexpr int kARing = TN == 256 ? 4 : kQMaxARing;
+  // split-K partials [S][128 rows][TN / S] fp32 reuse the x ring after the main loop
   static constexpr int kOffX = 0;
-  static constexpr int kOffP = kOffX + kQRing * kTileX;
-  static constexpr int kOffBar = kOffP + kQRing * PFmt<kInt4>::kTileP;
-  // barriers: full[R], emptyX[R], emptyP[R], afull[RA], aempty[RA], accFull; then the TMEM slot
-  static constexpr int kNumBars = 3 * kQRing + 2 * kQARing + 1;
+  static constexpr int kOffP = kOffX + kRing * kTileX;
+  static constexpr int kOffBar = kOffP + PFmt<kInt4>::kPRing * PFmt<kInt4>::kTileP;
+  // barriers: fullX[R], emptyX[R], fullP[RP], emptyP[RP], afull[RA], aempty[RA], accFull; then
+  // the TMEM slot
+  static constexpr int kNumBars = 2 * kRing + 2 * PFmt<kInt4>::kPRing + 2 * kARing + 1;
   static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffTmemSlot + 16;
-  static constexpr int kAlloc = kBytes + 1024;  // alignment slack
+  // alignment slack; at least 116 KB so that one CTA runs per SM: a CTA never waits in
+  // tcgen05.alloc for tensor memory held by another CTA (which may itself wait at a cluster
+  // barrier for a CTA that waits for tensor memory)
+  static constexpr int kAlloc = kBytes + 1024 > 116 * 1024 ? kBytes + 1024 : 116 * 1024;
+  // partials with a padded row pitch (TN / S + 1 floats: conflict-free) in the freed x and
+  // packed rings
+  static_assert(kQM * (TN + 8) * 4 <= kRing * kTileX + PFmt<kInt4>::kPRing * PFmt<kInt4>::kTileP,
+                "split-K partials fit");
   // tensor memory: accumulator columns [0, TN), decoded-weight slots after it
   static constexpr uint32_t kColA = TN;
-  static constexpr uint32_t kTmemCols = TN + 32 * kQARing <= 256 ? 256u : 512u;
+  static constexpr uint32_t kTmemCols = TN + 32 * kARing <= 256 ? 256u : 512u;
   // epilogue staging (reuses the x ring): 32 tokens x 128 rows fp16
-  static_assert(32 * kQM * 2 <= kQRing * kTileX, "staging fits in the x ring");
+  static_assert(32 * kQM * 2 <= kRing * kTileX, "staging fits in the x ring");
+  static_assert(kRing <= kQMaxRing && kARing <= kQMaxARing && TN + 32 * kARing <= 512, "rings");
 };
 
 struct PrefillArgs {
@@ -73,6 +91,7 @@ struct PrefillArgs {
   const __half* bias;  // may be null
   __half* y;
   int64_t M, N, K;
+  int S;               // K-slices: CTAs per cluster (grid z), reduced through DSMEM
 };
 
 __device__ __forceinline__ uint32_t hsub2_u32(uint32_t a, uint32_t b) {
@@ -125,28 +144,35 @@ __global__ void __launch_bounds__(kQThreads, 1)
   // space visible to the compiler (plain ld/st.shared instead of generic accesses)
   uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kOffBar);
-  uint64_t* full = bars;                     // x tile + packed tile landed (TMA)
-  uint64_t* emptyX = bars + kQRing;          // x tile consumed (MMA commit)
-  uint64_t* emptyP = bars + 2 * kQRing;      // packed tile consumed (decode warps)
-  uint64_t* afull = bars + 3 * kQRing;       // decoded weights in tensor memory
-  uint64_t* aempty = afull + kQARing;        // ... consumed (MMA commit)
-  uint64_t* accFull = aempty + kQARing;
+  uint64_t* full = bars;                       // x tile landed (TMA)
+  uint64_t* emptyX = bars + L::kRing;          // x tile consumed (MMA commit)
+  uint64_t* fullP = bars + 2 * L::kRing;       // packed tile landed (TMA)
+  uint64_t* emptyP = fullP + F::kPRing;        // packed tile consumed (decode warps)
+  uint64_t* afull = emptyP + F::kPRing;        // decoded weights in tensor memory
+  uint64_t* aempty = afull + L::kARing;        // ... consumed (MMA commit)
+  uint64_t* accFull = aempty + L::kARing;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::kOffTmemSlot);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kQM;  // first weight row
   const int64_t m0 = static_cast<int64_t>(blockIdx.y) * TN;   // first token
-  const int nk = static_cast<int>(a.K / kQK);
+  const int nk_all = static_cast<int>(a.K / kQK);
+  const int rank = static_cast<int>(blockIdx.z);              // K-slice = rank in the cluster
+  const int kb0 = static_cast<int>((static_cast<int64_t>(rank) * nk_all) / a.S);
+  const int nk = static_cast<int>((static_cast<int64_t>(rank + 1) * nk_all) / a.S) - kb0;  // >= 1
   const int64_t G = a.K >> 7;
 
   pdl_allow_dependents();
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kQRing; ++i) {
+    for (int i = 0; i < L::kRing; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&emptyX[i], 1);
+    }
+    for (int i = 0; i < F::kPRing; ++i) {
+      mbar_init(&fullP[i], 1);
       mbar_init(&emptyP[i], 4);
     }
-    for (int i = 0; i < kQARing; ++i) {
+    for (int i = 0; i < L::kARing; ++i) {
       mbar_init(&afull[i], 4);
       mbar_init(&aempty[i], 1);
     }
@@ -164,21 +190,34 @@ __global__ void __launch_bounds__(kQThreads, 1)
 
   bool ok = true;
   if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------------ TMA producer: x
     pdl_wait_prior_grids();
     if (lane == 0) {
       tma_prefetch_desc(&tmap_x);
-      tma_prefetch_desc(&tmap_w);
       for (int kb = 0; kb < nk && ok; ++kb) {
-        const int s = kb % kQRing;
-        if (kb >= kQRing) {
-          const uint32_t par = static_cast<uint32_t>((kb / kQRing) - 1) & 1u;
-          ok = mbar_wait(&emptyX[s], par) && mbar_wait(&emptyP[s], par);
+        const int s = kb % L::kRing;
+        if (kb >= L::kRing) {
+          ok = mbar_wait(&emptyX[s], static_cast<uint32_t>((kb / L::kRing) - 1) & 1u);
           if (!ok) break;
         }
-        mbar_arrive_expect_tx(&full[s], L::kTileX + F::kTileP);
-        tma_load_2d(sm + L::kOffX + s * L::kTileX, &tmap_x, &full[s], kb * kQK, static_cast<int32_t>(m0));
-        tma_load_2d(sm + L::kOffP + s * F::kTileP, &tmap_w, &full[s], kb * F::kRowBytes,
+        mbar_arrive_expect_tx(&full[s], L::kTileX);
+        tma_load_2d(sm + L::kOffX + s * L::kTileX, &tmap_x, &full[s], (kb0 + kb) * kQK, static_cast<int32_t>(m0));
+      }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------------ TMA producer: weights
+    // (model constants: issued before the wait for the previous kernel)
+    if (lane == 0) {
+      tma_prefetch_desc(&tmap_w);
+      const int npt = (nk + F::kSPP - 1) / F::kSPP;
+      for (int pt = 0; pt < npt && ok; ++pt) {
+        const int s = pt % F::kPRing;
+        if (pt >= F::kPRing) {
+          ok = mbar_wait(&emptyP[s], static_cast<uint32_t>((pt / F::kPRing) - 1) & 1u);
+          if (!ok) break;
+        }
+        mbar_arrive_expect_tx(&fullP[s], F::kTileP);
+        tma_load_2d(sm + L::kOffP + s * F::kTileP, &tmap_w, &fullP[s], (kb0 + pt * F::kSPP) * F::kRowBytes,
                     static_cast<int32_t>(n0));
       }
     }
@@ -189,9 +228,9 @@ __global__ void __launch_bounds__(kQThreads, 1)
       const uint32_t idesc = idesc_f16_f32(kQM, TN);
       const uint32_t x_base = smem_u32(sm + L::kOffX);
       for (int kb = 0; kb < nk && ok; ++kb) {
-        const int s = kb % kQRing, as = kb % kQARing;
-        ok = mbar_wait(&full[s], static_cast<uint32_t>(kb / kQRing) & 1u) &&
-             mbar_wait(&afull[as], static_cast<uint32_t>(kb / kQARing) & 1u);
+        const int s = kb % L::kRing, as = kb % L::kARing;
+        ok = mbar_wait(&full[s], static_cast<uint32_t>(kb / L::kRing) & 1u) &&
+             mbar_wait(&afull[as], static_cast<uint32_t>(kb / L::kARing) & 1u);
         if (!ok) break;
         tc_fence_after_sync();
         const uint64_t bdesc = sdesc_kmajor_sw128(x_base + s * L::kTileX);
@@ -217,18 +256,25 @@ __global__ void __launch_bounds__(kQThreads, 1)
       if (a.bias) ep_b = __half2float(a.bias[n]);
     }
     for (int kb = 0; kb < nk && ok; ++kb) {
-      const int s = kb % kQRing, as = kb % kQARing;
-      ok = mbar_wait(&full[s], static_cast<uint32_t>(kb / kQRing) & 1u);
-      if (!ok) break;
-      const uint8_t* prow = sm + L::kOffP + s * F::kTileP + r * F::kRowBytes;
-      const uint4 p0 = *reinterpret_cast<const uint4*>(prow);
+      const int as = kb % L::kARing, pt = kb / F::kSPP, ci = kb - pt * F::kSPP, ps = pt % F::kPRing;
+      if (ci == 0) {
+        ok = mbar_wait(&fullP[ps], static_cast<uint32_t>(pt / F::kPRing) & 1u);
+        if (!ok) break;
+      }
+      // this stage's 16 (ternary) or 32 (W4A16) bytes of row r: 16-byte chunk(s) of the
+      // 128-byte swizzled row (chunk c at position c ^ (r & 7): conflict free)
+      const uint8_t* prow = sm + L::kOffP + ps * F::kTileP + r * 128;
+      const int c0 = kInt4 ? 2 * ci : ci;
+      const uint4 p0 = *reinterpret_cast<const uint4*>(prow + ((c0 ^ (r & 7)) << 4));
       uint4 p1 = make_uint4(0u, 0u, 0u, 0u);
-      if (kInt4) p1 = *reinterpret_cast<const uint4*>(prow + 16);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&emptyP[s]);
+      if (kInt4) p1 = *reinterpret_cast<const uint4*>(prow + (((c0 + 1) ^ (r & 7)) << 4));
+      if (ci == F::kSPP - 1 || kb == nk - 1) {  // done with this packed tile
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&emptyP[ps]);
+      }
       uint32_t s2 = 0u;
       if (kInt4) {
-        const uint16_t sb = (n < a.N) ? __half_as_ushort(a.sc[n * G + (kb >> 1)]) : static_cast<uint16_t>(0);
+        const uint16_t sb = (n < a.N) ? __half_as_ushort(a.sc[n * G + ((kb0 + kb) >> 1)]) : static_cast<uint16_t>(0);
         s2 = static_cast<uint32_t>(sb) | (static_cast<uint32_t>(sb) << 16);
       }
       const uint32_t pw[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
@@ -241,8 +287,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
         v[4 * j + 2] = d.z;
         v[4 * j + 3] = d.w;
       }
-      if (kb >= kQARing) {
-        ok = mbar_wait(&aempty[as], static_cast<uint32_t>((kb / kQARing) - 1) & 1u);
+      if (kb >= L::kARing) {
+        ok = mbar_wait(&aempty[as], static_cast<uint32_t>((kb / L::kARing) - 1) & 1u);
         if (!ok) break;
         tc_fence_after_sync();
       }
@@ -257,38 +303,79 @@ __global__ void __launch_bounds__(kQThreads, 1)
     pdl_wait_prior_grids();  // y may still be read by the previous kernel
     const bool acc_ok = ok && mbar_wait(accFull, 0u);
     tc_fence_after_sync();
-    __half* stage = reinterpret_cast<__half*>(sm + L::kOffX);  // [32 tokens][128 rows]
-    const int et = threadIdx.x - 128;                           // 0..127
     const bool vec = (a.N & 7) == 0;
+    if (a.S == 1) {
+      __half* stage = reinterpret_cast<__half*>(sm + L::kOffX);  // [32 tokens][128 rows]
+      const int et = threadIdx.x - 128;                           // 0..127
 #pragma unroll 1
-    for (int c = 0; c < TN / 32 && acc_ok; ++c) {
-      uint32_t rr[32];
-      tmem_ld_32x32b_x32(lane_base + c * 32, rr);
-      tmem_ld_wait();
+      for (int c = 0; c < TN / 32 && acc_ok; ++c) {
+        uint32_t rr[32];
+        tmem_ld_32x32b_x32(lane_base + c * 32, rr);
+        tmem_ld_wait();
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const float v = __uint_as_float(rr[j]);
-        stage[j * kQM + r] = __float2half_rn(kInt4 ? v + ep_b : fmaf(v, ep_s, ep_b));
-      }
-      named_barrier_sync(1, 128);
-      // 32 tokens x 128 rows: 16 chunks of 16 bytes per token, four per thread
+        for (int j = 0; j < 32; ++j) {
+          const float v = __uint_as_float(rr[j]);
+          stage[j * kQM + r] = __float2half_rn(kInt4 ? v + ep_b : fmaf(v, ep_s, ep_b));
+        }
+        named_barrier_sync(1, 128);
+        // 32 tokens x 128 rows: 16 chunks of 16 bytes per token, four per thread
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int idx = et + 128 * q, tok = idx >> 4, ch = idx & 15;
-        const int64_t m = m0 + c * 32 + tok, nb = n0 + ch * 8;
-        if (m < a.M && nb < a.N) {
-          const uint4 val = *reinterpret_cast<const uint4*>(stage + tok * kQM + ch * 8);
-          __half* dst = a.y + m * a.N + nb;
-          if (vec && nb + 8 <= a.N) {
-            *reinterpret_cast<uint4*>(dst) = val;
-          } else {
-            const __half* hv = reinterpret_cast<const __half*>(&val);
-            for (int e = 0; e < 8 && nb + e < a.N; ++e) dst[e] = hv[e];
+        for (int q = 0; q < 4; ++q) {
+          const int idx = et + 128 * q, tok = idx >> 4, ch = idx & 15;
+          const int64_t m = m0 + c * 32 + tok, nb = n0 + ch * 8;
+          if (m < a.M && nb < a.N) {
+            const uint4 val = *reinterpret_cast<const uint4*>(stage + tok * kQM + ch * 8);
+            __half* dst = a.y + m * a.N + nb;
+            if (vec && nb + 8 <= a.N) {
+              *reinterpret_cast<uint4*>(dst) = val;
+            } else {
+              const __half* hv = reinterpret_cast<const __half*>(&val);
+              for (int e = 0; e < 8 && nb + e < a.N; ++e) dst[e] = hv[e];
+            }
           }
         }
+        named_barrier_sync(1, 128);
       }
-      named_barrier_sync(1, 128);
+    } else {
+      // split K: the tokens of the tile are split evenly over the S CTAs of the cluster; each
+      // CTA sends its partial sums of the other CTAs' tokens into their shared memory
+      // ([source rank][row][token], row pitch tpo + 1, in the freed x and packed rings) and
+      // adds the S partials of its own tokens in rank order (deterministic).
+      const int tpo = TN / a.S;  // tokens owned by each CTA
+      const int pitch = tpo + 1;
+      float* red = reinterpret_cast<float*>(sm + L::kOffX);
+      const uint32_t red_local = smem_u32(red);
+      cluster_sync_all();  // every CTA of the cluster is past its main loop: the x rings are free
+#pragma unroll 1
+      for (int c = 0; c < TN / 32; ++c) {
+        uint32_t rr[32];
+        if (acc_ok) {
+          tmem_ld_32x32b_x32(lane_base + c * 32, rr);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) rr[j] = 0u;
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int tok = c * 32 + j, q = tok / tpo;
+          const uint32_t off = ((rank * kQM + r) * pitch + (tok - q * tpo)) * 4;
+          st_shared_cluster_f32(mapa_shared(red_local + off, static_cast<uint32_t>(q)), __uint_as_float(rr[j]));
+        }
+      }
+      cluster_sync_all();  // all partials have landed
+      for (int j = 0; j < tpo; ++j) {
+        float v = 0.0f;
+        for (int src = 0; src < a.S; ++src) v += red[(src * kQM + r) * pitch + j];
+        const int64_t m = m0 + rank * tpo + j;
+        if (m < a.M && n < a.N) a.y[m * a.N + n] = __float2half_rn(kInt4 ? v + ep_b : fmaf(v, ep_s, ep_b));
+      }
     }
+  }
+  if (warp < 4 && a.S > 1) {
+    // every thread of the cluster takes part in the two barriers of the split-K epilogue
+    cluster_sync_all();
+    cluster_sync_all();
   }
 
   tc_fence_before_sync();
@@ -310,7 +397,7 @@ bool prefill_supported(bool int4, int64_t M, int64_t N, int64_t K) {
 template <bool kInt4, int TN>
 static cudaError_t launch_prefill_t(const __half* x, const void* w, const __half* sc,
                                     const __half* bias, __half* y, int64_t M, int64_t N, int64_t K,
-                                    cudaStream_t s) {
+                                    int S, cudaStream_t s) {
   using L = PrefillLayout<kInt4, TN>;
   using F = PFmt<kInt4>;
   CUtensorMap tx, tw;
@@ -320,7 +407,7 @@ static cudaError_t launch_prefill_t(const __half* x, const void* w, const __half
     return cudaErrorInvalidValue;
   const uint64_t kbytes = kInt4 ? static_cast<uint64_t>(K) / 2 : static_cast<uint64_t>(K) / 4;
   if (!make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w, kbytes, static_cast<uint64_t>(N), kbytes,
-                    F::kRowBytes, kQM, CU_TENSOR_MAP_SWIZZLE_NONE))
+                    128, kQM, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   auto* kern = prefill_gemm_kernel<kInt4, TN>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), L::kAlloc);
@@ -332,28 +419,47 @@ static cudaError_t launch_prefill_t(const __half* x, const void* w, const __half
   a.M = M;
   a.N = N;
   a.K = K;
+  a.S = S;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>((N + kQM - 1) / kQM), static_cast<unsigned>((M + TN - 1) / TN), 1);
+  cfg.gridDim = dim3(static_cast<unsigned>((N + kQM - 1) / kQM), static_cast<unsigned>((M + TN - 1) / TN),
+                     static_cast<unsigned>(S));
   cfg.blockDim = dim3(kQThreads, 1, 1);
   cfg.dynamicSmemBytes = L::kAlloc;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  int na = 1;
+  if (S > 1) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 1;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = static_cast<unsigned>(S);
+    na = 2;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = na;
   return cudaLaunchKernelEx(&cfg, kern, tx, tw, a);
 }
 
-// 256 tokens per CTA (each x tile then feeds twice the MMA work) unless that leaves SMs idle.
+// Tile choice: 64 tokens for M <= 64 (an N < 64 MMA costs as much as N = 64), 256 when those
+// tiles alone fill the GPU (each decoded weight then feeds the most MMAs), else 128 (as
+// efficient per MMA as 256); K split over a cluster of S CTAs (1, 2, 4 or 8) while the tiles
+// alone leave SMs idle.
 template <bool kInt4>
 static cudaError_t launch_prefill(const __half* x, const void* w, const __half* sc,
                                   const __half* bias, __half* y, int64_t M, int64_t N, int64_t K,
                                   cudaStream_t s) {
   const DeviceInfo di = current_device_info();
-  const int64_t tiles256 = ((N + kQM - 1) / kQM) * ((M + 255) / 256);
-  if (tiles256 >= di.num_sms) return launch_prefill_t<kInt4, 256>(x, w, sc, bias, y, M, N, K, s);
-  return launch_prefill_t<kInt4, 128>(x, w, sc, bias, y, M, N, K, s);
+  const int64_t rt = (N + kQM - 1) / kQM;
+  const int nk = static_cast<int>(K / kQK);
+  const int TN = M <= 64 ? 64 : ((M <= 128 || rt * ((M + 255) / 256) < di.num_sms) ? 128 : 256);
+  const int64_t base = rt * ((M + TN - 1) / TN);
+  int S = 1;
+  while (S < 8 && base * S * 2 <= di.num_sms && S * 2 <= nk) S *= 2;
+  if (TN == 64) return launch_prefill_t<kInt4, 64>(x, w, sc, bias, y, M, N, K, S, s);
+  if (TN == 128) return launch_prefill_t<kInt4, 128>(x, w, sc, bias, y, M, N, K, S, s);
+  return launch_prefill_t<kInt4, 256>(x, w, sc, bias, y, M, N, K, S, s);
 }
 
 cudaError_t launch_tq_gemm_prefill(const __half* x, const uint8_t* packed, const __half* scale,

@@ -136,3 +136,16 @@ def test_decode_m_gt_8_layouts(M, N, K):
     xw, qw, sc, bw = _w4_problem(M, N, K, 800 + M)
     yw = tq.w4g_gemm(xw, qw, sc, bw, path=tq.PATH_DECODE)
     check_w4g_gemm(xw, qw, sc, bw, yw, cols=np.arange(0, N, 7), label=f"w4g decode M={M} {N}x{K}")
+
+
+# Mid-M prefill: narrow token tiles and K split over a cluster (S = 2..8 CTAs, uneven K slices),
+# reduced through distributed shared memory.
+@pytest.mark.parametrize("M,N,K", [(40, 384, 1088), (100, 1000, 1152), (64, 3584, 3584), (130, 4608, 3584)])
+def test_prefill_split_k(M, N, K):
+    need_cuda()
+    x, p, s, b = _tq_problem(M, N, K, 900 + M)
+    y = tq.tq_gemm(x, p, s, b, path=tq.PATH_PREFILL)
+    check_tq_gemm(x, p, s, b, y, cols=np.arange(0, N, 3), label=f"tq prefill split-K M={M} {N}x{K}")
+    xw, qw, sc, bw = _w4_problem(M, N, K // 128 * 128, 950 + M)
+    yw = tq.w4g_gemm(xw, qw, sc, bw, path=tq.PATH_PREFILL)
+    check_w4g_gemm(xw, qw, sc, bw, yw, cols=np.arange(0, N, 3), label=f"w4g prefill split-K M={M} {N}x{K}")
