@@ -523,9 +523,48 @@ def secondary_rows(args, rank, layers, peaks):
         del g, xk, yn
     rows["qwen2_sweep_28_layers"] = {"unit": "per M: ms for 28 layers x 4 shapes; attainable_frac = "
                                              "max(bytes / HBM, flops / fp16 peak) / time", "values": sweep}
+    rows["dispatch_crossover_qwen2"] = dispatch_crossover(tq, I, pq[:8], qshapes)
     del pq
     torch.cuda.synchronize()
     return rows
+
+
+def dispatch_crossover(tq, I, pq, qshapes):
+    """Both GEMM paths forced at M around the ridge, on Qwen2-7B shapes (ternary: the given
+    packed layers; W4A16: four layers packed here), to place the automatic decode/prefill
+    switch by measurement."""
+    import torch
+
+    nl = len(pq)
+    p4 = []
+    for l in range(4):
+        row = []
+        for mid, (N, K) in enumerate(qshapes):
+            w = I.weights(N, K, I.seed_for(4, 50 + l, mid), device="cuda", outlier_frac=0.001)
+            row.append(tq.w4g_quantize_pack(w))
+            del w
+        p4.append(row)
+    out = {"unit": "ms per pass (ternary: %d layers, W4A16: 4 layers) x 4 shapes" % nl, "values": {}}
+    for M in (16, 24, 32, 40, 48, 64):
+        xk = {K: I.activations(M, K, I.seed_for(4, 98, M) + K, device="cuda") for K in (3584, 18944)}
+        yn = {N: torch.empty(M, N, dtype=torch.float16, device="cuda") for N, _ in qshapes}
+        ent = {}
+        for fmt, layers, fn in (("ternary", pq, tq.tq_gemm), ("w4g", p4, tq.w4g_gemm)):
+            for name, path in (("decode", tq.PATH_DECODE), ("prefill", tq.PATH_PREFILL)):
+                def run():
+                    for lay in layers:
+                        for mid, (N, K) in enumerate(qshapes):
+                            fn(xk[K], lay[mid][0], lay[mid][1], None, yn[N], path=path)
+
+                g = capture(run)
+                ent[f"{fmt}_{name}_ms"] = round(time_graph(g, 10), 4)
+                del g
+            fcode = 0 if fmt == "ternary" else 1
+            ent[f"{fmt}_auto"] = "decode" if tq.tq_select_path(fcode, M, 3584, 3584, 1) == tq.PATH_DECODE else "prefill"
+        out["values"][f"M{M}"] = ent
+        del xk, yn
+    del p4
+    return out
 
 
 def load_traffic():

@@ -156,7 +156,8 @@ static int gemm_grouped_impl(const uint16_t* x, int count, const WT* const* w,
   if (!w || !sc || !y || !N) return TQ_ERR_NULL;
   if (M < 0 || K <= 0 || K > (int64_t(1) << 28) || M > (int64_t(1) << 31)) return TQ_ERR_SHAPE;
   if (kInt4 && K % 128 != 0) return TQ_ERR_SHAPE;
-  bool all_decode = M >= 1 && M <= 16 && x && aligned16(x);
+  bool all_decode = M >= 1 && M <= (kInt4 ? tq::kDecodeAutoMaxM_W4g : tq::kDecodeAutoMaxM_Ternary) && x &&
+                    aligned16(x);
   for (int g = 0; g < count; ++g) {
     if (N[g] < 0 || N[g] > (int64_t(1) << 31)) return TQ_ERR_SHAPE;
     if (M > 0 && N[g] > 0 && (!w[g] || !sc[g] || !y[g])) return TQ_ERR_NULL;
@@ -207,11 +208,11 @@ int tq_select_path(int fmt, int64_t M, int64_t N, int64_t K, int aligned) {
   if (M < 0 || N < 0 || K <= 0) return TQ_ERR_SHAPE;
   if (int4 && K % 128 != 0) return TQ_ERR_SHAPE;
   if (M == 0 || N == 0 || !aligned) return TQ_PATH_GENERIC;
-  // Ridge of the fp16 tensor-core roofline: the decode kernel streams weights at HBM speed and
-  // wins for skinny M; the tensor-core prefill kernel takes over above 16 tokens.
-  if (M <= 16 && tq::decode_ok(int4, M, N, K)) return TQ_PATH_DECODE;
+  // Around the ridge of the fp16 tensor-core roofline the faster path was picked by measurement:
+  // the decode kernel for skinny M, the tensor-core prefill kernel above the crossover.
+  const int64_t dmax = int4 ? tq::kDecodeAutoMaxM_W4g : tq::kDecodeAutoMaxM_Ternary;
+  if (M <= dmax && tq::decode_ok(int4, M, N, K)) return TQ_PATH_DECODE;
   if (tq::prefill_supported(int4, M, N, K)) return TQ_PATH_PREFILL;
-  if (M <= 16) return TQ_PATH_GENERIC;
   return TQ_PATH_GENERIC;
 }
 

@@ -189,6 +189,12 @@ cudaError_t launch_w4g_gemm_generic(const __half* x, const int32_t* qweight, con
                                     int64_t K, cudaStream_t s);
 cudaError_t launch_tq_validate(const uint8_t* packed, int64_t N, int64_t K, int* bad,
                                cudaStream_t s);
+// Decode (skinny) path: at most 16 tokens per CTA; larger M runs token chunks of 16 over grid z.
+constexpr int64_t kDecodeMaxM = 64;
+// Largest M the automatic dispatch sends to the decode path, per format (the measured crossover
+// with the tensor-core path on Llama-3-8B and Qwen2-7B shaped linears).
+constexpr int64_t kDecodeAutoMaxM_Ternary = 48;
+constexpr int64_t kDecodeAutoMaxM_W4g = 16;
 cudaError_t launch_tq_gemm_decode(const __half* x, const uint8_t* packed, const __half* scale,
                                   const __half* bias, __half* y, int64_t M, int64_t N, int64_t K,
                                   cudaStream_t s);

@@ -1,4 +1,8 @@
-// tq_decode.cu -- memory-bound skinny GEMM (M <= 16) for ternary and W4A16 weights.
+// tq_decode.cu -- memory-bound skinny GEMM (M <= 64) for ternary and W4A16 weights.
+//
+// A CTA computes at most 16 tokens; 17 <= M <= 64 runs ceil(M / 16) token chunks over grid z
+// in the same launch (the chunks of a row block stream the same weights at about the same time,
+// so all but the first mostly read them from L2).
 //
 // [TQ] §1: decode time is spent fetching weights, so the kernel is built around the HBM stream
 // of packed codes; [TQ] §4.2: codes are decoded into fp16 tensor-core fragments, accumulated in
@@ -75,6 +79,7 @@ constexpr int kDMaxGroup = 4;  // weight matrices sharing x in one launch (e.g. 
 
 struct DecodeArgs {
   int64_t M, K;
+  int Mbox;       // tokens per CTA: M, or 16 when M > 16 (grid z = token chunks of 16)
   int C;          // stages along K
   int S;          // CTAs per cluster (K-slices)
   int ring;       // stages resident in shared memory
@@ -162,12 +167,16 @@ __device__ __forceinline__ void decode_gemm_body(const DecodeMaps& maps, const D
   const int64_t Nm = a.N[grp];
   const __half* scm = a.sc[grp];
   const __half* biasm = a.bias[grp];
-  __half* ym = a.y[grp];
+  __half* ym = a.y[grp] + static_cast<int64_t>(blockIdx.z) * 16 * a.N[grp];
   const int st_begin = static_cast<int>((static_cast<int64_t>(rank) * a.C) / a.S);
   const int st_end = static_cast<int>((static_cast<int64_t>(rank + 1) * a.C) / a.S);
   const int nst = st_end - st_begin;
   const int own_cap = (F::kRows + a.S - 1) / a.S;  // row slots per owner in `red`
-  const int Mi = static_cast<int>(a.M);
+  // token chunk of this CTA (M > 16 runs ceil(M / 16) chunks of 16 tokens over grid z: the CTAs
+  // of one row block read the same weights at about the same time, so the chunks after the
+  // first mostly hit L2)
+  const int64_t tok0 = static_cast<int64_t>(blockIdx.z) * 16;
+  const int Mi = static_cast<int>(a.M - tok0 < a.Mbox ? a.M - tok0 : a.Mbox);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < a.ring; ++i) {
@@ -194,7 +203,7 @@ __device__ __forceinline__ void decode_gemm_body(const DecodeMaps& maps, const D
 
   if (warp == W::kCons) {
     // ================================================================== producer warp
-    const uint32_t tx = static_cast<uint32_t>(kDWBytes + F::kKB * Mi * 128);
+    const uint32_t tx = static_cast<uint32_t>(kDWBytes + F::kKB * a.Mbox * 128);  // whole boxes
     auto load_w = [&](int i) {
       tma_load_2d(stg + (i % a.ring) * a.stage, tmap, &full[i % a.ring], (st_begin + i) * 128,
                   static_cast<int>(row0));
@@ -203,7 +212,8 @@ __device__ __forceinline__ void decode_gemm_body(const DecodeMaps& maps, const D
       uint8_t* dst = stg + (i % a.ring) * a.stage + kDWBytes;
 #pragma unroll
       for (int hb = 0; hb < F::kKB / 4; ++hb)
-        tma_load_3d(dst + hb * a.xhalf, &maps.x, &full[i % a.ring], 0, (st_begin + i) * F::kKB + 4 * hb, 0);
+        tma_load_3d(dst + hb * a.xhalf, &maps.x, &full[i % a.ring], 0, (st_begin + i) * F::kKB + 4 * hb,
+                    static_cast<int32_t>(tok0));
     };
     const int pre = nst < a.ring ? nst : a.ring;
     if (lane == 0) {
@@ -554,9 +564,9 @@ struct DecodePlan {
   int S, C, ring, stage, xhalf, smem;
 };
 
-// Stage ring and cluster size for RB row blocks of one launch.
+// Stage ring and cluster size for RB row blocks x `chunks` token chunks of M tokens each.
 template <bool kInt4>
-static bool plan_decode_t(int64_t RB, int64_t M, int64_t K, int num_sms, DecodePlan* p) {
+static bool plan_decode_t(int64_t RB, int64_t M, int64_t K, int num_sms, DecodePlan* p, int64_t chunks) {
   using F = DecFmt<kInt4>;
   using L = DecLayout<kInt4>;
   const int C = static_cast<int>((K + F::kStageK - 1) / F::kStageK);
@@ -570,7 +580,7 @@ static bool plan_decode_t(int64_t RB, int64_t M, int64_t K, int num_sms, DecodeP
   const int smem = L::bytes(ring, stage);
   if (smem > kDSmemBudget) return false;
   // one wave of two CTAs per SM, at most 8 K-slices per row block
-  int64_t S = (2 * static_cast<int64_t>(num_sms)) / RB;
+  int64_t S = (2 * static_cast<int64_t>(num_sms)) / (RB * chunks);
   if (S < 1) S = 1;
   if (S > kDMaxCluster) S = kDMaxCluster;
   if (S > C) S = C;
@@ -578,8 +588,9 @@ static bool plan_decode_t(int64_t RB, int64_t M, int64_t K, int num_sms, DecodeP
   return true;
 }
 
-static bool plan_decode(bool int4, int64_t RB, int64_t M, int64_t K, int num_sms, DecodePlan* p) {
-  return int4 ? plan_decode_t<true>(RB, M, K, num_sms, p) : plan_decode_t<false>(RB, M, K, num_sms, p);
+static bool plan_decode(bool int4, int64_t RB, int64_t M, int64_t K, int num_sms, DecodePlan* p,
+                        int64_t chunks = 1) {
+  return int4 ? plan_decode_t<true>(RB, M, K, num_sms, p, chunks) : plan_decode_t<false>(RB, M, K, num_sms, p, chunks);
 }
 
 template <bool kInt4, int NT, int TW>
@@ -590,7 +601,8 @@ static cudaError_t launch_decode_t(const DecodeMaps& maps, const DecodeArgs& a, 
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), kDSmemBudget);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(p.S), static_cast<unsigned>(a.rb_start[a.count]), 1);
+  cfg.gridDim = dim3(static_cast<unsigned>(p.S), static_cast<unsigned>(a.rb_start[a.count]),
+                     static_cast<unsigned>((a.M + 15) / 16));
   cfg.blockDim = dim3(DecWarps<NT, TW>::kThreads, 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(p.smem);
   cfg.stream = s;
@@ -620,10 +632,13 @@ static cudaError_t launch_decode_group(const __half* x, int count, const void* c
   using F = DecFmt<kInt4>;
   if (count < 1 || count > kDMaxGroup) return cudaErrorInvalidValue;
   const DeviceInfo di = current_device_info();
-  const int NT = M > 8 ? 2 : 1;
+  const int64_t Mbox = M > 16 ? 16 : M;
+  const int64_t chunks = (M + 15) / 16;
+  const int NT = Mbox > 8 ? 2 : 1;
   DecodeArgs a = {};
   DecodeMaps maps;
   a.M = M;
+  a.Mbox = static_cast<int>(Mbox);
   a.K = K;
   a.count = count;
   int64_t rbs = 0;
@@ -641,10 +656,10 @@ static cudaError_t launch_decode_group(const __half* x, int count, const void* c
       return cudaErrorInvalidValue;
   }
   for (int g = count; g < kDMaxGroup; ++g) maps.m[g] = maps.m[0];
-  {  // activations viewed as [M][K/64][64]: one box = four 64-element blocks x all M tokens
+  {  // activations viewed as [M][K/64][64]: one box = four 64-element blocks x Mbox tokens
     const uint64_t dims[3] = {64, static_cast<uint64_t>(K / 64), static_cast<uint64_t>(M)};
     const uint64_t strides[2] = {128, static_cast<uint64_t>(K) * 2};
-    const uint32_t box[3] = {64, 4, static_cast<uint32_t>(M)};
+    const uint32_t box[3] = {64, 4, static_cast<uint32_t>(Mbox)};
     if (!make_tmap_3d(&maps.x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, dims, strides, box,
                       CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
@@ -652,7 +667,7 @@ static cudaError_t launch_decode_group(const __half* x, int count, const void* c
   a.rb_start[count] = static_cast<int>(rbs);
   if (rbs > 65535) return cudaErrorInvalidValue;
   DecodePlan p;
-  if (!plan_decode(kInt4, rbs, M, K, di.num_sms, &p)) return cudaErrorInvalidValue;
+  if (!plan_decode(kInt4, rbs, Mbox, K, di.num_sms, &p, chunks)) return cudaErrorInvalidValue;
   a.C = p.C;
   a.S = p.S;
   a.ring = p.ring;
@@ -660,16 +675,16 @@ static cudaError_t launch_decode_group(const __half* x, int count, const void* c
   a.xhalf = p.xhalf;
   if (NT == 1) return launch_decode_t<kInt4, 1, 1>(maps, a, p, s);
   // a CTA with a single stage and two CTAs per SM: more, lighter warps hide the latency better
-  const bool single = (p.C + p.S - 1) / p.S <= 1 && static_cast<int64_t>(p.S) * rbs > di.num_sms;
+  const bool single = (p.C + p.S - 1) / p.S <= 1 && static_cast<int64_t>(p.S) * rbs * chunks > di.num_sms;
   return single ? launch_decode_t<kInt4, 2, 1>(maps, a, p, s) : launch_decode_t<kInt4, 2, 2>(maps, a, p, s);
 }
 
 bool decode_supported(bool int4, int64_t M, int64_t N, int64_t K) {
-  if (M < 1 || M > 16 || N < 1) return false;
+  if (M < 1 || M > kDecodeMaxM || N < 1) return false;
   if (int4 ? (K % 128 != 0) : (K % 64 != 0)) return false;
   DecodePlan p;
   const int64_t rows = int4 ? DecFmt<true>::kRows : DecFmt<false>::kRows;
-  return plan_decode(int4, (N + rows - 1) / rows, M, K, 148, &p);
+  return plan_decode(int4, (N + rows - 1) / rows, M > 16 ? 16 : M, K, 148, &p, (M + 15) / 16);
 }
 
 cudaError_t launch_tq_gemm_decode(const __half* x, const uint8_t* packed, const __half* scale,

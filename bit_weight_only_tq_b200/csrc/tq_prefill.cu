@@ -55,16 +55,21 @@ struct PFmt {
   static constexpr int kPRing = 3;
 };
 
-template <bool kInt4, int TN>
+// kSS: the decoded weights go to shared memory (128-byte-swizzled K-major tiles, the layout TMA
+// gives the x tile) and the MMA reads both operands from there; otherwise they go to tensor
+// memory.
+template <bool kInt4, int TN, bool kSS>
 struct PrefillLayout {
   static constexpr int kTileX = TN * kQK * 2;  // x tile of one stage
+  static constexpr int kTileA = kQM * kQK * 2;  // decoded-weight tile of one stage (kSS)
   // ring depths: narrow tiles move little data per stage, so they keep more stages in flight
-  static constexpr int kRing = TN == 256 ? 4 : (TN == 128 ? 6 : 10);
-  static constexpr int kARing = TN == 256 ? 4 : kQMaxARing;
+  static constexpr int kRing = kSS ? (TN == 64 ? 8 : 4) : (TN == 256 ? 4 : (TN == 128 ? 6 : 10));
+  static constexpr int kARing = kSS ? 4 : (TN == 256 ? 4 : kQMaxARing);
   // split-K partials [S][128 rows][TN / S] fp32 reuse the x ring after the main loop
   static constexpr int kOffX = 0;
   static constexpr int kOffP = kOffX + kRing * kTileX;
-  static constexpr int kOffBar = kOffP + PFmt<kInt4>::kPRing * PFmt<kInt4>::kTileP;
+  static constexpr int kOffA = kOffP + PFmt<kInt4>::kPRing * PFmt<kInt4>::kTileP;
+  static constexpr int kOffBar = kOffA + (kSS ? kARing * kTileA : 0);
   // barriers: fullX[R], emptyX[R], fullP[RP], emptyP[RP], afull[RA], aempty[RA], accFull; then
   // the TMEM slot
   static constexpr int kNumBars = 2 * kRing + 2 * PFmt<kInt4>::kPRing + 2 * kARing + 1;
@@ -78,12 +83,13 @@ struct PrefillLayout {
   // packed rings
   static_assert(kQM * (TN + 8) * 4 <= kRing * kTileX + PFmt<kInt4>::kPRing * PFmt<kInt4>::kTileP,
                 "split-K partials fit");
-  // tensor memory: accumulator columns [0, TN), decoded-weight slots after it
+  // tensor memory: accumulator columns [0, TN), decoded-weight slots after it (not kSS)
   static constexpr uint32_t kColA = TN;
-  static constexpr uint32_t kTmemCols = TN + 32 * kARing <= 256 ? 256u : 512u;
+  static constexpr uint32_t kTmemCols = kSS ? static_cast<uint32_t>(TN) : (TN + 32 * kARing <= 256 ? 256u : 512u);
   // epilogue staging (reuses the x ring): 32 tokens x 128 rows fp16
   static_assert(32 * kQM * 2 <= kRing * kTileX, "staging fits in the x ring");
-  static_assert(kRing <= kQMaxRing && kARing <= kQMaxARing && TN + 32 * kARing <= 512, "rings");
+  static_assert(kRing <= kQMaxRing && kARing <= kQMaxARing && (kSS || TN + 32 * kARing <= 512), "rings");
+  static_assert(kAlloc <= 227 * 1024, "shared memory");
 };
 
 struct PrefillArgs {
@@ -133,11 +139,11 @@ __device__ __forceinline__ uint4 decode_w4_8(uint32_t w, uint32_t s2) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-template <bool kInt4, int TN>
+template <bool kInt4, int TN, bool kSS>
 __global__ void __launch_bounds__(kQThreads, 1)
     prefill_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
                         const __grid_constant__ CUtensorMap tmap_w, const PrefillArgs a) {
-  using L = PrefillLayout<kInt4, TN>;
+  using L = PrefillLayout<kInt4, TN, kSS>;
   using F = PFmt<kInt4>;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned; pointer arithmetic on the __shared__ array keeps the shared address
@@ -227,6 +233,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
     if (lane == 0) {
       const uint32_t idesc = idesc_f16_f32(kQM, TN);
       const uint32_t x_base = smem_u32(sm + L::kOffX);
+      const uint32_t a_base = smem_u32(sm + L::kOffA);
       for (int kb = 0; kb < nk && ok; ++kb) {
         const int s = kb % L::kRing, as = kb % L::kARing;
         ok = mbar_wait(&full[s], static_cast<uint32_t>(kb / L::kRing) & 1u) &&
@@ -235,10 +242,15 @@ __global__ void __launch_bounds__(kQThreads, 1)
         tc_fence_after_sync();
         const uint64_t bdesc = sdesc_kmajor_sw128(x_base + s * L::kTileX);
         const uint32_t a_tmem = tmem + L::kColA + 32 * as;
+        const uint64_t adesc = sdesc_kmajor_sw128(a_base + as * L::kTileA);
 #pragma unroll
         for (int k16 = 0; k16 < kQK / 16; ++k16) {
-          // A: 8 columns (16 fp16) per K=16 step; B: +32 bytes along K = +2 in the descriptor
-          umma_f16_ts(tmem, a_tmem + 8 * k16, bdesc + 2 * k16, idesc, (kb | k16) != 0 ? 1u : 0u);
+          // A in tensor memory: 8 columns (16 fp16) per K=16 step; in shared memory (and B):
+          // +32 bytes along K = +2 in the descriptor
+          if (kSS)
+            umma_f16(tmem, adesc + 2 * k16, bdesc + 2 * k16, idesc, (kb | k16) != 0 ? 1u : 0u);
+          else
+            umma_f16_ts(tmem, a_tmem + 8 * k16, bdesc + 2 * k16, idesc, (kb | k16) != 0 ? 1u : 0u);
         }
         umma_commit(&emptyX[s]);
         umma_commit(&aempty[as]);
@@ -278,23 +290,39 @@ __global__ void __launch_bounds__(kQThreads, 1)
         s2 = static_cast<uint32_t>(sb) | (static_cast<uint32_t>(sb) << 16);
       }
       const uint32_t pw[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-      uint32_t v[32];  // column j = fp16 pair (k = 2j, 2j + 1) of this row
+      if (kSS) {
+        if (kb >= L::kARing) {
+          ok = mbar_wait(&aempty[as], static_cast<uint32_t>((kb / L::kARing) - 1) & 1u);
+          if (!ok) break;
+        }
+        // 16-byte chunk j (k = 8j .. 8j + 7) of row r at chunk position j ^ (r & 7) of the
+        // 128-byte row: the 128-byte swizzle; eight consecutive rows fill all 32 banks
+        uint8_t* arow = sm + L::kOffA + as * L::kTileA + r * 128;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint4 d = kInt4 ? decode_w4_8(pw[j], s2) : decode_tq_8(pw[j >> 1], j & 1);
-        v[4 * j] = d.x;
-        v[4 * j + 1] = d.y;
-        v[4 * j + 2] = d.z;
-        v[4 * j + 3] = d.w;
+        for (int j = 0; j < 8; ++j) {
+          const uint4 d = kInt4 ? decode_w4_8(pw[j], s2) : decode_tq_8(pw[j >> 1], j & 1);
+          *reinterpret_cast<uint4*>(arow + ((j ^ (r & 7)) << 4)) = d;
+        }
+        fence_proxy_async_smem();  // visible to the tensor core's operand reads
+      } else {
+        uint32_t v[32];  // column j = fp16 pair (k = 2j, 2j + 1) of this row
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint4 d = kInt4 ? decode_w4_8(pw[j], s2) : decode_tq_8(pw[j >> 1], j & 1);
+          v[4 * j] = d.x;
+          v[4 * j + 1] = d.y;
+          v[4 * j + 2] = d.z;
+          v[4 * j + 3] = d.w;
+        }
+        if (kb >= L::kARing) {
+          ok = mbar_wait(&aempty[as], static_cast<uint32_t>((kb / L::kARing) - 1) & 1u);
+          if (!ok) break;
+          tc_fence_after_sync();
+        }
+        tmem_st_32x32b_x32(lane_base + L::kColA + 32 * as, v);
+        tmem_st_wait();
+        tc_fence_before_sync();
       }
-      if (kb >= L::kARing) {
-        ok = mbar_wait(&aempty[as], static_cast<uint32_t>((kb / L::kARing) - 1) & 1u);
-        if (!ok) break;
-        tc_fence_after_sync();
-      }
-      tmem_st_32x32b_x32(lane_base + L::kColA + 32 * as, v);
-      tmem_st_wait();
-      tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&afull[as]);
     }
@@ -394,12 +422,11 @@ bool prefill_supported(bool int4, int64_t M, int64_t N, int64_t K) {
   return true;
 }
 
-template <bool kInt4, int TN>
+template <bool kInt4, int TN, bool kSS>
 static cudaError_t launch_prefill_t(const __half* x, const void* w, const __half* sc,
                                     const __half* bias, __half* y, int64_t M, int64_t N, int64_t K,
                                     int S, cudaStream_t s) {
-  using L = PrefillLayout<kInt4, TN>;
-  using F = PFmt<kInt4>;
+  using L = PrefillLayout<kInt4, TN, kSS>;
   CUtensorMap tx, tw;
   if (!make_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, static_cast<uint64_t>(K),
                     static_cast<uint64_t>(M), static_cast<uint64_t>(K) * 2, kQK, TN,
@@ -409,7 +436,7 @@ static cudaError_t launch_prefill_t(const __half* x, const void* w, const __half
   if (!make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w, kbytes, static_cast<uint64_t>(N), kbytes,
                     128, kQM, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  auto* kern = prefill_gemm_kernel<kInt4, TN>;
+  auto* kern = prefill_gemm_kernel<kInt4, TN, kSS>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), L::kAlloc);
   if (e != cudaSuccess) return e;
   PrefillArgs a;
@@ -446,6 +473,8 @@ static cudaError_t launch_prefill_t(const __half* x, const void* w, const __half
 // tiles alone fill the GPU (each decoded weight then feeds the most MMAs), else 128 (as
 // efficient per MMA as 256); K split over a cluster of S CTAs (1, 2, 4 or 8) while the tiles
 // alone leave SMs idle.
+constexpr int kPrefillSSMaxTN = 128;  // token tiles up to this width read A from shared memory
+
 template <bool kInt4>
 static cudaError_t launch_prefill(const __half* x, const void* w, const __half* sc,
                                   const __half* bias, __half* y, int64_t M, int64_t N, int64_t K,
@@ -457,9 +486,9 @@ static cudaError_t launch_prefill(const __half* x, const void* w, const __half* 
   const int64_t base = rt * ((M + TN - 1) / TN);
   int S = 1;
   while (S < 8 && base * S * 2 <= di.num_sms && S * 2 <= nk) S *= 2;
-  if (TN == 64) return launch_prefill_t<kInt4, 64>(x, w, sc, bias, y, M, N, K, S, s);
-  if (TN == 128) return launch_prefill_t<kInt4, 128>(x, w, sc, bias, y, M, N, K, S, s);
-  return launch_prefill_t<kInt4, 256>(x, w, sc, bias, y, M, N, K, S, s);
+  if (TN == 64) return launch_prefill_t<kInt4, 64, kPrefillSSMaxTN >= 64>(x, w, sc, bias, y, M, N, K, S, s);
+  if (TN == 128) return launch_prefill_t<kInt4, 128, kPrefillSSMaxTN >= 128>(x, w, sc, bias, y, M, N, K, S, s);
+  return launch_prefill_t<kInt4, 256, false>(x, w, sc, bias, y, M, N, K, S, s);
 }
 
 cudaError_t launch_tq_gemm_prefill(const __half* x, const uint8_t* packed, const __half* scale,

@@ -68,10 +68,13 @@ typedef enum {
 
 typedef enum { TQ_F32 = 0, TQ_F16 = 1 } tq_dtype;
 
-/* GEMM execution paths.  AUTO applies tq_select_path(); the others force one path (tests). */
+/* GEMM execution paths.  AUTO applies tq_select_path(); the others force one path (tests).
+ * The decode path runs at most 16 tokens per CTA; 17 <= M <= 64 runs ceil(M/16) token chunks
+ * in the same launch.  tq_select_path picks decode up to the crossover measured on Llama-3-8B /
+ * Qwen2-7B shaped linears (ternary M <= 48, W4A16 M <= 16) and the tensor-core path above. */
 typedef enum {
     TQ_PATH_AUTO = 0,
-    TQ_PATH_DECODE = 1,  /* memory-bound skinny path, M <= 16: mma.sync on in-register decode  */
+    TQ_PATH_DECODE = 1,  /* memory-bound skinny path, M <= 64: mma.sync on in-register decode  */
     TQ_PATH_PREFILL = 2, /* tensor-core path: TMA + smem decode + tcgen05.mma into TMEM         */
     TQ_PATH_GENERIC = 3  /* any shape / alignment: CUDA-core kernel (correct, not fast)         */
 } tq_path;
@@ -108,7 +111,7 @@ TQ_API int tq_quantize_pack(const void* w, int w_dtype, uint8_t* packed, uint16_
  *   scale   [N] fp16, device.                bias    [N] fp16 or NULL.
  *   y       [M,N] fp16, device, written.  x and y must not overlap.
  * Codes 0b11 are invalid; the output for a row holding one is unspecified (tq_validate_packed
- * finds them).  tq_gemm_ex forces a path: DECODE needs M <= 16, K % 64 == 0 and 16-byte aligned
+ * finds them).  tq_gemm_ex forces a path: DECODE needs M <= 64, K % 64 == 0 and 16-byte aligned
  * x / packed; PREFILL needs K % 64 == 0 and 16-byte aligned x / packed / y; otherwise
  * TQ_ERR_PATH (shape) or TQ_ERR_ALIGN (pointers).  GENERIC takes any shape.
  * ------------------------------------------------------------------------------------------ */
@@ -136,7 +139,7 @@ TQ_API int w4g_quantize_pack(const void* w, int w_dtype, int32_t* qweight, uint1
 
 /* w4g_gemm -- y = x . What^T (+ bias), What = scales[n,k/128] * (u - 8) ([VQ] §5 forward:
  * INT4 weight x fp16 activation -> fp16 output).  Shapes as tq_gemm with K % 128 == 0.
- * DECODE needs M <= 16 and 16-byte aligned x / qweight; PREFILL needs 16-byte aligned pointers. */
+ * DECODE needs M <= 64 and 16-byte aligned x / qweight; PREFILL needs 16-byte aligned pointers. */
 TQ_API int w4g_gemm(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
              const uint16_t* bias, uint16_t* y, int64_t M, int64_t N, int64_t K, void* stream);
 TQ_API int w4g_gemm_ex(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
@@ -148,8 +151,9 @@ TQ_API int w4g_gemm_ex(const uint16_t* x, const int32_t* qweight, const uint16_t
  * engine's fused q/k/v or gate/up projections do: for g < count,
  *     y_g[M, N_g] = x[M, K] . What_g[N_g, K]^T (+ bias_g)
  * Same results contract as `count` separate tq_gemm / w4g_gemm calls (each element within the
- * stated bound; the split of K over CTAs may differ, so the bits may differ).  With M <= 16 on
- * shapes the decode path takes, all matrices run in ONE kernel launch (one kernel boundary
+ * stated bound; the split of K over CTAs may differ, so the bits may differ).  When
+ * tq_select_path picks the decode path (M up to the crossover) on shapes it takes, all
+ * matrices run in ONE kernel launch (one kernel boundary
  * instead of `count`); otherwise the call issues `count` single-matrix GEMMs.
  *   count              1 .. 4
  *   packed / qweight   HOST array of `count` device pointers (layouts as in tq_gemm / w4g_gemm)

@@ -54,7 +54,7 @@ def test_gemm_argument_errors_without_gpu():
     assert tq.lib.tq_gemm_ex(p, p, p, NULL, p, 1, 4, 64, 9, NULL) == -8       # unknown path
     assert tq.lib.w4g_gemm(p, p, p, NULL, p, 1, 4, 100, NULL) == -2           # K % 128
     # forced fast paths refuse shapes they cannot take / misaligned pointers
-    assert tq.lib.tq_gemm_ex(p, p, p, NULL, p, 17, 4, 64, 1, NULL) == -8      # decode needs M<=16
+    assert tq.lib.tq_gemm_ex(p, p, p, NULL, p, 65, 4, 64, 1, NULL) == -8      # decode needs M<=64
     assert tq.lib.tq_gemm_ex(p, p, p, NULL, p, 1, 4, 100, 1, NULL) == -8      # decode needs K%64
     assert tq.lib.tq_gemm_ex(p, p, p, NULL, p, 256, 4, 100, 2, NULL) == -8    # prefill needs K%64
     q = ctypes.c_void_p(4098)
@@ -76,9 +76,14 @@ def test_dispatch_rule():
     assert tq.tq_select_path(T, 1, 4096, 14336) == tq.PATH_DECODE
     assert tq.tq_select_path(T, 1, 3584, 18944) == tq.PATH_DECODE
     assert tq.tq_select_path(T, 16, 37888, 3584) == tq.PATH_DECODE
-    # tensor-core path above the ridge
-    for M in (17, 32, 512, 2048, 8192):
+    # measured crossover (Qwen2-7B shapes): ternary decode in 16-token chunks up to M = 48,
+    # W4A16 decode up to M = 16; the tensor-core path above
+    for M in (17, 32, 33, 48):
+        assert tq.tq_select_path(T, M, 4096, 4096) == tq.PATH_DECODE
+        assert tq.tq_select_path(T, M, 37888, 3584) == tq.PATH_DECODE
+    for M in (49, 64, 512, 2048, 8192):
         assert tq.tq_select_path(T, M, 4096, 4096) == tq.PATH_PREFILL
+    for M in (17, 24, 32, 512, 2048, 8192):
         assert tq.tq_select_path(W, M, 14336, 4096) == tq.PATH_PREFILL
     # shapes / alignment the fast kernels do not take
     assert tq.tq_select_path(T, 1, 4096, 4100) == tq.PATH_GENERIC

@@ -149,3 +149,26 @@ def test_prefill_split_k(M, N, K):
     xw, qw, sc, bw = _w4_problem(M, N, K // 128 * 128, 950 + M)
     yw = tq.w4g_gemm(xw, qw, sc, bw, path=tq.PATH_PREFILL)
     check_w4g_gemm(xw, qw, sc, bw, yw, cols=np.arange(0, N, 3), label=f"w4g prefill split-K M={M} {N}x{K}")
+
+
+# M > 16 on the decode path: token chunks of 16 over grid z (ragged last chunk, several row
+# blocks and K slices per chunk), both formats; M = 16 is the single-chunk reference point.
+@pytest.mark.parametrize("M", [17, 24, 32, 33, 48, 64])
+@pytest.mark.parametrize("N,K", [(1000, 1088), (4096, 4096), (3584, 18944)])
+def test_decode_token_chunks(M, N, K):
+    need_cuda()
+    cols = None if N <= 1000 else np.arange(0, N, 11)
+    x, p, s, b = _tq_problem(M, N, K, 1200 + M + N // 64)
+    y = tq.tq_gemm(x, p, s, b, path=tq.PATH_DECODE)
+    check_tq_gemm(x, p, s, b, y, cols=cols, label=f"tq decode chunks M={M} {N}x{K}")
+    Kw = K // 128 * 128
+    xw, qw, sc, bw = _w4_problem(M, N, Kw, 1300 + M)
+    yw = tq.w4g_gemm(xw, qw, sc, bw, path=tq.PATH_DECODE)
+    check_w4g_gemm(xw, qw, sc, bw, yw, cols=cols, label=f"w4g decode chunks M={M} {N}x{Kw}")
+
+
+def test_decode_token_chunks_limit():
+    need_cuda()
+    x, p, s, b = _tq_problem(65, 256, 512, 1400)
+    with pytest.raises(tq.TQError):
+        tq.tq_gemm(x, p, s, b, path=tq.PATH_DECODE)   # 64 tokens at most on the decode path
