@@ -44,6 +44,7 @@ constexpr int kQK = 64;          // K per stage: one 128-byte swizzle row of fp1
 constexpr int kQMaxRing = 12;    // stages of (x tile, packed tile), at most
 constexpr int kQMaxARing = 8;    // tensor-memory slots of decoded weights (32 columns each)
 constexpr int kQThreads = 256;   // warp 0 TMA, warp 1 MMA, warps 4-7 decode + epilogue
+constexpr bool kMergeStageBarriers = true;
 
 template <bool kInt4>
 struct PFmt {
@@ -63,8 +64,11 @@ struct PrefillLayout {
   static constexpr int kTileX = TN * kQK * 2;  // x tile of one stage
   static constexpr int kTileA = kQM * kQK * 2;  // decoded-weight tile of one stage (kSS)
   // ring depths: narrow tiles move little data per stage, so they keep more stages in flight
-  static constexpr int kRing = kSS ? (TN == 64 ? 8 : 4) : (TN == 256 ? 4 : (TN == 128 ? 6 : 10));
-  static constexpr int kARing = kSS ? 4 : (TN == 256 ? 4 : kQMaxARing);
+  static constexpr int kRing = kSS ? (TN == 64 ? 6 : 4) : (TN == 256 ? 4 : (TN == 128 ? 6 : 10));
+  static constexpr int kARing = kSS ? (TN == 64 ? 6 : 4) : (TN == 256 ? 4 : kQMaxARing);
+  // equal rings: one barrier per stage for "x tile landed and weights decoded" and one for
+  // "stage consumed", so the MMA thread tests one barrier and commits once per stage
+  static constexpr bool kMergedBars = kMergeStageBarriers && kRing == kARing;
   // split-K partials [S][128 rows][TN / S] fp32 reuse the x ring after the main loop
   static constexpr int kOffX = 0;
   static constexpr int kOffP = kOffX + kRing * kTileX;
@@ -154,9 +158,11 @@ __global__ void __launch_bounds__(kQThreads, 1)
   uint64_t* emptyX = bars + L::kRing;          // x tile consumed (MMA commit)
   uint64_t* fullP = bars + 2 * L::kRing;       // packed tile landed (TMA)
   uint64_t* emptyP = fullP + F::kPRing;        // packed tile consumed (decode warps)
-  uint64_t* afull = emptyP + F::kPRing;        // decoded weights in tensor memory
-  uint64_t* aempty = afull + L::kARing;        // ... consumed (MMA commit)
-  uint64_t* accFull = aempty + L::kARing;
+  // decoded weights written / consumed (MMA commit); with merged barriers the same barriers as
+  // the x tile's (stage s of both rings), `full` then also counts the four decode warps
+  uint64_t* afull = L::kMergedBars ? full : emptyP + F::kPRing;
+  uint64_t* aempty = L::kMergedBars ? emptyX : emptyP + F::kPRing + L::kARing;
+  uint64_t* accFull = emptyP + F::kPRing + 2 * L::kARing;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::kOffTmemSlot);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -171,14 +177,14 @@ __global__ void __launch_bounds__(kQThreads, 1)
   pdl_allow_dependents();
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::kRing; ++i) {
-      mbar_init(&full[i], 1);
+      mbar_init(&full[i], L::kMergedBars ? 5 : 1);
       mbar_init(&emptyX[i], 1);
     }
     for (int i = 0; i < F::kPRing; ++i) {
       mbar_init(&fullP[i], 1);
       mbar_init(&emptyP[i], 4);
     }
-    for (int i = 0; i < L::kARing; ++i) {
+    for (int i = 0; i < L::kARing && !L::kMergedBars; ++i) {
       mbar_init(&afull[i], 4);
       mbar_init(&aempty[i], 1);
     }
@@ -237,7 +243,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
       for (int kb = 0; kb < nk && ok; ++kb) {
         const int s = kb % L::kRing, as = kb % L::kARing;
         ok = mbar_wait(&full[s], static_cast<uint32_t>(kb / L::kRing) & 1u) &&
-             mbar_wait(&afull[as], static_cast<uint32_t>(kb / L::kARing) & 1u);
+             (L::kMergedBars || mbar_wait(&afull[as], static_cast<uint32_t>(kb / L::kARing) & 1u));
         if (!ok) break;
         tc_fence_after_sync();
         const uint64_t bdesc = sdesc_kmajor_sw128(x_base + s * L::kTileX);
@@ -253,7 +259,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
             umma_f16_ts(tmem, a_tmem + 8 * k16, bdesc + 2 * k16, idesc, (kb | k16) != 0 ? 1u : 0u);
         }
         umma_commit(&emptyX[s]);
-        umma_commit(&aempty[as]);
+        if (!L::kMergedBars) umma_commit(&aempty[as]);
       }
       if (ok) umma_commit(accFull);
     }
@@ -267,6 +273,13 @@ __global__ void __launch_bounds__(kQThreads, 1)
       if (!kInt4) ep_s = __half2float(a.sc[n]);
       if (a.bias) ep_b = __half2float(a.bias[n]);
     }
+    // W4A16 group scales of this row: the next group's is loaded when a group starts, a stage
+    // or two before it is needed, so the load latency stays off the decode
+    auto group_scale = [&](int64_t gi) -> uint16_t {
+      return (n < a.N && gi < G) ? __half_as_ushort(a.sc[n * G + gi]) : static_cast<uint16_t>(0);
+    };
+    int64_t g_cur = -1;
+    uint16_t sc_cur = 0, sc_nxt = 0;
     for (int kb = 0; kb < nk && ok; ++kb) {
       const int as = kb % L::kARing, pt = kb / F::kSPP, ci = kb - pt * F::kSPP, ps = pt % F::kPRing;
       if (ci == 0) {
@@ -286,8 +299,13 @@ __global__ void __launch_bounds__(kQThreads, 1)
       }
       uint32_t s2 = 0u;
       if (kInt4) {
-        const uint16_t sb = (n < a.N) ? __half_as_ushort(a.sc[n * G + ((kb0 + kb) >> 1)]) : static_cast<uint16_t>(0);
-        s2 = static_cast<uint32_t>(sb) | (static_cast<uint32_t>(sb) << 16);
+        const int64_t gi = (kb0 + kb) >> 1;  // 128-wide group of this 64-wide stage
+        if (gi != g_cur) {
+          sc_cur = g_cur < 0 ? group_scale(gi) : sc_nxt;
+          sc_nxt = group_scale(gi + 1);
+          g_cur = gi;
+        }
+        s2 = static_cast<uint32_t>(sc_cur) | (static_cast<uint32_t>(sc_cur) << 16);
       }
       const uint32_t pw[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
       if (kSS) {
