@@ -399,26 +399,27 @@ def secondary_rows(args, rank, layers, peaks):
     hbm = float(peaks["hbm_gbs"])
     tc = float(peaks["bf16_tflops"])
     rows = {}
-    # ---- ternary prefill (config 2): 4 layers x 7 shapes, M = 2048, bias, outlier tokens
-    M = 2048
-    xs = {K: I.activations(M, K, I.seed_for(2, 0, K), device="cuda", outlier_row_frac=0.01)
-          for K in (4096, 14336)}
+    # ---- ternary prefill (config 2): 4 layers x 7 shapes, M in {2048, 512, 8192}, bias, outlier
+    # tokens
     bs = {N: I.bias(N, I.seed_for(2, 1, N), device="cuda") for N in (1024, 4096, 14336)}
-    ys = {N: torch.empty(M, N, dtype=torch.float16, device="cuda") for N in (1024, 4096, 14336)}
     sub = layers[:4]
+    for M in (2048, 512, 8192):
+        xs = {K: I.activations(M, K, I.seed_for(2, 0, K), device="cuda", outlier_row_frac=0.01)
+              for K in (4096, 14336)}
+        ys = {N: torch.empty(M, N, dtype=torch.float16, device="cuda") for N in (1024, 4096, 14336)}
 
-    def pf():
-        for row in sub:
-            for name, N, K, p, s in row:
-                tq.tq_gemm(xs[K], p, s, bs[N], ys[N])
+        def pf():
+            for row in sub:
+                for name, N, K, p, s in row:
+                    tq.tq_gemm(xs[K], p, s, bs[N], ys[N])
 
-    g = capture(pf)
-    ms = time_graph(g, 3)
-    flops = sum(2 * M * N * K for row in sub for _, N, K, _, _ in row)
-    tf = flops / (ms * 1e-3) / 1e12
-    rows["ternary_prefill_M2048"] = {"value": round(tf, 1), "unit": "TFLOP/s", "frac": round(tf / tc, 4),
-                                     "peak": tc, "bound": "tensor", "sample": "4 layers x 7 shapes, M=2048"}
-    del g
+        g = capture(pf)
+        ms = time_graph(g, 3)
+        flops = sum(2 * M * N * K for row in sub for _, N, K, _, _ in row)
+        tf = flops / (ms * 1e-3) / 1e12
+        rows[f"ternary_prefill_M{M}"] = {"value": round(tf, 1), "unit": "TFLOP/s", "frac": round(tf / tc, 4),
+                                         "peak": tc, "bound": "tensor", "sample": f"4 layers x 7 shapes, M={M}"}
+        del g, xs, ys
     # ---- W4A16 decode / prefill (config 3): 8 layers
     w4 = []
     for l in range(8):
@@ -445,21 +446,24 @@ def secondary_rows(args, rank, layers, peaks):
         rows[f"w4g_decode_M{M}"] = {"value": round(gbs, 1), "unit": "GB/s", "frac": round(gbs / hbm, 4),
                                     "peak": hbm, "bound": "hbm", "sample": "8 layers x 7 shapes"}
         del g
-    M = 4096
-    xq = {K: I.activations(M, K, I.seed_for(3, 3, K), device="cuda") for K in (4096, 14336)}
-    yq = {N: torch.empty(M, N, dtype=torch.float16, device="cuda") for N in (1024, 4096, 14336)}
+    for M, wl in ((4096, w4[:1]), (256, w4)):
+        xq = {K: I.activations(M, K, I.seed_for(3, 3, K), device="cuda") for K in (4096, 14336)}
+        yq = {N: torch.empty(M, N, dtype=torch.float16, device="cuda") for N in (1024, 4096, 14336)}
 
-    def wp():
-        for name, N, K, qw, sc in w4[0]:
-            tq.w4g_gemm(xq[K], qw, sc, None, yq[N])
+        def wp():
+            for row in wl:
+                for name, N, K, qw, sc in row:
+                    tq.w4g_gemm(xq[K], qw, sc, None, yq[N])
 
-    g = capture(wp)
-    ms = time_graph(g, 3)
-    flops = sum(2 * M * N * K for _, N, K, _, _ in w4[0])
-    tf = flops / (ms * 1e-3) / 1e12
-    rows["w4g_prefill_M4096"] = {"value": round(tf, 1), "unit": "TFLOP/s", "frac": round(tf / tc, 4),
-                                 "peak": tc, "bound": "tensor", "sample": "1 layer x 7 shapes, M=4096"}
-    del g, w4
+        g = capture(wp)
+        ms = time_graph(g, 3 if M > 256 else 10)
+        flops = sum(2 * M * N * K for row in wl for _, N, K, _, _ in row)
+        tf = flops / (ms * 1e-3) / 1e12
+        rows[f"w4g_prefill_M{M}"] = {"value": round(tf, 1), "unit": "TFLOP/s", "frac": round(tf / tc, 4),
+                                     "peak": tc, "bound": "tensor",
+                                     "sample": f"{len(wl)} layer{'s' if len(wl) > 1 else ''} x 7 shapes, M={M}"}
+        del g, xq, yq
+    del w4
     # ---- config 0: one ternary linear 1024x1024 at M = 1 (L2-resident: the time of one call)
     w = I.weights(1024, 1024, I.seed_for(0, 0, 0), device="cuda")
     p0, s0 = tq.tq_quantize_pack(w)

@@ -10,7 +10,9 @@ from gpu_util import check_tq_gemm, check_w4g_gemm, gpu, need_cuda
 pytestmark = gpu
 
 
-@pytest.mark.parametrize("M", [1, 5, 16])
+# M = 32 and 41 take the decode path in token chunks of 16 (the last one ragged), one launch for
+# all three matrices
+@pytest.mark.parametrize("M", [1, 5, 16, 32, 41])
 def test_tq_grouped_qkv(M):
     need_cuda()
     K = 4096
