@@ -339,17 +339,7 @@ def run_ours(args, world, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
         "data": "synthetic (seeded N(0,0.02) weights ternarised on the GPU; x ~ N(0,1) fp16)",
-        "config": {"workload": "Llama-3-8B-shaped ternary decode linears: 32 layers x "
-                               "{q,k,v,o 4096x4096/1024x4096, gate/up 14336x4096, down 4096x14336} "
-                               "x M in {1,4,16}",
-                   "calls": ("7 tq_gemm calls per layer" if args.separate else
-                             "per layer: tq_gemm_grouped(q,k,v), tq_gemm(o), tq_gemm_grouped(gate,up), "
-                             "tq_gemm(down) -- the grouping a serving engine's fused QKV / gate-up "
-                             "projections use; same linears, same outputs"),
-                   "layers": n_layers, "M": list(DECODE_M), "launches_per_step": launches_step,
-                   "bytes_per_step": bytes_step, "l2": "inputs larger than L2 (1.745 GB packed)",
-                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
-                   "graph": "one CUDA graph per step, PDL between GEMMs"},
+        "config": dict(decode_config(args, world), launches_per_step=launches_step),
         "roofline": roof,
         "e2e": {"value": round(e2e_val, 1), "unit": "GB/s", "h2d_bytes_per_step": bi,
                 "d2h_bytes_per_step": bo, "ms_per_step": round(e2e_ms, 4)},
@@ -595,59 +585,104 @@ def load_traffic():
 # ------------------------------------------------------------------------------------------------
 # CPU oracle (reference arm and cpu_baseline)
 # ------------------------------------------------------------------------------------------------
-def cpu_baseline(seconds=12.0):
-    """The oracle as it stands, on the host cores, on a bounded sample of the decode workload:
-    the first 1024 output rows of each layer-0 Llama linear (q, k, v, o, gate, up, down), packed
-    by the oracle, then oracle tq_gemm at M = 1, 4, 16 cycled until `seconds` of GEMM time."""
+def decode_config(args, world):
+    """`config` of the headline decode workload (both arms)."""
+    return {"workload": "Llama-3-8B-shaped ternary decode linears: 32 layers x "
+                        "{q,k,v,o 4096x4096/1024x4096, gate/up 14336x4096, down 4096x14336} "
+                        "x M in {1,4,16}",
+            "calls": ("7 tq_gemm calls per layer" if args.separate else
+                      "per layer: tq_gemm_grouped(q,k,v), tq_gemm(o), tq_gemm_grouped(gate,up), "
+                      "tq_gemm(down) -- the grouping a serving engine's fused QKV / gate-up "
+                      "projections use; same linears, same outputs"),
+            "layers": 32, "M": list(DECODE_M),
+            "bytes_per_step": sum(decode_bytes(M, N, K) for M in DECODE_M for _ in range(32) for _, N, K in LLAMA),
+            "l2": "inputs larger than L2 (1.745 GB packed)",
+            "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+            "graph": "one CUDA graph per step, PDL between GEMMs"}
+
+
+ORACLE_SAMPLE_ROWS = 1024
+
+
+def oracle_sample_setup():
+    """The bounded sample of the decode workload the oracle is timed on: the first 1024 output
+    rows of each layer-0 Llama linear (q, k, v, o, gate, up, down), packed by the oracle."""
     import oracle as O
     import tq_inputs as I
 
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:  # noqa: BLE001
-        cores = os.cpu_count() or 1
-    rows = 1024
     mats = []
     for mid, (name, N, K) in enumerate(LLAMA):
-        w = I.weights(N, K, I.seed_for(1, 0, mid))[:rows].numpy()
+        w = I.weights(N, K, I.seed_for(1, 0, mid))[:ORACLE_SAMPLE_ROWS].numpy()
         p, s = O.tq_quantize_pack(w)
-        mats.append((name, min(N, rows), K, p, s))
+        mats.append((name, min(N, ORACLE_SAMPLE_ROWS), K, p, s))
     xs = {(M, K): I.activations(M, K, 1).numpy() for M in DECODE_M for K in {4096, 14336}}
+    return mats, xs
+
+
+def oracle_sample_run(sample, seconds, start=0):
+    """Oracle tq_gemm at M = 1, 4, 16 over the sample's linears, cycled until `seconds` of GEMM
+    time (at least one call). Returns (bytes, seconds, calls)."""
+    import oracle as O
+
+    mats, xs = sample
     done_b, gemm_time, n_items = 0, 0.0, 0
-    while gemm_time < seconds:
-        name, N, K, p, s = mats[n_items % len(mats)]
-        M = DECODE_M[(n_items // len(mats)) % len(DECODE_M)]
+    while gemm_time < seconds or n_items == 0:
+        i = start + n_items
+        name, N, K, p, s = mats[i % len(mats)]
+        M = DECODE_M[(i // len(mats)) % len(DECODE_M)]
         t1 = time.perf_counter()
         O.tq_gemm(xs[(M, K)], p, s, None, K)
         gemm_time += time.perf_counter() - t1
         done_b += decode_bytes(M, N, K)
         n_items += 1
-    return {"value": round(done_b / gemm_time / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"{n_items} oracle tq_gemm calls on the first {rows} output rows of each layer-0 "
-                      f"Llama linear, M cycling 1/4/16 ({gemm_time:.1f} s of GEMM)"}
+    return done_b, gemm_time, n_items
+
+
+def oracle_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # noqa: BLE001
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(seconds=12.0):
+    """The oracle as it stands, on the host cores, on the bounded sample of the decode workload
+    (`oracle_sample_setup`), timed for `seconds` of GEMM."""
+    done_b, gemm_time, n_items = oracle_sample_run(oracle_sample_setup(), seconds)
+    return {"value": round(done_b / gemm_time / 1e9, 4), "unit": "GB/s", "cores": oracle_cores(), "kind": "oracle",
+            "sample": f"{n_items} oracle tq_gemm calls on the first {ORACLE_SAMPLE_ROWS} output rows of each "
+                      f"layer-0 Llama linear, M cycling 1/4/16 ({gemm_time:.1f} s of GEMM)"}
 
 
 def run_reference(args, world, rank):
-    """Reference arm: the CPU oracle timed on this host, same metric/config (bounded sample)."""
+    """Reference arm: the CPU oracle timed on this host on the GPU arm's metric and config; each
+    step is a bounded sample of the workload (oracle GEMMs on the sample of `oracle_sample_setup`),
+    sized so that warm-up + timed steps take about `--cpu-seconds` of GEMM in total."""
     t0 = time.perf_counter()
-    per_step = []
-    res = None
+    sample = oracle_sample_setup()
+    per_step_s = min(2.0, max(0.02, args.cpu_seconds / max(1, args.steps + args.warmup)))
+    tot_b, tot_s, calls, step_ms = 0, 0.0, 0, []
     for i in range(args.warmup + args.steps):
-        r = cpu_baseline(seconds=max(2.0, args.cpu_seconds / max(1, args.steps)))
+        b, sec, n = oracle_sample_run(sample, per_step_s, start=calls)
+        calls += n
         if i >= args.warmup:
-            per_step.append(r)
-        res = r
-    val = statistics.median([r["value"] for r in per_step]) if per_step else res["value"]
+            tot_b += b
+            tot_s += sec
+            step_ms.append(sec * 1e3)
+    val = round(tot_b / tot_s / 1e9, 4) if tot_s > 0 else 0.0
+    timed_calls = calls
     return {
         "metric": METRIC, "value": val, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": round(statistics.median(step_ms), 3) if step_ms else None,
+        "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (same seeds as the GPU arm)",
-        "config": {"workload": "Llama-3-8B-shaped ternary decode linears (oracle on a bounded sample)",
-                   "M": list(DECODE_M)},
+        "config": decode_config(args, world),
         "impl": "reference",
-        "cpu_baseline": {"value": val, "unit": "GB/s", "cores": res["cores"], "kind": "oracle",
-                         "sample": res["sample"]},
+        "cpu_baseline": {"value": val, "unit": "GB/s", "cores": oracle_cores(), "kind": "oracle",
+                         "sample": f"each step: oracle tq_gemm calls for ~{per_step_s:.2f} s on the first "
+                                   f"{ORACLE_SAMPLE_ROWS} output rows of each layer-0 Llama linear, M cycling "
+                                   f"1/4/16 ({timed_calls} calls in warm-up and timed steps)"},
         "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "wall_s": round(time.perf_counter() - t0, 1),
     }
