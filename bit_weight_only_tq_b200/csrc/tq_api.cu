@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "../../include/tq.h"
@@ -20,17 +21,20 @@ bool prefill_supported(bool int4, int64_t M, int64_t N, int64_t K);
 static constexpr int kMaxDevices = 64;
 
 DeviceInfo current_device_info() {
-  static int sms[kMaxDevices] = {0};
+  // SM count per device, queried once; atomics because calls may come from several host threads
+  static std::atomic<int> sms[kMaxDevices];
   int dev = 0;
   cudaGetDevice(&dev);
   DeviceInfo d{dev, 148};
   if (dev >= 0 && dev < kMaxDevices) {
-    if (sms[dev] == 0) {
-      int v = 0;
+    int v = sms[dev].load(std::memory_order_relaxed);
+    if (v == 0) {
       if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
-        sms[dev] = v;
+        sms[dev].store(v, std::memory_order_relaxed);
+      else
+        v = 0;
     }
-    if (sms[dev] > 0) d.num_sms = sms[dev];
+    if (v > 0) d.num_sms = v;
   }
   return d;
 }
