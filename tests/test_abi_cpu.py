@@ -2,8 +2,10 @@
 declared in include/tq.h, validates arguments before touching the device, and applies the
 documented dispatch rule."""
 import ctypes
+import os
 
 import pytest
+import torch
 
 import bit_weight_only_tq_b200 as tq
 
@@ -105,3 +107,31 @@ def test_grouped_argument_errors_without_gpu():
     assert tq.lib.tq_gemm_grouped(p, 3, arr, arr, None, arr, bad, 1, 64, None) == -2
     assert tq.lib.w4g_gemm_grouped(p, 3, arr, arr, None, arr, ns, 1, 100, None) == -2  # K % 128
     assert tq.lib.tq_gemm_grouped(p, 3, arr, arr, None, arr, ns, 0, 64, None) == 0    # M = 0
+
+
+def test_no_cpu_fallback_for_host_tensors():
+    # the product path runs only in the CUDA library: host tensors are refused, never computed
+    x = torch.zeros(1, 64, dtype=torch.float16)
+    p = torch.full((8, 16), 0x55, dtype=torch.uint8)
+    s = torch.zeros(8, dtype=torch.float16)
+    with pytest.raises(ValueError):
+        tq.tq_gemm(x, p, s)
+    with pytest.raises(ValueError):
+        tq.tq_quantize_pack(torch.zeros(8, 64))
+
+
+def test_import_fails_loudly_without_the_library(tmp_path):
+    # a copy of the package with no libtq.so and no compiler: importing it must fail
+    import shutil
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    shutil.copytree(os.path.join(root, "bit_weight_only_tq_b200"), tmp_path / "bit_weight_only_tq_b200",
+                    ignore=shutil.ignore_patterns("*.so", "*.so.tmp", "__pycache__"))
+    shutil.copytree(os.path.join(root, "include"), tmp_path / "include")
+    env = dict(os.environ, NVCC=str(tmp_path / "no-such-nvcc"))
+    r = subprocess.run([sys.executable, "-c", "import bit_weight_only_tq_b200"], cwd=tmp_path, env=env,
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0
+    assert not (tmp_path / "bit_weight_only_tq_b200" / "libtq.so").exists()
