@@ -59,3 +59,25 @@ def test_two_gloo_ranks_replicas():
 def test_single_rank_aggregation():
     assert bench.max_over_ranks(1.5, 1) == 1.5
     assert bench.weak_scaling_value(6_530_000_000, 1, 1000.0) == pytest.approx(6.53)
+
+
+def test_reference_arm_json_line():
+    # `bench.py --impl reference` runs the CPU oracle on the host (no GPU) and prints one JSON
+    # line with the GPU arm's metric and config plus the reference-arm keys
+    import json
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--steps", "2",
+                        "--warmup", "3", "--cpu-seconds", "0.3"], cwd=root, capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.strip().splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["higher_is_better"] is True
+    assert d["value"] > 0 and d["steps"] == 2 and d["warmup"] == 3 and d["ms_per_step"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"] == {"value": d["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert "Llama-3-8B" in d["config"]["workload"]
