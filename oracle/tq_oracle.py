@@ -21,7 +21,11 @@ Readings adopted where the sources are silent or garbled (each is repeated at it
     by the count in fp64), rounded to fp16 with ties-to-even; 0 if the row has no nonzero code;
   * the 2-bit code table is 00 -> -1, 01 -> 0, 10 -> +1; 11 is invalid;
   * INT4: s = fp16(max|w| / 7) per (row, group of 128 along K); q = clamp(rint(w / s), -8, 7)
-    using the stored fp16 s, ties-to-even; nibble i of int32 word j holds q + 8 for k = 8j + i.
+    using the stored fp16 s, ties-to-even; nibble i of int32 word j holds q + 8 for k = 8j + i;
+  * asymmetric INT4: lo = min(0, min w), hi = max(0, max w) over the group, s = fp16((hi-lo)/15),
+    z = clamp(rint(-lo/s), 0, 15), q = clamp(rint(w/s) + z, 0, 15); zeros stored one byte per group;
+  * activation order: a given column permutation perm defines the groups (g_idx[perm[j]] =
+    j // 128); packed weights stay in the original column order.
 
 Every function here is pinned by tests in ``tests/test_oracle_*.py`` against values derived by
 hand from the sources, exact rational arithmetic, exhaustive enumeration and library routines.
@@ -48,6 +52,14 @@ __all__ = [
     "w4g_quantize_pack",
     "w4g_unpack",
     "w4g_gemm",
+    "pack_nibbles",
+    "unpack_nibbles",
+    "w4z_quantize_group",
+    "w4z_quantize_pack",
+    "w4z_unpack",
+    "w4z_gemm",
+    "w4g_quantize_pack_actorder",
+    "w4g_gemm_actorder",
     "gemm_reference",
     "quant_check",
     "InvalidCode",
@@ -300,6 +312,132 @@ def w4g_gemm(x_f16, qweight, scales_bits, bias_f16, K: int):
     """W4A16 linear layer reference: dequantise, then matmul ([VQ] §5 forward)."""
     What = w4g_unpack(qweight, scales_bits)
     assert What.shape[1] == K
+    return gemm_reference(x_f16, What, bias_f16)
+
+
+# ----------------------------------------------------------------------------------------------
+# INT4 variants ([VQ] §5): asymmetric zero-points and activation ordering (g_idx)
+# ----------------------------------------------------------------------------------------------
+def w4z_quantize_group(w_group, order_of_zero=True):
+    """Asymmetric INT4 of one group (the weight_zp / GroupQuantZeroPointParameter of [VQ] §5's
+    GPTQ-Marlin create_weights; the qweight / scales / zeros triple of an AWQ checkpoint, [TQ] §2.1).
+
+    The pages name the zero-point but give no formula; the min-max rule that keeps 0 inside the
+    range is read here:
+      lo = min(0, min w), hi = max(0, max w)            (fp64, exact)
+      s  = fp16(( hi - lo ) / 15)                        (fp64 division, binary16 ties-to-even)
+      s == 0 (an all-zero group): z = 0, every q = 0
+      else z = clamp(rint(-lo / s), 0, 15) and q = clamp(rint(w / s) + z, 0, 15), both with the
+           STORED fp16 s, fp64 quotients, rint = round half to even
+    Returns (q int64 array, s bits uint16, z int).
+    """
+    w = np.asarray(w_group, dtype=np.float64)
+    lo = min(0.0, float(w.min()))
+    hi = max(0.0, float(w.max()))
+    s_bits = f64_to_f16_bits((hi - lo) / 15.0)
+    s = float(f16_bits_to_f64(s_bits))
+    if s == 0.0:
+        return np.zeros(w.shape, np.int64), np.uint16(s_bits), 0
+    z = int(np.clip(np.rint(-lo / s), 0, 15))
+    q = np.clip(np.rint(w / s) + z, 0, 15).astype(np.int64)
+    return q, np.uint16(s_bits), z
+
+
+def pack_nibbles(u):
+    """u int64 [N, K] in 0..15 -> int32 [N, K/8], nibble i of word j = element 8j + i."""
+    N, K = u.shape
+    u = u.reshape(N, K // 8, 8)
+    word = np.zeros((N, K // 8), np.int64)
+    for i in range(8):
+        word |= u[:, :, i] << (4 * i)
+    return word.astype(np.uint32).view(np.int32)
+
+
+def unpack_nibbles(qweight):
+    qw = np.asarray(qweight).view(np.uint32).astype(np.int64)
+    N, KW = qw.shape
+    return np.stack([(qw >> (4 * i)) & 0xF for i in range(8)], axis=2).reshape(N, KW * 8)
+
+
+def w4z_quantize_pack(W, perm=None):
+    """Asymmetric INT4, group 128 along K, optionally in activation order.
+
+    perm (optional int array [K], a permutation of 0..K-1): the order in which GPTQ with
+    desc_act processes the input columns ([VQ] §5: "optional g_idx (activation ordering)"); here it
+    is an input (the pages' Hessian order needs calibration data).  Column perm[j] belongs to
+    group j // 128, i.e. g_idx[perm[j]] = j // 128.  Without perm, g_idx[k] = k // 128.
+    The packed weights stay in the ORIGINAL column order (nibble i of word j = column 8j + i, the
+    checkpoint layout); scales and zeros are [N, K/128] by group.
+    Returns (qweight int32 [N, K/8], scales uint16 fp16-bits [N, K/128], zeros uint8 [N, K/128],
+    g_idx int32 [K]).
+    """
+    W = np.asarray(W)
+    if W.dtype not in (np.float32, np.float16):
+        raise TypeError("W must be float32 or float16")
+    N, K = W.shape
+    if K % GROUP != 0 or K <= 0:
+        raise ValueError("K must be a positive multiple of 128")
+    perm = np.arange(K) if perm is None else np.asarray(perm, dtype=np.int64)
+    if sorted(perm.tolist()) != list(range(K)):
+        raise ValueError("perm must be a permutation of 0..K-1")
+    G = K // GROUP
+    g_idx = np.empty(K, np.int32)
+    g_idx[perm] = np.arange(K) // GROUP
+    q = np.zeros((N, K), np.int64)
+    scales = np.zeros((N, G), np.uint16)
+    zeros = np.zeros((N, G), np.uint8)
+    Wd = W.astype(np.float64)
+    for n in range(N):
+        for g in range(G):
+            cols = perm[g * GROUP:(g + 1) * GROUP]
+            qg, sb, z = w4z_quantize_group(Wd[n, cols])
+            q[n, cols] = qg
+            scales[n, g] = sb
+            zeros[n, g] = z
+    return pack_nibbles(q), scales, zeros, g_idx
+
+
+def w4z_unpack(qweight, scales_bits, zeros, g_idx=None) -> np.ndarray:
+    """What[n,k] = s[n, g_idx[k]] * (q[n,k] - z[n, g_idx[k]]) in fp64 (g_idx default k // 128)."""
+    q = unpack_nibbles(qweight)
+    N, K = q.shape
+    g = (np.arange(K) // GROUP) if g_idx is None else np.asarray(g_idx, dtype=np.int64)
+    s = f16_bits_to_f64(scales_bits)
+    z = np.asarray(zeros, dtype=np.int64)
+    return s[:, g] * (q - z[:, g]).astype(np.float64)
+
+
+def w4z_gemm(x_f16, qweight, scales_bits, zeros, bias_f16, K: int, g_idx=None):
+    """Asymmetric / act-order W4A16 linear layer reference: dequantise, then matmul."""
+    What = w4z_unpack(qweight, scales_bits, zeros, g_idx)
+    assert What.shape[1] == K
+    return gemm_reference(x_f16, What, bias_f16)
+
+
+def w4g_quantize_pack_actorder(W, perm):
+    """Symmetric INT4 ([VQ] §5 sym=true) with activation ordering: the rule of w4g_quantize_pack
+    applied to the columns of each group perm[128 g .. 128 g + 127].  Returns (qweight [N, K/8]
+    in the original column order, scales [N, K/128], g_idx [K])."""
+    W = np.asarray(W)
+    N, K = W.shape
+    perm = np.asarray(perm, dtype=np.int64)
+    if sorted(perm.tolist()) != list(range(K)) or K % GROUP != 0:
+        raise ValueError("perm must be a permutation of 0..K-1, K % 128 == 0")
+    qw_p, s = w4g_quantize_pack(W[:, perm])            # contiguous groups in processing order
+    u_p = unpack_nibbles(qw_p)
+    u = np.empty_like(u_p)
+    u[:, perm] = u_p                                   # back to the original column order
+    g_idx = np.empty(K, np.int32)
+    g_idx[perm] = np.arange(K) // GROUP
+    return pack_nibbles(u), s, g_idx
+
+
+def w4g_gemm_actorder(x_f16, qweight, scales_bits, g_idx, bias_f16, K: int):
+    """What[n,k] = s[n, g_idx[k]] * (u[n,k] - 8); then y = x . What^T (+ bias)."""
+    u = unpack_nibbles(qweight)
+    s = f16_bits_to_f64(scales_bits)
+    g = np.asarray(g_idx, dtype=np.int64)
+    What = s[:, g] * (u - 8).astype(np.float64)
     return gemm_reference(x_f16, What, bias_f16)
 
 
