@@ -6,6 +6,7 @@ this package fails loudly if the shared library is missing and cannot be built.
 
 Functions mirror the C ABI in include/tq.h:
     tq_quantize_pack, tq_gemm, w4g_quantize_pack, w4g_gemm, tq_validate_packed,
+    tq_gemm_grouped, w4g_gemm_grouped, tq_gemm_batch, w4g_gemm_batch, tq_batch_workspace_size,
     tq_select_path, tq_device_status, tq_status_string
 """
 from __future__ import annotations
@@ -23,7 +24,9 @@ __all__ = [
     "TQ_OK", "TQ_F32", "TQ_F16", "PATH_AUTO", "PATH_DECODE", "PATH_PREFILL", "PATH_GENERIC",
     "FMT_TERNARY", "FMT_W4G128",
     "tq_quantize_pack", "tq_gemm", "w4g_quantize_pack", "w4g_gemm", "tq_validate_packed",
-    "tq_gemm_grouped", "w4g_gemm_grouped",
+    "tq_gemm_grouped", "w4g_gemm_grouped", "tq_gemm_batch", "w4g_gemm_batch", "batch_workspace",
+    "tq_batch_workspace_size", "TqLinear", "w4g_quantize_pack_ex", "w4g_gemm_zp", "w4g_repack_act_order",
+    "tq_permute_columns",
     "tq_select_path", "tq_device_status", "tq_status_string", "header_functions",
 ]
 
@@ -48,6 +51,15 @@ def _load():
 lib, lib_path = _load()
 
 _vp, _i64, _int = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+
+
+class TqLinear(ctypes.Structure):
+    """struct tq_linear of include/tq.h: one linear of a batch call (device pointers)."""
+    _fields_ = [("x", ctypes.c_void_p), ("w", ctypes.c_void_p), ("scale", ctypes.c_void_p),
+                ("bias", ctypes.c_void_p), ("y", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("zeros", ctypes.c_void_p)]
+
+
 _SIGS = {
     "tq_quantize_pack": [_vp, _int, _vp, _vp, _i64, _i64, _vp],
     "tq_gemm": [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp],
@@ -58,6 +70,16 @@ _SIGS = {
     "tq_validate_packed": [_vp, _i64, _i64, _vp, _vp],
     "tq_gemm_grouped": [_vp, _int, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _vp],
     "w4g_gemm_grouped": [_vp, _int, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _vp],
+    "tq_gemm_batch": [_vp, _int, _i64, _vp, ctypes.c_size_t, _vp],
+    "w4g_gemm_batch": [_vp, _int, _i64, _vp, ctypes.c_size_t, _vp],
+    "tq_batch_workspace_size": [],
+    "tq_debug_set_wait_limit": [ctypes.c_longlong],
+    "tq_debug_skip_activation_loads": [_int],
+    "w4g_quantize_pack_ex": [_vp, _int, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _vp],
+    "w4g_gemm_zp": [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp],
+    "w4g_gemm_zp_ex": [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _vp],
+    "w4g_repack_act_order": [_vp, _vp, _vp, _i64, _i64, _vp],
+    "tq_permute_columns": [_vp, _vp, _vp, _i64, _i64, _vp],
     "tq_select_path": [_int, _i64, _i64, _i64, _int],
     "tq_device_status": [],
     "tq_status_string": [_int],
@@ -66,14 +88,14 @@ _SIGS = {
 for _name, _args in _SIGS.items():
     _f = getattr(lib, _name)
     _f.argtypes = _args
-    _f.restype = ctypes.c_char_p if _name == "tq_status_string" else ctypes.c_int
+    _f.restype = {"tq_status_string": ctypes.c_char_p, "tq_batch_workspace_size": ctypes.c_size_t}.get(_name, ctypes.c_int)
 
 
 def header_functions(path: str = HEADER):
     """Names of the functions declared in include/tq.h."""
     with open(path) as f:
         txt = f.read()
-    return sorted(set(re.findall(r"^\s*TQ_API\s+(?:int|const char\*)\s+(\w+)\s*\(", txt, re.M)))
+    return sorted(set(re.findall(r"^\s*TQ_API\s+(?:int|size_t|const char\*)\s+(\w+)\s*\(", txt, re.M)))
 
 
 class TQError(RuntimeError):
@@ -186,6 +208,69 @@ def w4g_gemm(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, bias=
     return y
 
 
+def w4g_quantize_pack_ex(w: torch.Tensor, zero_point: bool = False, perm: torch.Tensor | None = None,
+                         stream=None):
+    """General INT4 pack (group 128): symmetric or asymmetric (zero_point=True), in activation order
+    when `perm` (int32 [K], the column processing order) is given.  Returns
+    (qweight int32 [N, K/8] in the original column order, scales fp16 [N, K/128],
+    zeros uint8 [N, K/128] or None, g_idx int32 [K])."""
+    if w.dtype not in (torch.float32, torch.float16):
+        raise ValueError("w must be float32 or float16")
+    _need(w, w.dtype, "w", 2)
+    _need(perm, torch.int32, "perm", 1)
+    N, K = w.shape
+    qweight = torch.empty(N, K // 8, dtype=torch.int32, device=w.device)
+    scales = torch.empty(N, K // 128, dtype=torch.float16, device=w.device)
+    zeros = torch.empty(N, K // 128, dtype=torch.uint8, device=w.device) if zero_point else None
+    g_idx = torch.empty(K, dtype=torch.int32, device=w.device)
+    dt = TQ_F16 if w.dtype == torch.float16 else TQ_F32
+    _check(lib.w4g_quantize_pack_ex(_ptr(w), dt, _ptr(perm), _ptr(qweight), _ptr(scales), _ptr(zeros), _ptr(g_idx),
+                                    N, K, _stream(stream)), "w4g_quantize_pack_ex")
+    return qweight, scales, zeros, g_idx
+
+
+def w4g_gemm_zp(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor, bias=None,
+                y=None, path: int = PATH_AUTO, stream=None) -> torch.Tensor:
+    """y = x . What^T (+ bias), What = scales[n, k/128] * (u - zeros[n, k/128])."""
+    _need(x, torch.float16, "x", 2)
+    _need(qweight, torch.int32, "qweight", 2)
+    _need(scales, torch.float16, "scales", 2)
+    _need(zeros, torch.uint8, "zeros", 2)
+    _need(bias, torch.float16, "bias", 1)
+    M, K = x.shape
+    N = qweight.shape[0]
+    if qweight.shape[1] * 8 != K or tuple(scales.shape) != (N, K // 128) or tuple(zeros.shape) != (N, K // 128):
+        raise ValueError("qweight / scales / zeros shapes do not match x")
+    if y is None:
+        y = torch.empty(M, N, dtype=torch.float16, device=x.device)
+    _need(y, torch.float16, "y", 2)
+    _check(lib.w4g_gemm_zp_ex(_ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros), _ptr(bias), _ptr(y), M, N, K,
+                              int(path), _stream(stream)), "w4g_gemm_zp")
+    return y
+
+
+def w4g_repack_act_order(qweight: torch.Tensor, perm: torch.Tensor, stream=None) -> torch.Tensor:
+    """Columns reordered into the quantisation order: out[:, j] = qweight column perm[j]."""
+    _need(qweight, torch.int32, "qweight", 2)
+    _need(perm, torch.int32, "perm", 1)
+    out = torch.empty_like(qweight)
+    _check(lib.w4g_repack_act_order(_ptr(qweight), _ptr(perm), _ptr(out), qweight.shape[0], qweight.shape[1] * 8,
+                                    _stream(stream)), "w4g_repack_act_order")
+    return out
+
+
+def tq_permute_columns(x: torch.Tensor, perm: torch.Tensor, out=None, stream=None) -> torch.Tensor:
+    """out[m, j] = x[m, perm[j]] (fp16)."""
+    _need(x, torch.float16, "x", 2)
+    _need(perm, torch.int32, "perm", 1)
+    if out is None:
+        out = torch.empty_like(x)
+    _need(out, torch.float16, "out", 2)
+    _check(lib.tq_permute_columns(_ptr(x), _ptr(perm), _ptr(out), x.shape[0], x.shape[1], _stream(stream)),
+           "tq_permute_columns")
+    return out
+
+
 def _ptr_array(ts):
     arr = (ctypes.c_void_p * len(ts))()
     for i, t in enumerate(ts):
@@ -229,6 +314,65 @@ def w4g_gemm_grouped(x, qweight_list, scales_list, bias_list=None, y_list=None, 
     """Several W4A16 linears sharing x in one launch: returns [y_g]."""
     return _grouped(lib.w4g_gemm_grouped, x, qweight_list, scales_list, bias_list, y_list, torch.int32, 2,
                     "w4g_gemm_grouped", stream)
+
+
+def tq_batch_workspace_size() -> int:
+    """Bytes of workspace the batch calls need on the current device."""
+    return int(lib.tq_batch_workspace_size())
+
+
+def batch_workspace(device=None) -> torch.Tensor:
+    """A zero-filled workspace for tq_gemm_batch / w4g_gemm_batch on `device` (default: the
+    current device).  Zero it again only after a call that failed."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        n = tq_batch_workspace_size()
+    return torch.zeros(n, dtype=torch.uint8, device=dev)
+
+
+def _batch(fn, xs, weights, scales, biases, ys, workspace, wdtype, sdim, what, stream, zeros=None):
+    count = len(weights)
+    if not (1 <= count <= 8) or len(scales) != count or len(xs) != count:
+        raise ValueError("1..8 linears, each with its x, weights and scales")
+    biases = [None] * count if biases is None else list(biases)
+    M = xs[0].shape[0]
+    items = (TqLinear * count)()
+    out = []
+    for i, (x, w, s, b) in enumerate(zip(xs, weights, scales, biases)):
+        _need(x, torch.float16, "x", 2)
+        _need(w, wdtype, "weights", 2)
+        _need(s, torch.float16, "scales", sdim)
+        _need(b, torch.float16, "bias", 1)
+        if x.shape[0] != M:
+            raise ValueError("every x of a batch has the same number of tokens M")
+        N, K = w.shape[0], x.shape[1]
+        y = torch.empty(M, N, dtype=torch.float16, device=x.device) if ys is None else ys[i]
+        _need(y, torch.float16, "y", 2)
+        if tuple(y.shape) != (M, N):
+            raise ValueError("y shape mismatch")
+        z = None if zeros is None else zeros[i]
+        _need(z, torch.uint8, "zeros", 2)
+        items[i] = TqLinear(x.data_ptr(), w.data_ptr(), s.data_ptr(), None if b is None else b.data_ptr(),
+                            y.data_ptr(), N, K, None if z is None else z.data_ptr())
+        out.append(y)
+    if workspace is None:
+        raise ValueError("a workspace from batch_workspace() is required")
+    _need(workspace, torch.uint8, "workspace", 1)
+    _check(fn(items, count, M, _ptr(workspace), workspace.numel(), _stream(stream)), what)
+    return out
+
+
+def tq_gemm_batch(xs, packed_list, scale_list, bias_list=None, y_list=None, workspace=None, stream=None):
+    """Independent ternary linears sharing M (each with its own x) in one persistent launch."""
+    return _batch(lib.tq_gemm_batch, xs, packed_list, scale_list, bias_list, y_list, workspace, torch.uint8, 1,
+                  "tq_gemm_batch", stream)
+
+
+def w4g_gemm_batch(xs, qweight_list, scales_list, bias_list=None, y_list=None, workspace=None, stream=None,
+                   zeros_list=None):
+    """Independent W4A16 linears sharing M in one persistent launch (zero-points optional)."""
+    return _batch(lib.w4g_gemm_batch, xs, qweight_list, scales_list, bias_list, y_list, workspace, torch.int32, 2,
+                  "w4g_gemm_batch", stream, zeros=zeros_list)
 
 
 def tq_validate_packed(packed: torch.Tensor, K: int, stream=None) -> int:

@@ -81,6 +81,18 @@ bool make_tmap_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
   return r == CUDA_SUCCESS;
 }
 
+// An empty kernel launched in plain stream order after every call that writes packed weights,
+// scales or zero-points.  The GEMM kernels read those model constants before
+// griddepcontrol.wait (programmatic dependent launch lets them start while the previous kernel
+// on the stream finishes); after this kernel, the previous kernel is always this one, which
+// itself started only once the writer had completed and its writes were visible.
+__global__ void constants_written_kernel() {}
+
+cudaError_t after_constants_written(cudaStream_t s) {
+  constants_written_kernel<<<1, 32, 0, s>>>();
+  return cudaGetLastError();
+}
+
 cudaError_t ensure_smem_attr(const void* func, int bytes) {
   struct Entry {
     const void* f;
@@ -226,7 +238,8 @@ int tq_quantize_pack(const void* w, int w_dtype, uint8_t* packed, uint16_t* scal
   if (N < 0 || K <= 0 || K > (int64_t(1) << 28)) return TQ_ERR_SHAPE;
   if (N == 0) return TQ_OK;
   if (!w || !packed || !scale) return TQ_ERR_NULL;
-  return to_status(tq::launch_tq_pack(w, w_dtype == TQ_F16, packed, scale, N, K, as_stream(stream)));
+  const cudaError_t e = tq::launch_tq_pack(w, w_dtype == TQ_F16, packed, scale, N, K, as_stream(stream));
+  return to_status(e != cudaSuccess ? e : tq::after_constants_written(as_stream(stream)));
 }
 
 int w4g_quantize_pack(const void* w, int w_dtype, int32_t* qweight, uint16_t* scales, int64_t N,
@@ -235,7 +248,8 @@ int w4g_quantize_pack(const void* w, int w_dtype, int32_t* qweight, uint16_t* sc
   if (N < 0 || K <= 0 || K % 128 != 0 || K > (int64_t(1) << 28)) return TQ_ERR_SHAPE;
   if (N == 0) return TQ_OK;
   if (!w || !qweight || !scales) return TQ_ERR_NULL;
-  return to_status(tq::launch_w4g_pack(w, w_dtype == TQ_F16, qweight, scales, N, K, as_stream(stream)));
+  const cudaError_t e = tq::launch_w4g_pack(w, w_dtype == TQ_F16, qweight, scales, N, K, as_stream(stream));
+  return to_status(e != cudaSuccess ? e : tq::after_constants_written(as_stream(stream)));
 }
 
 int tq_gemm_ex(const uint16_t* x, const uint8_t* packed, const uint16_t* scale,
@@ -266,9 +280,12 @@ int tq_gemm(const uint16_t* x, const uint8_t* packed, const uint16_t* scale, con
   return tq_gemm_ex(x, packed, scale, bias, y, M, N, K, TQ_PATH_AUTO, stream);
 }
 
-int w4g_gemm_ex(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
-                const uint16_t* bias, uint16_t* y, int64_t M, int64_t N, int64_t K, int path,
-                void* stream) {
+}  // extern "C"
+
+namespace {
+
+int w4_gemm_impl(const uint16_t* x, const int32_t* qweight, const uint16_t* scales, const uint8_t* zeros,
+                 const uint16_t* bias, uint16_t* y, int64_t M, int64_t N, int64_t K, int path, void* stream) {
   bool empty = false;
   int st = check_gemm_args(x, qweight, scales, y, M, N, K, &empty);
   if (st != TQ_OK) return st;
@@ -284,10 +301,61 @@ int w4g_gemm_ex(const uint16_t* x, const int32_t* qweight, const uint16_t* scale
   __half* yh = reinterpret_cast<__half*>(y);
   cudaStream_t s = as_stream(stream);
   switch (p) {
-    case TQ_PATH_DECODE: return to_status(tq::launch_w4g_gemm_decode(xh, qweight, sh, bh, yh, M, N, K, s));
-    case TQ_PATH_PREFILL: return to_status(tq::launch_w4g_gemm_prefill(xh, qweight, sh, bh, yh, M, N, K, s));
-    default: return to_status(tq::launch_w4g_gemm_generic(xh, qweight, sh, bh, yh, M, N, K, s));
+    case TQ_PATH_DECODE: return to_status(tq::launch_w4g_gemm_decode(xh, qweight, sh, zeros, bh, yh, M, N, K, s));
+    case TQ_PATH_PREFILL: return to_status(tq::launch_w4g_gemm_prefill(xh, qweight, sh, zeros, bh, yh, M, N, K, s));
+    default: return to_status(tq::launch_w4g_gemm_generic(xh, qweight, sh, zeros, bh, yh, M, N, K, s));
   }
+}
+
+}  // namespace
+
+extern "C" {
+
+int w4g_gemm_ex(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
+                const uint16_t* bias, uint16_t* y, int64_t M, int64_t N, int64_t K, int path,
+                void* stream) {
+  return w4_gemm_impl(x, qweight, scales, nullptr, bias, y, M, N, K, path, stream);
+}
+
+int w4g_gemm_zp_ex(const uint16_t* x, const int32_t* qweight, const uint16_t* scales, const uint8_t* zeros,
+                   const uint16_t* bias, uint16_t* y, int64_t M, int64_t N, int64_t K, int path, void* stream) {
+  if (!zeros && M > 0 && N > 0) return TQ_ERR_NULL;
+  return w4_gemm_impl(x, qweight, scales, zeros, bias, y, M, N, K, path, stream);
+}
+
+int w4g_gemm_zp(const uint16_t* x, const int32_t* qweight, const uint16_t* scales, const uint8_t* zeros,
+                const uint16_t* bias, uint16_t* y, int64_t M, int64_t N, int64_t K, void* stream) {
+  return w4g_gemm_zp_ex(x, qweight, scales, zeros, bias, y, M, N, K, TQ_PATH_AUTO, stream);
+}
+
+int w4g_quantize_pack_ex(const void* w, int w_dtype, const int32_t* perm, int32_t* qweight, uint16_t* scales,
+                         uint8_t* zeros, int32_t* g_idx, int64_t N, int64_t K, void* stream) {
+  if (w_dtype != TQ_F32 && w_dtype != TQ_F16) return TQ_ERR_DTYPE;
+  if (N < 0 || K <= 0 || K % 128 != 0 || K > (int64_t(1) << 28)) return TQ_ERR_SHAPE;
+  if (N == 0) {
+    if (g_idx && perm) return TQ_ERR_SHAPE;  // g_idx of an empty matrix in act order: nothing defines it
+    return g_idx ? to_status(tq::launch_iota_groups(g_idx, K, as_stream(stream))) : TQ_OK;
+  }
+  if (!w || !qweight || !scales) return TQ_ERR_NULL;
+  const cudaError_t e =
+      tq::launch_w4g_pack_ex(w, w_dtype == TQ_F16, perm, qweight, scales, zeros, g_idx, N, K, as_stream(stream));
+  return to_status(e != cudaSuccess ? e : tq::after_constants_written(as_stream(stream)));
+}
+
+int tq_permute_columns(const uint16_t* x, const int32_t* perm, uint16_t* out, int64_t M, int64_t K, void* stream) {
+  if (M < 0 || K <= 0) return TQ_ERR_SHAPE;
+  if (M == 0) return TQ_OK;
+  if (!x || !perm || !out) return TQ_ERR_NULL;
+  return to_status(tq::launch_permute_cols(x, perm, out, M, K, as_stream(stream)));
+}
+
+int w4g_repack_act_order(const int32_t* qweight, const int32_t* perm, int32_t* out, int64_t N, int64_t K,
+                         void* stream) {
+  if (N < 0 || K <= 0 || K % 8 != 0) return TQ_ERR_SHAPE;
+  if (N == 0) return TQ_OK;
+  if (!qweight || !perm || !out) return TQ_ERR_NULL;
+  const cudaError_t e = tq::launch_repack_act_order(qweight, perm, out, N, K, as_stream(stream));
+  return to_status(e != cudaSuccess ? e : tq::after_constants_written(as_stream(stream)));
 }
 
 int w4g_gemm(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
@@ -307,6 +375,66 @@ int w4g_gemm_grouped(const uint16_t* x, int count, const int32_t* const* qweight
                      uint16_t* const* y, const int64_t* N, int64_t M, int64_t K, void* stream) {
   return gemm_grouped_impl<true>(x, count, qweight, scales, bias, y, N, M, K, stream, w4g_gemm,
                                  tq::launch_w4g_gemm_decode_group);
+}
+
+int tq_debug_set_wait_limit(long long cycles) {
+  const long long v = cycles > 0 ? cycles : tq::kWaitLimitCycles;
+  return to_status(cudaMemcpyToSymbol(tq::g_tq_wait_limit, &v, sizeof(v)));
+}
+
+int tq_debug_skip_activation_loads(int on) {
+  const int v = on ? 1 : 0;
+  return to_status(cudaMemcpyToSymbol(tq::g_tq_skip_x_loads, &v, sizeof(v)));
+}
+
+size_t tq_batch_workspace_size(void) { return static_cast<size_t>(tq::batch_workspace_bytes()); }
+
+}  // extern "C"
+
+namespace {
+
+template <bool kInt4>
+int gemm_batch_impl(const tq_linear* items, int count, int64_t M, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+  if (count < 1 || count > tq::kBatchMaxItems) return TQ_ERR_SHAPE;
+  if (M < 0 || M > tq::kBatchMaxM) return TQ_ERR_SHAPE;
+  if (!items) return TQ_ERR_NULL;
+  tq::BatchLinear lin[tq::kBatchMaxItems];
+  int n = 0;
+  for (int i = 0; i < count; ++i) {
+    const tq_linear& it = items[i];
+    if (it.N < 0 || it.N > (int64_t(1) << 31) || it.K <= 0 || it.K > (int64_t(1) << 28)) return TQ_ERR_SHAPE;
+    if (kInt4 ? (it.K % 128 != 0) : (it.K % 64 != 0)) return TQ_ERR_SHAPE;
+    if (it.N == 0) continue;
+    if (!it.x || !it.w || !it.scale || !it.y) return TQ_ERR_NULL;
+    if (!aligned16(it.x) || !aligned16(it.w)) return TQ_ERR_ALIGN;
+    lin[n++] = tq::BatchLinear{reinterpret_cast<const __half*>(it.x), it.w, reinterpret_cast<const __half*>(it.scale),
+                               reinterpret_cast<const __half*>(it.bias), reinterpret_cast<__half*>(it.y), it.N, it.K,
+                               kInt4 ? it.zeros : nullptr};
+  }
+  if (M == 0 || n == 0) return TQ_OK;
+  if (!workspace) return TQ_ERR_NULL;
+  if (!aligned16(workspace)) return TQ_ERR_ALIGN;
+  if (static_cast<int64_t>(workspace_bytes) < tq::batch_workspace_bytes()) return TQ_ERR_SHAPE;
+  const cudaError_t e = kInt4 ? tq::launch_w4g_gemm_batch(lin, n, M, workspace, static_cast<int64_t>(workspace_bytes),
+                                                          as_stream(stream))
+                              : tq::launch_tq_gemm_batch(lin, n, M, workspace, static_cast<int64_t>(workspace_bytes),
+                                                         as_stream(stream));
+  return to_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+int tq_gemm_batch(const tq_linear* items, int count, int64_t M, void* workspace, size_t workspace_bytes,
+                  void* stream) {
+  return gemm_batch_impl<false>(items, count, M, workspace, workspace_bytes, stream);
+}
+
+int w4g_gemm_batch(const tq_linear* items, int count, int64_t M, void* workspace, size_t workspace_bytes,
+                   void* stream) {
+  return gemm_batch_impl<true>(items, count, M, workspace, workspace_bytes, stream);
 }
 
 int tq_validate_packed(const uint8_t* packed, int64_t N, int64_t K, int* bad_count, void* stream) {

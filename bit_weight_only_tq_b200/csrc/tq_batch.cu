@@ -1,0 +1,398 @@
+// tq_batch.cu -- persistent decode GEMM over a work list of independent linears (M <= 16).
+//
+// [TQ] §1: a decode step is bound by the HBM stream of packed weights, and a serving engine's
+// step runs many small linears; every launch boundary leaves SMs idle for microseconds (the
+// previous grid drains, the next one starts, the first activations arrive).  This kernel takes up
+// to kBMaxItems linears that share M -- the linears of one decoder layer, say -- and streams all
+// their packed weights in ONE launch, with a fixed set of CTAs (two per SM):
+//
+//   * The work is the sequence of stages (item, block of 128 rows, 128 bytes of every row of the
+//     block), item-major, then row-block-major, then along K; T stages in total.  CTA c takes the
+//     contiguous range [c T / G, (c + 1) T / G): every CTA streams the same number of bytes, so
+//     the launch ends when the bytes are through, whatever the shapes.
+//   * A row block whose stages all fall to one CTA is finished there (scale, bias, fp16 y).  A row
+//     block split between CTAs (only at the ends of a CTA's range) is summed through a
+//     caller-provided workspace: each contributor stores its fp32 partial in its own slot and
+//     counts itself in on the row block's counter; the last to arrive adds the slots in K order
+//     (deterministic: the same sum whichever CTA arrives last), writes y and resets the counter,
+//     so the workspace is ready for the next call.  Nobody waits for anybody.
+//   * The producer warp streams the next row blocks' weights into the ring while the consumer
+//     warps finish a row block; the weights of the first stages are requested before
+//     griddepcontrol.wait (model constants), so they arrive while the previous grid drains.
+//
+// The per-stage math is the decode kernel's (tq_decode.cu): mma.sync m16n8k16 with the weights
+// as the A operand, decoded exactly into fp16 in registers; fp32 accumulation.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "tq_common.cuh"
+
+namespace tq {
+
+constexpr int kBMaxItems = kBatchMaxItems;
+constexpr int kBRows = 128;       // rows of a row block (one packed TMA tile)
+constexpr int kBResPitch = 132;   // fp32 row pitch of the result buffer [token][row]
+constexpr int kBCtasPerSm = 2;
+
+struct BatchItem {
+  const __half* sc;    // ternary: scale[N]; W4A16: scales[N, K/128]
+  const uint8_t* zp;   // W4A16 zero-points [N, K/128], or null (symmetric)
+  const __half* bias;  // may be null
+  __half* y;           // [M, N]
+  int64_t N, K;
+  int64_t begin;       // first stage of this item in the launch's sequence
+  int C;               // stages per row block (along K)
+  int RB;              // row blocks
+};
+
+struct BatchParams {
+  CUtensorMap w[kBMaxItems];  // packed weights: [N rows][row bytes], box 128 B x 128 rows, 128-B swizzle
+  CUtensorMap x[kBMaxItems];  // activations viewed as [M][K/64][64], box 64 x 4 x M, 128-B swizzle
+  BatchItem it[kBMaxItems];
+  int count;
+  int M;
+  int G;                      // CTAs
+  int ring, stage, xhalf;
+  int64_t T;                  // stages in total
+  int* counters;              // [G] arrivals per split row block, indexed by its first contributor
+  float* slots;               // [2 G][16][128] fp32 partials: slot 2c = CTA c's first row block,
+                              // 2c + 1 = its last
+};
+
+template <bool kInt4>
+struct BatchLayout {
+  static constexpr int kRes = 16 * kBResPitch * 4;
+  __host__ __device__ static constexpr int fixed() { return 1024 + kRes + 2 * kDMaxRing * 8 + 16; }
+  __host__ __device__ static constexpr int bytes(int ring, int stage) { return fixed() + ring * stage; }
+};
+
+// Workspace layout: counters first (256-byte padded), then the partial slots.
+__host__ __device__ inline int64_t batch_counter_bytes(int G) { return ((static_cast<int64_t>(G) * 4 + 255) / 256) * 256; }
+__host__ __device__ inline int64_t batch_workspace_bytes_for(int G) {
+  return batch_counter_bytes(G) + 2 * static_cast<int64_t>(G) * 16 * kBRows * 4;
+}
+
+// First stage of CTA c's range, and the CTA whose range holds stage s.
+__device__ __forceinline__ int64_t range_begin(int c, int64_t T, int G) { return (static_cast<int64_t>(c) * T) / G; }
+__device__ __forceinline__ int range_owner(int64_t s, int64_t T, int G) {
+  return static_cast<int>(((s + 1) * G - 1) / T);
+}
+
+template <bool kInt4, int NT, int TW>
+__device__ __forceinline__ void batch_body(const BatchParams& P) {
+  using F = DecFmt<kInt4>;
+  using W = DecWarps<NT, TW>;
+  constexpr int kEp = W::kCons * 32;  // consumer threads (epilogue)
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* stg = base;                                                 // ring x [weights | x]
+  float* res = reinterpret_cast<float*>(stg + P.ring * P.stage);       // [16 tokens][kBResPitch]
+  uint64_t* full = reinterpret_cast<uint64_t*>(res + 16 * kBResPitch);
+  uint64_t* empty = full + kDMaxRing;
+  volatile int* flags = reinterpret_cast<volatile int*>(empty + kDMaxRing);  // [0] abort, [1] last
+
+  pdl_allow_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = static_cast<int>(blockIdx.x);
+  const int64_t s0 = range_begin(c, P.T, P.G), s1 = range_begin(c + 1, P.T, P.G);
+  const int nst = static_cast<int>(s1 - s0);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < P.ring; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], W::kCons);
+    }
+    flags[0] = 0;
+    flags[1] = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (nst <= 0) return;
+
+  // position of the range's first stage: item, row block, stage within the row block
+  int it0 = 0;
+  while (it0 + 1 < P.count && P.it[it0 + 1].begin <= s0) ++it0;
+  const int rb0 = static_cast<int>((s0 - P.it[it0].begin) / P.it[it0].C);
+  const int k0 = static_cast<int>((s0 - P.it[it0].begin) % P.it[it0].C);
+
+  if (warp == W::kCons) {
+    // ==================================================================== producer warp
+    if (lane == 0) {
+      const uint32_t tx = static_cast<uint32_t>(kDWBytes + F::kKB * P.M * 128);  // whole boxes
+      for (int q = 0; q < P.count; ++q) {
+        tma_prefetch_desc(&P.w[q]);
+        tma_prefetch_desc(&P.x[q]);
+      }
+      int it = it0, rb = rb0, kst = k0;
+      auto advance = [&]() {
+        if (++kst == P.it[it].C) {
+          kst = 0;
+          if (++rb == P.it[it].RB) {
+            rb = 0;
+            ++it;
+          }
+        }
+      };
+      auto load_w = [&](int i) {
+        tma_load_2d(stg + (i % P.ring) * P.stage, &P.w[it], &full[i % P.ring], kst * 128, rb * kBRows);
+      };
+      const bool skipx = skip_x_loads();  // failure-path test hook: never set in normal use
+      auto load_x = [&](int i) {
+        if (skipx) return;
+        uint8_t* dst = stg + (i % P.ring) * P.stage + kDWBytes;
+#pragma unroll
+        for (int hb = 0; hb < F::kKB / 4; ++hb)
+          tma_load_3d(dst + hb * P.xhalf, &P.x[it], &full[i % P.ring], 0, kst * F::kKB + 4 * hb, 0);
+      };
+      const int pre = nst < P.ring ? nst : P.ring;
+      for (int i = 0; i < pre; ++i) {  // weights are model constants: before the wait
+        mbar_arrive_expect_tx(&full[i], tx);
+        load_w(i);
+        advance();
+      }
+      pdl_wait_prior_grids();  // the activations may come from the previous kernel
+      it = it0, rb = rb0, kst = k0;
+      for (int i = 0; i < pre; ++i) {
+        load_x(i);
+        advance();
+      }
+      for (int i = pre; i < nst; ++i) {
+        const int slot = i % P.ring;
+        if (!mbar_wait(&empty[slot], static_cast<uint32_t>((i / P.ring) - 1) & 1u)) {
+          flags[0] = 1;
+          break;
+        }
+        mbar_arrive_expect_tx(&full[slot], tx);
+        load_w(i);
+        load_x(i);
+        advance();
+      }
+    }
+    return;
+  }
+
+  // ====================================================================== consumer warps
+  const int g = lane >> 2, t = lane & 3;
+  const int rs = warp & (kDRowSets - 1), hi = warp / kDRowSets;  // hi: K half (M <= 8) or token group
+  const int sub_lo = NT == 1 ? hi : 0, sub_hi = NT == 1 ? hi + 1 : 2;
+  const int Tb = TW < NT ? hi : 0;
+  bool tokv[TW];
+#pragma unroll
+  for (int T = 0; T < TW; ++T) tokv[T] = 8 * (Tb + T) + g < P.M;
+  const int gp = (g >> 1) | ((g & 1) << 2);
+  const int rw = rs * 16 * kDRT + gp;
+  const DecLane L{g, t, gp, rw, sub_lo, sub_hi, Tb};
+  const int e = threadIdx.x;          // epilogue thread: row e % 128, tokens e / 128 + step
+  const int er = e & (kBRows - 1);
+
+  float acc[kDRT][TW][4];
+  auto zero_acc = [&]() {
+#pragma unroll
+    for (int rt = 0; rt < kDRT; ++rt)
+#pragma unroll
+      for (int T = 0; T < TW; ++T)
+#pragma unroll
+        for (int ci = 0; ci < 4; ++ci) acc[rt][T][ci] = 0.0f;
+  };
+  zero_acc();
+
+  int it = it0, rb = rb0, kst = k0;
+  bool ok = true;
+  float ep_s = 1.0f, ep_b = 0.0f;  // this thread's epilogue row: scale (ternary) and bias
+  pdl_wait_prior_grids();          // x, y and the workspace belong to the previous kernel until now
+  for (int i = 0; i < nst; ++i) {
+    const BatchItem& I = P.it[it];
+    const int64_t row0 = static_cast<int64_t>(rb) * kBRows;
+    if (i == 0 || kst == 0) {  // a row block starts: fetch its epilogue constants early
+      const int64_t n = row0 + er;
+      ep_s = 1.0f;
+      ep_b = 0.0f;
+      if (n < I.N) {
+        if (!kInt4) ep_s = __half2float(I.sc[n]);
+        if (I.bias) ep_b = __half2float(I.bias[n]);
+      }
+    }
+    const int slot = i % P.ring;
+    if (ok) ok = mbar_wait_warp(&full[slot], static_cast<uint32_t>(i / P.ring) & 1u);
+    if (ok) {
+      dec_stage<kInt4, NT, TW>(acc, stg + slot * P.stage, P.xhalf, L, tokv, static_cast<int64_t>(kst) * 2, row0,
+                               I.N, I.sc, I.zp, I.K >> 7);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot]);
+    } else {
+      flags[0] = 1;  // a wait ran out (recorded in the device status word): results are void
+    }
+
+    if (kst == I.C - 1 || i == nst - 1) {
+      // ---------------------------------------------------------------- finish the row block
+      float v[kDRT][TW][4];
+      dec_values<kInt4, TW>(acc, v);
+      zero_acc();
+      // this CTA's sum over its stages of the block, [token][row] in `res`; for M <= 8 the two
+      // K halves (warps 4-7, then 0-3) are added in a fixed order
+      if (NT == 1 && hi == 0) named_barrier_sync(1, kEp);
+#pragma unroll
+      for (int rt = 0; rt < kDRT; ++rt)
+#pragma unroll
+        for (int T = 0; T < TW; ++T)
+#pragma unroll
+          for (int ci = 0; ci < 4; ++ci) {
+            float* dst = res + (8 * (Tb + T) + 2 * t + (ci & 1)) * kBResPitch + rw + 16 * rt + 8 * (ci >> 1);
+            if (NT == 1 && hi == 0)
+              *dst += v[rt][T][ci];
+            else
+              *dst = v[rt][T][ci];
+          }
+      if (NT == 1 && hi == 1) named_barrier_sync(1, kEp);
+      named_barrier_sync(1, kEp);
+
+      const int64_t gB0 = I.begin + static_cast<int64_t>(rb) * I.C;  // the block's stages [gB0, gB1)
+      const int64_t gB1 = gB0 + I.C;
+      const bool whole = gB0 >= s0 && gB1 <= s1;
+      const bool abort = flags[0] != 0;
+      const int64_t n = row0 + er;
+      auto out = [&](float acc_v, int tok) {
+        const float r = kInt4 ? acc_v + ep_b : fmaf(acc_v, ep_s, ep_b);
+        I.y[static_cast<int64_t>(tok) * I.N + n] = __float2half_rn(r);
+      };
+      if (!abort && whole) {
+        if (n < I.N)
+          for (int tok = e >> 7; tok < P.M; tok += kEp / kBRows) out(res[tok * kBResPitch + er], tok);
+      } else if (!abort) {
+        // split block: my partial to my slot, count in; the last contributor sums the slots
+        const int cf = range_owner(gB0, P.T, P.G), cl = range_owner(gB1 - 1, P.T, P.G);
+        float* mine = P.slots + (2 * static_cast<int64_t>(c) + (gB0 <= s0 ? 0 : 1)) * 16 * kBRows;
+        for (int tok = e >> 7; tok < P.M; tok += kEp / kBRows) mine[tok * kBRows + er] = res[tok * kBResPitch + er];
+        named_barrier_sync(1, kEp);
+        if (e == 0) {
+          __threadfence();
+          const int old = atomicAdd(&P.counters[cf], 1);
+          const int last = old == cl - cf;
+          if (last) __threadfence();
+          flags[1] = last;
+        }
+        named_barrier_sync(1, kEp);
+        if (flags[1]) {
+          if (n < I.N)
+            for (int tok = e >> 7; tok < P.M; tok += kEp / kBRows) {
+              float sum = 0.0f;
+              for (int cc = cf; cc <= cl; ++cc) {  // K order: deterministic
+                const int64_t sl = 2 * static_cast<int64_t>(cc) + (gB0 <= range_begin(cc, P.T, P.G) ? 0 : 1);
+                sum += __ldcg(P.slots + sl * 16 * kBRows + tok * kBRows + er);
+              }
+              out(sum, tok);
+            }
+          if (e == 0) P.counters[cf] = 0;  // ready for the next call
+        }
+      }
+      named_barrier_sync(1, kEp);  // `res` and the flag are free again
+    }
+    if (++kst == I.C) {
+      kst = 0;
+      if (++rb == I.RB) {
+        rb = 0;
+        ++it;
+      }
+    }
+  }
+}
+
+template <bool kInt4>
+__global__ void __maxnreg__(96) batch_decode_kernel_m8(const __grid_constant__ BatchParams P) {
+  batch_body<kInt4, 1, 1>(P);
+}
+
+template <bool kInt4>
+__global__ void __launch_bounds__(DecWarps<2, 2>::kThreads, 2) batch_decode_kernel_m16(const __grid_constant__ BatchParams P) {
+  batch_body<kInt4, 2, 2>(P);
+}
+
+// ---------------------------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------------------------
+int64_t batch_workspace_bytes() { return batch_workspace_bytes_for(kBCtasPerSm * current_device_info().num_sms); }
+
+template <bool kInt4>
+static cudaError_t launch_batch_t(const BatchLinear* items, int count, int64_t M, void* ws, int64_t ws_bytes,
+                                  cudaStream_t s) {
+  using F = DecFmt<kInt4>;
+  using L = BatchLayout<kInt4>;
+  if (count < 1 || count > kBMaxItems || M < 1 || M > 16) return cudaErrorInvalidValue;
+  const DeviceInfo di = current_device_info();
+  BatchParams P;
+  P.count = count;
+  P.M = static_cast<int>(M);
+  int64_t T = 0;
+  for (int q = 0; q < count; ++q) {
+    const BatchLinear& b = items[q];
+    BatchItem& I = P.it[q];
+    I.sc = b.sc;
+    I.zp = b.zp;
+    I.bias = b.bias;
+    I.y = b.y;
+    I.N = b.N;
+    I.K = b.K;
+    I.C = static_cast<int>((b.K + F::kStageK - 1) / F::kStageK);
+    I.RB = static_cast<int>((b.N + kBRows - 1) / kBRows);
+    I.begin = T;
+    T += static_cast<int64_t>(I.C) * I.RB;
+    const int64_t kbytes = kInt4 ? b.K / 2 : b.K / 4;
+    if (!make_tmap_2d(&P.w[q], CU_TENSOR_MAP_DATA_TYPE_UINT8, b.w, static_cast<uint64_t>(kbytes),
+                      static_cast<uint64_t>(b.N), static_cast<uint64_t>(kbytes), 128, kBRows,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+    const uint64_t dims[3] = {64, static_cast<uint64_t>(b.K / 64), static_cast<uint64_t>(M)};
+    const uint64_t strides[2] = {128, static_cast<uint64_t>(b.K) * 2};
+    const uint32_t box[3] = {64, 4, static_cast<uint32_t>(M)};
+    if (!make_tmap_3d(&P.x[q], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, b.x, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
+  for (int q = count; q < kBMaxItems; ++q) {
+    P.w[q] = P.w[0];
+    P.x[q] = P.x[0];
+    P.it[q] = P.it[0];
+    P.it[q].begin = T;  // never reached
+  }
+  const int Gmax = kBCtasPerSm * di.num_sms;
+  if (ws_bytes < batch_workspace_bytes_for(Gmax)) return cudaErrorInvalidValue;
+  P.T = T;
+  P.G = static_cast<int>(T < Gmax ? T : Gmax);
+  P.xhalf = ((static_cast<int>(M) * 4 * 128 + 1023) / 1024) * 1024;
+  P.stage = kDWBytes + (F::kKB / 4) * P.xhalf;
+  int ring = kDMaxRing;
+  while (ring > 2 && L::bytes(ring, P.stage) > kDSmemBudget) --ring;
+  P.ring = ring;
+  const int smem = L::bytes(ring, P.stage);
+  if (smem > kDSmemBudget) return cudaErrorInvalidValue;
+  P.counters = reinterpret_cast<int*>(ws);
+  P.slots = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + batch_counter_bytes(Gmax));
+
+  const bool m16 = M > 8;
+  auto* kern = m16 ? batch_decode_kernel_m16<kInt4> : batch_decode_kernel_m8<kInt4>;
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), kDSmemBudget);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(P.G), 1, 1);
+  cfg.blockDim = dim3(m16 ? DecWarps<2, 2>::kThreads : DecWarps<1, 1>::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, P);
+}
+
+cudaError_t launch_tq_gemm_batch(const BatchLinear* items, int count, int64_t M, void* ws, int64_t ws_bytes,
+                                 cudaStream_t s) {
+  return launch_batch_t<false>(items, count, M, ws, ws_bytes, s);
+}
+
+cudaError_t launch_w4g_gemm_batch(const BatchLinear* items, int count, int64_t M, void* ws, int64_t ws_bytes,
+                                  cudaStream_t s) {
+  return launch_batch_t<true>(items, count, M, ws, ws_bytes, s);
+}
+
+}  // namespace tq

@@ -181,11 +181,22 @@ cudaError_t launch_tq_pack(const void* w, bool w_f16, uint8_t* packed, uint16_t*
                            int64_t K, cudaStream_t s);
 cudaError_t launch_w4g_pack(const void* w, bool w_f16, int32_t* qweight, uint16_t* scales,
                             int64_t N, int64_t K, cudaStream_t s);
+// General W4 pack: zeros != null -> asymmetric (zero-point per group); perm != null -> the groups
+// are the columns perm[128 g ..] (activation order); g_idx (nullable) receives each column's group.
+cudaError_t launch_w4g_pack_ex(const void* w, bool w_f16, const int32_t* perm, int32_t* qweight, uint16_t* scales,
+                               uint8_t* zeros, int32_t* g_idx, int64_t N, int64_t K, cudaStream_t s);
+cudaError_t launch_permute_cols(const uint16_t* x, const int32_t* perm, uint16_t* out, int64_t M, int64_t K,
+                                cudaStream_t s);
+cudaError_t launch_repack_act_order(const int32_t* qweight, const int32_t* perm, int32_t* out, int64_t N,
+                                    int64_t K, cudaStream_t s);
+cudaError_t launch_iota_groups(int32_t* g_idx, int64_t K, cudaStream_t s);
 cudaError_t launch_tq_gemm_generic(const __half* x, const uint8_t* packed, const __half* scale,
                                    const __half* bias, __half* y, int64_t M, int64_t N, int64_t K,
                                    cudaStream_t s);
+// W4A16 GEMMs: zeros == null is the symmetric format (What = s (u - 8)); otherwise
+// What = s (u - zeros[n, k / 128]).
 cudaError_t launch_w4g_gemm_generic(const __half* x, const int32_t* qweight, const __half* scales,
-                                    const __half* bias, __half* y, int64_t M, int64_t N,
+                                    const uint8_t* zeros, const __half* bias, __half* y, int64_t M, int64_t N,
                                     int64_t K, cudaStream_t s);
 cudaError_t launch_tq_validate(const uint8_t* packed, int64_t N, int64_t K, int* bad,
                                cudaStream_t s);
@@ -207,14 +218,33 @@ cudaError_t launch_w4g_gemm_decode_group(const __half* x, int count, const int32
                                          __half* const* y, const int64_t* N, int64_t M, int64_t K,
                                          cudaStream_t s);
 cudaError_t launch_w4g_gemm_decode(const __half* x, const int32_t* qweight, const __half* scales,
-                                   const __half* bias, __half* y, int64_t M, int64_t N, int64_t K,
-                                   cudaStream_t s);
+                                   const uint8_t* zeros, const __half* bias, __half* y, int64_t M, int64_t N,
+                                   int64_t K, cudaStream_t s);
 cudaError_t launch_tq_gemm_prefill(const __half* x, const uint8_t* packed, const __half* scale,
                                    const __half* bias, __half* y, int64_t M, int64_t N, int64_t K,
                                    cudaStream_t s);
 cudaError_t launch_w4g_gemm_prefill(const __half* x, const int32_t* qweight, const __half* scales,
-                                    const __half* bias, __half* y, int64_t M, int64_t N,
+                                    const uint8_t* zeros, const __half* bias, __half* y, int64_t M, int64_t N,
                                     int64_t K, cudaStream_t s);
+
+// Work list of the persistent batch decode kernel (tq_batch.cu): independent linears sharing M.
+struct BatchLinear {
+  const __half* x;     // [M, K]
+  const void* w;       // ternary uint8 [N, K/4] or W4A16 int32 [N, K/8]
+  const __half* sc;    // ternary [N]; W4A16 [N, K/128]
+  const __half* bias;  // [N] or null
+  __half* y;           // [M, N]
+  int64_t N, K;
+  const uint8_t* zp;   // W4A16 zero-points [N, K/128], or null (symmetric)
+};
+constexpr int kBatchMaxItems = 8;
+constexpr int64_t kBatchMaxM = 16;
+// Workspace bytes the batch kernel needs on the current device.
+int64_t batch_workspace_bytes();
+cudaError_t launch_tq_gemm_batch(const BatchLinear* items, int count, int64_t M, void* ws, int64_t ws_bytes,
+                                 cudaStream_t s);
+cudaError_t launch_w4g_gemm_batch(const BatchLinear* items, int count, int64_t M, void* ws, int64_t ws_bytes,
+                                  cudaStream_t s);
 
 // Encode a 2-D row-major tensor map (driver entry point fetched through the runtime, so the
 // library does not link libcuda).  Returns false on failure.
@@ -225,6 +255,9 @@ bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
 // 3-D variant: dims[0] innermost (elements), strides_bytes[i] = stride of dimension i + 1.
 bool make_tmap_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, const uint64_t dims[3],
                   const uint64_t strides_bytes[2], const uint32_t box[3], CUtensorMapSwizzle swizzle);
+
+// Enqueue the empty kernel that separates a write of model constants from a following GEMM.
+cudaError_t after_constants_written(cudaStream_t s);
 
 // Set the dynamic shared-memory limit of `func` on the current device once.
 cudaError_t ensure_smem_attr(const void* func, int bytes);

@@ -8,16 +8,14 @@
 // of packed codes; [TQ] §4.2: codes are decoded into fp16 tensor-core fragments, accumulated in
 // fp32, and the per-row scale is applied after the MMA.
 //
-// Work layout.  One CTA = one block of output rows (127 ternary rows plus one virtual row, or 128
-// W4A16 rows) x one K-slice; a cluster of S CTAs (S <= 8) covers the whole K of its rows and
+// Work layout.  One CTA = one block of 128 output rows x one K-slice; a cluster of S CTAs (S <= 8) covers the whole K of its rows and
 // reduces through distributed shared memory in a fixed order (deterministic, no global scratch).
 // A stage is 128 bytes of every packed row (512 ternary or 256 INT4 codes) plus the activations
 // of those k for all M tokens.  Per CTA:
 //   * the last warp (producer) streams each stage with TMA into a ring: the 128-row x 128-byte packed
 //     tile (issued before griddepcontrol.wait, weights never depend on the previous kernel) and
 //     the activations, one 64-element block x M tokens per box (issued after it), both
-//     128-byte swizzled so that every 16-byte read below is bank-conflict free.  For W4A16 it
-//     also sums each 128-wide group of x per token;
+//     128-byte swizzled so that every 16-byte read below is bank-conflict free;
 //   * consumers: warp w owns rows 32 (w & 3) .. +31 (two 16-row MMA tiles).  For M <= 8 there
 //     are eight, warp w taking the K half w >> 2 of every stage (the two halves are added in
 //     shared memory, in a fixed order, at the end); for M > 8 there are four, each holding both
@@ -27,18 +25,19 @@
 //     shared memory (byte permutes into the k order the decode produces, see below); with two
 //     row tiles per warp one fragment feeds four MMAs.
 //
-// In-register decode ("subnormal" trick).  ANDing a packed 32-bit word with 0x00030003 << 2p
-// leaves, in each fp16 half, the code at bits 2p..2p+1: the exact value c * 2^(2p-24) (fp16
-// subnormals for p <= 4, and still exactly linear for p = 5 where the code fills the two lowest
-// exponent bits).  Positions 6, 7 are shifted down by 12 first.  So one word of 16 codes costs
-// 1 shift + 8 ANDs for 8 fp16x2 registers, ~0.56 integer operations per weight.  The odd
-// positions carry an extra factor 4, folded into their activation fragments (x / 4); the
-// factors 2^-24 (position pairs 0 and 3), 2^-20 (pair 1) and 2^-16 (pair 2) are kept in three
-// accumulators and applied exactly (powers of two) after the loop.  The codes are c = w + 1, so
-// the result is sum_k c x - sum_k x; sum_k x comes out of the same MMAs as a virtual 128th row
-// whose codes are all 01 (c = 1).
-// W4A16 uses the same scheme with 4-bit fields (masks 0x000F000F / 0x00F000F0, x / 16 fold) and
-// one 128-wide quantisation group per 64-byte sub-chunk: y += s[n,g] * (2^24 * C_g - 8 sum_g x).
+// In-register decode, exact.  The MMA multiplies the weight values themselves, so the fp32
+// accumulators only ever hold partial sums of x * What (no large sum of x is formed and
+// subtracted at the end: that cancellation would cost accuracy on rows with few nonzero codes).
+//   ternary: code position p (0..7) of a 32-bit word holds the codes of k = p and k = p + 8 in
+//     its two fp16 halves.  Shifting them to bits 14-15 of each half and keeping the complement
+//     of those two bits gives the fp16 values -2 / -0 / +2 = 2 (c - 1) (the code's high bit lands
+//     on the sign): one shift and one LOP3 per register of two weights; the result is halved
+//     after the loop.  The activation fragments are x pairs (p, p + 8), picked with byte permutes.
+//   W4A16: ANDing a word with 0x000F000F (nibbles at bits 0-3) or 0x00F000F0 (bits 4-7) leaves
+//     u * 2^-24 or u * 2^-20 in each half (fp16 subnormals, exactly linear in u); one fp16x2
+//     subtraction of 8 units gives (u - 8) times that power of two exactly.  The two fields
+//     accumulate in separate chains, combined with an exact factor 16, and each 128-wide
+//     quantisation group (one 64-byte sub-chunk) is scaled as y += s[n,g] * 2^24 * sum_g (u - 8) x.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -72,7 +71,7 @@ template <bool kInt4>
 struct DecFmt {
   static constexpr int kStageK = kInt4 ? 256 : 512;  // codes per stage (128 bytes of a row)
   static constexpr int kKB = kStageK / 64;           // 64-element activation blocks per stage
-  static constexpr int kRows = kInt4 ? 128 : 127;    // real output rows per CTA
+  static constexpr int kRows = 128;                   // output rows per CTA
 };
 
 constexpr int kDMaxGroup = 4;  // weight matrices sharing x in one launch (e.g. q, k, v)
@@ -89,6 +88,7 @@ struct DecodeArgs {
   int rb_start[kDMaxGroup + 1];     // first row block of each matrix in grid.y
   int64_t N[kDMaxGroup];
   const __half* sc[kDMaxGroup];     // ternary: scale[N]; W4A16: scales[N, K/128]
+  const uint8_t* zp[kDMaxGroup];    // W4A16 zero-points [N, K/128], or null (symmetric: 8)
   const __half* bias[kDMaxGroup];   // may be null
   __half* y[kDMaxGroup];
 };
@@ -101,12 +101,10 @@ struct DecodeMaps {
 
 template <bool kInt4>
 struct DecLayout {
-  static constexpr int kXg = kInt4 ? 2 * 16 * 4 : 0;  // W4A16 group sums of a stage [2][16]
   static constexpr int kRed = kDRedRows * 16 * 4;
-  static constexpr int kSxr = kDMaxCluster * 16 * 4;
   static constexpr int kPart = kDTile * 8 * 4;        // second K half's partials (M <= 8)
-  __host__ __device__ static constexpr int fixed() { return 1024 + kRed + kSxr + kPart + 3 * kDMaxRing * 8; }
-  __host__ __device__ static constexpr int bytes(int ring, int stage) { return fixed() + ring * (stage + kXg); }
+  __host__ __device__ static constexpr int fixed() { return 1024 + kRed + kPart + 2 * kDMaxRing * 8; }
+  __host__ __device__ static constexpr int bytes(int ring, int stage) { return fixed() + ring * stage; }
 };
 
 // Activations of a stage: one TMA box per four 64-element blocks (a ternary stage has two, a
@@ -119,18 +117,209 @@ __device__ __forceinline__ uint4 ld_x_chunk(const uint8_t* box, int row, int c) 
   return *reinterpret_cast<const uint4*>(box + row * 128 + ((c ^ (row & 7)) << 4));
 }
 
-// B fragments of one MMA pair from four activation words: even positions (x) and odd positions
-// (x times `fold`), in the k order of the decode.
-__device__ __forceinline__ void make_frag(uint32_t Pa, uint32_t Pb, uint32_t Pc, uint32_t Pd,
-                                          __half2 fold, uint32_t& e0, uint32_t& e1, uint32_t& o0,
-                                          uint32_t& o1) {
+// B fragments of one MMA pair from four activation words: the low fp16 halves (even positions)
+// and the high halves (odd positions) of (Pa, Pb) and of (Pc, Pd), in the k order of the decode.
+__device__ __forceinline__ void make_frag(uint32_t Pa, uint32_t Pb, uint32_t Pc, uint32_t Pd, uint32_t& e0,
+                                          uint32_t& e1, uint32_t& o0, uint32_t& o1) {
   e0 = __byte_perm(Pa, Pb, 0x5410);
   e1 = __byte_perm(Pc, Pd, 0x5410);
-  uint32_t u01 = __byte_perm(Pa, Pb, 0x7632), u23 = __byte_perm(Pc, Pd, 0x7632);
-  __half2 s01 = __hmul2(*reinterpret_cast<__half2*>(&u01), fold);
-  __half2 s23 = __hmul2(*reinterpret_cast<__half2*>(&u23), fold);
-  o0 = *reinterpret_cast<uint32_t*>(&s01);
-  o1 = *reinterpret_cast<uint32_t*>(&s23);
+  o0 = __byte_perm(Pa, Pb, 0x7632);
+  o1 = __byte_perm(Pc, Pd, 0x7632);
+}
+
+// One A-fragment register.  `mask` selects one code field in each fp16 half, which then holds
+// the code times the field's unit (a power of two: the pattern 0x0001 << field offset);
+// subtracting `unit` (the offset times that field unit: 1 for ternary, 8 for W4A16) leaves
+// (code - offset) * field unit, i.e. the weight value -1 / 0 / +1 or -8..7 times a power of two.
+// fp16 arithmetic is exact here: operands and result are multiples of the subnormal quantum
+// 2^-24 below 2^-12.
+__device__ __forceinline__ uint32_t dec_field(uint32_t w, uint32_t mask, uint32_t unit) {
+  uint32_t a = w & mask;
+  __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&unit));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+// Lane constants of a consumer warp: MMA fragment coordinates (g = lane / 4, t = lane % 4), the
+// stored row of tile row g (gp) and of this warp's first tile row (rw), the sub-chunks of a stage
+// this warp covers and its first token group.
+struct DecLane {
+  int g, t, gp, rw, sub_lo, sub_hi, Tb;
+};
+
+// One stage of the consumer loop: this warp's rows (two 16-row tiles) x its sub-chunks of the
+// stage's 128 bytes per row, for its token groups, accumulated into `acc` (ternary: three
+// exact power-of-two classes; W4A16: one, the group scales already applied).  `st` is the
+// stage's weight tile, followed by its activation boxes (`xhalf` bytes each).  W4A16 needs the
+// first quantisation group of the stage (`gi_base`), the block's first row and the scales.
+// One ternary A-fragment register: code position p (0..7) of a packed word, i.e. the codes of
+// k = p (low fp16 half) and k = p + 8 (high half) of the word's 16.  Shifting the code to bits
+// 14-15 of each half puts its high bit b1 at the sign bit and its low bit b0 at the top exponent
+// bit; complementing both and clearing the rest leaves the fp16 value
+//   c = 0b00 -> 0xC000 = -2,  c = 0b01 -> 0x8000 = -0,  c = 0b10 -> 0x4000 = +2,
+// i.e. exactly 2 (c - 1): one shift and one LOP3 per two weights, no arithmetic.  (Code 0b11 is
+// invalid and decodes to +0.)
+__device__ __forceinline__ uint32_t dec_tq_pos(uint32_t w, int p) {
+  const uint32_t s = p == 7 ? w : (w << (14 - 2 * p));
+  return ~s & 0xC000C000u;
+}
+
+template <bool kInt4, int NT, int TW>
+__device__ __forceinline__ void dec_stage(float (&acc)[kDRT][TW][4], const uint8_t* st, int xhalf,
+                                          const DecLane& L, const bool (&tokv)[TW], int64_t gi_base,
+                                          int64_t row0, int64_t Nm, const __half* scm, const uint8_t* zpm,
+                                          int64_t G) {
+  const int g = L.g, t = L.t, gp = L.gp, rw = L.rw, Tb = L.Tb, sub_lo = L.sub_lo, sub_hi = L.sub_hi;
+  const uint8_t* xs = st + kDWBytes;
+#pragma unroll 1
+  for (int sub = sub_lo; sub < sub_hi; ++sub) {
+    const int chunk = sub * 4 + t;  // this lane's 16 bytes of the packed rows
+    // rows rw + 16 rt + 8 hr all have (row & 7) == gp: swizzled chunk position chunk ^ gp
+    uint32_t w[kDRT][2][4];
+#pragma unroll
+    for (int rt = 0; rt < kDRT; ++rt)
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        uint4 U = *reinterpret_cast<const uint4*>(st + (rw + 16 * rt + 8 * hr) * 128 + ((chunk ^ gp) << 4));
+        w[rt][hr][0] = U.x;
+        w[rt][hr][1] = U.y;
+        w[rt][hr][2] = U.z;
+        w[rt][hr][3] = U.w;
+      }
+    if (!kInt4) {
+      // the 64 codes of the chunk are k = 64*chunk + 0..63: activation block `chunk`, i.e.
+      // block t of the box of sub-chunk `sub`
+      const uint8_t* xbox = xs + sub * xhalf;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        // P[T][j] = x[8(Tb+T)+g][64*chunk + 32h + 2j .. +1]
+        uint32_t P[TW][16];
+#pragma unroll
+        for (int T = 0; T < TW; ++T)
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) {
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (tokv[T]) v = ld_x_chunk(xbox, 4 * (8 * (Tb + T) + g) + t, 4 * h + jj);
+            P[T][4 * jj] = v.x;
+            P[T][4 * jj + 1] = v.y;
+            P[T][4 * jj + 2] = v.z;
+            P[T][4 * jj + 3] = v.w;
+          }
+        // position p of words 2h (k = 64 chunk + 32h + p, + p + 8) and 2h + 1 (+ 16 + p, + 24 + p):
+        // x pairs (p, p + 8) are the even (p even) or odd halves of P[p / 2] and P[p / 2 + 4]
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+          const uint32_t sel = (p & 1) ? 0x7632u : 0x5410u;
+          uint32_t b0[TW], b1[TW];
+#pragma unroll
+          for (int T = 0; T < TW; ++T) {
+            b0[T] = __byte_perm(P[T][p >> 1], P[T][(p >> 1) + 4], sel);
+            b1[T] = __byte_perm(P[T][8 + (p >> 1)], P[T][12 + (p >> 1)], sel);
+          }
+#pragma unroll
+          for (int rt = 0; rt < kDRT; ++rt) {
+            const uint32_t a0 = dec_tq_pos(w[rt][0][2 * h], p), a1 = dec_tq_pos(w[rt][1][2 * h], p);
+            const uint32_t a2 = dec_tq_pos(w[rt][0][2 * h + 1], p), a3 = dec_tq_pos(w[rt][1][2 * h + 1], p);
+#pragma unroll
+            for (int T = 0; T < TW; ++T) mma_16816(acc[rt][T], a0, a1, a2, a3, b0[T], b1[T]);
+          }
+        }
+      }
+    } else {
+      // the group scales of this lane's rows, requested before the MMAs that they follow
+      const int64_t gi = gi_base + sub;
+      float sg[kDRT][2];
+      uint32_t zz[kDRT][2];  // zero-point of each row's group (8 for the symmetric format)
+#pragma unroll
+      for (int rt = 0; rt < kDRT; ++rt)
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+          const int64_t n = row0 + rw + 16 * rt + 8 * hr;
+          // groups past K (a zero-filled half stage) contribute nothing
+          const bool in = n < Nm && gi < G;
+          sg[rt][hr] = in ? __half2float(scm[n * G + gi]) : 0.0f;
+          zz[rt][hr] = (zpm && in) ? static_cast<uint32_t>(zpm[n * G + gi]) : 8u;
+        }
+      // the 32 codes of the chunk are k = 32*chunk + 0..31: half (chunk & 1) of activation
+      // block chunk / 2, its 16-byte chunks 4*(chunk & 1) + 0..3
+      uint32_t P[TW][16];
+#pragma unroll
+      for (int T = 0; T < TW; ++T)
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          uint4 v = make_uint4(0u, 0u, 0u, 0u);
+          if (tokv[T]) v = ld_x_chunk(xs, 4 * (8 * (Tb + T) + g) + (chunk >> 1), 4 * (chunk & 1) + jj);
+          P[T][4 * jj] = v.x;
+          P[T][4 * jj + 1] = v.y;
+          P[T][4 * jj + 2] = v.z;
+          P[T][4 * jj + 3] = v.w;
+        }
+      float cg[2][kDRT][TW][4];  // two chains: nibble fields at bits 0-3 (unit 2^-24) and 4-7 (2^-20)
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int rt = 0; rt < kDRT; ++rt)
+#pragma unroll
+          for (int T = 0; T < TW; ++T)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) cg[j][rt][T][c] = 0.0f;
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int s2 = 0; s2 < 2; ++s2) {
+          uint32_t be0[TW], be1[TW], bo0[TW], bo1[TW];
+#pragma unroll
+          for (int T = 0; T < TW; ++T)
+            make_frag(P[T][8 * h + s2], P[T][8 * h + 2 + s2], P[T][8 * h + 4 + s2], P[T][8 * h + 6 + s2], be0[T],
+                      be1[T], bo0[T], bo1[T]);
+#pragma unroll
+          for (int rt = 0; rt < kDRT; ++rt) {
+            const uint32_t x0 = w[rt][0][2 * h] >> (8 * s2), x1 = w[rt][1][2 * h] >> (8 * s2);
+            const uint32_t x2 = w[rt][0][2 * h + 1] >> (8 * s2), x3 = w[rt][1][2 * h + 1] >> (8 * s2);
+#pragma unroll
+            for (int cls = 0; cls < 2; ++cls) {
+              // u at bits 0-3 (value u 2^-24) or 4-7 (u 2^-20); minus z units: (u - z) exactly
+              const uint32_t mk = cls ? 0x00F000F0u : 0x000F000Fu;
+              const uint32_t unit = cls ? 0x00100010u : 0x00010001u;
+              const uint32_t zg = zz[rt][0] * unit, zh = zz[rt][1] * unit;  // rows g and g + 8
+              const uint32_t d0 = dec_field(x0, mk, zg), d1 = dec_field(x1, mk, zh);
+              const uint32_t d2 = dec_field(x2, mk, zg), d3 = dec_field(x3, mk, zh);
+#pragma unroll
+              for (int T = 0; T < TW; ++T)
+                mma_16816(cg[cls][rt][T], d0, d1, d2, d3, cls ? bo0[T] : be0[T], cls ? bo1[T] : be1[T]);
+            }
+          }
+        }
+#pragma unroll
+      for (int rt = 0; rt < kDRT; ++rt) {
+        // the group's sum of (u - 8) x in units of 2^-24: the second field's chain times 16
+        // (exact powers of two)
+        const float s0u = sg[rt][0] * 16777216.0f, s1u = sg[rt][1] * 16777216.0f;
+#pragma unroll
+        for (int T = 0; T < TW; ++T) {
+          float c4[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) c4[c] = fmaf(cg[1][rt][T][c], 16.0f, cg[0][rt][T][c]);
+          acc[rt][T][0] = fmaf(s0u, c4[0], acc[rt][T][0]);
+          acc[rt][T][1] = fmaf(s0u, c4[1], acc[rt][T][1]);
+          acc[rt][T][2] = fmaf(s1u, c4[2], acc[rt][T][2]);
+          acc[rt][T][3] = fmaf(s1u, c4[3], acc[rt][T][3]);
+        }
+      }
+    }
+  }
+}
+
+// Final fp32 values of a warp's tiles: ternary accumulates 2 (c - 1) x (the decoded weights are
+// -2, -0, +2), halved here exactly; W4A16 has the group scales applied already.  Rows
+// rw + 16 rt + 8 (ci >> 1), tokens 8 (Tb + T) + 2t + (ci & 1).
+template <bool kInt4, int TW>
+__device__ __forceinline__ void dec_values(const float (&acc)[kDRT][TW][4], float (&v)[kDRT][TW][4]) {
+#pragma unroll
+  for (int rt = 0; rt < kDRT; ++rt)
+#pragma unroll
+    for (int T = 0; T < TW; ++T)
+#pragma unroll
+      for (int ci = 0; ci < 4; ++ci) v[rt][T][ci] = kInt4 ? acc[rt][T][ci] : 0.5f * acc[rt][T][ci];
 }
 
 template <bool kInt4, int NT, int TW>
@@ -143,13 +332,10 @@ __device__ __forceinline__ void decode_gemm_body(const DecodeMaps& maps, const D
   // space visible to the compiler (plain ld/st.shared instead of generic accesses)
   uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* stg = base;                                                  // ring x [weights | x]
-  float* xg = reinterpret_cast<float*>(stg + a.ring * a.stage);         // ring x [2][16]
-  float* red = xg + a.ring * (L::kXg / 4);                              // [S][16][own_cap]
-  float* sxr = red + kDRedRows * 16;                                    // [S][16] slice sums of x
-  float* part = sxr + kDMaxCluster * 16;                                // [128 rows][8 tokens]
+  float* red = reinterpret_cast<float*>(stg + a.ring * a.stage);        // [S][16][own_cap]
+  float* part = red + kDRedRows * 16;                                   // [128 rows][8 tokens]
   uint64_t* full = reinterpret_cast<uint64_t*>(part + kDTile * 8);
-  uint64_t* xready = full + kDMaxRing;  // W4A16 group sums of the stage written
-  uint64_t* empty = xready + kDMaxRing;
+  uint64_t* empty = full + kDMaxRing;
 
   pdl_allow_dependents();
 
@@ -166,6 +352,7 @@ __device__ __forceinline__ void decode_gemm_body(const DecodeMaps& maps, const D
   const CUtensorMap* tmap = &maps.m[grp];
   const int64_t Nm = a.N[grp];
   const __half* scm = a.sc[grp];
+  const uint8_t* zpm = a.zp[grp];
   const __half* biasm = a.bias[grp];
   __half* ym = a.y[grp] + static_cast<int64_t>(blockIdx.z) * 16 * a.N[grp];
   const int st_begin = static_cast<int>((static_cast<int64_t>(rank) * a.C) / a.S);
@@ -181,7 +368,6 @@ __device__ __forceinline__ void decode_gemm_body(const DecodeMaps& maps, const D
   if (threadIdx.x == 0) {
     for (int i = 0; i < a.ring; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&xready[i], 32);
       mbar_init(&empty[i], W::kCons);
     }
     fence_mbar_init();
@@ -208,7 +394,9 @@ __device__ __forceinline__ void decode_gemm_body(const DecodeMaps& maps, const D
       tma_load_2d(stg + (i % a.ring) * a.stage, tmap, &full[i % a.ring], (st_begin + i) * 128,
                   static_cast<int>(row0));
     };
+    const bool skipx = skip_x_loads();  // failure-path test hook: never set in normal use
     auto load_x = [&](int i) {
+      if (skipx) return;
       uint8_t* dst = stg + (i % a.ring) * a.stage + kDWBytes;
 #pragma unroll
       for (int hb = 0; hb < F::kKB / 4; ++hb)
@@ -227,251 +415,48 @@ __device__ __forceinline__ void decode_gemm_body(const DecodeMaps& maps, const D
     pdl_wait_prior_grids();  // the activations may come from the previous kernel
     if (lane == 0)
       for (int i = 0; i < pre; ++i) load_x(i);
-    if (!kInt4) {
-      if (lane == 0)
-        for (int j = a.ring; j < nst; ++j) {
-          const int slot = j % a.ring;
-          if (!mbar_wait(&empty[slot], static_cast<uint32_t>((j / a.ring) - 1) & 1u)) break;
-          mbar_arrive_expect_tx(&full[slot], tx);
-          load_w(j);
-          load_x(j);
-        }
-    } else {
-      // group sums: lane -> token m = lane % (8*NT), block part = lane / (8*NT)
-      constexpr int MP = 8 * NT, PARTS = 32 / MP, KBL = F::kKB / PARTS;
-      const int m = lane % MP, part = lane / MP;
-      for (int i = 0; i < nst; ++i) {
-        const int slot = i % a.ring;
-        const uint32_t ph = static_cast<uint32_t>(i / a.ring) & 1u;
-        if (!mbar_wait_warp(&full[slot], ph)) break;  // warp-uniform exit
-        const uint8_t* xs = stg + slot * a.stage + kDWBytes;
-        float ps = 0.0f;
-        if (m < Mi) {
-#pragma unroll
-          for (int bb = 0; bb < KBL; ++bb) {
-            const int b = part * KBL + bb;  // W4A16: one box, rows 4 m + b
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              const uint4 v = ld_x_chunk(xs, 4 * m + b, c);
-              const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&u[j]));
-                ps += f2.x + f2.y;
-              }
-            }
-          }
-        }
-        // a group is 128 elements = 2 blocks: combine the two parts of one group
-        if (KBL == 1) ps += __shfl_xor_sync(0xFFFFFFFFu, ps, MP);
-        const int gq = (part * KBL) >> 1;
-        if (KBL == 2 || (part & 1) == 0) xg[(slot * 2 + gq) * 16 + m] = ps;
-        mbar_arrive(&xready[slot]);
-        const int j = i + a.ring;
-        if (j < nst) {
-          if (!mbar_wait_warp(&empty[slot], ph)) break;
-          if (lane == 0) {
-            mbar_arrive_expect_tx(&full[slot], tx);
-            load_w(j);
-            load_x(j);
-          }
-        }
+    if (lane == 0)
+      for (int j = a.ring; j < nst; ++j) {
+        const int slot = j % a.ring;
+        if (!mbar_wait(&empty[slot], static_cast<uint32_t>((j / a.ring) - 1) & 1u)) break;
+        mbar_arrive_expect_tx(&full[slot], tx);
+        load_w(j);
+        load_x(j);
       }
-    }
   } else {
     // ================================================================== consumer warps
-    // accumulator groups by exact power-of-two factor: pairs 0 and 3 (2^-24), 1 (2^-20), 2 (2^-16)
-    constexpr int NG = kInt4 ? 1 : 3;
     const int rs = warp & (kDRowSets - 1), hi = warp / kDRowSets;  // hi: K half or token group
     const int sub_lo = NT == 1 ? hi : 0, sub_hi = NT == 1 ? hi + 1 : 2;
     const int Tb = TW < NT ? hi : 0;  // first token group of this warp
     bool tokv[TW];  // this lane's token 8(Tb+T) + g (B column g of token group Tb+T) exists
 #pragma unroll
     for (int T = 0; T < TW; ++T) tokv[T] = 8 * (Tb + T) + g < Mi;
-    float acc[NG][kDRT][TW][4];
+    float acc[kDRT][TW][4];
 #pragma unroll
-    for (int q = 0; q < NG; ++q)
+    for (int rt = 0; rt < kDRT; ++rt)
 #pragma unroll
-      for (int rt = 0; rt < kDRT; ++rt)
+      for (int T = 0; T < TW; ++T)
 #pragma unroll
-        for (int T = 0; T < TW; ++T)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) acc[q][rt][T][c] = 0.0f;
-    const __half2 fold = kInt4 ? __floats2half2_rn(0.0625f, 0.0625f) : __floats2half2_rn(0.25f, 0.25f);
+        for (int c = 0; c < 4; ++c) acc[rt][T][c] = 0.0f;
     // MMA tile row g is stored row gp of its group of eight, gp = (g >> 1) | (g & 1) << 2: the
     // eight lanes of a quarter warp then read rows of different swizzle phases (conflict free)
     const int gp = (g >> 1) | ((g & 1) << 2);
     const int rw = rs * 16 * kDRT + gp;  // row of tile 0, lower half; tile rt adds 16 rt, upper +8
-    // ternary: tile row 127 is the virtual all-01 row (its result is sum_k x)
-    const bool virt = !kInt4 && rw + 16 * (kDRT - 1) + 8 == kDTile - 1;
     const int64_t G = a.K >> 7;
+    const DecLane L{g, t, gp, rw, sub_lo, sub_hi, Tb};
     pdl_wait_prior_grids();  // block (not poll) until the previous kernel is done
     for (int i = 0; i < nst; ++i) {
       const int slot = i % a.ring;
       const uint32_t ph = static_cast<uint32_t>(i / a.ring) & 1u;
       if (!mbar_wait_warp(&full[slot], ph)) break;  // warp-uniform exit
       const uint8_t* st = stg + slot * a.stage;
-      const uint8_t* xs = st + kDWBytes;
-#pragma unroll 1
-      for (int sub = sub_lo; sub < sub_hi; ++sub) {
-        const int chunk = sub * 4 + t;  // this lane's 16 bytes of the packed rows
-        // rows rw + 16 rt + 8 hr all have (row & 7) == gp: swizzled chunk position chunk ^ gp
-        uint32_t w[kDRT][2][4];
-#pragma unroll
-        for (int rt = 0; rt < kDRT; ++rt)
-#pragma unroll
-          for (int hr = 0; hr < 2; ++hr) {
-            uint4 U = *reinterpret_cast<const uint4*>(st + (rw + 16 * rt + 8 * hr) * 128 + ((chunk ^ gp) << 4));
-            if (virt && rt == kDRT - 1 && hr == 1) U = make_uint4(0x55555555u, 0x55555555u, 0x55555555u, 0x55555555u);
-            w[rt][hr][0] = U.x;
-            w[rt][hr][1] = U.y;
-            w[rt][hr][2] = U.z;
-            w[rt][hr][3] = U.w;
-          }
-        if (!kInt4) {
-          // the 64 codes of the chunk are k = 64*chunk + 0..63: activation block `chunk`, i.e.
-          // block t of the box of sub-chunk `sub`
-          const uint8_t* xbox = xs + sub * a.xhalf;
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            // P[T][j] = x[8(Tb+T)+g][64*chunk + 32h + 2j .. +1]
-            uint32_t P[TW][16];
-#pragma unroll
-            for (int T = 0; T < TW; ++T)
-#pragma unroll
-              for (int jj = 0; jj < 4; ++jj) {
-                uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                if (tokv[T]) v = ld_x_chunk(xbox, 4 * (8 * (Tb + T) + g) + t, 4 * h + jj);
-                P[T][4 * jj] = v.x;
-                P[T][4 * jj + 1] = v.y;
-                P[T][4 * jj + 2] = v.z;
-                P[T][4 * jj + 3] = v.w;
-              }
-            uint32_t sh[kDRT][4];
-#pragma unroll
-            for (int rt = 0; rt < kDRT; ++rt) {
-              sh[rt][0] = w[rt][0][2 * h] >> 12;
-              sh[rt][1] = w[rt][1][2 * h] >> 12;
-              sh[rt][2] = w[rt][0][2 * h + 1] >> 12;
-              sh[rt][3] = w[rt][1][2 * h + 1] >> 12;
-            }
-#pragma unroll
-            for (int pp = 0; pp < 4; ++pp) {
-              uint32_t be0[TW], be1[TW], bo0[TW], bo1[TW];
-#pragma unroll
-              for (int T = 0; T < TW; ++T)
-                make_frag(P[T][pp], P[T][4 + pp], P[T][8 + pp], P[T][12 + pp], fold, be0[T], be1[T], bo0[T], bo1[T]);
-#pragma unroll
-              for (int q = 0; q < 2; ++q) {
-                const int p = 2 * pp + q;
-#pragma unroll
-                for (int rt = 0; rt < kDRT; ++rt) {
-                  uint32_t a0, a1, a2, a3;
-                  if (p < 6) {
-                    const uint32_t mk = 0x00030003u << (2 * p);
-                    a0 = w[rt][0][2 * h] & mk;
-                    a1 = w[rt][1][2 * h] & mk;
-                    a2 = w[rt][0][2 * h + 1] & mk;
-                    a3 = w[rt][1][2 * h + 1] & mk;
-                  } else {
-                    const uint32_t mk = (p == 6) ? 0x00030003u : 0x000C000Cu;
-                    a0 = sh[rt][0] & mk;
-                    a1 = sh[rt][1] & mk;
-                    a2 = sh[rt][2] & mk;
-                    a3 = sh[rt][3] & mk;
-                  }
-#pragma unroll
-                  for (int T = 0; T < TW; ++T)
-                    mma_16816(acc[pp == 3 ? 0 : pp][rt][T], a0, a1, a2, a3, q ? bo0[T] : be0[T], q ? bo1[T] : be1[T]);
-                }
-              }
-            }
-          }
-        } else {
-          // the 32 codes of the chunk are k = 32*chunk + 0..31: half (chunk & 1) of activation
-          // block chunk / 2, its 16-byte chunks 4*(chunk & 1) + 0..3
-          uint32_t P[TW][16];
-#pragma unroll
-          for (int T = 0; T < TW; ++T)
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-              uint4 v = make_uint4(0u, 0u, 0u, 0u);
-              if (tokv[T]) v = ld_x_chunk(xs, 4 * (8 * (Tb + T) + g) + (chunk >> 1), 4 * (chunk & 1) + jj);
-              P[T][4 * jj] = v.x;
-              P[T][4 * jj + 1] = v.y;
-              P[T][4 * jj + 2] = v.z;
-              P[T][4 * jj + 3] = v.w;
-            }
-          float cg[2][kDRT][TW][4];  // two chains (class 0 / class 1 fields)
-#pragma unroll
-          for (int j = 0; j < 2; ++j)
-#pragma unroll
-            for (int rt = 0; rt < kDRT; ++rt)
-#pragma unroll
-              for (int T = 0; T < TW; ++T)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) cg[j][rt][T][c] = 0.0f;
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int s2 = 0; s2 < 2; ++s2) {
-              uint32_t be0[TW], be1[TW], bo0[TW], bo1[TW];
-#pragma unroll
-              for (int T = 0; T < TW; ++T)
-                make_frag(P[T][8 * h + s2], P[T][8 * h + 2 + s2], P[T][8 * h + 4 + s2], P[T][8 * h + 6 + s2], fold,
-                          be0[T], be1[T], bo0[T], bo1[T]);
-#pragma unroll
-              for (int rt = 0; rt < kDRT; ++rt) {
-                const uint32_t x0 = w[rt][0][2 * h] >> (8 * s2), x1 = w[rt][1][2 * h] >> (8 * s2);
-                const uint32_t x2 = w[rt][0][2 * h + 1] >> (8 * s2), x3 = w[rt][1][2 * h + 1] >> (8 * s2);
-#pragma unroll
-                for (int cls = 0; cls < 2; ++cls) {
-                  const uint32_t mk = cls ? 0x00F000F0u : 0x000F000Fu;
-#pragma unroll
-                  for (int T = 0; T < TW; ++T)
-                    mma_16816(cg[cls][rt][T], x0 & mk, x1 & mk, x2 & mk, x3 & mk, cls ? bo0[T] : be0[T],
-                              cls ? bo1[T] : be1[T]);
-                }
-              }
-            }
-          if (sub == sub_lo) (void)mbar_wait_warp(&xready[slot], ph);
-          const int64_t gi = static_cast<int64_t>(st_begin + i) * 2 + sub;
-#pragma unroll
-          for (int rt = 0; rt < kDRT; ++rt) {
-            const int64_t n0 = row0 + rw + 16 * rt, n1 = n0 + 8;
-            // groups past K (a zero-filled half stage) contribute nothing
-            const float s0 = (n0 < Nm && gi < G) ? __half2float(scm[n0 * G + gi]) : 0.0f;
-            const float s1 = (n1 < Nm && gi < G) ? __half2float(scm[n1 * G + gi]) : 0.0f;
-#pragma unroll
-            for (int T = 0; T < TW; ++T) {
-              const float xg0 = 8.0f * xg[(slot * 2 + sub) * 16 + 8 * (Tb + T) + 2 * t];
-              const float xg1 = 8.0f * xg[(slot * 2 + sub) * 16 + 8 * (Tb + T) + 2 * t + 1];
-              float c4[4];
-#pragma unroll
-              for (int c = 0; c < 4; ++c) c4[c] = cg[0][rt][T][c] + cg[1][rt][T][c];
-              acc[0][rt][T][0] = fmaf(s0, fmaf(c4[0], 16777216.0f, -xg0), acc[0][rt][T][0]);
-              acc[0][rt][T][1] = fmaf(s0, fmaf(c4[1], 16777216.0f, -xg1), acc[0][rt][T][1]);
-              acc[0][rt][T][2] = fmaf(s1, fmaf(c4[2], 16777216.0f, -xg0), acc[0][rt][T][2]);
-              acc[0][rt][T][3] = fmaf(s1, fmaf(c4[3], 16777216.0f, -xg1), acc[0][rt][T][3]);
-            }
-          }
-        }
-      }
+      dec_stage<kInt4, NT, TW>(acc, st, a.xhalf, L, tokv, static_cast<int64_t>(st_begin + i) * 2, row0, Nm, scm, zpm,
+                               G);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);
     }
-    // this warp's results: factors 2^-24 (pairs 0 and 3), 2^-20 (pair 1), 2^-16 (pair 2) applied
-    // exactly; rows rw + 16 rt + 8 hr, tokens 8 (Tb + T) + 2t + c
     float v[kDRT][TW][4];
-#pragma unroll
-    for (int rt = 0; rt < kDRT; ++rt)
-#pragma unroll
-      for (int T = 0; T < TW; ++T)
-#pragma unroll
-        for (int ci = 0; ci < 4; ++ci)
-          v[rt][T][ci] = kInt4 ? acc[0][rt][T][ci]
-                               : fmaf(acc[0][rt][T][ci], 16777216.0f,
-                                      fmaf(acc[1 % NG][rt][T][ci], 1048576.0f, acc[2 % NG][rt][T][ci] * 65536.0f));
+    dec_values<kInt4, TW>(acc, v);
     if (NT == 1) {  // M <= 8: add the second K half (warps 4-7) to the first, fixed order
       if (hi == 1) {
 #pragma unroll
@@ -489,14 +474,13 @@ __device__ __forceinline__ void decode_gemm_body(const DecodeMaps& maps, const D
     }
     {
       // push this slice's partial results to the CTA that owns each row (owner q holds rows
-      // [q*R/S, (q+1)*R/S) of the R real rows); the virtual row goes to every owner
-      const uint32_t red_local = smem_u32(red), sxr_local = smem_u32(sxr);
+      // [q*R/S, (q+1)*R/S) of the R rows)
+      const uint32_t red_local = smem_u32(red);
 #pragma unroll
       for (int rt = 0; rt < kDRT; ++rt)
 #pragma unroll
         for (int hr = 0; hr < 2; ++hr) {
           const int r = rw + 16 * rt + 8 * hr;
-          const bool vrow = virt && rt == kDRT - 1 && hr == 1;
           const int q = ((r + 1) * a.S - 1) / F::kRows;
           const int slot = r - (q * F::kRows) / a.S;
 #pragma unroll
@@ -505,13 +489,8 @@ __device__ __forceinline__ void decode_gemm_body(const DecodeMaps& maps, const D
             for (int c = 0; c < 2; ++c) {
               const float val = v[rt][T][2 * hr + c];
               const int tok = 8 * (Tb + T) + 2 * t + c;
-              if (vrow) {
-                for (int o = 0; o < a.S; ++o)
-                  st_shared_cluster_f32(mapa_shared(sxr_local + (rank * 16 + tok) * 4, static_cast<uint32_t>(o)), val);
-              } else if (r < F::kRows) {
-                st_shared_cluster_f32(
-                    mapa_shared(red_local + ((rank * 16 + tok) * own_cap + slot) * 4, static_cast<uint32_t>(q)), val);
-              }
+              st_shared_cluster_f32(
+                  mapa_shared(red_local + ((rank * 16 + tok) * own_cap + slot) * 4, static_cast<uint32_t>(q)), val);
             }
         }
     }
@@ -519,17 +498,15 @@ __device__ __forceinline__ void decode_gemm_body(const DecodeMaps& maps, const D
   }
 
   // ==================================================================== cluster reduction
-  cluster_sync_all();  // every partial and slice sum has landed in its owner's shared memory
+  cluster_sync_all();  // every partial has landed in its owner's shared memory
   pdl_wait_prior_grids();
   if (ep_on) {
     const int Mv = Mi < 8 * NT ? Mi : 8 * NT;
     for (int mm = 0; mm < Mv; ++mm) {
-      float v = 0.0f, sx = 0.0f;
-      for (int q = 0; q < a.S; ++q) {  // fixed order: deterministic
+      float v = 0.0f;
+      for (int q = 0; q < a.S; ++q)  // fixed order: deterministic
         v += red[(q * 16 + mm) * own_cap + ep_row];  // consecutive rows: conflict free
-        if (!kInt4) sx += sxr[q * 16 + mm];
-      }
-      if (!kInt4) v = (v - sx) * ep_s;
+      if (!kInt4) v *= ep_s;
       ym[mm * Nm + ep_n] = __float2half_rn(v + ep_b);
     }
   }
@@ -628,7 +605,7 @@ template <bool kInt4>
 static cudaError_t launch_decode_group(const __half* x, int count, const void* const* w,
                                        const __half* const* sc, const __half* const* bias,
                                        __half* const* y, const int64_t* N, int64_t M, int64_t K,
-                                       cudaStream_t s) {
+                                       cudaStream_t s, const uint8_t* const* zp = nullptr) {
   using F = DecFmt<kInt4>;
   if (count < 1 || count > kDMaxGroup) return cudaErrorInvalidValue;
   const DeviceInfo di = current_device_info();
@@ -648,6 +625,7 @@ static cudaError_t launch_decode_group(const __half* x, int count, const void* c
     rbs += (N[g] + F::kRows - 1) / F::kRows;
     a.N[g] = N[g];
     a.sc[g] = sc[g];
+    a.zp[g] = zp ? zp[g] : nullptr;
     a.bias[g] = bias ? bias[g] : nullptr;
     a.y[g] = y[g];
     if (!make_tmap_2d(&maps.m[g], CU_TENSOR_MAP_DATA_TYPE_UINT8, w[g], static_cast<uint64_t>(kbytes),
@@ -684,7 +662,8 @@ bool decode_supported(bool int4, int64_t M, int64_t N, int64_t K) {
   if (int4 ? (K % 128 != 0) : (K % 64 != 0)) return false;
   DecodePlan p;
   const int64_t rows = int4 ? DecFmt<true>::kRows : DecFmt<false>::kRows;
-  return plan_decode(int4, (N + rows - 1) / rows, M > 16 ? 16 : M, K, 148, &p, (M + 15) / 16);
+  return plan_decode(int4, (N + rows - 1) / rows, M > 16 ? 16 : M, K, current_device_info().num_sms, &p,
+                     (M + 15) / 16);
 }
 
 cudaError_t launch_tq_gemm_decode(const __half* x, const uint8_t* packed, const __half* scale,
@@ -695,10 +674,10 @@ cudaError_t launch_tq_gemm_decode(const __half* x, const uint8_t* packed, const 
 }
 
 cudaError_t launch_w4g_gemm_decode(const __half* x, const int32_t* qweight, const __half* scales,
-                                   const __half* bias, __half* y, int64_t M, int64_t N, int64_t K,
-                                   cudaStream_t s) {
+                                   const uint8_t* zeros, const __half* bias, __half* y, int64_t M, int64_t N,
+                                   int64_t K, cudaStream_t s) {
   const void* w = qweight;
-  return launch_decode_group<true>(x, 1, &w, &scales, &bias, &y, &N, M, K, s);
+  return launch_decode_group<true>(x, 1, &w, &scales, &bias, &y, &N, M, K, s, &zeros);
 }
 
 cudaError_t launch_tq_gemm_decode_group(const __half* x, int count, const uint8_t* const* packed,

@@ -4,4 +4,5 @@
 #include "tq_generic.cu"
 #include "tq_pack.cu"
 #include "tq_decode.cu"
+#include "tq_batch.cu"
 #include "tq_prefill.cu"

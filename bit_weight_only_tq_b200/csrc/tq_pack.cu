@@ -312,10 +312,54 @@ __global__ void __launch_bounds__(kPackThreads)
 // ---------------------------------------------------------------------------------------------
 // W4A16 pack: one warp per (row n, group g of 128).  Lane l holds k = 128g + 4l .. 4l+3.
 // ---------------------------------------------------------------------------------------------
+// The group quantiser shared by both W4 pack kernels: this lane's four weights wf of one
+// 128-wide group (the warp holds the group).  Symmetric ([VQ] §5 "sym": true): s = fp16(max|w|/7),
+// q = clamp(rint(w / s), -8, 7), stored u = q + 8.  Asymmetric (zeros requested, the weight_zp of
+// the same section): lo = min(0, min w), hi = max(0, max w), s = fp16((hi - lo) / 15),
+// z = clamp(rint(-lo / s), 0, 15), stored u = clamp(rint(w / s) + z, 0, 15).  All quotients in
+// fp64 with the STORED fp16 s; s == 0 gives u = 0 (asymmetric, z = 0) or u = 8 (symmetric).
+__device__ __forceinline__ void w4_quantize_group(const float (&wf)[4], bool asym, uint16_t& sb, int& z,
+                                                  int (&u)[4]) {
+  float a = 0.0f, b = 0.0f;  // symmetric: a = max|w|; asymmetric: a = min(0, w), b = max(0, w)
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if (asym) {
+      a = fminf(a, wf[i]);
+      b = fmaxf(b, wf[i]);
+    } else {
+      a = fmaxf(a, fabsf(wf[i]));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    if (asym) {
+      a = fminf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+      b = fmaxf(b, __shfl_xor_sync(0xFFFFFFFFu, b, o));
+    } else {
+      a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+    }
+  }
+  sb = asym ? f64_to_f16_rne((static_cast<double>(b) - static_cast<double>(a)) / 15.0)
+            : f64_to_f16_rne(static_cast<double>(a) / 7.0);
+  const double sd = f16_bits_to_f64(sb);
+  z = asym ? 0 : 8;
+  if (asym && sd != 0.0) z = static_cast<int>(fmin(fmax(rint(-static_cast<double>(a) / sd), 0.0), 15.0));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if (sd == 0.0) {
+      u[i] = asym ? 0 : 8;
+    } else {
+      const double r = rint(static_cast<double>(wf[i]) / sd);
+      u[i] = asym ? static_cast<int>(fmin(fmax(r + z, 0.0), 15.0)) : static_cast<int>(fmin(fmax(r, -8.0), 7.0)) + 8;
+    }
+  }
+}
+
+// One warp per (row, group of 128 consecutive columns): four columns per lane, whole words out.
 template <bool kF16>
 __global__ void __launch_bounds__(256)
     w4g_pack_kernel(const void* __restrict__ w, int32_t* __restrict__ qweight,
-                    uint16_t* __restrict__ scales, int64_t N, int64_t K, int vec) {
+                    uint16_t* __restrict__ scales, uint8_t* __restrict__ zeros, int64_t N, int64_t K, int vec) {
   const int lane = threadIdx.x & 31;
   const int64_t G = K >> 7;
   const int64_t warps_total = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
@@ -328,31 +372,64 @@ __global__ void __launch_bounds__(256)
     uint32_t v[4];
     load4<kF16>(row, k0 >> 2, K, vec, v);
     float wf[4];
-    float mx = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 4; ++i)
       wf[i] = kF16 ? __half2float(__ushort_as_half(static_cast<uint16_t>(v[i]))) : __uint_as_float(v[i]);
-      mx = fmaxf(mx, fabsf(wf[i]));
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-    const uint16_t sb = f64_to_f16_rne(static_cast<double>(mx) / 7.0);
-    const double sd = f16_bits_to_f64(sb);
+    uint16_t sb;
+    int z, u[4];
+    w4_quantize_group(wf, zeros != nullptr, sb, z, u);
     uint32_t nib = 0;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      int q = 0;
-      if (sd != 0.0) {
-        const double r = rint(static_cast<double>(wf[i]) / sd);
-        q = static_cast<int>(fmin(fmax(r, -8.0), 7.0));
-      }
-      nib |= static_cast<uint32_t>(q + 8) << (4 * i);
-    }
+    for (int i = 0; i < 4; ++i) nib |= static_cast<uint32_t>(u[i]) << (4 * i);
     const uint32_t other = __shfl_down_sync(0xFFFFFFFFu, nib, 1);
     if ((lane & 1) == 0) {
       qweight[n * (K >> 3) + g * 16 + (lane >> 1)] = static_cast<int32_t>(nib | (other << 16));
     }
-    if (lane == 0) scales[n * G + g] = sb;
+    if (lane == 0) {
+      scales[n * G + g] = sb;
+      if (zeros) zeros[n * G + g] = static_cast<uint8_t>(z);
+    }
+  }
+}
+
+// Activation order: one warp per (row, group), the group being the columns perm[128 g .. +127];
+// the nibbles go to the columns' ORIGINAL positions (OR into a zeroed qweight, since one word
+// gathers columns of several groups).  The warps of row 0 also write g_idx[perm[j]] = j / 128.
+template <bool kF16>
+__global__ void __launch_bounds__(256)
+    w4g_pack_perm_kernel(const void* __restrict__ w, const int32_t* __restrict__ perm, int32_t* __restrict__ qweight,
+                         uint16_t* __restrict__ scales, uint8_t* __restrict__ zeros, int32_t* __restrict__ g_idx,
+                         int64_t N, int64_t K) {
+  const int lane = threadIdx.x & 31;
+  const int64_t G = K >> 7;
+  const int64_t warps_total = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t item = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       item < N * G; item += warps_total) {
+    const int64_t n = item / G, g = item - n * G;
+    int64_t col[4];
+    float wf[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      col[i] = __ldg(perm + g * 128 + 4 * lane + i);
+      const bool in = col[i] >= 0 && col[i] < K;  // a perm that is not a permutation: no stray access
+      wf[i] = !in ? 0.0f
+                  : kF16 ? __half2float(__ushort_as_half(__ldg(static_cast<const uint16_t*>(w) + n * K + col[i])))
+                         : __ldg(static_cast<const float*>(w) + n * K + col[i]);
+    }
+    uint16_t sb;
+    int z, u[4];
+    w4_quantize_group(wf, zeros != nullptr, sb, z, u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (col[i] < 0 || col[i] >= K) continue;
+      atomicOr(reinterpret_cast<unsigned int*>(qweight + n * (K >> 3) + (col[i] >> 3)),
+               static_cast<unsigned int>(u[i]) << (4 * (col[i] & 7)));
+      if (n == 0 && g_idx) g_idx[col[i]] = static_cast<int32_t>(g);
+    }
+    if (lane == 0) {
+      scales[n * G + g] = sb;
+      if (zeros) zeros[n * G + g] = static_cast<uint8_t>(z);
+    }
   }
 }
 
@@ -387,16 +464,34 @@ cudaError_t launch_tq_pack(const void* w, bool w_f16, uint8_t* packed, uint16_t*
 
 cudaError_t launch_w4g_pack(const void* w, bool w_f16, int32_t* qweight, uint16_t* scales,
                             int64_t N, int64_t K, cudaStream_t s) {
+  return launch_w4g_pack_ex(w, w_f16, nullptr, qweight, scales, nullptr, nullptr, N, K, s);
+}
+
+cudaError_t launch_w4g_pack_ex(const void* w, bool w_f16, const int32_t* perm, int32_t* qweight, uint16_t* scales,
+                               uint8_t* zeros, int32_t* g_idx, int64_t N, int64_t K, cudaStream_t s) {
   const DeviceInfo di = current_device_info();
   const int64_t items = N * (K >> 7);
   int64_t grid = (items + 7) / 8;
   if (grid > int64_t(di.num_sms) * 16) grid = int64_t(di.num_sms) * 16;
+  if (perm) {
+    cudaError_t e = cudaMemsetAsync(qweight, 0, static_cast<size_t>(N) * static_cast<size_t>(K / 2), s);
+    if (e != cudaSuccess) return e;
+    if (w_f16)
+      w4g_pack_perm_kernel<true><<<static_cast<unsigned>(grid), 256, 0, s>>>(w, perm, qweight, scales, zeros, g_idx, N, K);
+    else
+      w4g_pack_perm_kernel<false><<<static_cast<unsigned>(grid), 256, 0, s>>>(w, perm, qweight, scales, zeros, g_idx, N, K);
+    return cudaGetLastError();
+  }
+  if (g_idx) {  // contiguous groups: g_idx[k] = k / 128
+    cudaError_t e = launch_iota_groups(g_idx, K, s);
+    if (e != cudaSuccess) return e;
+  }
   const uintptr_t a = reinterpret_cast<uintptr_t>(w);
   const int vec = (a % (w_f16 ? 8 : 16) == 0);
   if (w_f16)
-    w4g_pack_kernel<true><<<static_cast<unsigned>(grid), 256, 0, s>>>(w, qweight, scales, N, K, vec);
+    w4g_pack_kernel<true><<<static_cast<unsigned>(grid), 256, 0, s>>>(w, qweight, scales, zeros, N, K, vec);
   else
-    w4g_pack_kernel<false><<<static_cast<unsigned>(grid), 256, 0, s>>>(w, qweight, scales, N, K, vec);
+    w4g_pack_kernel<false><<<static_cast<unsigned>(grid), 256, 0, s>>>(w, qweight, scales, zeros, N, K, vec);
   return cudaGetLastError();
 }
 

@@ -98,6 +98,7 @@ struct PrefillLayout {
 
 struct PrefillArgs {
   const __half* sc;    // ternary: scale[N]; W4A16: scales[N, K/128]
+  const uint8_t* zp;   // W4A16 zero-points [N, K/128], or null (symmetric)
   const __half* bias;  // may be null
   __half* y;
   int64_t M, N, K;
@@ -130,15 +131,20 @@ __device__ __forceinline__ uint4 decode_tq_8(uint32_t w, int bpair) {
   return r;
 }
 
-// 8 consecutive INT4 codes (one int32 word) -> 8 fp16 q * s, s2 = (s, s).
-__device__ __forceinline__ uint4 decode_w4_8(uint32_t w, uint32_t s2) {
+// The fp16 pair (1024 + z, 64 + z) that decode_w4_8 subtracts for zero-point z (0..15): 1024 + z
+// has unit 1, 64 + z unit 1/16, so both are exact patterns.  z = 8 is the symmetric format.
+__device__ __forceinline__ uint32_t w4_zero_pair(uint32_t z) { return ((0x5400u + 16u * z) << 16) | (0x6400u + z); }
+
+// 8 consecutive INT4 codes (one int32 word) -> 8 fp16 (u - z) * s, s2 = (s, s), zsub =
+// w4_zero_pair(z).
+__device__ __forceinline__ uint4 decode_w4_8(uint32_t w, uint32_t s2, uint32_t zsub) {
   uint32_t o[4];
 #pragma unroll
   for (int bi = 0; bi < 4; ++bi) {
     const uint32_t t = byte_to_halves(w, bi);
     // low nibble -> 1024 + u (0x6400 base), high nibble -> 64 + u (0x5400 base, bits 4-7)
     const uint32_t h = (t & 0x00F0000Fu) | 0x54006400u;
-    o[bi] = hmul2_u32(hsub2_u32(h, 0x54806408u /* (1032, 72) */), s2);
+    o[bi] = hmul2_u32(hsub2_u32(h, zsub), s2);
   }
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
@@ -206,7 +212,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
     pdl_wait_prior_grids();
     if (lane == 0) {
       tma_prefetch_desc(&tmap_x);
-      for (int kb = 0; kb < nk && ok; ++kb) {
+      const bool skipx = skip_x_loads();  // failure-path test hook: never set in normal use
+      for (int kb = 0; kb < nk && ok && !skipx; ++kb) {
         const int s = kb % L::kRing;
         if (kb >= L::kRing) {
           ok = mbar_wait(&emptyX[s], static_cast<uint32_t>((kb / L::kRing) - 1) & 1u);
@@ -278,8 +285,12 @@ __global__ void __launch_bounds__(kQThreads, 1)
     auto group_scale = [&](int64_t gi) -> uint16_t {
       return (n < a.N && gi < G) ? __half_as_ushort(a.sc[n * G + gi]) : static_cast<uint16_t>(0);
     };
+    auto group_zero = [&](int64_t gi) -> uint32_t {
+      return (a.zp && n < a.N && gi < G) ? static_cast<uint32_t>(a.zp[n * G + gi]) : 8u;
+    };
     int64_t g_cur = -1;
     uint16_t sc_cur = 0, sc_nxt = 0;
+    uint32_t zp_cur = 8u, zp_nxt = 8u;
     for (int kb = 0; kb < nk && ok; ++kb) {
       const int as = kb % L::kARing, pt = kb / F::kSPP, ci = kb - pt * F::kSPP, ps = pt % F::kPRing;
       if (ci == 0) {
@@ -302,11 +313,14 @@ __global__ void __launch_bounds__(kQThreads, 1)
         const int64_t gi = (kb0 + kb) >> 1;  // 128-wide group of this 64-wide stage
         if (gi != g_cur) {
           sc_cur = g_cur < 0 ? group_scale(gi) : sc_nxt;
+          zp_cur = g_cur < 0 ? group_zero(gi) : zp_nxt;
           sc_nxt = group_scale(gi + 1);
+          zp_nxt = group_zero(gi + 1);
           g_cur = gi;
         }
         s2 = static_cast<uint32_t>(sc_cur) | (static_cast<uint32_t>(sc_cur) << 16);
       }
+      const uint32_t zsub = w4_zero_pair(zp_cur);
       const uint32_t pw[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
       if (kSS) {
         if (kb >= L::kARing) {
@@ -318,7 +332,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
         uint8_t* arow = sm + L::kOffA + as * L::kTileA + r * 128;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const uint4 d = kInt4 ? decode_w4_8(pw[j], s2) : decode_tq_8(pw[j >> 1], j & 1);
+          const uint4 d = kInt4 ? decode_w4_8(pw[j], s2, zsub) : decode_tq_8(pw[j >> 1], j & 1);
           *reinterpret_cast<uint4*>(arow + ((j ^ (r & 7)) << 4)) = d;
         }
         fence_proxy_async_smem();  // visible to the tensor core's operand reads
@@ -326,7 +340,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
         uint32_t v[32];  // column j = fp16 pair (k = 2j, 2j + 1) of this row
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const uint4 d = kInt4 ? decode_w4_8(pw[j], s2) : decode_tq_8(pw[j >> 1], j & 1);
+          const uint4 d = kInt4 ? decode_w4_8(pw[j], s2, zsub) : decode_tq_8(pw[j >> 1], j & 1);
           v[4 * j] = d.x;
           v[4 * j + 1] = d.y;
           v[4 * j + 2] = d.z;
@@ -441,7 +455,7 @@ bool prefill_supported(bool int4, int64_t M, int64_t N, int64_t K) {
 }
 
 template <bool kInt4, int TN, bool kSS>
-static cudaError_t launch_prefill_t(const __half* x, const void* w, const __half* sc,
+static cudaError_t launch_prefill_t(const __half* x, const void* w, const __half* sc, const uint8_t* zp,
                                     const __half* bias, __half* y, int64_t M, int64_t N, int64_t K,
                                     int S, cudaStream_t s) {
   using L = PrefillLayout<kInt4, TN, kSS>;
@@ -459,6 +473,7 @@ static cudaError_t launch_prefill_t(const __half* x, const void* w, const __half
   if (e != cudaSuccess) return e;
   PrefillArgs a;
   a.sc = sc;
+  a.zp = zp;
   a.bias = bias;
   a.y = y;
   a.M = M;
@@ -494,7 +509,7 @@ static cudaError_t launch_prefill_t(const __half* x, const void* w, const __half
 constexpr int kPrefillSSMaxTN = 128;  // token tiles up to this width read A from shared memory
 
 template <bool kInt4>
-static cudaError_t launch_prefill(const __half* x, const void* w, const __half* sc,
+static cudaError_t launch_prefill(const __half* x, const void* w, const __half* sc, const uint8_t* zp,
                                   const __half* bias, __half* y, int64_t M, int64_t N, int64_t K,
                                   cudaStream_t s) {
   const DeviceInfo di = current_device_info();
@@ -504,21 +519,21 @@ static cudaError_t launch_prefill(const __half* x, const void* w, const __half* 
   const int64_t base = rt * ((M + TN - 1) / TN);
   int S = 1;
   while (S < 8 && base * S * 2 <= di.num_sms && S * 2 <= nk) S *= 2;
-  if (TN == 64) return launch_prefill_t<kInt4, 64, kPrefillSSMaxTN >= 64>(x, w, sc, bias, y, M, N, K, S, s);
-  if (TN == 128) return launch_prefill_t<kInt4, 128, kPrefillSSMaxTN >= 128>(x, w, sc, bias, y, M, N, K, S, s);
-  return launch_prefill_t<kInt4, 256, false>(x, w, sc, bias, y, M, N, K, S, s);
+  if (TN == 64) return launch_prefill_t<kInt4, 64, kPrefillSSMaxTN >= 64>(x, w, sc, zp, bias, y, M, N, K, S, s);
+  if (TN == 128) return launch_prefill_t<kInt4, 128, kPrefillSSMaxTN >= 128>(x, w, sc, zp, bias, y, M, N, K, S, s);
+  return launch_prefill_t<kInt4, 256, false>(x, w, sc, zp, bias, y, M, N, K, S, s);
 }
 
 cudaError_t launch_tq_gemm_prefill(const __half* x, const uint8_t* packed, const __half* scale,
                                    const __half* bias, __half* y, int64_t M, int64_t N, int64_t K,
                                    cudaStream_t s) {
-  return launch_prefill<false>(x, packed, scale, bias, y, M, N, K, s);
+  return launch_prefill<false>(x, packed, scale, nullptr, bias, y, M, N, K, s);
 }
 
 cudaError_t launch_w4g_gemm_prefill(const __half* x, const int32_t* qweight, const __half* scales,
-                                    const __half* bias, __half* y, int64_t M, int64_t N, int64_t K,
-                                    cudaStream_t s) {
-  return launch_prefill<true>(x, qweight, scales, bias, y, M, N, K, s);
+                                    const uint8_t* zeros, const __half* bias, __half* y, int64_t M, int64_t N,
+                                    int64_t K, cudaStream_t s) {
+  return launch_prefill<true>(x, qweight, scales, zeros, bias, y, M, N, K, s);
 }
 
 }  // namespace tq

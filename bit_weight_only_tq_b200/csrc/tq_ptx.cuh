@@ -18,8 +18,16 @@ __device__ int g_tq_device_status = 0;
 
 static constexpr int kStatusTimeout = 1;
 
-// A wait gives up after this many SM clock cycles (~2 s at 1.9 GHz).
+// A wait gives up after this many SM clock cycles (~2 s at 1.9 GHz).  Tests of the failure path
+// shorten it through tq_debug_set_wait_limit().
 static constexpr long long kWaitLimitCycles = 4000000000LL;
+__device__ long long g_tq_wait_limit = kWaitLimitCycles;
+
+// Failure-path test hook (tq_debug_skip_activation_loads): when nonzero, the producers of the
+// GEMM kernels issue no activation (x) loads, so the stage barriers that count those bytes never
+// complete and the consumers' bounded waits run out.  Nothing in the library sets it.
+__device__ int g_tq_skip_x_loads = 0;
+__device__ __forceinline__ bool skip_x_loads() { return *reinterpret_cast<volatile int*>(&g_tq_skip_x_loads) != 0; }
 
 __device__ __forceinline__ void record_timeout() {
   atomicExch(&g_tq_device_status, kStatusTimeout);
@@ -77,7 +85,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     if (mbar_try_wait(a, parity)) return true;
     if (backoff < 256) backoff += 32;
     __nanosleep(backoff);
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > *reinterpret_cast<volatile long long*>(&g_tq_wait_limit)) {
       record_timeout();
       return false;
     }

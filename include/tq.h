@@ -34,14 +34,17 @@
  *   - Inputs must be finite; results for Inf/NaN weights or activations are unspecified.
  *   - The tensor-core GEMM kernels are launched with programmatic dependent launch: they start
  *     while the preceding kernel on the stream is still running and wait for it before reading x
- *     or writing y, but they read the packed weights, scales and bias (model constants) before
- *     that wait.  Those must therefore not be written by the kernel enqueued immediately before
- *     a GEMM call on the same stream (e.g. tq_quantize_pack followed directly by tq_gemm): put
- *     any other operation, an event wait or a synchronisation in between.
+ *     or writing y, but they read the packed weights, scales, zero-points and bias (model
+ *     constants) before that wait.  The library's own writers of packed data (the pack and
+ *     repack calls) therefore end with an empty kernel in plain stream order, so a GEMM enqueued
+ *     right after them sees their results.  A caller that writes weights, scales or bias with
+ *     its OWN kernel must not enqueue a GEMM immediately after that kernel on the same stream:
+ *     put any other operation, an event wait or a synchronisation in between.
  */
 #ifndef TQ_H
 #define TQ_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #if defined(__GNUC__)
@@ -147,6 +150,57 @@ TQ_API int w4g_gemm_ex(const uint16_t* x, const int32_t* qweight, const uint16_t
                 void* stream);
 
 /* --------------------------------------------------------------------------------------------
+ * INT4 variants ([VQ] §5: GPTQ's sym / desc_act options, the weight_zp zero-point parameter and
+ * the optional g_idx of activation ordering; [TQ] §2.1: AWQ checkpoints carry qweight, scales
+ * and zeros).
+ *
+ * w4g_quantize_pack_ex -- the general INT4 packer, group size 128 along K.
+ *   w        [N,K] fp32 or fp16, device; K % 128 == 0.
+ *   perm     NULL, or device int32 [K]: a permutation of 0..K-1, the order in which the columns
+ *            are quantised (activation order: column perm[j] belongs to group j / 128).  NULL:
+ *            group g is columns 128 g .. 128 g + 127.
+ *   qweight  [N, K/8] int32, written, in the ORIGINAL column order: nibble i of word j holds the
+ *            code of column 8j + i.
+ *   scales   [N, K/128] fp16, written, by group.
+ *   zeros    NULL: symmetric, exactly as w4g_quantize_pack (u = q + 8, s = fp16(max|w|/7)).
+ *            Else [N, K/128] uint8, written: asymmetric, per group lo = min(0, min w),
+ *            hi = max(0, max w), s = fp16((hi - lo) / 15), z = clamp(rint(-lo / s), 0, 15),
+ *            u = clamp(rint(w / s) + z, 0, 15) (fp64 quotients by the stored fp16 s, ties to
+ *            even; an all-zero group gives s = 0, z = 0, u = 0).  What = s * (u - z).
+ *   g_idx    NULL, or device int32 [K], written: the group of each column (k / 128 without perm).
+ * Bit-exact.  With perm, qweight is cleared first (the kernel ORs nibbles into it).
+ * Returns TQ_OK, TQ_ERR_DTYPE, TQ_ERR_SHAPE (K % 128), TQ_ERR_NULL or TQ_ERR_CUDA.
+ *
+ * w4g_gemm_zp / w4g_gemm_zp_ex -- y = x . What^T (+ bias) with What[n,k] = s[n, k/128] *
+ *   (u[n,k] - zeros[n, k/128]) (asymmetric, consecutive groups); shapes, paths and errors as
+ *   w4g_gemm / w4g_gemm_ex; zeros must not be NULL.
+ *
+ * Activation order at run time, the way the Marlin path of [VQ] §4.3 takes it: the product is
+ * summed over k in the quantisation order, x . What^T = (x P) . (What P)^T, where P is the
+ * column permutation perm.  Once, after packing:
+ *   w4g_repack_act_order(qweight, perm, out, N, K): out[n, column j] = qweight[n, column
+ *     perm[j]] (nibbles moved; out must not overlap qweight); the groups of `out` are then
+ *     consecutive, so it is an ordinary W4A16 / zero-point matrix for the scales and zeros.
+ * Per call:
+ *   tq_permute_columns(x, perm, x_out, M, K): x_out[m, j] = x[m, perm[j]] (fp16 [M, K]; no
+ *     overlap), then w4g_gemm / w4g_gemm_zp (or the batch calls) on (x_out, out, scales[, zeros]).
+ * Both return TQ_OK, TQ_ERR_SHAPE, TQ_ERR_NULL or TQ_ERR_CUDA.
+ * ------------------------------------------------------------------------------------------ */
+TQ_API int w4g_quantize_pack_ex(const void* w, int w_dtype, const int32_t* perm, int32_t* qweight,
+                                uint16_t* scales, uint8_t* zeros, int32_t* g_idx, int64_t N, int64_t K,
+                                void* stream);
+TQ_API int w4g_gemm_zp(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
+                       const uint8_t* zeros, const uint16_t* bias, uint16_t* y, int64_t M, int64_t N,
+                       int64_t K, void* stream);
+TQ_API int w4g_gemm_zp_ex(const uint16_t* x, const int32_t* qweight, const uint16_t* scales,
+                          const uint8_t* zeros, const uint16_t* bias, uint16_t* y, int64_t M, int64_t N,
+                          int64_t K, int path, void* stream);
+TQ_API int w4g_repack_act_order(const int32_t* qweight, const int32_t* perm, int32_t* out, int64_t N,
+                                int64_t K, void* stream);
+TQ_API int tq_permute_columns(const uint16_t* x, const int32_t* perm, uint16_t* x_out, int64_t M,
+                              int64_t K, void* stream);
+
+/* --------------------------------------------------------------------------------------------
  * tq_gemm_grouped / w4g_gemm_grouped -- several linears that read the same input, as a serving
  * engine's fused q/k/v or gate/up projections do: for g < count,
  *     y_g[M, N_g] = x[M, K] . What_g[N_g, K]^T (+ bias_g)
@@ -172,6 +226,59 @@ TQ_API int w4g_gemm_grouped(const uint16_t* x, int count, const int32_t* const* 
                             uint16_t* const* y, const int64_t* N, int64_t M, int64_t K,
                             void* stream);
 
+/* --------------------------------------------------------------------------------------------
+ * tq_gemm_batch / w4g_gemm_batch -- a work list of independent linears that share M, all in ONE
+ * persistent kernel launch ([TQ] §1: decode time goes to fetching packed weights; a serving
+ * engine's decode step runs many small linears, and every launch boundary costs microseconds of
+ * idle SMs).  For i < count:
+ *     y_i[M, N_i] = x_i[M, K_i] . What_i[N_i, K_i]^T (+ bias_i)
+ * The items must be independent: no item's y may overlap any item's x, weights, scales or bias,
+ * nor another item's y.  Items may share x (fused q/k/v, gate/up).
+ *
+ *   items      HOST array of `count` tq_linear descriptors (read during the call only):
+ *                x      [M, K] fp16, device, 16-byte aligned
+ *                w      ternary: packed uint8 [N, K/4] (tq_quantize_pack), K % 64 == 0;
+ *                       W4A16:   qweight int32 [N, K/8] (w4g_quantize_pack), K % 128 == 0;
+ *                       device, 16-byte aligned
+ *                scale  ternary: fp16 [N]; W4A16: fp16 [N, K/128]
+ *                zeros  W4A16 only: NULL (symmetric) or uint8 [N, K/128] zero-points
+ *                       (w4g_quantize_pack_ex); ignored by tq_gemm_batch
+ *                bias   fp16 [N] or NULL
+ *                y      [M, N] fp16, written
+ *                N, K   N >= 0 (an item with N == 0 is skipped), 0 < K <= 2^28
+ *   count      1 .. 8
+ *   M          0 .. 16 tokens (0: nothing is launched)
+ *   workspace  device buffer of at least tq_batch_workspace_size() bytes, 16-byte aligned,
+ *              ZERO-FILLED before its first use (e.g. cudaMemset).  It holds the partial sums of
+ *              row blocks that the kernel splits between CTAs and one arrival counter per split;
+ *              every call leaves the counters at zero again, so a workspace is zeroed once and
+ *              then reused by any number of calls.  Calls that may run concurrently (different
+ *              streams) need different workspaces.  After a call that ended in TQ_ERR_TIMEOUT
+ *              (tq_device_status) or a CUDA error, zero it again.
+ * Results: the same bound as tq_gemm / w4g_gemm; deterministic (partial sums are added in K
+ * order whichever CTA finishes last).  Errors: TQ_ERR_SHAPE (count, M, N, K out of range or
+ * workspace too small), TQ_ERR_NULL, TQ_ERR_ALIGN, TQ_ERR_CUDA.
+ * ------------------------------------------------------------------------------------------ */
+typedef struct tq_linear {
+    const uint16_t* x;
+    const void* w;
+    const uint16_t* scale;
+    const uint16_t* bias;
+    uint16_t* y;
+    int64_t N;
+    int64_t K;
+    const uint8_t* zeros;
+} tq_linear;
+
+TQ_API int tq_gemm_batch(const tq_linear* items, int count, int64_t M, void* workspace,
+                         size_t workspace_bytes, void* stream);
+TQ_API int w4g_gemm_batch(const tq_linear* items, int count, int64_t M, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
+/* tq_batch_workspace_size -- bytes of workspace tq_gemm_batch / w4g_gemm_batch need on the
+ * device that is current in the calling thread (it depends on the number of SMs). */
+TQ_API size_t tq_batch_workspace_size(void);
+
 /* tq_validate_packed -- count the bytes of a packed ternary matrix [N, ceil(K/4)] that hold
  * the unused code 0b11 in one of their first K codes of the row ([TQ] §3.1: the table maps
  * 00/01/10 only).  *bad_count (device int) is OVERWRITTEN with the count (set to 0 first, on
@@ -187,6 +294,25 @@ TQ_API int tq_select_path(int fmt, int64_t M, int64_t N, int64_t K, int aligned1
  * status word written by kernels whose bounded waits ran out.  Returns TQ_OK,
  * TQ_ERR_TIMEOUT, or TQ_ERR_CUDA if the synchronisation itself failed. */
 TQ_API int tq_device_status(void);
+
+/* --------------------------------------------------------------------------------------------
+ * Failure-path test hooks ([TQ] §5.4-5.5: kernels that fail by status, never by hanging).
+ * They exist so that tests can make a bounded device-side wait run out on purpose without
+ * faulting or hanging the GPU; a serving process never calls them.  Both apply to the current
+ * device, synchronise it, and stay in effect until changed.
+ *
+ * tq_debug_set_wait_limit -- every bounded wait (mbarrier polls of the GEMM kernels) gives up
+ *   after `cycles` SM clock cycles instead of the default 4e9 (~2 s); cycles <= 0 restores the
+ *   default.  A wait that gives up records TQ_ERR_TIMEOUT for tq_device_status(); the kernel
+ *   then skips the rest of its work (its outputs are unspecified), frees what it holds and exits.
+ * tq_debug_skip_activation_loads -- on != 0: the GEMM kernels' producers issue no activation
+ *   (x) loads, so the stage barriers that count those bytes never complete and the consumers'
+ *   waits run out; 0 restores normal operation.  Batch calls made while it is set leave their
+ *   workspace counters untouched.
+ * Returns TQ_OK or TQ_ERR_CUDA.
+ * ------------------------------------------------------------------------------------------ */
+TQ_API int tq_debug_set_wait_limit(long long cycles);
+TQ_API int tq_debug_skip_activation_loads(int on);
 
 /* tq_status_string -- static, human-readable text for a tq_status value. */
 TQ_API const char* tq_status_string(int status);

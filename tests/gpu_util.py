@@ -57,3 +57,24 @@ def check_w4g_gemm(x, qweight, scales, bias, y, rows=None, cols=None, label=""):
     r = O.quant_check(yref, yt, bound=bound)
     assert r["ok"], (label, r)
     return r
+
+
+# Output canaries: every output buffer is allocated with guard elements on both sides, filled
+# with a quiet-NaN payload no kernel writes, and checked after the call (replaces the
+# sanitizer's out-of-bounds detection for the output side).
+GUARD = 64               # elements (128 bytes: keeps the output 16-byte aligned)
+CANARY = 0x7E5A          # quiet NaN with a payload
+
+
+def guarded_empty(M, N, device="cuda"):
+    """(y [M,N] fp16 view, whole buffer) with GUARD canary elements before and after y."""
+    buf = torch.empty(M * N + 2 * GUARD, dtype=torch.int16, device=device)
+    buf.fill_(CANARY - 0x10000 if CANARY > 0x7FFF else CANARY)
+    buf = buf.view(torch.float16)
+    return buf[GUARD:GUARD + M * N].view(M, N), buf
+
+
+def check_canaries(buf, M, N, label=""):
+    b = buf.detach().cpu().view(torch.int16).numpy().view(np.uint16)
+    head, tail = b[:GUARD], b[GUARD + M * N:]
+    assert (head == CANARY).all() and (tail == CANARY).all(), f"{label}: write outside y [{M},{N}]"

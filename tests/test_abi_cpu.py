@@ -12,11 +12,12 @@ import bit_weight_only_tq_b200 as tq
 
 def test_library_exports_every_header_function():
     names = tq.header_functions()
-    assert len(names) == 13
+    assert len(names) == 23
     for n in names:
         assert hasattr(tq.lib, n), n
     for n in ("tq_quantize_pack", "tq_gemm", "w4g_quantize_pack", "w4g_gemm", "tq_validate_packed",
-              "tq_select_path", "tq_device_status", "tq_status_string"):
+              "tq_select_path", "tq_device_status", "tq_status_string", "tq_gemm_batch", "w4g_gemm_batch",
+              "tq_batch_workspace_size"):
         assert n in names
 
 
@@ -107,6 +108,38 @@ def test_grouped_argument_errors_without_gpu():
     assert tq.lib.tq_gemm_grouped(p, 3, arr, arr, None, arr, bad, 1, 64, None) == -2
     assert tq.lib.w4g_gemm_grouped(p, 3, arr, arr, None, arr, ns, 1, 100, None) == -2  # K % 128
     assert tq.lib.tq_gemm_grouped(p, 3, arr, arr, None, arr, ns, 0, 64, None) == 0    # M = 0
+
+
+def _items(*specs):
+    arr = (tq.TqLinear * len(specs))()
+    for i, (x, w, sc, y, N, K) in enumerate(specs):
+        arr[i] = tq.TqLinear(x, w, sc, None, y, N, K)
+    return arr
+
+
+def test_batch_argument_errors_without_gpu():
+    a, q = 4096, 4098  # a 16-byte aligned and a misaligned fake device address
+    ws, big = ctypes.c_void_p(1 << 20), 1 << 40
+    ok = _items((a, a, a, a, 64, 128))
+    assert tq.lib.tq_gemm_batch(ok, 0, 1, ws, big, None) == -2                 # count
+    assert tq.lib.tq_gemm_batch(ok, 9, 1, ws, big, None) == -2
+    assert tq.lib.tq_gemm_batch(ok, 1, 17, ws, big, None) == -2                # M > 16
+    assert tq.lib.tq_gemm_batch(ok, 1, -1, ws, big, None) == -2
+    assert tq.lib.tq_gemm_batch(None, 1, 1, ws, big, None) == -1
+    assert tq.lib.tq_gemm_batch(_items((a, a, a, a, 64, 100)), 1, 1, ws, big, None) == -2   # K % 64
+    assert tq.lib.w4g_gemm_batch(_items((a, a, a, a, 64, 192)), 1, 1, ws, big, None) == -2  # K % 128
+    assert tq.lib.tq_gemm_batch(_items((a, a, a, a, -1, 128)), 1, 1, ws, big, None) == -2
+    assert tq.lib.tq_gemm_batch(_items((0, a, a, a, 64, 128)), 1, 1, ws, big, None) == -1   # null x
+    assert tq.lib.tq_gemm_batch(_items((q, a, a, a, 64, 128)), 1, 1, ws, big, None) == -3   # misaligned x
+    assert tq.lib.tq_gemm_batch(_items((a, q, a, a, 64, 128)), 1, 1, ws, big, None) == -3   # misaligned w
+    assert tq.lib.tq_gemm_batch(ok, 1, 1, None, big, None) == -1                # no workspace
+    assert tq.lib.tq_gemm_batch(ok, 1, 1, ctypes.c_void_p(1 << 20 | 4), big, None) == -3
+    need = tq.tq_batch_workspace_size()
+    assert need > 0
+    assert tq.lib.tq_gemm_batch(ok, 1, 1, ws, need - 1, None) == -2            # workspace too small
+    # nothing to do: no launch, no workspace needed
+    assert tq.lib.tq_gemm_batch(ok, 1, 0, None, 0, None) == 0                   # M = 0
+    assert tq.lib.tq_gemm_batch(_items((0, 0, 0, 0, 0, 128)), 1, 4, None, 0, None) == 0  # N = 0
 
 
 def test_no_cpu_fallback_for_host_tensors():

@@ -1,6 +1,7 @@
 """Boundary properties of the C ABI on the GPU: CUDA-graph capture ([TQ] §5.4 stateless
 kernels), no temporary device allocations ([TQ] §5.5), determinism, non-default streams,
 device ordinal of the caller ([TQ] §5.1), and the device status word."""
+import numpy as np
 import pytest
 import torch
 
@@ -93,3 +94,28 @@ def test_current_device_is_used():
         torch.cuda.synchronize()
         assert y.device.index == dev
         check_tq_gemm(x, p, s, b, y)
+
+
+def test_pack_then_gemm_back_to_back():
+    # the GEMMs read weights before waiting for the previous kernel; the pack calls end with a
+    # plain-order empty kernel, so a GEMM enqueued right after a pack (no sync) sees its output
+    need_cuda()
+    import oracle as O
+    from gpu_util import bits, check_tq_gemm, check_w4g_gemm
+    for trial in range(3):
+        w = I.weights(4096, 4096, 70 + trial, device="cuda")
+        x = I.activations(4, 4096, 71 + trial, device="cuda")
+        p = torch.empty(4096, 1024, dtype=torch.uint8, device="cuda")
+        s = torch.empty(4096, dtype=torch.float16, device="cuda")
+        p.fill_(0x55)
+        s.fill_(0)
+        tq.tq_quantize_pack(w, p, s)
+        y = tq.tq_gemm(x, p, s, path=tq.PATH_DECODE)
+        yb = tq.tq_gemm(x.repeat(64, 1)[:200].contiguous(), p, s, path=tq.PATH_PREFILL)
+        qw, sc = tq.w4g_quantize_pack(w)
+        yw = tq.w4g_gemm(x, qw, sc, path=tq.PATH_DECODE)
+        torch.cuda.synchronize()
+        cols = np.arange(0, 4096, 17)
+        check_tq_gemm(x, p, s, None, y, cols=cols)
+        check_tq_gemm(x.repeat(64, 1)[:200].contiguous(), p, s, None, yb, rows=np.arange(0, 200, 13), cols=cols)
+        check_w4g_gemm(x, qw, sc, None, yw, cols=cols)

@@ -8,7 +8,7 @@ import torch
 
 import bit_weight_only_tq_b200 as tq
 import tq_inputs as I
-from gpu_util import check_tq_gemm, check_w4g_gemm, gpu, need_cuda
+from gpu_util import check_canaries, check_tq_gemm, check_w4g_gemm, gpu, guarded_empty, need_cuda
 
 pytestmark = gpu
 
@@ -144,10 +144,16 @@ def test_decode_m_gt_8_layouts(M, N, K):
 def test_prefill_split_k(M, N, K):
     need_cuda()
     x, p, s, b = _tq_problem(M, N, K, 900 + M)
-    y = tq.tq_gemm(x, p, s, b, path=tq.PATH_PREFILL)
+    y, buf = guarded_empty(M, N)
+    tq.tq_gemm(x, p, s, b, y=y, path=tq.PATH_PREFILL)
+    torch.cuda.synchronize()
+    check_canaries(buf, M, N, f"split-K M={M}")
     check_tq_gemm(x, p, s, b, y, cols=np.arange(0, N, 3), label=f"tq prefill split-K M={M} {N}x{K}")
     xw, qw, sc, bw = _w4_problem(M, N, K // 128 * 128, 950 + M)
-    yw = tq.w4g_gemm(xw, qw, sc, bw, path=tq.PATH_PREFILL)
+    yw, bufw = guarded_empty(M, N)
+    tq.w4g_gemm(xw, qw, sc, bw, y=yw, path=tq.PATH_PREFILL)
+    torch.cuda.synchronize()
+    check_canaries(bufw, M, N, f"w4g split-K M={M}")
     check_w4g_gemm(xw, qw, sc, bw, yw, cols=np.arange(0, N, 3), label=f"w4g prefill split-K M={M} {N}x{K}")
 
 
@@ -159,11 +165,17 @@ def test_decode_token_chunks(M, N, K):
     need_cuda()
     cols = None if N <= 1000 else np.arange(0, N, 11)
     x, p, s, b = _tq_problem(M, N, K, 1200 + M + N // 64)
-    y = tq.tq_gemm(x, p, s, b, path=tq.PATH_DECODE)
+    y, buf = guarded_empty(M, N)
+    tq.tq_gemm(x, p, s, b, y=y, path=tq.PATH_DECODE)
+    torch.cuda.synchronize()
+    check_canaries(buf, M, N, f"chunks M={M}")
     check_tq_gemm(x, p, s, b, y, cols=cols, label=f"tq decode chunks M={M} {N}x{K}")
     Kw = K // 128 * 128
     xw, qw, sc, bw = _w4_problem(M, N, Kw, 1300 + M)
-    yw = tq.w4g_gemm(xw, qw, sc, bw, path=tq.PATH_DECODE)
+    yw, bufw = guarded_empty(M, N)
+    tq.w4g_gemm(xw, qw, sc, bw, y=yw, path=tq.PATH_DECODE)
+    torch.cuda.synchronize()
+    check_canaries(bufw, M, N, f"w4g chunks M={M}")
     check_w4g_gemm(xw, qw, sc, bw, yw, cols=cols, label=f"w4g decode chunks M={M} {N}x{Kw}")
 
 

@@ -5,7 +5,7 @@ import torch
 
 import bit_weight_only_tq_b200 as tq
 import tq_inputs as I
-from gpu_util import check_tq_gemm, check_w4g_gemm, gpu, need_cuda
+from gpu_util import check_canaries, check_tq_gemm, check_w4g_gemm, gpu, guarded_empty, need_cuda
 
 pytestmark = gpu
 
@@ -20,8 +20,11 @@ def test_tq_grouped_qkv(M):
     ws = [tq.tq_quantize_pack(I.weights(N, K, 11 + i, device="cuda")) for i, N in enumerate(shapes)]
     x = I.activations(M, K, 3, device="cuda")
     biases = [I.bias(shapes[0], 1, device="cuda"), None, I.bias(shapes[2], 2, device="cuda")]
-    ys = tq.tq_gemm_grouped(x, [p for p, _ in ws], [s for _, s in ws], biases)
+    outs = [guarded_empty(M, N) for N in shapes]
+    ys = tq.tq_gemm_grouped(x, [p for p, _ in ws], [s for _, s in ws], biases, [y for y, _ in outs])
     torch.cuda.synchronize()
+    for (_, buf), N in zip(outs, shapes):
+        check_canaries(buf, M, N, f"grouped N={N} M={M}")
     for (p, s), b, y, N in zip(ws, biases, ys, shapes):
         cols = np.arange(0, N, 3)
         check_tq_gemm(x, p, s, b, y, cols=cols, label=f"grouped N={N} M={M}")
