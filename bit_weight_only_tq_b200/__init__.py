@@ -26,7 +26,7 @@ __all__ = [
     "tq_quantize_pack", "tq_gemm", "w4g_quantize_pack", "w4g_gemm", "tq_validate_packed",
     "tq_gemm_grouped", "w4g_gemm_grouped", "tq_gemm_batch", "w4g_gemm_batch", "batch_workspace",
     "tq_batch_workspace_size", "TqLinear", "w4g_quantize_pack_ex", "w4g_gemm_zp", "w4g_repack_act_order",
-    "tq_permute_columns",
+    "tq_permute_columns", "BATCH_AUTO", "BATCH_MMA_SYNC", "BATCH_TENSOR_CORE",
     "tq_select_path", "tq_device_status", "tq_status_string", "header_functions",
 ]
 
@@ -73,6 +73,8 @@ _SIGS = {
     "tq_gemm_batch": [_vp, _int, _i64, _vp, ctypes.c_size_t, _vp],
     "w4g_gemm_batch": [_vp, _int, _i64, _vp, ctypes.c_size_t, _vp],
     "tq_batch_workspace_size": [],
+    "tq_gemm_batch_ex": [_vp, _int, _i64, _vp, ctypes.c_size_t, _int, _vp],
+    "w4g_gemm_batch_ex": [_vp, _int, _i64, _vp, ctypes.c_size_t, _int, _vp],
     "tq_debug_set_wait_limit": [ctypes.c_longlong],
     "tq_debug_skip_activation_loads": [_int],
     "w4g_quantize_pack_ex": [_vp, _int, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _vp],
@@ -330,7 +332,10 @@ def batch_workspace(device=None) -> torch.Tensor:
     return torch.zeros(n, dtype=torch.uint8, device=dev)
 
 
-def _batch(fn, xs, weights, scales, biases, ys, workspace, wdtype, sdim, what, stream, zeros=None):
+BATCH_AUTO, BATCH_MMA_SYNC, BATCH_TENSOR_CORE = 0, 1, 2
+
+
+def _batch(fn, xs, weights, scales, biases, ys, workspace, wdtype, sdim, what, stream, zeros=None, variant=0):
     count = len(weights)
     if not (1 <= count <= 8) or len(scales) != count or len(xs) != count:
         raise ValueError("1..8 linears, each with its x, weights and scales")
@@ -358,21 +363,22 @@ def _batch(fn, xs, weights, scales, biases, ys, workspace, wdtype, sdim, what, s
     if workspace is None:
         raise ValueError("a workspace from batch_workspace() is required")
     _need(workspace, torch.uint8, "workspace", 1)
-    _check(fn(items, count, M, _ptr(workspace), workspace.numel(), _stream(stream)), what)
+    _check(fn(items, count, M, _ptr(workspace), workspace.numel(), int(variant), _stream(stream)), what)
     return out
 
 
-def tq_gemm_batch(xs, packed_list, scale_list, bias_list=None, y_list=None, workspace=None, stream=None):
+def tq_gemm_batch(xs, packed_list, scale_list, bias_list=None, y_list=None, workspace=None, stream=None,
+                  variant=BATCH_AUTO):
     """Independent ternary linears sharing M (each with its own x) in one persistent launch."""
-    return _batch(lib.tq_gemm_batch, xs, packed_list, scale_list, bias_list, y_list, workspace, torch.uint8, 1,
-                  "tq_gemm_batch", stream)
+    return _batch(lib.tq_gemm_batch_ex, xs, packed_list, scale_list, bias_list, y_list, workspace, torch.uint8, 1,
+                  "tq_gemm_batch", stream, variant=variant)
 
 
 def w4g_gemm_batch(xs, qweight_list, scales_list, bias_list=None, y_list=None, workspace=None, stream=None,
-                   zeros_list=None):
+                   zeros_list=None, variant=BATCH_AUTO):
     """Independent W4A16 linears sharing M in one persistent launch (zero-points optional)."""
-    return _batch(lib.w4g_gemm_batch, xs, qweight_list, scales_list, bias_list, y_list, workspace, torch.int32, 2,
-                  "w4g_gemm_batch", stream, zeros=zeros_list)
+    return _batch(lib.w4g_gemm_batch_ex, xs, qweight_list, scales_list, bias_list, y_list, workspace, torch.int32, 2,
+                  "w4g_gemm_batch", stream, zeros=zeros_list, variant=variant)
 
 
 def tq_validate_packed(packed: torch.Tensor, K: int, stream=None) -> int:

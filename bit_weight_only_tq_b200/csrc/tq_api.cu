@@ -395,9 +395,12 @@ namespace {
 
 template <bool kInt4>
 int gemm_batch_impl(const tq_linear* items, int count, int64_t M, void* workspace, size_t workspace_bytes,
-                    void* stream) {
+                    int variant, void* stream) {
   if (count < 1 || count > tq::kBatchMaxItems) return TQ_ERR_SHAPE;
+  if (variant < TQ_BATCH_AUTO || variant > TQ_BATCH_TENSOR_CORE) return TQ_ERR_PATH;
   if (M < 0 || M > tq::kBatchMaxM) return TQ_ERR_SHAPE;
+  if (variant == TQ_BATCH_AUTO) variant = M <= 16 ? TQ_BATCH_MMA_SYNC : TQ_BATCH_TENSOR_CORE;
+  if (variant == TQ_BATCH_MMA_SYNC && M > 16) return TQ_ERR_PATH;
   if (!items) return TQ_ERR_NULL;
   tq::BatchLinear lin[tq::kBatchMaxItems];
   int n = 0;
@@ -416,10 +419,13 @@ int gemm_batch_impl(const tq_linear* items, int count, int64_t M, void* workspac
   if (!workspace) return TQ_ERR_NULL;
   if (!aligned16(workspace)) return TQ_ERR_ALIGN;
   if (static_cast<int64_t>(workspace_bytes) < tq::batch_workspace_bytes()) return TQ_ERR_SHAPE;
-  const cudaError_t e = kInt4 ? tq::launch_w4g_gemm_batch(lin, n, M, workspace, static_cast<int64_t>(workspace_bytes),
-                                                          as_stream(stream))
-                              : tq::launch_tq_gemm_batch(lin, n, M, workspace, static_cast<int64_t>(workspace_bytes),
-                                                         as_stream(stream));
+  const int64_t wb = static_cast<int64_t>(workspace_bytes);
+  cudaError_t e;
+  if (variant == TQ_BATCH_TENSOR_CORE)
+    e = tq::launch_gemm_batch_tc(kInt4, lin, n, M, workspace, wb, as_stream(stream));
+  else
+    e = kInt4 ? tq::launch_w4g_gemm_batch(lin, n, M, workspace, wb, as_stream(stream))
+              : tq::launch_tq_gemm_batch(lin, n, M, workspace, wb, as_stream(stream));
   return to_status(e);
 }
 
@@ -429,12 +435,22 @@ extern "C" {
 
 int tq_gemm_batch(const tq_linear* items, int count, int64_t M, void* workspace, size_t workspace_bytes,
                   void* stream) {
-  return gemm_batch_impl<false>(items, count, M, workspace, workspace_bytes, stream);
+  return gemm_batch_impl<false>(items, count, M, workspace, workspace_bytes, TQ_BATCH_AUTO, stream);
 }
 
 int w4g_gemm_batch(const tq_linear* items, int count, int64_t M, void* workspace, size_t workspace_bytes,
                    void* stream) {
-  return gemm_batch_impl<true>(items, count, M, workspace, workspace_bytes, stream);
+  return gemm_batch_impl<true>(items, count, M, workspace, workspace_bytes, TQ_BATCH_AUTO, stream);
+}
+
+int tq_gemm_batch_ex(const tq_linear* items, int count, int64_t M, void* workspace, size_t workspace_bytes,
+                     int variant, void* stream) {
+  return gemm_batch_impl<false>(items, count, M, workspace, workspace_bytes, variant, stream);
+}
+
+int w4g_gemm_batch_ex(const tq_linear* items, int count, int64_t M, void* workspace, size_t workspace_bytes,
+                      int variant, void* stream) {
+  return gemm_batch_impl<true>(items, count, M, workspace, workspace_bytes, variant, stream);
 }
 
 int tq_validate_packed(const uint8_t* packed, int64_t N, int64_t K, int* bad_count, void* stream) {

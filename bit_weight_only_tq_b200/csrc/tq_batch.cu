@@ -311,7 +311,12 @@ __global__ void __launch_bounds__(DecWarps<2, 2>::kThreads, 2) batch_decode_kern
 // ---------------------------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------------------------
-int64_t batch_workspace_bytes() { return batch_workspace_bytes_for(kBCtasPerSm * current_device_info().num_sms); }
+int64_t tc_batch_workspace_bytes_for(int G);
+int64_t batch_workspace_bytes() {
+  const int sms = current_device_info().num_sms;
+  const int64_t a = batch_workspace_bytes_for(kBCtasPerSm * sms), b = tc_batch_workspace_bytes_for(sms);
+  return a > b ? a : b;
+}
 
 template <bool kInt4>
 static cudaError_t launch_batch_t(const BatchLinear* items, int count, int64_t M, void* ws, int64_t ws_bytes,

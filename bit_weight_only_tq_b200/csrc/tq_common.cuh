@@ -238,13 +238,17 @@ struct BatchLinear {
   const uint8_t* zp;   // W4A16 zero-points [N, K/128], or null (symmetric)
 };
 constexpr int kBatchMaxItems = 8;
-constexpr int64_t kBatchMaxM = 16;
+constexpr int64_t kBatchMaxM = 32;        // the tensor-core variant; the mma.sync variant takes M <= 16
 // Workspace bytes the batch kernel needs on the current device.
 int64_t batch_workspace_bytes();
 cudaError_t launch_tq_gemm_batch(const BatchLinear* items, int count, int64_t M, void* ws, int64_t ws_bytes,
                                  cudaStream_t s);
 cudaError_t launch_w4g_gemm_batch(const BatchLinear* items, int count, int64_t M, void* ws, int64_t ws_bytes,
                                   cudaStream_t s);
+// The tensor-core variant of the batch kernel (tq_tcbatch.cu), 1 <= M <= 32.
+cudaError_t launch_gemm_batch_tc(bool int4, const BatchLinear* items, int count, int64_t M, void* ws,
+                                 int64_t ws_bytes, cudaStream_t s);
+int64_t tc_batch_workspace_bytes_for(int G);
 
 // Encode a 2-D row-major tensor map (driver entry point fetched through the runtime, so the
 // library does not link libcuda).  Returns false on failure.

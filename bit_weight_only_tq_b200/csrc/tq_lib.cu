@@ -5,4 +5,5 @@
 #include "tq_pack.cu"
 #include "tq_decode.cu"
 #include "tq_batch.cu"
+#include "tq_tcbatch.cu"
 #include "tq_prefill.cu"

@@ -247,7 +247,7 @@ TQ_API int w4g_gemm_grouped(const uint16_t* x, int count, const int32_t* const* 
  *                y      [M, N] fp16, written
  *                N, K   N >= 0 (an item with N == 0 is skipped), 0 < K <= 2^28
  *   count      1 .. 8
- *   M          0 .. 16 tokens (0: nothing is launched)
+ *   M          0 .. 32 tokens (0: nothing is launched)
  *   workspace  device buffer of at least tq_batch_workspace_size() bytes, 16-byte aligned,
  *              ZERO-FILLED before its first use (e.g. cudaMemset).  It holds the partial sums of
  *              row blocks that the kernel splits between CTAs and one arrival counter per split;
@@ -274,6 +274,19 @@ TQ_API int tq_gemm_batch(const tq_linear* items, int count, int64_t M, void* wor
                          size_t workspace_bytes, void* stream);
 TQ_API int w4g_gemm_batch(const tq_linear* items, int count, int64_t M, void* workspace,
                           size_t workspace_bytes, void* stream);
+
+/* The batch calls run one of two kernels over the same work split (tests and benchmarks force
+ * one with the _ex forms; AUTO picks by M):
+ *   TQ_BATCH_MMA_SYNC     M <= 16: two CTAs per SM, mma.sync on the in-register decode;
+ *   TQ_BATCH_TENSOR_CORE  M <= 32: one CTA per SM, decoded weights stored to tensor memory as
+ *                         the A operand of tcgen05.mma (N = 16 or 32 tokens), accumulators in
+ *                         tensor memory.
+ * Errors as above, plus TQ_ERR_PATH for an unknown variant or M > 16 with TQ_BATCH_MMA_SYNC. */
+typedef enum { TQ_BATCH_AUTO = 0, TQ_BATCH_MMA_SYNC = 1, TQ_BATCH_TENSOR_CORE = 2 } tq_batch_variant;
+TQ_API int tq_gemm_batch_ex(const tq_linear* items, int count, int64_t M, void* workspace,
+                            size_t workspace_bytes, int variant, void* stream);
+TQ_API int w4g_gemm_batch_ex(const tq_linear* items, int count, int64_t M, void* workspace,
+                             size_t workspace_bytes, int variant, void* stream);
 
 /* tq_batch_workspace_size -- bytes of workspace tq_gemm_batch / w4g_gemm_batch need on the
  * device that is current in the calling thread (it depends on the number of SMs). */

@@ -12,7 +12,7 @@ import bit_weight_only_tq_b200 as tq
 
 def test_library_exports_every_header_function():
     names = tq.header_functions()
-    assert len(names) == 23
+    assert len(names) == 25
     for n in names:
         assert hasattr(tq.lib, n), n
     for n in ("tq_quantize_pack", "tq_gemm", "w4g_quantize_pack", "w4g_gemm", "tq_validate_packed",
@@ -123,7 +123,9 @@ def test_batch_argument_errors_without_gpu():
     ok = _items((a, a, a, a, 64, 128))
     assert tq.lib.tq_gemm_batch(ok, 0, 1, ws, big, None) == -2                 # count
     assert tq.lib.tq_gemm_batch(ok, 9, 1, ws, big, None) == -2
-    assert tq.lib.tq_gemm_batch(ok, 1, 17, ws, big, None) == -2                # M > 16
+    assert tq.lib.tq_gemm_batch(ok, 1, 33, ws, big, None) == -2                # M > 32
+    assert tq.lib.tq_gemm_batch_ex(ok, 1, 17, ws, big, tq.BATCH_MMA_SYNC, None) == -8   # mma.sync: M <= 16
+    assert tq.lib.tq_gemm_batch_ex(ok, 1, 4, ws, big, 7, None) == -8                     # unknown variant
     assert tq.lib.tq_gemm_batch(ok, 1, -1, ws, big, None) == -2
     assert tq.lib.tq_gemm_batch(None, 1, 1, ws, big, None) == -1
     assert tq.lib.tq_gemm_batch(_items((a, a, a, a, 64, 100)), 1, 1, ws, big, None) == -2   # K % 64

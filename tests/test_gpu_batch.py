@@ -57,15 +57,19 @@ SHAPES = [
 ]
 
 
-@pytest.mark.parametrize("M", [1, 3, 8, 9, 16])
+VARIANTS = [(tq.BATCH_MMA_SYNC, M) for M in (1, 3, 8, 9, 16)] + \
+           [(tq.BATCH_TENSOR_CORE, M) for M in (1, 3, 8, 16, 17, 32)]
+
+
+@pytest.mark.parametrize("variant,M", VARIANTS)
 @pytest.mark.parametrize("si", range(len(SHAPES)))
-def test_tq_batch(si, M):
+def test_tq_batch(si, variant, M):
     need_cuda()
     shapes = SHAPES[si]
     xs, ps, ss, bs = _tq_items(shapes, M, 40 * si + M, share_x=(si == 2))
     ys, bufs = _guarded_ys(M, shapes)
     ws = _workspace()
-    tq.tq_gemm_batch(xs, ps, ss, bs, ys, workspace=ws)
+    tq.tq_gemm_batch(xs, ps, ss, bs, ys, workspace=ws, variant=variant)
     torch.cuda.synchronize()
     for (N, K), x, p, s, b, y, buf in zip(shapes, xs, ps, ss, bs, ys, bufs):
         check_canaries(buf, M, N, f"batch {shapes} M={M}")
@@ -75,15 +79,16 @@ def test_tq_batch(si, M):
     assert tq.tq_device_status() == 0
 
 
-def test_tq_batch_deterministic_and_reusable():
+@pytest.mark.parametrize("variant", [tq.BATCH_MMA_SYNC, tq.BATCH_TENSOR_CORE])
+def test_tq_batch_deterministic_and_reusable(variant):
     need_cuda()
     shapes = SHAPES[2]
     M = 4
     xs, ps, ss, bs = _tq_items(shapes, M, 7, share_x=True)
     ws = _workspace()
-    first = [y.clone() for y in tq.tq_gemm_batch(xs, ps, ss, bs, workspace=ws)]
+    first = [y.clone() for y in tq.tq_gemm_batch(xs, ps, ss, bs, workspace=ws, variant=variant)]
     for _ in range(3):
-        again = tq.tq_gemm_batch(xs, ps, ss, bs, workspace=ws)
+        again = tq.tq_gemm_batch(xs, ps, ss, bs, workspace=ws, variant=variant)
         for a, b in zip(first, again):
             assert torch.equal(a.view(torch.int16), b.view(torch.int16))
     _counters_zero(ws)
@@ -103,8 +108,9 @@ def test_tq_batch_matches_single_calls():
         assert d <= 2e-2, d
 
 
-@pytest.mark.parametrize("M", [1, 16])
-def test_tq_batch_edge_rows(M):
+@pytest.mark.parametrize("variant,M", [(tq.BATCH_MMA_SYNC, 1), (tq.BATCH_MMA_SYNC, 16), (tq.BATCH_TENSOR_CORE, 1),
+                                       (tq.BATCH_TENSOR_CORE, 16), (tq.BATCH_TENSOR_CORE, 32)])
+def test_tq_batch_edge_rows(variant, M):
     need_cuda()
     from test_gpu_edge_gemm import adversarial_ternary, edge_activations
     shapes = [(200, 4096), (200, 14336)]
@@ -116,15 +122,17 @@ def test_tq_batch_edge_rows(M):
         ss.append(s)
         bs.append(I.bias(N, i, device="cuda"))
     ys, bufs = _guarded_ys(M, shapes)
-    tq.tq_gemm_batch(xs, ps, ss, bs, ys, workspace=_workspace())
+    tq.tq_gemm_batch(xs, ps, ss, bs, ys, workspace=_workspace(), variant=variant)
     torch.cuda.synchronize()
     for (N, K), x, p, s, b, y, buf in zip(shapes, xs, ps, ss, bs, ys, bufs):
         check_canaries(buf, M, N)
-        check_tq_gemm(x, p, s, b, y, label=f"batch edge {N}x{K} M={M}")
+        check_tq_gemm(x, p, s, b, y, label=f"batch edge {N}x{K} M={M} variant={variant}")
 
 
-@pytest.mark.parametrize("M", [1, 5, 16])
-def test_w4g_batch(M):
+@pytest.mark.parametrize("variant,M", [(tq.BATCH_MMA_SYNC, 1), (tq.BATCH_MMA_SYNC, 5), (tq.BATCH_MMA_SYNC, 16),
+                                       (tq.BATCH_TENSOR_CORE, 1), (tq.BATCH_TENSOR_CORE, 16),
+                                       (tq.BATCH_TENSOR_CORE, 24)])
+def test_w4g_batch(variant, M):
     need_cuda()
     shapes = [(1000, 1152), (4096, 4096), (200, 14336), (129, 128)]
     xs, qs, ss, bs = [], [], [], []
@@ -136,7 +144,7 @@ def test_w4g_batch(M):
         bs.append(I.bias(N, i, device="cuda") if i != 1 else None)
     ys, bufs = _guarded_ys(M, shapes)
     ws = _workspace()
-    tq.w4g_gemm_batch(xs, qs, ss, bs, ys, workspace=ws)
+    tq.w4g_gemm_batch(xs, qs, ss, bs, ys, workspace=ws, variant=variant)
     torch.cuda.synchronize()
     for (N, K), x, q, s, b, y, buf in zip(shapes, xs, qs, ss, bs, ys, bufs):
         check_canaries(buf, M, N)

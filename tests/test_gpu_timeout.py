@@ -40,18 +40,19 @@ def _case(kind):
         x = I.activations(M, 1024, 4, device="cuda")
         return lambda y: tq.w4g_gemm(x, qw, sc, None, y=y, path=path), (M, 384)
     p, s = tq.tq_quantize_pack(I.weights(384, 1024, 1, device="cuda"))
-    if kind == "batch":
+    if kind in ("batch", "batch_tc"):
         M = 8
         x = I.activations(M, 1024, 2, device="cuda")
         ws = tq.batch_workspace()
-        return lambda y: tq.tq_gemm_batch([x], [p], [s], None, [y], workspace=ws), (M, 384), ws
+        v = tq.BATCH_TENSOR_CORE if kind == "batch_tc" else tq.BATCH_MMA_SYNC
+        return lambda y: tq.tq_gemm_batch([x], [p], [s], None, [y], workspace=ws, variant=v), (M, 384), ws
     M, path = {"decode": (1, tq.PATH_DECODE), "decode_m16": (16, tq.PATH_DECODE),
                "prefill": (256, tq.PATH_PREFILL), "prefill_splitk": (64, tq.PATH_PREFILL)}[kind]
     x = I.activations(M, 1024, 2, device="cuda")
     return lambda y: tq.tq_gemm(x, p, s, None, y=y, path=path), (M, 384)
 
 
-@pytest.mark.parametrize("kind", ["decode", "decode_m16", "prefill", "prefill_splitk", "batch",
+@pytest.mark.parametrize("kind", ["decode", "decode_m16", "prefill", "prefill_splitk", "batch", "batch_tc",
                                   "w4g_decode", "w4g_prefill"])
 def test_wait_runs_out_then_recovers(kind):
     need_cuda()
@@ -65,7 +66,7 @@ def test_wait_runs_out_then_recovers(kind):
         run(y)                                   # returns: the launch itself is fine
         assert tq.tq_device_status() == TQ_ERR_TIMEOUT
     assert tq.tq_device_status() == 0            # read and cleared
-    if kind == "batch":                          # an aborted batch leaves its counters alone
+    if kind.startswith("batch"):                 # an aborted batch leaves its counters alone
         ws = case[2]
         n = 2 * torch.cuda.get_device_properties(0).multi_processor_count
         assert int(ws[: 4 * n].view(torch.int32).abs().sum().item()) == 0

@@ -129,14 +129,15 @@ def test_repack_moves_every_nibble():
     assert np.array_equal(got, u.numpy()[:, perm.numpy()])
 
 
-@pytest.mark.parametrize("M", [1, 16])
-def test_zero_point_batch(M):
+@pytest.mark.parametrize("variant,M", [(tq.BATCH_MMA_SYNC, 1), (tq.BATCH_MMA_SYNC, 16), (tq.BATCH_TENSOR_CORE, 1),
+                                       (tq.BATCH_TENSOR_CORE, 32)])
+def test_zero_point_batch(variant, M):
     need_cuda()
     shapes = [(1000, 1152), (200, 4096), (4096, 4096)]
     probs = [_zp_problem(M, N, K, 31 + i) for i, (N, K) in enumerate(shapes)]
     ws = tq.batch_workspace()
     ys = tq.w4g_gemm_batch([p[0] for p in probs], [p[1] for p in probs], [p[2] for p in probs],
-                           [p[4] for p in probs], workspace=ws, zeros_list=[p[3] for p in probs])
+                           [p[4] for p in probs], workspace=ws, zeros_list=[p[3] for p in probs], variant=variant)
     torch.cuda.synchronize()
     for (x, qw, sc, zp, b), y, (N, K) in zip(probs, ys, shapes):
         _check_zp(x, qw, sc, zp, b, y, cols=None if N <= 1000 else np.arange(0, N, 7), label=f"zp batch {N}x{K}")
