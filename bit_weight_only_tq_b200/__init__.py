@@ -82,6 +82,7 @@ _SIGS = {
     "w4g_gemm_zp_ex": [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _vp],
     "w4g_repack_act_order": [_vp, _vp, _vp, _i64, _i64, _vp],
     "tq_permute_columns": [_vp, _vp, _vp, _i64, _i64, _vp],
+    "tq_shard_plan": [_int, _int, _i64, _i64, _int, _int, _vp],
     "tq_select_path": [_int, _i64, _i64, _i64, _int],
     "tq_device_status": [],
     "tq_status_string": [_int],

@@ -453,6 +453,42 @@ int w4g_gemm_batch_ex(const tq_linear* items, int count, int64_t M, void* worksp
   return gemm_batch_impl<true>(items, count, M, workspace, workspace_bytes, variant, stream);
 }
 
+int tq_shard_plan(int fmt, int mode, int64_t N, int64_t K, int world, int rank, tq_shard* out) {
+  if (!out) return TQ_ERR_NULL;
+  if (fmt != TQ_FMT_TERNARY && fmt != TQ_FMT_W4G128) return TQ_ERR_PATH;
+  if (mode != TQ_SHARD_ROWS && mode != TQ_SHARD_K) return TQ_ERR_PATH;
+  if (world < 1 || rank < 0 || rank >= world || N < 0 || K <= 0) return TQ_ERR_SHAPE;
+  const bool int4 = fmt == TQ_FMT_W4G128;
+  if (int4 && K % 128 != 0) return TQ_ERR_SHAPE;
+  const int64_t pf = int4 ? 8 : 4;  // packed factor: elements per byte (ternary) / per int32 word
+  tq_shard r{};
+  if (mode == TQ_SHARD_ROWS) {
+    r.row0 = N * rank / world;
+    r.rows = N * (rank + 1) / world - r.row0;
+    r.k0 = 0;
+    r.cols = K;
+    r.packed0 = 0;
+    r.packed = (K + pf - 1) / pf;
+    r.group0 = 0;
+    r.groups = int4 ? K / 128 : 0;
+    r.scale_full = 0;
+  } else {
+    const int64_t unit = int4 ? 128 : 4;
+    if (K % world != 0 || (K / world) % unit != 0) return TQ_ERR_SHAPE;
+    r.row0 = 0;
+    r.rows = N;
+    r.cols = K / world;
+    r.k0 = r.cols * rank;
+    r.packed0 = r.k0 / pf;
+    r.packed = r.cols / pf;
+    r.group0 = int4 ? r.k0 / 128 : 0;
+    r.groups = int4 ? r.cols / 128 : 0;
+    r.scale_full = int4 ? 0 : 1;
+  }
+  *out = r;
+  return TQ_OK;
+}
+
 int tq_validate_packed(const uint8_t* packed, int64_t N, int64_t K, int* bad_count, void* stream) {
   if (N < 0 || K <= 0) return TQ_ERR_SHAPE;
   if (!bad_count) return TQ_ERR_NULL;

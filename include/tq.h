@@ -292,6 +292,35 @@ TQ_API int w4g_gemm_batch_ex(const tq_linear* items, int count, int64_t M, void*
  * device that is current in the calling thread (it depends on the number of SMs). */
 TQ_API size_t tq_batch_workspace_size(void);
 
+/* --------------------------------------------------------------------------------------------
+ * tq_shard_plan -- what one rank of a tensor-parallel group holds of a packed matrix [N, K]
+ * ([TQ] §5.2: under tensor parallelism each GPU keeps a part of the weight but the FULL per-row
+ * scale, shared by broadcast, never gathered; [VQ] §4.2 _adjust_shard_indexes_for_packing: a
+ * shard's offset and size along the packed dimension are divided by the packed factor).
+ *   fmt    tq_format; mode: TQ_SHARD_ROWS or TQ_SHARD_K; world >= 1; 0 <= rank < world.
+ *   TQ_SHARD_ROWS  output rows [row0, row0 + rows) with row0 = floor(N rank / world) (sizes
+ *                  differ by at most one); every column; the scales of the rank's rows.  The
+ *                  ranks' y are concatenated along N.
+ *   TQ_SHARD_K     every row; input columns [k0, k0 + K/world); K / world must be a multiple of
+ *                  4 (ternary: whole bytes) or 128 (W4A16: whole groups), else TQ_ERR_SHAPE.
+ *                  Ternary scales are the full-row scales of all N rows (scale_full = 1); W4A16
+ *                  scales / zero-points are the rank's groups.  The ranks' y are summed.
+ *   out    packed0 / packed: the same columns in packed units (bytes for ternary, int32 words
+ *          for W4A16), i.e. k0 / packed factor and (K / world) / packed factor; group0 / groups:
+ *          W4A16 scale and zero-point columns.
+ * Host arithmetic only (no device access).  Returns TQ_OK, TQ_ERR_SHAPE, TQ_ERR_PATH (fmt or
+ * mode unknown) or TQ_ERR_NULL.
+ * ------------------------------------------------------------------------------------------ */
+typedef enum { TQ_SHARD_ROWS = 0, TQ_SHARD_K = 1 } tq_shard_mode;
+typedef struct tq_shard {
+    int64_t row0, rows;
+    int64_t k0, cols;
+    int64_t packed0, packed;
+    int64_t group0, groups;
+    int scale_full;
+} tq_shard;
+TQ_API int tq_shard_plan(int fmt, int mode, int64_t N, int64_t K, int world, int rank, tq_shard* out);
+
 /* tq_validate_packed -- count the bytes of a packed ternary matrix [N, ceil(K/4)] that hold
  * the unused code 0b11 in one of their first K codes of the row ([TQ] §3.1: the table maps
  * 00/01/10 only).  *bad_count (device int) is OVERWRITTEN with the count (set to 0 first, on

@@ -12,7 +12,7 @@ import bit_weight_only_tq_b200 as tq
 
 def test_library_exports_every_header_function():
     names = tq.header_functions()
-    assert len(names) == 25
+    assert len(names) == 26
     for n in names:
         assert hasattr(tq.lib, n), n
     for n in ("tq_quantize_pack", "tq_gemm", "w4g_quantize_pack", "w4g_gemm", "tq_validate_packed",
