@@ -64,7 +64,7 @@ struct BatchParams {
 template <bool kInt4>
 struct BatchLayout {
   static constexpr int kRes = 16 * kBResPitch * 4;
-  __host__ __device__ static constexpr int fixed() { return 1024 + kRes + 2 * kDMaxRing * 8 + 16; }
+  __host__ __device__ static constexpr int fixed() { return 1024 + kRes + 2 * kDMaxRing * 8 + 2 * 8 + 16; }
   __host__ __device__ static constexpr int bytes(int ring, int stage) { return fixed() + ring * stage; }
 };
 
@@ -91,7 +91,9 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
   float* res = reinterpret_cast<float*>(stg + P.ring * P.stage);       // [16 tokens][kBResPitch]
   uint64_t* full = reinterpret_cast<uint64_t*>(res + 16 * kBResPitch);
   uint64_t* empty = full + kDMaxRing;
-  volatile int* flags = reinterpret_cast<volatile int*>(empty + kDMaxRing);  // [0] abort, [1] last
+  uint64_t* resfull = empty + kDMaxRing;   // a row block's sum is in `res` (consumers)      count 1
+  uint64_t* resempty = resfull + 1;        // `res` read by the epilogue warp                 count 1
+  volatile int* flags = reinterpret_cast<volatile int*>(resempty + 1);  // [0] abort
 
   pdl_allow_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -103,8 +105,9 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], W::kCons);
     }
+    mbar_init(resfull, 1);
+    mbar_init(resempty, 1);
     flags[0] = 0;
-    flags[1] = 0;
     fence_mbar_init();
   }
   __syncthreads();
@@ -172,6 +175,84 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
     return;
   }
 
+  if (warp == W::kCons + 1) {
+    // ==================================================================== epilogue warp
+    // Walks the row blocks of the range in order.  Per block: the scale and bias of its rows
+    // (lane + 32 j) are requested, then it waits until the consumers have put the block's sum
+    // in `res`, writes y (a block finished in this CTA) or, for a block split between CTAs,
+    // stores this CTA's partial in its workspace slot and counts itself in; the last
+    // contributor adds the slots in K order and writes y.  The consumers meanwhile go on with
+    // the next stages: they only wait for `res` at their next block end.
+    pdl_wait_prior_grids();  // y and the workspace belong to the previous kernel until now
+    int it = it0, rb = rb0, kst = k0, u = 0;
+    bool ok = true;
+    for (int i = 0; i < nst; ++i) {
+      const BatchItem& I = P.it[it];
+      if (kst == I.C - 1 || i == nst - 1) {
+        const int64_t row0 = static_cast<int64_t>(rb) * kBRows;
+        float es[4], eb[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int64_t n = row0 + lane + 32 * j;
+          es[j] = 1.0f;
+          eb[j] = 0.0f;
+          if (n < I.N) {
+            if (!kInt4) es[j] = __half2float(I.sc[n]);
+            if (I.bias) eb[j] = __half2float(I.bias[n]);
+          }
+        }
+        if (ok) ok = mbar_wait_warp(resfull, static_cast<uint32_t>(u & 1));
+        const bool abort = !ok || flags[0] != 0;
+        const int64_t gB0 = I.begin + static_cast<int64_t>(rb) * I.C, gB1 = gB0 + I.C;  // the block's stages
+        auto out = [&](float v, int tok, int j) {
+          const int64_t n = row0 + lane + 32 * j;
+          if (n < I.N) I.y[static_cast<int64_t>(tok) * I.N + n] = __float2half_rn(kInt4 ? v + eb[j] : fmaf(v, es[j], eb[j]));
+        };
+        if (!abort && gB0 >= s0 && gB1 <= s1) {
+          for (int tok = 0; tok < P.M; ++tok)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) out(res[tok * kBResPitch + lane + 32 * j], tok, j);
+        } else if (!abort) {
+          const int cf = range_owner(gB0, P.T, P.G), cl = range_owner(gB1 - 1, P.T, P.G);
+          float* mine = P.slots + (2 * static_cast<int64_t>(c) + (gB0 <= s0 ? 0 : 1)) * 16 * kBRows;
+          for (int tok = 0; tok < P.M; ++tok)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) mine[tok * kBRows + lane + 32 * j] = res[tok * kBResPitch + lane + 32 * j];
+          __threadfence();
+          __syncwarp();
+          int last = 0;
+          if (lane == 0) last = atomicAdd(&P.counters[cf], 1) == cl - cf;
+          last = __shfl_sync(0xFFFFFFFFu, last, 0);
+          if (last) {
+            __threadfence();
+            for (int tok = 0; tok < P.M; ++tok)
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                float sum = 0.0f;
+                for (int cc = cf; cc <= cl; ++cc) {  // K order: deterministic
+                  const int64_t sl = 2 * static_cast<int64_t>(cc) + (gB0 <= range_begin(cc, P.T, P.G) ? 0 : 1);
+                  sum += __ldcg(P.slots + sl * 16 * kBRows + tok * kBRows + lane + 32 * j);
+                }
+                out(sum, tok, j);
+              }
+            if (lane == 0) P.counters[cf] = 0;  // ready for the next call
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(resempty);  // `res` is free again
+        ++u;
+      }
+      if (++kst == I.C) {
+        kst = 0;
+        if (++rb == I.RB) {
+          rb = 0;
+          ++it;
+        }
+      }
+    }
+    return;
+  }
+
   // ====================================================================== consumer warps
   const int g = lane >> 2, t = lane & 3;
   const int rs = warp & (kDRowSets - 1), hi = warp / kDRowSets;  // hi: K half (M <= 8) or token group
@@ -183,8 +264,6 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
   const int gp = (g >> 1) | ((g & 1) << 2);
   const int rw = rs * 16 * kDRT + gp;
   const DecLane L{g, t, gp, rw, sub_lo, sub_hi, Tb};
-  const int e = threadIdx.x;          // epilogue thread: row e % 128, tokens e / 128 + step
-  const int er = e & (kBRows - 1);
 
   float acc[kDRT][TW][4];
   auto zero_acc = [&]() {
@@ -197,22 +276,12 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
   };
   zero_acc();
 
-  int it = it0, rb = rb0, kst = k0;
+  int it = it0, rb = rb0, kst = k0, u = 0;
   bool ok = true;
-  float ep_s = 1.0f, ep_b = 0.0f;  // this thread's epilogue row: scale (ternary) and bias
-  pdl_wait_prior_grids();          // x, y and the workspace belong to the previous kernel until now
+  pdl_wait_prior_grids();          // x belongs to the previous kernel until now
   for (int i = 0; i < nst; ++i) {
     const BatchItem& I = P.it[it];
     const int64_t row0 = static_cast<int64_t>(rb) * kBRows;
-    if (i == 0 || kst == 0) {  // a row block starts: fetch its epilogue constants early
-      const int64_t n = row0 + er;
-      ep_s = 1.0f;
-      ep_b = 0.0f;
-      if (n < I.N) {
-        if (!kInt4) ep_s = __half2float(I.sc[n]);
-        if (I.bias) ep_b = __half2float(I.bias[n]);
-      }
-    }
     const int slot = i % P.ring;
     if (ok) ok = mbar_wait_warp(&full[slot], static_cast<uint32_t>(i / P.ring) & 1u);
     if (ok) {
@@ -229,8 +298,10 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
       float v[kDRT][TW][4];
       dec_values<kInt4, TW>(acc, v);
       zero_acc();
-      // this CTA's sum over its stages of the block, [token][row] in `res`; for M <= 8 the two
-      // K halves (warps 4-7, then 0-3) are added in a fixed order
+      // this CTA's sum over its stages of the block, [token][row] in `res`, once the epilogue
+      // warp has taken the previous block's; for M <= 8 the two K halves (warps 4-7, then 0-3)
+      // are added in a fixed order
+      if (u > 0 && ok) ok = mbar_wait_warp(resempty, static_cast<uint32_t>((u - 1) & 1));
       if (NT == 1 && hi == 0) named_barrier_sync(1, kEp);
 #pragma unroll
       for (int rt = 0; rt < kDRT; ++rt)
@@ -246,47 +317,9 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
           }
       if (NT == 1 && hi == 1) named_barrier_sync(1, kEp);
       named_barrier_sync(1, kEp);
-
-      const int64_t gB0 = I.begin + static_cast<int64_t>(rb) * I.C;  // the block's stages [gB0, gB1)
-      const int64_t gB1 = gB0 + I.C;
-      const bool whole = gB0 >= s0 && gB1 <= s1;
-      const bool abort = flags[0] != 0;
-      const int64_t n = row0 + er;
-      auto out = [&](float acc_v, int tok) {
-        const float r = kInt4 ? acc_v + ep_b : fmaf(acc_v, ep_s, ep_b);
-        I.y[static_cast<int64_t>(tok) * I.N + n] = __float2half_rn(r);
-      };
-      if (!abort && whole) {
-        if (n < I.N)
-          for (int tok = e >> 7; tok < P.M; tok += kEp / kBRows) out(res[tok * kBResPitch + er], tok);
-      } else if (!abort) {
-        // split block: my partial to my slot, count in; the last contributor sums the slots
-        const int cf = range_owner(gB0, P.T, P.G), cl = range_owner(gB1 - 1, P.T, P.G);
-        float* mine = P.slots + (2 * static_cast<int64_t>(c) + (gB0 <= s0 ? 0 : 1)) * 16 * kBRows;
-        for (int tok = e >> 7; tok < P.M; tok += kEp / kBRows) mine[tok * kBRows + er] = res[tok * kBResPitch + er];
-        named_barrier_sync(1, kEp);
-        if (e == 0) {
-          __threadfence();
-          const int old = atomicAdd(&P.counters[cf], 1);
-          const int last = old == cl - cf;
-          if (last) __threadfence();
-          flags[1] = last;
-        }
-        named_barrier_sync(1, kEp);
-        if (flags[1]) {
-          if (n < I.N)
-            for (int tok = e >> 7; tok < P.M; tok += kEp / kBRows) {
-              float sum = 0.0f;
-              for (int cc = cf; cc <= cl; ++cc) {  // K order: deterministic
-                const int64_t sl = 2 * static_cast<int64_t>(cc) + (gB0 <= range_begin(cc, P.T, P.G) ? 0 : 1);
-                sum += __ldcg(P.slots + sl * 16 * kBRows + tok * kBRows + er);
-              }
-              out(sum, tok);
-            }
-          if (e == 0) P.counters[cf] = 0;  // ready for the next call
-        }
-      }
-      named_barrier_sync(1, kEp);  // `res` and the flag are free again
+      if (!ok) flags[0] = 1;
+      if (threadIdx.x == 0) mbar_arrive(resfull);  // hand the block to the epilogue warp
+      ++u;
     }
     if (++kst == I.C) {
       kst = 0;
@@ -298,13 +331,19 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
   }
 }
 
+// Threads: the consumer warps, the producer warp, the epilogue warp.
+template <int NT, int TW>
+constexpr int batch_threads() { return DecWarps<NT, TW>::kThreads + 32; }
+
+// M <= 8: two CTAs of ten warps per SM; five warps share one SM sub-partition's 16K registers,
+// so a thread may use at most 102 (96 it is).
 template <bool kInt4>
 __global__ void __maxnreg__(96) batch_decode_kernel_m8(const __grid_constant__ BatchParams P) {
   batch_body<kInt4, 1, 1>(P);
 }
 
 template <bool kInt4>
-__global__ void __launch_bounds__(DecWarps<2, 2>::kThreads, 2) batch_decode_kernel_m16(const __grid_constant__ BatchParams P) {
+__global__ void __launch_bounds__(batch_threads<2, 2>(), 2) batch_decode_kernel_m16(const __grid_constant__ BatchParams P) {
   batch_body<kInt4, 2, 2>(P);
 }
 
@@ -379,7 +418,7 @@ static cudaError_t launch_batch_t(const BatchLinear* items, int count, int64_t M
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(P.G), 1, 1);
-  cfg.blockDim = dim3(m16 ? DecWarps<2, 2>::kThreads : DecWarps<1, 1>::kThreads, 1, 1);
+  cfg.blockDim = dim3(m16 ? batch_threads<2, 2>() : batch_threads<1, 1>(), 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = s;
   cudaLaunchAttribute attr[1];

@@ -35,8 +35,8 @@
 //     after the loop.  The activation fragments are x pairs (p, p + 8), picked with byte permutes.
 //   W4A16: ANDing a word with 0x000F000F (nibbles at bits 0-3) or 0x00F000F0 (bits 4-7) leaves
 //     u * 2^-24 or u * 2^-20 in each half (fp16 subnormals, exactly linear in u); one fp16x2
-//     subtraction of 8 units gives (u - 8) times that power of two exactly.  The two fields
-//     accumulate in separate chains, combined with an exact factor 16, and each 128-wide
+//     subtraction of z units gives (u - z) times that power of two exactly.  The two fields
+//     accumulate in separate chains, combined with an exact factor 1/16, and each 128-wide
 //     quantisation group (one 64-byte sub-chunk) is scaled as y += s[n,g] * 2^24 * sum_g (u - 8) x.
 #include <cuda.h>
 #include <cuda_fp16.h>
@@ -291,14 +291,14 @@ __device__ __forceinline__ void dec_stage(float (&acc)[kDRT][TW][4], const uint8
         }
 #pragma unroll
       for (int rt = 0; rt < kDRT; ++rt) {
-        // the group's sum of (u - 8) x in units of 2^-24: the second field's chain times 16
-        // (exact powers of two)
+        // the group's sum of (u - z) x in units of 2^-24: the second field's chain (units of
+        // 2^-20) times 1/16 (exact powers of two)
         const float s0u = sg[rt][0] * 16777216.0f, s1u = sg[rt][1] * 16777216.0f;
 #pragma unroll
         for (int T = 0; T < TW; ++T) {
           float c4[4];
 #pragma unroll
-          for (int c = 0; c < 4; ++c) c4[c] = fmaf(cg[1][rt][T][c], 16.0f, cg[0][rt][T][c]);
+          for (int c = 0; c < 4; ++c) c4[c] = fmaf(cg[1][rt][T][c], 0.0625f, cg[0][rt][T][c]);
           acc[rt][T][0] = fmaf(s0u, c4[0], acc[rt][T][0]);
           acc[rt][T][1] = fmaf(s0u, c4[1], acc[rt][T][1]);
           acc[rt][T][2] = fmaf(s1u, c4[2], acc[rt][T][2]);

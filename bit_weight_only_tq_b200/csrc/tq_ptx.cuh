@@ -73,18 +73,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
 }
 
 // Wait for the phase with the given parity to complete.  Returns false (and records a timeout
-// in the device status word) if it has not completed within kWaitLimitCycles.
-// Retries back off with nanosleep so that a waiting warp leaves the issue slots to the warps
-// (of this or a co-resident CTA) that do the work.
+// in the device status word) if it has not completed within the wait limit (g_tq_wait_limit SM
+// clock cycles).  mbarrier.try_wait itself suspends the thread in hardware until the phase
+// completes or a short system-defined window passes, so the loop polls it back to back (a
+// software sleep would only add latency after the phase completes); the clock is read every
+// 64 polls.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const long long t0 = clock64();
-  uint32_t backoff = 0;
   while (true) {
-    if (mbar_try_wait(a, parity)) return true;
-    if (backoff < 256) backoff += 32;
-    __nanosleep(backoff);
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(a, parity)) return true;
     if (clock64() - t0 > *reinterpret_cast<volatile long long*>(&g_tq_wait_limit)) {
       record_timeout();
       return false;

@@ -294,14 +294,29 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_batch_kernel(const __grid_co
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp - 4) * 32) << 16);
     TcPos p = pos0;
     int a = 0;
-    int64_t g_cur = -1;
-    uint16_t sc_cur = 0;
-    uint32_t zp_cur = 8u;
+    // W4A16: the scales and zero-points of a stage's two groups, fetched one stage ahead so that
+    // their latency stays off the decode
+    uint32_t scv[2] = {0u, 0u}, zv[2] = {8u, 8u}, scn[2] = {0u, 0u}, zn[2] = {8u, 8u};
+    auto fetch_groups = [&](const TcPos& q, uint32_t (&sc)[2], uint32_t (&z)[2]) {
+      const TcItem& J = P.it[q.it];
+      const int64_t nn = static_cast<int64_t>(q.rb) * 128 + r, G = J.K >> 7;
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int64_t gi = static_cast<int64_t>(q.kst) * 2 + j;
+        const bool in = nn < J.N && gi < G;
+        sc[j] = in ? static_cast<uint32_t>(__half_as_ushort(J.sc[nn * G + gi])) : 0u;
+        z[j] = (in && J.zp) ? static_cast<uint32_t>(J.zp[nn * G + gi]) : 8u;
+      }
+    };
+    if (kInt4 && nst > 0) fetch_groups(pos0, scv, zv);
     for (int i = 0; i < nst; ++i) {
       const int slot = i % P.ring;
+      if (kInt4 && i + 1 < nst) {
+        TcPos q = p;
+        q.advance(P);
+        fetch_groups(q, scn, zn);
+      }
       if (ok) ok = mbar_wait_warp(&full[slot], static_cast<uint32_t>(i / P.ring) & 1u);
-      const TcItem& I = P.it[p.it];
-      const int64_t n = static_cast<int64_t>(p.rb) * 128 + r;
       const uint8_t* prow = stg + slot * L::kStage + r * 128;
       for (int sub = 0; sub < L::kSubs; ++sub, ++a) {
         const int as = a % kTcARing;
@@ -314,16 +329,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_batch_kernel(const __grid_co
 #pragma unroll
             for (int pp = 0; pp < 8; ++pp) v[8 * q + pp] = tc_dec_tq(wq[q], pp);
         } else {
-          const int64_t G = I.K >> 7;
-          const int64_t gi = static_cast<int64_t>(p.kst) * 2 + (sub >> 1);
-          if (gi != g_cur) {
-            const bool in = n < I.N && gi < G;
-            sc_cur = in ? __half_as_ushort(I.sc[n * G + gi]) : static_cast<uint16_t>(0);
-            zp_cur = (in && I.zp) ? static_cast<uint32_t>(I.zp[n * G + gi]) : 8u;
-            g_cur = gi;
-          }
-          const uint32_t s2 = static_cast<uint32_t>(sc_cur) | (static_cast<uint32_t>(sc_cur) << 16);
-          const uint32_t zsub = ((0x5400u + 16u * zp_cur) << 16) | (0x6400u + zp_cur);
+          const uint32_t sg = scv[sub >> 1], zg = zv[sub >> 1];
+          const uint32_t s2 = sg | (sg << 16);
+          const uint32_t zsub = ((0x5400u + 16u * zg) << 16) | (0x6400u + zg);
           const uint4 p0 = *reinterpret_cast<const uint4*>(prow + (((2 * sub) ^ (r & 7)) << 4));
           const uint4 p1 = *reinterpret_cast<const uint4*>(prow + (((2 * sub + 1) ^ (r & 7)) << 4));
           const uint32_t wq[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
@@ -346,6 +354,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_batch_kernel(const __grid_co
       if (lane == 0 && ok) mbar_arrive(&empty[slot]);
       if (!ok) flags[0] = 1;
       p.advance(P);
+      if (kInt4) {
+        scv[0] = scn[0];
+        scv[1] = scn[1];
+        zv[0] = zn[0];
+        zv[1] = zn[1];
+      }
     }
   } else {
     // ==================================================================== epilogue
@@ -440,8 +454,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_batch_kernel(const __grid_co
 // ---------------------------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------------------------
+// Workspace: the counter region of the mma.sync variant (sized for two CTAs per SM, so that one
+// layout serves both variants), then [2 G][32][128] fp32 slots.
 int64_t tc_batch_workspace_bytes_for(int G) {
-  return ((static_cast<int64_t>(G) * 4 + 255) / 256) * 256 + 2 * static_cast<int64_t>(G) * kTcSlotTokens * 128 * 4;
+  return batch_counter_bytes(kBCtasPerSm * G) + 2 * static_cast<int64_t>(G) * kTcSlotTokens * 128 * 4;
 }
 
 template <bool kInt4, int TN>
@@ -492,7 +508,7 @@ static cudaError_t launch_tc_t(const BatchLinear* items, int count, int64_t M, v
   P.ring = ring;
   const int smem = L::bytes(ring);
   P.counters = reinterpret_cast<int*>(ws);
-  P.slots = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + ((static_cast<int64_t>(Gmax) * 4 + 255) / 256) * 256);
+  P.slots = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + batch_counter_bytes(kBCtasPerSm * Gmax));
   auto* kern = tc_batch_kernel<kInt4, TN>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
