@@ -74,6 +74,7 @@ _SIGS = {
     "w4g_gemm_batch": [_vp, _int, _i64, _vp, ctypes.c_size_t, _vp],
     "tq_batch_workspace_size": [],
     "tq_gemm_batch_ex": [_vp, _int, _i64, _vp, ctypes.c_size_t, _int, _vp],
+    "tq_gemm_batch_noalloc": [_vp, _int, _i64, _vp],
     "w4g_gemm_batch_ex": [_vp, _int, _i64, _vp, ctypes.c_size_t, _int, _vp],
     "tq_debug_set_wait_limit": [ctypes.c_longlong],
     "tq_debug_skip_activation_loads": [_int],
@@ -380,6 +381,36 @@ def w4g_gemm_batch(xs, qweight_list, scales_list, bias_list=None, y_list=None, w
     """Independent W4A16 linears sharing M in one persistent launch (zero-points optional)."""
     return _batch(lib.w4g_gemm_batch_ex, xs, qweight_list, scales_list, bias_list, y_list, workspace, torch.int32, 2,
                   "w4g_gemm_batch", stream, zeros=zeros_list, variant=variant)
+
+
+def tq_gemm_batch_noalloc(xs, packed_list, scale_list, bias_list=None, y_list=None, stream=None):
+    """tq_gemm_batch with the library's own static scratch: no workspace argument, nothing
+    allocated by the library (the outputs are allocated here only when y_list is None).  Calls
+    that may overlap on one device share that scratch and must be serialised."""
+    count = len(packed_list)
+    if not (1 <= count <= 8) or len(scale_list) != count or len(xs) != count:
+        raise ValueError("1..8 linears, each with its x, weights and scales")
+    biases = [None] * count if bias_list is None else list(bias_list)
+    M = xs[0].shape[0]
+    items = (TqLinear * count)()
+    out = []
+    for i, (x, w, s, b) in enumerate(zip(xs, packed_list, scale_list, biases)):
+        _need(x, torch.float16, "x", 2)
+        _need(w, torch.uint8, "packed", 2)
+        _need(s, torch.float16, "scale", 1)
+        _need(b, torch.float16, "bias", 1)
+        if x.shape[0] != M:
+            raise ValueError("every x of a batch has the same number of tokens M")
+        N, K = w.shape[0], x.shape[1]
+        y = torch.empty(M, N, dtype=torch.float16, device=x.device) if y_list is None else y_list[i]
+        _need(y, torch.float16, "y", 2)
+        if tuple(y.shape) != (M, N):
+            raise ValueError("y shape mismatch")
+        items[i] = TqLinear(x.data_ptr(), w.data_ptr(), s.data_ptr(), None if b is None else b.data_ptr(),
+                            y.data_ptr(), N, K, None)
+        out.append(y)
+    _check(lib.tq_gemm_batch_noalloc(items, count, M, _stream(stream)), "tq_gemm_batch_noalloc")
+    return out
 
 
 def tq_validate_packed(packed: torch.Tensor, K: int, stream=None) -> int:

@@ -440,3 +440,54 @@ cudaError_t launch_w4g_gemm_batch(const BatchLinear* items, int count, int64_t M
 }
 
 }  // namespace tq
+
+namespace tq {
+
+// =============================================================================================
+// Allocation-free batch entry point (tq_gemm_batch_noalloc)
+// =============================================================================================
+// Some callers cannot hand the batch call a workspace and must not allocate one: a custom
+// operator behind an interface that passes only its inputs and outputs, or a process whose
+// device memory is all reserved by its framework's caching allocator (a raw cudaMalloc there
+// fails, or synchronises the device in the middle of a step).  For them the workspace lives in
+// this file-scope device array, which every GPU that loads the library holds until the process
+// exits.  Its size covers GPUs with up to kNoAllocMaxSms SMs (5.0 MiB).
+constexpr int kNoAllocMaxSms = 160;
+constexpr int64_t kNoAllocCounterBytes = ((static_cast<int64_t>(kBCtasPerSm) * kNoAllocMaxSms * 4 + 255) / 256) * 256;
+constexpr int64_t kNoAllocScratchBytes =
+    kNoAllocCounterBytes + 2 * static_cast<int64_t>(kBCtasPerSm) * kNoAllocMaxSms * 16 * kBRows * 4;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+// The device address of the array on the current device.  In host code `g_noalloc_scratch` is
+// only a host-side stand-in for the symbol (a kernel given it would fault, or silently use host
+// memory): the address is looked up once per device with that device current, and cached.
+static void* noalloc_scratch_on_current_device() {
+  static std::atomic<void*> addr[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  void* p = addr[dev].load(std::memory_order_acquire);
+  if (p) return p;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return nullptr;
+  addr[dev].store(p, std::memory_order_release);
+  return p;
+}
+
+}  // namespace tq
+
+extern "C" TQ_API int tq_gemm_batch_noalloc(const tq_linear* items, int count, int64_t M, void* stream) {
+  // the argument checks of tq_gemm_batch, before any device work
+  if (count < 1 || count > tq::kBatchMaxItems || M < 0 || M > tq::kBatchMaxM) return TQ_ERR_SHAPE;
+  if (!items) return TQ_ERR_NULL;
+  if (M == 0) return TQ_OK;
+  // the workspace this device needs must fit in the static array
+  if (tq::batch_workspace_bytes() > tq::kNoAllocScratchBytes) return TQ_ERR_SHAPE;
+  void* ws = tq::noalloc_scratch_on_current_device();
+  if (!ws) return TQ_ERR_CUDA;
+  // every call shares the array: the arrival counters must start at zero (a completed call
+  // leaves them zero, a failed one may not), so they are cleared on the caller's stream
+  if (cudaMemsetAsync(ws, 0, static_cast<size_t>(tq::kNoAllocCounterBytes), reinterpret_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return TQ_ERR_CUDA;
+  return gemm_batch_impl<false>(items, count, M, ws, static_cast<size_t>(tq::kNoAllocScratchBytes), TQ_BATCH_AUTO,
+                                stream);
+}

@@ -288,6 +288,30 @@ TQ_API int tq_gemm_batch_ex(const tq_linear* items, int count, int64_t M, void* 
 TQ_API int w4g_gemm_batch_ex(const tq_linear* items, int count, int64_t M, void* workspace,
                              size_t workspace_bytes, int variant, void* stream);
 
+/* --------------------------------------------------------------------------------------------
+ * tq_gemm_batch_noalloc -- tq_gemm_batch without a workspace argument and without allocating.
+ * (An addition of this library for its callers; the pages have no counterpart.)
+ *
+ * For callers that get no workspace buffer from their host framework and must not allocate
+ * one: a custom operator behind an interface that passes only inputs and outputs, or a process
+ * whose device memory is all reserved by its framework's caching allocator, where a raw
+ * cudaMalloc fails or synchronises the device mid-step.  The batch kernel's scratch (arrival
+ * counters and partial sums) lives instead in one static device array of 5.0 MiB inside the
+ * library, which every GPU that loads the library holds until the process exits; it covers
+ * GPUs with up to 160 SMs.
+ *
+ *   items, count, M, stream  as tq_gemm_batch (ternary linears, AUTO variant).
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
+ * that device current and caches it: make that first call before any stream capture.  Every
+ * call clears the array's counters on `stream` before its kernel, and all calls share the
+ * array: calls that may overlap on the GPU (different streams, or different host threads on
+ * one device) race and give wrong results; serialise them.  No cudaMalloc, cudaFree or other
+ * allocating call is made.
+ * Errors: as tq_gemm_batch; TQ_ERR_SHAPE also when the current device has more SMs than the
+ * array covers; TQ_ERR_CUDA when the address lookup or the clear fails.
+ * ------------------------------------------------------------------------------------------ */
+TQ_API int tq_gemm_batch_noalloc(const tq_linear* items, int count, int64_t M, void* stream);
+
 /* tq_batch_workspace_size -- bytes of workspace tq_gemm_batch / w4g_gemm_batch need on the
  * device that is current in the calling thread (it depends on the number of SMs). */
 TQ_API size_t tq_batch_workspace_size(void);

@@ -12,7 +12,7 @@ import bit_weight_only_tq_b200 as tq
 
 def test_library_exports_every_header_function():
     names = tq.header_functions()
-    assert len(names) == 26
+    assert len(names) == 27
     for n in names:
         assert hasattr(tq.lib, n), n
     for n in ("tq_quantize_pack", "tq_gemm", "w4g_quantize_pack", "w4g_gemm", "tq_validate_packed",
@@ -135,6 +135,13 @@ def test_batch_argument_errors_without_gpu():
     assert tq.lib.tq_gemm_batch(_items((q, a, a, a, 64, 128)), 1, 1, ws, big, None) == -3   # misaligned x
     assert tq.lib.tq_gemm_batch(_items((a, q, a, a, 64, 128)), 1, 1, ws, big, None) == -3   # misaligned w
     assert tq.lib.tq_gemm_batch(ok, 1, 1, None, big, None) == -1                # no workspace
+    # the allocation-free variant checks the same arguments before any device work
+    assert tq.lib.tq_gemm_batch_noalloc(ok, 0, 1, None) == -2
+    assert tq.lib.tq_gemm_batch_noalloc(ok, 9, 1, None) == -2
+    assert tq.lib.tq_gemm_batch_noalloc(ok, 1, 33, None) == -2
+    assert tq.lib.tq_gemm_batch_noalloc(ok, 1, -1, None) == -2
+    assert tq.lib.tq_gemm_batch_noalloc(None, 1, 1, None) == -1
+    assert tq.lib.tq_gemm_batch_noalloc(ok, 1, 0, None) == 0
     assert tq.lib.tq_gemm_batch(ok, 1, 1, ctypes.c_void_p(1 << 20 | 4), big, None) == -3
     need = tq.tq_batch_workspace_size()
     assert need > 0
