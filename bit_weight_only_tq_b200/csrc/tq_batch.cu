@@ -177,23 +177,29 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
 
   if (warp == W::kCons + 1) {
     // ==================================================================== epilogue warp
-    // Walks the row blocks of the range in order.  Per block: the scale and bias of its rows
-    // (lane + 32 j) are requested, then it waits until the consumers have put the block's sum
-    // in `res`, writes y (a block finished in this CTA) or, for a block split between CTAs,
-    // stores this CTA's partial in its workspace slot and counts itself in; the last
-    // contributor adds the slots in K order and writes y.  The consumers meanwhile go on with
+    // Walks the row blocks of the range in order.  Lane l owns rows 4l .. 4l + 3 of a block for
+    // every token: one float4 of each token's row of `res` or of a workspace slot.  Per block:
+    // the scale and bias of its rows are requested, then it waits until the consumers have put
+    // the block's sum in `res`, writes y (a block finished in this CTA) or, for a block split
+    // between CTAs, stores this CTA's partial in its workspace slot, frees `res` and counts
+    // itself in; the last contributor adds the slots in K order and writes y.  Every load of
+    // one slot is issued before the first add (one round trip per contributor: under the
+    // weight stream an L2 round trip takes microseconds).  The consumers meanwhile go on with
     // the next stages: they only wait for `res` at their next block end.
+    constexpr int kTok = 8 * NT;  // tokens a launch of this shape holds at most
+    constexpr int kQ = kBRows / 4;  // float4 per token row of a slot
+    constexpr int kCh = NT == 1 ? 4 : 8;
     pdl_wait_prior_grids();  // y and the workspace belong to the previous kernel until now
     int it = it0, rb = rb0, kst = k0, u = 0;
     bool ok = true;
     for (int i = 0; i < nst; ++i) {
       const BatchItem& I = P.it[it];
       if (kst == I.C - 1 || i == nst - 1) {
-        const int64_t row0 = static_cast<int64_t>(rb) * kBRows;
+        const int64_t n0 = static_cast<int64_t>(rb) * kBRows + 4 * lane;
         float es[4], eb[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const int64_t n = row0 + lane + 32 * j;
+          const int64_t n = n0 + j;
           es[j] = 1.0f;
           eb[j] = 0.0f;
           if (n < I.N) {
@@ -201,23 +207,46 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
             if (I.bias) eb[j] = __half2float(I.bias[n]);
           }
         }
+        // y rows n0 .. n0 + 3 of one token from its four fp32 sums
+        const bool vec = (I.N & 3) == 0 && (reinterpret_cast<uintptr_t>(I.y) & 7) == 0;
+        auto put = [&](int tok, const float4& a) {
+          const float r[4] = {a.x, a.y, a.z, a.w};
+          __half h[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) h[j] = __float2half_rn(kInt4 ? r[j] + eb[j] : fmaf(r[j], es[j], eb[j]));
+          __half* yp = I.y + static_cast<int64_t>(tok) * I.N + n0;
+          if (vec && n0 + 3 < I.N) {
+            uint2 pk;
+            pk.x = static_cast<uint32_t>(__half_as_ushort(h[0])) | (static_cast<uint32_t>(__half_as_ushort(h[1])) << 16);
+            pk.y = static_cast<uint32_t>(__half_as_ushort(h[2])) | (static_cast<uint32_t>(__half_as_ushort(h[3])) << 16);
+            *reinterpret_cast<uint2*>(yp) = pk;
+          } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              if (n0 + j < I.N) yp[j] = h[j];
+          }
+        };
+        auto res4 = [&](int tok) { return *reinterpret_cast<const float4*>(res + tok * kBResPitch + 4 * lane); };
         if (ok) ok = mbar_wait_warp(resfull, static_cast<uint32_t>(u & 1));
         const bool abort = !ok || flags[0] != 0;
         const int64_t gB0 = I.begin + static_cast<int64_t>(rb) * I.C, gB1 = gB0 + I.C;  // the block's stages
-        auto out = [&](float v, int tok, int j) {
-          const int64_t n = row0 + lane + 32 * j;
-          if (n < I.N) I.y[static_cast<int64_t>(tok) * I.N + n] = __float2half_rn(kInt4 ? v + eb[j] : fmaf(v, es[j], eb[j]));
-        };
         if (!abort && gB0 >= s0 && gB1 <= s1) {
-          for (int tok = 0; tok < P.M; ++tok)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) out(res[tok * kBResPitch + lane + 32 * j], tok, j);
-        } else if (!abort) {
+          for (int q = 0; q < kTok; ++q)
+            if (q < P.M) put(q, res4(q));
+          __syncwarp();
+          if (lane == 0) mbar_arrive(resempty);  // `res` is free again
+        } else if (abort) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(resempty);
+        } else {
           const int cf = range_owner(gB0, P.T, P.G), cl = range_owner(gB1 - 1, P.T, P.G);
-          float* mine = P.slots + (2 * static_cast<int64_t>(c) + (gB0 <= s0 ? 0 : 1)) * 16 * kBRows;
-          for (int tok = 0; tok < P.M; ++tok)
+          float4* mine = reinterpret_cast<float4*>(P.slots + (2 * static_cast<int64_t>(c) + (gB0 <= s0 ? 0 : 1)) * 16 * kBRows);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) mine[tok * kBRows + lane + 32 * j] = res[tok * kBResPitch + lane + 32 * j];
+          for (int q = 0; q < kTok; ++q)
+            if (q < P.M) mine[q * kQ + lane] = res4(q);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(resempty);
           __threadfence();
           __syncwarp();
           int last = 0;
@@ -225,21 +254,37 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
           last = __shfl_sync(0xFFFFFFFFu, last, 0);
           if (last) {
             __threadfence();
-            for (int tok = 0; tok < P.M; ++tok)
+            // kCh tokens at a time (what the registers allow): all loads of a slot for them in flight
+            // together, K order kept
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                float sum = 0.0f;
-                for (int cc = cf; cc <= cl; ++cc) {  // K order: deterministic
-                  const int64_t sl = 2 * static_cast<int64_t>(cc) + (gB0 <= range_begin(cc, P.T, P.G) ? 0 : 1);
-                  sum += __ldcg(P.slots + sl * 16 * kBRows + tok * kBRows + lane + 32 * j);
-                }
-                out(sum, tok, j);
+            for (int q0 = 0; q0 < kTok; q0 += kCh) {
+              if (q0 >= P.M) break;
+              float4 v[kCh];
+#pragma unroll
+              for (int q = 0; q < kCh; ++q) v[q] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+              for (int cc = cf; cc <= cl; ++cc) {  // K order: deterministic
+                const int64_t sl = 2 * static_cast<int64_t>(cc) + (gB0 <= range_begin(cc, P.T, P.G) ? 0 : 1);
+                const float4* src = reinterpret_cast<const float4*>(P.slots + sl * 16 * kBRows) + lane;
+                float4 t[kCh];
+#pragma unroll
+                for (int q = 0; q < kCh; ++q)
+                  if (q0 + q < P.M) t[q] = __ldcg(src + (q0 + q) * kQ);
+#pragma unroll
+                for (int q = 0; q < kCh; ++q)
+                  if (q0 + q < P.M) {
+                    v[q].x += t[q].x;
+                    v[q].y += t[q].y;
+                    v[q].z += t[q].z;
+                    v[q].w += t[q].w;
+                  }
               }
+#pragma unroll
+              for (int q = 0; q < kCh; ++q)
+                if (q0 + q < P.M) put(q0 + q, v[q]);
+            }
             if (lane == 0) P.counters[cf] = 0;  // ready for the next call
           }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(resempty);  // `res` is free again
         ++u;
       }
       if (++kst == I.C) {

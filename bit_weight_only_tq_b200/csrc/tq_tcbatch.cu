@@ -422,14 +422,29 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_batch_kernel(const __grid_co
           }
           named_barrier_sync(2, 128);
           if (flags[1]) {
+            // eight tokens at a time: every load of a slot for them is in flight before the first
+            // add (one L2 round trip per contributor, not one per token)
             if (n < I.N)
-              for (int tok = 0; tok < Mt; ++tok) {
-                float sum = 0.0f;
+#pragma unroll
+              for (int q0 = 0; q0 < TN; q0 += 8) {
+                if (q0 >= Mt) break;
+                float v[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) v[q] = 0.0f;
                 for (int cc = cf; cc <= cl; ++cc) {  // K order: deterministic
                   const int64_t sl = 2 * static_cast<int64_t>(cc) + (gB0 <= tc_range_begin(cc, P.T, P.G) ? 0 : 1);
-                  sum += __ldcg(P.slots + sl * kTcSlotTokens * 128 + tok * 128 + e);
+                  const float* src = P.slots + sl * kTcSlotTokens * 128 + e;
+                  float t[8];
+#pragma unroll
+                  for (int q = 0; q < 8; ++q)
+                    if (q0 + q < Mt) t[q] = __ldcg(src + (q0 + q) * 128);
+#pragma unroll
+                  for (int q = 0; q < 8; ++q)
+                    if (q0 + q < Mt) v[q] += t[q];
                 }
-                I.y[static_cast<int64_t>(tok) * I.N + n] = __float2half_rn(fmaf(sum, ep_s, ep_b));
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                  if (q0 + q < Mt) I.y[static_cast<int64_t>(q0 + q) * I.N + n] = __float2half_rn(fmaf(v[q], ep_s, ep_b));
               }
             if (e == 0) P.counters[cf] = 0;
           }
