@@ -55,6 +55,7 @@ struct BatchParams {
   int M;
   int G;                      // CTAs
   int ring, stage, xhalf;
+  uint32_t four;              // 4 (decode multiplier, see DecLane)
   int64_t T;                  // stages in total
   int* counters;              // [G] arrivals per split row block, indexed by its first contributor
   float* slots;               // [2 G][16][128] fp32 partials: slot 2c = CTA c's first row block,
@@ -64,7 +65,8 @@ struct BatchParams {
 template <bool kInt4>
 struct BatchLayout {
   static constexpr int kRes = 16 * kBResPitch * 4;
-  __host__ __device__ static constexpr int fixed() { return 1024 + kRes + 2 * kDMaxRing * 8 + 2 * 8 + 16; }
+  static constexpr int kItems = kBMaxItems * static_cast<int>(sizeof(BatchItem));
+  __host__ __device__ static constexpr int fixed() { return 1024 + kRes + 2 * kDMaxRing * 8 + 2 * 8 + 16 + kItems; }
   __host__ __device__ static constexpr int bytes(int ring, int stage) { return fixed() + ring * stage; }
 };
 
@@ -75,9 +77,12 @@ __host__ __device__ inline int64_t batch_workspace_bytes_for(int G) {
 }
 
 // First stage of CTA c's range, and the CTA whose range holds stage s.
-__device__ __forceinline__ int64_t range_begin(int c, int64_t T, int G) { return (static_cast<int64_t>(c) * T) / G; }
+// (The host keeps T * G below 2^32, so both are exact in 32-bit arithmetic.)
+__device__ __forceinline__ int64_t range_begin(int c, int64_t T, int G) {
+  return static_cast<int64_t>(static_cast<uint32_t>(c) * static_cast<uint32_t>(T) / static_cast<uint32_t>(G));
+}
 __device__ __forceinline__ int range_owner(int64_t s, int64_t T, int G) {
-  return static_cast<int>(((s + 1) * G - 1) / T);
+  return static_cast<int>((static_cast<uint32_t>(s + 1) * static_cast<uint32_t>(G) - 1u) / static_cast<uint32_t>(T));
 }
 
 template <bool kInt4, int NT, int TW>
@@ -94,12 +99,18 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
   uint64_t* resfull = empty + kDMaxRing;   // a row block's sum is in `res` (consumers)      count 1
   uint64_t* resempty = resfull + 1;        // `res` read by the epilogue warp                 count 1
   volatile int* flags = reinterpret_cast<volatile int*>(resempty + 1);  // [0] abort
+  // the items, copied from the launch parameters once: indexed reads of a parameter block go
+  // through the generic load path, shared memory is a short-latency read
+  BatchItem* its = reinterpret_cast<BatchItem*>(resempty + 3);
 
   pdl_allow_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = static_cast<int>(blockIdx.x);
   const int64_t s0 = range_begin(c, P.T, P.G), s1 = range_begin(c + 1, P.T, P.G);
   const int nst = static_cast<int>(s1 - s0);
+  static_assert(sizeof(BatchItem) % 4 == 0, "items are copied as words");
+  if (threadIdx.x < P.count * static_cast<int>(sizeof(BatchItem) / 4))
+    reinterpret_cast<uint32_t*>(its)[threadIdx.x] = reinterpret_cast<const uint32_t*>(P.it)[threadIdx.x];
   if (threadIdx.x == 0) {
     for (int i = 0; i < P.ring; ++i) {
       mbar_init(&full[i], 1);
@@ -115,9 +126,10 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
 
   // position of the range's first stage: item, row block, stage within the row block
   int it0 = 0;
-  while (it0 + 1 < P.count && P.it[it0 + 1].begin <= s0) ++it0;
-  const int rb0 = static_cast<int>((s0 - P.it[it0].begin) / P.it[it0].C);
-  const int k0 = static_cast<int>((s0 - P.it[it0].begin) % P.it[it0].C);
+  while (it0 + 1 < P.count && its[it0 + 1].begin <= s0) ++it0;
+  const uint32_t off0 = static_cast<uint32_t>(s0 - its[it0].begin);
+  const int rb0 = static_cast<int>(off0 / static_cast<uint32_t>(its[it0].C));
+  const int k0 = static_cast<int>(off0 % static_cast<uint32_t>(its[it0].C));
 
   if (warp == W::kCons) {
     // ==================================================================== producer warp
@@ -127,49 +139,56 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
         tma_prefetch_desc(&P.w[q]);
         tma_prefetch_desc(&P.x[q]);
       }
-      int it = it0, rb = rb0, kst = k0;
+      const int ring = P.ring;
+      int it = it0, rb = rb0, kst = k0, C = its[it0].C;
       auto advance = [&]() {
-        if (++kst == P.it[it].C) {
+        if (++kst == C) {
           kst = 0;
-          if (++rb == P.it[it].RB) {
+          if (++rb == its[it].RB) {
             rb = 0;
             ++it;
+            if (it < P.count) C = its[it].C;
           }
         }
       };
-      auto load_w = [&](int i) {
-        tma_load_2d(stg + (i % P.ring) * P.stage, &P.w[it], &full[i % P.ring], kst * 128, rb * kBRows);
+      auto load_w = [&](int slot) {
+        tma_load_2d(stg + slot * P.stage, &P.w[it], &full[slot], kst * 128, rb * kBRows);
       };
       const bool skipx = skip_x_loads();  // failure-path test hook: never set in normal use
-      auto load_x = [&](int i) {
+      auto load_x = [&](int slot) {
         if (skipx) return;
-        uint8_t* dst = stg + (i % P.ring) * P.stage + kDWBytes;
+        uint8_t* dst = stg + slot * P.stage + kDWBytes;
 #pragma unroll
         for (int hb = 0; hb < F::kKB / 4; ++hb)
-          tma_load_3d(dst + hb * P.xhalf, &P.x[it], &full[i % P.ring], 0, kst * F::kKB + 4 * hb, 0);
+          tma_load_3d(dst + hb * P.xhalf, &P.x[it], &full[slot], 0, kst * F::kKB + 4 * hb, 0);
       };
-      const int pre = nst < P.ring ? nst : P.ring;
+      const int pre = nst < ring ? nst : ring;
       for (int i = 0; i < pre; ++i) {  // weights are model constants: before the wait
         mbar_arrive_expect_tx(&full[i], tx);
         load_w(i);
         advance();
       }
       pdl_wait_prior_grids();  // the activations may come from the previous kernel
-      it = it0, rb = rb0, kst = k0;
+      it = it0, rb = rb0, kst = k0, C = its[it0].C;
       for (int i = 0; i < pre; ++i) {
         load_x(i);
         advance();
       }
+      int slot = 0;
+      uint32_t ph = 0;  // parity of the slot's last completed `empty` phase
       for (int i = pre; i < nst; ++i) {
-        const int slot = i % P.ring;
-        if (!mbar_wait(&empty[slot], static_cast<uint32_t>((i / P.ring) - 1) & 1u)) {
+        if (!mbar_wait(&empty[slot], ph)) {
           flags[0] = 1;
           break;
         }
         mbar_arrive_expect_tx(&full[slot], tx);
-        load_w(i);
-        load_x(i);
+        load_w(slot);
+        load_x(slot);
         advance();
+        if (++slot == ring) {
+          slot = 0;
+          ph ^= 1u;
+        }
       }
     }
     return;
@@ -193,7 +212,7 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
     int it = it0, rb = rb0, kst = k0, u = 0;
     bool ok = true;
     for (int i = 0; i < nst; ++i) {
-      const BatchItem& I = P.it[it];
+      const BatchItem& I = its[it];
       if (kst == I.C - 1 || i == nst - 1) {
         const int64_t n0 = static_cast<int64_t>(rb) * kBRows + 4 * lane;
         float es[4], eb[4];
@@ -241,21 +260,10 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
           if (lane == 0) mbar_arrive(resempty);
         } else {
           const int cf = range_owner(gB0, P.T, P.G), cl = range_owner(gB1 - 1, P.T, P.G);
-          float4* mine = reinterpret_cast<float4*>(P.slots + (2 * static_cast<int64_t>(c) + (gB0 <= s0 ? 0 : 1)) * 16 * kBRows);
-#pragma unroll
-          for (int q = 0; q < kTok; ++q)
-            if (q < P.M) mine[q * kQ + lane] = res4(q);
-          __syncwarp();
-          if (lane == 0) mbar_arrive(resempty);
-          __threadfence();
-          __syncwarp();
-          int last = 0;
-          if (lane == 0) last = atomicAdd(&P.counters[cf], 1) == cl - cf;
-          last = __shfl_sync(0xFFFFFFFFu, last, 0);
-          if (last) {
-            __threadfence();
-            // kCh tokens at a time (what the registers allow): all loads of a slot for them in flight
-            // together, K order kept
+          // Adds the contributors' partials in K order (CTA cf first) and writes y: kCh tokens at
+          // a time (what the registers allow), all loads of a slot for them in flight together.
+          // This CTA's own partial comes from `res` when `own` is set, else from its slot.
+          auto sum_and_write = [&](bool own) {
 #pragma unroll
             for (int q0 = 0; q0 < kTok; q0 += kCh) {
               if (q0 >= P.M) break;
@@ -263,12 +271,18 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
 #pragma unroll
               for (int q = 0; q < kCh; ++q) v[q] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
               for (int cc = cf; cc <= cl; ++cc) {  // K order: deterministic
-                const int64_t sl = 2 * static_cast<int64_t>(cc) + (gB0 <= range_begin(cc, P.T, P.G) ? 0 : 1);
-                const float4* src = reinterpret_cast<const float4*>(P.slots + sl * 16 * kBRows) + lane;
                 float4 t[kCh];
+                if (own && cc == c) {
 #pragma unroll
-                for (int q = 0; q < kCh; ++q)
-                  if (q0 + q < P.M) t[q] = __ldcg(src + (q0 + q) * kQ);
+                  for (int q = 0; q < kCh; ++q)
+                    if (q0 + q < P.M) t[q] = res4(q0 + q);
+                } else {
+                  const int64_t sl = 2 * static_cast<int64_t>(cc) + (gB0 <= range_begin(cc, P.T, P.G) ? 0 : 1);
+                  const float4* src = reinterpret_cast<const float4*>(P.slots + sl * 16 * kBRows) + lane;
+#pragma unroll
+                  for (int q = 0; q < kCh; ++q)
+                    if (q0 + q < P.M) t[q] = __ldcg(src + (q0 + q) * kQ);
+                }
 #pragma unroll
                 for (int q = 0; q < kCh; ++q)
                   if (q0 + q < P.M) {
@@ -282,7 +296,37 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
               for (int q = 0; q < kCh; ++q)
                 if (q0 + q < P.M) put(q0 + q, v[q]);
             }
-            if (lane == 0) P.counters[cf] = 0;  // ready for the next call
+          };
+          // every other contributor already counted in (the usual case for the block that ends
+          // a range: the CTA after this one finished its part at its start): this CTA is last
+          // and needs neither its slot nor the atomic
+          int all = 0;
+          if (lane == 0) all = ld_acquire_gpu(&P.counters[cf]) == cl - cf;
+          all = __shfl_sync(0xFFFFFFFFu, all, 0);
+          if (all) {
+            sum_and_write(true);
+            __syncwarp();
+            if (lane == 0) {
+              mbar_arrive(resempty);
+              P.counters[cf] = 0;  // ready for the next call
+            }
+          } else {
+            float4* mine = reinterpret_cast<float4*>(P.slots + (2 * static_cast<int64_t>(c) + (gB0 <= s0 ? 0 : 1)) * 16 * kBRows);
+#pragma unroll
+            for (int q = 0; q < kTok; ++q)
+              if (q < P.M) mine[q * kQ + lane] = res4(q);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(resempty);
+            __threadfence();
+            __syncwarp();
+            int last = 0;
+            if (lane == 0) last = atomicAdd(&P.counters[cf], 1) == cl - cf;
+            last = __shfl_sync(0xFFFFFFFFu, last, 0);
+            if (last) {
+              __threadfence();
+              sum_and_write(false);
+              if (lane == 0) P.counters[cf] = 0;  // ready for the next call
+            }
           }
         }
         ++u;
@@ -308,7 +352,7 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
   for (int T = 0; T < TW; ++T) tokv[T] = 8 * (Tb + T) + g < P.M;
   const int gp = (g >> 1) | ((g & 1) << 2);
   const int rw = rs * 16 * kDRT + gp;
-  const DecLane L{g, t, gp, rw, sub_lo, sub_hi, Tb};
+  const DecLane L{g, t, gp, rw, sub_lo, sub_hi, Tb, P.four};
 
   float acc[kDRT][TW][4];
   auto zero_acc = [&]() {
@@ -322,13 +366,14 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
   zero_acc();
 
   int it = it0, rb = rb0, kst = k0, u = 0;
+  int slot = 0;
+  uint32_t ph = 0;  // parity of the slot's next `full` phase
   bool ok = true;
   pdl_wait_prior_grids();          // x belongs to the previous kernel until now
   for (int i = 0; i < nst; ++i) {
-    const BatchItem& I = P.it[it];
+    const BatchItem& I = its[it];
     const int64_t row0 = static_cast<int64_t>(rb) * kBRows;
-    const int slot = i % P.ring;
-    if (ok) ok = mbar_wait_warp(&full[slot], static_cast<uint32_t>(i / P.ring) & 1u);
+    if (ok) ok = mbar_wait_warp(&full[slot], ph);
     if (ok) {
       dec_stage<kInt4, NT, TW>(acc, stg + slot * P.stage, P.xhalf, L, tokv, static_cast<int64_t>(kst) * 2, row0,
                                I.N, I.sc, I.zp, I.K >> 7);
@@ -336,6 +381,10 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
       if (lane == 0) mbar_arrive(&empty[slot]);
     } else {
       flags[0] = 1;  // a wait ran out (recorded in the device status word): results are void
+    }
+    if (++slot == P.ring) {
+      slot = 0;
+      ph ^= 1u;
     }
 
     if (kst == I.C - 1 || i == nst - 1) {
@@ -447,7 +496,9 @@ static cudaError_t launch_batch_t(const BatchLinear* items, int count, int64_t M
   if (ws_bytes < batch_workspace_bytes_for(Gmax)) return cudaErrorInvalidValue;
   P.T = T;
   P.G = static_cast<int>(T < Gmax ? T : Gmax);
+  if (T * P.G >= (static_cast<int64_t>(1) << 32)) return cudaErrorInvalidValue;  // 32-bit range arithmetic
   P.xhalf = ((static_cast<int>(M) * 4 * 128 + 1023) / 1024) * 1024;
+  P.four = 4u;
   P.stage = kDWBytes + (F::kKB / 4) * P.xhalf;
   int ring = kDMaxRing;
   while (ring > 2 && L::bytes(ring, P.stage) > kDSmemBudget) --ring;

@@ -84,6 +84,7 @@ struct DecodeArgs {
   int ring;       // stages resident in shared memory
   int stage;      // bytes of one stage (weights + activations, multiple of 1024)
   int xhalf;      // bytes of one activation box [M][4 blocks][64] (multiple of 1024)
+  uint32_t four;  // 4 (decode multiplier, see DecLane)
   int count;                        // matrices in the group
   int rb_start[kDMaxGroup + 1];     // first row block of each matrix in grid.y
   int64_t N[kDMaxGroup];
@@ -144,6 +145,7 @@ __device__ __forceinline__ uint32_t dec_field(uint32_t w, uint32_t mask, uint32_
 // this warp covers and its first token group.
 struct DecLane {
   int g, t, gp, rw, sub_lo, sub_hi, Tb;
+  uint32_t four;  // 4, from the launch parameters: the compiler cannot turn `x * four` into a shift
 };
 
 // One stage of the consumer loop: this warp's rows (two 16-row tiles) x its sub-chunks of the
@@ -158,10 +160,6 @@ struct DecLane {
 //   c = 0b00 -> 0xC000 = -2,  c = 0b01 -> 0x8000 = -0,  c = 0b10 -> 0x4000 = +2,
 // i.e. exactly 2 (c - 1): one shift and one LOP3 per two weights, no arithmetic.  (Code 0b11 is
 // invalid and decodes to +0.)
-__device__ __forceinline__ uint32_t dec_tq_pos(uint32_t w, int p) {
-  const uint32_t s = p == 7 ? w : (w << (14 - 2 * p));
-  return ~s & 0xC000C000u;
-}
 
 template <bool kInt4, int NT, int TW>
 __device__ __forceinline__ void dec_stage(float (&acc)[kDRT][TW][4], const uint8_t* st, int xhalf,
@@ -205,9 +203,21 @@ __device__ __forceinline__ void dec_stage(float (&acc)[kDRT][TW][4], const uint8
             P[T][4 * jj + 3] = v.w;
           }
         // position p of words 2h (k = 64 chunk + 32h + p, + p + 8) and 2h + 1 (+ 16 + p, + 24 + p):
-        // x pairs (p, p + 8) are the even (p even) or odd halves of P[p / 2] and P[p / 2 + 4]
+        // x pairs (p, p + 8) are the even (p even) or odd halves of P[p / 2] and P[p / 2 + 4].
+        // Positions run 7 .. 0 on running copies of the words moved two bits left per step
+        // (code p at bits 14-15 / 30-31); the move is a multiply by four, which runs on the FMA
+        // pipe and leaves the integer ALU pipe to the masks and the x permutes.
+        uint32_t sw[kDRT][4];
 #pragma unroll
-        for (int p = 0; p < 8; ++p) {
+        for (int rt = 0; rt < kDRT; ++rt) {
+          sw[rt][0] = w[rt][0][2 * h];
+          sw[rt][1] = w[rt][1][2 * h];
+          sw[rt][2] = w[rt][0][2 * h + 1];
+          sw[rt][3] = w[rt][1][2 * h + 1];
+        }
+#pragma unroll
+        for (int pp = 0; pp < 8; ++pp) {
+          const int p = 7 - pp;
           const uint32_t sel = (p & 1) ? 0x7632u : 0x5410u;
           uint32_t b0[TW], b1[TW];
 #pragma unroll
@@ -217,8 +227,12 @@ __device__ __forceinline__ void dec_stage(float (&acc)[kDRT][TW][4], const uint8
           }
 #pragma unroll
           for (int rt = 0; rt < kDRT; ++rt) {
-            const uint32_t a0 = dec_tq_pos(w[rt][0][2 * h], p), a1 = dec_tq_pos(w[rt][1][2 * h], p);
-            const uint32_t a2 = dec_tq_pos(w[rt][0][2 * h + 1], p), a3 = dec_tq_pos(w[rt][1][2 * h + 1], p);
+            if (pp > 0) {
+#pragma unroll
+              for (int j = 0; j < 4; ++j) sw[rt][j] *= L.four;
+            }
+            const uint32_t a0 = ~sw[rt][0] & 0xC000C000u, a1 = ~sw[rt][1] & 0xC000C000u;
+            const uint32_t a2 = ~sw[rt][2] & 0xC000C000u, a3 = ~sw[rt][3] & 0xC000C000u;
 #pragma unroll
             for (int T = 0; T < TW; ++T) mma_16816(acc[rt][T], a0, a1, a2, a3, b0[T], b1[T]);
           }
@@ -443,7 +457,7 @@ __device__ __forceinline__ void decode_gemm_body(const DecodeMaps& maps, const D
     const int gp = (g >> 1) | ((g & 1) << 2);
     const int rw = rs * 16 * kDRT + gp;  // row of tile 0, lower half; tile rt adds 16 rt, upper +8
     const int64_t G = a.K >> 7;
-    const DecLane L{g, t, gp, rw, sub_lo, sub_hi, Tb};
+    const DecLane L{g, t, gp, rw, sub_lo, sub_hi, Tb, a.four};
     pdl_wait_prior_grids();  // block (not poll) until the previous kernel is done
     for (int i = 0; i < nst; ++i) {
       const int slot = i % a.ring;
@@ -651,6 +665,7 @@ static cudaError_t launch_decode_group(const __half* x, int count, const void* c
   a.ring = p.ring;
   a.stage = p.stage;
   a.xhalf = p.xhalf;
+  a.four = 4u;
   if (NT == 1) return launch_decode_t<kInt4, 1, 1>(maps, a, p, s);
   // a CTA with a single stage and two CTAs per SM: more, lighter warps hide the latency better
   const bool single = (p.C + p.S - 1) / p.S <= 1 && static_cast<int64_t>(p.S) * rbs * chunks > di.num_sms;

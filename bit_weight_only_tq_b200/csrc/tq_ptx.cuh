@@ -72,25 +72,44 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
   return ok != 0;
 }
 
+// try_wait with an explicit suspend-time hint: a thread whose phase has not completed is
+// suspended in hardware until the phase completes or `hint_ns` nanoseconds pass, issuing
+// nothing meanwhile (the default window is short, and a warp that polls takes issue slots
+// from the warps that compute beside it on its SM sub-partition).
+__device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar_addr, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar_addr), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete.  Returns false (and records a timeout
 // in the device status word) if it has not completed within the wait limit (g_tq_wait_limit SM
-// clock cycles).  mbarrier.try_wait itself suspends the thread in hardware until the phase
-// completes or a short system-defined window passes, so the loop polls it back to back (a
-// software sleep would only add latency after the phase completes); the clock is read every
-// 64 polls.
+// clock cycles).  Each try_wait suspends the thread until the phase completes or 20 us pass, so
+// the loop issues a few instructions per 20 us at most; the clock is read after every try.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const long long t0 = clock64();
   while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 64; ++i)
-      if (mbar_try_wait(a, parity)) return true;
+    if (mbar_try_wait_hint(a, parity, 20000u)) return true;
     if (clock64() - t0 > *reinterpret_cast<volatile long long*>(&g_tq_wait_limit)) {
       record_timeout();
       return false;
     }
   }
+}
+
+// Load with acquire semantics at GPU scope (pairs with a release, or a fence and a relaxed write).
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
 }
 
 // Named barrier `id` (1..15) over the first `nthreads` threads (a multiple of 32) that use it.

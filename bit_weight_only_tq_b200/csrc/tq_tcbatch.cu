@@ -83,8 +83,13 @@ struct TcParams {
   float* slots;                   // [2G][32][128]
 };
 
-__device__ __forceinline__ int64_t tc_range_begin(int c, int64_t T, int G) { return (static_cast<int64_t>(c) * T) / G; }
-__device__ __forceinline__ int tc_range_owner(int64_t s, int64_t T, int G) { return static_cast<int>(((s + 1) * G - 1) / T); }
+// (The host keeps T * G below 2^32, so both are exact in 32-bit arithmetic.)
+__device__ __forceinline__ int64_t tc_range_begin(int c, int64_t T, int G) {
+  return static_cast<int64_t>(static_cast<uint32_t>(c) * static_cast<uint32_t>(T) / static_cast<uint32_t>(G));
+}
+__device__ __forceinline__ int tc_range_owner(int64_t s, int64_t T, int G) {
+  return static_cast<int>((static_cast<uint32_t>(s + 1) * static_cast<uint32_t>(G) - 1u) / static_cast<uint32_t>(T));
+}
 
 // Position (item, row block, stage within the row block) walked stage by stage.
 struct TcPos {
@@ -175,8 +180,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_batch_kernel(const __grid_co
   TcPos pos0{0, 0, 0};
   if (nst > 0) {
     while (pos0.it + 1 < P.count && P.it[pos0.it + 1].begin <= s0) ++pos0.it;
-    pos0.rb = static_cast<int>((s0 - P.it[pos0.it].begin) / P.it[pos0.it].C);
-    pos0.kst = static_cast<int>((s0 - P.it[pos0.it].begin) % P.it[pos0.it].C);
+    const uint32_t off0 = static_cast<uint32_t>(s0 - P.it[pos0.it].begin);
+    pos0.rb = static_cast<int>(off0 / static_cast<uint32_t>(P.it[pos0.it].C));
+    pos0.kst = static_cast<int>(off0 % static_cast<uint32_t>(P.it[pos0.it].C));
   }
   auto unit_end = [&](const TcPos& p, int i) { return p.kst == P.it[p.it].C - 1 || i == nst - 1; };
 
@@ -518,6 +524,7 @@ static cudaError_t launch_tc_t(const BatchLinear* items, int count, int64_t M, v
   if (ws_bytes < tc_batch_workspace_bytes_for(Gmax)) return cudaErrorInvalidValue;
   P.T = T;
   P.G = static_cast<int>(T < Gmax ? T : Gmax);
+  if (T * P.G >= (static_cast<int64_t>(1) << 32)) return cudaErrorInvalidValue;  // 32-bit range arithmetic
   int ring = kTcMaxRing;
   while (ring > 2 && L::bytes(ring) > 227 * 1024) --ring;
   P.ring = ring;
