@@ -35,6 +35,7 @@ constexpr int kBMaxItems = kBatchMaxItems;
 constexpr int kBRows = 128;       // rows of a row block (one packed TMA tile)
 constexpr int kBResPitch = 132;   // fp32 row pitch of the result buffer [token][row]
 constexpr int kBCtasPerSm = 2;
+constexpr bool kBatchM8FourWarps = false;  // M <= 8: four consumer warps over whole stages
 
 struct BatchItem {
   const __half* sc;    // ternary: scale[N]; W4A16: scales[N, K/128]
@@ -85,11 +86,15 @@ __device__ __forceinline__ int range_owner(int64_t s, int64_t T, int G) {
   return static_cast<int>((static_cast<uint32_t>(s + 1) * static_cast<uint32_t>(G) - 1u) / static_cast<uint32_t>(T));
 }
 
-template <bool kInt4, int NT, int TW>
+// NT token groups of eight, TW of them per consumer warp, CW consumer warps.  With eight
+// consumer warps and one token group the two K halves of a stage go to two warp sets (kSplitK);
+// otherwise every consumer warp takes its rows over the whole stage.
+template <bool kInt4, int NT, int TW, int CW>
 __device__ __forceinline__ void batch_body(const BatchParams& P) {
   using F = DecFmt<kInt4>;
-  using W = DecWarps<NT, TW>;
-  constexpr int kEp = W::kCons * 32;  // consumer threads (epilogue)
+  constexpr int kCons = CW;
+  constexpr bool kSplitK = NT == 1 && CW == 8;
+  constexpr int kEp = kCons * 32;  // consumer threads (epilogue)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* stg = base;                                                 // ring x [weights | x]
@@ -114,7 +119,7 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
   if (threadIdx.x == 0) {
     for (int i = 0; i < P.ring; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], W::kCons);
+      mbar_init(&empty[i], kCons);
     }
     mbar_init(resfull, 1);
     mbar_init(resempty, 1);
@@ -131,7 +136,7 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
   const int rb0 = static_cast<int>(off0 / static_cast<uint32_t>(its[it0].C));
   const int k0 = static_cast<int>(off0 % static_cast<uint32_t>(its[it0].C));
 
-  if (warp == W::kCons) {
+  if (warp == kCons) {
     // ==================================================================== producer warp
     if (lane == 0) {
       const uint32_t tx = static_cast<uint32_t>(kDWBytes + F::kKB * P.M * 128);  // whole boxes
@@ -194,7 +199,7 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
     return;
   }
 
-  if (warp == W::kCons + 1) {
+  if (warp == kCons + 1) {
     // ==================================================================== epilogue warp
     // Walks the row blocks of the range in order.  Lane l owns rows 4l .. 4l + 3 of a block for
     // every token: one float4 of each token's row of `res` or of a workspace slot.  Per block:
@@ -207,7 +212,7 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
     // the next stages: they only wait for `res` at their next block end.
     constexpr int kTok = 8 * NT;  // tokens a launch of this shape holds at most
     constexpr int kQ = kBRows / 4;  // float4 per token row of a slot
-    constexpr int kCh = NT == 1 ? 4 : 8;
+    constexpr int kCh = kSplitK ? 4 : 8;  // the eight-consumer kernel has 96 registers a thread
     pdl_wait_prior_grids();  // y and the workspace belong to the previous kernel until now
     int it = it0, rb = rb0, kst = k0, u = 0;
     bool ok = true;
@@ -345,11 +350,14 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
   // ====================================================================== consumer warps
   const int g = lane >> 2, t = lane & 3;
   const int rs = warp & (kDRowSets - 1), hi = warp / kDRowSets;  // hi: K half (M <= 8) or token group
-  const int sub_lo = NT == 1 ? hi : 0, sub_hi = NT == 1 ? hi + 1 : 2;
+  const int sub_lo = kSplitK ? hi : 0, sub_hi = kSplitK ? hi + 1 : 2;
   const int Tb = TW < NT ? hi : 0;
-  bool tokv[TW];
+  // activation row of this lane's token 8 (Tb + T) + g (B column g of token group Tb + T); a
+  // lane past the last token reads the last token's row instead (its column is never stored),
+  // so the loads need neither a predicate nor zero fill
+  int xrow[TW];
 #pragma unroll
-  for (int T = 0; T < TW; ++T) tokv[T] = 8 * (Tb + T) + g < P.M;
+  for (int T = 0; T < TW; ++T) xrow[T] = 4 * min(8 * (Tb + T) + g, P.M - 1);
   const int gp = (g >> 1) | ((g & 1) << 2);
   const int rw = rs * 16 * kDRT + gp;
   const DecLane L{g, t, gp, rw, sub_lo, sub_hi, Tb, P.four};
@@ -375,7 +383,7 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
     const int64_t row0 = static_cast<int64_t>(rb) * kBRows;
     if (ok) ok = mbar_wait_warp(&full[slot], ph);
     if (ok) {
-      dec_stage<kInt4, NT, TW>(acc, stg + slot * P.stage, P.xhalf, L, tokv, static_cast<int64_t>(kst) * 2, row0,
+      dec_stage<kInt4, NT, TW>(acc, stg + slot * P.stage, P.xhalf, L, xrow, static_cast<int64_t>(kst) * 2, row0,
                                I.N, I.sc, I.zp, I.K >> 7);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);
@@ -396,7 +404,7 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
       // warp has taken the previous block's; for M <= 8 the two K halves (warps 4-7, then 0-3)
       // are added in a fixed order
       if (u > 0 && ok) ok = mbar_wait_warp(resempty, static_cast<uint32_t>((u - 1) & 1));
-      if (NT == 1 && hi == 0) named_barrier_sync(1, kEp);
+      if (kSplitK && hi == 0) named_barrier_sync(1, kEp);
 #pragma unroll
       for (int rt = 0; rt < kDRT; ++rt)
 #pragma unroll
@@ -404,12 +412,12 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
 #pragma unroll
           for (int ci = 0; ci < 4; ++ci) {
             float* dst = res + (8 * (Tb + T) + 2 * t + (ci & 1)) * kBResPitch + rw + 16 * rt + 8 * (ci >> 1);
-            if (NT == 1 && hi == 0)
+            if (kSplitK && hi == 0)
               *dst += v[rt][T][ci];
             else
               *dst = v[rt][T][ci];
           }
-      if (NT == 1 && hi == 1) named_barrier_sync(1, kEp);
+      if (kSplitK && hi == 1) named_barrier_sync(1, kEp);
       named_barrier_sync(1, kEp);
       if (!ok) flags[0] = 1;
       if (threadIdx.x == 0) mbar_arrive(resfull);  // hand the block to the epilogue warp
@@ -426,19 +434,25 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
 }
 
 // Threads: the consumer warps, the producer warp, the epilogue warp.
-template <int NT, int TW>
-constexpr int batch_threads() { return DecWarps<NT, TW>::kThreads + 32; }
+template <int CW>
+constexpr int batch_threads() { return (CW + 2) * 32; }
 
-// M <= 8: two CTAs of ten warps per SM; five warps share one SM sub-partition's 16K registers,
-// so a thread may use at most 102 (96 it is).
+// M <= 8, eight consumer warps (K halves split): two CTAs of ten warps per SM; five warps share
+// one SM sub-partition's 16K registers, so a thread may use at most 102 (96 it is).
 template <bool kInt4>
 __global__ void __maxnreg__(96) batch_decode_kernel_m8(const __grid_constant__ BatchParams P) {
-  batch_body<kInt4, 1, 1>(P);
+  batch_body<kInt4, 1, 1, 8>(P);
+}
+
+// M <= 8, four consumer warps, each over the whole stage (twice the MMAs per stage and warp).
+template <bool kInt4>
+__global__ void __launch_bounds__(batch_threads<4>(), 2) batch_decode_kernel_m8w4(const __grid_constant__ BatchParams P) {
+  batch_body<kInt4, 1, 1, 4>(P);
 }
 
 template <bool kInt4>
-__global__ void __launch_bounds__(batch_threads<2, 2>(), 2) batch_decode_kernel_m16(const __grid_constant__ BatchParams P) {
-  batch_body<kInt4, 2, 2>(P);
+__global__ void __launch_bounds__(batch_threads<4>(), 2) batch_decode_kernel_m16(const __grid_constant__ BatchParams P) {
+  batch_body<kInt4, 2, 2, 4>(P);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -509,12 +523,13 @@ static cudaError_t launch_batch_t(const BatchLinear* items, int count, int64_t M
   P.slots = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + batch_counter_bytes(Gmax));
 
   const bool m16 = M > 8;
-  auto* kern = m16 ? batch_decode_kernel_m16<kInt4> : batch_decode_kernel_m8<kInt4>;
+  const bool w4 = !m16 && kBatchM8FourWarps;
+  auto* kern = m16 ? batch_decode_kernel_m16<kInt4> : w4 ? batch_decode_kernel_m8w4<kInt4> : batch_decode_kernel_m8<kInt4>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), kDSmemBudget);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(P.G), 1, 1);
-  cfg.blockDim = dim3(m16 ? batch_threads<2, 2>() : batch_threads<1, 1>(), 1, 1);
+  cfg.blockDim = dim3(m16 || w4 ? batch_threads<4>() : batch_threads<8>(), 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = s;
   cudaLaunchAttribute attr[1];

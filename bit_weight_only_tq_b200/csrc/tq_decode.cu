@@ -163,10 +163,10 @@ struct DecLane {
 
 template <bool kInt4, int NT, int TW>
 __device__ __forceinline__ void dec_stage(float (&acc)[kDRT][TW][4], const uint8_t* st, int xhalf,
-                                          const DecLane& L, const bool (&tokv)[TW], int64_t gi_base,
+                                          const DecLane& L, const int (&xrow)[TW], int64_t gi_base,
                                           int64_t row0, int64_t Nm, const __half* scm, const uint8_t* zpm,
                                           int64_t G) {
-  const int g = L.g, t = L.t, gp = L.gp, rw = L.rw, Tb = L.Tb, sub_lo = L.sub_lo, sub_hi = L.sub_hi;
+  const int t = L.t, gp = L.gp, rw = L.rw, sub_lo = L.sub_lo, sub_hi = L.sub_hi;
   const uint8_t* xs = st + kDWBytes;
 #pragma unroll 1
   for (int sub = sub_lo; sub < sub_hi; ++sub) {
@@ -195,8 +195,7 @@ __device__ __forceinline__ void dec_stage(float (&acc)[kDRT][TW][4], const uint8
         for (int T = 0; T < TW; ++T)
 #pragma unroll
           for (int jj = 0; jj < 4; ++jj) {
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (tokv[T]) v = ld_x_chunk(xbox, 4 * (8 * (Tb + T) + g) + t, 4 * h + jj);
+            const uint4 v = ld_x_chunk(xbox, xrow[T] + t, 4 * h + jj);
             P[T][4 * jj] = v.x;
             P[T][4 * jj + 1] = v.y;
             P[T][4 * jj + 2] = v.z;
@@ -260,8 +259,7 @@ __device__ __forceinline__ void dec_stage(float (&acc)[kDRT][TW][4], const uint8
       for (int T = 0; T < TW; ++T)
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
-          uint4 v = make_uint4(0u, 0u, 0u, 0u);
-          if (tokv[T]) v = ld_x_chunk(xs, 4 * (8 * (Tb + T) + g) + (chunk >> 1), 4 * (chunk & 1) + jj);
+          const uint4 v = ld_x_chunk(xs, xrow[T] + (chunk >> 1), 4 * (chunk & 1) + jj);
           P[T][4 * jj] = v.x;
           P[T][4 * jj + 1] = v.y;
           P[T][4 * jj + 2] = v.z;
@@ -442,9 +440,9 @@ __device__ __forceinline__ void decode_gemm_body(const DecodeMaps& maps, const D
     const int rs = warp & (kDRowSets - 1), hi = warp / kDRowSets;  // hi: K half or token group
     const int sub_lo = NT == 1 ? hi : 0, sub_hi = NT == 1 ? hi + 1 : 2;
     const int Tb = TW < NT ? hi : 0;  // first token group of this warp
-    bool tokv[TW];  // this lane's token 8(Tb+T) + g (B column g of token group Tb+T) exists
+    int xrow[TW];  // activation row of this lane's token 8(Tb+T) + g (B column g of group Tb+T)
 #pragma unroll
-    for (int T = 0; T < TW; ++T) tokv[T] = 8 * (Tb + T) + g < Mi;
+    for (int T = 0; T < TW; ++T) xrow[T] = 4 * min(8 * (Tb + T) + g, static_cast<int>(Mi) - 1);
     float acc[kDRT][TW][4];
 #pragma unroll
     for (int rt = 0; rt < kDRT; ++rt)
@@ -464,7 +462,7 @@ __device__ __forceinline__ void decode_gemm_body(const DecodeMaps& maps, const D
       const uint32_t ph = static_cast<uint32_t>(i / a.ring) & 1u;
       if (!mbar_wait_warp(&full[slot], ph)) break;  // warp-uniform exit
       const uint8_t* st = stg + slot * a.stage;
-      dec_stage<kInt4, NT, TW>(acc, st, a.xhalf, L, tokv, static_cast<int64_t>(st_begin + i) * 2, row0, Nm, scm, zpm,
+      dec_stage<kInt4, NT, TW>(acc, st, a.xhalf, L, xrow, static_cast<int64_t>(st_begin + i) * 2, row0, Nm, scm, zpm,
                                G);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);

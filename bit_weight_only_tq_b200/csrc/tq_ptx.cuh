@@ -117,16 +117,10 @@ __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// Warp-wide wait (all 32 lanes call it): lane 0 polls with backoff; once the phase has completed
-// every lane performs one acquiring test of it, which then succeeds at once, so that each thread
-// itself observes the completion.  Returns the same value in every lane.
-__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity) {
-  int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity) ? 1 : 0;
-  ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-  if (ok) (void)mbar_try_wait(smem_u32(bar), parity);
-  return ok != 0;
-}
+// Warp-wide wait (all 32 lanes call it, converged): the lanes run the same bounded loop and see
+// the same phase, so every thread itself observes the completion with one try_wait per round
+// for the whole warp.  Returns the same value in every lane.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity) { return mbar_wait(bar, parity); }
 
 // ---------------------------------------------------------------------------------------------
 // Proxy fences
