@@ -373,57 +373,66 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
   };
   zero_acc();
 
-  int it = it0, rb = rb0, kst = k0, u = 0;
+  // The range is walked unit by unit (the stages of one row block that fall in this range); the
+  // per-stage loop only waits, decodes, releases and moves the ring slot.
+  int it = it0, rb = rb0, kst = k0, u = 0, left = nst;
   int slot = 0;
   uint32_t ph = 0;  // parity of the slot's next `full` phase
   bool ok = true;
   pdl_wait_prior_grids();          // x belongs to the previous kernel until now
-  for (int i = 0; i < nst; ++i) {
+  while (left > 0) {
     const BatchItem& I = its[it];
+    const int C = I.C;
+    const int n = C - kst < left ? C - kst : left;
     const int64_t row0 = static_cast<int64_t>(rb) * kBRows;
-    if (ok) ok = mbar_wait_warp(&full[slot], ph);
-    if (ok) {
-      dec_stage<kInt4, NT, TW>(acc, stg + slot * P.stage, P.xhalf, L, xrow, static_cast<int64_t>(kst) * 2, row0,
-                               I.N, I.sc, I.zp, I.K >> 7);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[slot]);
-    } else {
-      flags[0] = 1;  // a wait ran out (recorded in the device status word): results are void
+    const int64_t Nm = I.N, G = I.K >> 7;
+    const __half* scm = I.sc;
+    const uint8_t* zpm = I.zp;
+    for (int j = 0; j < n; ++j) {
+      if (ok) ok = mbar_wait_warp(&full[slot], ph);
+      if (ok) {
+        dec_stage<kInt4, NT, TW>(acc, stg + slot * P.stage, P.xhalf, L, xrow, static_cast<int64_t>(kst + j) * 2, row0,
+                                 Nm, scm, zpm, G);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[slot]);
+      } else {
+        flags[0] = 1;  // a wait ran out (recorded in the device status word): results are void
+      }
+      if (++slot == P.ring) {
+        slot = 0;
+        ph ^= 1u;
+      }
     }
-    if (++slot == P.ring) {
-      slot = 0;
-      ph ^= 1u;
-    }
+    left -= n;
 
-    if (kst == I.C - 1 || i == nst - 1) {
-      // ---------------------------------------------------------------- finish the row block
-      float v[kDRT][TW][4];
-      dec_values<kInt4, TW>(acc, v);
-      zero_acc();
-      // this CTA's sum over its stages of the block, [token][row] in `res`, once the epilogue
-      // warp has taken the previous block's; for M <= 8 the two K halves (warps 4-7, then 0-3)
-      // are added in a fixed order
-      if (u > 0 && ok) ok = mbar_wait_warp(resempty, static_cast<uint32_t>((u - 1) & 1));
-      if (kSplitK && hi == 0) named_barrier_sync(1, kEp);
+    // ------------------------------------------------------------------ finish the unit
+    float v[kDRT][TW][4];
+    dec_values<kInt4, TW>(acc, v);
+    zero_acc();
+    // this CTA's sum over its stages of the block, [token][row] in `res`, once the epilogue
+    // warp has taken the previous block's; for M <= 8 the two K halves (warps 4-7, then 0-3)
+    // are added in a fixed order
+    if (u > 0 && ok) ok = mbar_wait_warp(resempty, static_cast<uint32_t>((u - 1) & 1));
+    if (kSplitK && hi == 0) named_barrier_sync(1, kEp);
 #pragma unroll
-      for (int rt = 0; rt < kDRT; ++rt)
+    for (int rt = 0; rt < kDRT; ++rt)
 #pragma unroll
-        for (int T = 0; T < TW; ++T)
+      for (int T = 0; T < TW; ++T)
 #pragma unroll
-          for (int ci = 0; ci < 4; ++ci) {
-            float* dst = res + (8 * (Tb + T) + 2 * t + (ci & 1)) * kBResPitch + rw + 16 * rt + 8 * (ci >> 1);
-            if (kSplitK && hi == 0)
-              *dst += v[rt][T][ci];
-            else
-              *dst = v[rt][T][ci];
-          }
-      if (kSplitK && hi == 1) named_barrier_sync(1, kEp);
-      named_barrier_sync(1, kEp);
-      if (!ok) flags[0] = 1;
-      if (threadIdx.x == 0) mbar_arrive(resfull);  // hand the block to the epilogue warp
-      ++u;
-    }
-    if (++kst == I.C) {
+        for (int ci = 0; ci < 4; ++ci) {
+          float* dst = res + (8 * (Tb + T) + 2 * t + (ci & 1)) * kBResPitch + rw + 16 * rt + 8 * (ci >> 1);
+          if (kSplitK && hi == 0)
+            *dst += v[rt][T][ci];
+          else
+            *dst = v[rt][T][ci];
+        }
+    if (kSplitK && hi == 1) named_barrier_sync(1, kEp);
+    named_barrier_sync(1, kEp);
+    if (!ok) flags[0] = 1;
+    if (threadIdx.x == 0) mbar_arrive(resfull);  // hand the block to the epilogue warp
+    ++u;
+    kst += n;
+    if (kst == C) {
       kst = 0;
       if (++rb == I.RB) {
         rb = 0;
