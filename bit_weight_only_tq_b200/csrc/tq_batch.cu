@@ -322,13 +322,13 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
               if (q < P.M) mine[q * kQ + lane] = res4(q);
             __syncwarp();
             if (lane == 0) mbar_arrive(resempty);
-            __threadfence();
-            __syncwarp();
+            // the warp barrier orders every lane's partial before lane 0's release; the count's
+            // acquire orders the other contributors' partials before the warp reads them
             int last = 0;
-            if (lane == 0) last = atomicAdd(&P.counters[cf], 1) == cl - cf;
+            if (lane == 0) last = atom_add_acq_rel_gpu(&P.counters[cf], 1) == cl - cf;
             last = __shfl_sync(0xFFFFFFFFu, last, 0);
             if (last) {
-              __threadfence();
+              __syncwarp();
               sum_and_write(false);
               if (lane == 0) P.counters[cf] = 0;  // ready for the next call
             }

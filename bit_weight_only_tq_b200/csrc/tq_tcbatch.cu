@@ -420,11 +420,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_batch_kernel(const __grid_co
             if (tok < Mt) mine[tok * 128 + e] = __uint_as_float(acc[tok]);
           named_barrier_sync(2, 128);
           if (e == 0) {
-            __threadfence();
-            const int old = atomicAdd(&P.counters[cf], 1);
-            const int last = old == cl - cf;
-            if (last) __threadfence();
-            flags[1] = last;
+            // the barrier orders the 128 threads' partials before this release; the acquire
+            // orders the other contributors' partials before the reads after the next barrier
+            const int old = atom_add_acq_rel_gpu(&P.counters[cf], 1);
+            flags[1] = old == cl - cf;
           }
           named_barrier_sync(2, 128);
           if (flags[1]) {
