@@ -35,7 +35,8 @@ constexpr int kBMaxItems = kBatchMaxItems;
 constexpr int kBRows = 128;       // rows of a row block (one packed TMA tile)
 constexpr int kBResPitch = 132;   // fp32 row pitch of the result buffer [token][row]
 constexpr int kBCtasPerSm = 2;
-constexpr bool kBatchM8FourWarps = false;  // M <= 8: four consumer warps over whole stages
+constexpr bool kBatchM8FourWarps = false;
+constexpr int kBatchPreW = 8;              // stages whose weights are loaded before the PDL wait  // M <= 8: four consumer warps over whole stages
 
 struct BatchItem {
   const __half* sc;    // ternary: scale[N]; W4A16: scales[N, K/128]
@@ -57,6 +58,7 @@ struct BatchParams {
   int G;                      // CTAs
   int ring, stage, xhalf;
   uint32_t four;              // 4 (decode multiplier, see DecLane)
+  int pre_w;                  // stages whose weights are requested before the wait on the previous kernel
   int64_t T;                  // stages in total
   int* counters;              // [G] arrivals per split row block, indexed by its first contributor
   float* slots;               // [2 G][16][128] fp32 partials: slot 2c = CTA c's first row block,
@@ -168,14 +170,19 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
           tma_load_3d(dst + hb * P.xhalf, &P.x[it], &full[slot], 0, kst * F::kKB + 4 * hb, 0);
       };
       const int pre = nst < ring ? nst : ring;
-      for (int i = 0; i < pre; ++i) {  // weights are model constants: before the wait
+      // weights are model constants: the first `pw` stages' weights are requested before the
+      // wait for the previous kernel (their latency overlaps its tail), the rest after it (a
+      // full ring of requests at once would queue the previous kernel's last L2 round trips)
+      const int pw = pre < P.pre_w ? pre : P.pre_w;
+      for (int i = 0; i < pre; ++i) {
         mbar_arrive_expect_tx(&full[i], tx);
-        load_w(i);
+        if (i < pw) load_w(i);
         advance();
       }
       pdl_wait_prior_grids();  // the activations may come from the previous kernel
       it = it0, rb = rb0, kst = k0, C = its[it0].C;
       for (int i = 0; i < pre; ++i) {
+        if (i >= pw) load_w(i);
         load_x(i);
         advance();
       }
@@ -522,6 +529,7 @@ static cudaError_t launch_batch_t(const BatchLinear* items, int count, int64_t M
   if (T * P.G >= (static_cast<int64_t>(1) << 32)) return cudaErrorInvalidValue;  // 32-bit range arithmetic
   P.xhalf = ((static_cast<int>(M) * 4 * 128 + 1023) / 1024) * 1024;
   P.four = 4u;
+  P.pre_w = kBatchPreW;
   P.stage = kDWBytes + (F::kKB / 4) * P.xhalf;
   int ring = kDMaxRing;
   while (ring > 2 && L::bytes(ring, P.stage) > kDSmemBudget) --ring;
