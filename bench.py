@@ -654,25 +654,35 @@ def dispatch_crossover(tq, I, pq, qshapes):
     return out
 
 
-def load_traffic():
-    """DRAM bytes per decode launch from the committed ncu summary, only if it was taken on this
-    kernel source (the summary records the SHA-256 of the decode source file)."""
+TRAFFIC_SOURCES = ("tq_batch.cu", "tq_decode.cu", "tq_ptx.cuh", "tq_common.cuh")
+
+
+def kernel_source_sha():
+    """SHA-256 over the sources of the batch decode kernel (the headline's dominant kernel)."""
     import hashlib
 
+    h = hashlib.sha256()
+    for f in TRAFFIC_SOURCES:
+        with open(os.path.join(ROOT, "bit_weight_only_tq_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def load_traffic():
+    """DRAM bytes per batch-decode launch from the committed ncu summary, only if it was taken on
+    this kernel source (the summary records the SHA-256 of the kernel's source files)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
-    src = os.path.join(ROOT, "bit_weight_only_tq_b200", "csrc", "tq_decode.cu")
-    if not os.path.exists(p) or not os.path.exists(src):
+    if not os.path.exists(p):
         return None
     try:
         with open(p) as f:
             d = json.load(f)
-        with open(src, "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()
+        sha = kernel_source_sha()
     except (OSError, ValueError):
         return None
     if d.get("kernel_source_sha256") != sha:
         return None
-    return d.get("decode_gemm_bytes_per_launch")
+    return d.get("batch_decode_bytes_per_launch")
 
 
 # ------------------------------------------------------------------------------------------------
