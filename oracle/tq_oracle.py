@@ -49,6 +49,8 @@ __all__ = [
     "tq_quantize_pack",
     "tq_unpack",
     "tq_gemm",
+    "tq_interleave",
+    "tq_deinterleave",
     "w4g_quantize_pack",
     "w4g_unpack",
     "w4g_gemm",
@@ -190,6 +192,39 @@ def unpack_codes(packed, K: int) -> np.ndarray:
     codes = (p[..., :, None] >> shifts) & 3
     codes = codes.reshape(p.shape[:-1] + (p.shape[-1] * 4,))
     return codes[..., :K].astype(np.uint8)
+
+
+# The pair-interleaved layout: a post-load relayout of the packed codes (the repack step that
+# [VQ] §4.3 describes for GPTQ/AWQ checkpoints, applied here to the ternary format).  It is a
+# layout of this library, not of the pages: the same bytes per row, the codes of every group of
+# 16 moved so that the two fp16 halves of a 32-bit word read at one bit position hold the codes
+# of two consecutive k.
+IL_SOURCE = np.array([0, 2, 4, 6, 8, 10, 12, 14, 1, 3, 5, 7, 9, 11, 13, 15], np.int64)
+
+
+def tq_interleave(packed) -> np.ndarray:
+    """Canonical packed rows [N, KB] (KB % 4 == 0: whole 32-bit words of 16 codes) to the
+    pair-interleaved layout.  Code slot s of a little-endian word (bits 2s..2s+1) holds, in the
+    canonical layout, code k = 16q + s; in the interleaved layout slot j (j < 8) holds
+    k = 16q + 2j and slot 8 + j holds k = 16q + 2j + 1."""
+    p = np.asarray(packed, np.uint8)
+    N, KB = p.shape
+    if KB % 4:
+        raise ValueError("the interleaved layout needs whole 32-bit words (K a multiple of 16)")
+    codes = unpack_codes(p, KB * 4).reshape(N, KB // 4, 16)
+    return pack_codes(codes[:, :, IL_SOURCE].reshape(N, KB * 4))
+
+
+def tq_deinterleave(packed_il) -> np.ndarray:
+    """Inverse of tq_interleave."""
+    p = np.asarray(packed_il, np.uint8)
+    N, KB = p.shape
+    if KB % 4:
+        raise ValueError("the interleaved layout needs whole 32-bit words (K a multiple of 16)")
+    il = unpack_codes(p, KB * 4).reshape(N, KB // 4, 16)
+    codes = np.empty_like(il)
+    codes[:, :, IL_SOURCE] = il
+    return pack_codes(codes.reshape(N, KB * 4))
 
 
 def tq_quantize_pack(W):
