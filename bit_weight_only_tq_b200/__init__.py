@@ -75,6 +75,7 @@ _SIGS = {
     "tq_batch_workspace_size": [],
     "tq_gemm_batch_ex": [_vp, _int, _i64, _vp, ctypes.c_size_t, _int, _vp],
     "tq_gemm_batch_noalloc": [_vp, _int, _i64, _vp],
+    "tq_interleave_packed": [_vp, _vp, _i64, _i64, _vp],
     "w4g_gemm_batch_ex": [_vp, _int, _i64, _vp, ctypes.c_size_t, _int, _vp],
     "tq_debug_set_wait_limit": [ctypes.c_longlong],
     "tq_debug_skip_activation_loads": [_int],
@@ -334,7 +335,20 @@ def batch_workspace(device=None) -> torch.Tensor:
     return torch.zeros(n, dtype=torch.uint8, device=dev)
 
 
-BATCH_AUTO, BATCH_MMA_SYNC, BATCH_TENSOR_CORE = 0, 1, 2
+BATCH_AUTO, BATCH_MMA_SYNC, BATCH_TENSOR_CORE, BATCH_INTERLEAVED = 0, 1, 2, 16
+
+
+def tq_interleave_packed(packed: torch.Tensor, out: torch.Tensor = None, stream=None) -> torch.Tensor:
+    """Relayout packed ternary rows [N, K/4] (K % 16 == 0) into the pair-interleaved layout that
+    tq_gemm_batch(..., interleaved=True) reads; `out` may be `packed` itself."""
+    _need(packed, torch.uint8, "packed", 2)
+    out = torch.empty_like(packed) if out is None else out
+    _need(out, torch.uint8, "out", 2)
+    if tuple(out.shape) != tuple(packed.shape):
+        raise ValueError("out shape mismatch")
+    N, K = packed.shape[0], packed.shape[1] * 4
+    _check(lib.tq_interleave_packed(_ptr(packed), _ptr(out), N, K, _stream(stream)), "tq_interleave_packed")
+    return out
 
 
 def _batch(fn, xs, weights, scales, biases, ys, workspace, wdtype, sdim, what, stream, zeros=None, variant=0):
@@ -370,10 +384,12 @@ def _batch(fn, xs, weights, scales, biases, ys, workspace, wdtype, sdim, what, s
 
 
 def tq_gemm_batch(xs, packed_list, scale_list, bias_list=None, y_list=None, workspace=None, stream=None,
-                  variant=BATCH_AUTO):
-    """Independent ternary linears sharing M (each with its own x) in one persistent launch."""
+                  variant=BATCH_AUTO, interleaved=False):
+    """Independent ternary linears sharing M (each with its own x) in one persistent launch.
+    interleaved=True: the packed weights come from tq_interleave_packed."""
+    v = int(variant) | (BATCH_INTERLEAVED if interleaved else 0)
     return _batch(lib.tq_gemm_batch_ex, xs, packed_list, scale_list, bias_list, y_list, workspace, torch.uint8, 1,
-                  "tq_gemm_batch", stream, variant=variant)
+                  "tq_gemm_batch", stream, variant=v)
 
 
 def w4g_gemm_batch(xs, qweight_list, scales_list, bias_list=None, y_list=None, workspace=None, stream=None,

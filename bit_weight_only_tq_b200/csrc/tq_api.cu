@@ -397,10 +397,13 @@ template <bool kInt4>
 int gemm_batch_impl(const tq_linear* items, int count, int64_t M, void* workspace, size_t workspace_bytes,
                     int variant, void* stream) {
   if (count < 1 || count > tq::kBatchMaxItems) return TQ_ERR_SHAPE;
+  const bool il = (variant & TQ_BATCH_INTERLEAVED) != 0;  // ternary weights in the interleaved layout
+  variant &= ~TQ_BATCH_INTERLEAVED;
   if (variant < TQ_BATCH_AUTO || variant > TQ_BATCH_TENSOR_CORE) return TQ_ERR_PATH;
   if (M < 0 || M > tq::kBatchMaxM) return TQ_ERR_SHAPE;
   if (variant == TQ_BATCH_AUTO) variant = M <= 16 ? TQ_BATCH_MMA_SYNC : TQ_BATCH_TENSOR_CORE;
   if (variant == TQ_BATCH_MMA_SYNC && M > 16) return TQ_ERR_PATH;
+  if (il && (kInt4 || variant != TQ_BATCH_MMA_SYNC)) return TQ_ERR_PATH;
   if (!items) return TQ_ERR_NULL;
   tq::BatchLinear lin[tq::kBatchMaxItems];
   int n = 0;
@@ -425,7 +428,7 @@ int gemm_batch_impl(const tq_linear* items, int count, int64_t M, void* workspac
     e = tq::launch_gemm_batch_tc(kInt4, lin, n, M, workspace, wb, as_stream(stream));
   else
     e = kInt4 ? tq::launch_w4g_gemm_batch(lin, n, M, workspace, wb, as_stream(stream))
-              : tq::launch_tq_gemm_batch(lin, n, M, workspace, wb, as_stream(stream));
+              : tq::launch_tq_gemm_batch(lin, n, M, workspace, wb, as_stream(stream), il);
   return to_status(e);
 }
 
@@ -451,6 +454,17 @@ int tq_gemm_batch_ex(const tq_linear* items, int count, int64_t M, void* workspa
 int w4g_gemm_batch_ex(const tq_linear* items, int count, int64_t M, void* workspace, size_t workspace_bytes,
                       int variant, void* stream) {
   return gemm_batch_impl<true>(items, count, M, workspace, workspace_bytes, variant, stream);
+}
+
+int tq_interleave_packed(const uint8_t* packed, uint8_t* out, int64_t N, int64_t K, void* stream) {
+  if (N < 0 || K <= 0 || K % 16 != 0 || N > (int64_t(1) << 31) || K > (int64_t(1) << 28)) return TQ_ERR_SHAPE;
+  if (N == 0) return TQ_OK;
+  if (!packed || !out) return TQ_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(packed) | reinterpret_cast<uintptr_t>(out)) & 3u) return TQ_ERR_ALIGN;
+  cudaError_t e = tq::launch_tq_interleave(reinterpret_cast<const uint32_t*>(packed), reinterpret_cast<uint32_t*>(out),
+                                           N * (K / 16), as_stream(stream));
+  if (e == cudaSuccess) e = tq::after_constants_written(as_stream(stream));
+  return to_status(e);
 }
 
 int tq_shard_plan(int fmt, int mode, int64_t N, int64_t K, int world, int rank, tq_shard* out) {

@@ -91,7 +91,7 @@ __device__ __forceinline__ int range_owner(int64_t s, int64_t T, int G) {
 // NT token groups of eight, TW of them per consumer warp, CW consumer warps.  With eight
 // consumer warps and one token group the two K halves of a stage go to two warp sets (kSplitK);
 // otherwise every consumer warp takes its rows over the whole stage.
-template <bool kInt4, int NT, int TW, int CW>
+template <bool kInt4, int NT, int TW, int CW, bool kIL = false>
 __device__ __forceinline__ void batch_body(const BatchParams& P) {
   using F = DecFmt<kInt4>;
   constexpr int kCons = CW;
@@ -398,7 +398,7 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
     for (int j = 0; j < n; ++j) {
       if (ok) ok = mbar_wait_warp(&full[slot], ph);
       if (ok) {
-        dec_stage<kInt4, NT, TW>(acc, stg + slot * P.stage, P.xhalf, L, xrow, static_cast<int64_t>(kst + j) * 2, row0,
+        dec_stage<kInt4, NT, TW, kIL>(acc, stg + slot * P.stage, P.xhalf, L, xrow, static_cast<int64_t>(kst + j) * 2, row0,
                                  Nm, scm, zpm, G);
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[slot]);
@@ -455,20 +455,20 @@ constexpr int batch_threads() { return (CW + 2) * 32; }
 
 // M <= 8, eight consumer warps (K halves split): two CTAs of ten warps per SM; five warps share
 // one SM sub-partition's 16K registers, so a thread may use at most 102 (96 it is).
-template <bool kInt4>
+template <bool kInt4, bool kIL>
 __global__ void __maxnreg__(96) batch_decode_kernel_m8(const __grid_constant__ BatchParams P) {
-  batch_body<kInt4, 1, 1, 8>(P);
+  batch_body<kInt4, 1, 1, 8, kIL>(P);
 }
 
 // M <= 8, four consumer warps, each over the whole stage (twice the MMAs per stage and warp).
-template <bool kInt4>
+template <bool kInt4, bool kIL>
 __global__ void __launch_bounds__(batch_threads<4>(), 2) batch_decode_kernel_m8w4(const __grid_constant__ BatchParams P) {
-  batch_body<kInt4, 1, 1, 4>(P);
+  batch_body<kInt4, 1, 1, 4, kIL>(P);
 }
 
-template <bool kInt4>
+template <bool kInt4, bool kIL>
 __global__ void __launch_bounds__(batch_threads<4>(), 2) batch_decode_kernel_m16(const __grid_constant__ BatchParams P) {
-  batch_body<kInt4, 2, 2, 4>(P);
+  batch_body<kInt4, 2, 2, 4, kIL>(P);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -481,7 +481,7 @@ int64_t batch_workspace_bytes() {
   return a > b ? a : b;
 }
 
-template <bool kInt4>
+template <bool kInt4, bool kIL>
 static cudaError_t launch_batch_t(const BatchLinear* items, int count, int64_t M, void* ws, int64_t ws_bytes,
                                   cudaStream_t s) {
   using F = DecFmt<kInt4>;
@@ -541,7 +541,8 @@ static cudaError_t launch_batch_t(const BatchLinear* items, int count, int64_t M
 
   const bool m16 = M > 8;
   const bool w4 = !m16 && kBatchM8FourWarps;
-  auto* kern = m16 ? batch_decode_kernel_m16<kInt4> : w4 ? batch_decode_kernel_m8w4<kInt4> : batch_decode_kernel_m8<kInt4>;
+  auto* kern = m16 ? batch_decode_kernel_m16<kInt4, kIL>
+                   : w4 ? batch_decode_kernel_m8w4<kInt4, kIL> : batch_decode_kernel_m8<kInt4, kIL>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), kDSmemBudget);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -558,13 +559,14 @@ static cudaError_t launch_batch_t(const BatchLinear* items, int count, int64_t M
 }
 
 cudaError_t launch_tq_gemm_batch(const BatchLinear* items, int count, int64_t M, void* ws, int64_t ws_bytes,
-                                 cudaStream_t s) {
-  return launch_batch_t<false>(items, count, M, ws, ws_bytes, s);
+                                 cudaStream_t s, bool interleaved) {
+  return interleaved ? launch_batch_t<false, true>(items, count, M, ws, ws_bytes, s)
+                     : launch_batch_t<false, false>(items, count, M, ws, ws_bytes, s);
 }
 
 cudaError_t launch_w4g_gemm_batch(const BatchLinear* items, int count, int64_t M, void* ws, int64_t ws_bytes,
                                   cudaStream_t s) {
-  return launch_batch_t<true>(items, count, M, ws, ws_bytes, s);
+  return launch_batch_t<true, false>(items, count, M, ws, ws_bytes, s);
 }
 
 }  // namespace tq

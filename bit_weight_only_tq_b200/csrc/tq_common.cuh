@@ -242,7 +242,9 @@ constexpr int64_t kBatchMaxM = 32;        // the tensor-core variant; the mma.sy
 // Workspace bytes the batch kernel needs on the current device.
 int64_t batch_workspace_bytes();
 cudaError_t launch_tq_gemm_batch(const BatchLinear* items, int count, int64_t M, void* ws, int64_t ws_bytes,
-                                 cudaStream_t s);
+                                 cudaStream_t s, bool interleaved = false);
+// The pair-interleaved relayout of packed ternary rows (words of 16 codes, flat).
+cudaError_t launch_tq_interleave(const uint32_t* in, uint32_t* out, int64_t words, cudaStream_t s);
 cudaError_t launch_w4g_gemm_batch(const BatchLinear* items, int count, int64_t M, void* ws, int64_t ws_bytes,
                                   cudaStream_t s);
 // The tensor-core variant of the batch kernel (tq_tcbatch.cu), 1 <= M <= 32.

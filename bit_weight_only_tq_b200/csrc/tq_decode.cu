@@ -161,7 +161,10 @@ struct DecLane {
 // i.e. exactly 2 (c - 1): one shift and one LOP3 per two weights, no arithmetic.  (Code 0b11 is
 // invalid and decodes to +0.)
 
-template <bool kInt4, int NT, int TW>
+// kIL: the ternary weights are in the pair-interleaved layout (slot j of a word holds k = 2j,
+// slot 8 + j holds k = 2j + 1), so the activation pair of code position p is the p-th 32-bit
+// word of x as it lies in shared memory: no byte permutes.
+template <bool kInt4, int NT, int TW, bool kIL = false>
 __device__ __forceinline__ void dec_stage(float (&acc)[kDRT][TW][4], const uint8_t* st, int xhalf,
                                           const DecLane& L, const int (&xrow)[TW], int64_t gi_base,
                                           int64_t row0, int64_t Nm, const __half* scm, const uint8_t* zpm,
@@ -221,8 +224,13 @@ __device__ __forceinline__ void dec_stage(float (&acc)[kDRT][TW][4], const uint8
           uint32_t b0[TW], b1[TW];
 #pragma unroll
           for (int T = 0; T < TW; ++T) {
-            b0[T] = __byte_perm(P[T][p >> 1], P[T][(p >> 1) + 4], sel);
-            b1[T] = __byte_perm(P[T][8 + (p >> 1)], P[T][12 + (p >> 1)], sel);
+            if (kIL) {  // k = 2p, 2p + 1 of words 2h and 2h + 1
+              b0[T] = P[T][p];
+              b1[T] = P[T][8 + p];
+            } else {
+              b0[T] = __byte_perm(P[T][p >> 1], P[T][(p >> 1) + 4], sel);
+              b1[T] = __byte_perm(P[T][8 + (p >> 1)], P[T][12 + (p >> 1)], sel);
+            }
           }
 #pragma unroll
           for (int rt = 0; rt < kDRT; ++rt) {

@@ -310,6 +310,39 @@ __global__ void __launch_bounds__(kPackThreads)
 }
 
 // ---------------------------------------------------------------------------------------------
+// Pair-interleaved relayout (the post-load repack of [VQ] §4.3, applied to the ternary rows).
+// A 32-bit little-endian word holds 16 codes, code slot s at bits 2s..2s+1 (canonical: k = s).
+// The interleaved word holds the even slots (k = 0, 2, .., 14) in order in its low 16 bits and
+// the odd slots (k = 1, 3, .., 15) in its high 16 bits, so a decode that reads bit position 2p
+// of both halves gets k = 2p and 2p + 1.  Each 2-bit field is gathered by a three-step compaction.
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t compact_even_fields(uint32_t v) {  // fields at bits 4i..4i+1 -> 2i..2i+1
+  v &= 0x33333333u;
+  v = (v | (v >> 2)) & 0x0F0F0F0Fu;
+  v = (v | (v >> 4)) & 0x00FF00FFu;
+  v = (v | (v >> 8)) & 0x0000FFFFu;
+  return v;
+}
+
+__global__ void __launch_bounds__(256) tq_interleave_kernel(const uint32_t* in, uint32_t* out,  // may be the same buffer
+                                                          int64_t words) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < words; i += stride) {
+    const uint32_t w = in[i];
+    out[i] = compact_even_fields(w) | (compact_even_fields(w >> 2) << 16);
+  }
+}
+
+cudaError_t launch_tq_interleave(const uint32_t* in, uint32_t* out, int64_t words, cudaStream_t s) {
+  if (words <= 0) return cudaSuccess;
+  const int sms = current_device_info().num_sms;
+  int64_t blocks = (words + 255) / 256;
+  if (blocks > 8 * static_cast<int64_t>(sms)) blocks = 8 * static_cast<int64_t>(sms);
+  tq_interleave_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(in, out, words);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------------------------
 // W4A16 pack: one warp per (row n, group g of 128).  Lane l holds k = 128g + 4l .. 4l+3.
 // ---------------------------------------------------------------------------------------------
 // The group quantiser shared by both W4 pack kernels: this lane's four weights wf of one

@@ -281,12 +281,37 @@ TQ_API int w4g_gemm_batch(const tq_linear* items, int count, int64_t M, void* wo
  *   TQ_BATCH_TENSOR_CORE  M <= 32: one CTA per SM, decoded weights stored to tensor memory as
  *                         the A operand of tcgen05.mma (N = 16 or 32 tokens), accumulators in
  *                         tensor memory.
- * Errors as above, plus TQ_ERR_PATH for an unknown variant or M > 16 with TQ_BATCH_MMA_SYNC. */
-typedef enum { TQ_BATCH_AUTO = 0, TQ_BATCH_MMA_SYNC = 1, TQ_BATCH_TENSOR_CORE = 2 } tq_batch_variant;
+ * TQ_BATCH_INTERLEAVED may be OR-ed into the variant of tq_gemm_batch_ex: every item's ternary
+ * weights are then in the pair-interleaved layout of tq_interleave_packed (same scales, same
+ * results up to the fp32 summation order); the mma.sync kernel only (M <= 16).
+ * Errors as above, plus TQ_ERR_PATH for an unknown variant, M > 16 with TQ_BATCH_MMA_SYNC, or
+ * TQ_BATCH_INTERLEAVED with W4A16 items or the tensor-core kernel. */
+typedef enum { TQ_BATCH_AUTO = 0, TQ_BATCH_MMA_SYNC = 1, TQ_BATCH_TENSOR_CORE = 2,
+               TQ_BATCH_INTERLEAVED = 16 } tq_batch_variant;
 TQ_API int tq_gemm_batch_ex(const tq_linear* items, int count, int64_t M, void* workspace,
                             size_t workspace_bytes, int variant, void* stream);
 TQ_API int w4g_gemm_batch_ex(const tq_linear* items, int count, int64_t M, void* workspace,
                              size_t workspace_bytes, int variant, void* stream);
+
+/* --------------------------------------------------------------------------------------------
+ * tq_interleave_packed -- relayout of packed ternary rows for the decode kernels ([VQ] §4.3: the
+ * post-load repack a checkpoint's weights go through once before inference; the layout itself
+ * is this library's, the pages have no counterpart).
+ *
+ *   packed  device, [N][K/4] bytes in the canonical layout of tq_quantize_pack.
+ *   out     device, [N][K/4] bytes; may be `packed` itself (in place).
+ *   K       multiple of 16 (rows of whole 32-bit words of 16 codes).
+ * Per little-endian 32-bit word of a row (codes k = 16q .. 16q + 15, code s at bits 2s..2s+1 in
+ * the canonical layout) the interleaved word holds k = 16q + 2j at bits 2j..2j+1 and
+ * k = 16q + 2j + 1 at bits 16 + 2j.. (j = 0..7): the two fp16 halves a decode reads at one bit
+ * position then hold two consecutive k, matching the activations' natural fp16 pairs.  The
+ * scales are unchanged.  Pass the result to tq_gemm_batch_ex with TQ_BATCH_INTERLEAVED.
+ * Like the pack calls it ends with an empty kernel in plain stream order (safe before a GEMM
+ * that reads the weights before waiting for the previous kernel).
+ * Errors: TQ_ERR_SHAPE (K not a multiple of 16, N < 0), TQ_ERR_NULL, TQ_ERR_ALIGN (pointers not
+ * 4-byte aligned), TQ_ERR_CUDA.
+ * ------------------------------------------------------------------------------------------ */
+TQ_API int tq_interleave_packed(const uint8_t* packed, uint8_t* out, int64_t N, int64_t K, void* stream);
 
 /* --------------------------------------------------------------------------------------------
  * tq_gemm_batch_noalloc -- tq_gemm_batch without a workspace argument and without allocating.

@@ -12,7 +12,7 @@ import bit_weight_only_tq_b200 as tq
 
 def test_library_exports_every_header_function():
     names = tq.header_functions()
-    assert len(names) == 27
+    assert len(names) == 28
     for n in names:
         assert hasattr(tq.lib, n), n
     for n in ("tq_quantize_pack", "tq_gemm", "w4g_quantize_pack", "w4g_gemm", "tq_validate_packed",
@@ -135,6 +135,11 @@ def test_batch_argument_errors_without_gpu():
     assert tq.lib.tq_gemm_batch(_items((q, a, a, a, 64, 128)), 1, 1, ws, big, None) == -3   # misaligned x
     assert tq.lib.tq_gemm_batch(_items((a, q, a, a, 64, 128)), 1, 1, ws, big, None) == -3   # misaligned w
     assert tq.lib.tq_gemm_batch(ok, 1, 1, None, big, None) == -1                # no workspace
+    # the interleaved-layout flag: ternary items on the mma.sync kernel only
+    assert tq.lib.tq_gemm_batch_ex(ok, 1, 4, ws, big, tq.BATCH_TENSOR_CORE | tq.BATCH_INTERLEAVED, None) == -8
+    assert tq.lib.tq_gemm_batch_ex(ok, 1, 17, ws, big, tq.BATCH_AUTO | tq.BATCH_INTERLEAVED, None) == -8
+    assert tq.lib.w4g_gemm_batch_ex(ok, 1, 4, ws, big, tq.BATCH_MMA_SYNC | tq.BATCH_INTERLEAVED, None) == -8
+    assert tq.lib.tq_gemm_batch_ex(ok, 1, 4, ws, big, 3 | tq.BATCH_INTERLEAVED, None) == -8
     # the allocation-free variant checks the same arguments before any device work
     assert tq.lib.tq_gemm_batch_noalloc(ok, 0, 1, None) == -2
     assert tq.lib.tq_gemm_batch_noalloc(ok, 9, 1, None) == -2
@@ -177,3 +182,13 @@ def test_import_fails_loudly_without_the_library(tmp_path):
                        capture_output=True, text=True, timeout=300)
     assert r.returncode != 0
     assert not (tmp_path / "bit_weight_only_tq_b200" / "libtq.so").exists()
+
+
+def test_interleave_argument_errors_without_gpu():
+    a = ctypes.c_void_p(1 << 20)
+    q = ctypes.c_void_p((1 << 20) + 2)
+    assert tq.lib.tq_interleave_packed(a, a, 8, 24, None) == -2      # K % 16
+    assert tq.lib.tq_interleave_packed(a, a, -1, 64, None) == -2
+    assert tq.lib.tq_interleave_packed(a, a, 0, 64, None) == 0       # empty
+    assert tq.lib.tq_interleave_packed(None, a, 8, 64, None) == -1
+    assert tq.lib.tq_interleave_packed(q, a, 8, 64, None) == -3      # misaligned
