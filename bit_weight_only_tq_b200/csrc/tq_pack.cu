@@ -247,6 +247,45 @@ struct UnitsAcc {  // exact running sum of fp16 magnitudes
   }
 };
 
+// Fast exact sum of fp16 magnitudes in fp32 (FMA pipe) while the values stay small: each v is
+// split into h = v rounded to a multiple of 2^-12 ((v + 2048) - 2048, exact for v < 2^11) and
+// l = v - h (exact, |l| <= 2^-13, a multiple of 2^-24).  The h sums are exact while below 2^12
+// (multiples of 2^-12) and, h being >= 0, they only grow: a final sum below 2^11 proves every
+// partial sum and every v were in range.  The l sums stay exact while fewer than 2^13 values
+// are added (|partial| < 1, multiples of 2^-24).  Otherwise the caller recomputes the sum in fp64.
+struct FastAcc {
+  float hi = 0.0f, lo = 0.0f;
+  __device__ __forceinline__ void add(float v) {
+    const float h = __fadd_rn(__fadd_rn(v, 2048.0f), -2048.0f);
+    hi = __fadd_rn(hi, h);
+    lo = __fadd_rn(lo, __fadd_rn(v, -h));
+  }
+  __device__ __forceinline__ void add_pair(uint32_t mags) {  // two fp16 magnitude patterns
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&mags));
+    add(f.x);
+    add(f.y);
+  }
+  __device__ __forceinline__ bool valid() const { return hi < 2048.0f; }
+  // This lane's sum in units of 2^-24 (both parts are exact integers in those units).
+  __device__ __forceinline__ long long units() const {
+    return __double2ll_rn(static_cast<double>(hi) * 16777216.0) + __double2ll_rn(static_cast<double>(lo) * 16777216.0);
+  }
+};
+
+// Warp total of per-lane unit sums, correctly rounded once to fp64 (all lanes get it).
+__device__ __forceinline__ double warp_units_total(long long u) {
+  long long h = u >> 32, l = u & 0xFFFFFFFFll;  // two parts, so no row length overflows
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    h += __shfl_xor_sync(0xFFFFFFFFu, h, o);
+    l += __shfl_xor_sync(0xFFFFFFFFu, l, o);
+  }
+  return __ll2double_rn(h) * 256.0 + __ll2double_rn(l) * 0x1p-24;
+}
+
+// kFast: the row sums use FastAcc (fp32, FMA pipe) with an fp64 recomputation of a row whose
+// values leave its range; rows need fewer than 2^13 elements per lane (K < 2^18).
+template <bool kFast>
 __global__ void __launch_bounds__(kPackThreads)
     tq_pack_f16_kernel(const uint16_t* __restrict__ w, uint8_t* __restrict__ packed,
                        uint16_t* __restrict__ scale, int64_t N, int64_t K) {
@@ -256,25 +295,44 @@ __global__ void __launch_bounds__(kPackThreads)
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
   for (int64_t n = static_cast<int64_t>(blockIdx.x) * kWarps + wid; n < N; n += nwarps) {
     const uint4* row = reinterpret_cast<const uint4*>(w + n * K);
-    UnitsAcc accS;
-    int cnt = 0;
+    // exact sum of |w| over the row, fp64 (the fallback, and the path without kFast)
+    auto slow_sum = [&]() {
+      UnitsAcc acc;
+      int cnt = 0;
 #pragma unroll 2
-    for (int64_t j = lane; j < C; j += 32) {
-      const uint4 v = __ldg(row + j);
-      accS.part += ((f16_mag_f64(v.x) + f16_mag_f64(v.x >> 16)) + (f16_mag_f64(v.y) + f16_mag_f64(v.y >> 16))) +
-                   ((f16_mag_f64(v.z) + f16_mag_f64(v.z >> 16)) + (f16_mag_f64(v.w) + f16_mag_f64(v.w >> 16)));
-      if (++cnt == 1024) {  // 8192 elements < 2^13: the partial stays below 2^29
-        accS.flush();
-        cnt = 0;
+      for (int64_t j = lane; j < C; j += 32) {
+        const uint4 v = __ldg(row + j);
+        acc.part += ((f16_mag_f64(v.x) + f16_mag_f64(v.x >> 16)) + (f16_mag_f64(v.y) + f16_mag_f64(v.y >> 16))) +
+                    ((f16_mag_f64(v.z) + f16_mag_f64(v.z >> 16)) + (f16_mag_f64(v.w) + f16_mag_f64(v.w >> 16)));
+        if (++cnt == 1024) {  // 8192 elements < 2^13: the partial stays below 2^29
+          acc.flush();
+          cnt = 0;
+        }
       }
+      return acc.warp_total();
+    };
+    double S;
+    if (kFast) {
+      FastAcc fa;
+#pragma unroll 2
+      for (int64_t j = lane; j < C; j += 32) {
+        const uint4 v = __ldg(row + j);
+        fa.add_pair(v.x & 0x7FFF7FFFu);
+        fa.add_pair(v.y & 0x7FFF7FFFu);
+        fa.add_pair(v.z & 0x7FFF7FFFu);
+        fa.add_pair(v.w & 0x7FFF7FFFu);
+      }
+      S = __all_sync(0xFFFFFFFFu, fa.valid()) ? warp_units_total(fa.units()) : slow_sum();
+    } else {
+      S = slow_sum();
     }
-    const double S = accS.warp_total();
     const double t = 0.7 * (S / static_cast<double>(K));
     const uint32_t tb = magnitude_floor_bits<true>(t);
     const uint32_t tb2 = (tb | (tb << 16)) | 0x80008000u;
     UnitsAcc accA;
+    FastAcc faA;
     int nz = 0;
-    cnt = 0;
+    int cnt = 0;
     uint16_t* prow = reinterpret_cast<uint16_t*>(packed + n * (K >> 2));
 #pragma unroll 2
     for (int64_t j = lane; j < C; j += 32) {
@@ -292,17 +350,50 @@ __global__ void __launch_bounds__(kPackThreads)
         const uint32_t c = zero | pos;                            // else 00
         out |= ((c | (c >> 14)) & 0xFu) << (4 * i);
         nz += __popc(~D & 0x80008000u);
-        if (!(D & 0x8000u)) a += f16_mag_f64(wd[i]);
-        if (!(D & 0x80000000u)) a += f16_mag_f64(wd[i] >> 16);
+        if (kFast) {
+          // the magnitudes of the nonzero codes (a zero code's half is cleared)
+          const uint32_t keep = ((~D & 0x80008000u) >> 15) * 0xFFFFu;
+          faA.add_pair(wd[i] & 0x7FFF7FFFu & keep);
+        } else {
+          if (!(D & 0x8000u)) a += f16_mag_f64(wd[i]);
+          if (!(D & 0x80000000u)) a += f16_mag_f64(wd[i] >> 16);
+        }
       }
-      accA.part += a;
-      if (++cnt == 1024) {
-        accA.flush();
-        cnt = 0;
+      if (!kFast) {
+        accA.part += a;
+        if (++cnt == 1024) {
+          accA.flush();
+          cnt = 0;
+        }
       }
       prow[j] = static_cast<uint16_t>(out);
     }
-    const double A = accA.warp_total();
+    double A;
+    if (kFast && __all_sync(0xFFFFFFFFu, faA.valid())) {
+      A = warp_units_total(faA.units());
+    } else if (kFast) {  // recompute the sum of the nonzero magnitudes in fp64
+      UnitsAcc acc;
+      cnt = 0;
+      for (int64_t j = lane; j < C; j += 32) {
+        const uint4 v = __ldg(row + j);
+        const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+        double a2 = 0.0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t D = tb2 - (wd[i] & 0x7FFF7FFFu);
+          if (!(D & 0x8000u)) a2 += f16_mag_f64(wd[i]);
+          if (!(D & 0x80000000u)) a2 += f16_mag_f64(wd[i] >> 16);
+        }
+        acc.part += a2;
+        if (++cnt == 1024) {
+          acc.flush();
+          cnt = 0;
+        }
+      }
+      A = acc.warp_total();
+    } else {
+      A = accA.warp_total();
+    }
     const int nzt = warp_sum(nz);
     if (lane == 0)
       scale[n] = nzt > 0 ? f64_to_f16_rne(A / static_cast<double>(nzt)) : static_cast<uint16_t>(0);
@@ -481,8 +572,13 @@ cudaError_t launch_tq_pack(const void* w, bool w_f16, uint8_t* packed, uint16_t*
   const int binw = 30 - ceil_log2_i64(K);
   const uintptr_t a = reinterpret_cast<uintptr_t>(w);
   if (w_f16 && K % 8 == 0 && a % 16 == 0) {
-    tq_pack_f16_kernel<<<static_cast<unsigned>(grid), kPackThreads, 0, s>>>(
-        static_cast<const uint16_t*>(w), packed, scale, N, K);
+    // the fp32 row sums need fewer than 2^13 elements per lane
+    if (K < (int64_t(1) << 18))
+      tq_pack_f16_kernel<true><<<static_cast<unsigned>(grid), kPackThreads, 0, s>>>(
+          static_cast<const uint16_t*>(w), packed, scale, N, K);
+    else
+      tq_pack_f16_kernel<false><<<static_cast<unsigned>(grid), kPackThreads, 0, s>>>(
+          static_cast<const uint16_t*>(w), packed, scale, N, K);
     return cudaGetLastError();
   }
   const int vec = (K % 4 == 0) && (a % (w_f16 ? 8 : 16) == 0);

@@ -144,3 +144,32 @@ def test_pack_fp32_deep_bins_long_row():
     e = torch.randint(-120, 60, (3, K), generator=g).float()
     w = torch.randn(3, K, generator=g) * torch.exp2(e)
     _check_tq(w)
+
+
+def test_pack_fp16_fast_sum_boundaries():
+    # fp16 rows (16-byte aligned, K % 8 == 0) whose per-lane sums sit at the edges of the fast
+    # fp32 accumulation (values up to 2^11, lane sums around 2^11, many subnormals), and rows
+    # that must fall back to the fp64 sums; the result must match the oracle bit for bit
+    K = 2048
+    g = torch.Generator().manual_seed(21)
+    rows = []
+    r = torch.full((K,), 2047.0)                       # every value just below 2^11: lane sums overflow
+    rows.append(r)
+    r = torch.zeros(K)
+    r[::32] = 2047.0                                   # one such value per lane... and 63 more per lane
+    rows.append(r)
+    r = torch.zeros(K)
+    r[::64] = 2040.0                                   # lane sums just below 2^11 (one value each)
+    rows.append(r)
+    r = torch.randn(K, generator=g) * 6e-8             # fp16 subnormals and zeros
+    rows.append(r)
+    r = torch.randn(K, generator=g) * 0.02
+    r[::7] = 5e-5                                      # mixed normal and subnormal magnitudes
+    rows.append(r)
+    r = torch.randn(K, generator=g) * 30.0             # lane sums around 2^11
+    rows.append(r)
+    r = torch.randn(K, generator=g)
+    r[5] = 65504.0                                     # the largest fp16 value
+    rows.append(r)
+    w = torch.stack(rows).to(torch.float16)
+    _check_tq(w)
