@@ -83,8 +83,7 @@ struct PrefillLayout {
   // tcgen05.alloc for tensor memory held by another CTA (which may itself wait at a cluster
   // barrier for a CTA that waits for tensor memory)
   static constexpr int kAlloc = kBytes + 1024 > 116 * 1024 ? kBytes + 1024 : 116 * 1024;
-  // partials with a padded row pitch (TN / S + 1 floats: conflict-free) in the freed x and
-  // packed rings
+  // partials [S][TN / S][128 rows] fp32 (rows contiguous) in the freed x and packed rings
   static_assert(kQM * (TN + 8) * 4 <= kRing * kTileX + PFmt<kInt4>::kPRing * PFmt<kInt4>::kTileP,
                 "split-K partials fit");
   // tensor memory: accumulator columns [0, TN), decoded-weight slots after it (not kSS)
@@ -399,10 +398,11 @@ __global__ void __launch_bounds__(kQThreads, 1)
     } else {
       // split K: the tokens of the tile are split evenly over the S CTAs of the cluster; each
       // CTA sends its partial sums of the other CTAs' tokens into their shared memory
-      // ([source rank][row][token], row pitch tpo + 1, in the freed x and packed rings) and
-      // adds the S partials of its own tokens in rank order (deterministic).
+      // ([source rank][token][row], in the freed x and packed rings: the 32 lanes of a warp,
+      // rows r .. r + 31, write one contiguous 128-byte line per token, one remote transaction
+      // per store instead of one per lane) and adds the S partials of its own tokens in rank
+      // order (deterministic).
       const int tpo = TN / a.S;  // tokens owned by each CTA
-      const int pitch = tpo + 1;
       float* red = reinterpret_cast<float*>(sm + L::kOffX);
       const uint32_t red_local = smem_u32(red);
       cluster_sync_all();  // every CTA of the cluster is past its main loop: the x rings are free
@@ -419,14 +419,14 @@ __global__ void __launch_bounds__(kQThreads, 1)
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           const int tok = c * 32 + j, q = tok / tpo;
-          const uint32_t off = ((rank * kQM + r) * pitch + (tok - q * tpo)) * 4;
+          const uint32_t off = ((rank * tpo + (tok - q * tpo)) * kQM + r) * 4;
           st_shared_cluster_f32(mapa_shared(red_local + off, static_cast<uint32_t>(q)), __uint_as_float(rr[j]));
         }
       }
       cluster_sync_all();  // all partials have landed
       for (int j = 0; j < tpo; ++j) {
         float v = 0.0f;
-        for (int src = 0; src < a.S; ++src) v += red[(src * kQM + r) * pitch + j];
+        for (int src = 0; src < a.S; ++src) v += red[(src * tpo + j) * kQM + r];
         const int64_t m = m0 + rank * tpo + j;
         if (m < a.M && n < a.N) a.y[m * a.N + n] = __float2half_rn(kInt4 ? v + ep_b : fmaf(v, ep_s, ep_b));
       }
