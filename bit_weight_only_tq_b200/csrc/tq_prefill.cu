@@ -19,8 +19,9 @@
 //     registers in natural k order and store them with one tcgen05.st per stage;
 //       ternary: (c - 1) is exact in fp16; the row scale is applied in the epilogue;
 //       W4A16:   fp16(q * s[n, k/128]) (one rounding, <= 2^-11 relative);
-//     then the epilogue: tcgen05.ld 32 tokens of the row at a time, scale / bias, fp16, staged
-//     through shared memory for coalesced 16-byte stores of y.
+//   * the epilogue, all eight warps in two groups of four taking alternate 32-token chunks:
+//     tcgen05.ld 32 tokens of a row at a time, scale / bias, fp16, staged through shared memory
+//     for coalesced 16-byte stores of y.
 // Shared-memory traffic per MMA is the x tile only (read by the MMA, written by TMA); decoding
 // into shared memory would add the weight tile twice (written, then read).
 // Every wait is bounded; a wait that runs out records a timeout in the device status word and
@@ -34,6 +35,8 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+
+#include <atomic>
 
 #include "tq_common.cuh"
 
@@ -69,7 +72,6 @@ struct PrefillLayout {
   // equal rings: one barrier per stage for "x tile landed and weights decoded" and one for
   // "stage consumed", so the MMA thread tests one barrier and commits once per stage
   static constexpr bool kMergedBars = kMergeStageBarriers && kRing == kARing;
-  // split-K partials [S][128 rows][TN / S] fp32 reuse the x ring after the main loop
   static constexpr int kOffX = 0;
   static constexpr int kOffP = kOffX + kRing * kTileX;
   static constexpr int kOffA = kOffP + PFmt<kInt4>::kPRing * PFmt<kInt4>::kTileP;
@@ -83,14 +85,15 @@ struct PrefillLayout {
   // tcgen05.alloc for tensor memory held by another CTA (which may itself wait at a cluster
   // barrier for a CTA that waits for tensor memory)
   static constexpr int kAlloc = kBytes + 1024 > 116 * 1024 ? kBytes + 1024 : 116 * 1024;
-  // partials [S][TN / S][128 rows] fp32 (rows contiguous) in the freed x and packed rings
+  // split-K partials [S][TN / S / 4][128 rows][4] fp32 reuse the x and packed rings after the
+  // main loop
   static_assert(kQM * (TN + 8) * 4 <= kRing * kTileX + PFmt<kInt4>::kPRing * PFmt<kInt4>::kTileP,
                 "split-K partials fit");
   // tensor memory: accumulator columns [0, TN), decoded-weight slots after it (not kSS)
   static constexpr uint32_t kColA = TN;
   static constexpr uint32_t kTmemCols = kSS ? static_cast<uint32_t>(TN) : (TN + 32 * kARing <= 256 ? 256u : 512u);
-  // epilogue staging (reuses the x ring): 32 tokens x 128 rows fp16
-  static_assert(32 * kQM * 2 <= kRing * kTileX, "staging fits in the x ring");
+  // epilogue staging (reuses the x ring): two buffers of 32 tokens x 128 rows fp16
+  static_assert(2 * 32 * kQM * 2 <= kRing * kTileX, "staging fits in the x ring");
   static_assert(kRing <= kQMaxRing && kARing <= kQMaxARing && (kSS || TN + 32 * kARing <= 512), "rings");
   static_assert(kAlloc <= 227 * 1024, "shared memory");
 };
@@ -206,6 +209,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   bool ok = true;
+  bool acc_flag = false;  // decode warps: the accumulator is complete
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer: x
     pdl_wait_prior_grids();
@@ -274,11 +278,6 @@ __global__ void __launch_bounds__(kQThreads, 1)
     const int r = threadIdx.x - 128;  // weight row within the tile = TMEM lane
     const int64_t n = n0 + r;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp - 4) * 32) << 16);
-    float ep_s = 1.0f, ep_b = 0.0f;  // epilogue scale / bias of this row (constants)
-    if (n < a.N) {
-      if (!kInt4) ep_s = __half2float(a.sc[n]);
-      if (a.bias) ep_b = __half2float(a.bias[n]);
-    }
     // W4A16 group scales of this row: the next group's is loaded when a group starts, a stage
     // or two before it is needed, so the load latency stays off the decode
     auto group_scale = [&](int64_t gi) -> uint16_t {
@@ -357,85 +356,139 @@ __global__ void __launch_bounds__(kQThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&afull[as]);
     }
+    acc_flag = ok && mbar_wait(accFull, 0u);
+  }
 
-    // ---------------------------------------------------------------- epilogue (same warps)
-    pdl_wait_prior_grids();  // y may still be read by the previous kernel
-    const bool acc_ok = ok && mbar_wait(accFull, 0u);
-    tc_fence_after_sync();
+  // ------------------------------------------------------------------ epilogue (all eight warps)
+  // Two groups of four warps (warps 4-7, then 0-3) take alternate 32-token chunks of the
+  // accumulator; warp w reads tensor-memory lanes 32 (w % 4) .. + 31, i.e. weight row
+  // r = threadIdx.x % 128.  The decode warps saw the accumulator complete (or the wait run out).
+  if (threadIdx.x == 128) tmem_slot[1] = acc_flag ? 1u : 0u;
+  pdl_wait_prior_grids();  // y may still be read by the previous kernel
+  __syncwarp();            // the single-lane producer and MMA loops have ended
+  named_barrier_sync(3, kQThreads);
+  const bool acc_ok = tmem_slot[1] != 0u;
+  tc_fence_after_sync();
+  {
+    const int grp = warp < 4 ? 1 : 0;  // chunk parity of this warp's group
+    const int r = threadIdx.x & (kQM - 1);
+    const int64_t n = n0 + r;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    float ep_s = 1.0f, ep_b = 0.0f;  // scale / bias of this row
+    if (n < a.N) {
+      if (!kInt4) ep_s = __half2float(a.sc[n]);
+      if (a.bias) ep_b = __half2float(a.bias[n]);
+    }
     const bool vec = (a.N & 7) == 0;
-    if (a.S == 1) {
-      __half* stage = reinterpret_cast<__half*>(sm + L::kOffX);  // [32 tokens][128 rows]
-      const int et = threadIdx.x - 128;                           // 0..127
-#pragma unroll 1
-      for (int c = 0; c < TN / 32 && acc_ok; ++c) {
-        uint32_t rr[32];
-        tmem_ld_32x32b_x32(lane_base + c * 32, rr);
-        tmem_ld_wait();
+    // y[m0 + t0 + t, n0 + 0..127] for t < cnt (<= 32) from a staging buffer [cnt][128 rows]
+    // fp16 of this group: 16 chunks of 16 bytes per token, four per thread, then the buffer is
+    // free again
+    auto store_staged = [&](const __half* stage, int t0, int cnt) {
+      named_barrier_sync(1 + grp, 128);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float v = __uint_as_float(rr[j]);
-          stage[j * kQM + r] = __float2half_rn(kInt4 ? v + ep_b : fmaf(v, ep_s, ep_b));
-        }
-        named_barrier_sync(1, 128);
-        // 32 tokens x 128 rows: 16 chunks of 16 bytes per token, four per thread
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int idx = et + 128 * q, tok = idx >> 4, ch = idx & 15;
-          const int64_t m = m0 + c * 32 + tok, nb = n0 + ch * 8;
-          if (m < a.M && nb < a.N) {
-            const uint4 val = *reinterpret_cast<const uint4*>(stage + tok * kQM + ch * 8);
-            __half* dst = a.y + m * a.N + nb;
-            if (vec && nb + 8 <= a.N) {
-              *reinterpret_cast<uint4*>(dst) = val;
-            } else {
-              const __half* hv = reinterpret_cast<const __half*>(&val);
-              for (int e = 0; e < 8 && nb + e < a.N; ++e) dst[e] = hv[e];
-            }
+      for (int q = 0; q < 4; ++q) {
+        const int idx = r + 128 * q, tok = idx >> 4, ch = idx & 15;
+        const int64_t m = m0 + t0 + tok, nb = n0 + ch * 8;
+        if (tok < cnt && m < a.M && nb < a.N) {
+          const uint4 val = *reinterpret_cast<const uint4*>(stage + tok * kQM + ch * 8);
+          __half* dst = a.y + m * a.N + nb;
+          if (vec && nb + 8 <= a.N) {
+            *reinterpret_cast<uint4*>(dst) = val;
+          } else {
+            const __half* hv = reinterpret_cast<const __half*>(&val);
+            for (int e = 0; e < 8 && nb + e < a.N; ++e) dst[e] = hv[e];
           }
         }
-        named_barrier_sync(1, 128);
+      }
+      named_barrier_sync(1 + grp, 128);
+    };
+    auto out_h = [&](float v) { return __float2half_rn(kInt4 ? v + ep_b : fmaf(v, ep_s, ep_b)); };
+    auto load_chunk = [&](int c, uint32_t (&rr)[32]) {
+      if (acc_ok) {
+        tmem_ld_32x32b_x32(lane_base + c * 32, rr);
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) rr[j] = 0u;
+      }
+    };
+    if (a.S == 1) {
+      __half* stage = reinterpret_cast<__half*>(sm + L::kOffX) + grp * 32 * kQM;  // [32 tokens][128 rows]
+#pragma unroll 1
+      for (int c = grp; c < TN / 32 && acc_ok; c += 2) {
+        uint32_t rr[32];
+        load_chunk(c, rr);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) stage[j * kQM + r] = out_h(__uint_as_float(rr[j]));
+        store_staged(stage, c * 32, 32);
       }
     } else {
-      // split K: the tokens of the tile are split evenly over the S CTAs of the cluster; each
-      // CTA sends its partial sums of the other CTAs' tokens into their shared memory
-      // ([source rank][token][row], in the freed x and packed rings: the 32 lanes of a warp,
-      // rows r .. r + 31, write one contiguous 128-byte line per token, one remote transaction
-      // per store instead of one per lane) and adds the S partials of its own tokens in rank
-      // order (deterministic).
-      const int tpo = TN / a.S;  // tokens owned by each CTA
+      // split K: the tokens of the tile are split evenly over the S CTAs of the cluster (tpo =
+      // TN / S each, a multiple of 8).  Each CTA sends its partial sums of the other CTAs'
+      // tokens into their shared memory, laid out [source rank][token / 4][row][token % 4] fp32
+      // in the freed x and packed rings: one 16-byte store per thread of four tokens of its row,
+      // 512 contiguous bytes per warp.  Its own tokens stay in tensor memory; it adds the S
+      // partials of each of them in rank order (the same order on every run) and writes y
+      // through staging buffers in the slot of its own rank (no CTA writes there).
+      const int tpo = TN / a.S, own0 = rank * tpo, own1 = own0 + tpo;
       float* red = reinterpret_cast<float*>(sm + L::kOffX);
       const uint32_t red_local = smem_u32(red);
+      auto slot = [&](int src, int tl) { return ((src * (tpo >> 2) + (tl >> 2)) * kQM + r) * 4; };  // floats
       cluster_sync_all();  // every CTA of the cluster is past its main loop: the x rings are free
 #pragma unroll 1
-      for (int c = 0; c < TN / 32; ++c) {
+      for (int c = grp; c < TN / 32; c += 2) {
+        if (c * 32 >= own0 && c * 32 + 32 <= own1) continue;  // all 32 tokens are this CTA's
         uint32_t rr[32];
-        if (acc_ok) {
-          tmem_ld_32x32b_x32(lane_base + c * 32, rr);
-          tmem_ld_wait();
-        } else {
+        load_chunk(c, rr);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) rr[j] = 0u;
-        }
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int tok = c * 32 + j, q = tok / tpo;
-          const uint32_t off = ((rank * tpo + (tok - q * tpo)) * kQM + r) * 4;
-          st_shared_cluster_f32(mapa_shared(red_local + off, static_cast<uint32_t>(q)), __uint_as_float(rr[j]));
+        for (int j = 0; j < 32; j += 4) {
+          const int tok = c * 32 + j, q = tok / tpo;  // four consecutive tokens share an owner
+          if (q != rank) {
+            const uint32_t dst = red_local + 4u * static_cast<uint32_t>(slot(rank, tok - q * tpo));
+            st_shared_cluster_v4_f32(mapa_shared(dst, static_cast<uint32_t>(q)), rr[j], rr[j + 1], rr[j + 2],
+                                     rr[j + 3]);
+          }
         }
       }
       cluster_sync_all();  // all partials have landed
-      for (int j = 0; j < tpo; ++j) {
-        float v = 0.0f;
-        for (int src = 0; src < a.S; ++src) v += red[(src * tpo + j) * kQM + r];
-        const int64_t m = m0 + rank * tpo + j;
-        if (m < a.M && n < a.N) a.y[m * a.N + n] = __float2half_rn(kInt4 ? v + ep_b : fmaf(v, ep_s, ep_b));
+      // own chunks alternate between the groups; a second staging buffer is needed only when
+      // there are two or more own chunks (tpo >= 64: the own slot holds 32 KB or more)
+      const int oc0 = own0 / 32;
+      __half* stage = reinterpret_cast<__half*>(red + static_cast<size_t>(own0) * kQM) + grp * 32 * kQM;
+#pragma unroll 1
+      for (int c = oc0 + grp; c * 32 < own1; c += 2) {
+        const int b0 = max(c * 32, own0), b1 = min(c * 32 + 32, own1);  // own tokens of chunk c
+        uint32_t rr[32];
+        load_chunk(c, rr);
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+        for (int src = 0; src < a.S; ++src) {
+          if (src == rank) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] += __uint_as_float(rr[j]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              const int tok = c * 32 + j;
+              if (tok >= b0 && tok < b1) {
+                const float4 p = *reinterpret_cast<const float4*>(red + slot(src, tok - own0));
+                v[j] += p.x;
+                v[j + 1] += p.y;
+                v[j + 2] += p.z;
+                v[j + 3] += p.w;
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int tok = c * 32 + j;
+          if (tok >= b0 && tok < b1) stage[(tok - b0) * kQM + r] = out_h(v[j]);
+        }
+        store_staged(stage, b0, b1 - b0);
       }
     }
-  }
-  if (warp < 4 && a.S > 1) {
-    // every thread of the cluster takes part in the two barriers of the split-K epilogue
-    cluster_sync_all();
-    cluster_sync_all();
   }
 
   tc_fence_before_sync();
@@ -502,10 +555,46 @@ static cudaError_t launch_prefill_t(const __half* x, const void* w, const __half
   return cudaLaunchKernelEx(&cfg, kern, tx, tw, a);
 }
 
-// Tile choice: 64 tokens for M <= 64 (an N < 64 MMA costs as much as N = 64), 256 when those
-// tiles alone fill the GPU (each decoded weight then feeds the most MMAs), else 128 (as
-// efficient per MMA as 256); K split over a cluster of S CTAs (1, 2, 4 or 8) while the tiles
-// alone leave SMs idle.
+// Clusters of S CTAs of this kernel that can be resident at once (a cluster's CTAs share one
+// GPC, so the GPCs bound it below SMs / S), queried once per device and S; 0 when unknown.
+constexpr int kPfMaxDevices = 64;
+
+template <bool kInt4, int TN, bool kSS>
+static int prefill_cluster_capacity(int device, int S) {
+  using L = PrefillLayout<kInt4, TN, kSS>;
+  static std::atomic<int> cache[kPfMaxDevices][4];
+  if (device < 0 || device >= kPfMaxDevices || S < 2 || S > 8) return 0;
+  const int li = S == 2 ? 1 : (S == 4 ? 2 : 3);
+  int n = cache[device][li].load(std::memory_order_relaxed);
+  if (n > 0) return n;
+  auto* kern = prefill_gemm_kernel<kInt4, TN, kSS>;
+  if (ensure_smem_attr(reinterpret_cast<const void*>(kern), L::kAlloc) != cudaSuccess) return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1, 1, static_cast<unsigned>(S));
+  cfg.blockDim = dim3(kQThreads, 1, 1);
+  cfg.dynamicSmemBytes = L::kAlloc;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = 1;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = static_cast<unsigned>(S);
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  cache[device][li].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+// Tile choice: 64 tokens for M <= 64 (an N < 64 MMA costs as much as N = 64), 128 for M <= 128,
+// else 256: a stage of 256 tokens takes about as long as one of 128 (the issuing thread, not the
+// tensor pipe, sets the narrow tiles' stage time), so the wide tile does twice the work per SM
+// and stage; K split over a cluster of S CTAs (1, 2, 4 or 8) while the tiles alone leave SMs
+// idle and all the clusters fit on the GPU at once (a second wave of clusters costs more than
+// the narrower split saves).
 constexpr int kPrefillSSMaxTN = 128;  // token tiles up to this width read A from shared memory
 
 template <bool kInt4>
@@ -515,10 +604,19 @@ static cudaError_t launch_prefill(const __half* x, const void* w, const __half* 
   const DeviceInfo di = current_device_info();
   const int64_t rt = (N + kQM - 1) / kQM;
   const int nk = static_cast<int>(K / kQK);
-  const int TN = M <= 64 ? 64 : ((M <= 128 || rt * ((M + 255) / 256) < di.num_sms) ? 128 : 256);
+  const int TN = M <= 64 ? 64 : (M <= 128 ? 128 : 256);
   const int64_t base = rt * ((M + TN - 1) / TN);
+  auto capacity = [&](int cs) {
+    if (TN == 64) return prefill_cluster_capacity<kInt4, 64, kPrefillSSMaxTN >= 64>(di.device, cs);
+    if (TN == 128) return prefill_cluster_capacity<kInt4, 128, kPrefillSSMaxTN >= 128>(di.device, cs);
+    return prefill_cluster_capacity<kInt4, 256, false>(di.device, cs);
+  };
   int S = 1;
-  while (S < 8 && base * S * 2 <= di.num_sms && S * 2 <= nk) S *= 2;
+  while (S < 8 && base * S * 2 <= di.num_sms && S * 2 <= nk) {
+    const int cap = capacity(S * 2);
+    if (cap > 0 && base > cap) break;
+    S *= 2;
+  }
   if (TN == 64) return launch_prefill_t<kInt4, 64, kPrefillSSMaxTN >= 64>(x, w, sc, zp, bias, y, M, N, K, S, s);
   if (TN == 128) return launch_prefill_t<kInt4, 128, kPrefillSSMaxTN >= 128>(x, w, sc, zp, bias, y, M, N, K, S, s);
   return launch_prefill_t<kInt4, 256, false>(x, w, sc, zp, bias, y, M, N, K, S, s);
