@@ -3,8 +3,8 @@
 Headline workload (one "step"): the Llama-3-8B-shaped ternary decode sweep -- 32 distinct layers
 x 7 linears (q, k, v, o, gate, up, down) x M in {1, 4, 16} tokens, x ~ N(0,1) fp16, weights
 ~ N(0, 0.02) ternarised and packed by tq_quantize_pack (1.745 GB packed, larger than L2, so no
-L2 flush is needed between steps).  Every GEMM goes through the public tq_gemm C-ABI call
-(path chosen by the library's dispatch); the 672 calls of a step are captured in CUDA graphs.
+L2 flush is needed between steps).  Each layer and M is one tq_gemm_batch C-ABI call (its 7
+linears in one persistent launch); the 96 calls of a step are captured in one CUDA graph.
 
 metric: decode packed-weight GB/s (algorithmic bytes: packed weights + scales + x + y) ; the
 other hot-path rows (prefill TFLOP/s, W4A16, pack) are measured after the headline step and
@@ -188,6 +188,23 @@ def build_ternary_layers(rank, n_layers, config=1, shapes=LLAMA, dtype=None):
         layers.append(row)
     torch.cuda.synchronize()
     return layers
+
+
+def layer_calls(gemm, grouped, row, xs, ys, bs=None):
+    """The seven linears of one Llama layer as a serving engine issues them: q/k/v and gate/up
+    each through one grouped call (they read the same x), o and down alone."""
+    d = {name: (N, K, w, s) for name, N, K, w, s in row}
+
+    def grp(names):
+        grouped(xs[d[names[0]][1]], [d[n][2] for n in names], [d[n][3] for n in names],
+                None if bs is None else [bs[d[n][0]] for n in names], [ys[n] for n in names])
+
+    grp(("q_proj", "k_proj", "v_proj"))
+    N, K, w, s = d["o_proj"]
+    gemm(xs[K], w, s, None if bs is None else bs[N], ys["o_proj"])
+    grp(("gate_proj", "up_proj"))
+    N, K, w, s = d["down_proj"]
+    gemm(xs[K], w, s, None if bs is None else bs[N], ys["down_proj"])
 
 
 def capture(fn):
@@ -481,19 +498,19 @@ def secondary_rows(args, rank, layers, peaks):
     for M in (2048, 512, 8192):
         xs = {K: I.activations(M, K, I.seed_for(2, 0, K), device="cuda", outlier_row_frac=0.01)
               for K in (4096, 14336)}
-        ys = {N: torch.empty(M, N, dtype=torch.float16, device="cuda") for N in (1024, 4096, 14336)}
+        ys = {name: torch.empty(M, N, dtype=torch.float16, device="cuda") for name, N, _ in LLAMA}
 
         def pf():
             for row in sub:
-                for name, N, K, p, s in row:
-                    tq.tq_gemm(xs[K], p, s, bs[N], ys[N])
+                layer_calls(tq.tq_gemm, tq.tq_gemm_grouped, row, xs, ys, bs)
 
         g = capture(pf)
         ms = time_graph(g, 10)
         flops = sum(2 * M * N * K for row in sub for _, N, K, _, _ in row)
         tf = flops / (ms * 1e-3) / 1e12
         rows[f"ternary_prefill_M{M}"] = {"value": round(tf, 1), "unit": "TFLOP/s", "frac": round(tf / tc, 4),
-                                         "peak": tc, "bound": "tensor", "sample": f"4 layers x 7 shapes, M={M}"}
+                                         "peak": tc, "bound": "tensor",
+                                         "sample": f"4 layers x 7 shapes, M={M}; q/k/v and gate/up grouped"}
         del g, xs, ys
     # ---- W4A16 decode / prefill (config 3): 8 layers
     w4 = []
@@ -531,12 +548,11 @@ def secondary_rows(args, rank, layers, peaks):
             del g
     for M, wl in ((4096, w4[:1]), (256, w4)):
         xq = {K: I.activations(M, K, I.seed_for(3, 3, K), device="cuda") for K in (4096, 14336)}
-        yq = {N: torch.empty(M, N, dtype=torch.float16, device="cuda") for N in (1024, 4096, 14336)}
+        yq = {name: torch.empty(M, N, dtype=torch.float16, device="cuda") for name, N, _ in LLAMA}
 
         def wp():
             for row in wl:
-                for name, N, K, qw, sc in row:
-                    tq.w4g_gemm(xq[K], qw, sc, None, yq[N])
+                layer_calls(tq.w4g_gemm, tq.w4g_gemm_grouped, row, xq, yq)
 
         g = capture(wp)
         ms = time_graph(g, 10)
@@ -544,7 +560,8 @@ def secondary_rows(args, rank, layers, peaks):
         tf = flops / (ms * 1e-3) / 1e12
         rows[f"w4g_prefill_M{M}"] = {"value": round(tf, 1), "unit": "TFLOP/s", "frac": round(tf / tc, 4),
                                      "peak": tc, "bound": "tensor",
-                                     "sample": f"{len(wl)} layer{'s' if len(wl) > 1 else ''} x 7 shapes, M={M}"}
+                                     "sample": f"{len(wl)} layer{'s' if len(wl) > 1 else ''} x 7 shapes, M={M}; "
+                                               "q/k/v and gate/up grouped"}
         del g, xq, yq
     del w4
     # ---- config 0: one ternary linear 1024x1024 at M = 1 (L2-resident: the time of one call)

@@ -162,7 +162,8 @@ int resolve_path(int fmt, int path, int64_t M, int64_t N, int64_t K, bool all_al
 }
 
 // Shared driver of the grouped entry points: one decode launch when every matrix takes the
-// decode path, otherwise one single-matrix GEMM per matrix.
+// decode path, one tensor-core launch when every matrix takes the prefill path, otherwise one
+// single-matrix GEMM per matrix.
 template <bool kInt4, typename WT, typename Single, typename Group>
 static int gemm_grouped_impl(const uint16_t* x, int count, const WT* const* w,
                              const uint16_t* const* sc, const uint16_t* const* bias,
@@ -189,6 +190,31 @@ static int gemm_grouped_impl(const uint16_t* x, int count, const WT* const* w,
     return to_status(group(reinterpret_cast<const __half*>(x), count, w,
                            reinterpret_cast<const __half* const*>(sc), bh,
                            reinterpret_cast<__half* const*>(y), N, M, K, as_stream(stream)));
+  }
+  // every non-empty matrix on the tensor-core path: one launch over all their row tiles
+  {
+    const int fmt = kInt4 ? TQ_FMT_W4G128 : TQ_FMT_TERNARY;
+    int n = 0;
+    const void* gw[4];
+    const __half* gs[4];
+    const __half* gb[4];
+    __half* gy[4];
+    int64_t gn[4];
+    bool all_prefill = true;
+    for (int g = 0; g < count && all_prefill; ++g) {
+      if (N[g] == 0) continue;
+      const bool al = aligned16(x) && aligned16(w[g]) && aligned16(y[g]) && (!kInt4 || aligned16(sc[g]));
+      all_prefill = tq_select_path(fmt, M, N[g], K, al ? 1 : 0) == TQ_PATH_PREFILL;
+      gw[n] = w[g];
+      gs[n] = reinterpret_cast<const __half*>(sc[g]);
+      gb[n] = bias ? reinterpret_cast<const __half*>(bias[g]) : nullptr;
+      gy[n] = reinterpret_cast<__half*>(y[g]);
+      gn[n] = N[g];
+      ++n;
+    }
+    if (all_prefill && n > 1 && tq::prefill_grouping_pays(M, gn, n))
+      return to_status(tq::launch_gemm_prefill_grouped(kInt4, reinterpret_cast<const __half*>(x), n, gw, gs, gb, gy,
+                                                       gn, M, K, as_stream(stream)));
   }
   for (int g = 0; g < count; ++g) {
     const int st = single(x, w[g], sc[g], bias ? bias[g] : nullptr, y[g], M, N[g], K, stream);

@@ -204,7 +204,7 @@ cudaError_t launch_tq_validate(const uint8_t* packed, int64_t N, int64_t K, int*
 constexpr int64_t kDecodeMaxM = 64;
 // Largest M the automatic dispatch sends to the decode path, per format (the measured crossover
 // with the tensor-core path on Llama-3-8B and Qwen2-7B shaped linears).
-constexpr int64_t kDecodeAutoMaxM_Ternary = 48;
+constexpr int64_t kDecodeAutoMaxM_Ternary = 32;
 constexpr int64_t kDecodeAutoMaxM_W4g = 16;
 cudaError_t launch_tq_gemm_decode(const __half* x, const uint8_t* packed, const __half* scale,
                                   const __half* bias, __half* y, int64_t M, int64_t N, int64_t K,
@@ -226,6 +226,13 @@ cudaError_t launch_tq_gemm_prefill(const __half* x, const uint8_t* packed, const
 cudaError_t launch_w4g_gemm_prefill(const __half* x, const int32_t* qweight, const __half* scales,
                                     const uint8_t* zeros, const __half* bias, __half* y, int64_t M, int64_t N,
                                     int64_t K, cudaStream_t s);
+// Up to four matrices that read the same x in ONE tensor-core launch (symmetric W4A16 when int4);
+// every matrix must satisfy prefill_supported and the prefill path's alignment.  Worth it when
+// prefill_grouping_pays (their tiles together fill at most a few waves).
+bool prefill_grouping_pays(int64_t M, const int64_t* N, int count);
+cudaError_t launch_gemm_prefill_grouped(bool int4, const __half* x, int count, const void* const* w,
+                                        const __half* const* sc, const __half* const* bias, __half* const* y,
+                                        const int64_t* N, int64_t M, int64_t K, cudaStream_t s);
 
 // Work list of the persistent batch decode kernel (tq_batch.cu): independent linears sharing M.
 struct BatchLinear {

@@ -15,11 +15,12 @@
 //   * warp 1: allocates the tensor memory (accumulator + a ring of decoded-weight slots); one
 //     lane issues tcgen05.mma (M=128, N=TN, K=16, A from tensor memory) and commits to
 //     mbarriers that free the input stages;
-//   * warps 4-7 (thread r = weight row r = TMEM lane r): decode the packed row into 32 fp16x2
-//     registers in natural k order and store them with one tcgen05.st per stage;
+//   * warps 4-11, two groups of four taking alternate stages (thread r % 128 = weight row r =
+//     TMEM lane r): decode the packed row into 32 fp16x2 registers in natural k order and store
+//     them with one tcgen05.st per stage;
 //       ternary: (c - 1) is exact in fp16; the row scale is applied in the epilogue;
 //       W4A16:   fp16(q * s[n, k/128]) (one rounding, <= 2^-11 relative);
-//   * the epilogue, all eight warps in two groups of four taking alternate 32-token chunks:
+//   * the epilogue, all twelve warps in three groups of four taking 32-token chunks in turn:
 //     tcgen05.ld 32 tokens of a row at a time, scale / bias, fp16, staged through shared memory
 //     for coalesced 16-byte stores of y.
 // Shared-memory traffic per MMA is the x tile only (read by the MMA, written by TMA); decoding
@@ -46,7 +47,9 @@ constexpr int kQM = 128;         // weight rows per CTA (UMMA M, TMEM lanes)
 constexpr int kQK = 64;          // K per stage: one 128-byte swizzle row of fp16
 constexpr int kQMaxRing = 12;    // stages of (x tile, packed tile), at most
 constexpr int kQMaxARing = 8;    // tensor-memory slots of decoded weights (32 columns each)
-constexpr int kQThreads = 256;   // warp 0 TMA, warp 1 MMA, warps 4-7 decode + epilogue
+constexpr int kQDecGroups = 2;   // groups of four decode warps, taking alternate stages
+constexpr int kQThreads = 128 * (1 + kQDecGroups);  // warps 0-3: TMA, MMA; then the decode groups
+constexpr int kQEpiGroups = 1 + kQDecGroups;        // every group of four warps runs the epilogue
 constexpr bool kMergeStageBarriers = true;
 
 template <bool kInt4>
@@ -57,6 +60,7 @@ struct PFmt {
   static constexpr int kSPP = 128 / kRowBytes;       // stages per packed tile
   static constexpr int kTileP = kQM * 128;
   static constexpr int kPRing = 3;
+  static_assert(kSPP % kQDecGroups == 0, "the decode groups alternate within a packed tile");
 };
 
 // kSS: the decoded weights go to shared memory (128-byte-swizzled K-major tiles, the layout TMA
@@ -92,19 +96,31 @@ struct PrefillLayout {
   // tensor memory: accumulator columns [0, TN), decoded-weight slots after it (not kSS)
   static constexpr uint32_t kColA = TN;
   static constexpr uint32_t kTmemCols = kSS ? static_cast<uint32_t>(TN) : (TN + 32 * kARing <= 256 ? 256u : 512u);
-  // epilogue staging (reuses the x ring): two buffers of 32 tokens x 128 rows fp16
-  static_assert(2 * 32 * kQM * 2 <= kRing * kTileX, "staging fits in the x ring");
+  // epilogue staging (reuses the x ring): one buffer of 32 tokens x 128 rows fp16 per group
+  static_assert(kQEpiGroups * 32 * kQM * 2 <= kRing * kTileX, "staging fits in the x ring");
   static_assert(kRing <= kQMaxRing && kARing <= kQMaxARing && (kSS || TN + 32 * kARing <= 512), "rings");
   static_assert(kAlloc <= 227 * 1024, "shared memory");
 };
 
+// One launch covers up to kQMaxGroup matrices that share x (a serving engine's fused q/k/v or
+// gate/up): grid x runs over the row tiles of all of them, matrix g owning tiles
+// [tile0[g], tile0[g + 1]).
+constexpr int kQMaxGroup = 4;
+
 struct PrefillArgs {
-  const __half* sc;    // ternary: scale[N]; W4A16: scales[N, K/128]
-  const uint8_t* zp;   // W4A16 zero-points [N, K/128], or null (symmetric)
-  const __half* bias;  // may be null
-  __half* y;
-  int64_t M, N, K;
+  const __half* sc[kQMaxGroup];    // ternary: scale[N]; W4A16: scales[N, K/128]
+  const uint8_t* zp[kQMaxGroup];   // W4A16 zero-points [N, K/128], or null (symmetric)
+  const __half* bias[kQMaxGroup];  // may be null
+  __half* y[kQMaxGroup];
+  int64_t N[kQMaxGroup];
+  int tile0[kQMaxGroup + 1];
+  int count;
+  int64_t M, K;
   int S;               // K-slices: CTAs per cluster (grid z), reduced through DSMEM
+};
+
+struct PrefillWeightMaps {
+  CUtensorMap m[kQMaxGroup];  // packed weights of each matrix
 };
 
 __device__ __forceinline__ uint32_t hsub2_u32(uint32_t a, uint32_t b) {
@@ -154,7 +170,7 @@ __device__ __forceinline__ uint4 decode_w4_8(uint32_t w, uint32_t s2, uint32_t z
 template <bool kInt4, int TN, bool kSS>
 __global__ void __launch_bounds__(kQThreads, 1)
     prefill_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
-                        const __grid_constant__ CUtensorMap tmap_w, const PrefillArgs a) {
+                        const __grid_constant__ PrefillWeightMaps tmaps_w, const PrefillArgs a) {
   using L = PrefillLayout<kInt4, TN, kSS>;
   using F = PFmt<kInt4>;
   extern __shared__ uint8_t smem_raw[];
@@ -174,7 +190,15 @@ __global__ void __launch_bounds__(kQThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::kOffTmemSlot);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kQM;  // first weight row
+  int g = 0;  // matrix of this row tile
+  while (g + 1 < a.count && static_cast<int>(blockIdx.x) >= a.tile0[g + 1]) ++g;
+  const int64_t n0 = static_cast<int64_t>(static_cast<int>(blockIdx.x) - a.tile0[g]) * kQM;  // first weight row
+  const int64_t Ng = a.N[g];
+  const __half* const gsc = a.sc[g];
+  const uint8_t* const gzp = a.zp[g];
+  const __half* const gbias = a.bias[g];
+  __half* const gy = a.y[g];
+  const CUtensorMap* const tmap_w = &tmaps_w.m[g];
   const int64_t m0 = static_cast<int64_t>(blockIdx.y) * TN;   // first token
   const int nk_all = static_cast<int>(a.K / kQK);
   const int rank = static_cast<int>(blockIdx.z);              // K-slice = rank in the cluster
@@ -190,7 +214,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
     }
     for (int i = 0; i < F::kPRing; ++i) {
       mbar_init(&fullP[i], 1);
-      mbar_init(&emptyP[i], 4);
+      mbar_init(&emptyP[i], 4 * kQDecGroups);
     }
     for (int i = 0; i < L::kARing && !L::kMergedBars; ++i) {
       mbar_init(&afull[i], 4);
@@ -230,7 +254,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
     // ------------------------------------------------------------------ TMA producer: weights
     // (model constants: issued before the wait for the previous kernel)
     if (lane == 0) {
-      tma_prefetch_desc(&tmap_w);
+      tma_prefetch_desc(tmap_w);
       const int npt = (nk + F::kSPP - 1) / F::kSPP;
       for (int pt = 0; pt < npt && ok; ++pt) {
         const int s = pt % F::kPRing;
@@ -239,7 +263,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
           if (!ok) break;
         }
         mbar_arrive_expect_tx(&fullP[s], F::kTileP);
-        tma_load_2d(sm + L::kOffP + s * F::kTileP, &tmap_w, &fullP[s], (kb0 + pt * F::kSPP) * F::kRowBytes,
+        tma_load_2d(sm + L::kOffP + s * F::kTileP, tmap_w, &fullP[s], (kb0 + pt * F::kSPP) * F::kRowBytes,
                     static_cast<int32_t>(n0));
       }
     }
@@ -275,23 +299,26 @@ __global__ void __launch_bounds__(kQThreads, 1)
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------------ decode warps
-    const int r = threadIdx.x - 128;  // weight row within the tile = TMEM lane
+    // group dg decodes stages dg, dg + 2, ...: two warps per SM sub-partition hide each other's
+    // waits and tensor-memory store latency
+    const int dg = (warp >> 2) - 1;
+    const int r = threadIdx.x & (kQM - 1);  // weight row within the tile = TMEM lane
     const int64_t n = n0 + r;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp - 4) * 32) << 16);
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     // W4A16 group scales of this row: the next group's is loaded when a group starts, a stage
     // or two before it is needed, so the load latency stays off the decode
     auto group_scale = [&](int64_t gi) -> uint16_t {
-      return (n < a.N && gi < G) ? __half_as_ushort(a.sc[n * G + gi]) : static_cast<uint16_t>(0);
+      return (n < Ng && gi < G) ? __half_as_ushort(gsc[n * G + gi]) : static_cast<uint16_t>(0);
     };
     auto group_zero = [&](int64_t gi) -> uint32_t {
-      return (a.zp && n < a.N && gi < G) ? static_cast<uint32_t>(a.zp[n * G + gi]) : 8u;
+      return (gzp && n < Ng && gi < G) ? static_cast<uint32_t>(gzp[n * G + gi]) : 8u;
     };
     int64_t g_cur = -1;
     uint16_t sc_cur = 0, sc_nxt = 0;
     uint32_t zp_cur = 8u, zp_nxt = 8u;
-    for (int kb = 0; kb < nk && ok; ++kb) {
+    for (int kb = dg; kb < nk && ok; kb += kQDecGroups) {
       const int as = kb % L::kARing, pt = kb / F::kSPP, ci = kb - pt * F::kSPP, ps = pt % F::kPRing;
-      if (ci == 0) {
+      if (ci == dg) {  // this group's first stage of the packed tile (kSPP is even)
         ok = mbar_wait(&fullP[ps], static_cast<uint32_t>(pt / F::kPRing) & 1u);
         if (!ok) break;
       }
@@ -302,7 +329,9 @@ __global__ void __launch_bounds__(kQThreads, 1)
       const uint4 p0 = *reinterpret_cast<const uint4*>(prow + ((c0 ^ (r & 7)) << 4));
       uint4 p1 = make_uint4(0u, 0u, 0u, 0u);
       if (kInt4) p1 = *reinterpret_cast<const uint4*>(prow + (((c0 + 1) ^ (r & 7)) << 4));
-      if (ci == F::kSPP - 1 || kb == nk - 1) {  // done with this packed tile
+      // done with this packed tile: both groups arrive on every tile but a CTA's last, which
+      // no later load waits for
+      if (ci + kQDecGroups >= F::kSPP || kb + kQDecGroups >= nk) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&emptyP[ps]);
       }
@@ -359,44 +388,44 @@ __global__ void __launch_bounds__(kQThreads, 1)
     acc_flag = ok && mbar_wait(accFull, 0u);
   }
 
-  // ------------------------------------------------------------------ epilogue (all eight warps)
-  // Two groups of four warps (warps 4-7, then 0-3) take alternate 32-token chunks of the
-  // accumulator; warp w reads tensor-memory lanes 32 (w % 4) .. + 31, i.e. weight row
+  // ------------------------------------------------------------------ epilogue (all warps)
+  // The groups of four warps (the decode groups, then warps 0-3) take 32-token chunks of the
+  // accumulator in turn; warp w reads tensor-memory lanes 32 (w % 4) .. + 31, i.e. weight row
   // r = threadIdx.x % 128.  The decode warps saw the accumulator complete (or the wait run out).
   if (threadIdx.x == 128) tmem_slot[1] = acc_flag ? 1u : 0u;
   pdl_wait_prior_grids();  // y may still be read by the previous kernel
   __syncwarp();            // the single-lane producer and MMA loops have ended
-  named_barrier_sync(3, kQThreads);
+  named_barrier_sync(1 + kQEpiGroups, kQThreads);
   const bool acc_ok = tmem_slot[1] != 0u;
   tc_fence_after_sync();
   {
-    const int grp = warp < 4 ? 1 : 0;  // chunk parity of this warp's group
+    const int grp = ((warp >> 2) + kQEpiGroups - 1) % kQEpiGroups;  // chunks grp, grp + kQEpiGroups, ...
     const int r = threadIdx.x & (kQM - 1);
     const int64_t n = n0 + r;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     float ep_s = 1.0f, ep_b = 0.0f;  // scale / bias of this row
-    if (n < a.N) {
-      if (!kInt4) ep_s = __half2float(a.sc[n]);
-      if (a.bias) ep_b = __half2float(a.bias[n]);
+    if (n < Ng) {
+      if (!kInt4) ep_s = __half2float(gsc[n]);
+      if (gbias) ep_b = __half2float(gbias[n]);
     }
-    const bool vec = (a.N & 7) == 0;
+    const bool vec = (Ng & 7) == 0;
     // y[m0 + t0 + t, n0 + 0..127] for t < cnt (<= 32) from a staging buffer [cnt][128 rows]
-    // fp16 of this group: 16 chunks of 16 bytes per token, four per thread, then the buffer is
-    // free again
+    // fp16 of this group (named barrier 1 + grp): 16 chunks of 16 bytes per token, four per
+    // thread, then the buffer is free again
     auto store_staged = [&](const __half* stage, int t0, int cnt) {
       named_barrier_sync(1 + grp, 128);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const int idx = r + 128 * q, tok = idx >> 4, ch = idx & 15;
         const int64_t m = m0 + t0 + tok, nb = n0 + ch * 8;
-        if (tok < cnt && m < a.M && nb < a.N) {
+        if (tok < cnt && m < a.M && nb < Ng) {
           const uint4 val = *reinterpret_cast<const uint4*>(stage + tok * kQM + ch * 8);
-          __half* dst = a.y + m * a.N + nb;
-          if (vec && nb + 8 <= a.N) {
+          __half* dst = gy + m * Ng + nb;
+          if (vec && nb + 8 <= Ng) {
             *reinterpret_cast<uint4*>(dst) = val;
           } else {
             const __half* hv = reinterpret_cast<const __half*>(&val);
-            for (int e = 0; e < 8 && nb + e < a.N; ++e) dst[e] = hv[e];
+            for (int e = 0; e < 8 && nb + e < Ng; ++e) dst[e] = hv[e];
           }
         }
       }
@@ -415,7 +444,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
     if (a.S == 1) {
       __half* stage = reinterpret_cast<__half*>(sm + L::kOffX) + grp * 32 * kQM;  // [32 tokens][128 rows]
 #pragma unroll 1
-      for (int c = grp; c < TN / 32 && acc_ok; c += 2) {
+      for (int c = grp; c < TN / 32 && acc_ok; c += kQEpiGroups) {
         uint32_t rr[32];
         load_chunk(c, rr);
 #pragma unroll
@@ -436,7 +465,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
       auto slot = [&](int src, int tl) { return ((src * (tpo >> 2) + (tl >> 2)) * kQM + r) * 4; };  // floats
       cluster_sync_all();  // every CTA of the cluster is past its main loop: the x rings are free
 #pragma unroll 1
-      for (int c = grp; c < TN / 32; c += 2) {
+      for (int c = grp; c < TN / 32; c += kQEpiGroups) {
         if (c * 32 >= own0 && c * 32 + 32 <= own1) continue;  // all 32 tokens are this CTA's
         uint32_t rr[32];
         load_chunk(c, rr);
@@ -451,12 +480,12 @@ __global__ void __launch_bounds__(kQThreads, 1)
         }
       }
       cluster_sync_all();  // all partials have landed
-      // own chunks alternate between the groups; a second staging buffer is needed only when
-      // there are two or more own chunks (tpo >= 64: the own slot holds 32 KB or more)
+      // own chunks go to the groups in turn; group g's staging buffer (8 KB at 8 g KB) is used
+      // only when there are more than g own chunks (tpo > 32 g: the own slot holds 16 g KB or more)
       const int oc0 = own0 / 32;
       __half* stage = reinterpret_cast<__half*>(red + static_cast<size_t>(own0) * kQM) + grp * 32 * kQM;
 #pragma unroll 1
-      for (int c = oc0 + grp; c * 32 < own1; c += 2) {
+      for (int c = oc0 + grp; c * 32 < own1; c += kQEpiGroups) {
         const int b0 = max(c * 32, own0), b1 = min(c * 32 + 32, own1);  // own tokens of chunk c
         uint32_t rr[32];
         load_chunk(c, rr);
@@ -507,34 +536,55 @@ bool prefill_supported(bool int4, int64_t M, int64_t N, int64_t K) {
   return true;
 }
 
+// The matrices of one launch (all read the same x[M, K]).
+struct PrefillProblem {
+  int count;
+  const void* w[kQMaxGroup];
+  const __half* sc[kQMaxGroup];
+  const uint8_t* zp[kQMaxGroup];
+  const __half* bias[kQMaxGroup];
+  __half* y[kQMaxGroup];
+  int64_t N[kQMaxGroup];
+};
+
 template <bool kInt4, int TN, bool kSS>
-static cudaError_t launch_prefill_t(const __half* x, const void* w, const __half* sc, const uint8_t* zp,
-                                    const __half* bias, __half* y, int64_t M, int64_t N, int64_t K,
-                                    int S, cudaStream_t s) {
+static cudaError_t launch_prefill_t(const __half* x, const PrefillProblem& pb, int64_t M, int64_t K, int S,
+                                    cudaStream_t s) {
   using L = PrefillLayout<kInt4, TN, kSS>;
-  CUtensorMap tx, tw;
+  CUtensorMap tx;
+  PrefillWeightMaps tw;
   if (!make_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, static_cast<uint64_t>(K),
                     static_cast<uint64_t>(M), static_cast<uint64_t>(K) * 2, kQK, TN,
                     CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   const uint64_t kbytes = kInt4 ? static_cast<uint64_t>(K) / 2 : static_cast<uint64_t>(K) / 4;
-  if (!make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w, kbytes, static_cast<uint64_t>(N), kbytes,
-                    128, kQM, CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
+  PrefillArgs a = {};
+  a.count = pb.count;
+  a.tile0[0] = 0;
+  for (int g = 0; g < kQMaxGroup; ++g) {
+    if (g < pb.count) {
+      if (!make_tmap_2d(&tw.m[g], CU_TENSOR_MAP_DATA_TYPE_UINT8, pb.w[g], kbytes, static_cast<uint64_t>(pb.N[g]),
+                        kbytes, 128, kQM, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+      a.sc[g] = pb.sc[g];
+      a.zp[g] = pb.zp[g];
+      a.bias[g] = pb.bias[g];
+      a.y[g] = pb.y[g];
+      a.N[g] = pb.N[g];
+      a.tile0[g + 1] = a.tile0[g] + static_cast<int>((pb.N[g] + kQM - 1) / kQM);
+    } else {
+      tw.m[g] = tw.m[0];
+      a.tile0[g + 1] = a.tile0[g];
+    }
+  }
   auto* kern = prefill_gemm_kernel<kInt4, TN, kSS>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), L::kAlloc);
   if (e != cudaSuccess) return e;
-  PrefillArgs a;
-  a.sc = sc;
-  a.zp = zp;
-  a.bias = bias;
-  a.y = y;
   a.M = M;
-  a.N = N;
   a.K = K;
   a.S = S;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>((N + kQM - 1) / kQM), static_cast<unsigned>((M + TN - 1) / TN),
+  cfg.gridDim = dim3(static_cast<unsigned>(a.tile0[pb.count]), static_cast<unsigned>((M + TN - 1) / TN),
                      static_cast<unsigned>(S));
   cfg.blockDim = dim3(kQThreads, 1, 1);
   cfg.dynamicSmemBytes = L::kAlloc;
@@ -597,14 +647,25 @@ static int prefill_cluster_capacity(int device, int S) {
 // the narrower split saves).
 constexpr int kPrefillSSMaxTN = 128;  // token tiles up to this width read A from shared memory
 
+static int prefill_tile_tokens(int64_t M) { return M <= 64 ? 64 : (M <= 128 ? 128 : 256); }
+
+// One launch for several matrices fills the GPU when each alone would leave SMs idle or end in
+// a part-empty wave; past a few waves each matrix's own launch keeps its weights' reuse across
+// token tiles closer together in L2 (measured: W4A16 gate+up at M = 4096 4 % slower grouped).
+bool prefill_grouping_pays(int64_t M, const int64_t* N, int count) {
+  int64_t rt = 0;
+  for (int g = 0; g < count; ++g) rt += (N[g] + kQM - 1) / kQM;
+  const int TN = prefill_tile_tokens(M);
+  return rt * ((M + TN - 1) / TN) <= 4 * static_cast<int64_t>(current_device_info().num_sms);
+}
+
 template <bool kInt4>
-static cudaError_t launch_prefill(const __half* x, const void* w, const __half* sc, const uint8_t* zp,
-                                  const __half* bias, __half* y, int64_t M, int64_t N, int64_t K,
-                                  cudaStream_t s) {
+static cudaError_t launch_prefill(const __half* x, const PrefillProblem& pb, int64_t M, int64_t K, cudaStream_t s) {
   const DeviceInfo di = current_device_info();
-  const int64_t rt = (N + kQM - 1) / kQM;
+  int64_t rt = 0;
+  for (int g = 0; g < pb.count; ++g) rt += (pb.N[g] + kQM - 1) / kQM;
   const int nk = static_cast<int>(K / kQK);
-  const int TN = M <= 64 ? 64 : (M <= 128 ? 128 : 256);
+  const int TN = prefill_tile_tokens(M);
   const int64_t base = rt * ((M + TN - 1) / TN);
   auto capacity = [&](int cs) {
     if (TN == 64) return prefill_cluster_capacity<kInt4, 64, kPrefillSSMaxTN >= 64>(di.device, cs);
@@ -617,21 +678,51 @@ static cudaError_t launch_prefill(const __half* x, const void* w, const __half* 
     if (cap > 0 && base > cap) break;
     S *= 2;
   }
-  if (TN == 64) return launch_prefill_t<kInt4, 64, kPrefillSSMaxTN >= 64>(x, w, sc, zp, bias, y, M, N, K, S, s);
-  if (TN == 128) return launch_prefill_t<kInt4, 128, kPrefillSSMaxTN >= 128>(x, w, sc, zp, bias, y, M, N, K, S, s);
-  return launch_prefill_t<kInt4, 256, false>(x, w, sc, zp, bias, y, M, N, K, S, s);
+  if (TN == 64) return launch_prefill_t<kInt4, 64, kPrefillSSMaxTN >= 64>(x, pb, M, K, S, s);
+  if (TN == 128) return launch_prefill_t<kInt4, 128, kPrefillSSMaxTN >= 128>(x, pb, M, K, S, s);
+  return launch_prefill_t<kInt4, 256, false>(x, pb, M, K, S, s);
+}
+
+static PrefillProblem one_matrix(const void* w, const __half* sc, const uint8_t* zp, const __half* bias, __half* y,
+                                 int64_t N) {
+  PrefillProblem pb = {};
+  pb.count = 1;
+  pb.w[0] = w;
+  pb.sc[0] = sc;
+  pb.zp[0] = zp;
+  pb.bias[0] = bias;
+  pb.y[0] = y;
+  pb.N[0] = N;
+  return pb;
 }
 
 cudaError_t launch_tq_gemm_prefill(const __half* x, const uint8_t* packed, const __half* scale,
                                    const __half* bias, __half* y, int64_t M, int64_t N, int64_t K,
                                    cudaStream_t s) {
-  return launch_prefill<false>(x, packed, scale, nullptr, bias, y, M, N, K, s);
+  return launch_prefill<false>(x, one_matrix(packed, scale, nullptr, bias, y, N), M, K, s);
 }
 
 cudaError_t launch_w4g_gemm_prefill(const __half* x, const int32_t* qweight, const __half* scales,
                                     const uint8_t* zeros, const __half* bias, __half* y, int64_t M, int64_t N,
                                     int64_t K, cudaStream_t s) {
-  return launch_prefill<true>(x, qweight, scales, zeros, bias, y, M, N, K, s);
+  return launch_prefill<true>(x, one_matrix(qweight, scales, zeros, bias, y, N), M, K, s);
+}
+
+cudaError_t launch_gemm_prefill_grouped(bool int4, const __half* x, int count, const void* const* w,
+                                        const __half* const* sc, const __half* const* bias, __half* const* y,
+                                        const int64_t* N, int64_t M, int64_t K, cudaStream_t s) {
+  if (count < 1 || count > kQMaxGroup) return cudaErrorInvalidValue;
+  PrefillProblem pb = {};
+  pb.count = count;
+  for (int g = 0; g < count; ++g) {
+    pb.w[g] = w[g];
+    pb.sc[g] = sc[g];
+    pb.zp[g] = nullptr;
+    pb.bias[g] = bias[g];
+    pb.y[g] = y[g];
+    pb.N[g] = N[g];
+  }
+  return int4 ? launch_prefill<true>(x, pb, M, K, s) : launch_prefill<false>(x, pb, M, K, s);
 }
 
 }  // namespace tq

@@ -74,7 +74,7 @@ typedef enum { TQ_F32 = 0, TQ_F16 = 1 } tq_dtype;
 /* GEMM execution paths.  AUTO applies tq_select_path(); the others force one path (tests).
  * The decode path runs at most 16 tokens per CTA; 17 <= M <= 64 runs ceil(M/16) token chunks
  * in the same launch.  tq_select_path picks decode up to the crossover measured on Llama-3-8B /
- * Qwen2-7B shaped linears (ternary M <= 48, W4A16 M <= 16) and the tensor-core path above. */
+ * Qwen2-7B shaped linears (ternary M <= 32, W4A16 M <= 16) and the tensor-core path above. */
 typedef enum {
     TQ_PATH_AUTO = 0,
     TQ_PATH_DECODE = 1,  /* memory-bound skinny path, M <= 64: mma.sync on in-register decode  */
@@ -206,9 +206,11 @@ TQ_API int tq_permute_columns(const uint16_t* x, const int32_t* perm, uint16_t* 
  *     y_g[M, N_g] = x[M, K] . What_g[N_g, K]^T (+ bias_g)
  * Same results contract as `count` separate tq_gemm / w4g_gemm calls (each element within the
  * stated bound; the split of K over CTAs may differ, so the bits may differ).  When
- * tq_select_path picks the decode path (M up to the crossover) on shapes it takes, all
- * matrices run in ONE kernel launch (one kernel boundary
- * instead of `count`); otherwise the call issues `count` single-matrix GEMMs.
+ * tq_select_path picks the decode path (M up to the crossover) for every matrix, all matrices
+ * run in ONE decode launch; when it picks the tensor-core prefill path for every matrix and their
+ * tiles together fill at most four waves of the GPU, in ONE prefill launch whose grid covers the
+ * row tiles of all of them (one kernel boundary instead of `count`, and small matrices fill the
+ * GPU together); otherwise the call issues `count` single-matrix GEMMs.
  *   count              1 .. 4
  *   packed / qweight   HOST array of `count` device pointers (layouts as in tq_gemm / w4g_gemm)
  *   scale / scales     HOST array of `count` device pointers
