@@ -822,7 +822,8 @@ def run_reference(args, world, rank):
 # ------------------------------------------------------------------------------------------------
 PROFILE_CASES = {
     "decode": "ternary gate_proj 14336x4096 at M=1, 3 launches; q/k/v group (4096+1024+1024)x4096 at M=16, 3 launches",
-    "prefill": "ternary q_proj 4096x4096 at M=2048 (1 % outlier rows), 3 launches; W4A16 gate_proj 14336x4096 at M=512, 3 launches",
+    "prefill": "ternary q_proj 4096x4096 at M=2048 (1 % outlier rows), 3 launches; W4A16 gate+up (2x14336)x4096 "
+               "grouped at M=256, 3 launches; ternary q/k/v (4096+1024+1024)x4096 grouped at M=512, 3 launches",
     "pack": "tq_quantize_pack of an fp16 Qwen2-7B gate_up 37888x3584 (2 launches) and an fp32 4096x4096 (2 launches); w4g_quantize_pack of the latter (2 launches)",
     "prefill_mid": "ternary Qwen2-7B down 3584x18944 at M=128, 3 launches; gate_up 37888x3584 at M=32, 3 launches",
     "batch": "tq_gemm_batch over one Llama-3-8B layer's 7 ternary linears (54.5 MB packed) at M=1, 3 launches; "
@@ -856,12 +857,22 @@ def run_profile_case(name):
         x = I.activations(2048, 4096, 2, device="cuda", outlier_row_frac=0.01)
         for _ in range(3):
             tq.tq_gemm(x, p, s)
-        w = I.weights(14336, 4096, 5, device="cuda")
-        q, sc = tq.w4g_quantize_pack(w)
-        del w
-        x = I.activations(512, 4096, 6, device="cuda")
+        gu = []
+        for i in range(2):
+            w = I.weights(14336, 4096, 5 + i, device="cuda")
+            gu.append(tq.w4g_quantize_pack(w))
+            del w
+        x = I.activations(256, 4096, 6, device="cuda")
         for _ in range(3):
-            tq.w4g_gemm(x, q, sc)
+            tq.w4g_gemm_grouped(x, [q for q, _ in gu], [sc for _, sc in gu])
+        qkv = []
+        for i, N in enumerate((4096, 1024, 1024)):
+            w = I.weights(N, 4096, 8 + i, device="cuda")
+            qkv.append(tq.tq_quantize_pack(w))
+            del w
+        x = I.activations(512, 4096, 9, device="cuda", outlier_row_frac=0.01)
+        for _ in range(3):
+            tq.tq_gemm_grouped(x, [p for p, _ in qkv], [sc for _, sc in qkv])
     elif name == "prefill_mid":
         w = I.weights(3584, 18944, 1, device="cuda")
         p, s = tq.tq_quantize_pack(w)
