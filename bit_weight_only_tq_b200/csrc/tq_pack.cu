@@ -18,6 +18,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
+
 #include "tq_common.cuh"
 
 namespace tq {
@@ -283,8 +285,170 @@ __device__ __forceinline__ double warp_units_total(long long u) {
   return __ll2double_rn(h) * 256.0 + __ll2double_rn(l) * 0x1p-24;
 }
 
-// kFast: the row sums use FastAcc (fp32, FMA pipe) with an fp64 recomputation of a row whose
-// values leave its range; rows need fewer than 2^13 elements per lane (K < 2^18).
+// Relative error bound of a row sum made of fp32 accumulators that each add at most n
+// nonnegative terms in order, starting from zero (at most gamma(n) = n u / (1 - n u), u = 2^-24),
+// then combined in fp64; the factor and the 2^-45 cover the fp64 roundings of the sum, of the
+// value derived from it and of the bounds computed from that value.
+__device__ __forceinline__ double fp32_sum_rel_bound(int64_t n) {
+  const double nu = static_cast<double>(n) * 0x1p-24;
+  return 1.02 * (nu / (1.0 - nu)) + 0x1p-45;
+}
+
+// kFast: both row sums are plain fp32 sums (eight accumulators per lane) whose error bound
+// decides whether they can be used: the threshold's fp16 bucket and the fp16 scale are taken
+// from them only when every value within the bound gives the same bucket / the same fp16 (both
+// maps are monotone), which then equals the result from the exact sums; otherwise the row's sum
+// is recomputed exactly (FastAcc, fp32 on the FMA pipe, with an fp64 recomputation when its
+// values leave its range).  Rows need fewer than 2^13 elements per lane (K < 2^18).
+// One warp packs one row: ld(j) returns its 16-byte chunk j (8 elements), prow receives the
+// packed bytes; returns the row's fp16 scale (every lane).
+template <bool kFast, typename Ld>
+__device__ __forceinline__ uint16_t pack_f16_row(Ld ld, uint16_t* prow, int64_t C, int64_t K, double rel, int lane) {
+  // exact sum of |w| over the row, fp64 (the fallback, and the path without kFast)
+  auto slow_sum = [&]() {
+    UnitsAcc acc;
+    int cnt = 0;
+#pragma unroll 2
+    for (int64_t j = lane; j < C; j += 32) {
+      const uint4 v = ld(j);
+      acc.part += ((f16_mag_f64(v.x) + f16_mag_f64(v.x >> 16)) + (f16_mag_f64(v.y) + f16_mag_f64(v.y >> 16))) +
+                  ((f16_mag_f64(v.z) + f16_mag_f64(v.z >> 16)) + (f16_mag_f64(v.w) + f16_mag_f64(v.w >> 16)));
+      if (++cnt == 1024) {  // 8192 elements < 2^13: the partial stays below 2^29
+        acc.flush();
+        cnt = 0;
+      }
+    }
+    return acc.warp_total();
+  };
+  auto exact_sum = [&]() {
+    if (!kFast) return slow_sum();
+    FastAcc fa;
+#pragma unroll 2
+    for (int64_t j = lane; j < C; j += 32) {
+      const uint4 v = ld(j);
+      fa.add_pair(v.x & 0x7FFF7FFFu);
+      fa.add_pair(v.y & 0x7FFF7FFFu);
+      fa.add_pair(v.z & 0x7FFF7FFFu);
+      fa.add_pair(v.w & 0x7FFF7FFFu);
+    }
+    return __all_sync(0xFFFFFFFFu, fa.valid()) ? warp_units_total(fa.units()) : slow_sum();
+  };
+  uint32_t tb;
+  bool Sh_finite = false;
+  if (kFast) {
+    float sa[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll 2
+    for (int64_t j = lane; j < C; j += 32) {
+      const uint4 v = ld(j);
+      const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t m = wd[i] & 0x7FFF7FFFu;
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&m));
+        sa[2 * i] += f.x;
+        sa[2 * i + 1] += f.y;
+      }
+    }
+    const double Sh = warp_sum(((static_cast<double>(sa[0]) + sa[1]) + (static_cast<double>(sa[2]) + sa[3])) +
+                                   ((static_cast<double>(sa[4]) + sa[5]) + (static_cast<double>(sa[6]) + sa[7])));
+    const double th = 0.7 * (Sh / static_cast<double>(K));
+    const uint32_t lo = magnitude_floor_bits<true>(th * (1.0 - rel));
+    const uint32_t hi = magnitude_floor_bits<true>(th * (1.0 + rel));
+    Sh_finite = Sh < INFINITY;
+    if (Sh_finite && lo == hi) {
+      tb = lo;
+    } else {
+      const double S = exact_sum();
+      tb = magnitude_floor_bits<true>(0.7 * (S / static_cast<double>(K)));
+    }
+  } else {
+    const double S = slow_sum();
+    tb = magnitude_floor_bits<true>(0.7 * (S / static_cast<double>(K)));
+  }
+  const uint32_t tb2 = (tb | (tb << 16)) | 0x80008000u;
+  // exact sum of the nonzero magnitudes, fp64
+  auto slow_nonzero_sum = [&]() {
+    UnitsAcc acc;
+    int cnt = 0;
+    for (int64_t j = lane; j < C; j += 32) {
+      const uint4 v = ld(j);
+      const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+      double a2 = 0.0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t D = tb2 - (wd[i] & 0x7FFF7FFFu);
+        if (!(D & 0x8000u)) a2 += f16_mag_f64(wd[i]);
+        if (!(D & 0x80000000u)) a2 += f16_mag_f64(wd[i] >> 16);
+      }
+      acc.part += a2;
+      if (++cnt == 1024) {
+        acc.flush();
+        cnt = 0;
+      }
+    }
+    return acc.warp_total();
+  };
+  // the fp32 sum of the nonzero magnitudes needs a finite row (the fp16 compare below then agrees
+  // with the integer one); otherwise the exact path sums them
+  const bool fin = kFast && Sh_finite;
+  const uint32_t tbh2 = tb | (tb << 16);  // the threshold's fp16 pattern, both halves
+  float sa[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+  int zeros = 0;  // fewer than 2^18 elements per lane
+  int elems = 0;
+#pragma unroll 2
+  for (int64_t j = lane; j < C; j += 32) {
+    const uint4 v = ld(j);
+    const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+    uint32_t dz[4], np[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      // per 16-bit half: bit 15 of D is set iff |h| <= t (0x8000 + tb - |h| never borrows
+      // across halves): code 01; bit 15 of ~(D | h) is set iff |h| > t and h >= 0: code 10
+      const uint32_t m = wd[i] & 0x7FFF7FFFu;
+      dz[i] = tb2 - m;
+      np[i] = ~(dz[i] | wd[i]);
+      if (fin) {  // the magnitudes of the nonzero codes (m > t as fp16; a zero code's half is 0)
+        const __half2 mh = *reinterpret_cast<const __half2*>(&m);
+        const __half2 keep = __hmul2(mh, __hgt2(mh, *reinterpret_cast<const __half2*>(&tbh2)));
+        const float2 f = __half22float2(keep);
+        sa[2 * i] += f.x;
+        sa[2 * i + 1] += f.y;
+      }
+    }
+    // bytes 1 and 3 of each word carry its two elements' flags in bit 7: one byte permute puts
+    // the flags of elements 4q .. 4q + 3 in bit 7 of bytes 0 .. 3; a multiply by
+    // 2^24 + 2^18 + 2^12 + 2^6 moves the flag of byte e (bit 8e) to bit 24 + 2e (2G: 25 + 2e),
+    // and its other partial products fall on distinct bits below 24 (no carries)
+    constexpr uint32_t G = 0x01041040u;
+    const uint32_t z0 = (__byte_perm(dz[0], dz[1], 0x7531) >> 7) & 0x01010101u;
+    const uint32_t z1 = (__byte_perm(dz[2], dz[3], 0x7531) >> 7) & 0x01010101u;
+    const uint32_t p0 = (__byte_perm(np[0], np[1], 0x7531) >> 7) & 0x01010101u;
+    const uint32_t p1 = (__byte_perm(np[2], np[3], 0x7531) >> 7) & 0x01010101u;
+    const uint32_t lo = z0 * G + p0 * (2u * G), hi = z1 * G + p1 * (2u * G);
+    const uint32_t out = (lo >> 24) | ((hi >> 24) << 8);  // element e: code at bits 2e, 2e + 1
+    zeros += __popc(out & 0x5555u);                        // code 01
+    elems += 8;
+    prow[j] = static_cast<uint16_t>(out);
+  }
+  const int64_t nzt = warp_sum(static_cast<int64_t>(elems - zeros));
+  uint16_t sc = 0;
+  if (nzt > 0) {
+    bool done = false;
+    if (fin) {
+      const double Ah = warp_sum(((static_cast<double>(sa[0]) + sa[1]) + (static_cast<double>(sa[2]) + sa[3])) +
+                                     ((static_cast<double>(sa[4]) + sa[5]) + (static_cast<double>(sa[6]) + sa[7])));
+      const uint16_t lo = f64_to_f16_rne(Ah * (1.0 - rel) / static_cast<double>(nzt));
+      const uint16_t hi = f64_to_f16_rne(Ah * (1.0 + rel) / static_cast<double>(nzt));
+      if (Ah < INFINITY && lo == hi) {
+        sc = lo;
+        done = true;
+      }
+    }
+    if (!done) sc = f64_to_f16_rne(slow_nonzero_sum() / static_cast<double>(nzt));
+  }
+  return sc;
+}
+
 template <bool kFast>
 __global__ void __launch_bounds__(kPackThreads)
     tq_pack_f16_kernel(const uint16_t* __restrict__ w, uint8_t* __restrict__ packed,
@@ -293,110 +457,249 @@ __global__ void __launch_bounds__(kPackThreads)
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int64_t C = K >> 3;  // 16-byte chunks (8 elements) per row
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
+  const double rel = fp32_sum_rel_bound((C + 31) / 32);  // terms per fp32 accumulator, at most
   for (int64_t n = static_cast<int64_t>(blockIdx.x) * kWarps + wid; n < N; n += nwarps) {
     const uint4* row = reinterpret_cast<const uint4*>(w + n * K);
-    // exact sum of |w| over the row, fp64 (the fallback, and the path without kFast)
-    auto slow_sum = [&]() {
-      UnitsAcc acc;
-      int cnt = 0;
-#pragma unroll 2
-      for (int64_t j = lane; j < C; j += 32) {
-        const uint4 v = __ldg(row + j);
-        acc.part += ((f16_mag_f64(v.x) + f16_mag_f64(v.x >> 16)) + (f16_mag_f64(v.y) + f16_mag_f64(v.y >> 16))) +
-                    ((f16_mag_f64(v.z) + f16_mag_f64(v.z >> 16)) + (f16_mag_f64(v.w) + f16_mag_f64(v.w >> 16)));
-        if (++cnt == 1024) {  // 8192 elements < 2^13: the partial stays below 2^29
-          acc.flush();
-          cnt = 0;
-        }
+    const uint16_t sc = pack_f16_row<kFast>([&](int64_t j) { return __ldg(row + j); },
+                                            reinterpret_cast<uint16_t*>(packed + n * (K >> 2)), C, K, rel, lane);
+    if (lane == 0) scale[n] = sc;
+  }
+}
+
+// Rows that fit in shared memory: each warp of the CTA brings its row in with one bulk copy
+// (global -> shared, completion counted on the warp's mbarrier) and every pass reads it from
+// there, so each element crosses HBM once and the warps hold whole rows in flight.
+__global__ void __launch_bounds__(kPackThreads)
+    tq_pack_f16_smem_kernel(const uint16_t* __restrict__ w, uint8_t* __restrict__ packed,
+                            uint16_t* __restrict__ scale, int64_t N, int64_t K) {
+  extern __shared__ __align__(16) uint8_t pk_smem[];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, W = static_cast<int>(blockDim.x >> 5);
+  const int64_t C = K >> 3;
+  const uint4* buf = reinterpret_cast<const uint4*>(pk_smem) + wid * C;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(pk_smem + static_cast<int64_t>(W) * C * 16) + wid;
+  if (lane == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  const double rel = fp32_sum_rel_bound((C + 31) / 32);
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * W;
+  uint32_t phase = 0;
+  for (int64_t n = static_cast<int64_t>(blockIdx.x) * W + wid; n < N; n += nwarps, phase ^= 1u) {
+    if (lane == 0) {
+      fence_proxy_async_smem();  // the warp's reads of the previous row before the copy's writes
+      mbar_arrive_expect_tx(bar, static_cast<uint32_t>(K * 2));
+      bulk_load_1d(const_cast<uint4*>(buf), w + n * K, static_cast<uint32_t>(K * 2), bar);
+    }
+    if (!mbar_wait(bar, phase)) {  // timeout (recorded): give the copy one more bounded wait
+      mbar_wait(bar, phase);
+      return;
+    }
+    const uint16_t sc = pack_f16_row<true>([&](int64_t j) { return buf[j]; },
+                                           reinterpret_cast<uint16_t*>(packed + n * (K >> 2)), C, K, rel, lane);
+    if (lane == 0) scale[n] = sc;
+    __syncwarp();
+  }
+}
+
+// Long rows (more than fit four per 55 KB): the kPackThreads threads of a CTA pack one row
+// together, double-buffered in shared memory (the next row's bulk copy runs under this row's
+// work).  Thread t takes the 16-byte chunks t, t + kPackThreads, ...; the row sums are reduced
+// over the CTA in a fixed order, and the exact fallbacks reduce integer parts (exact).
+struct PackCtaRed {
+  double d[kPackThreads / 32];
+  long long h[kPackThreads / 32], l[kPackThreads / 32];
+};
+
+// every thread of the block calls these; every thread gets the result
+__device__ __forceinline__ double cta_sum_f64(double v, PackCtaRed* red) {
+  v = warp_sum(v);
+  __syncthreads();  // the previous reduction's reads are done
+  if ((threadIdx.x & 31) == 0) red->d[threadIdx.x >> 5] = v;
+  __syncthreads();
+  double t = 0.0;
+#pragma unroll
+  for (int i = 0; i < kPackThreads / 32; ++i) t += red->d[i];
+  return t;
+}
+
+// Exact total of per-thread parts h (units of 2^8) and l (units of 2^-24), correctly rounded once.
+__device__ __forceinline__ double cta_units_total(long long h, long long l, PackCtaRed* red) {
+  h = warp_sum(h);
+  l = warp_sum(l);
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) {
+    red->h[threadIdx.x >> 5] = h;
+    red->l[threadIdx.x >> 5] = l;
+  }
+  __syncthreads();
+  long long H = 0, L = 0;
+#pragma unroll
+  for (int i = 0; i < kPackThreads / 32; ++i) {
+    H += red->h[i];
+    L += red->l[i];
+  }
+  return __ll2double_rn(H) * 256.0 + __ll2double_rn(L) * 0x1p-24;  // two exact terms, one rounding
+}
+
+__global__ void __launch_bounds__(kPackThreads)
+    tq_pack_f16_row_cta_kernel(const uint16_t* __restrict__ w, uint8_t* __restrict__ packed,
+                               uint16_t* __restrict__ scale, int64_t N, int64_t K) {
+  extern __shared__ __align__(16) uint8_t pk_smem[];
+  const int tid = threadIdx.x;
+  const int64_t C = K >> 3;
+  const uint4* bufs = reinterpret_cast<const uint4*>(pk_smem);  // [2][C]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(pk_smem + 2 * C * 16);
+  PackCtaRed* red = reinterpret_cast<PackCtaRed*>(bar + 2);
+  const uint32_t bytes = static_cast<uint32_t>(K * 2);
+  if (tid == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  auto issue = [&](int64_t row, int b) {
+    mbar_arrive_expect_tx(&bar[b], bytes);
+    bulk_load_1d(const_cast<uint4*>(bufs + b * C), w + row * K, bytes, &bar[b]);
+  };
+  const int64_t G = gridDim.x;
+  int64_t n = blockIdx.x;
+  if (tid == 0 && n < N) issue(n, 0);
+  const int64_t n_thr = (C + kPackThreads - 1) / kPackThreads;  // terms per fp32 accumulator
+  const double rel = fp32_sum_rel_bound(n_thr);
+  for (int it = 0; n < N; n += G, ++it) {
+    const int b = it & 1;
+    if (tid == 0) {
+      if (n + G < N) {
+        fence_proxy_async_smem();  // buffer b ^ 1 was last read two rows ago (a barrier since)
+        issue(n + G, b ^ 1);
       }
-      return acc.warp_total();
-    };
-    double S;
-    if (kFast) {
+    }
+    // a wait that runs out (recorded) ends the CTA, the same way in every thread, after a bounded
+    // wait for the copy issued into the other buffer
+    if (!__syncthreads_and(mbar_wait(&bar[b], static_cast<uint32_t>(it >> 1) & 1u))) {
+      if (n + G < N) mbar_wait(&bar[b ^ 1], static_cast<uint32_t>((it + 1) >> 1) & 1u);
+      return;
+    }
+    const uint4* buf = bufs + b * C;
+    // ---- threshold: fp32 sums when their bound decides the fp16 bucket, else exact
+    float sa[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+    for (int64_t j = tid; j < C; j += kPackThreads) {
+      const uint4 v = buf[j];
+      const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t m = wd[i] & 0x7FFF7FFFu;
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&m));
+        sa[2 * i] += f.x;
+        sa[2 * i + 1] += f.y;
+      }
+    }
+    const double Sh = cta_sum_f64(((static_cast<double>(sa[0]) + sa[1]) + (static_cast<double>(sa[2]) + sa[3])) +
+                                      ((static_cast<double>(sa[4]) + sa[5]) + (static_cast<double>(sa[6]) + sa[7])),
+                                  red);
+    const bool fin = Sh < INFINITY;
+    const double th = 0.7 * (Sh / static_cast<double>(K));
+    uint32_t tb = magnitude_floor_bits<true>(th * (1.0 - rel));
+    if (!fin || tb != magnitude_floor_bits<true>(th * (1.0 + rel))) {
       FastAcc fa;
-#pragma unroll 2
-      for (int64_t j = lane; j < C; j += 32) {
-        const uint4 v = __ldg(row + j);
+      for (int64_t j = tid; j < C; j += kPackThreads) {
+        const uint4 v = buf[j];
         fa.add_pair(v.x & 0x7FFF7FFFu);
         fa.add_pair(v.y & 0x7FFF7FFFu);
         fa.add_pair(v.z & 0x7FFF7FFFu);
         fa.add_pair(v.w & 0x7FFF7FFFu);
       }
-      S = __all_sync(0xFFFFFFFFu, fa.valid()) ? warp_units_total(fa.units()) : slow_sum();
-    } else {
-      S = slow_sum();
+      double S;
+      if (__syncthreads_and(fa.valid())) {
+        const long long u = fa.units();
+        S = cta_units_total(u >> 32, u & 0xFFFFFFFFll, red);
+      } else {
+        UnitsAcc acc;
+        int cnt = 0;
+        for (int64_t j = tid; j < C; j += kPackThreads) {
+          const uint4 v = buf[j];
+          acc.part += ((f16_mag_f64(v.x) + f16_mag_f64(v.x >> 16)) + (f16_mag_f64(v.y) + f16_mag_f64(v.y >> 16))) +
+                      ((f16_mag_f64(v.z) + f16_mag_f64(v.z >> 16)) + (f16_mag_f64(v.w) + f16_mag_f64(v.w >> 16)));
+          if (++cnt == 1024) {
+            acc.flush();
+            cnt = 0;
+          }
+        }
+        acc.flush();
+        S = cta_units_total(acc.hi, acc.lo, red);
+      }
+      tb = magnitude_floor_bits<true>(0.7 * (S / static_cast<double>(K)));
     }
-    const double t = 0.7 * (S / static_cast<double>(K));
-    const uint32_t tb = magnitude_floor_bits<true>(t);
     const uint32_t tb2 = (tb | (tb << 16)) | 0x80008000u;
-    UnitsAcc accA;
-    FastAcc faA;
-    int nz = 0;
-    int cnt = 0;
+    const uint32_t tbh2 = tb | (tb << 16);
+    // ---- codes, zero count, fp32 sum of the nonzero magnitudes
     uint16_t* prow = reinterpret_cast<uint16_t*>(packed + n * (K >> 2));
-#pragma unroll 2
-    for (int64_t j = lane; j < C; j += 32) {
-      const uint4 v = __ldg(row + j);
+    float sb[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+    int zeros = 0, elems = 0;
+    for (int64_t j = tid; j < C; j += kPackThreads) {
+      const uint4 v = buf[j];
       const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
-      uint32_t out = 0;
-      double a = 0.0;
+      uint32_t dz[4], np[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        // per 16-bit half: bit 15 of D is set iff |h| <= t (0x8000 + tb - |h| never borrows
-        // across halves)
-        const uint32_t D = tb2 - (wd[i] & 0x7FFF7FFFu);
-        const uint32_t zero = (D >> 15) & 0x00010001u;           // code 01
-        const uint32_t pos = (~(D | wd[i]) >> 14) & 0x00020002u;  // |h| > t and h >= 0: code 10
-        const uint32_t c = zero | pos;                            // else 00
-        out |= ((c | (c >> 14)) & 0xFu) << (4 * i);
-        nz += __popc(~D & 0x80008000u);
-        if (kFast) {
-          // the magnitudes of the nonzero codes (a zero code's half is cleared)
-          const uint32_t keep = ((~D & 0x80008000u) >> 15) * 0xFFFFu;
-          faA.add_pair(wd[i] & 0x7FFF7FFFu & keep);
-        } else {
-          if (!(D & 0x8000u)) a += f16_mag_f64(wd[i]);
-          if (!(D & 0x80000000u)) a += f16_mag_f64(wd[i] >> 16);
+        const uint32_t m = wd[i] & 0x7FFF7FFFu;
+        dz[i] = tb2 - m;
+        np[i] = ~(dz[i] | wd[i]);
+        if (fin) {
+          const __half2 mh = *reinterpret_cast<const __half2*>(&m);
+          const __half2 keep = __hmul2(mh, __hgt2(mh, *reinterpret_cast<const __half2*>(&tbh2)));
+          const float2 f = __half22float2(keep);
+          sb[2 * i] += f.x;
+          sb[2 * i + 1] += f.y;
         }
       }
-      if (!kFast) {
-        accA.part += a;
-        if (++cnt == 1024) {
-          accA.flush();
-          cnt = 0;
-        }
-      }
+      constexpr uint32_t Gm = 0x01041040u;  // the flag gather of pack_f16_row
+      const uint32_t z0 = (__byte_perm(dz[0], dz[1], 0x7531) >> 7) & 0x01010101u;
+      const uint32_t z1 = (__byte_perm(dz[2], dz[3], 0x7531) >> 7) & 0x01010101u;
+      const uint32_t p0 = (__byte_perm(np[0], np[1], 0x7531) >> 7) & 0x01010101u;
+      const uint32_t p1 = (__byte_perm(np[2], np[3], 0x7531) >> 7) & 0x01010101u;
+      const uint32_t lo = z0 * Gm + p0 * (2u * Gm), hi = z1 * Gm + p1 * (2u * Gm);
+      const uint32_t out = (lo >> 24) | ((hi >> 24) << 8);
+      zeros += __popc(out & 0x5555u);
+      elems += 8;
       prow[j] = static_cast<uint16_t>(out);
     }
-    double A;
-    if (kFast && __all_sync(0xFFFFFFFFu, faA.valid())) {
-      A = warp_units_total(faA.units());
-    } else if (kFast) {  // recompute the sum of the nonzero magnitudes in fp64
-      UnitsAcc acc;
-      cnt = 0;
-      for (int64_t j = lane; j < C; j += 32) {
-        const uint4 v = __ldg(row + j);
-        const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
-        double a2 = 0.0;
+    const int64_t nzt = static_cast<int64_t>(
+        cta_sum_f64(static_cast<double>(elems - zeros), red));  // integers below 2^31: exact in fp64
+    uint16_t sc = 0;
+    if (nzt > 0) {
+      const double Ah = cta_sum_f64(((static_cast<double>(sb[0]) + sb[1]) + (static_cast<double>(sb[2]) + sb[3])) +
+                                        ((static_cast<double>(sb[4]) + sb[5]) + (static_cast<double>(sb[6]) + sb[7])),
+                                    red);
+      const uint16_t slo = f64_to_f16_rne(Ah * (1.0 - rel) / static_cast<double>(nzt));
+      if (fin && Ah < INFINITY && slo == f64_to_f16_rne(Ah * (1.0 + rel) / static_cast<double>(nzt))) {
+        sc = slo;
+      } else {
+        UnitsAcc acc;
+        int cnt = 0;
+        for (int64_t j = tid; j < C; j += kPackThreads) {
+          const uint4 v = buf[j];
+          const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+          double a2 = 0.0;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint32_t D = tb2 - (wd[i] & 0x7FFF7FFFu);
-          if (!(D & 0x8000u)) a2 += f16_mag_f64(wd[i]);
-          if (!(D & 0x80000000u)) a2 += f16_mag_f64(wd[i] >> 16);
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t D = tb2 - (wd[i] & 0x7FFF7FFFu);
+            if (!(D & 0x8000u)) a2 += f16_mag_f64(wd[i]);
+            if (!(D & 0x80000000u)) a2 += f16_mag_f64(wd[i] >> 16);
+          }
+          acc.part += a2;
+          if (++cnt == 1024) {
+            acc.flush();
+            cnt = 0;
+          }
         }
-        acc.part += a2;
-        if (++cnt == 1024) {
-          acc.flush();
-          cnt = 0;
-        }
+        acc.flush();
+        sc = f64_to_f16_rne(cta_units_total(acc.hi, acc.lo, red) / static_cast<double>(nzt));
       }
-      A = acc.warp_total();
-    } else {
-      A = accA.warp_total();
     }
-    const int nzt = warp_sum(nz);
-    if (lane == 0)
-      scale[n] = nzt > 0 ? f64_to_f16_rne(A / static_cast<double>(nzt)) : static_cast<uint16_t>(0);
+    if (tid == 0) scale[n] = sc;
+    __syncthreads();  // every thread is done with buffer b before it is refilled
   }
 }
 
@@ -572,6 +875,44 @@ cudaError_t launch_tq_pack(const void* w, bool w_f16, uint8_t* packed, uint16_t*
   const int binw = 30 - ceil_log2_i64(K);
   const uintptr_t a = reinterpret_cast<uintptr_t>(w);
   if (w_f16 && K % 8 == 0 && a % 16 == 0) {
+    // rows that fit in shared memory: one bulk copy per row, every pass from shared memory; four
+    // to eight warps per CTA, one row each, within 55 KB (four CTAs per SM); longer rows (up to
+    // 100 KB) one per CTA, double-buffered; the grid is what stays resident
+    const int64_t row_bytes = 2 * K;
+    const int W = static_cast<int>(std::min<int64_t>(8, (55 * 1024) / (row_bytes + 8)));
+    if (W < 4 && 2 * row_bytes + 1024 <= 200 * 1024) {
+      const int smem = static_cast<int>(2 * row_bytes + 16 + sizeof(PackCtaRed));
+      const void* kern = reinterpret_cast<const void*>(tq_pack_f16_row_cta_kernel);
+      cudaError_t e = ensure_smem_attr(kern, smem);
+      if (e != cudaSuccess) return e;
+      int bps = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, tq_pack_f16_row_cta_kernel, kPackThreads, smem) !=
+              cudaSuccess ||
+          bps < 1) {
+        (void)cudaGetLastError();
+        bps = 1;
+      }
+      const int64_t g = std::min<int64_t>(N, static_cast<int64_t>(di.num_sms) * bps);
+      tq_pack_f16_row_cta_kernel<<<static_cast<unsigned>(g), kPackThreads, smem, s>>>(
+          static_cast<const uint16_t*>(w), packed, scale, N, K);
+      return cudaGetLastError();
+    }
+    if (W >= 4) {
+      const int smem = static_cast<int>(W * (row_bytes + 8));
+      const void* kern = reinterpret_cast<const void*>(tq_pack_f16_smem_kernel);
+      cudaError_t e = ensure_smem_attr(kern, smem);
+      if (e != cudaSuccess) return e;
+      int bps = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, tq_pack_f16_smem_kernel, W * 32, smem) != cudaSuccess ||
+          bps < 1) {
+        (void)cudaGetLastError();
+        bps = 1;
+      }
+      const int64_t g = std::min<int64_t>((N + W - 1) / W, static_cast<int64_t>(di.num_sms) * bps);
+      tq_pack_f16_smem_kernel<<<static_cast<unsigned>(g), W * 32, smem, s>>>(static_cast<const uint16_t*>(w), packed,
+                                                                             scale, N, K);
+      return cudaGetLastError();
+    }
     // the fp32 row sums need fewer than 2^13 elements per lane
     if (K < (int64_t(1) << 18))
       tq_pack_f16_kernel<true><<<static_cast<unsigned>(grid), kPackThreads, 0, s>>>(

@@ -47,9 +47,10 @@ def test_pack_unaligned_input():
     _check_tq(I.weights(33, 4096, 6, dtype=torch.float16), offset=3)
 
 
-def test_pack_adversarial_rows():
+# K = 2048: one row per warp; K = 18944: one row per CTA (long rows); both from shared memory
+@pytest.mark.parametrize("K", [2048, 18944])
+def test_pack_adversarial_rows(K):
     g = torch.Generator().manual_seed(11)
-    K = 2048
     rows = []
     rows.append(torch.zeros(K))                                           # all zero
     rows.append(torch.full((K,), 0.02))                                   # constant
@@ -146,11 +147,11 @@ def test_pack_fp32_deep_bins_long_row():
     _check_tq(w)
 
 
-def test_pack_fp16_fast_sum_boundaries():
+@pytest.mark.parametrize("K", [2048, 7168, 18944])
+def test_pack_fp16_fast_sum_boundaries(K):
     # fp16 rows (16-byte aligned, K % 8 == 0) whose per-lane sums sit at the edges of the fast
     # fp32 accumulation (values up to 2^11, lane sums around 2^11, many subnormals), and rows
     # that must fall back to the fp64 sums; the result must match the oracle bit for bit
-    K = 2048
     g = torch.Generator().manual_seed(21)
     rows = []
     r = torch.full((K,), 2047.0)                       # every value just below 2^11: lane sums overflow
@@ -173,3 +174,44 @@ def test_pack_fp16_fast_sum_boundaries():
     rows.append(r)
     w = torch.stack(rows).to(torch.float16)
     _check_tq(w)
+
+
+def _near_decision_edges(K, n_rows, seed, rel):
+    """Rows of N(0, 0.02) fp16 weights whose threshold 0.7 mean|w| lies within 4 rel (relative)
+    of an fp16 value (where the threshold's fp16 bucket changes), or whose scale mean lies within
+    4 rel of a midpoint between fp16 values (where its rounding changes): there an approximate
+    row sum must not decide.  Found by search; the sums here are plain fp64 sums, exact for fp16
+    values with K < 2^13 (multiples of 2^-24 below 2^29)."""
+    rng = np.random.default_rng(seed)
+    w = (rng.standard_normal((n_rows, K)) * 0.02).astype(np.float16)
+    d_t, d_s = np.empty(n_rows), np.empty(n_rows)
+    for r0 in range(0, n_rows, 512):
+        a = np.abs(w[r0:r0 + 512].astype(np.float64))
+        t = 0.7 * (a.sum(axis=1) / K)
+        tv = np.float16(t).astype(np.float64)               # nearest fp16 value
+        d_t[r0:r0 + 512] = np.abs(t - tv) / t
+        keep = a > t[:, None]
+        nz = keep.sum(axis=1)
+        m = (a * keep).sum(axis=1) / np.maximum(nz, 1)
+        f = np.float16(m).astype(np.float64)
+        nxt = np.where(m >= f, np.nextafter(np.float16(m), np.float16(np.inf)).astype(np.float64),
+                       np.nextafter(np.float16(m), np.float16(0)).astype(np.float64))
+        d_s[r0:r0 + 512] = np.abs(m - (f + nxt) / 2) / m
+    return w, d_t, d_s
+
+
+# K = 3584: one row per warp (14 terms per fp32 accumulator); K = 18944: one row per CTA of 256
+# threads (10 terms)
+@pytest.mark.parametrize("K,terms,n_rows,least", [(3584, 14, 8192, 4), (18944, 10, 4096, 2)])
+def test_pack_fp16_bounded_sums_at_decision_edges(K, terms, n_rows, least):
+    # the fp16 pack takes its row sums from fp32 accumulators when their error bound cannot change
+    # the threshold's bucket or the scale's rounding, and sums exactly otherwise: rows right at
+    # (and just beyond) those edges must still match the oracle bit for bit
+    rel = 1.02 * (terms * 2.0 ** -24)                       # the kernel's bound
+    w, d_t, d_s = _near_decision_edges(K, n_rows, 5, rel)
+    near_t = np.argsort(d_t)[:32]
+    near_s = np.argsort(d_s)[:32]
+    assert (d_t[near_t] < rel).sum() >= least, "too few rows inside the threshold band"
+    assert (d_s[near_s] < rel).sum() >= least, "too few rows inside the scale band"
+    idx = np.unique(np.concatenate([near_t, near_s]))
+    _check_tq(torch.from_numpy(w[idx]))
