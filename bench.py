@@ -442,8 +442,7 @@ def run_ours(args, world, rank, local):
     traffic = load_traffic()
     roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
             "frac": round(achieved / hbm, 4), "traffic": traffic,
-            "kernel": ("batch_decode_kernel (persistent, equal stage ranges per CTA, mma.sync on exact decode)"
-                       if args.calls == "batch" else "decode_gemm_kernel (mma.sync, TMA ring, cluster split-K)"),
+            "kernel": "batch_decode_kernel" if args.calls == "batch" else "decode_gemm_kernel",
             "peak_source": f"{peak_src} hbm_gbs"}
 
     detail = {}
@@ -476,8 +475,8 @@ def run_ours(args, world, rank, local):
         "roofline": roof,
         "e2e": {"value": round(e2e_val, 1), "unit": "GB/s", "h2d_bytes_per_step": bi,
                 "d2h_bytes_per_step": bo, "ms_per_step": round(e2e_ms, 4),
-                "calls": ("graph replay; outputs copied out per 8 layers on a second stream under the next "
-                          "layers' compute" if args.calls == "batch" else "graph replay"),
+                "calls": ("graph; y of each 8 layers copied out on a 2nd stream under the next"
+                          if args.calls == "batch" else "graph replay"),
                 "eager_value": round(eager_val, 1), "eager_ms_per_step": round(eager_ms, 4)},
         "gpu_launches": launches_step * args.steps,
         "clocks": clocks,
