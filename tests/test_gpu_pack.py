@@ -36,6 +36,13 @@ def test_pack_fp16_rows():
     _check_tq(I.weights(300, 3584, I.seed_for(4, 0, 1), dtype=torch.float16))
 
 
+# fp16 rows on each pack kernel: one row per warp (K = 6912: four warps' rows in 55 KB), one row
+# per CTA (K = 7040, just past that), rows too long for shared memory (K = 65536, streamed)
+@pytest.mark.parametrize("K", [6912, 7040, 65536])
+def test_pack_fp16_kernel_boundaries(K):
+    _check_tq(I.weights(37, K, 90 + K, dtype=torch.float16, outlier_frac=0.001))
+
+
 @pytest.mark.parametrize("K", [1, 2, 3, 5, 63, 65, 1001, 4095])
 def test_pack_ragged_k(K):
     _check_tq(I.weights(17, K, 77 + K))
