@@ -52,12 +52,15 @@ constexpr int kQThreads = 128 * (1 + kQDecGroups);  // warps 0-3: TMA, MMA; then
 constexpr int kQEpiGroups = 1 + kQDecGroups;        // every group of four warps runs the epilogue
 constexpr bool kMergeStageBarriers = true;
 
-template <bool kInt4>
+// kKS: K per stage, 64 (one 128-byte swizzle row of fp16 per operand row) or 128 (two of them,
+// eight MMAs per barrier test and commit instead of four)
+template <bool kInt4, int kKS>
 struct PFmt {
-  static constexpr int kRowBytes = kInt4 ? 32 : 16;  // packed bytes per row per stage (64 k)
-  // the packed weights arrive in tiles of 128 bytes per row (8 ternary / 4 W4A16 stages),
-  // 128-byte swizzled: one DRAM burst per row instead of one 16- or 32-byte piece per stage
-  static constexpr int kSPP = 128 / kRowBytes;       // stages per packed tile
+  static constexpr int kSub = kKS / kQK;                       // 64-k sub-tiles per stage
+  static constexpr int kRowBytes = (kInt4 ? 32 : 16) * kSub;  // packed bytes per row per stage
+  // the packed weights arrive in tiles of 128 bytes per row (512 ternary / 256 W4A16 k),
+  // 128-byte swizzled: one DRAM burst per row instead of one small piece per stage
+  static constexpr int kSPP = 128 / kRowBytes;                 // stages per packed tile
   static constexpr int kTileP = kQM * 128;
   static constexpr int kPRing = 3;
   static_assert(kSPP % kQDecGroups == 0, "the decode groups alternate within a packed tile");
@@ -66,23 +69,28 @@ struct PFmt {
 // kSS: the decoded weights go to shared memory (128-byte-swizzled K-major tiles, the layout TMA
 // gives the x tile) and the MMA reads both operands from there; otherwise they go to tensor
 // memory.
-template <bool kInt4, int TN, bool kSS>
+template <bool kInt4, int TN, bool kSS, int kKS>
 struct PrefillLayout {
-  static constexpr int kTileX = TN * kQK * 2;  // x tile of one stage
-  static constexpr int kTileA = kQM * kQK * 2;  // decoded-weight tile of one stage (kSS)
+  static_assert(kSS || kKS == kQK, "tensor-memory A slots hold 64 k");
+  static constexpr int kSub = kKS / kQK;
+  static constexpr int kTileXs = TN * kQK * 2;   // x sub-tile: TN rows x 128 bytes
+  static constexpr int kTileAs = kQM * kQK * 2;  // decoded-weight sub-tile (kSS): 128 rows x 128 bytes
+  static constexpr int kTileX = kSub * kTileXs;  // x tile of one stage
+  static constexpr int kTileA = kSub * kTileAs;  // decoded-weight tile of one stage (kSS)
   // ring depths: narrow tiles move little data per stage, so they keep more stages in flight
-  static constexpr int kRing = kSS ? (TN == 64 ? 6 : 4) : (TN == 256 ? 4 : (TN == 128 ? 6 : 10));
-  static constexpr int kARing = kSS ? (TN == 64 ? 6 : 4) : (TN == 256 ? 4 : kQMaxARing);
+  static constexpr int kRing = kSS ? (kSub == 2 ? (TN == 64 ? 3 : 2) : (TN == 64 ? 6 : 4))
+                                   : (TN == 256 ? 4 : (TN == 128 ? 6 : 10));
+  static constexpr int kARing = kSS ? kRing : (TN == 256 ? 4 : kQMaxARing);
   // equal rings: one barrier per stage for "x tile landed and weights decoded" and one for
   // "stage consumed", so the MMA thread tests one barrier and commits once per stage
   static constexpr bool kMergedBars = kMergeStageBarriers && kRing == kARing;
   static constexpr int kOffX = 0;
   static constexpr int kOffP = kOffX + kRing * kTileX;
-  static constexpr int kOffA = kOffP + PFmt<kInt4>::kPRing * PFmt<kInt4>::kTileP;
+  static constexpr int kOffA = kOffP + PFmt<kInt4, kKS>::kPRing * PFmt<kInt4, kKS>::kTileP;
   static constexpr int kOffBar = kOffA + (kSS ? kARing * kTileA : 0);
   // barriers: fullX[R], emptyX[R], fullP[RP], emptyP[RP], afull[RA], aempty[RA], accFull; then
   // the TMEM slot
-  static constexpr int kNumBars = 2 * kRing + 2 * PFmt<kInt4>::kPRing + 2 * kARing + 1;
+  static constexpr int kNumBars = 2 * kRing + 2 * PFmt<kInt4, kKS>::kPRing + 2 * kARing + 1;
   static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffTmemSlot + 16;
   // alignment slack; at least 116 KB so that one CTA runs per SM: a CTA never waits in
@@ -91,7 +99,7 @@ struct PrefillLayout {
   static constexpr int kAlloc = kBytes + 1024 > 116 * 1024 ? kBytes + 1024 : 116 * 1024;
   // split-K partials [S][TN / S / 4][128 rows][4] fp32 reuse the x and packed rings after the
   // main loop
-  static_assert(kQM * (TN + 8) * 4 <= kRing * kTileX + PFmt<kInt4>::kPRing * PFmt<kInt4>::kTileP,
+  static_assert(kQM * (TN + 8) * 4 <= kRing * kTileX + PFmt<kInt4, kKS>::kPRing * PFmt<kInt4, kKS>::kTileP,
                 "split-K partials fit");
   // tensor memory: accumulator columns [0, TN), decoded-weight slots after it (not kSS)
   static constexpr uint32_t kColA = TN;
@@ -167,12 +175,12 @@ __device__ __forceinline__ uint4 decode_w4_8(uint32_t w, uint32_t s2, uint32_t z
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-template <bool kInt4, int TN, bool kSS>
+template <bool kInt4, int TN, bool kSS, int kKS>
 __global__ void __launch_bounds__(kQThreads, 1)
     prefill_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
                         const __grid_constant__ PrefillWeightMaps tmaps_w, const PrefillArgs a) {
-  using L = PrefillLayout<kInt4, TN, kSS>;
-  using F = PFmt<kInt4>;
+  using L = PrefillLayout<kInt4, TN, kSS, kKS>;
+  using F = PFmt<kInt4, kKS>;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned; pointer arithmetic on the __shared__ array keeps the shared address
   // space visible to the compiler (plain ld/st.shared instead of generic accesses)
@@ -200,7 +208,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
   __half* const gy = a.y[g];
   const CUtensorMap* const tmap_w = &tmaps_w.m[g];
   const int64_t m0 = static_cast<int64_t>(blockIdx.y) * TN;   // first token
-  const int nk_all = static_cast<int>(a.K / kQK);
+  const int nk_all = static_cast<int>((a.K + kKS - 1) / kKS);  // a last half stage reads zeros
   const int rank = static_cast<int>(blockIdx.z);              // K-slice = rank in the cluster
   const int kb0 = static_cast<int>((static_cast<int64_t>(rank) * nk_all) / a.S);
   const int nk = static_cast<int>((static_cast<int64_t>(rank + 1) * nk_all) / a.S) - kb0;  // >= 1
@@ -247,7 +255,10 @@ __global__ void __launch_bounds__(kQThreads, 1)
           if (!ok) break;
         }
         mbar_arrive_expect_tx(&full[s], L::kTileX);
-        tma_load_2d(sm + L::kOffX + s * L::kTileX, &tmap_x, &full[s], (kb0 + kb) * kQK, static_cast<int32_t>(m0));
+#pragma unroll
+        for (int q = 0; q < L::kSub; ++q)
+          tma_load_2d(sm + L::kOffX + s * L::kTileX + q * L::kTileXs, &tmap_x, &full[s], (kb0 + kb) * kKS + q * kQK,
+                      static_cast<int32_t>(m0));
       }
     }
   } else if (warp == 2) {
@@ -280,17 +291,21 @@ __global__ void __launch_bounds__(kQThreads, 1)
              (L::kMergedBars || mbar_wait(&afull[as], static_cast<uint32_t>(kb / L::kARing) & 1u));
         if (!ok) break;
         tc_fence_after_sync();
-        const uint64_t bdesc = sdesc_kmajor_sw128(x_base + s * L::kTileX);
         const uint32_t a_tmem = tmem + L::kColA + 32 * as;
-        const uint64_t adesc = sdesc_kmajor_sw128(a_base + as * L::kTileA);
 #pragma unroll
-        for (int k16 = 0; k16 < kQK / 16; ++k16) {
-          // A in tensor memory: 8 columns (16 fp16) per K=16 step; in shared memory (and B):
-          // +32 bytes along K = +2 in the descriptor
-          if (kSS)
-            umma_f16(tmem, adesc + 2 * k16, bdesc + 2 * k16, idesc, (kb | k16) != 0 ? 1u : 0u);
-          else
-            umma_f16_ts(tmem, a_tmem + 8 * k16, bdesc + 2 * k16, idesc, (kb | k16) != 0 ? 1u : 0u);
+        for (int q = 0; q < L::kSub; ++q) {
+          const uint64_t bdesc = sdesc_kmajor_sw128(x_base + s * L::kTileX + q * L::kTileXs);
+          const uint64_t adesc = sdesc_kmajor_sw128(a_base + as * L::kTileA + q * L::kTileAs);
+#pragma unroll
+          for (int k16 = 0; k16 < kQK / 16; ++k16) {
+            // A in tensor memory: 8 columns (16 fp16) per K=16 step; in shared memory (and B):
+            // +32 bytes along K = +2 in the descriptor
+            const uint32_t accum = (kb | q | k16) != 0 ? 1u : 0u;
+            if (kSS)
+              umma_f16(tmem, adesc + 2 * k16, bdesc + 2 * k16, idesc, accum);
+            else
+              umma_f16_ts(tmem, a_tmem + 8 * k16, bdesc + 2 * k16, idesc, accum);
+          }
         }
         umma_commit(&emptyX[s]);
         if (!L::kMergedBars) umma_commit(&aempty[as]);
@@ -313,7 +328,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
     auto group_zero = [&](int64_t gi) -> uint32_t {
       return (gzp && n < Ng && gi < G) ? static_cast<uint32_t>(gzp[n * G + gi]) : 8u;
     };
-    int64_t g_cur = -1;
+    int64_t g_cur = -1, g_nxt = -1;
     uint16_t sc_cur = 0, sc_nxt = 0;
     uint32_t zp_cur = 8u, zp_nxt = 8u;
     for (int kb = dg; kb < nk && ok; kb += kQDecGroups) {
@@ -322,13 +337,14 @@ __global__ void __launch_bounds__(kQThreads, 1)
         ok = mbar_wait(&fullP[ps], static_cast<uint32_t>(pt / F::kPRing) & 1u);
         if (!ok) break;
       }
-      // this stage's 16 (ternary) or 32 (W4A16) bytes of row r: 16-byte chunk(s) of the
+      // this stage's 16 (ternary) or 32 (W4A16) bytes per 64 k of row r: 16-byte chunks of the
       // 128-byte swizzled row (chunk c at position c ^ (r & 7): conflict free)
+      constexpr int kCh = (kInt4 ? 2 : 1) * L::kSub;  // chunks per stage
       const uint8_t* prow = sm + L::kOffP + ps * F::kTileP + r * 128;
-      const int c0 = kInt4 ? 2 * ci : ci;
-      const uint4 p0 = *reinterpret_cast<const uint4*>(prow + ((c0 ^ (r & 7)) << 4));
-      uint4 p1 = make_uint4(0u, 0u, 0u, 0u);
-      if (kInt4) p1 = *reinterpret_cast<const uint4*>(prow + (((c0 + 1) ^ (r & 7)) << 4));
+      uint4 pc[kCh];
+#pragma unroll
+      for (int c = 0; c < kCh; ++c)
+        pc[c] = *reinterpret_cast<const uint4*>(prow + (((kCh * ci + c) ^ (r & 7)) << 4));
       // done with this packed tile: both groups arrive on every tile but a CTA's last, which
       // no later load waits for
       if (ci + kQDecGroups >= F::kSPP || kb + kQDecGroups >= nk) {
@@ -337,18 +353,32 @@ __global__ void __launch_bounds__(kQThreads, 1)
       }
       uint32_t s2 = 0u;
       if (kInt4) {
-        const int64_t gi = (kb0 + kb) >> 1;  // 128-wide group of this 64-wide stage
+        const int64_t gi = (static_cast<int64_t>(kb0 + kb) * kKS) >> 7;  // 128-wide group of this stage
         if (gi != g_cur) {
-          sc_cur = g_cur < 0 ? group_scale(gi) : sc_nxt;
-          zp_cur = g_cur < 0 ? group_zero(gi) : zp_nxt;
-          sc_nxt = group_scale(gi + 1);
-          zp_nxt = group_zero(gi + 1);
+          sc_cur = gi == g_nxt ? sc_nxt : group_scale(gi);
+          zp_cur = gi == g_nxt ? zp_nxt : group_zero(gi);
+          // the group of this decode group's next stage (kQDecGroups stages on)
+          g_nxt = (static_cast<int64_t>(kb0 + kb + kQDecGroups) * kKS) >> 7;
+          sc_nxt = group_scale(g_nxt);
+          zp_nxt = group_zero(g_nxt);
           g_cur = gi;
         }
         s2 = static_cast<uint32_t>(sc_cur) | (static_cast<uint32_t>(sc_cur) << 16);
       }
       const uint32_t zsub = w4_zero_pair(zp_cur);
-      const uint32_t pw[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+      // the packed words of 64-k sub-tile q
+      auto words = [&](int q, uint32_t (&pw)[8]) {
+        const uint4 u0 = pc[(kInt4 ? 2 : 1) * q];
+        const uint4 u1 = kInt4 ? pc[2 * q + 1] : make_uint4(0u, 0u, 0u, 0u);
+        pw[0] = u0.x;
+        pw[1] = u0.y;
+        pw[2] = u0.z;
+        pw[3] = u0.w;
+        pw[4] = u1.x;
+        pw[5] = u1.y;
+        pw[6] = u1.z;
+        pw[7] = u1.w;
+      };
       if (kSS) {
         if (kb >= L::kARing) {
           ok = mbar_wait(&aempty[as], static_cast<uint32_t>((kb / L::kARing) - 1) & 1u);
@@ -356,14 +386,21 @@ __global__ void __launch_bounds__(kQThreads, 1)
         }
         // 16-byte chunk j (k = 8j .. 8j + 7) of row r at chunk position j ^ (r & 7) of the
         // 128-byte row: the 128-byte swizzle; eight consecutive rows fill all 32 banks
-        uint8_t* arow = sm + L::kOffA + as * L::kTileA + r * 128;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint4 d = kInt4 ? decode_w4_8(pw[j], s2, zsub) : decode_tq_8(pw[j >> 1], j & 1);
-          *reinterpret_cast<uint4*>(arow + ((j ^ (r & 7)) << 4)) = d;
+        for (int q = 0; q < L::kSub; ++q) {
+          uint32_t pw[8];
+          words(q, pw);
+          uint8_t* arow = sm + L::kOffA + as * L::kTileA + q * L::kTileAs + r * 128;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint4 d = kInt4 ? decode_w4_8(pw[j], s2, zsub) : decode_tq_8(pw[j >> 1], j & 1);
+            *reinterpret_cast<uint4*>(arow + ((j ^ (r & 7)) << 4)) = d;
+          }
         }
         fence_proxy_async_smem();  // visible to the tensor core's operand reads
       } else {
+        uint32_t pw[8];
+        words(0, pw);
         uint32_t v[32];  // column j = fp16 pair (k = 2j, 2j + 1) of this row
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -547,10 +584,10 @@ struct PrefillProblem {
   int64_t N[kQMaxGroup];
 };
 
-template <bool kInt4, int TN, bool kSS>
+template <bool kInt4, int TN, bool kSS, int kKS>
 static cudaError_t launch_prefill_t(const __half* x, const PrefillProblem& pb, int64_t M, int64_t K, int S,
                                     cudaStream_t s) {
-  using L = PrefillLayout<kInt4, TN, kSS>;
+  using L = PrefillLayout<kInt4, TN, kSS, kKS>;
   CUtensorMap tx;
   PrefillWeightMaps tw;
   if (!make_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, static_cast<uint64_t>(K),
@@ -577,7 +614,7 @@ static cudaError_t launch_prefill_t(const __half* x, const PrefillProblem& pb, i
       a.tile0[g + 1] = a.tile0[g];
     }
   }
-  auto* kern = prefill_gemm_kernel<kInt4, TN, kSS>;
+  auto* kern = prefill_gemm_kernel<kInt4, TN, kSS, kKS>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), L::kAlloc);
   if (e != cudaSuccess) return e;
   a.M = M;
@@ -609,15 +646,15 @@ static cudaError_t launch_prefill_t(const __half* x, const PrefillProblem& pb, i
 // GPC, so the GPCs bound it below SMs / S), queried once per device and S; 0 when unknown.
 constexpr int kPfMaxDevices = 64;
 
-template <bool kInt4, int TN, bool kSS>
+template <bool kInt4, int TN, bool kSS, int kKS>
 static int prefill_cluster_capacity(int device, int S) {
-  using L = PrefillLayout<kInt4, TN, kSS>;
+  using L = PrefillLayout<kInt4, TN, kSS, kKS>;
   static std::atomic<int> cache[kPfMaxDevices][4];
   if (device < 0 || device >= kPfMaxDevices || S < 2 || S > 8) return 0;
   const int li = S == 2 ? 1 : (S == 4 ? 2 : 3);
   int n = cache[device][li].load(std::memory_order_relaxed);
   if (n > 0) return n;
-  auto* kern = prefill_gemm_kernel<kInt4, TN, kSS>;
+  auto* kern = prefill_gemm_kernel<kInt4, TN, kSS, kKS>;
   if (ensure_smem_attr(reinterpret_cast<const void*>(kern), L::kAlloc) != cudaSuccess) return 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(1, 1, static_cast<unsigned>(S));
@@ -646,6 +683,7 @@ static int prefill_cluster_capacity(int device, int S) {
 // idle and all the clusters fit on the GPU at once (a second wave of clusters costs more than
 // the narrower split saves).
 constexpr int kPrefillSSMaxTN = 128;  // token tiles up to this width read A from shared memory
+constexpr int kPrefillSSStageK = 128;  // and take 128 k per stage (eight MMAs per barrier test)
 
 static int prefill_tile_tokens(int64_t M) { return M <= 64 ? 64 : (M <= 128 ? 128 : 256); }
 
@@ -664,13 +702,14 @@ static cudaError_t launch_prefill(const __half* x, const PrefillProblem& pb, int
   const DeviceInfo di = current_device_info();
   int64_t rt = 0;
   for (int g = 0; g < pb.count; ++g) rt += (pb.N[g] + kQM - 1) / kQM;
-  const int nk = static_cast<int>(K / kQK);
   const int TN = prefill_tile_tokens(M);
+  const int KS = TN <= kPrefillSSMaxTN ? kPrefillSSStageK : kQK;
+  const int nk = static_cast<int>((K + KS - 1) / KS);
   const int64_t base = rt * ((M + TN - 1) / TN);
   auto capacity = [&](int cs) {
-    if (TN == 64) return prefill_cluster_capacity<kInt4, 64, kPrefillSSMaxTN >= 64>(di.device, cs);
-    if (TN == 128) return prefill_cluster_capacity<kInt4, 128, kPrefillSSMaxTN >= 128>(di.device, cs);
-    return prefill_cluster_capacity<kInt4, 256, false>(di.device, cs);
+    if (TN == 64) return prefill_cluster_capacity<kInt4, 64, true, kPrefillSSStageK>(di.device, cs);
+    if (TN == 128) return prefill_cluster_capacity<kInt4, 128, true, kPrefillSSStageK>(di.device, cs);
+    return prefill_cluster_capacity<kInt4, 256, false, kQK>(di.device, cs);
   };
   int S = 1;
   while (S < 8 && base * S * 2 <= di.num_sms && S * 2 <= nk) {
@@ -678,9 +717,9 @@ static cudaError_t launch_prefill(const __half* x, const PrefillProblem& pb, int
     if (cap > 0 && base > cap) break;
     S *= 2;
   }
-  if (TN == 64) return launch_prefill_t<kInt4, 64, kPrefillSSMaxTN >= 64>(x, pb, M, K, S, s);
-  if (TN == 128) return launch_prefill_t<kInt4, 128, kPrefillSSMaxTN >= 128>(x, pb, M, K, S, s);
-  return launch_prefill_t<kInt4, 256, false>(x, pb, M, K, S, s);
+  if (TN == 64) return launch_prefill_t<kInt4, 64, true, kPrefillSSStageK>(x, pb, M, K, S, s);
+  if (TN == 128) return launch_prefill_t<kInt4, 128, true, kPrefillSSStageK>(x, pb, M, K, S, s);
+  return launch_prefill_t<kInt4, 256, false, kQK>(x, pb, M, K, S, s);
 }
 
 static PrefillProblem one_matrix(const void* w, const __half* sc, const uint8_t* zp, const __half* bias, __half* y,
