@@ -204,7 +204,7 @@ cudaError_t launch_tq_validate(const uint8_t* packed, int64_t N, int64_t K, int*
 constexpr int64_t kDecodeMaxM = 64;
 // Largest M the automatic dispatch sends to the decode path, per format (the measured crossover
 // with the tensor-core path on Llama-3-8B and Qwen2-7B shaped linears).
-constexpr int64_t kDecodeAutoMaxM_Ternary = 32;
+constexpr int64_t kDecodeAutoMaxM_Ternary = 16;
 constexpr int64_t kDecodeAutoMaxM_W4g = 16;
 cudaError_t launch_tq_gemm_decode(const __half* x, const uint8_t* packed, const __half* scale,
                                   const __half* bias, __half* y, int64_t M, int64_t N, int64_t K,

@@ -74,7 +74,7 @@ typedef enum { TQ_F32 = 0, TQ_F16 = 1 } tq_dtype;
 /* GEMM execution paths.  AUTO applies tq_select_path(); the others force one path (tests).
  * The decode path runs at most 16 tokens per CTA; 17 <= M <= 64 runs ceil(M/16) token chunks
  * in the same launch.  tq_select_path picks decode up to the crossover measured on Llama-3-8B /
- * Qwen2-7B shaped linears (ternary M <= 32, W4A16 M <= 16) and the tensor-core path above. */
+ * Qwen2-7B shaped linears (M <= 16 for both formats) and the tensor-core path above. */
 typedef enum {
     TQ_PATH_AUTO = 0,
     TQ_PATH_DECODE = 1,  /* memory-bound skinny path, M <= 64: mma.sync on in-register decode  */

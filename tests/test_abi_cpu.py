@@ -79,12 +79,9 @@ def test_dispatch_rule():
     assert tq.tq_select_path(T, 1, 4096, 14336) == tq.PATH_DECODE
     assert tq.tq_select_path(T, 1, 3584, 18944) == tq.PATH_DECODE
     assert tq.tq_select_path(T, 16, 37888, 3584) == tq.PATH_DECODE
-    # measured crossover (Qwen2-7B shapes): ternary decode in 16-token chunks up to M = 32,
-    # W4A16 decode up to M = 16; the tensor-core path above
-    for M in (17, 24, 32):
-        assert tq.tq_select_path(T, M, 4096, 4096) == tq.PATH_DECODE
-        assert tq.tq_select_path(T, M, 37888, 3584) == tq.PATH_DECODE
-    for M in (33, 40, 48, 64, 512, 2048, 8192):
+    # measured crossover (Qwen2-7B shapes): decode up to M = 16 for both formats (a second
+    # 16-token chunk costs more than the tensor-core path); the tensor-core path above
+    for M in (17, 24, 32, 33, 40, 48, 64, 512, 2048, 8192):
         assert tq.tq_select_path(T, M, 4096, 4096) == tq.PATH_PREFILL
     for M in (17, 24, 32, 512, 2048, 8192):
         assert tq.tq_select_path(W, M, 14336, 4096) == tq.PATH_PREFILL

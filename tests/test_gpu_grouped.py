@@ -10,8 +10,7 @@ from gpu_util import check_canaries, check_tq_gemm, check_w4g_gemm, gpu, guarded
 pytestmark = gpu
 
 
-# M = 29 and 32 take the decode path in token chunks of 16 (29: the last one ragged), one launch
-# for all three matrices; M = 41 the tensor-core path, also one launch
+# M <= 16: one decode launch for all three matrices; M = 29, 32, 41: one tensor-core launch
 @pytest.mark.parametrize("M", [1, 5, 16, 29, 32, 41])
 def test_tq_grouped_qkv(M):
     need_cuda()
