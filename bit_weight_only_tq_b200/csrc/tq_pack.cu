@@ -791,10 +791,11 @@ cudaError_t launch_tq_interleave(const uint32_t* in, uint32_t* out, int64_t word
 }
 
 // ---------------------------------------------------------------------------------------------
-// W4A16 pack: one warp per (row n, group g of 128).  Lane l holds k = 128g + 4l .. 4l+3.
+// W4A16 pack.  A warp quantises whole groups of 128; lane l holds weights 4l .. 4l+3 of a group.
 // ---------------------------------------------------------------------------------------------
-// The group quantiser shared by both W4 pack kernels: this lane's four weights wf of one
-// 128-wide group (the warp holds the group).  Symmetric ([VQ] §5 "sym": true): s = fp16(max|w|/7),
+// The group quantiser of the activation-order kernel: this lane's four weights wf of one
+// 128-wide group (the warp holds the group).  The contiguous-group kernel below computes the same
+// codes, scales and zeros, sixteen groups per warp at a time.  Symmetric ([VQ] §5 "sym": true): s = fp16(max|w|/7),
 // q = clamp(rint(w / s), -8, 7), stored u = q + 8.  Asymmetric (zeros requested, the weight_zp of
 // the same section): lo = min(0, min w), hi = max(0, max w), s = fp16((hi - lo) / 15),
 // z = clamp(rint(-lo / s), 0, 15), stored u = clamp(rint(w / s) + z, 0, 15).  All quotients in
@@ -823,52 +824,209 @@ __device__ __forceinline__ void w4_quantize_group(const float (&wf)[4], bool asy
   sb = asym ? f64_to_f16_rne((static_cast<double>(b) - static_cast<double>(a)) / 15.0)
             : f64_to_f16_rne(static_cast<double>(a) / 7.0);
   const double sd = f16_bits_to_f64(sb);
+  // rint(v / s) in fp32 with the same result as the fp64 quotient: r = v * (1 / s) is within a
+  // few fp32 ulps of q = v / s, so floor(r) + 1/2 is the half-integer h next to q (r is clamped
+  // to +-64 first: every q beyond that saturates the code alike); whether q lies below, at or
+  // above h is the sign of h s - v, which one fused multiply-add gives exactly (h s is exact, and
+  // h s - v is a multiple of 2^-149, so it never rounds to zero unless it is zero: this needs
+  // fp32 subnormals, i.e. no flush-to-zero); at q == h the even neighbour wins, as rint's does.
+  // An infinite s or a non-finite v takes the fp64 quotient (clamped alike; a NaN quotient gives
+  // the lowest code, as the clamps of the fp64 form do).  The result lies in [-64, 65].
+  const float sf = static_cast<float>(sd);
+  const bool fin_s = sd != 0.0 && sd < INFINITY;
+  const float inv = fin_s ? 1.0f / sf : 0.0f;
+  auto q_of = [&](float v) -> int {
+    if (!fin_s || !(fabsf(v) < INFINITY))
+      return static_cast<int>(fmin(fmax(rint(static_cast<double>(v) / sd), -64.0), 65.0));
+    const int fl = static_cast<int>(floorf(fminf(fmaxf(__fmul_rn(v, inv), -64.0f), 64.0f)));
+    const float d = __fmaf_rn(static_cast<float>(fl) + 0.5f, sf, -v);
+    return d < 0.0f ? fl + 1 : d > 0.0f ? fl : fl + (fl & 1);
+  };
   z = asym ? 0 : 8;
-  if (asym && sd != 0.0) z = static_cast<int>(fmin(fmax(rint(-static_cast<double>(a) / sd), 0.0), 15.0));
+  if (asym && sd != 0.0) z = min(max(q_of(-a), 0), 15);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     if (sd == 0.0) {
       u[i] = asym ? 0 : 8;
     } else {
-      const double r = rint(static_cast<double>(wf[i]) / sd);
-      u[i] = asym ? static_cast<int>(fmin(fmax(r + z, 0.0), 15.0)) : static_cast<int>(fmin(fmax(r, -8.0), 7.0)) + 8;
+      const int r = q_of(wf[i]);
+      u[i] = asym ? min(max(r + z, 0), 15) : min(max(r, -8), 7) + 8;
     }
   }
 }
 
-// One warp per (row, group of 128 consecutive columns): four columns per lane, whole words out.
-template <bool kF16>
+// Contiguous groups.  Item i = n G + g (row n, group g of 128 columns; K = 128 G) is the 128
+// weights at element 128 i of the row-major W, and its outputs are qweight words 16 i .. 16 i + 15,
+// scale i and zero i, so W is walked as one flat run of items.  A warp takes kB = 16 consecutive
+// items per pass; lane l holds weights 4 l .. 4 l + 3 of each, all sixteen loads issued first.
+// The group statistics (max |w|, or min and max) are reduced across the warp for all sixteen
+// items at once by recursive halving (each exchange step halves the items a lane still holds, so
+// lane l ends with item l mod 16 after 16 shuffles instead of 80), the lane then derives that
+// item's scale (and zero) in fp64 as the group quantiser above does, and the quantiser of each
+// item reads them back from lane j with one shuffle per item.
+//
+// Codes in fp32, equal to rint(v / s) of the fp64 quotient: r = v * (1 / s) is within a few fp32
+// ulps of q = v / s, so h = floor(r) + 1/2 is a half-integer within one of q; q > h, q = h or
+// q < h is the sign of d = h s - v, which one fused multiply-add gives exactly (h s is exact, h s
+// - v is a multiple of 2^-149 and so rounds to zero only when it is zero: this needs fp32
+// subnormals, i.e. no flush-to-zero), so the code is h + 1/2, h (a tie) or h - 1/2; adding
+// 1.5 * 2^23 rounds a tie to even, as rint does, and leaves the code in the low mantissa bits.
+// Overflowing or non-finite quotients (huge v, v = +-inf or NaN, s = inf) end at the same clamped
+// codes as the fp64 form; s = 0 gives code 8 (symmetric) or 0 (asymmetric), as there.
+constexpr int kW4PackItems = 16;
+
+template <bool kF16, bool kAsym>
 __global__ void __launch_bounds__(256)
-    w4g_pack_kernel(const void* __restrict__ w, int32_t* __restrict__ qweight,
-                    uint16_t* __restrict__ scales, uint8_t* __restrict__ zeros, int64_t N, int64_t K, int vec) {
+    w4g_pack_kernel(const void* __restrict__ w, int32_t* __restrict__ qweight, uint16_t* __restrict__ scales,
+                    uint8_t* __restrict__ zeros, int64_t items, int vec) {
+  constexpr int kB = kW4PackItems;
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23: integers in the low mantissa bits
   const int lane = threadIdx.x & 31;
-  const int64_t G = K >> 7;
   const int64_t warps_total = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  for (int64_t item = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-       item < N * G; item += warps_total) {
-    const int64_t n = item / G, g = item - n * G;
-    const int64_t k0 = g * 128 + 4 * lane;
-    const void* row = kF16 ? static_cast<const void*>(static_cast<const uint16_t*>(w) + n * K)
-                           : static_cast<const void*>(static_cast<const float*>(w) + n * K);
-    uint32_t v[4];
-    load4<kF16>(row, k0 >> 2, K, vec, v);
-    float wf[4];
+  for (int64_t base = (static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5)) * kB;
+       base < items; base += warps_total * kB) {
+    const int nb = items - base < kB ? static_cast<int>(items - base) : kB;  // the same for the whole warp
+    const void* grp0 = kF16 ? static_cast<const void*>(static_cast<const uint16_t*>(w) + base * 128)
+                            : static_cast<const void*>(static_cast<const float*>(w) + base * 128);
+    // fp32: four values per lane and item; fp16: two half pairs
+    constexpr int kWords = kF16 ? 2 : 4;
+    uint32_t v[kB][kWords];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      wf[i] = kF16 ? __half2float(__ushort_as_half(static_cast<uint16_t>(v[i]))) : __uint_as_float(v[i]);
-    uint16_t sb;
-    int z, u[4];
-    w4_quantize_group(wf, zeros != nullptr, sb, z, u);
-    uint32_t nib = 0;
+    for (int j = 0; j < kB; ++j) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) nib |= static_cast<uint32_t>(u[i]) << (4 * i);
-    const uint32_t other = __shfl_down_sync(0xFFFFFFFFu, nib, 1);
-    if ((lane & 1) == 0) {
-      qweight[n * (K >> 3) + g * 16 + (lane >> 1)] = static_cast<int32_t>(nib | (other << 16));
+      for (int i = 0; i < kWords; ++i) v[j][i] = 0u;
+      if (j >= nb) continue;
+      if (kF16) {
+        const uint16_t* p = static_cast<const uint16_t*>(grp0) + j * 128 + 4 * lane;
+        if (vec) {
+          const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+          v[j][0] = u.x;
+          v[j][1] = u.y;
+        } else {
+          v[j][0] = static_cast<uint32_t>(__ldg(p)) | (static_cast<uint32_t>(__ldg(p + 1)) << 16);
+          v[j][1] = static_cast<uint32_t>(__ldg(p + 2)) | (static_cast<uint32_t>(__ldg(p + 3)) << 16);
+        }
+      } else {
+        const float* p = static_cast<const float*>(grp0) + j * 128 + 4 * lane;
+        if (vec) {
+          const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+          v[j][0] = u.x;
+          v[j][1] = u.y;
+          v[j][2] = u.z;
+          v[j][3] = u.w;
+        } else {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) v[j][i] = __float_as_uint(__ldg(p + i));
+        }
+      }
     }
-    if (lane == 0) {
-      scales[n * G + g] = sb;
-      if (zeros) zeros[n * G + g] = static_cast<uint8_t>(z);
+    auto vals = [&](int j, float (&f)[4]) {
+      if (kF16) {
+        const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&v[j][0]));
+        const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&v[j][1]));
+        f[0] = f01.x;
+        f[1] = f01.y;
+        f[2] = f23.x;
+        f[3] = f23.y;
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) f[i] = __uint_as_float(v[j][i]);
+      }
+    };
+    // this lane's statistics of every item: symmetric a = max|w|; asymmetric a = min(0, w),
+    // b = max(0, w) (fp16: taken on the half pairs, exact; a NaN loses to any number, as in fminf)
+    float a[kB], b[kB];
+#pragma unroll
+    for (int j = 0; j < kB; ++j) {
+      if (kF16) {
+        const __half2 h0 = *reinterpret_cast<const __half2*>(&v[j][0]);
+        const __half2 h1 = *reinterpret_cast<const __half2*>(&v[j][1]);
+        if (kAsym) {
+          const __half2 lo = __hmin2(h0, h1), hi = __hmax2(h0, h1);
+          a[j] = fminf(fminf(0.0f, __low2float(lo)), __high2float(lo));
+          b[j] = fmaxf(fmaxf(0.0f, __low2float(hi)), __high2float(hi));
+        } else {
+          const __half2 m = __hmax2(__habs2(h0), __habs2(h1));
+          a[j] = fmaxf(fmaxf(0.0f, __low2float(m)), __high2float(m));
+          b[j] = 0.0f;
+        }
+      } else {
+        a[j] = 0.0f;
+        b[j] = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          if (kAsym) {
+            a[j] = fminf(a[j], __uint_as_float(v[j][i]));
+            b[j] = fmaxf(b[j], __uint_as_float(v[j][i]));
+          } else {
+            a[j] = fmaxf(a[j], fabsf(__uint_as_float(v[j][i])));
+          }
+        }
+      }
+    }
+    // recursive halving: after the step over lane bit k, a lane keeps the upper half of the items
+    // it held when that bit is set and the lower half otherwise, combined with its partner's copy
+#pragma unroll
+    for (int k = kB / 2; k >= 1; k >>= 1) {
+      const bool up = (lane & k) != 0;
+#pragma unroll
+      for (int i = 0; i < k; ++i) {
+        const float ra = __shfl_xor_sync(0xFFFFFFFFu, up ? a[i] : a[i + k], k);
+        a[i] = kAsym ? fminf(up ? a[i + k] : a[i], ra) : fmaxf(up ? a[i + k] : a[i], ra);
+        if (kAsym) {
+          const float rb = __shfl_xor_sync(0xFFFFFFFFu, up ? b[i] : b[i + k], k);
+          b[i] = fmaxf(up ? b[i + k] : b[i], rb);
+        }
+      }
+    }
+    a[0] = kAsym ? fminf(a[0], __shfl_xor_sync(0xFFFFFFFFu, a[0], 16))
+                 : fmaxf(a[0], __shfl_xor_sync(0xFFFFFFFFu, a[0], 16));
+    if (kAsym) b[0] = fmaxf(b[0], __shfl_xor_sync(0xFFFFFFFFu, b[0], 16));
+    // item lane mod 16: its scale, 1 / scale and zero point
+    const uint16_t sb = kAsym ? f64_to_f16_rne((static_cast<double>(b[0]) - static_cast<double>(a[0])) / 15.0)
+                              : f64_to_f16_rne(static_cast<double>(a[0]) / 7.0);
+    const float sf = __half2float(__ushort_as_half(sb));
+    const float inv = 1.0f / sf;  // +inf for s = 0 (then unused), 0 for s = inf
+    auto round_q = [&](float x, float s, float rs) -> float {  // rint(x / s), exact (see above)
+      const float h = floorf(__fmul_rn(x, rs)) + 0.5f;
+      const float d = __fmaf_rn(h, s, -x);
+      return d < 0.0f ? h + 0.5f : d > 0.0f ? h - 0.5f : h;
+    };
+    int z = kAsym ? 0 : 8;
+    if (kAsym && sf != 0.0f) {
+      const float n = (round_q(-a[0], sf, inv) + kMagic) - kMagic;  // ties to even; NaN stays NaN
+      z = static_cast<int>(fminf(fmaxf(n, 0.0f), 15.0f));
+    }
+    if (lane < nb) {
+      scales[base + lane] = sb;
+      if (kAsym) zeros[base + lane] = static_cast<uint8_t>(z);
+    }
+    const uint32_t sz = static_cast<uint32_t>(sb) | (static_cast<uint32_t>(z) << 16);
+#pragma unroll
+    for (int j = 0; j < kB; ++j) {
+      if (j >= nb) break;
+      const uint32_t szj = __shfl_sync(0xFFFFFFFFu, sz, j);
+      const float invj = __shfl_sync(0xFFFFFFFFu, inv, j);
+      const float sj = __half2float(__ushort_as_half(static_cast<uint16_t>(szj & 0xFFFFu)));
+      const float zj = static_cast<float>(szj >> 16);
+      float f[4];
+      vals(j, f);
+      uint32_t nib = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float y = round_q(f[i], sj, invj);
+        float t;
+        if (kAsym) {
+          const float n = (y + kMagic) - kMagic;
+          t = fminf(fmaxf(n + zj, 0.0f), 15.0f) + kMagic;
+        } else {
+          t = fminf(fmaxf(y, -8.0f), 7.0f) + (kMagic + 8.0f);
+        }
+        nib |= (__float_as_uint(t) & 15u) << (4 * i);
+      }
+      if (sj == 0.0f) nib = kAsym ? 0u : 0x8888u;
+      const uint32_t other = __shfl_down_sync(0xFFFFFFFFu, nib, 1);
+      if ((lane & 1) == 0) qweight[(base + j) * 16 + (lane >> 1)] = static_cast<int32_t>(nib | (other << 16));
     }
   }
 }
@@ -1012,11 +1170,20 @@ cudaError_t launch_w4g_pack_ex(const void* w, bool w_f16, const int32_t* perm, i
   }
   const uintptr_t a = reinterpret_cast<uintptr_t>(w);
   const int vec = (a % (w_f16 ? 8 : 16) == 0);
-  if (w_f16)
-    w4g_pack_kernel<true><<<static_cast<unsigned>(grid), 256, 0, s>>>(w, qweight, scales, zeros, N, K, vec);
-  else
-    w4g_pack_kernel<false><<<static_cast<unsigned>(grid), 256, 0, s>>>(w, qweight, scales, zeros, N, K, vec);
-  return cudaGetLastError();
+  // eight warps per CTA, each taking 16 items a pass; the grid is what stays resident
+  auto go = [&](auto kern) {
+    int bps = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, kern, 256, 0) != cudaSuccess || bps < 1) {
+      (void)cudaGetLastError();
+      bps = 1;
+    }
+    const int64_t g = std::min<int64_t>((items + 8 * kW4PackItems - 1) / (8 * kW4PackItems),
+                                        static_cast<int64_t>(bps) * di.num_sms);
+    kern<<<static_cast<unsigned>(g), 256, 0, s>>>(w, qweight, scales, zeros, items, vec);
+    return cudaGetLastError();
+  };
+  if (w_f16) return zeros ? go(w4g_pack_kernel<true, true>) : go(w4g_pack_kernel<true, false>);
+  return zeros ? go(w4g_pack_kernel<false, true>) : go(w4g_pack_kernel<false, false>);
 }
 
 }  // namespace tq
