@@ -57,6 +57,44 @@ def test_pack_bit_exact(zero_point, act_order, dtype):
     _check_pack(w, zero_point, perm)
 
 
+def _tie_weights(N, K, seed, np_dtype):
+    """Groups whose weights sit exactly on the rounding ties (k + 1/2) s of their own scale s and
+    on the representable values next to them: every group holds 7 s (so max|w| / 7 = s for the
+    symmetric rule) and every other group also -8 s (so (hi - lo) / 15 = s for the zero-point
+    rule, zero 8).  s ranges over fp16 normals and subnormals; for fp16 weights s = m 2^e with a
+    5-bit m, so that every tie is itself an fp16 value."""
+    rng = np.random.default_rng(seed)
+    G = K // 128
+    w = np.empty((N, G, 128), dtype=np_dtype)
+    for n in range(N):
+        for g in range(G):
+            if np_dtype == np.float16:
+                s0 = np.ldexp(float(rng.integers(1, 32)), int(rng.integers(-23, 6)))
+            else:
+                s0 = float(np.array([rng.integers(1, 0x5800)], dtype=np.uint16).view(np.float16)[0])
+            tie = ((rng.integers(-7, 7, 128) + 0.5) * s0).astype(np_dtype)
+            side = rng.integers(0, 3, 128)
+            vals = np.where(side == 0, tie, np.where(side == 1, np.nextafter(tie, np_dtype(np.inf)),
+                                                     np.nextafter(tie, np_dtype(-np.inf))))
+            vals[0] = 7 * s0
+            if (n + g) % 2:
+                vals[1] = -8 * s0
+            w[n, g] = vals
+    return w.reshape(N, K)
+
+
+# 37 x 384: 111 groups, so the last pass of the contiguous-group kernel (16 groups a warp) is ragged
+@pytest.mark.parametrize("zero_point", [False, True])
+@pytest.mark.parametrize("act_order", [False, True])
+@pytest.mark.parametrize("np_dtype", [np.float32, np.float16])
+def test_pack_rounding_ties(zero_point, act_order, np_dtype):
+    need_cuda()
+    N, K = 37, 384
+    w = torch.from_numpy(_tie_weights(N, K, 17, np_dtype))
+    perm = torch.randperm(K, generator=torch.Generator().manual_seed(5)).to(torch.int32) if act_order else None
+    _check_pack(w, zero_point, perm)
+
+
 def _zp_problem(M, N, K, seed, outlier_rows=0.0):
     w = _edge_weights(N, K, seed)
     qw, sc, zp, _ = tq.w4g_quantize_pack_ex(w.cuda(), zero_point=True)
