@@ -562,6 +562,32 @@ def secondary_rows(args, rank, layers, peaks):
                                          "peak": tc, "bound": "tensor",
                                          "sample": f"4 layers x 7 shapes, M={M}; q/k/v and gate/up grouped"}
         del g, xs, ys
+    # ---- W4A16 pack (config 3 weights, fp32): 2 layers x 7 shapes, 1.75 GB read
+    wf = [[I.weights(N, K, I.seed_for(3, l, mid) + rank_seed_offset(rank), device="cuda", outlier_frac=0.001)
+           for mid, (name, N, K) in enumerate(LLAMA)] for l in range(2)]
+    po = [[(torch.empty(N, K // 8, dtype=torch.int32, device="cuda"),
+            torch.empty(N, K // 128, dtype=torch.float16, device="cuda")) for (name, N, K) in LLAMA] for _ in range(2)]
+
+    def pack4():
+        for l in range(2):
+            for mid in range(len(LLAMA)):
+                tq.w4g_quantize_pack(wf[l][mid], po[l][mid][0], po[l][mid][1])
+
+    pack4()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(True), torch.cuda.Event(True)
+    a.record()
+    pack4()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    byts = 2 * sum(N * K * 4 + N * K // 2 + 2 * N * (K // 128) for _, N, K in LLAMA)
+    gbs = byts / (ms * 1e-3) / 1e9
+    rows["w4g_quantize_pack_llama_fp32"] = {"value": round(gbs, 1), "unit": "GB/s", "frac": round(gbs / hbm, 4),
+                                            "peak": hbm, "bound": "hbm", "ms": round(ms, 3),
+                                            "sample": f"2 Llama-3-8B layers x 7 shapes, fp32 in "
+                                                      f"({byts / 1e9:.2f} GB moved), inputs larger than L2"}
+    del wf, po
     # ---- W4A16 decode / prefill (config 3): 8 layers
     w4 = []
     for l in range(8):
