@@ -35,8 +35,8 @@ constexpr int kBMaxItems = kBatchMaxItems;
 constexpr int kBRows = 128;       // rows of a row block (one packed TMA tile)
 constexpr int kBResPitch = 132;   // fp32 row pitch of the result buffer [token][row]
 constexpr int kBCtasPerSm = 2;
-constexpr bool kBatchM8FourWarps = false;
-constexpr int kBatchPreW = 8;              // stages whose weights are loaded before the PDL wait  // M <= 8: four consumer warps over whole stages
+constexpr bool kBatchM8FourWarps = false;  // M <= 8: four consumer warps over whole stages (measured slower)
+constexpr int kBatchPreW = 8;              // stages whose weights are loaded before the PDL wait
 
 struct BatchItem {
   const __half* sc;    // ternary: scale[N]; W4A16: scales[N, K/128]
