@@ -121,6 +121,7 @@ struct PrefillArgs {
   const __half* bias[kQMaxGroup];  // may be null
   __half* y[kQMaxGroup];
   int64_t N[kQMaxGroup];
+  int64_t ldy[kQMaxGroup];         // y row stride (elements): N, or more for a block of y's columns
   int tile0[kQMaxGroup + 1];
   int count;
   int64_t M, K;
@@ -206,6 +207,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
   const uint8_t* const gzp = a.zp[g];
   const __half* const gbias = a.bias[g];
   __half* const gy = a.y[g];
+  const int64_t gldy = a.ldy[g];
   const CUtensorMap* const tmap_w = &tmaps_w.m[g];
   const int64_t m0 = static_cast<int64_t>(blockIdx.y) * TN;   // first token
   const int nk_all = static_cast<int>((a.K + kKS - 1) / kKS);  // a last half stage reads zeros
@@ -445,7 +447,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
       if (!kInt4) ep_s = __half2float(gsc[n]);
       if (gbias) ep_b = __half2float(gbias[n]);
     }
-    const bool vec = (Ng & 7) == 0;
+    const bool vec = ((Ng | gldy) & 7) == 0 && (reinterpret_cast<uintptr_t>(gy) & 15u) == 0;
     // y[m0 + t0 + t, n0 + 0..127] for t < cnt (<= 32) from a staging buffer [cnt][128 rows]
     // fp16 of this group (named barrier 1 + grp): 16 chunks of 16 bytes per token, four per
     // thread, then the buffer is free again
@@ -457,7 +459,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
         const int64_t m = m0 + t0 + tok, nb = n0 + ch * 8;
         if (tok < cnt && m < a.M && nb < Ng) {
           const uint4 val = *reinterpret_cast<const uint4*>(stage + tok * kQM + ch * 8);
-          __half* dst = gy + m * Ng + nb;
+          __half* dst = gy + m * gldy + nb;
           if (vec && nb + 8 <= Ng) {
             *reinterpret_cast<uint4*>(dst) = val;
           } else {
@@ -582,6 +584,7 @@ struct PrefillProblem {
   const __half* bias[kQMaxGroup];
   __half* y[kQMaxGroup];
   int64_t N[kQMaxGroup];
+  int64_t ldy[kQMaxGroup];  // 0: N
 };
 
 template <bool kInt4, int TN, bool kSS, int kKS>
@@ -608,6 +611,7 @@ static cudaError_t launch_prefill_t(const __half* x, const PrefillProblem& pb, i
       a.bias[g] = pb.bias[g];
       a.y[g] = pb.y[g];
       a.N[g] = pb.N[g];
+      a.ldy[g] = pb.ldy[g] > 0 ? pb.ldy[g] : pb.N[g];
       a.tile0[g + 1] = a.tile0[g] + static_cast<int>((pb.N[g] + kQM - 1) / kQM);
     } else {
       tw.m[g] = tw.m[0];
@@ -697,6 +701,73 @@ bool prefill_grouping_pays(int64_t M, const int64_t* N, int count) {
   return rt * ((M + TN - 1) / TN) <= 4 * static_cast<int64_t>(current_device_info().num_sms);
 }
 
+// Row tiles [r0, r1) of a problem (numbered matrix by matrix, as the grid runs over them) as a
+// problem of its own: each matrix's part starts at its weights', scales', zeros', bias' and y's
+// row offset, and y keeps its row stride.
+template <bool kInt4>
+static PrefillProblem sub_rows(const PrefillProblem& pb, int64_t K, int64_t r0, int64_t r1) {
+  PrefillProblem out = {};
+  const int64_t kbytes = kInt4 ? K / 2 : K / 4, G = K >> 7;
+  int64_t t0 = 0;  // first row tile of matrix g
+  for (int g = 0; g < pb.count; ++g) {
+    const int64_t nt = (pb.N[g] + kQM - 1) / kQM;
+    const int64_t lo = r0 > t0 ? r0 : t0, hi = r1 < t0 + nt ? r1 : t0 + nt;
+    if (lo < hi) {
+      const int64_t row = (lo - t0) * kQM, end = (hi - t0) * kQM < pb.N[g] ? (hi - t0) * kQM : pb.N[g];
+      const int i = out.count++;
+      out.w[i] = static_cast<const uint8_t*>(pb.w[g]) + row * kbytes;
+      out.sc[i] = pb.sc[g] + (kInt4 ? row * G : row);
+      out.zp[i] = pb.zp[g] ? pb.zp[g] + row * G : nullptr;
+      out.bias[i] = pb.bias[g] ? pb.bias[g] + row : nullptr;
+      out.y[i] = pb.y[g] + row;
+      out.N[i] = end - row;
+      out.ldy[i] = pb.ldy[g] > 0 ? pb.ldy[g] : pb.N[g];
+    }
+    t0 += nt;
+  }
+  return out;
+}
+
+// A launch whose tiles end in a part-empty wave (tiles = W waves + a few) leaves most SMs idle for
+// a whole tile time.  Split instead: the row tiles that fill whole waves (of CTAs, with K split
+// over Sm when that makes the waves come out whole) in one launch, the few row tiles left in a
+// second launch with K split over a cluster of St, which then takes about 1 / St of a tile time.
+// Cost model, in units of one full-K tile's time: a wave of CTAs that each take 1 / S of K costs
+// 1 / S + 0.12 (a CTA's fixed prologue and epilogue, about 3 us against about 25 us for a tile
+// of K = 4096) + 0.08 when S > 1 (the cluster's partial-sum exchange).
+struct PrefillTailPlan {
+  int64_t rows_main = 0;  // row tiles of the first launch; 0: no split
+  int Sm = 1, St = 1;
+};
+
+template <typename Cap>
+static PrefillTailPlan prefill_tail_plan(int64_t rt, int64_t TT, int nk, int sms, Cap capacity) {
+  PrefillTailPlan best;
+  const int64_t base = rt * TT;
+  if (base <= sms) return best;
+  auto waves_cost = [&](int64_t ctas, int S) {
+    return static_cast<double>((ctas + sms - 1) / sms) * (1.0 / S + 0.12 + (S > 1 ? 0.08 : 0.0));
+  };
+  double best_cost = waves_cost(base, 1) * 0.92;  // a split must save 8 % by this model
+  for (int Sm = 1; Sm <= 4; Sm *= 2) {
+    if (Sm > nk || (Sm > 1 && capacity(Sm) <= 0)) break;
+    const int64_t W = base * Sm / sms;  // whole waves of CTAs
+    const int64_t rows_main = W * sms / (static_cast<int64_t>(Sm) * TT);
+    if (rows_main <= 0 || rows_main >= rt) continue;
+    const int64_t tail = (rt - rows_main) * TT;
+    int St = 8;
+    while (St > 1 && (tail * St > sms || St > nk || capacity(St) < tail)) St /= 2;
+    const double cost = waves_cost(rows_main * TT * Sm, Sm) + waves_cost(tail * St, St);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best.rows_main = rows_main;
+      best.Sm = Sm;
+      best.St = St;
+    }
+  }
+  return best;
+}
+
 template <bool kInt4>
 static cudaError_t launch_prefill(const __half* x, const PrefillProblem& pb, int64_t M, int64_t K, cudaStream_t s) {
   const DeviceInfo di = current_device_info();
@@ -705,11 +776,17 @@ static cudaError_t launch_prefill(const __half* x, const PrefillProblem& pb, int
   const int TN = prefill_tile_tokens(M);
   const int KS = TN <= kPrefillSSMaxTN ? kPrefillSSStageK : kQK;
   const int nk = static_cast<int>((K + KS - 1) / KS);
-  const int64_t base = rt * ((M + TN - 1) / TN);
+  const int64_t TT = (M + TN - 1) / TN;
+  const int64_t base = rt * TT;
   auto capacity = [&](int cs) {
     if (TN == 64) return prefill_cluster_capacity<kInt4, 64, true, kPrefillSSStageK>(di.device, cs);
     if (TN == 128) return prefill_cluster_capacity<kInt4, 128, true, kPrefillSSStageK>(di.device, cs);
     return prefill_cluster_capacity<kInt4, 256, false, kQK>(di.device, cs);
+  };
+  auto run = [&](const PrefillProblem& p, int S) {
+    if (TN == 64) return launch_prefill_t<kInt4, 64, true, kPrefillSSStageK>(x, p, M, K, S, s);
+    if (TN == 128) return launch_prefill_t<kInt4, 128, true, kPrefillSSStageK>(x, p, M, K, S, s);
+    return launch_prefill_t<kInt4, 256, false, kQK>(x, p, M, K, S, s);
   };
   int S = 1;
   while (S < 8 && base * S * 2 <= di.num_sms && S * 2 <= nk) {
@@ -717,9 +794,15 @@ static cudaError_t launch_prefill(const __half* x, const PrefillProblem& pb, int
     if (cap > 0 && base > cap) break;
     S *= 2;
   }
-  if (TN == 64) return launch_prefill_t<kInt4, 64, true, kPrefillSSStageK>(x, pb, M, K, S, s);
-  if (TN == 128) return launch_prefill_t<kInt4, 128, true, kPrefillSSStageK>(x, pb, M, K, S, s);
-  return launch_prefill_t<kInt4, 256, false, kQK>(x, pb, M, K, S, s);
+  if (S == 1) {
+    const PrefillTailPlan tp = prefill_tail_plan(rt, TT, nk, di.num_sms, capacity);
+    if (tp.rows_main > 0) {
+      const cudaError_t e = run(sub_rows<kInt4>(pb, K, 0, tp.rows_main), tp.Sm);
+      if (e != cudaSuccess) return e;
+      return run(sub_rows<kInt4>(pb, K, tp.rows_main, rt), tp.St);
+    }
+  }
+  return run(pb, S);
 }
 
 static PrefillProblem one_matrix(const void* w, const __half* sc, const uint8_t* zp, const __half* bias, __half* y,

@@ -63,6 +63,10 @@ def test_w4g_grouped():
     ("w4", 256, [512, 200, 128], 2048),
     ("w4", 100, [256, 136], 1152),
     ("tq", 4096, [4096, 4096], 256),      # more than four waves: one launch per matrix
+    # 150 row tiles x one token tile: 148 in a first launch, the last 2 (the second matrix's,
+    # one of them ragged) in a second launch split over K
+    ("tq", 256, [9600, 9550], 1024),
+    ("w4", 512, [9600], 1024),            # 75 row tiles x 2 token tiles: the last row tile apart
 ])
 def test_grouped_prefill(fmt, M, shapes, K):
     need_cuda()

@@ -122,6 +122,16 @@ def _check_zp(x, qw, sc, zp, b, y, g_idx=None, x_ref=None, cols=None, label=""):
                                     (3, tq.PATH_GENERIC), (5, tq.PATH_AUTO), (600, tq.PATH_AUTO)])
 @pytest.mark.parametrize("N,K", [(300, 1024), (4096, 4096)])
 def test_zero_point_gemm(M, path, N, K):
+    _zero_point_gemm(M, path, N, K)
+
+
+# 150 row tiles at M = 256: the last two run in a second launch (their zero points, scales and
+# bias from the row offset)
+def test_zero_point_prefill_tail_launch():
+    _zero_point_gemm(256, tq.PATH_PREFILL, 19150, 1024)
+
+
+def _zero_point_gemm(M, path, N, K):
     need_cuda()
     x, qw, sc, zp, b = _zp_problem(M, N, K, 11 + M, outlier_rows=0.01)
     y, buf = guarded_empty(M, N)
