@@ -210,7 +210,9 @@ TQ_API int tq_permute_columns(const uint16_t* x, const int32_t* perm, uint16_t* 
  * run in ONE decode launch; when it picks the tensor-core prefill path for every matrix and their
  * tiles together fill at most four waves of the GPU, in ONE prefill launch whose grid covers the
  * row tiles of all of them (one kernel boundary instead of `count`, and small matrices fill the
- * GPU together); otherwise the call issues `count` single-matrix GEMMs.
+ * GPU together; when those tiles would end in a nearly empty wave, the last few row tiles run in
+ * a second launch with K split over a cluster); otherwise the call issues `count` single-matrix
+ * GEMMs (each of which may split off its last row tiles the same way).
  *   count              1 .. 4
  *   packed / qweight   HOST array of `count` device pointers (layouts as in tq_gemm / w4g_gemm)
  *   scale / scales     HOST array of `count` device pointers
