@@ -293,9 +293,12 @@ def run_ours(args, world, rank, local):
             Y = [yv[(M, li, j)] for j in range(len(row))]
             batch_args.append((X, P, S, Y))
 
+    # every call names the call after it (the first of the next step after the last), whose
+    # first weight tiles it prefetches into L2 (tq_gemm_batch_next)
     def step_batch():
-        for X, P, S, Y in batch_args:
-            tq.tq_gemm_batch(X, P, S, None, Y, workspace=ws)
+        for i, (X, P, S, Y) in enumerate(batch_args):
+            Xn, Pn, _, _ = batch_args[(i + 1) % len(batch_args)]
+            tq.tq_gemm_batch(X, P, S, None, Y, workspace=ws, next_packed=Pn, next_M=Xn[0].shape[0])
 
     steps = {"batch": (step_batch, 1), "grouped": (step_grouped, 4), "separate": (step_separate, len(LLAMA))}
     step_fn, per_layer = steps[args.calls]
@@ -331,6 +334,9 @@ def run_ours(args, world, rank, local):
     copy_stream = torch.cuda.Stream()
     chunk = 8
     per_m = len(batch_args) // len(DECODE_M) if args.calls == "batch" else 0
+    # the end-to-end order (largest M first): the index of the call that follows each call
+    e2e_order = [mi * per_m + li for mi in reversed(range(len(DECODE_M))) for li in range(per_m)]
+    e2e_next = {a: e2e_order[(i + 1) % len(e2e_order)] for i, a in enumerate(e2e_order)}
 
     def e2e_fn():
         cs = torch.cuda.current_stream()
@@ -347,7 +353,8 @@ def run_ours(args, world, rank, local):
                 l1 = min(l0 + chunk, n_layers)
                 for li in range(l0, l1):
                     X, P, S, Y = batch_args[mi * per_m + li]
-                    tq.tq_gemm_batch(X, P, S, None, Y, workspace=ws)
+                    Xn, Pn, _, _ = batch_args[e2e_next[mi * per_m + li]]
+                    tq.tq_gemm_batch(X, P, S, None, Y, workspace=ws, next_packed=Pn, next_M=Xn[0].shape[0])
                 ev = torch.cuda.Event()
                 ev.record(cs)
                 copy_stream.wait_event(ev)
@@ -390,10 +397,15 @@ def run_ours(args, world, rank, local):
                                      P[j].shape[0], X[j].shape[1])
             prebuilt.append((arr, len(P), X[0].shape[0]))
         ws_p, ws_n = ctypes.c_void_p(ws.data_ptr()), ws.numel()
+        # each call with the call after it in that order (tq_gemm_batch_next)
+        def batch_call(a, nxt):
+            arr, n, M = prebuilt[a]
+            narr, nn, nM = prebuilt[nxt]
+            return tq.lib.tq_gemm_batch_next(arr, n, M, ws_p, ws_n, 0, narr, nn, nM, stream_h)
 
         def eager_calls():
-            for arr, n, M in prebuilt:
-                st = tq.lib.tq_gemm_batch(arr, n, M, ws_p, ws_n, stream_h)
+            for a in range(len(prebuilt)):
+                st = batch_call(a, (a + 1) % len(prebuilt))
                 if st != 0:
                     raise RuntimeError(tq.tq_status_string(st))
 
@@ -412,8 +424,8 @@ def run_ours(args, world, rank, local):
         for mi, M in reversed(list(enumerate(DECODE_M))):
             for l0 in range(0, n_layers, chunk):
                 l1 = min(l0 + chunk, n_layers)
-                for arr, n, Mi in prebuilt[mi * per_m + l0: mi * per_m + l1]:
-                    st = tq.lib.tq_gemm_batch(arr, n, Mi, ws_p, ws_n, stream_h)
+                for a in range(mi * per_m + l0, mi * per_m + l1):
+                    st = batch_call(a, e2e_next[a])
                     if st != 0:
                         raise RuntimeError(tq.tq_status_string(st))
                 ev = torch.cuda.Event()
@@ -902,8 +914,8 @@ PROFILE_CASES = {
                "grouped at M=256, 3 launches; ternary q/k/v (4096+1024+1024)x4096 grouped at M=512, 3 launches",
     "pack": "tq_quantize_pack of an fp16 Qwen2-7B gate_up 37888x3584 (2 launches) and an fp32 4096x4096 (2 launches); w4g_quantize_pack of the latter (2 launches)",
     "prefill_mid": "ternary Qwen2-7B down 3584x18944 at M=128, 3 launches; gate_up 37888x3584 at M=32, 3 launches",
-    "batch": "tq_gemm_batch over one Llama-3-8B layer's 7 ternary linears (54.5 MB packed) at M=1, 3 launches; "
-             "then at M=16, 3 launches",
+    "batch": "tq_gemm_batch over the 7 ternary linears of a Llama-3-8B layer (54.5 MB packed; four layers in "
+             "turn, 218 MB, each call naming the next) at M=1, 6 launches; then at M=16, 6 launches",
     "w4g_batch": "w4g_gemm_batch over one Llama-3-8B layer's 7 W4A16 linears (109 MB) at M=1, 3 launches; "
                  "then at M=16, 3 launches",
 }
@@ -965,16 +977,27 @@ def run_profile_case(name):
     elif name in ("batch", "w4g_batch"):
         int4 = name == "w4g_batch"
         ws = tq.batch_workspace()
-        mats = []
-        for mid, (_, N, K) in enumerate(LLAMA):
-            w = I.weights(N, K, 10 + mid, device="cuda", outlier_frac=0.001 if int4 else 0.0)
-            mats.append((tq.w4g_quantize_pack(w) if int4 else tq.tq_quantize_pack(w)) + (K,))
-            del w
-        fn = tq.w4g_gemm_batch if int4 else tq.tq_gemm_batch
-        for M in (1, 16):
-            xs = {K: I.activations(M, K, 20 + K, device="cuda") for K in (4096, 14336)}
-            for _ in range(3):
-                fn([xs[K] for _, _, K in mats], [p for p, _, _ in mats], [s for _, s, _ in mats], workspace=ws)
+        nl = 1 if int4 else 4
+        layers = []
+        for li in range(nl):
+            mats = []
+            for mid, (_, N, K) in enumerate(LLAMA):
+                w = I.weights(N, K, 10 + 7 * li + mid, device="cuda", outlier_frac=0.001 if int4 else 0.0)
+                mats.append((tq.w4g_quantize_pack(w) if int4 else tq.tq_quantize_pack(w)) + (K,))
+                del w
+            layers.append(mats)
+        calls = [(M, i % nl) for M in (1, 16) for i in range(3)] if int4 else \
+            [(1 if i < 6 else 16, i % nl) for i in range(12)]
+        xs = {(M, K): I.activations(M, K, 20 + K, device="cuda") for M in (1, 16) for K in (4096, 14336)}
+        for i, (M, li) in enumerate(calls):
+            mats = layers[li]
+            args3 = ([xs[(M, K)] for _, _, K in mats], [p for p, _, _ in mats], [s for _, s, _ in mats])
+            if int4:
+                tq.w4g_gemm_batch(*args3, workspace=ws)
+            else:
+                nxt = calls[i + 1] if i + 1 < len(calls) else None
+                tq.tq_gemm_batch(*args3, workspace=ws, next_packed=None if nxt is None else
+                                 [p for p, _, _ in layers[nxt[1]]], next_M=0 if nxt is None else nxt[0])
     elif name == "pack":
         w = I.weights(37888, 3584, 1, device="cuda", dtype=torch.float16)
         for _ in range(2):

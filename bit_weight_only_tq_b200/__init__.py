@@ -71,6 +71,8 @@ _SIGS = {
     "tq_gemm_grouped": [_vp, _int, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _vp],
     "w4g_gemm_grouped": [_vp, _int, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _vp],
     "tq_gemm_batch": [_vp, _int, _i64, _vp, ctypes.c_size_t, _vp],
+    "tq_gemm_batch_next": [_vp, _int, _i64, _vp, ctypes.c_size_t, _int, _vp, _int, _i64, _vp],
+    "w4g_gemm_batch_next": [_vp, _int, _i64, _vp, ctypes.c_size_t, _int, _vp, _int, _i64, _vp],
     "w4g_gemm_batch": [_vp, _int, _i64, _vp, ctypes.c_size_t, _vp],
     "tq_batch_workspace_size": [],
     "tq_gemm_batch_ex": [_vp, _int, _i64, _vp, ctypes.c_size_t, _int, _vp],
@@ -351,7 +353,8 @@ def tq_interleave_packed(packed: torch.Tensor, out: torch.Tensor = None, stream=
     return out
 
 
-def _batch(fn, xs, weights, scales, biases, ys, workspace, wdtype, sdim, what, stream, zeros=None, variant=0):
+def _batch(fn, xs, weights, scales, biases, ys, workspace, wdtype, sdim, what, stream, zeros=None, variant=0,
+           next_fn=None, next_weights=None, next_M=0, k_per_col=4):
     count = len(weights)
     if not (1 <= count <= 8) or len(scales) != count or len(xs) != count:
         raise ValueError("1..8 linears, each with its x, weights and scales")
@@ -379,24 +382,39 @@ def _batch(fn, xs, weights, scales, biases, ys, workspace, wdtype, sdim, what, s
     if workspace is None:
         raise ValueError("a workspace from batch_workspace() is required")
     _need(workspace, torch.uint8, "workspace", 1)
+    if next_weights:
+        nxt = (TqLinear * len(next_weights))()
+        for i, w in enumerate(next_weights):
+            _need(w, wdtype, "next weights", 2)
+            nxt[i] = TqLinear(None, w.data_ptr(), None, None, None, w.shape[0], w.shape[1] * k_per_col, None)
+        _check(next_fn(items, count, M, _ptr(workspace), workspace.numel(), int(variant), nxt, len(next_weights),
+                       int(next_M), _stream(stream)), what)
+        return out
     _check(fn(items, count, M, _ptr(workspace), workspace.numel(), int(variant), _stream(stream)), what)
     return out
 
 
 def tq_gemm_batch(xs, packed_list, scale_list, bias_list=None, y_list=None, workspace=None, stream=None,
-                  variant=BATCH_AUTO, interleaved=False):
+                  variant=BATCH_AUTO, interleaved=False, next_packed=None, next_M=0):
     """Independent ternary linears sharing M (each with its own x) in one persistent launch.
-    interleaved=True: the packed weights come from tq_interleave_packed."""
+    interleaved=True: the packed weights come from tq_interleave_packed.  next_packed / next_M:
+    the packed weights and token count of the batch call that follows on this stream (its first
+    tiles are prefetched into L2 during this one; tq_gemm_batch_next)."""
     v = int(variant) | (BATCH_INTERLEAVED if interleaved else 0)
     return _batch(lib.tq_gemm_batch_ex, xs, packed_list, scale_list, bias_list, y_list, workspace, torch.uint8, 1,
-                  "tq_gemm_batch", stream, variant=v)
+                  "tq_gemm_batch", stream, variant=v, next_fn=lib.tq_gemm_batch_next if next_packed else None,
+                  next_weights=next_packed,
+                  next_M=next_M, k_per_col=4)
 
 
 def w4g_gemm_batch(xs, qweight_list, scales_list, bias_list=None, y_list=None, workspace=None, stream=None,
-                   zeros_list=None, variant=BATCH_AUTO):
-    """Independent W4A16 linears sharing M in one persistent launch (zero-points optional)."""
+                   zeros_list=None, variant=BATCH_AUTO, next_qweight=None, next_M=0):
+    """Independent W4A16 linears sharing M in one persistent launch (zero-points optional);
+    next_qweight / next_M name the batch call that follows (w4g_gemm_batch_next)."""
     return _batch(lib.w4g_gemm_batch_ex, xs, qweight_list, scales_list, bias_list, y_list, workspace, torch.int32, 2,
-                  "w4g_gemm_batch", stream, zeros=zeros_list, variant=variant)
+                  "w4g_gemm_batch", stream, zeros=zeros_list, variant=variant,
+                  next_fn=lib.w4g_gemm_batch_next if next_qweight else None, next_weights=next_qweight,
+                  next_M=next_M, k_per_col=8)
 
 
 def tq_gemm_batch_noalloc(xs, packed_list, scale_list, bias_list=None, y_list=None, stream=None):

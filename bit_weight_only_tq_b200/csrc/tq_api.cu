@@ -421,8 +421,26 @@ namespace {
 
 template <bool kInt4>
 int gemm_batch_impl(const tq_linear* items, int count, int64_t M, void* workspace, size_t workspace_bytes,
-                    int variant, void* stream) {
+                    int variant, void* stream, const tq_linear* next = nullptr, int next_count = 0,
+                    int64_t next_M = 0) {
   if (count < 1 || count > tq::kBatchMaxItems) return TQ_ERR_SHAPE;
+  if (next_count < 0 || next_count > tq::kBatchMaxItems || next_M < 0 || next_M > tq::kBatchMaxM) return TQ_ERR_SHAPE;
+  if (next_count > 0 && !next) return TQ_ERR_NULL;
+  tq::BatchLinear nlin[tq::kBatchMaxItems];
+  int nn = 0;
+  for (int i = 0; i < next_count; ++i) {
+    const tq_linear& it = next[i];
+    if (it.N < 0 || it.N > (int64_t(1) << 31) || it.K <= 0 || it.K > (int64_t(1) << 28)) return TQ_ERR_SHAPE;
+    if (kInt4 ? (it.K % 128 != 0) : (it.K % 64 != 0)) return TQ_ERR_SHAPE;
+    if (it.N == 0) continue;
+    if (!it.w) return TQ_ERR_NULL;
+    if (!aligned16(it.w)) return TQ_ERR_ALIGN;
+    nlin[nn++] = tq::BatchLinear{nullptr, it.w, nullptr, nullptr, nullptr, it.N, it.K, nullptr};
+  }
+  tq::BatchNext nx;
+  nx.items = nlin;
+  nx.count = nn;
+  nx.M = next_M;
   const bool il = (variant & TQ_BATCH_INTERLEAVED) != 0;  // ternary weights in the interleaved layout
   variant &= ~TQ_BATCH_INTERLEAVED;
   if (variant < TQ_BATCH_AUTO || variant > TQ_BATCH_TENSOR_CORE) return TQ_ERR_PATH;
@@ -453,8 +471,8 @@ int gemm_batch_impl(const tq_linear* items, int count, int64_t M, void* workspac
   if (variant == TQ_BATCH_TENSOR_CORE)
     e = tq::launch_gemm_batch_tc(kInt4, lin, n, M, workspace, wb, as_stream(stream));
   else
-    e = kInt4 ? tq::launch_w4g_gemm_batch(lin, n, M, workspace, wb, as_stream(stream))
-              : tq::launch_tq_gemm_batch(lin, n, M, workspace, wb, as_stream(stream), il);
+    e = kInt4 ? tq::launch_w4g_gemm_batch(lin, n, M, workspace, wb, as_stream(stream), nx)
+              : tq::launch_tq_gemm_batch(lin, n, M, workspace, wb, as_stream(stream), il, nx);
   return to_status(e);
 }
 
@@ -480,6 +498,18 @@ int tq_gemm_batch_ex(const tq_linear* items, int count, int64_t M, void* workspa
 int w4g_gemm_batch_ex(const tq_linear* items, int count, int64_t M, void* workspace, size_t workspace_bytes,
                       int variant, void* stream) {
   return gemm_batch_impl<true>(items, count, M, workspace, workspace_bytes, variant, stream);
+}
+
+int tq_gemm_batch_next(const tq_linear* items, int count, int64_t M, void* workspace, size_t workspace_bytes,
+                       int variant, const tq_linear* next, int next_count, int64_t next_M, void* stream) {
+  return gemm_batch_impl<false>(items, count, M, workspace, workspace_bytes, variant, stream, next, next_count,
+                                next_M);
+}
+
+int w4g_gemm_batch_next(const tq_linear* items, int count, int64_t M, void* workspace, size_t workspace_bytes,
+                        int variant, const tq_linear* next, int next_count, int64_t next_M, void* stream) {
+  return gemm_batch_impl<true>(items, count, M, workspace, workspace_bytes, variant, stream, next, next_count,
+                               next_M);
 }
 
 int tq_interleave_packed(const uint8_t* packed, uint8_t* out, int64_t N, int64_t K, void* stream) {

@@ -49,6 +49,12 @@ struct BatchItem {
   int RB;              // row blocks
 };
 
+// The next call's linears (an L2 prefetch of the stages its CTAs load first).
+struct BatchNextItem {
+  int64_t begin;  // first stage of this item in the next call's sequence
+  int C, RB;      // stages per row block, row blocks
+};
+
 struct BatchParams {
   CUtensorMap w[kBMaxItems];  // packed weights: [N rows][row bytes], box 128 B x 128 rows, 128-B swizzle
   CUtensorMap x[kBMaxItems];  // activations viewed as [M][K/64][64], box 64 x 4 x M, 128-B swizzle
@@ -63,6 +69,12 @@ struct BatchParams {
   int* counters;              // [G] arrivals per split row block, indexed by its first contributor
   float* slots;               // [2 G][16][128] fp32 partials: slot 2c = CTA c's first row block,
                               // 2c + 1 = its last
+  // the next call on this stream, when the caller names it: its packed weights, its stage
+  // sequence, its CTAs and ring depth (0 items: none)
+  CUtensorMap wn[kBMaxItems];
+  BatchNextItem nit[kBMaxItems];
+  int ncount, Gn, nring;
+  int64_t Tn;
 };
 
 template <bool kInt4>
@@ -188,9 +200,11 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
       }
       int slot = 0;
       uint32_t ph = 0;  // parity of the slot's last completed `empty` phase
+      bool fine = true;
       for (int i = pre; i < nst; ++i) {
         if (!mbar_wait(&empty[slot], ph)) {
           flags[0] = 1;
+          fine = false;
           break;
         }
         mbar_arrive_expect_tx(&full[slot], tx);
@@ -200,6 +214,28 @@ __device__ __forceinline__ void batch_body(const BatchParams& P) {
         if (++slot == ring) {
           slot = 0;
           ph ^= 1u;
+        }
+      }
+      // All of this CTA's loads are issued.  The stages that the next call's CTA of this index
+      // loads first (its ring fill) are requested into L2 now, while this launch computes: that
+      // launch then starts on L2 hits instead of the HBM burst of every CTA's fill at once.
+      if (fine && P.ncount > 0 && c < P.Gn) {
+        const int64_t b0 = range_begin(c, P.Tn, P.Gn), b1 = range_begin(c + 1, P.Tn, P.Gn);
+        const int nn = static_cast<int>(b1 - b0 < P.nring ? b1 - b0 : P.nring);
+        int q = 0;
+        while (q + 1 < P.ncount && P.nit[q + 1].begin <= b0) ++q;
+        const uint32_t o = static_cast<uint32_t>(b0 - P.nit[q].begin);
+        int qC = P.nit[q].C, qrb = static_cast<int>(o / static_cast<uint32_t>(qC)),
+            qk = static_cast<int>(o % static_cast<uint32_t>(qC));
+        for (int i = 0; i < nn && q < P.ncount; ++i) {
+          tma_prefetch_l2_2d(&P.wn[q], qk * 128, qrb * kBRows);
+          if (++qk == qC) {
+            qk = 0;
+            if (++qrb == P.nit[q].RB) {
+              qrb = 0;
+              if (++q < P.ncount) qC = P.nit[q].C;
+            }
+          }
         }
       }
     }
@@ -483,7 +519,7 @@ int64_t batch_workspace_bytes() {
 
 template <bool kInt4, bool kIL>
 static cudaError_t launch_batch_t(const BatchLinear* items, int count, int64_t M, void* ws, int64_t ws_bytes,
-                                  cudaStream_t s) {
+                                  cudaStream_t s, const BatchNext& next) {
   using F = DecFmt<kInt4>;
   using L = BatchLayout<kInt4>;
   if (count < 1 || count > kBMaxItems || M < 1 || M > 16) return cudaErrorInvalidValue;
@@ -538,6 +574,33 @@ static cudaError_t launch_batch_t(const BatchLinear* items, int count, int64_t M
   if (smem > kDSmemBudget) return cudaErrorInvalidValue;
   P.counters = reinterpret_cast<int*>(ws);
   P.slots = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + batch_counter_bytes(Gmax));
+  // the next call's stage sequence, CTAs and ring depth, as its own launch will compute them
+  P.ncount = 0;
+  if (next.count > 0 && next.count <= kBMaxItems && next.M >= 1 && next.M <= 16) {
+    int64_t Tn = 0;
+    for (int q = 0; q < next.count; ++q) {
+      const BatchLinear& b = next.items[q];
+      const int64_t kbytes = kInt4 ? b.K / 2 : b.K / 4;
+      if (!make_tmap_2d(&P.wn[q], CU_TENSOR_MAP_DATA_TYPE_UINT8, b.w, static_cast<uint64_t>(kbytes),
+                        static_cast<uint64_t>(b.N), static_cast<uint64_t>(kbytes), 128, kBRows,
+                        CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+      P.nit[q].begin = Tn;
+      P.nit[q].C = static_cast<int>((b.K + F::kStageK - 1) / F::kStageK);
+      P.nit[q].RB = static_cast<int>((b.N + kBRows - 1) / kBRows);
+      Tn += static_cast<int64_t>(P.nit[q].C) * P.nit[q].RB;
+    }
+    if (Tn * (Tn < Gmax ? Tn : Gmax) < (static_cast<int64_t>(1) << 32)) {
+      P.Tn = Tn;
+      P.Gn = static_cast<int>(Tn < Gmax ? Tn : Gmax);
+      const int xh = ((static_cast<int>(next.M) * 4 * 128 + 1023) / 1024) * 1024;
+      const int st = kDWBytes + (F::kKB / 4) * xh;
+      int rn = kDMaxRing;
+      while (rn > 2 && L::bytes(rn, st) > kDSmemBudget) --rn;
+      P.nring = rn;
+      P.ncount = next.count;
+    }
+  }
 
   const bool m16 = M > 8;
   const bool w4 = !m16 && kBatchM8FourWarps;
@@ -559,14 +622,14 @@ static cudaError_t launch_batch_t(const BatchLinear* items, int count, int64_t M
 }
 
 cudaError_t launch_tq_gemm_batch(const BatchLinear* items, int count, int64_t M, void* ws, int64_t ws_bytes,
-                                 cudaStream_t s, bool interleaved) {
-  return interleaved ? launch_batch_t<false, true>(items, count, M, ws, ws_bytes, s)
-                     : launch_batch_t<false, false>(items, count, M, ws, ws_bytes, s);
+                                 cudaStream_t s, bool interleaved, const BatchNext& next) {
+  return interleaved ? launch_batch_t<false, true>(items, count, M, ws, ws_bytes, s, next)
+                     : launch_batch_t<false, false>(items, count, M, ws, ws_bytes, s, next);
 }
 
 cudaError_t launch_w4g_gemm_batch(const BatchLinear* items, int count, int64_t M, void* ws, int64_t ws_bytes,
-                                  cudaStream_t s) {
-  return launch_batch_t<true, false>(items, count, M, ws, ws_bytes, s);
+                                  cudaStream_t s, const BatchNext& next) {
+  return launch_batch_t<true, false>(items, count, M, ws, ws_bytes, s, next);
 }
 
 }  // namespace tq

@@ -245,15 +245,22 @@ struct BatchLinear {
   const uint8_t* zp;   // W4A16 zero-points [N, K/128], or null (symmetric)
 };
 constexpr int kBatchMaxItems = 8;
+// The call that will follow a batch call on its stream, when the caller names it (its weights
+// are then prefetched into L2 during this call; only w, N and K of its items are read).
+struct BatchNext {
+  const BatchLinear* items = nullptr;
+  int count = 0;
+  int64_t M = 0;
+};
 constexpr int64_t kBatchMaxM = 32;        // the tensor-core variant; the mma.sync variant takes M <= 16
 // Workspace bytes the batch kernel needs on the current device.
 int64_t batch_workspace_bytes();
 cudaError_t launch_tq_gemm_batch(const BatchLinear* items, int count, int64_t M, void* ws, int64_t ws_bytes,
-                                 cudaStream_t s, bool interleaved = false);
+                                 cudaStream_t s, bool interleaved = false, const BatchNext& next = BatchNext());
 // The pair-interleaved relayout of packed ternary rows (words of 16 codes, flat).
 cudaError_t launch_tq_interleave(const uint32_t* in, uint32_t* out, int64_t words, cudaStream_t s);
 cudaError_t launch_w4g_gemm_batch(const BatchLinear* items, int count, int64_t M, void* ws, int64_t ws_bytes,
-                                  cudaStream_t s);
+                                  cudaStream_t s, const BatchNext& next = BatchNext());
 // The tensor-core variant of the batch kernel (tq_tcbatch.cu), 1 <= M <= 32.
 cudaError_t launch_gemm_batch_tc(bool int4, const BatchLinear* items, int count, int64_t M, void* ws,
                                  int64_t ws_bytes, cudaStream_t s);

@@ -297,6 +297,23 @@ TQ_API int tq_gemm_batch_ex(const tq_linear* items, int count, int64_t M, void* 
 TQ_API int w4g_gemm_batch_ex(const tq_linear* items, int count, int64_t M, void* workspace,
                              size_t workspace_bytes, int variant, void* stream);
 
+/* tq_gemm_batch_next / w4g_gemm_batch_next -- tq_gemm_batch_ex / w4g_gemm_batch_ex that also
+ * names the batch call which will follow it on the same stream (a serving engine knows its next
+ * layer): `next` is a HOST array of `next_count` (0 .. 8) items of which only w, N and K are read
+ * (w 16-byte aligned, the same format and shape rules as `items`), and next_M its token count
+ * (0 .. 32).  While this call computes, each CTA requests into L2 the packed-weight tiles that
+ * the next call's CTA of the same index loads first (the mma.sync variant's ring fill, for
+ * next_M <= 16; larger next_M prefetch nothing), so that launch starts on L2 hits.  Results are
+ * exactly those of tq_gemm_batch_ex: the prefetch is a hint that moves no output.  Naming a
+ * call that does not follow only costs the prefetched bytes.
+ * ------------------------------------------------------------------------------------------ */
+TQ_API int tq_gemm_batch_next(const tq_linear* items, int count, int64_t M, void* workspace,
+                              size_t workspace_bytes, int variant, const tq_linear* next, int next_count,
+                              int64_t next_M, void* stream);
+TQ_API int w4g_gemm_batch_next(const tq_linear* items, int count, int64_t M, void* workspace,
+                               size_t workspace_bytes, int variant, const tq_linear* next, int next_count,
+                               int64_t next_M, void* stream);
+
 /* --------------------------------------------------------------------------------------------
  * tq_interleave_packed -- relayout of packed ternary rows for the decode kernels ([VQ] §4.3: the
  * post-load repack a checkpoint's weights go through once before inference; the layout itself

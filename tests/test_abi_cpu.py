@@ -12,7 +12,7 @@ import bit_weight_only_tq_b200 as tq
 
 def test_library_exports_every_header_function():
     names = tq.header_functions()
-    assert len(names) == 28
+    assert len(names) == 30
     for n in names:
         assert hasattr(tq.lib, n), n
     for n in ("tq_quantize_pack", "tq_gemm", "w4g_quantize_pack", "w4g_gemm", "tq_validate_packed",
@@ -137,6 +137,18 @@ def test_batch_argument_errors_without_gpu():
     assert tq.lib.tq_gemm_batch_ex(ok, 1, 17, ws, big, tq.BATCH_AUTO | tq.BATCH_INTERLEAVED, None) == -8
     assert tq.lib.w4g_gemm_batch_ex(ok, 1, 4, ws, big, tq.BATCH_MMA_SYNC | tq.BATCH_INTERLEAVED, None) == -8
     assert tq.lib.tq_gemm_batch_ex(ok, 1, 4, ws, big, 3 | tq.BATCH_INTERLEAVED, None) == -8
+    # the call-with-next entry: the next items' count, token count, pointers and shapes are
+    # checked before anything else
+    nxt = _items((0, a, 0, 0, 64, 128))
+    assert tq.lib.tq_gemm_batch_next(ok, 1, 1, ws, big, 0, nxt, 9, 1, None) == -2   # next count
+    assert tq.lib.tq_gemm_batch_next(ok, 1, 1, ws, big, 0, nxt, -1, 1, None) == -2
+    assert tq.lib.tq_gemm_batch_next(ok, 1, 1, ws, big, 0, nxt, 1, 33, None) == -2  # next M
+    assert tq.lib.tq_gemm_batch_next(ok, 1, 1, ws, big, 0, None, 1, 1, None) == -1  # null next
+    assert tq.lib.tq_gemm_batch_next(ok, 1, 1, ws, big, 0, _items((0, 0, 0, 0, 64, 128)), 1, 1, None) == -1
+    assert tq.lib.tq_gemm_batch_next(ok, 1, 1, ws, big, 0, _items((0, q, 0, 0, 64, 128)), 1, 1, None) == -3
+    assert tq.lib.tq_gemm_batch_next(ok, 1, 1, ws, big, 0, _items((0, a, 0, 0, 64, 100)), 1, 1, None) == -2
+    assert tq.lib.w4g_gemm_batch_next(ok, 1, 1, ws, big, 0, _items((0, a, 0, 0, 64, 192)), 1, 1, None) == -2
+    assert tq.lib.tq_gemm_batch_next(ok, 0, 1, ws, big, 0, nxt, 1, 1, None) == -2   # this call's count
     # the allocation-free variant checks the same arguments before any device work
     assert tq.lib.tq_gemm_batch_noalloc(ok, 0, 1, None) == -2
     assert tq.lib.tq_gemm_batch_noalloc(ok, 9, 1, None) == -2

@@ -94,6 +94,44 @@ def test_tq_batch_deterministic_and_reusable(variant):
     _counters_zero(ws)
 
 
+# naming the next call (an L2 prefetch of its first weight tiles) moves no output bit: the same
+# layer sequence with and without the hints, including a next call of another M, one above the
+# mma.sync range (nothing prefetched), one with an empty matrix, and W4A16
+@pytest.mark.parametrize("int4", [False, True])
+def test_batch_next_hint_changes_nothing(int4):
+    need_cuda()
+    shapes = SHAPES[2]
+    layers = []
+    for li in range(2):
+        mats = []
+        for i, (N, K) in enumerate(shapes):
+            w = I.weights(N, K, 60 + 7 * li + i, device="cuda")
+            mats.append(tq.w4g_quantize_pack(w) if int4 else tq.tq_quantize_pack(w))
+        layers.append(mats)
+    ws = _workspace()
+    fn = tq.w4g_gemm_batch if int4 else tq.tq_gemm_batch
+    key = "next_qweight" if int4 else "next_packed"
+    calls = [(1, 0, (1, 1)), (1, 1, (4, 0)), (4, 0, (16, 1)), (16, 1, (32, 0)), (4, 1, (1, 0)), (16, 0, None)]
+    xs = {(M, K): I.activations(M, K, 70 + M + K, device="cuda") for M in (1, 4, 16) for K in (4096, 14336)}
+    for M, li, nxt in calls:
+        X = [xs[(M, K)] for _, K in shapes]
+        P = [p for p, _ in layers[li]]
+        S = [s for _, s in layers[li]]
+        plain = [y.clone() for y in fn(X, P, S, workspace=ws)]
+        if nxt is None:
+            continue
+        nM, nl = nxt
+        named = [p for p, _ in layers[nl]]
+        if nM == 4:
+            named = named[:3] + [named[3][:0]] + named[4:]  # an empty matrix among the next items
+        hinted = fn(X, P, S, workspace=ws, **{key: named, "next_M": nM})
+        torch.cuda.synchronize()
+        for a, b in zip(plain, hinted):
+            assert torch.equal(a.view(torch.int16), b.view(torch.int16)), (M, li, nxt)
+    _counters_zero(ws)
+    assert tq.tq_device_status() == 0
+
+
 def test_tq_batch_matches_single_calls():
     need_cuda()
     shapes = SHAPES[1]
