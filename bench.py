@@ -615,10 +615,12 @@ def secondary_rows(args, rank, layers, peaks):
         xq = {K: I.activations(M, K, I.seed_for(3, 2, K) + M, device="cuda") for K in (4096, 14336)}
         yq = {N: torch.empty(M, N, dtype=torch.float16, device="cuda") for N in (1024, 4096, 14336)}
 
-        def wd():  # one w4g_gemm_batch launch per layer (its 7 linears)
-            for row in w4:
+        def wd():  # one w4g_gemm_batch launch per layer (its 7 linears), each naming the next
+            for li, row in enumerate(w4):
+                nxt = w4[(li + 1) % len(w4)]
                 tq.w4g_gemm_batch([xq[K] for _, _, K, _, _ in row], [r[3] for r in row], [r[4] for r in row],
-                                  None, [yq[N] for _, N, _, _, _ in row], workspace=ws)
+                                  None, [yq[N] for _, N, _, _, _ in row], workspace=ws,
+                                  next_qweight=[r[3] for r in nxt], next_M=M)
 
         def wc():  # one w4g_gemm call per linear
             for row in w4:
